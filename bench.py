@@ -1,0 +1,534 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized paged KV-cache decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--fmt F]
+    python bench.py --impl reference ...        # the CPU oracle, same metric
+
+One step = the whole hot path for one decode step of the workload: append one
+new token per sequence into the quantized paged cache (kvq_append), paged GQA
+decode attention split into chunk partials (kvq_decode_partial) and the
+log-sum-exp merge into the BF16 output (kvq_decode_merge).
+
+Headline `value`: decode KV bytes read per step (all ranks) / step time, GB/s.
+Inputs live in HBM before timing; L2 is flushed (a 256 MB write) before every
+timed step and each step is timed on its stream with CUDA events; K steps are
+bracketed by a barrier and a device synchronize; the max over ranks is taken.
+Multi-GPU runs are weak-scaled replicas: each rank holds its own batch of
+sequences (the path has no exchange step), so `value` sums all ranks' bytes.
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int8_quantized_paged_quantize_b200 import workloads as WL  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama3-8b-fp8"
+META_BYTES = {"fp8": 4, "int8": 8, "bf16": 0}       # per (token, KV head): K and V metadata
+ELEM = {"fp8": 1, "int8": 1, "bf16": 2}
+DTYPE_TAG = {"fp8": "e4m3 cache / f32 accumulate", "int8": "s8 cache / f32 accumulate",
+             "bf16": "bf16 cache / f32 accumulate"}
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kv_bytes_per_step(ctx, w, fmt):
+    """Algorithmic bytes one decode step reads: the K and V codes plus their
+    per-token metadata for every attended token and KV head, the queries and
+    the block-table entries."""
+    ctx = np.asarray(ctx, dtype=np.int64)
+    kv = int(ctx.sum()) * w.n_kv_heads * (2 * w.head_dim * ELEM[fmt] + META_BYTES[fmt])
+    q = w.batch * w.n_q_heads * w.head_dim * 2
+    tables = 4 * int(((ctx + 15) // 16).sum())
+    return kv, kv + q + tables
+
+
+def append_bytes_per_token(w, fmt):
+    """Append: read K and V BF16 rows, write codes and metadata."""
+    return w.n_kv_heads * (2 * w.head_dim * 2 + 2 * w.head_dim * ELEM[fmt] + META_BYTES[fmt])
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.proc, self.path = None, None
+        try:
+            self.id = "GPU-" + str(torch.cuda.get_device_properties(index).uuid)
+        except Exception:
+            self.id = str(index)
+
+    def start(self):
+        try:
+            import tempfile
+            self.path = tempfile.mktemp(suffix=".csv")
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.id}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            c = [x.strip() for x in line.split(",")]
+            if len(c) < 9:
+                continue
+            try:
+                sm.append(float(c[1]))
+                mx.append(float(c[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, c[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, device="cuda"):
+    """Max of a float over all ranks (identity on one rank)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world, device="cuda"):
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- GPU setup
+class Setup:
+    """Device-resident state of one workload in one format: the filled cache,
+    per-step inputs, slots, context lengths, workspace and output."""
+
+    def __init__(self, w, fmt, steps, seed, hist=None):
+        from int8_quantized_paged_quantize_b200 import kvq
+        self.kvq = kvq
+        self.w, self.fmt, self.steps = w, fmt, steps
+        self.tables_np, nb = WL.block_tables(w, seed)
+        self.ctx0 = WL.context_lengths(w, seed) + w.bulk_append
+        d = kvq.dims(nb, w.n_kv_heads, w.n_q_heads, w.head_dim, self.tables_np.shape[1])
+        self.dims = d
+        self.cache = kvq.LayerCache.allocate(fmt, d)
+        dev = torch.device("cuda")
+        self.tables = torch.from_numpy(self.tables_np).to(dev)
+        self.hist = hist if hist is not None else self.make_history(w, seed)
+        self.fill()
+        # per-step inputs, resident in HBM
+        self.q, self.k, self.v, self.slots, self.ctx = [], [], [], [], []
+        ctx = self.ctx0.copy()
+        for s in range(steps):
+            q, k, v = WL.step_inputs(w, s, seed)
+            self.q.append(q.to(dev))
+            self.k.append(k.to(dev))
+            self.v.append(v.to(dev))
+            sl = self.tables_np[np.arange(w.batch), ctx // 16].astype(np.int64) * 16 + ctx % 16
+            self.slots.append(torch.from_numpy(sl).to(dev))
+            ctx = ctx + 1
+            self.ctx.append(torch.from_numpy(ctx.astype(np.int32)).to(dev))
+        self.ctx_np = [self.ctx0 + s + 1 for s in range(steps)]
+        self.max_ctx = int(self.ctx_np[-1].max())
+        self.ws = self.cache.workspace(w.batch, self.max_ctx)
+        self.out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+
+    @staticmethod
+    def make_history(w, seed):
+        """BF16 K/V of every sequence's cached tokens (history + bulk append),
+        concatenated, with their slots."""
+        tables, _ = WL.block_tables(w, seed)
+        ctx = WL.context_lengths(w, seed)
+        ks, vs, ss = [], [], []
+        for b in range(w.batch):
+            k, v = WL.kv_history(w, b, seed)
+            ks.append(k)
+            vs.append(v)
+            pos = np.arange(ctx[b])
+            if w.bulk_append:
+                kb, vb = WL.kv_bulk(w, b, seed)
+                ks.append(kb)
+                vs.append(vb)
+                pos = np.arange(ctx[b] + w.bulk_append)
+            ss.append(torch.from_numpy(tables[b][pos // 16].astype(np.int64) * 16 + pos % 16))
+        return torch.cat(ks), torch.cat(vs), torch.cat(ss)
+
+    def fill(self, chunk=1 << 16):
+        K, V, S = self.hist
+        dev = torch.device("cuda")
+        for a in range(0, S.numel(), chunk):
+            self.cache.append(K[a:a + chunk].to(dev), V[a:a + chunk].to(dev), S[a:a + chunk].to(dev))
+        torch.cuda.synchronize()
+
+    def reset_tail(self):
+        """Nothing to undo: step s appends at position ctx0 + s, so re-running the
+        steps overwrites the same slots with the same values."""
+
+    # one step of the hot path, with events between its phases
+    def step(self, s, ev=None):
+        kvq, c = self.kvq, self.cache
+        w = self.w
+        c.append(self.k[s], self.v[s], self.slots[s])
+        if ev is not None:
+            ev[1].record()
+        kvq.decode_partial(self.q[s], c.k, c.v, c.k_scale, c.v_scale, self.tables, self.ctx[s],
+                           self.max_ctx, w.sm_scale, self.ws, self.fmt, self.dims)
+        if ev is not None:
+            ev[2].record()
+        kvq.decode_merge(w.batch, self.ctx[s], self.max_ctx, self.out, self.ws, self.fmt, self.dims)
+
+
+def timed_loop(st, steps, warmup, world, flush):
+    """Run warmup + steps; returns per-phase mean milliseconds over the timed steps."""
+    for s in range(warmup):
+        st.step(s % st.steps)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev = evs[i]
+        ev[0].record()
+        st.step(i % st.steps, ev)
+        ev[3].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    mrg_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    return {"step": float(np.mean(step_ms)), "append": float(np.mean(app_ms)),
+            "decode": float(np.mean(dec_ms)), "merge": float(np.mean(mrg_ms)),
+            "launches": 3 * steps}
+
+
+def e2e_loop(st, steps, warmup, world, flush):
+    """The same step through the public API with host inputs: per step the
+    step's inputs are copied from pinned host memory (q, k, v, slots, context
+    lengths, the block tables) and the output is read back, inside the timing."""
+    w = st.w
+    host = []
+    for s in range(st.steps):
+        host.append([t.cpu().pin_memory() for t in (st.q[s], st.k[s], st.v[s], st.slots[s], st.ctx[s])])
+    tables_h = st.tables.cpu().pin_memory()
+    out_h = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    dq = [torch.empty_like(t) for t in (st.q[0], st.k[0], st.v[0], st.slots[0], st.ctx[0])]
+    tables_d = torch.empty_like(st.tables)
+    h2d = sum(t.numel() * t.element_size() for t in host[0]) + tables_h.numel() * 4
+    d2h = out_h.numel() * out_h.element_size()
+
+    def one(s):
+        for d, h in zip(dq, host[s]):
+            d.copy_(h, non_blocking=True)
+        tables_d.copy_(tables_h, non_blocking=True)
+        q, k, v, sl, cl = dq
+        st.cache.append(k, v, sl)
+        st.cache.decode(q, tables_d, cl, st.max_ctx, sm_scale=w.sm_scale, out=st.out,
+                        workspace=st.ws)
+        out_h.copy_(st.out, non_blocking=True)
+
+    for s in range(warmup):
+        one(s % st.steps)
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record()
+        one(i % st.steps)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    return ms, h2d, d2h
+
+
+def bulk_append_rate(st, tokens=32768, reps=5):
+    """Append throughput for one bulk call of `tokens` tokens (prefill-style)."""
+    K, V, S = st.hist
+    n = min(tokens, S.numel())
+    dev = torch.device("cuda")
+    k, v, s = K[:n].to(dev), V[:n].to(dev), S[:n].to(dev)
+    for _ in range(2):
+        st.cache.append(k, v, s)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        st.cache.append(k, v, s)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    return n / (ms * 1e-3), ms, n
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_decode_sample(w, fmt, seed, budget_s=12.0):
+    """Time the CPU oracle on a bounded sample of the workload: for sequences in
+    order until the time budget is spent, quantize the sequence's cached K/V into
+    an oracle pool (append) and run the decode step's attention over it for all
+    query heads (dequantising gather + FP64 softmax attention). Returns
+    (decode KV GB/s, append tok/s, sample description, threads)."""
+    from oracle import attention as OA
+    from oracle import paged as OP
+    tables, nb = WL.block_tables(w, seed)
+    ctx = WL.context_lengths(w, seed)
+    q, kn, vn = WL.step_inputs(w, 0, seed)
+    t_app = t_dec = 0.0
+    n_tok = 0
+    kv_bytes = 0
+    done = []
+    t_start = time.perf_counter()
+    for b in range(w.batch):
+        if time.perf_counter() - t_start > budget_s and done:
+            break
+        k, v = WL.kv_history(w, b, seed)
+        k = torch.cat([k, kn[b:b + 1]]).float().numpy()
+        v = torch.cat([v, vn[b:b + 1]]).float().numpy()
+        n = k.shape[0]
+        pages = (n + 15) // 16
+        pool = OP.LogicalPool(fmt, pages, w.n_kv_heads, 16, w.head_dim)
+        row = np.arange(pages)
+        t0 = time.perf_counter()
+        pool.append(k, v, OP.slot_of(row, np.arange(n), 16))
+        t1 = time.perf_counter()
+        K, V = pool.gather(row, n)
+        OA.decode_attention(q[b:b + 1].float().numpy(), [(K, V)], w.sm_scale, w.n_kv_heads)
+        t2 = time.perf_counter()
+        t_app += t1 - t0
+        t_dec += t2 - t1
+        n_tok += n
+        kv_bytes += n * w.n_kv_heads * (2 * w.head_dim * ELEM[fmt] + META_BYTES[fmt])
+        done.append(b)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    desc = (f"{len(done)} of {w.batch} sequences ({n_tok} tokens, all {w.n_q_heads} query heads): "
+            f"oracle append of their cached tokens + one decode step")
+    return kv_bytes / t_dec / 1e9, n_tok / t_app, desc, threads
+
+
+def run_reference(args):
+    """The oracle as the reference arm: same metric/unit/config, each step a
+    bounded sample of the workload on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WL.WORKLOADS[args.workload]
+    fmt = args.fmt or w.fmt
+    vals = []
+    t0 = time.perf_counter()
+    for s in range(args.warmup + args.steps):
+        gbs, tok_s, desc, threads = oracle_decode_sample(w, fmt, seed=0, budget_s=args.ref_budget)
+        if s >= args.warmup:
+            vals.append(gbs)
+    value = float(np.mean(vals))
+    line = {"impl": "reference", "metric": metric_name(fmt), "value": value, "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * (time.perf_counter() - t0) / max(1, args.warmup + args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (seeded)",
+            "config": config_block(w, fmt, l2="host run (no GPU)"),
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": "GB/s", "cores": threads,
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def metric_name(fmt):
+    return f"paged decode-attn KV GB/s ({fmt.upper()} cache; step = append + decode + merge)"
+
+
+def config_block(w, fmt, l2):
+    lens = {"fixed": f"{w.ctx[0]}", "list": "list", "uniform": f"U[{w.ctx[0]},{w.ctx[1]}]",
+            "lognormal_mix": "lognormal(1500, 1) + 4x30000"}[w.lengths]
+    return {"workload": f"{w.name}: B={w.batch} Hq={w.n_q_heads} Hk={w.n_kv_heads} D={w.head_dim} "
+                        f"bs=16 ctx={lens}" + (f" +{w.bulk_append} bulk" if w.bulk_append else ""),
+            "fmt": fmt, "batch": w.batch, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "block_size": 16, "l2": l2}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WL.WORKLOADS))
+    ap.add_argument("--fmt", default=None, choices=["fp8", "int8", "bf16"])
+    ap.add_argument("--no-formats", action="store_true", help="skip the per-format comparison")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--ref-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    rank, world, local = dist_setup(args.gpus)
+    w = WL.WORKLOADS[args.workload]
+    fmt = args.fmt or w.fmt
+    steps_needed = args.warmup + args.steps
+    wb = dataclasses.replace(w, decode_steps=max(w.decode_steps, steps_needed))
+    seed = rank
+    hbm_peak, peak_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    hist = Setup.make_history(wb, seed)
+    st = Setup(wb, fmt, steps_needed, seed, hist=hist)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t = timed_loop(st, args.steps, args.warmup, world, flush)
+    clk = clocks.stop()
+
+    step_ms = max_over_ranks(t["step"], world)
+    dec_ms = max_over_ranks(t["decode"], world)
+    # bytes of the timed steps (contexts grow by one per step)
+    kv_list, all_list = zip(*[kv_bytes_per_step(st.ctx_np[i % st.steps], wb, fmt)
+                              for i in range(args.steps)])
+    kv_step = float(np.mean(kv_list))
+    alg_step = float(np.mean(all_list))
+    kv_total = sum_over_ranks(kv_step, world)
+    value = kv_total / (step_ms * 1e-3) / 1e9
+    achieved = alg_step / (t["decode"] * 1e-3) / 1e9
+    seqs_s = sum_over_ranks(wb.batch, world) / (step_ms * 1e-3)
+    app_tok_s = sum_over_ranks(wb.batch, world) / (max_over_ranks(t["append"], world) * 1e-3)
+    bulk_tok_s, bulk_ms, bulk_n = bulk_append_rate(st)
+
+    e2e_ms, h2d, d2h = e2e_loop(st, args.steps, args.warmup, world, flush)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_val = kv_total / (e2e_ms * 1e-3) / 1e9
+
+    formats = {}
+    if not args.no_formats:
+        for f in ("fp8", "int8", "bf16"):
+            if f == fmt:
+                tf, stf = t, st
+            else:
+                del st
+                torch.cuda.empty_cache()
+                stf = Setup(wb, f, steps_needed, seed, hist=hist)
+                tf = timed_loop(stf, args.steps, args.warmup, world, flush)
+            kvf = float(np.mean([kv_bytes_per_step(stf.ctx_np[i % stf.steps], wb, f)[0]
+                                 for i in range(args.steps)]))
+            algf = float(np.mean([kv_bytes_per_step(stf.ctx_np[i % stf.steps], wb, f)[1]
+                                  for i in range(args.steps)]))
+            bt, _, _ = bulk_append_rate(stf)
+            smax = max_over_ranks(tf["step"], world)
+            formats[f] = {
+                "kv_gbs_step": sum_over_ranks(kvf, world) / (smax * 1e-3) / 1e9,
+                "decode_kernel_gbs": algf / (tf["decode"] * 1e-3) / 1e9,
+                "decode_frac_of_peak": algf / (tf["decode"] * 1e-3) / 1e9 / hbm_peak,
+                "decode_seqs_per_s": sum_over_ranks(wb.batch, world) / (smax * 1e-3),
+                "append_tok_per_s_step": sum_over_ranks(wb.batch, world) / (tf["append"] * 1e-3),
+                "append_tok_per_s_bulk": bt,
+                "ms": {k: round(v, 5) for k, v in tf.items() if k != "launches"},
+                "kv_bytes_per_step": kvf,
+            }
+            st = stf
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        gbs, tok_s, desc, threads = oracle_decode_sample(wb, fmt, seed=0)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "append_tok_per_s": tok_s}
+
+    line = {
+        "metric": metric_name(fmt), "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": DTYPE_TAG[fmt], "data": "synthetic (seeded; no dataset or weights)",
+        "config": config_block(wb, fmt, l2="flushed before every timed step (256 MB write)"),
+        "decode_seqs_per_s": seqs_s, "append_tok_per_s_step": app_tok_s,
+        "append_tok_per_s_bulk": bulk_tok_s, "kv_frac_of_peak_step": value / world / hbm_peak,
+        "phase_ms": {k: round(v, 5) for k, v in t.items() if k != "launches"},
+        "roofline": {"bound": "hbm", "kernel": "decode partial (kvq_decode_partial)",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                     "alg_bytes_per_launch": alg_step, "traffic": None},
+        "e2e": {"value": e2e_val, "unit": "GB/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": t["launches"],
+        "clocks": clk,
+        "formats": formats,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,264 @@
+/*
+ * kvq.h - C ABI of libkvq: a quantized paged KV cache (FP8 E4M3 / INT8
+ * asymmetric) for autoregressive decode on NVIDIA B200 (sm_100a).
+ *
+ * The library has two hot operations, both CUDA kernels launched on the
+ * caller's stream:
+ *   kvq_append       quantize-on-append of new tokens' K and V into the paged pool
+ *   kvq_decode_attn  paged GQA decode attention over the quantized cache
+ * plus a host-side block allocator and size queries.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [LIMITS]   "KV cache quantization: what FP8/INT8 K and V really give, and
+ *              their limits" (molayo1419.me)
+ *   [76X]      "Fitting 76x concurrent requests with an FP8 KV cache"
+ *              (storycompiler.tistory.com/431)
+ *   [COMPRESS] "KV Cache compression" (ryotta.opik.net)
+ *   [GUIDE]    "From FP8 KV cache to INT4 weight-only: GPU LLM serving
+ *              optimisation guide (May 2026)" (daewooki.github.io)
+ *
+ * Conventions for every call
+ * --------------------------
+ * - Pointers marked "device" are CUDA device pointers on the current device;
+ *   "host" pointers are ordinary host memory. Every device pointer must be
+ *   16-byte aligned.
+ * - The caller owns every buffer and the stream. The hot calls (kvq_append,
+ *   kvq_decode_attn and its two phases) allocate no memory; the split-K
+ *   scratch of decode comes from the caller (kvq_decode_workspace_bytes).
+ * - Return value: KVQ_OK (0) or a negative kvq_status. Argument checks run on
+ *   the host before any launch; a failed check launches nothing. Launches are
+ *   asynchronous: KVQ_ERR_CUDA reports a launch failure only.
+ * - Data-dependent faults (a slot or block id outside the pool, a context
+ *   length beyond the block table or beyond max_context_len) cannot be seen on
+ *   the host. Kernels skip the offending token, page or sequence and set a bit
+ *   in a per-device error word that kvq_device_error() reads.
+ * - Supported shapes: block_size 16; head_dim 64 or 128; GQA group
+ *   G = n_q_heads / n_kv_heads in {1, 2, 4, 8}. Other shapes return
+ *   KVQ_ERR_UNSUPPORTED.
+ *
+ * Device layouts (one layer; K and V are separate arrays)
+ * -------------------------------------------------------
+ *   K cache  [num_blocks][n_kv_heads][block_size][head_dim]   element-major rows
+ *   V cache  [num_blocks][n_kv_heads][head_dim][block_size]   each (block, head)
+ *            page is stored transposed, so that a page row holds one channel
+ *            of 16 consecutive tokens
+ *   element  1 byte (FP8 E4M3 code or int8 code) or 2 bytes (BF16)
+ *   scales   FP8:  [num_blocks][n_kv_heads][block_size]    BF16 scale
+ *            INT8: [num_blocks][n_kv_heads][block_size][2] BF16 {scale, zero_point}
+ *            BF16: none (pass NULL)
+ * A token at sequence position p lives in slot
+ *   block_tables[b][p / block_size] * block_size + p % block_size.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t). NULL is the legacy default stream. */
+typedef struct CUstream_st* kvq_stream_t;
+
+typedef enum {
+  KVQ_BF16 = 0,      /* unquantized BF16 cache: the comparison baseline */
+  KVQ_FP8_E4M3 = 1,  /* OCP E4M3 codes (max 448, RNE, saturating) + BF16 scale */
+  KVQ_INT8_ASYM = 2  /* signed int8 codes + BF16 {scale, zero_point} */
+} kvq_fmt;
+
+typedef enum {
+  KVQ_OUT_BF16 = 0,  /* decode output rounded to BF16 (round to nearest even) */
+  KVQ_OUT_F32 = 1    /* decode output as the kernel's FP32 result */
+} kvq_out_dtype;
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_ARG = -1,            /* null/misaligned pointer, bad size or enum */
+  KVQ_ERR_UNSUPPORTED = -2,    /* shape outside the supported set */
+  KVQ_ERR_WORKSPACE = -3,      /* decode workspace smaller than required */
+  KVQ_ERR_CUDA = -4,           /* a CUDA call or launch failed */
+  KVQ_ERR_POOL_EXHAUSTED = -5, /* the block allocator has too few free blocks */
+  KVQ_ERR_DEVICE = -6          /* kvq_device_error found a flagged fault */
+} kvq_status;
+
+/* Bits of the per-device error word (kvq_device_error). */
+#define KVQ_DEVERR_SLOT 0x1u     /* append: slot >= num_blocks * block_size */
+#define KVQ_DEVERR_BLOCK 0x2u    /* decode: block id outside [0, num_blocks) */
+#define KVQ_DEVERR_CONTEXT 0x4u  /* decode: context_len < 0, > max_context_len,
+                                    or > max_blocks_per_seq * block_size */
+
+typedef struct {
+  int32_t num_blocks;         /* blocks in the pool */
+  int32_t block_size;         /* tokens per block; must be 16 */
+  int32_t n_kv_heads;         /* KV heads (Hk) */
+  int32_t n_q_heads;          /* query heads (Hq); Hq / Hk in {1, 2, 4, 8} */
+  int32_t head_dim;           /* D: 64 or 128 */
+  int32_t max_blocks_per_seq; /* W: the row length of block_tables */
+} kvq_dims;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int kvq_version(void);
+
+/* Static text for a kvq_status value. */
+const char* kvq_status_string(int status);
+
+/*
+ * Bytes of ONE cache array (K or V) and of its scale array for `dims`.
+ * [COMPRESS] "1. The KV cache memory problem" gives the element count
+ * 2 x layers x n_kv_heads x head_dim x tokens x bytes; one cache array is one
+ * of the two halves of one layer for num_blocks * block_size tokens.
+ * meta_bytes is 0 for KVQ_BF16. Host only; no CUDA call.
+ */
+int kvq_cache_bytes(const kvq_dims* dims, kvq_fmt fmt, size_t* cache_bytes,
+                    size_t* meta_bytes);
+
+/* ------------------------------------------------------------------------ */
+/* Host block allocator.                                                      */
+/* [GUIDE] "Core concepts 2) PagedAttention": the cache is a pool of fixed-    */
+/* size blocks and each request is mapped to just the blocks it needs.        */
+/* [COMPRESS] "6.2": low-bit K/V fit more tokens into each block's bytes.     */
+/* The allocator hands out block ids; device memory is the caller's. Not     */
+/* thread-safe: one pool per thread, or external locking.                     */
+/* ------------------------------------------------------------------------ */
+typedef struct kvq_pool kvq_pool;
+
+/* Create a pool of dims->num_blocks free blocks for `n_layers` layers of the
+ * given format. *out receives the handle (host memory owned by the library;
+ * release with kvq_pool_destroy). */
+int kvq_pool_create(const kvq_dims* dims, kvq_fmt fmt, int32_t n_layers, kvq_pool** out);
+void kvq_pool_destroy(kvq_pool* pool);
+
+/* Device bytes the pool stands for: element bytes of K and V over all layers
+ * (the closed form of [COMPRESS] section 1 for num_blocks * block_size tokens)
+ * and the bytes of their per-token scale arrays. */
+int kvq_pool_bytes(const kvq_pool* pool, size_t* element_bytes, size_t* meta_bytes);
+
+/* Number of free blocks. */
+int kvq_pool_num_free(const kvq_pool* pool, int32_t* n_free);
+
+/* Take n blocks (all or none) and write their ids to block_ids[0..n) (host).
+ * KVQ_ERR_POOL_EXHAUSTED if fewer than n are free. */
+int kvq_pool_alloc(kvq_pool* pool, int32_t n, int32_t* block_ids);
+
+/* Return n blocks. KVQ_ERR_ARG (and nothing freed) if an id is out of range,
+ * repeated, or not currently allocated. */
+int kvq_pool_free(kvq_pool* pool, int32_t n, const int32_t* block_ids);
+
+/* Grow one sequence from cur_len to cur_len + n_new tokens: allocate the new
+ * blocks it needs into block_table_row[ceil(cur_len/bs) .. ) (host, length
+ * dims->max_blocks_per_seq) and write the slot of each new token to
+ * slots[0..n_new) (host). All or nothing: KVQ_ERR_POOL_EXHAUSTED or
+ * KVQ_ERR_ARG (row too short) leave the row and the pool unchanged. */
+int kvq_pool_extend_seq(kvq_pool* pool, int32_t* block_table_row, int32_t cur_len,
+                        int32_t n_new, int64_t* slots);
+
+/* ------------------------------------------------------------------------ */
+/* Quantize-on-append.                                                        */
+/* [LIMITS] "What KV cache quantization actually is": K/V are quantized only */
+/* when stored, the scale comes from the full BF16 values, and the per-token */
+/* scales are kept in BF16. [LIMITS] "Formats you will actually meet": E4M3  */
+/* for K/V; INT8 per-token asymmetric with a (scale, zero_point) pair.       */
+/* [COMPRESS] "5.1" and "6.3": quantize right after K,V are computed.        */
+/* ------------------------------------------------------------------------ */
+/*
+ * k, v          device, [num_tokens][n_kv_heads][head_dim] BF16, contiguous:
+ *               the new tokens' keys and values.
+ * slot_mapping  device, [num_tokens] int64: destination slot of each token
+ *               (block = slot / block_size, offset = slot % block_size).
+ *               A negative slot skips the token; a slot >= num_blocks *
+ *               block_size skips it and sets KVQ_DEVERR_SLOT. Slots must be
+ *               distinct within one call.
+ * k_cache, v_cache  device, the layouts in the file header.
+ * k_scale, v_scale  device scale arrays (NULL for KVQ_BF16).
+ * Per (token, KV head) row of D values:
+ *   FP8:  s = bf16_rne(max|x| / 448); code = e4m3_rne_satfinite(x / s)
+ *   INT8: xmin = min(0, min x), xmax = max(0, max x);
+ *         s = bf16_rne((xmax - xmin) / 255); zp = clamp(-128 - rint(xmin / s), -128, 127);
+ *         code = clamp(rint(x / s) + zp, -128, 127)
+ *   (all divisions IEEE f32, rint ties to even; s == 0 stores zero codes and zp 0)
+ *   BF16: the values are copied.
+ */
+int kvq_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+               void* k_cache, void* v_cache, void* k_scale, void* v_scale, kvq_fmt fmt,
+               const kvq_dims* dims, kvq_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Paged GQA decode attention.                                                */
+/* [GUIDE] "Core concepts 1)": decode attends one query position against the */
+/* whole cached K/V and is bound by reading it. [LIMITS] "What KV cache      */
+/* quantization actually is": dequantization is fused into the attention    */
+/* kernel right before the matmuls. [76X] "4. Precision loss?": 8-bit        */
+/* storage, FP32 accumulation. [COMPRESS] "5.1": a separate dequantization   */
+/* kernel would give back the bandwidth gain.                                */
+/* ------------------------------------------------------------------------ */
+/*
+ * Scratch bytes kvq_decode_attn needs for these sizes. partition_tokens is the
+ * split-K chunk (a positive multiple of 128), or 0 to let the library choose
+ * from the batch, head count, max_context_len and the device's SM count.
+ * Returns 0 for invalid arguments.
+ */
+size_t kvq_decode_workspace_bytes(int32_t batch, int32_t max_context_len, int32_t partition_tokens,
+                                  kvq_fmt fmt, const kvq_dims* dims);
+
+/*
+ * out[b][h] = softmax_t(sm_scale * q[b][h] . K_b[t][h/G]) weighted sum of V_b[t][h/G],
+ * t = 0 .. context_lens[b]-1, where K_b/V_b are the dequantized cache rows read
+ * through block_tables[b]; G = n_q_heads / n_kv_heads (query head h uses KV head h / G).
+ *
+ * q             device, [batch][n_q_heads][head_dim] BF16.
+ * k_cache, v_cache  device, the layouts in the file header.
+ * scales        host array of 2 device pointers {k_scale, v_scale} (both NULL, or
+ *               scales itself NULL, for KVQ_BF16).
+ * block_tables  device, [batch][max_blocks_per_seq] int32.
+ * context_lens  device, [batch] int32: cached tokens per sequence, the token
+ *               appended in this step included. 0 gives an all-zero output row.
+ * max_context_len  host bound on every context_lens[b]; sizes the split grid.
+ * sm_scale      softmax scale (usually 1/sqrt(head_dim)).
+ * out           device, [batch][n_q_heads][head_dim], BF16 or FP32 per out_dtype.
+ * out_dtype     KVQ_OUT_BF16 or KVQ_OUT_F32. The kernel computes in FP32; BF16
+ *               output is that result rounded to nearest even.
+ * workspace     device scratch of at least kvq_decode_workspace_bytes(...) bytes;
+ *               contents on entry do not matter.
+ * partition_tokens  as for kvq_decode_workspace_bytes (0 = automatic).
+ * The sequence's tokens are split into chunks of partition_tokens; each chunk
+ * computes an online-softmax partial (max, sum, unnormalized output) and a
+ * merge kernel combines the partials with a log-sum-exp rescale.
+ */
+int kvq_decode_attn(const void* q, int32_t batch, const void* k_cache, const void* v_cache,
+                    const void* const* scales, const int32_t* block_tables,
+                    const int32_t* context_lens, int32_t max_context_len, float sm_scale,
+                    void* out, kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                    int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                    kvq_stream_t stream);
+
+/* The two phases of kvq_decode_attn, for callers that time or overlap them.
+ * kvq_decode_partial writes per-chunk partials into the workspace;
+ * kvq_decode_merge reads them and writes out. Same arguments and errors as
+ * kvq_decode_attn; the two calls must use the same batch, max_context_len,
+ * partition_tokens, dims and workspace. */
+int kvq_decode_partial(const void* q, int32_t batch, const void* k_cache, const void* v_cache,
+                       const void* const* scales, const int32_t* block_tables,
+                       const int32_t* context_lens, int32_t max_context_len, float sm_scale,
+                       void* workspace, size_t workspace_bytes, int32_t partition_tokens,
+                       kvq_fmt fmt, const kvq_dims* dims, kvq_stream_t stream);
+int kvq_decode_merge(int32_t batch, const int32_t* context_lens, int32_t max_context_len,
+                     void* out, kvq_out_dtype out_dtype, const void* workspace,
+                     size_t workspace_bytes,
+                     int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                     kvq_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Device error word.                                                          */
+/* ------------------------------------------------------------------------ */
+/* Read (and if `clear` is non-zero, reset) the current device's error word
+ * (KVQ_DEVERR_* bits) into *flags (host). Synchronizes the device. Returns
+ * KVQ_ERR_DEVICE if any bit was set, KVQ_OK otherwise. */
+int kvq_device_error(uint32_t* flags, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

@@ -19,6 +19,6 @@ __all__ = ["workloads", "kvq"]
 
 def __getattr__(name):
     if name == "kvq":
-        from . import kvq as _kvq
-        return _kvq
+        import importlib
+        return importlib.import_module(__name__ + ".kvq")
     raise AttributeError(name)

@@ -1,0 +1,194 @@
+// C ABI of libkvq: host-side argument checks, the split-K plan, and dispatch to
+// the CUDA kernels in kvq_kernels.cu. See include/kvq.h for the contract.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+namespace {
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dev_ok(const void* p) { return p != nullptr && aligned16(p); }
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+int cuda_rc(int e) { return e == 0 ? KVQ_OK : KVQ_ERR_CUDA; }
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();  // clear a sticky "no device" error from the query
+    return 148;
+  }
+  return n;
+}
+
+// Split-K chunking. A chunk is a whole number of 128-token tiles. Automatic
+// choice: the smallest power-of-two chunk (>= 128 tokens) for which the grid of
+// (sequence, KV head, chunk) CTAs of the longest sequence fits in 16 CTAs per
+// SM, so long contexts are spread over every SM while short ones stay in one
+// chunk (no merge traffic to speak of).
+int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kvq_dims* d,
+              DecodePlan* plan) {
+  if (batch < 0 || max_ctx < 0 || partition_tokens < 0) return KVQ_ERR_ARG;
+  if (partition_tokens % kTileTokens != 0) return KVQ_ERR_ARG;
+  int64_t part = partition_tokens;
+  if (part == 0) {
+    const int64_t budget = int64_t(16) * device_sm_count();
+    const int64_t rows = int64_t(batch) * d->n_kv_heads;
+    part = kTileTokens;
+    while (part < (int64_t(1) << 20) &&
+           rows * ((int64_t(max_ctx) + part - 1) / part) > budget)
+      part *= 2;
+  }
+  const int64_t splits = std::max<int64_t>(1, (int64_t(max_ctx) + part - 1) / part);
+  plan->partition = int32_t(part);
+  plan->max_splits = int32_t(splits);
+  const size_t rows = size_t(batch) * d->n_q_heads * size_t(splits);
+  plan->o_bytes = round256(rows * d->head_dim * sizeof(float));
+  plan->ml_bytes = round256(rows * 2 * sizeof(float));
+  plan->total = plan->o_bytes + plan->ml_bytes;
+  return KVQ_OK;
+}
+
+}  // namespace kvq
+
+using namespace kvq;
+
+namespace {
+
+int check_decode_common(int32_t batch, int32_t max_ctx, int32_t partition_tokens, kvq_fmt fmt,
+                        const kvq_dims* dims, DecodePlan* plan) {
+  if (!fmt_valid(fmt)) return KVQ_ERR_ARG;
+  int rc = check_dims(dims);
+  if (rc != KVQ_OK) return rc;
+  if (batch < 0 || max_ctx < 0) return KVQ_ERR_ARG;
+  if (int64_t(max_ctx) > int64_t(dims->max_blocks_per_seq) * dims->block_size) return KVQ_ERR_ARG;
+  return make_plan(batch, max_ctx, partition_tokens, dims, plan);
+}
+
+int check_decode_inputs(const void* q, const void* kc, const void* vc, const void* const* scales,
+                        const int32_t* tables, const int32_t* ctx, float sm_scale, kvq_fmt fmt,
+                        const void** ks, const void** vs) {
+  if (!dev_ok(q) || !dev_ok(kc) || !dev_ok(vc) || !dev_ok(tables) || !dev_ok(ctx))
+    return KVQ_ERR_ARG;
+  if (!std::isfinite(sm_scale)) return KVQ_ERR_ARG;
+  *ks = *vs = nullptr;
+  if (fmt != KVQ_BF16) {
+    if (!scales || !dev_ok(scales[0]) || !dev_ok(scales[1])) return KVQ_ERR_ARG;
+    *ks = scales[0];
+    *vs = scales[1];
+  }
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvq_version(void) { return 100; }
+
+const char* kvq_status_string(int status) {
+  switch (status) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_ARG: return "invalid argument (null or misaligned pointer, bad size or enum)";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported shape (block_size 16, head_dim 64/128, GQA group 1/2/4/8)";
+    case KVQ_ERR_WORKSPACE: return "decode workspace too small";
+    case KVQ_ERR_CUDA: return "CUDA launch or call failed";
+    case KVQ_ERR_POOL_EXHAUSTED: return "block pool exhausted";
+    case KVQ_ERR_DEVICE: return "a kernel flagged a data fault (see kvq_device_error)";
+    default: return "unknown status";
+  }
+}
+
+int kvq_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+               void* k_cache, void* v_cache, void* k_scale, void* v_scale, kvq_fmt fmt,
+               const kvq_dims* dims, kvq_stream_t stream) {
+  if (!fmt_valid(fmt) || num_tokens < 0) return KVQ_ERR_ARG;
+  int rc = check_dims(dims);
+  if (rc != KVQ_OK) return rc;
+  if (num_tokens == 0) return KVQ_OK;
+  if (!dev_ok(k) || !dev_ok(v) || !dev_ok(slot_mapping) || !dev_ok(k_cache) || !dev_ok(v_cache))
+    return KVQ_ERR_ARG;
+  if (fmt != KVQ_BF16 && (!dev_ok(k_scale) || !dev_ok(v_scale))) return KVQ_ERR_ARG;
+  return cuda_rc(launch_append(k, v, slot_mapping, num_tokens, k_cache, v_cache, k_scale, v_scale,
+                               fmt, *dims, stream));
+}
+
+size_t kvq_decode_workspace_bytes(int32_t batch, int32_t max_context_len, int32_t partition_tokens,
+                                  kvq_fmt fmt, const kvq_dims* dims) {
+  DecodePlan plan;
+  if (check_decode_common(batch, max_context_len, partition_tokens, fmt, dims, &plan) != KVQ_OK)
+    return 0;
+  return plan.total;
+}
+
+int kvq_decode_partial(const void* q, int32_t batch, const void* k_cache, const void* v_cache,
+                       const void* const* scales, const int32_t* block_tables,
+                       const int32_t* context_lens, int32_t max_context_len, float sm_scale,
+                       void* workspace, size_t workspace_bytes, int32_t partition_tokens,
+                       kvq_fmt fmt, const kvq_dims* dims, kvq_stream_t stream) {
+  DecodePlan plan;
+  int rc = check_decode_common(batch, max_context_len, partition_tokens, fmt, dims, &plan);
+  if (rc != KVQ_OK) return rc;
+  if (batch == 0) return KVQ_OK;
+  const void *ks, *vs;
+  rc = check_decode_inputs(q, k_cache, v_cache, scales, block_tables, context_lens, sm_scale, fmt,
+                           &ks, &vs);
+  if (rc != KVQ_OK) return rc;
+  if (!dev_ok(workspace)) return KVQ_ERR_ARG;
+  if (workspace_bytes < plan.total) return KVQ_ERR_WORKSPACE;
+  return cuda_rc(launch_decode_partial(q, batch, k_cache, v_cache, ks, vs, block_tables,
+                                       context_lens, max_context_len, sm_scale, plan, workspace,
+                                       fmt, *dims, stream));
+}
+
+int kvq_decode_merge(int32_t batch, const int32_t* context_lens, int32_t max_context_len,
+                     void* out, kvq_out_dtype out_dtype, const void* workspace,
+                     size_t workspace_bytes,
+                     int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                     kvq_stream_t stream) {
+  DecodePlan plan;
+  int rc = check_decode_common(batch, max_context_len, partition_tokens, fmt, dims, &plan);
+  if (rc != KVQ_OK) return rc;
+  if (out_dtype != KVQ_OUT_BF16 && out_dtype != KVQ_OUT_F32) return KVQ_ERR_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!dev_ok(context_lens) || !dev_ok(out) || !dev_ok(workspace)) return KVQ_ERR_ARG;
+  if (workspace_bytes < plan.total) return KVQ_ERR_WORKSPACE;
+  return cuda_rc(launch_decode_merge(batch, context_lens, max_context_len, out,
+                                     out_dtype == KVQ_OUT_F32, workspace, plan, *dims, stream));
+}
+
+int kvq_decode_attn(const void* q, int32_t batch, const void* k_cache, const void* v_cache,
+                    const void* const* scales, const int32_t* block_tables,
+                    const int32_t* context_lens, int32_t max_context_len, float sm_scale,
+                    void* out, kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                    int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                    kvq_stream_t stream) {
+  DecodePlan plan;
+  int rc = check_decode_common(batch, max_context_len, partition_tokens, fmt, dims, &plan);
+  if (rc != KVQ_OK) return rc;
+  if (out_dtype != KVQ_OUT_BF16 && out_dtype != KVQ_OUT_F32) return KVQ_ERR_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!dev_ok(out)) return KVQ_ERR_ARG;
+  rc = kvq_decode_partial(q, batch, k_cache, v_cache, scales, block_tables, context_lens,
+                          max_context_len, sm_scale, workspace, workspace_bytes, partition_tokens,
+                          fmt, dims, stream);
+  if (rc != KVQ_OK) return rc;
+  return kvq_decode_merge(batch, context_lens, max_context_len, out, out_dtype, workspace,
+                          workspace_bytes, partition_tokens, fmt, dims, stream);
+}
+
+int kvq_device_error(uint32_t* flags, int clear) {
+  if (!flags) return KVQ_ERR_ARG;
+  const int e = read_device_error(flags, clear);
+  if (e != 0) return KVQ_ERR_CUDA;
+  return *flags ? KVQ_ERR_DEVICE : KVQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Internal declarations shared by the host translation units of libkvq.
+// Device code lives in kvq_kernels.cu; the C ABI in kvq_api.cpp; the block
+// allocator in kvq_pool.cpp.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kBlockSize = 16;     // tokens per page
+constexpr int kTileTokens = 128;   // partition_tokens granularity
+
+// Element bytes of the cache arrays and BF16 metadata values per (token, head).
+inline int elem_bytes(kvq_fmt f) { return f == KVQ_BF16 ? 2 : 1; }
+inline int meta_values(kvq_fmt f) { return f == KVQ_FP8_E4M3 ? 1 : (f == KVQ_INT8_ASYM ? 2 : 0); }
+inline bool fmt_valid(int f) { return f == KVQ_BF16 || f == KVQ_FP8_E4M3 || f == KVQ_INT8_ASYM; }
+
+// Checks the shape rules of kvq.h. Returns KVQ_OK, KVQ_ERR_ARG or KVQ_ERR_UNSUPPORTED.
+int check_dims(const kvq_dims* d);
+
+// Split-K plan of one decode call.
+struct DecodePlan {
+  int32_t partition;   // tokens per split (multiple of kTileTokens)
+  int32_t max_splits;  // splits of the longest sequence
+  size_t o_bytes;      // partial outputs  [B][Hq][max_splits][D] f32
+  size_t ml_bytes;     // partial (max, sum) [B][Hq][max_splits][2] f32
+  size_t total;        // workspace bytes (256-aligned pieces)
+};
+// Fills `plan`; returns KVQ_OK or KVQ_ERR_ARG.
+int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kvq_dims* d,
+              DecodePlan* plan);
+
+// Number of SMs of the current device (148 if no device can be queried).
+int device_sm_count();
+
+// Kernel launchers (kvq_kernels.cu). They assume validated arguments and return
+// a cudaError_t value as int.
+int launch_append(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
+                  void* vc, void* ks, void* vs, kvq_fmt fmt, const kvq_dims& d, void* stream);
+int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* vc,
+                          const void* ks, const void* vs, const int32_t* tables,
+                          const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                          const DecodePlan& plan, void* ws, kvq_fmt fmt, const kvq_dims& d,
+                          void* stream);
+int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* out, bool out_f32,
+                        const void* ws, const DecodePlan& plan, const kvq_dims& d, void* stream);
+int read_device_error(uint32_t* flags, int clear);
+
+}  // namespace kvq

@@ -1,0 +1,594 @@
+// CUDA kernels of libkvq for sm_100a: quantize-on-append, paged GQA decode
+// attention (split-K partials) and the log-sum-exp merge.
+//
+// Sources (web pages, by title and section):
+//  "KV cache quantization: what FP8/INT8 K and V really give, and their limits"
+//     - "What KV cache quantization actually is": quantize only when storing,
+//       scale from the full BF16 values, BF16 per-token scales, dequantization
+//       fused into the attention kernel right before the matmuls.
+//     - "Formats you will actually meet": E4M3 for K/V; INT8 per-token
+//       asymmetric (scale, zero_point).
+//  "Fitting 76x concurrent requests with an FP8 KV cache" - "4. Precision
+//     loss?": 8-bit storage, FP32 accumulation of the attention dot products.
+//  "KV Cache compression" - "5.1 Quantization pipeline" (a separate dequant
+//     kernel gives the bandwidth gain back), "6.3" (quantize right after K/V
+//     are computed).
+//  "From FP8 KV cache to INT4 weight-only" - "Core concepts" 1) decode reads the
+//     whole cache once per step and is memory bound; 2) PagedAttention.
+//
+// Numerics that must match the oracle bit for bit (codes and scales):
+//  IEEE f32 division (__fdiv_rn), BF16 round-to-nearest-even of the scale,
+//  hardware E4M3 conversion with round-to-nearest-even and saturation, rint
+//  (ties to even) for INT8. This file is compiled without fast-math.
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+// Per-device error word (KVQ_DEVERR_* bits), read by kvq_device_error().
+__device__ unsigned int g_error_word;
+
+__device__ __forceinline__ void flag_error(unsigned int bit) { atomicOr(&g_error_word, bit); }
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_min(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Two E4M3 codes (low byte first) -> two floats (exact).
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t two_codes) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu),
+                                              __NV_E4M3);
+  return __half22float2(*reinterpret_cast<__half2*>(&h));
+}
+
+// Eight 1-byte codes held in a uint2 / four in a uint32 -> floats.
+template <int FMT>
+__device__ __forceinline__ void codes4_to_f32(uint32_t w, float* o) {
+  if constexpr (FMT == KVQ_FP8_E4M3) {
+    const float2 a = e4m3x2_to_f2(w), b = e4m3x2_to_f2(w >> 16);
+    o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+  } else {  // INT8: signed bytes
+    o[0] = float(int8_t(w & 0xff));
+    o[1] = float(int8_t((w >> 8) & 0xff));
+    o[2] = float(int8_t((w >> 16) & 0xff));
+    o[3] = float(int8_t(w >> 24));
+  }
+}
+
+// ------------------------------------------------------------------ append
+// One warp per (token, KV head, K|V) row of D BF16 values: E = D/32 values per
+// lane. Range reduction by warp shuffles, scale on every lane, encode, store.
+// K rows go to the page row [off][0..D); V rows go down the transposed page
+// column [0..D)[off].
+template <int D, int FMT>
+__global__ void __launch_bounds__(256) append_kernel(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const int64_t* __restrict__ slots, int T, int Hk, int NB, uint8_t* __restrict__ kc,
+    uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs) {
+  constexpr int E = D / 32;
+  constexpr int ELT = (FMT == KVQ_BF16) ? 2 : 1;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+  if (row >= int64_t(T) * Hk * 2) return;
+  const int which = int(row & 1);           // 0: K, 1: V
+  const int64_t th = row >> 1;
+  const int h = int(th % Hk);
+  const int64_t t = th / Hk;
+  const int64_t slot = slots[t];
+  if (slot < 0) return;
+  if (slot >= int64_t(NB) * kBlockSize) {
+    if (lane == 0) flag_error(KVQ_DEVERR_SLOT);
+    return;
+  }
+  const int64_t blk = slot / kBlockSize;
+  const int off = int(slot % kBlockSize);
+  const __nv_bfloat16* src = (which ? v : k) + (t * Hk + h) * D + lane * E;
+
+  // E BF16 values of this lane
+  uint32_t raw[E / 2];
+  if constexpr (E == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(src);
+    raw[0] = u.x; raw[1] = u.y;
+  } else {
+    raw[0] = *reinterpret_cast<const uint32_t*>(src);
+  }
+  float x[E];
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) { x[2 * i] = bf16_lo(raw[i]); x[2 * i + 1] = bf16_hi(raw[i]); }
+
+  const int64_t page = blk * Hk + h;                       // (block, head) page index
+  uint8_t* cache = which ? vc : kc;
+  __nv_bfloat16* meta = which ? vs : ks;
+
+  if constexpr (FMT == KVQ_BF16) {
+    if (which == 0) {
+      uint8_t* dst = cache + ((page * kBlockSize + off) * D + lane * E) * ELT;
+      if constexpr (E == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(raw[0], raw[1]);
+      else *reinterpret_cast<uint32_t*>(dst) = raw[0];
+    } else {
+      uint16_t* dst = reinterpret_cast<uint16_t*>(cache) + page * D * kBlockSize + off;
+#pragma unroll
+      for (int i = 0; i < E; ++i)
+        dst[(lane * E + i) * kBlockSize] = uint16_t(i & 1 ? raw[i / 2] >> 16 : raw[i / 2] & 0xffff);
+    }
+    return;
+  } else {
+    uint8_t code[E];
+    __nv_bfloat16 s_bf;
+    int zp = 0;
+    if constexpr (FMT == KVQ_FP8_E4M3) {
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(x[i]));
+      amax = warp_max(amax);
+      s_bf = __float2bfloat16_rn(__fdiv_rn(amax, 448.0f));
+      const float s = __bfloat162float(s_bf);
+#pragma unroll
+      for (int i = 0; i < E; i += 2) {
+        uint16_t two = 0;
+        if (s != 0.f) {
+          const float2 qv = make_float2(__fdiv_rn(x[i], s), __fdiv_rn(x[i + 1], s));
+          two = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
+        }
+        code[i] = uint8_t(two & 0xff);
+        code[i + 1] = uint8_t(two >> 8);
+      }
+    } else {  // INT8 asymmetric
+      float lo = 0.f, hi = 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) { lo = fminf(lo, x[i]); hi = fmaxf(hi, x[i]); }
+      lo = warp_min(lo);
+      hi = warp_max(hi);
+      s_bf = __float2bfloat16_rn(__fdiv_rn(__fsub_rn(hi, lo), 255.0f));
+      const float s = __bfloat162float(s_bf);
+      if (s != 0.f) {
+        const float zq = fminf(fmaxf(__fdiv_rn(lo, s), -1024.f), 1024.f);
+        zp = min(127, max(-128, -128 - __float2int_rn(zq)));
+      }
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        int c = 0;
+        if (s != 0.f) {
+          const float qf = fminf(fmaxf(__fdiv_rn(x[i], s), -1024.f), 1024.f);
+          c = min(127, max(-128, __float2int_rn(qf) + zp));
+        }
+        code[i] = uint8_t(int8_t(c));
+      }
+    }
+    if (which == 0) {
+      uint8_t* dst = cache + (page * kBlockSize + off) * D + lane * E;
+      if constexpr (E == 4)
+        *reinterpret_cast<uint32_t*>(dst) =
+            uint32_t(code[0]) | (uint32_t(code[1]) << 8) | (uint32_t(code[2]) << 16) | (uint32_t(code[3]) << 24);
+      else
+        *reinterpret_cast<uint16_t*>(dst) = uint16_t(code[0] | (code[1] << 8));
+    } else {
+      uint8_t* dst = cache + page * D * kBlockSize + off;
+#pragma unroll
+      for (int i = 0; i < E; ++i) dst[(lane * E + i) * kBlockSize] = code[i];
+    }
+    if (lane == 0) {
+      if constexpr (FMT == KVQ_FP8_E4M3) {
+        meta[page * kBlockSize + off] = s_bf;
+      } else {
+        meta[(page * kBlockSize + off) * 2] = s_bf;
+        meta[(page * kBlockSize + off) * 2 + 1] = __int2bfloat16_rn(zp);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ decode (CUDA cores)
+// One CTA of 4 warps per (sequence b, KV head h, chunk). Warp w takes pages
+// w, w+4, ... of the chunk. For a page of 16 tokens:
+//   QK: lane = (token t = lane & 15, half of head_dim); partial dot products
+//       over the half, completed with one xor-16 shuffle; every query head of
+//       the GQA group is done from the same K bytes, so each byte is read once.
+//   online softmax (base 2) per warp: page max by shuffles, rescale of the
+//       running sums by exp2(m_old - m_new).
+//   PV: the V page is stored transposed, so a lane owns D/32 channels and reads
+//       16 consecutive tokens per channel; the weights p*s_v of the page's 16
+//       tokens come from a small shared buffer.
+// Quantized values are never materialised: the K scale multiplies the finished
+// dot product, the V scale is folded into the softmax weight, and INT8 zero
+// points are subtracted as zp * sum(q) (K) and as sum(w * zp) (V).
+template <int D, int G, int FMT>
+struct SimtCfg {
+  static constexpr int ELT = (FMT == KVQ_BF16) ? 2 : 1;
+  static constexpr int KU4 = D * ELT / 32;          // uint4 per lane for a K half-row
+  static constexpr int ROWS = D / 32;               // V channels per lane
+  static constexpr int VU4 = ROWS * ELT;            // uint4 per lane for its V rows
+  static constexpr int PAGE_BYTES = kBlockSize * D * ELT;
+};
+
+template <int D, int G, int FMT>
+__global__ void __launch_bounds__(128) decode_simt_kernel(
+    const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kc,
+    const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
+    const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
+    const int32_t* __restrict__ ctx_lens, int Hk, int NB, int W, int max_ctx, int part,
+    int max_splits, float qscale, float* __restrict__ part_o, float* __restrict__ part_ml) {
+  using C = SimtCfg<D, G, FMT>;
+  constexpr int ELT = C::ELT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x % max_splits;
+  const int bh = blockIdx.x / max_splits;
+  const int b = bh / Hk, h = bh % Hk;
+  const int Hq = Hk * G;
+
+  __shared__ __align__(16) float qs[G][D];
+  __shared__ float qsum[G];
+  __shared__ __align__(16) float wsm[4][kBlockSize][G];
+  __shared__ float red_m[4][G], red_l[4][G];
+  __shared__ __align__(16) float red_o[4][G][D];
+
+  int ctx = ctx_lens[b];
+  const int64_t cap = int64_t(W) * kBlockSize;
+  if (ctx < 0 || ctx > max_ctx || ctx > cap) {
+    if (threadIdx.x == 0 && split == 0) flag_error(KVQ_DEVERR_CONTEXT);
+    ctx = 0;
+  }
+  const int n_splits = (ctx + part - 1) / part;
+  if (split >= n_splits) return;                 // the merge never reads this chunk
+  const int t0 = split * part, t1 = min(ctx, t0 + part);
+  const int p0 = t0 / kBlockSize, p1 = (t1 + kBlockSize - 1) / kBlockSize;
+
+  // query group of this KV head, pre-scaled into the base-2 softmax domain
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int g = i / D, d = i % D;
+    qs[g][d] = __bfloat162float(q[(int64_t(b) * Hq + h * G + g) * D + d]) * qscale;
+  }
+  __syncthreads();
+  if (threadIdx.x < G) {
+    float s = 0.f;
+    for (int d = 0; d < D; ++d) s += qs[threadIdx.x][d];
+    qsum[threadIdx.x] = s;
+  }
+  __syncthreads();
+
+  const int t_in = lane & 15, half = lane >> 4;
+  float m_run[G], l_part[G], corr_part[G], acc[G][C::ROWS];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m_run[g] = -INFINITY; l_part[g] = 0.f; corr_part[g] = 0.f;
+#pragma unroll
+    for (int j = 0; j < C::ROWS; ++j) acc[g][j] = 0.f;
+  }
+
+  const int32_t* trow = tables + int64_t(b) * W;
+  for (int pg = p0 + warp; pg < p1; pg += 4) {
+    const int blk = trow[pg];
+    if (blk < 0 || blk >= NB) {
+      if (lane == 0) flag_error(KVQ_DEVERR_BLOCK);
+      continue;
+    }
+    const int64_t page = int64_t(blk) * Hk + h;
+    const int nvalid = min(kBlockSize, t1 - pg * kBlockSize);
+    const bool valid = t_in < nvalid && pg * kBlockSize + t_in >= t0;
+
+    // ---- loads
+    uint4 kr[C::KU4], vr[C::VU4];
+    const uint4* kp = reinterpret_cast<const uint4*>(kc + page * C::PAGE_BYTES +
+                                                     (t_in * D + half * (D / 2)) * ELT);
+#pragma unroll
+    for (int i = 0; i < C::KU4; ++i) kr[i] = __ldg(kp + i);
+    const uint4* vp = reinterpret_cast<const uint4*>(vc + page * C::PAGE_BYTES) + lane * C::VU4;
+#pragma unroll
+    for (int i = 0; i < C::VU4; ++i) vr[i] = __ldg(vp + i);
+    float sk = 1.f, sv = 1.f, zk = 0.f, zv = 0.f;
+    if constexpr (FMT == KVQ_FP8_E4M3) {
+      sk = __bfloat162float(ks[page * kBlockSize + t_in]);
+      sv = __bfloat162float(vs[page * kBlockSize + t_in]);
+    } else if constexpr (FMT == KVQ_INT8_ASYM) {
+      const __nv_bfloat162 mk = reinterpret_cast<const __nv_bfloat162*>(ks)[page * kBlockSize + t_in];
+      const __nv_bfloat162 mv = reinterpret_cast<const __nv_bfloat162*>(vs)[page * kBlockSize + t_in];
+      sk = __low2float(mk); zk = __high2float(mk);
+      sv = __low2float(mv); zv = __high2float(mv);
+    }
+
+    // ---- QK over this lane's half of head_dim
+    float dot[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) dot[g] = 0.f;
+    const uint32_t* kw = reinterpret_cast<const uint32_t*>(kr);
+#pragma unroll
+    for (int i = 0; i < C::KU4 * 4; ++i) {       // 32-bit words
+      float kv[4];
+      int nv;
+      if constexpr (FMT == KVQ_BF16) {
+        kv[0] = bf16_lo(kw[i]); kv[1] = bf16_hi(kw[i]); nv = 2;
+      } else {
+        codes4_to_f32<FMT>(kw[i], kv); nv = 4;
+      }
+      const int d0 = half * (D / 2) + i * nv;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (e < nv) dot[g] = fmaf(qs[g][d0 + e], kv[e], dot[g]);
+      }
+    }
+    float x[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float full = dot[g] + __shfl_xor_sync(0xffffffffu, dot[g], 16);
+      if constexpr (FMT == KVQ_FP8_E4M3) full *= sk;
+      if constexpr (FMT == KVQ_INT8_ASYM) full = (full - zk * qsum[g]) * sk;
+      x[g] = valid ? full : -INFINITY;
+    }
+
+    // ---- online softmax for the page
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float pm = x[g];
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, o));
+      const float m_new = fmaxf(m_run[g], pm);
+      const float alpha = exp2f(m_run[g] - m_new);     // 0 when m_run is -inf
+      const float p = valid ? exp2f(x[g] - m_new) : 0.f;
+      m_run[g] = m_new;
+      l_part[g] = l_part[g] * alpha + (half == 0 ? p : 0.f);
+#pragma unroll
+      for (int j = 0; j < C::ROWS; ++j) acc[g][j] *= alpha;
+      const float w = valid ? p * sv : 0.f;
+      if constexpr (FMT == KVQ_INT8_ASYM)
+        corr_part[g] = corr_part[g] * alpha + (half == 0 && valid ? w * zv : 0.f);
+      if (half == 0) wsm[warp][t_in][g] = w;
+    }
+    __syncwarp();
+
+    // ---- PV: this lane's channels, 16 tokens each
+    if (nvalid < kBlockSize) {                       // zero the tokens past the end
+#pragma unroll
+      for (int j = 0; j < C::ROWS; ++j) {
+#pragma unroll
+        for (int wd = 0; wd < 4 * ELT; ++wd) {
+          uint32_t* u = reinterpret_cast<uint32_t*>(&vr[j * ELT]) + wd;
+          const int tok0 = wd * 4 / ELT;           // first token in this word
+          uint32_t keep = 0;
+#pragma unroll
+          for (int bq = 0; bq < 4; ++bq)
+            if (tok0 + bq / ELT < nvalid) keep |= 0xffu << (8 * bq);
+          *u &= keep;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < C::ROWS; ++j) {
+      const uint32_t* vw = reinterpret_cast<const uint32_t*>(&vr[j * ELT]);
+#pragma unroll
+      for (int wd = 0; wd < 4 * ELT; ++wd) {
+        float vv[4];
+        int nv;
+        if constexpr (FMT == KVQ_BF16) {
+          vv[0] = bf16_lo(vw[wd]); vv[1] = bf16_hi(vw[wd]); nv = 2;
+        } else {
+          codes4_to_f32<FMT>(vw[wd], vv); nv = 4;
+        }
+        const int tb = wd * nv;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (e < nv) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) acc[g][j] = fmaf(wsm[warp][tb + e][g], vv[e], acc[g][j]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  // ---- combine the 4 warps of the CTA and write the chunk's partial
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float l = warp_sum(l_part[g]);
+    const float corr = warp_sum(corr_part[g]);
+    if (lane == 0) { red_m[warp][g] = m_run[g]; red_l[warp][g] = l; }
+#pragma unroll
+    for (int j = 0; j < C::ROWS; ++j) {
+      float a = acc[g][j];
+      if constexpr (FMT == KVQ_INT8_ASYM) a -= corr;
+      red_o[warp][g][lane * C::ROWS + j] = a;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int g = i / D, d = i % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w][g]);
+    float o = 0.f, l = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float f = (M == -INFINITY) ? 0.f : exp2f(red_m[w][g] - M);
+      o += red_o[w][g][d] * f;
+      l += red_l[w][g] * f;
+    }
+    const int64_t r = (int64_t(b) * Hq + h * G + g) * max_splits + split;
+    part_o[r * D + d] = o;
+    if (d == 0) { part_ml[r * 2] = M; part_ml[r * 2 + 1] = l; }
+  }
+}
+
+// ------------------------------------------------------------------ merge
+// One CTA of D threads per (sequence, query head): combine the chunk partials
+// (m_i, l_i, o_i) as m = max m_i, l = sum l_i 2^(m_i - m), o = sum o_i 2^(m_i - m) / l.
+template <int D, typename OutT>
+__global__ void __launch_bounds__(128) merge_kernel(const int32_t* __restrict__ ctx_lens, int Hq,
+                                                    int part, int max_splits, int max_ctx, int W,
+                                                    const float* __restrict__ part_o,
+                                                    const float* __restrict__ part_ml,
+                                                    OutT* __restrict__ out) {
+  const int bq = blockIdx.x;                 // b * Hq + head
+  const int b = bq / Hq;
+  const int d = threadIdx.x;
+  int ctx = ctx_lens[b];
+  if (ctx < 0 || ctx > max_ctx || int64_t(ctx) > int64_t(W) * kBlockSize) ctx = 0;
+  const int n = (ctx + part - 1) / part;
+  const int64_t r0 = int64_t(bq) * max_splits;
+  float M = -INFINITY;
+  for (int s = 0; s < n; ++s) M = fmaxf(M, part_ml[(r0 + s) * 2]);
+  float o = 0.f, l = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < n; ++s) {
+      const float f = exp2f(part_ml[(r0 + s) * 2] - M);
+      l += part_ml[(r0 + s) * 2 + 1] * f;
+      o += part_o[(r0 + s) * D + d] * f;
+    }
+  }
+  const float r = l > 0.f ? o / l : 0.f;
+  if constexpr (sizeof(OutT) == 4) out[int64_t(bq) * D + d] = r;
+  else out[int64_t(bq) * D + d] = __float2bfloat16_rn(r);
+}
+
+// ------------------------------------------------------------------ launchers
+namespace {
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D, int FMT>
+cudaError_t append_dispatch(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
+                            void* vc, void* ks, void* vs, const kvq_dims& d, cudaStream_t st) {
+  const int64_t rows = int64_t(T) * d.n_kv_heads * 2;
+  const int warps = 8;
+  const int64_t grid = (rows + warps - 1) / warps;
+  append_kernel<D, FMT><<<dim3(unsigned(grid)), 32 * warps, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), slots, T,
+      d.n_kv_heads, d.num_blocks, static_cast<uint8_t*>(kc), static_cast<uint8_t*>(vc),
+      static_cast<__nv_bfloat16*>(ks), static_cast<__nv_bfloat16*>(vs));
+  return cudaGetLastError();
+}
+
+template <int D, int G, int FMT>
+cudaError_t decode_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
+                             const void* ks, const void* vs, const int32_t* tables,
+                             const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                             const DecodePlan& plan, void* ws, const kvq_dims& d,
+                             cudaStream_t st) {
+  float* po = static_cast<float*>(ws);
+  float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
+  const int64_t grid = int64_t(B) * d.n_kv_heads * plan.max_splits;
+  decode_simt_kernel<D, G, FMT><<<dim3(unsigned(grid)), 128, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
+      static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
+      static_cast<const __nv_bfloat16*>(vs), tables, ctx, d.n_kv_heads, d.num_blocks,
+      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml);
+  return cudaGetLastError();
+}
+
+template <int D, int FMT>
+cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, const void* vc,
+                             const void* ks, const void* vs, const int32_t* tables,
+                             const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                             const DecodePlan& plan, void* ws, const kvq_dims& d,
+                             cudaStream_t st) {
+  switch (G) {
+    case 1: return decode_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+    case 2: return decode_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+    case 4: return decode_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+    default: return decode_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+  }
+}
+}  // namespace
+
+int launch_append(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
+                  void* vc, void* ks, void* vs, kvq_fmt fmt, const kvq_dims& d, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d.head_dim == 128) {
+    if (fmt == KVQ_FP8_E4M3) e = append_dispatch<128, KVQ_FP8_E4M3>(k, v, slots, T, kc, vc, ks, vs, d, st);
+    else if (fmt == KVQ_INT8_ASYM) e = append_dispatch<128, KVQ_INT8_ASYM>(k, v, slots, T, kc, vc, ks, vs, d, st);
+    else e = append_dispatch<128, KVQ_BF16>(k, v, slots, T, kc, vc, ks, vs, d, st);
+  } else {
+    if (fmt == KVQ_FP8_E4M3) e = append_dispatch<64, KVQ_FP8_E4M3>(k, v, slots, T, kc, vc, ks, vs, d, st);
+    else if (fmt == KVQ_INT8_ASYM) e = append_dispatch<64, KVQ_INT8_ASYM>(k, v, slots, T, kc, vc, ks, vs, d, st);
+    else e = append_dispatch<64, KVQ_BF16>(k, v, slots, T, kc, vc, ks, vs, d, st);
+  }
+  return int(e);
+}
+
+int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* vc,
+                          const void* ks, const void* vs, const int32_t* tables,
+                          const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                          const DecodePlan& plan, void* ws, kvq_fmt fmt, const kvq_dims& d,
+                          void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = d.n_q_heads / d.n_kv_heads;
+  cudaError_t e;
+#define KVQ_DEC(DD, FF) decode_dispatch2<DD, FF>(G, q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st)
+  if (d.head_dim == 128) {
+    if (fmt == KVQ_FP8_E4M3) e = KVQ_DEC(128, KVQ_FP8_E4M3);
+    else if (fmt == KVQ_INT8_ASYM) e = KVQ_DEC(128, KVQ_INT8_ASYM);
+    else e = KVQ_DEC(128, KVQ_BF16);
+  } else {
+    if (fmt == KVQ_FP8_E4M3) e = KVQ_DEC(64, KVQ_FP8_E4M3);
+    else if (fmt == KVQ_INT8_ASYM) e = KVQ_DEC(64, KVQ_INT8_ASYM);
+    else e = KVQ_DEC(64, KVQ_BF16);
+  }
+#undef KVQ_DEC
+  return int(e);
+}
+
+int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* out, bool out_f32,
+                        const void* ws, const DecodePlan& plan, const kvq_dims& d, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float* po = static_cast<const float*>(ws);
+  const float* pml = reinterpret_cast<const float*>(static_cast<const char*>(ws) + plan.o_bytes);
+  const dim3 grid(unsigned(int64_t(B) * d.n_q_heads));
+  const int W = d.max_blocks_per_seq, Hq = d.n_q_heads;
+  if (d.head_dim == 128) {
+    if (out_f32)
+      merge_kernel<128, float><<<grid, 128, 0, st>>>(ctx, Hq, plan.partition, plan.max_splits,
+          max_ctx, W, po, pml, static_cast<float*>(out));
+    else
+      merge_kernel<128, __nv_bfloat16><<<grid, 128, 0, st>>>(ctx, Hq, plan.partition,
+          plan.max_splits, max_ctx, W, po, pml, static_cast<__nv_bfloat16*>(out));
+  } else {
+    if (out_f32)
+      merge_kernel<64, float><<<grid, 64, 0, st>>>(ctx, Hq, plan.partition, plan.max_splits,
+          max_ctx, W, po, pml, static_cast<float*>(out));
+    else
+      merge_kernel<64, __nv_bfloat16><<<grid, 64, 0, st>>>(ctx, Hq, plan.partition,
+          plan.max_splits, max_ctx, W, po, pml, static_cast<__nv_bfloat16*>(out));
+  }
+  return int(cudaGetLastError());
+}
+
+int read_device_error(uint32_t* flags, int clear) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return int(e);
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v));
+  if (e != cudaSuccess) return int(e);
+  *flags = v;
+  if (clear && v) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return int(e);
+  }
+  return 0;
+}
+
+}  // namespace kvq

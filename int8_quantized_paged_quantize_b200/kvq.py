@@ -1,0 +1,297 @@
+"""Thin ctypes binding of libkvq (include/kvq.h).
+
+Argument marshalling only: PyTorch tensors supply device pointers, the current
+CUDA stream supplies the stream; every computation runs in the library's CUDA
+kernels. If ``libkvq.so`` is missing or a call fails, a ``KvqError`` is raised;
+there is no CPU path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
+
+FMT = {"bf16": 0, "fp8": 1, "int8": 2}
+ELEM_BYTES = {"bf16": 2, "fp8": 1, "int8": 1}
+META_VALUES = {"bf16": 0, "fp8": 1, "int8": 2}
+BLOCK_SIZE = 16
+
+DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT = 0x1, 0x2, 0x4
+
+# Every function the header declares: (name, restype, argtypes)
+_c = ctypes
+_P = _c.c_void_p
+_SIGNATURES = [
+    ("kvq_version", _c.c_int, []),
+    ("kvq_status_string", _c.c_char_p, [_c.c_int]),
+    ("kvq_cache_bytes", _c.c_int, [_P, _c.c_int, _c.POINTER(_c.c_size_t), _c.POINTER(_c.c_size_t)]),
+    ("kvq_pool_create", _c.c_int, [_P, _c.c_int, _c.c_int32, _c.POINTER(_P)]),
+    ("kvq_pool_destroy", None, [_P]),
+    ("kvq_pool_bytes", _c.c_int, [_P, _c.POINTER(_c.c_size_t), _c.POINTER(_c.c_size_t)]),
+    ("kvq_pool_num_free", _c.c_int, [_P, _c.POINTER(_c.c_int32)]),
+    ("kvq_pool_alloc", _c.c_int, [_P, _c.c_int32, _P]),
+    ("kvq_pool_free", _c.c_int, [_P, _c.c_int32, _P]),
+    ("kvq_pool_extend_seq", _c.c_int, [_P, _P, _c.c_int32, _c.c_int32, _P]),
+    ("kvq_append", _c.c_int, [_P, _P, _P, _c.c_int32, _P, _P, _P, _P, _c.c_int, _P, _P]),
+    ("kvq_decode_workspace_bytes", _c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _P]),
+    ("kvq_decode_attn", _c.c_int, [_P, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32, _c.c_float, _P,
+                                   _c.c_int, _P, _c.c_size_t, _c.c_int32, _c.c_int, _P, _P]),
+    ("kvq_decode_partial", _c.c_int, [_P, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32, _c.c_float,
+                                      _P, _c.c_size_t, _c.c_int32, _c.c_int, _P, _P]),
+    ("kvq_decode_merge", _c.c_int, [_c.c_int32, _P, _c.c_int32, _P, _c.c_int, _P, _c.c_size_t,
+                                    _c.c_int32, _c.c_int, _P, _P]),
+    ("kvq_device_error", _c.c_int, [_c.POINTER(_c.c_uint32), _c.c_int]),
+]
+
+_lib = None
+
+
+class KvqError(RuntimeError):
+    pass
+
+
+def lib():
+    """The loaded libkvq (raises KvqError if the library has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise KvqError(f"libkvq.so not built (expected at {_LIB_PATH}); "
+                           "run python -m int8_quantized_paged_quantize_b200.build")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, res, args in _SIGNATURES:
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        msg = lib().kvq_status_string(rc).decode()
+        raise KvqError(f"{what}: {msg} (status {rc})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32)]
+
+
+def dims(num_blocks, n_kv_heads, n_q_heads, head_dim, max_blocks_per_seq, block_size=BLOCK_SIZE):
+    return Dims(num_blocks, block_size, n_kv_heads, n_q_heads, head_dim, max_blocks_per_seq)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _out_dtype(out):
+    if out.dtype == torch.bfloat16:
+        return 0
+    if out.dtype == torch.float32:
+        return 1
+    raise KvqError("out must be bfloat16 or float32")
+
+
+def _need(t, dtype, name):
+    if not t.is_cuda or not t.is_contiguous() or t.dtype != dtype:
+        raise KvqError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+# --------------------------------------------------------------------------- sizes / allocator
+def cache_bytes(d: Dims, fmt: str):
+    cb, mb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().kvq_cache_bytes(ctypes.byref(d), FMT[fmt], ctypes.byref(cb), ctypes.byref(mb)),
+           "kvq_cache_bytes")
+    return cb.value, mb.value
+
+
+class Pool:
+    """Host block allocator (kvq_pool_*)."""
+
+    def __init__(self, d: Dims, fmt: str, n_layers: int = 1):
+        self._d = d
+        h = ctypes.c_void_p()
+        _check(lib().kvq_pool_create(ctypes.byref(d), FMT[fmt], n_layers, ctypes.byref(h)),
+               "kvq_pool_create")
+        self._h = h
+
+    def close(self):
+        if self._h:
+            lib().kvq_pool_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def bytes(self):
+        eb, mb = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().kvq_pool_bytes(self._h, ctypes.byref(eb), ctypes.byref(mb)), "kvq_pool_bytes")
+        return eb.value, mb.value
+
+    def num_free(self):
+        n = ctypes.c_int32()
+        _check(lib().kvq_pool_num_free(self._h, ctypes.byref(n)), "kvq_pool_num_free")
+        return n.value
+
+    def alloc(self, n):
+        ids = (ctypes.c_int32 * max(n, 1))()
+        _check(lib().kvq_pool_alloc(self._h, n, ids), "kvq_pool_alloc")
+        return list(ids[:n])
+
+    def free(self, ids):
+        arr = (ctypes.c_int32 * max(len(ids), 1))(*ids)
+        _check(lib().kvq_pool_free(self._h, len(ids), arr), "kvq_pool_free")
+
+    def extend_seq(self, row, cur_len, n_new):
+        """row: a mutable list of max_blocks_per_seq ints (updated in place); returns slots."""
+        arr = (ctypes.c_int32 * len(row))(*row)
+        slots = (ctypes.c_int64 * max(n_new, 1))()
+        _check(lib().kvq_pool_extend_seq(self._h, arr, cur_len, n_new, slots), "kvq_pool_extend_seq")
+        row[:] = list(arr)
+        return list(slots[:n_new])
+
+
+# --------------------------------------------------------------------------- hot calls
+def append(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale, fmt: str, d: Dims, stream=None):
+    """Quantize-on-append (kvq_append). k, v: [T][Hk][D] bf16; slot_mapping [T] int64."""
+    _need(k, torch.bfloat16, "k")
+    _need(v, torch.bfloat16, "v")
+    _need(slot_mapping, torch.int64, "slot_mapping")
+    T = slot_mapping.numel()
+    _check(lib().kvq_append(_ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_cache), _ptr(v_cache),
+                            _ptr(k_scale), _ptr(v_scale), FMT[fmt], ctypes.byref(d),
+                            _stream(stream)), "kvq_append")
+
+
+def decode_workspace_bytes(batch, max_context_len, fmt, d: Dims, partition_tokens=0):
+    n = lib().kvq_decode_workspace_bytes(batch, max_context_len, partition_tokens, FMT[fmt],
+                                         ctypes.byref(d))
+    if n == 0 and batch > 0:
+        raise KvqError("kvq_decode_workspace_bytes: invalid arguments")
+    return n
+
+
+def _scales(k_scale, v_scale):
+    arr = (ctypes.c_void_p * 2)(k_scale.data_ptr() if k_scale is not None else 0,
+                                v_scale.data_ptr() if v_scale is not None else 0)
+    return arr
+
+
+def decode_attn(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                max_context_len, sm_scale, out, workspace, fmt: str, d: Dims,
+                partition_tokens=0, stream=None):
+    """Paged GQA decode attention (kvq_decode_attn): partials + merge into out."""
+    _need(q, torch.bfloat16, "q")
+    _need(out, out.dtype, "out")
+    _need(block_tables, torch.int32, "block_tables")
+    _need(context_lens, torch.int32, "context_lens")
+    B = q.shape[0]
+    _check(lib().kvq_decode_attn(_ptr(q), B, _ptr(k_cache), _ptr(v_cache), _scales(k_scale, v_scale),
+                                 _ptr(block_tables), _ptr(context_lens), int(max_context_len),
+                                 float(sm_scale), _ptr(out), _out_dtype(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), partition_tokens,
+                                 FMT[fmt], ctypes.byref(d), _stream(stream)), "kvq_decode_attn")
+
+
+def decode_partial(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                   max_context_len, sm_scale, workspace, fmt: str, d: Dims, partition_tokens=0,
+                   stream=None):
+    B = q.shape[0]
+    _check(lib().kvq_decode_partial(_ptr(q), B, _ptr(k_cache), _ptr(v_cache),
+                                    _scales(k_scale, v_scale), _ptr(block_tables),
+                                    _ptr(context_lens), int(max_context_len), float(sm_scale),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    partition_tokens, FMT[fmt], ctypes.byref(d), _stream(stream)),
+           "kvq_decode_partial")
+
+
+def decode_merge(batch, context_lens, max_context_len, out, workspace, fmt: str, d: Dims,
+                 partition_tokens=0, stream=None):
+    _check(lib().kvq_decode_merge(batch, _ptr(context_lens), int(max_context_len), _ptr(out),
+                                  _out_dtype(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  partition_tokens, FMT[fmt], ctypes.byref(d), _stream(stream)),
+           "kvq_decode_merge")
+
+
+def device_error(clear=True) -> int:
+    """KVQ_DEVERR_* bits flagged by kernels on the current device (synchronizes)."""
+    f = ctypes.c_uint32()
+    rc = lib().kvq_device_error(ctypes.byref(f), 1 if clear else 0)
+    if rc not in (0, -6):
+        _check(rc, "kvq_device_error")
+    return f.value
+
+
+# --------------------------------------------------------------------------- convenience
+@dataclass
+class LayerCache:
+    """Device buffers of one layer's quantized K/V cache (torch-owned memory)."""
+    fmt: str
+    dims: Dims
+    k: torch.Tensor
+    v: torch.Tensor
+    k_scale: torch.Tensor | None
+    v_scale: torch.Tensor | None
+
+    @staticmethod
+    def allocate(fmt, d: Dims, device="cuda"):
+        nb, hk, D = d.num_blocks, d.n_kv_heads, d.head_dim
+        edt = torch.bfloat16 if fmt == "bf16" else torch.uint8
+        k = torch.zeros((nb, hk, BLOCK_SIZE, D), dtype=edt, device=device)
+        v = torch.zeros((nb, hk, D, BLOCK_SIZE), dtype=edt, device=device)
+        mv = META_VALUES[fmt]
+        if mv:
+            shape = (nb, hk, BLOCK_SIZE) if mv == 1 else (nb, hk, BLOCK_SIZE, 2)
+            ks = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+            vs = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        else:
+            ks = vs = None
+        return LayerCache(fmt, d, k, v, ks, vs)
+
+    def append(self, k, v, slot_mapping, stream=None):
+        append(k, v, slot_mapping, self.k, self.v, self.k_scale, self.v_scale, self.fmt, self.dims,
+               stream)
+
+    def workspace(self, batch, max_context_len, partition_tokens=0, device="cuda"):
+        n = decode_workspace_bytes(batch, max_context_len, self.fmt, self.dims, partition_tokens)
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+    def decode(self, q, block_tables, context_lens, max_context_len, sm_scale=None, out=None,
+               workspace=None, partition_tokens=0, stream=None, out_dtype=torch.bfloat16):
+        if sm_scale is None:
+            sm_scale = 1.0 / math.sqrt(self.dims.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        if workspace is None:
+            workspace = self.workspace(q.shape[0], max_context_len, partition_tokens, q.device)
+        decode_attn(q, self.k, self.v, self.k_scale, self.v_scale, block_tables, context_lens,
+                    max_context_len, sm_scale, out, workspace, self.fmt, self.dims,
+                    partition_tokens, stream)
+        return out
+
+    # ---- views in the logical layout [NB][Hk][bs][D] (for inspection and tests)
+    def k_logical(self):
+        return self.k
+
+    def v_logical(self):
+        return self.v.transpose(2, 3)

@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import math
 import zlib
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 
 import numpy as np
 import torch
@@ -45,7 +45,6 @@ class Workload:
     pool: str = "shuffled"        # shuffled | permutation16 | fragmented
     bulk_append: int = 0          # tokens appended per sequence in one bulk call before decode
     decode_steps: int = 1
-    extra: dict = field(default_factory=dict)
 
     @property
     def group(self) -> int:

@@ -1,0 +1,203 @@
+"""Helpers for the GPU parity tests: run one workload through libkvq (append of the
+cached history, append of the step's tokens, decode) and through the CPU oracle
+on the same seeded inputs, then compare.
+
+Comparison rules:
+  * cache codes and BF16 scales/zero points: bit-exact;
+  * attention output (FP32 out of the kernel) vs the oracle's FP64 attention
+    over the same dequantised K/V: max |err| <= 4e-3 and mean |err| <= 5e-4.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+
+import numpy as np
+import torch
+
+from int8_quantized_paged_quantize_b200 import kvq
+from int8_quantized_paged_quantize_b200 import workloads as W
+from oracle import attention as OA
+from oracle import formats as OF
+
+MAX_ABS = 4e-3
+MEAN_ABS = 5e-4
+
+
+@dataclass
+class GpuRun:
+    w: W.Workload
+    fmt: str
+    cache: kvq.LayerCache
+    tables: np.ndarray          # [B][W] int32
+    ctx_before: np.ndarray      # cached tokens before the step (history + bulk append)
+    ctx_after: np.ndarray       # attended tokens (step token included)
+    q: torch.Tensor             # [B][Hq][D] bf16 (CPU)
+    k_new: torch.Tensor
+    v_new: torch.Tensor
+    out: torch.Tensor           # [B][Hq][D] (CPU, dtype of the run)
+    seed: int = 0
+
+
+def slots_for(tables, b, positions, bs=16):
+    positions = np.asarray(positions, dtype=np.int64)
+    return tables[b][positions // bs].astype(np.int64) * bs + positions % bs
+
+
+def with_lengths(w: W.Workload, ctx_list):
+    """The same shapes with an explicit list of cached lengths (no bulk append)."""
+    return replace(w, lengths="list", ctx=tuple(int(c) for c in ctx_list),
+                   batch=len(ctx_list), bulk_append=0, decode_steps=1)
+
+
+_INPUTS = {}
+
+
+def inputs(w: W.Workload, seed=0):
+    """Seeded inputs of one workload, generated once per process: per-sequence
+    history and bulk-append K/V (BF16, CPU) and the first step's q/k/v."""
+    key = (w, seed)
+    if key not in _INPUTS:
+        hist = [W.kv_history(w, b, seed) for b in range(w.batch)]
+        bulk = [W.kv_bulk(w, b, seed) for b in range(w.batch)] if w.bulk_append else None
+        _INPUTS.clear()                      # keep one workload's data at a time
+        _INPUTS[key] = (hist, bulk, W.step_inputs(w, 0, seed))
+    return _INPUTS[key]
+
+
+def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch.float32,
+            history_chunks=1):
+    """Append every sequence's cached history (in `history_chunks` calls), then the
+    bulk append if the workload has one, then one token per sequence, and run one
+    decode step over ctx + 1 tokens. Returns a GpuRun."""
+    tables, nb = W.block_tables(w, seed)
+    ctx = W.context_lengths(w, seed)
+    hist, bulk, (q, k_new, v_new) = inputs(w, seed)
+    d = kvq.dims(nb, w.n_kv_heads, w.n_q_heads, w.head_dim, tables.shape[1])
+    cache = kvq.LayerCache.allocate(fmt, d)
+    dev = torch.device("cuda")
+    S = [torch.from_numpy(slots_for(tables, b, np.arange(ctx[b]))) for b in range(w.batch)]
+    S = torch.cat(S) if S else torch.zeros(0, dtype=torch.int64)
+    n = S.numel()
+    if n:
+        K = torch.cat([h[0] for h in hist])
+        V = torch.cat([h[1] for h in hist])
+        bounds = np.linspace(0, n, history_chunks + 1).astype(int)
+        for a, z in zip(bounds[:-1], bounds[1:]):
+            if z > a:
+                cache.append(K[a:z].to(dev), V[a:z].to(dev), S[a:z].to(dev))
+        del K, V
+    if bulk is not None:
+        nb_tok = w.bulk_append
+        K = torch.cat([x[0] for x in bulk]).to(dev)
+        V = torch.cat([x[1] for x in bulk]).to(dev)
+        S = torch.cat([torch.from_numpy(slots_for(tables, b, ctx[b] + np.arange(nb_tok)))
+                       for b in range(w.batch)]).to(dev)
+        cache.append(K, V, S)
+        del K, V
+        ctx = ctx + nb_tok
+    step_slots = torch.from_numpy(np.array([slots_for(tables, b, [ctx[b]])[0]
+                                            for b in range(w.batch)], dtype=np.int64))
+    cache.append(k_new.to(dev), v_new.to(dev), step_slots.to(dev))
+    ctx_after = ctx + 1
+    tbl = torch.from_numpy(tables).to(dev)
+    cl = torch.from_numpy(ctx_after.astype(np.int32)).to(dev)
+    out = cache.decode(q.to(dev), tbl, cl, int(ctx_after.max()), sm_scale=w.sm_scale,
+                       partition_tokens=partition_tokens, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert kvq.device_error(clear=True) == 0
+    return GpuRun(w, fmt, cache, tables, ctx, ctx_after, q, k_new, v_new, out.cpu(), seed)
+
+
+# ----------------------------------------------------------------------------- oracle side
+def oracle_sequence(run: GpuRun, b: int):
+    """Oracle codes/scales and dequantised K/V of sequence b's ctx_after tokens,
+    quantised by the oracle from the same seeded BF16 inputs.
+
+    Returns dict with 'k_codes','v_codes' [n][Hk][D], 'k_scale','v_scale' [n][Hk],
+    'k_zp','v_zp', 'K','V' float64 [n][Hk][D] and the raw BF16 'Kraw','Vraw'."""
+    w = run.w
+    hist, bulk, _ = inputs(w, run.seed)
+    parts_k, parts_v = [hist[b][0]], [hist[b][1]]
+    if bulk is not None:
+        parts_k.append(bulk[b][0])
+        parts_v.append(bulk[b][1])
+    k = torch.cat(parts_k + [run.k_new[b:b + 1]]).float().numpy()
+    v = torch.cat(parts_v + [run.v_new[b:b + 1]]).float().numpy()
+    res = {"Kraw": k.astype(np.float64), "Vraw": v.astype(np.float64)}
+    for name, x in (("k", k), ("v", v)):
+        if run.fmt == "fp8":
+            c, s = OF.fp8_quantize(x)
+            res[name + "_codes"], res[name + "_scale"] = c, s
+            res[name.upper()] = OF.fp8_dequantize(c, s)
+        elif run.fmt == "int8":
+            c, s, z = OF.int8_quantize(x)
+            res[name + "_codes"], res[name + "_scale"], res[name + "_zp"] = c, s, z
+            res[name.upper()] = OF.int8_dequantize(c, s, z)
+        else:
+            res[name + "_codes"] = OF.bf16_round(x)
+            res[name.upper()] = x.astype(np.float64)
+    return res
+
+
+def gpu_sequence(run: GpuRun, b: int):
+    """The GPU cache contents of sequence b's ctx_after tokens in logical order:
+    codes [n][Hk][D] and metadata [n][Hk] (scale, zero point)."""
+    n = int(run.ctx_after[b])
+    pages = int(math.ceil(n / 16))
+    ids = torch.from_numpy(run.tables[b][:pages].astype(np.int64)).to(run.cache.k.device)
+    kl = run.cache.k_logical()[ids]                      # [pages][Hk][16][D]
+    vl = run.cache.v_logical()[ids]
+    kl = kl.permute(0, 2, 1, 3).reshape(pages * 16, kl.shape[1], kl.shape[3])[:n].cpu()
+    vl = vl.permute(0, 2, 1, 3).reshape(pages * 16, vl.shape[1], vl.shape[3])[:n].cpu()
+    out = {"k_codes": kl, "v_codes": vl}
+    if run.fmt != "bf16":
+        for name, t in (("k", run.cache.k_scale), ("v", run.cache.v_scale)):
+            m = t[ids]                                       # [pages][Hk][16](,2)
+            if run.fmt == "fp8":
+                m = m.permute(0, 2, 1).reshape(pages * 16, -1)[:n].float().cpu().numpy()
+                out[name + "_scale"] = m
+            else:
+                m = m.permute(0, 2, 1, 3).reshape(pages * 16, m.shape[1], 2)[:n].float().cpu().numpy()
+                out[name + "_scale"] = m[..., 0]
+                out[name + "_zp"] = m[..., 1]
+    return out
+
+
+def assert_codes_equal(run: GpuRun, b: int, ref: dict):
+    g = gpu_sequence(run, b)
+    for name in ("k", "v"):
+        gc = g[name + "_codes"]
+        if run.fmt == "bf16":
+            assert torch.equal(gc.float(), torch.from_numpy(ref[name + "_codes"])), name
+        elif run.fmt == "fp8":
+            assert np.array_equal(gc.numpy(), ref[name + "_codes"]), f"{name} codes b={b}"
+        else:
+            assert np.array_equal(gc.numpy().view(np.int8), ref[name + "_codes"]), f"{name} codes b={b}"
+        if run.fmt != "bf16":
+            assert np.array_equal(OF.bf16_bits(g[name + "_scale"]), OF.bf16_bits(ref[name + "_scale"])), \
+                f"{name} scales b={b}"
+        if run.fmt == "int8":
+            assert np.array_equal(g[name + "_zp"], ref[name + "_zp"].astype(np.float32)), f"{name} zp b={b}"
+
+
+def oracle_attention(run: GpuRun, b: int, ref: dict, raw=False):
+    """FP64 attention of sequence b, [Hq][D]: over the dequantised cache, or with
+    raw=True over the unquantised BF16 values (the quality reference)."""
+    K, V = (ref["Kraw"], ref["Vraw"]) if raw else (ref["K"], ref["V"])
+    q = run.q[b:b + 1].float().numpy().astype(np.float64)
+    return OA.decode_attention(q, [(K, V)], run.w.sm_scale, run.w.n_kv_heads)[0]
+
+
+def attention_errors(run: GpuRun, seqs, check_codes=True):
+    """(max abs err, mean abs err) of the GPU output vs the oracle over `seqs`."""
+    errs = []
+    for b in seqs:
+        ref = oracle_sequence(run, b)
+        if check_codes:
+            assert_codes_equal(run, b, ref)
+        o = oracle_attention(run, b, ref)
+        errs.append(np.abs(run.out[b].float().numpy().astype(np.float64) - o).ravel())
+    e = np.concatenate(errs) if errs else np.zeros(1)
+    return float(e.max()), float(e.mean())
