@@ -250,6 +250,38 @@ int kvq_decode_merge(int32_t batch, const int32_t* context_lens, int32_t max_con
                      kvq_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Decode without a caller workspace. The pages have no counterpart to this:   */
+/* it is kvq_decode_attn with its scratch taken from the library itself.       */
+/* ------------------------------------------------------------------------ */
+/* Size of the scratch array compiled into the library (64 MiB per device). */
+#define KVQ_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * Same arguments, result and errors as kvq_decode_attn, minus the workspace.
+ * For callers that cannot allocate device memory while decoding (a plugin
+ * inside another framework's step, where the framework owns all device memory;
+ * a latency-critical loop that must not hit the device synchronisation of
+ * cudaMalloc/cudaFree). The split-K scratch comes from one static device array
+ * of KVQ_NOALLOC_SCRATCH_BYTES, held by every GPU that loads the library until
+ * the process exits; the call allocates nothing.
+ * - Returns KVQ_ERR_WORKSPACE, before touching the device, when the split plan
+ *   (kvq_decode_workspace_bytes for the same arguments) needs more than
+ *   KVQ_NOALLOC_SCRATCH_BYTES; use a larger partition_tokens or kvq_decode_attn.
+ * - The first call on each device looks up the array's device address (with
+ *   that device current) and caches it; make that first call before any stream
+ *   capture.
+ * - All calls share the array and it keeps the last call's contents (nothing in
+ *   it needs to start at zero). Calls whose kernels overlap on the GPU (other
+ *   streams, other host threads) race on it: serialise them.
+ */
+int kvq_decode_attn_noalloc(const void* q, int32_t batch, const void* k_cache,
+                            const void* v_cache, const void* const* scales,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            int32_t max_context_len, float sm_scale, void* out,
+                            kvq_out_dtype out_dtype, int32_t partition_tokens, kvq_fmt fmt,
+                            const kvq_dims* dims, kvq_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Device error word.                                                          */
 /* ------------------------------------------------------------------------ */
 /* Read (and if `clear` is non-zero, reset) the current device's error word

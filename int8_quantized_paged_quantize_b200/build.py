@@ -24,7 +24,7 @@ LIB = os.path.join(PKG, "libkvq.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3", "-I", INCLUDE, "-I", CSRC]
-SOURCES = ["kvq_kernels.cu", "kvq_api.cpp", "kvq_pool.cpp"]
+SOURCES = ["kvq_kernels.cu", "kvq_api.cpp", "kvq_pool.cpp", "kvq_noalloc.cu"]
 
 
 def nvcc() -> str:

@@ -47,7 +47,12 @@ _SIGNATURES = [
     ("kvq_decode_merge", _c.c_int, [_c.c_int32, _P, _c.c_int32, _P, _c.c_int, _P, _c.c_size_t,
                                     _c.c_int32, _c.c_int, _P, _P]),
     ("kvq_device_error", _c.c_int, [_c.POINTER(_c.c_uint32), _c.c_int]),
+    ("kvq_decode_attn_noalloc", _c.c_int, [_P, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32,
+                                           _c.c_float, _P, _c.c_int, _c.c_int32, _c.c_int, _P,
+                                           _P]),
 ]
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 _lib = None
 
@@ -231,6 +236,24 @@ def decode_merge(batch, context_lens, max_context_len, out, workspace, fmt: str,
                                   _out_dtype(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   partition_tokens, FMT[fmt], ctypes.byref(d), _stream(stream)),
            "kvq_decode_merge")
+
+
+def decode_attn_noalloc(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                        max_context_len, sm_scale, out, fmt: str, d: Dims, partition_tokens=0,
+                        stream=None):
+    """kvq_decode_attn_noalloc: decode attention with the library's own static
+    scratch instead of a caller workspace (for callers that cannot allocate)."""
+    _need(q, torch.bfloat16, "q")
+    _need(out, out.dtype, "out")
+    _need(block_tables, torch.int32, "block_tables")
+    _need(context_lens, torch.int32, "context_lens")
+    B = q.shape[0]
+    _check(lib().kvq_decode_attn_noalloc(_ptr(q), B, _ptr(k_cache), _ptr(v_cache),
+                                         _scales(k_scale, v_scale), _ptr(block_tables),
+                                         _ptr(context_lens), int(max_context_len), float(sm_scale),
+                                         _ptr(out), _out_dtype(out), partition_tokens, FMT[fmt],
+                                         ctypes.byref(d), _stream(stream)),
+           "kvq_decode_attn_noalloc")
 
 
 def device_error(clear=True) -> int:
