@@ -38,14 +38,20 @@
  *
  * Device layouts (one layer; K and V are separate arrays)
  * -------------------------------------------------------
- *   K cache  [num_blocks][n_kv_heads][block_size][head_dim]   element-major rows
- *   V cache  [num_blocks][n_kv_heads][head_dim][block_size]   each (block, head)
- *            page is stored transposed, so that a page row holds one channel
- *            of 16 consecutive tokens
- *   element  1 byte (FP8 E4M3 code or int8 code) or 2 bytes (BF16)
+ *   element  E = 1 byte (FP8 E4M3 code or int8 code) or 2 bytes (BF16)
+ *   page     one (block, KV head): 16 tokens x head_dim elements = 16*D*E bytes,
+ *            made of 16-byte chunks
+ *   K cache  [num_blocks][n_kv_heads][D*E/16][16][16/E]: chunk (c, t) holds
+ *            elements d in [c*16/E, (c+1)*16/E) of token t, at page offset
+ *            (c*16 + t)*16
+ *   V cache  [num_blocks][n_kv_heads][E][D][16/E]: chunk (u, d) holds tokens
+ *            t in [u*16/E, (u+1)*16/E) of channel d, at page offset (u*D + d)*16
+ *            (the page is stored transposed)
  *   scales   FP8:  [num_blocks][n_kv_heads][block_size]    BF16 scale
  *            INT8: [num_blocks][n_kv_heads][block_size][2] BF16 {scale, zero_point}
  *            BF16: none (pass NULL)
+ * A thread that owns one token (K) or one channel (V) reads its row as whole
+ * 16-byte chunks, and the threads of a page together read contiguous bytes.
  * A token at sequence position p lives in slot
  *   block_tables[b][p / block_size] * block_size + p % block_size.
  */
@@ -88,6 +94,8 @@ typedef enum {
 #define KVQ_DEVERR_BLOCK 0x2u    /* decode: block id outside [0, num_blocks) */
 #define KVQ_DEVERR_CONTEXT 0x4u  /* decode: context_len < 0, > max_context_len,
                                     or > max_blocks_per_seq * block_size */
+#define KVQ_DEVERR_TIMEOUT 0x8u  /* decode: a pipeline wait ran out (about 1 s);
+                                    that chunk's output is not valid */
 
 typedef struct {
   int32_t num_blocks;         /* blocks in the pool */

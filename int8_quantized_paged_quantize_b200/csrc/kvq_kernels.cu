@@ -78,36 +78,33 @@ __device__ __forceinline__ void codes4_to_f32(uint32_t w, float* o) {
   }
 }
 
-// ------------------------------------------------------------------ append
-// One warp per (token, KV head, K|V) row of D BF16 values: E = D/32 values per
-// lane. Range reduction by warp shuffles, scale on every lane, encode, store.
-// K rows go to the page row [off][0..D); V rows go down the transposed page
-// column [0..D)[off].
-template <int D, int FMT>
-__global__ void __launch_bounds__(256) append_kernel(
-    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-    const int64_t* __restrict__ slots, int T, int Hk, int NB, uint8_t* __restrict__ kc,
-    uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs) {
-  constexpr int E = D / 32;
-  constexpr int ELT = (FMT == KVQ_BF16) ? 2 : 1;
-  const int lane = threadIdx.x & 31;
-  const int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
-  if (row >= int64_t(T) * Hk * 2) return;
-  const int which = int(row & 1);           // 0: K, 1: V
-  const int64_t th = row >> 1;
-  const int h = int(th % Hk);
-  const int64_t t = th / Hk;
-  const int64_t slot = slots[t];
-  if (slot < 0) return;
-  if (slot >= int64_t(NB) * kBlockSize) {
-    if (lane == 0) flag_error(KVQ_DEVERR_SLOT);
-    return;
-  }
-  const int64_t blk = slot / kBlockSize;
-  const int off = int(slot % kBlockSize);
-  const __nv_bfloat16* src = (which ? v : k) + (t * Hk + h) * D + lane * E;
+}  // namespace kvq
 
-  // E BF16 values of this lane
+#include <cstdlib>
+#include <cstring>
+#include <utility>
+
+#include "kvq_decode_tc.cuh"
+
+namespace kvq {
+
+// ------------------------------------------------------------------ append
+// Quantize one (token, KV head) row of D BF16 values held by a warp (E = D/32
+// values per lane): range by warp shuffles, the BF16 scale (+ zero point) on
+// every lane, codes in d order packed little-endian into `w`.
+template <int D, int FMT>
+struct RowCodes {
+  static constexpr int E = D / 32;
+  static constexpr int ELT = (FMT == KVQ_BF16) ? 2 : 1;
+  static constexpr int WORDS = (E * ELT + 3) / 4;
+  uint32_t w[WORDS];
+  __nv_bfloat16 s;
+  int zp;
+};
+
+template <int D, int FMT>
+__device__ __forceinline__ void quantize_row(const __nv_bfloat16* src, RowCodes<D, FMT>& rc) {
+  constexpr int E = D / 32;
   uint32_t raw[E / 2];
   if constexpr (E == 4) {
     const uint2 u = *reinterpret_cast<const uint2*>(src);
@@ -115,46 +112,31 @@ __global__ void __launch_bounds__(256) append_kernel(
   } else {
     raw[0] = *reinterpret_cast<const uint32_t*>(src);
   }
-  float x[E];
-#pragma unroll
-  for (int i = 0; i < E / 2; ++i) { x[2 * i] = bf16_lo(raw[i]); x[2 * i + 1] = bf16_hi(raw[i]); }
-
-  const int64_t page = blk * Hk + h;                       // (block, head) page index
-  uint8_t* cache = which ? vc : kc;
-  __nv_bfloat16* meta = which ? vs : ks;
-
+  rc.zp = 0;
+  rc.s = __float2bfloat16_rn(0.f);
   if constexpr (FMT == KVQ_BF16) {
-    if (which == 0) {
-      uint8_t* dst = cache + ((page * kBlockSize + off) * D + lane * E) * ELT;
-      if constexpr (E == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(raw[0], raw[1]);
-      else *reinterpret_cast<uint32_t*>(dst) = raw[0];
-    } else {
-      uint16_t* dst = reinterpret_cast<uint16_t*>(cache) + page * D * kBlockSize + off;
 #pragma unroll
-      for (int i = 0; i < E; ++i)
-        dst[(lane * E + i) * kBlockSize] = uint16_t(i & 1 ? raw[i / 2] >> 16 : raw[i / 2] & 0xffff);
-    }
+    for (int i = 0; i < E / 2; ++i) rc.w[i] = raw[i];
     return;
   } else {
-    uint8_t code[E];
-    __nv_bfloat16 s_bf;
-    int zp = 0;
+    float x[E];
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) { x[2 * i] = bf16_lo(raw[i]); x[2 * i + 1] = bf16_hi(raw[i]); }
+    uint32_t packed = 0;
     if constexpr (FMT == KVQ_FP8_E4M3) {
       float amax = 0.f;
 #pragma unroll
       for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(x[i]));
       amax = warp_max(amax);
-      s_bf = __float2bfloat16_rn(__fdiv_rn(amax, 448.0f));
-      const float s = __bfloat162float(s_bf);
+      rc.s = __float2bfloat16_rn(__fdiv_rn(amax, 448.0f));
+      const float s = __bfloat162float(rc.s);
+      if (s != 0.f) {
 #pragma unroll
-      for (int i = 0; i < E; i += 2) {
-        uint16_t two = 0;
-        if (s != 0.f) {
+        for (int i = 0; i < E; i += 2) {
           const float2 qv = make_float2(__fdiv_rn(x[i], s), __fdiv_rn(x[i + 1], s));
-          two = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
+          const uint32_t two = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
+          packed |= two << (8 * i);
         }
-        code[i] = uint8_t(two & 0xff);
-        code[i + 1] = uint8_t(two >> 8);
       }
     } else {  // INT8 asymmetric
       float lo = 0.f, hi = 0.f;
@@ -162,41 +144,148 @@ __global__ void __launch_bounds__(256) append_kernel(
       for (int i = 0; i < E; ++i) { lo = fminf(lo, x[i]); hi = fmaxf(hi, x[i]); }
       lo = warp_min(lo);
       hi = warp_max(hi);
-      s_bf = __float2bfloat16_rn(__fdiv_rn(__fsub_rn(hi, lo), 255.0f));
-      const float s = __bfloat162float(s_bf);
+      rc.s = __float2bfloat16_rn(__fdiv_rn(__fsub_rn(hi, lo), 255.0f));
+      const float s = __bfloat162float(rc.s);
       if (s != 0.f) {
         const float zq = fminf(fmaxf(__fdiv_rn(lo, s), -1024.f), 1024.f);
-        zp = min(127, max(-128, -128 - __float2int_rn(zq)));
-      }
+        rc.zp = min(127, max(-128, -128 - __float2int_rn(zq)));
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        int c = 0;
-        if (s != 0.f) {
+        for (int i = 0; i < E; ++i) {
           const float qf = fminf(fmaxf(__fdiv_rn(x[i], s), -1024.f), 1024.f);
-          c = min(127, max(-128, __float2int_rn(qf) + zp));
+          const int c = min(127, max(-128, __float2int_rn(qf) + rc.zp));
+          packed |= uint32_t(uint8_t(int8_t(c))) << (8 * i);
         }
-        code[i] = uint8_t(int8_t(c));
       }
     }
-    if (which == 0) {
-      uint8_t* dst = cache + (page * kBlockSize + off) * D + lane * E;
-      if constexpr (E == 4)
-        *reinterpret_cast<uint32_t*>(dst) =
-            uint32_t(code[0]) | (uint32_t(code[1]) << 8) | (uint32_t(code[2]) << 16) | (uint32_t(code[3]) << 24);
-      else
-        *reinterpret_cast<uint16_t*>(dst) = uint16_t(code[0] | (code[1] << 8));
-    } else {
-      uint8_t* dst = cache + page * D * kBlockSize + off;
+    rc.w[0] = packed;
+  }
+}
+
+// One CTA of 8 warps per (16 consecutive input tokens, KV head); each warp
+// quantizes K and V rows of its tokens. When the 16 tokens fill one page in
+// order (the bulk / prefill case) the codes are staged in shared memory and the
+// page is written as whole 16-byte chunks: K in its chunk-major layout, V
+// transposed. Otherwise every row is stored on its own: its K chunks, and one
+// element per channel down the transposed V page.
+template <int D, int FMT>
+__global__ void __launch_bounds__(256) append_kernel(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const int64_t* __restrict__ slots, int T, int Hk, int NB, uint8_t* __restrict__ kc,
+    uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs) {
+  using RC = RowCodes<D, FMT>;
+  constexpr int E = RC::E, ELT = RC::ELT;
+  constexpr int ROWB = D * ELT;                 // bytes of one token row
+  constexpr int PADB = ROWB + 16;               // padded smem row (bank spread)
+  constexpr int PAGEB = kBlockSize * ROWB;
+  constexpr int MV = (FMT == KVQ_FP8_E4M3) ? 1 : (FMT == KVQ_INT8_ASYM ? 2 : 0);
+  __shared__ __align__(16) uint8_t kbuf[kBlockSize * PADB];
+  __shared__ __align__(16) uint8_t vbuf[kBlockSize * PADB];
+  __shared__ __nv_bfloat16 kmb[kBlockSize][2], vmb[kBlockSize][2];
+  __shared__ int64_t sl[kBlockSize];
+
+  const int h = blockIdx.y;
+  const int64_t tb = int64_t(blockIdx.x) * kBlockSize;
+  const int n = int(min(int64_t(kBlockSize), int64_t(T) - tb));
+  if (threadIdx.x < kBlockSize) sl[threadIdx.x] = threadIdx.x < n ? slots[tb + threadIdx.x] : -1;
+  __syncthreads();
+  const int64_t s0 = sl[0];
+  bool fast = n == kBlockSize && s0 >= 0 && s0 % kBlockSize == 0 && s0 < int64_t(NB) * kBlockSize;
 #pragma unroll
-      for (int i = 0; i < E; ++i) dst[(lane * E + i) * kBlockSize] = code[i];
+  for (int i = 1; i < kBlockSize; ++i) fast = fast && sl[i] == s0 + i;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d0 = lane * E;
+  for (int rr = warp; rr < 2 * kBlockSize; rr += 8) {
+    const int i = rr >> 1, which = rr & 1;          // token in the group, K or V
+    if (i >= n) continue;
+    const int64_t slot = sl[i];
+    if (slot < 0) continue;
+    if (slot >= int64_t(NB) * kBlockSize) {
+      if (lane == 0) flag_error(KVQ_DEVERR_SLOT);
+      continue;
     }
-    if (lane == 0) {
-      if constexpr (FMT == KVQ_FP8_E4M3) {
-        meta[page * kBlockSize + off] = s_bf;
-      } else {
-        meta[(page * kBlockSize + off) * 2] = s_bf;
-        meta[(page * kBlockSize + off) * 2 + 1] = __int2bfloat16_rn(zp);
+    RC rc;
+    quantize_row<D, FMT>((which ? v : k) + ((tb + i) * Hk + h) * D + d0, rc);
+    if (fast) {
+      uint8_t* dst = (which ? vbuf : kbuf) + i * PADB + d0 * ELT;
+      if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
+      else if constexpr (E * ELT == 4) *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
+      else *reinterpret_cast<uint16_t*>(dst) = uint16_t(rc.w[0]);
+      if (lane == 0) {
+        (which ? vmb : kmb)[i][0] = rc.s;
+        (which ? vmb : kmb)[i][1] = __int2bfloat16_rn(rc.zp);
       }
+      continue;
+    }
+    const int64_t page = (slot / kBlockSize) * Hk + h;
+    const int off = int(slot % kBlockSize);
+    if (which == 0) {
+      // this token's chunk(s) of the K page: element d at chunk d*ELT/16
+      uint8_t* dst = kc + page * PAGEB + ((d0 * ELT) / 16) * 256 + off * 16 + (d0 * ELT) % 16;
+      if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
+      else if constexpr (E * ELT == 4) *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
+      else *reinterpret_cast<uint16_t*>(dst) = uint16_t(rc.w[0]);
+    } else {
+      // down the transposed V page: (token off, channel d) at chunk (off*ELT/16, d)
+      uint8_t* base = vc + page * PAGEB + ((off * ELT) / 16) * (D * 16) + (off * ELT) % 16;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const uint32_t word = rc.w[(e * ELT) / 4];
+        if constexpr (ELT == 2)
+          *reinterpret_cast<uint16_t*>(base + (d0 + e) * 16) = uint16_t(word >> (16 * (e & 1)));
+        else
+          base[(d0 + e) * 16] = uint8_t(word >> (8 * (e & 3)));
+      }
+    }
+    if (MV > 0 && lane == 0) {
+      __nv_bfloat16* meta = which ? vs : ks;
+      if (MV == 1) {
+        meta[page * kBlockSize + off] = rc.s;
+      } else {
+        meta[(page * kBlockSize + off) * 2] = rc.s;
+        meta[(page * kBlockSize + off) * 2 + 1] = __int2bfloat16_rn(rc.zp);
+      }
+    }
+  }
+  if (!fast) return;                                 // uniform over the CTA
+  __syncthreads();
+  const int64_t page = (s0 / kBlockSize) * Hk + h;
+  uint8_t* kp = kc + page * PAGEB;
+  uint8_t* vp = vc + page * PAGEB;
+  // K: chunk j = (c, t) <- bytes [16c, 16c+16) of token t's row
+  for (int j = threadIdx.x; j < PAGEB / 16; j += blockDim.x) {
+    const int c = j >> 4, t = j & 15;
+    *reinterpret_cast<uint4*>(kp + j * 16) = *reinterpret_cast<const uint4*>(kbuf + t * PADB + c * 16);
+  }
+  // V: chunk j = (u, d) <- tokens [u*16/ELT, (u+1)*16/ELT) of channel d
+  for (int j = threadIdx.x; j < ELT * D; j += blockDim.x) {
+    const int u = j / D, d = j % D;
+    uint32_t wv[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t word = 0;
+      if constexpr (ELT == 1) {
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) word |= uint32_t(vbuf[(q4 * 4 + bb) * PADB + d]) << (8 * bb);
+      } else {
+        const int t0 = u * 8 + q4 * 2;
+        word = uint32_t(*reinterpret_cast<const uint16_t*>(vbuf + t0 * PADB + 2 * d)) |
+               (uint32_t(*reinterpret_cast<const uint16_t*>(vbuf + (t0 + 1) * PADB + 2 * d)) << 16);
+      }
+      wv[q4] = word;
+    }
+    *reinterpret_cast<uint4*>(vp + j * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  }
+  if (MV > 0 && threadIdx.x < 2 * kBlockSize) {
+    const int t = threadIdx.x & 15;
+    const bool isv = threadIdx.x >= kBlockSize;
+    __nv_bfloat16* meta = isv ? vs : ks;
+    const __nv_bfloat16 (*mb)[2] = isv ? vmb : kmb;
+    if (MV == 1) {
+      meta[page * kBlockSize + t] = mb[t][0];
+    } else {
+      meta[(page * kBlockSize + t) * 2] = mb[t][0];
+      meta[(page * kBlockSize + t) * 2 + 1] = mb[t][1];
     }
   }
 }
@@ -289,15 +378,19 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
     const int nvalid = min(kBlockSize, t1 - pg * kBlockSize);
     const bool valid = t_in < nvalid && pg * kBlockSize + t_in >= t0;
 
-    // ---- loads
+    // ---- loads (K: chunks of this lane's half row; V: this lane's channel rows)
     uint4 kr[C::KU4], vr[C::VU4];
-    const uint4* kp = reinterpret_cast<const uint4*>(kc + page * C::PAGE_BYTES +
-                                                     (t_in * D + half * (D / 2)) * ELT);
+    const uint8_t* kpage = kc + page * C::PAGE_BYTES;
 #pragma unroll
-    for (int i = 0; i < C::KU4; ++i) kr[i] = __ldg(kp + i);
-    const uint4* vp = reinterpret_cast<const uint4*>(vc + page * C::PAGE_BYTES) + lane * C::VU4;
+    for (int i = 0; i < C::KU4; ++i)
+      kr[i] = __ldg(reinterpret_cast<const uint4*>(kpage + (half * C::KU4 + i) * 256 + t_in * 16));
+    const uint8_t* vpage = vc + page * C::PAGE_BYTES;
 #pragma unroll
-    for (int i = 0; i < C::VU4; ++i) vr[i] = __ldg(vp + i);
+    for (int j = 0; j < C::ROWS; ++j) {
+#pragma unroll
+      for (int u = 0; u < ELT; ++u)
+        vr[j * ELT + u] = __ldg(reinterpret_cast<const uint4*>(vpage + u * (D * 16) + (lane * C::ROWS + j) * 16));
+    }
     float sk = 1.f, sv = 1.f, zk = 0.f, zv = 0.f;
     if constexpr (FMT == KVQ_FP8_E4M3) {
       sk = __bfloat162float(ks[page * kBlockSize + t_in]);
@@ -471,10 +564,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int D, int FMT>
 cudaError_t append_dispatch(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
                             void* vc, void* ks, void* vs, const kvq_dims& d, cudaStream_t st) {
-  const int64_t rows = int64_t(T) * d.n_kv_heads * 2;
-  const int warps = 8;
-  const int64_t grid = (rows + warps - 1) / warps;
-  append_kernel<D, FMT><<<dim3(unsigned(grid)), 32 * warps, 0, st>>>(
+  const dim3 grid(unsigned((int64_t(T) + kBlockSize - 1) / kBlockSize), unsigned(d.n_kv_heads));
+  append_kernel<D, FMT><<<grid, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), slots, T,
       d.n_kv_heads, d.num_blocks, static_cast<uint8_t*>(kc), static_cast<uint8_t*>(vc),
       static_cast<__nv_bfloat16*>(ks), static_cast<__nv_bfloat16*>(vs));
@@ -498,12 +589,51 @@ cudaError_t decode_dispatch3(const void* q, int32_t B, const void* kc, const voi
   return cudaGetLastError();
 }
 
+template <int D, int G, int FMT>
+cudaError_t decode_tc_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
+                                const void* ks, const void* vs, const int32_t* tables,
+                                const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                                const DecodePlan& plan, void* ws, const kvq_dims& d,
+                                cudaStream_t st) {
+  using C = TcCfg<D, FMT>;
+  auto kern = decode_tc_kernel<D, G, FMT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  float* po = static_cast<float*>(ws);
+  float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
+  const int64_t grid = int64_t(B) * d.n_kv_heads * plan.max_splits;
+  kern<<<dim3(unsigned(grid)), 192, C::SMEM, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
+      static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
+      static_cast<const __nv_bfloat16*>(vs), tables, ctx, d.n_kv_heads, d.num_blocks,
+      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml);
+  return cudaGetLastError();
+}
+
+// The tensor-core kernel is the decode path; KVQ_DECODE_KERNEL=simt selects the
+// CUDA-core kernel instead (kept to measure one against the other).
+bool use_simt_decode() {
+  static const bool simt = [] {
+    const char* v = std::getenv("KVQ_DECODE_KERNEL");
+    return v != nullptr && std::strcmp(v, "simt") == 0;
+  }();
+  return simt;
+}
+
 template <int D, int FMT>
 cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, const void* vc,
                              const void* ks, const void* vs, const int32_t* tables,
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
                              const DecodePlan& plan, void* ws, const kvq_dims& d,
                              cudaStream_t st) {
+  if (!use_simt_decode()) {
+    switch (G) {
+      case 1: return decode_tc_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+      case 2: return decode_tc_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+      case 4: return decode_tc_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+      default: return decode_tc_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+    }
+  }
   switch (G) {
     case 1: return decode_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
     case 2: return decode_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);

@@ -22,7 +22,7 @@ ELEM_BYTES = {"bf16": 2, "fp8": 1, "int8": 1}
 META_VALUES = {"bf16": 0, "fp8": 1, "int8": 2}
 BLOCK_SIZE = 16
 
-DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT = 0x1, 0x2, 0x4
+DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 # Every function the header declares: (name, restype, argtypes)
 _c = ctypes
@@ -278,10 +278,12 @@ class LayerCache:
 
     @staticmethod
     def allocate(fmt, d: Dims, device="cuda"):
+        """Zeroed K/V caches and scales in the library's page layout (include/kvq.h)."""
         nb, hk, D = d.num_blocks, d.n_kv_heads, d.head_dim
+        E = ELEM_BYTES[fmt]
         edt = torch.bfloat16 if fmt == "bf16" else torch.uint8
-        k = torch.zeros((nb, hk, BLOCK_SIZE, D), dtype=edt, device=device)
-        v = torch.zeros((nb, hk, D, BLOCK_SIZE), dtype=edt, device=device)
+        k = torch.zeros((nb, hk, D * E // 16, BLOCK_SIZE, 16 // E), dtype=edt, device=device)
+        v = torch.zeros((nb, hk, E, D, 16 // E), dtype=edt, device=device)
         mv = META_VALUES[fmt]
         if mv:
             shape = (nb, hk, BLOCK_SIZE) if mv == 1 else (nb, hk, BLOCK_SIZE, 2)
@@ -312,9 +314,15 @@ class LayerCache:
                     partition_tokens, stream)
         return out
 
-    # ---- views in the logical layout [NB][Hk][bs][D] (for inspection and tests)
-    def k_logical(self):
-        return self.k
+    # ---- copies in the logical layout [NB][Hk][block_size][D] (for inspection and tests)
+    def k_logical(self, blocks=None):
+        """K of all blocks (or of the block ids `blocks`) as [n][Hk][block_size][D]."""
+        k = self.k if blocks is None else self.k[blocks]
+        return k.permute(0, 1, 3, 2, 4).reshape(k.shape[0], k.shape[1], BLOCK_SIZE,
+                                                self.dims.head_dim)
 
-    def v_logical(self):
-        return self.v.transpose(2, 3)
+    def v_logical(self, blocks=None):
+        """V of all blocks (or of the block ids `blocks`) as [n][Hk][block_size][D]."""
+        v = self.v if blocks is None else self.v[blocks]
+        return v.permute(0, 1, 2, 4, 3).reshape(v.shape[0], v.shape[1], BLOCK_SIZE,
+                                                self.dims.head_dim)

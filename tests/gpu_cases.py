@@ -147,8 +147,8 @@ def gpu_sequence(run: GpuRun, b: int):
     n = int(run.ctx_after[b])
     pages = int(math.ceil(n / 16))
     ids = torch.from_numpy(run.tables[b][:pages].astype(np.int64)).to(run.cache.k.device)
-    kl = run.cache.k_logical()[ids]                      # [pages][Hk][16][D]
-    vl = run.cache.v_logical()[ids]
+    kl = run.cache.k_logical(ids)                        # [pages][Hk][16][D]
+    vl = run.cache.v_logical(ids)
     kl = kl.permute(0, 2, 1, 3).reshape(pages * 16, kl.shape[1], kl.shape[3])[:n].cpu()
     vl = vl.permute(0, 2, 1, 3).reshape(pages * 16, vl.shape[1], vl.shape[3])[:n].cpu()
     out = {"k_codes": kl, "v_codes": vl}

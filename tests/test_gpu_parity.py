@@ -120,7 +120,7 @@ def test_zero_rows_store_zero_scale(fmt):
     v[1] = 1.0
     c.append(k, v, torch.tensor([0, 1, 2], dtype=torch.int64, device="cuda"))
     torch.cuda.synchronize()
-    assert torch.all(c.k_scale.float().cpu() == 0) and torch.all(c.k.cpu() == 0)
+    assert torch.all(c.k_scale.float().cpu() == 0) and torch.all(c.k_logical().cpu() == 0)
     q = torch.randn(1, 4, 64, device="cuda").to(torch.bfloat16)
     tbl = torch.tensor([[0, -1, -1, -1]], dtype=torch.int32, device="cuda")
     cl = torch.tensor([3], dtype=torch.int32, device="cuda")
@@ -173,7 +173,7 @@ def test_negative_slots_are_skipped_and_bad_slots_flagged():
     c.append(k, k, torch.tensor([-1, 5, 40], dtype=torch.int64, device="cuda"))  # 40 >= 2*16
     torch.cuda.synchronize()
     assert kvq.device_error() == kvq.DEVERR_SLOT
-    written = (c.k.cpu() != 0).any(-1).any(1)                    # [blocks][offsets]
+    written = (c.k_logical().cpu() != 0).any(-1).any(1)          # [blocks][offsets]
     assert written.sum().item() == 1 and bool(written[0, 5])
 
 
@@ -246,4 +246,27 @@ def test_multiple_decode_steps_track_the_oracle(fmt):
         assert err.max() <= GC.MAX_ABS and err.mean() <= GC.MEAN_ABS, (step, err.max())
     assert np.array_equal(c.k_logical().cpu().numpy().view(np.int8 if fmt == "int8" else np.uint8),
                           pool.k)
+    assert kvq.device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("D", [64, 128])
+def test_bulk_and_per_row_append_write_the_same_bytes(fmt, D):
+    """Whole pages appended in order take the staged bulk path; the same tokens in
+    a shuffled order take the per-row path. Both must leave identical caches."""
+    d = kvq.dims(12, 2, 4, D, 12)
+    n = 16 * 10 + 5
+    g = torch.Generator().manual_seed(3)
+    k = (torch.randn(n, 2, D, generator=g) * 2 + 0.3).to(torch.bfloat16).cuda()
+    v = torch.randn(n, 2, D, generator=g).to(torch.bfloat16).cuda()
+    slots = torch.arange(n, dtype=torch.int64).cuda() + 16          # pages 1..11, in order
+    a = kvq.LayerCache.allocate(fmt, d)
+    a.append(k, v, slots)
+    perm = torch.randperm(n, generator=g).cuda()
+    b = kvq.LayerCache.allocate(fmt, d)
+    b.append(k[perm].contiguous(), v[perm].contiguous(), slots[perm].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
+    if fmt != "bf16":
+        assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
     assert kvq.device_error() == 0
