@@ -65,7 +65,8 @@ struct TcCfg {
   static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;         // float [2][4][16]
   static constexpr int OFF_RED2 = OFF_RED + 2 * 4 * 16 * 4;  // float [2][4][8]
   static constexpr int OFF_QSC = OFF_RED2 + 2 * 4 * 8 * 4;   // float [8]
-  static constexpr int OFF_MISC = OFF_QSC + 8 * 4;           // tmem base, abort flag
+  static constexpr int OFF_PMASK = OFF_QSC + 8 * 4;          // uint32 [NST] valid-page masks
+  static constexpr int OFF_MISC = OFF_PMASK + 4 * NST;       // tmem base, abort flag
   static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + alignment slack
 };
 
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
   float* red2 = reinterpret_cast<float*>(smem + C::OFF_RED2);
   float* qsc = reinterpret_cast<float*>(smem + C::OFF_QSC);
+  volatile uint32_t* pmask = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_PMASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -209,7 +211,11 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
           }
           nvalid += blk[p] >= 0;
         }
+        uint32_t mask = 0;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) mask |= (blk[p] >= 0 ? 1u : 0u) << p;
         if (!mbar_wait(kempty + s, ph ^ 1, abort_flag, kWaitLimitCycles)) break;
+        pmask[s] = mask;                       // published by the arrive below
         mbar_arrive_expect_tx(kfull + s, nvalid * uint32_t(C::PAGE + C::METAB));
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
@@ -303,30 +309,18 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
     }
     float einv_pend = 1.f;
     bool ok = true;
+    // byte offset of (row g, token r) in a P buffer; row part*8 + g adds part*1024
+    uint32_t poff[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) poff[g] = sw128_offset(g, r, C::NPR);
     // carried from the K conversion of tile j to the softmax/V of tile j
     float sk_carry = 0.f, sk_cur = 0.f;
     uint32_t valid_carry = 0, valid_cur = 0;
 
-    // page p of tile j is valid when inside the chunk and its block id is legal
-    auto page_mask = [&](int j) -> uint32_t {
-      const int tok0 = t0 + 128 * j;
-      const int pg0 = tok0 / kBlockSize;
-      const int npg = min(8, (t1 - tok0 + kBlockSize - 1) / kBlockSize);
-      uint32_t mask = 0;
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        if (p < npg) {
-          const int bk = trow[pg0 + p];
-          if (bk >= 0 && bk < NB) mask |= 1u << p;
-        }
-      }
-      return mask;
-    };
-
     auto conv_k = [&](int j) {
       const int s = j % C::NST;
       if (ok) ok = mbar_wait(kfull + s, (j / C::NST) & 1, abort_flag, kWaitLimitCycles);
-      const uint32_t mask = page_mask(j);
+      const uint32_t mask = ok ? pmask[s] : 0u;   // pages of tile j inside the chunk with legal ids
       const int p = r >> 4, t = r & 15;
       const bool valid = ok && (mask >> p & 1) && (t0 + 128 * j + r < t1);
       uint32_t w[C::KWORDS];
@@ -356,10 +350,7 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
             for (int e = 0; e < 4; ++e) {
               uint32_t lo, hi;
               if constexpr (FMT == KVQ_FP8_E4M3) {
-                __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(__nv_fp8x2_storage_t(uw[e] & 0xffff), __NV_E4M3);
-                __half2_raw bb = __nv_cvt_fp8x2_to_halfraw2(__nv_fp8x2_storage_t(uw[e] >> 16), __NV_E4M3);
-                lo = uint32_t(a.x) | (uint32_t(a.y) << 16);
-                hi = uint32_t(bb.x) | (uint32_t(bb.y) << 16);
+                e4m3x4_to_f16x4(uw[e], lo, hi);
               } else {
                 const uint32_t x = uw[e] ^ 0x80808080u;          // c + 128 as unsigned bytes
                 const uint32_t p0 = __byte_perm(x, 0x64646464u, 0x4140);   // 1024 + byte0|1
@@ -417,10 +408,7 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               if constexpr (FMT == KVQ_FP8_E4M3) {
-                __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(__nv_fp8x2_storage_t(uw[e] & 0xffff), __NV_E4M3);
-                __half2_raw bb = __nv_cvt_fp8x2_to_halfraw2(__nv_fp8x2_storage_t(uw[e] >> 16), __NV_E4M3);
-                pw[2 * e] = uint32_t(a.x) | (uint32_t(a.y) << 16);
-                pw[2 * e + 1] = uint32_t(bb.x) | (uint32_t(bb.y) << 16);
+                e4m3x4_to_f16x4(uw[e], pw[2 * e], pw[2 * e + 1]);
               } else {
                 const uint32_t x = uw[e] ^ 0x80808080u;
                 const uint32_t p0 = __byte_perm(x, 0x64646464u, 0x4140);
@@ -549,15 +537,15 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
           const float r1 = pr - __bfloat162float(hi);
           const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
           const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-          *reinterpret_cast<uint16_t*>(pb + sw128_offset(g, r, C::NPR)) = __bfloat16_as_ushort(hi);
-          *reinterpret_cast<uint16_t*>(pb + sw128_offset(8 + g, r, C::NPR)) = __bfloat16_as_ushort(mid);
-          *reinterpret_cast<uint16_t*>(pb + sw128_offset(16 + g, r, C::NPR)) = __bfloat16_as_ushort(lo);
+          *reinterpret_cast<uint16_t*>(pb + poff[g]) = __bfloat16_as_ushort(hi);
+          *reinterpret_cast<uint16_t*>(pb + poff[g] + 1024) = __bfloat16_as_ushort(mid);
+          *reinterpret_cast<uint16_t*>(pb + poff[g] + 2048) = __bfloat16_as_ushort(lo);
         } else {
           const float pp = pr * sv * escale;
           const __half hi = __float2half_rn(pp);
           const __half lo = __float2half_rn(pp - __half2float(hi));
-          *reinterpret_cast<uint16_t*>(pb + sw128_offset(g, r, C::NPR)) = __half_as_ushort(hi);
-          *reinterpret_cast<uint16_t*>(pb + sw128_offset(8 + g, r, C::NPR)) = __half_as_ushort(lo);
+          *reinterpret_cast<uint16_t*>(pb + poff[g]) = __half_as_ushort(hi);
+          *reinterpret_cast<uint16_t*>(pb + poff[g] + 1024) = __half_as_ushort(lo);
           if constexpr (FMT == KVQ_INT8_ASYM)
             corr[g] = corr[g] * alpha[g] + (__half2float(hi) + __half2float(lo)) * zv * einv;
         }
