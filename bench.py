@@ -145,6 +145,7 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+
 def max_over_ranks(x, world, device="cuda"):
     """Max of a float over all ranks (identity on one rank)."""
     if world == 1:
@@ -409,8 +410,14 @@ def metric_name(fmt):
 
 
 def config_block(w, fmt, l2):
-    lens = {"fixed": f"{w.ctx[0]}", "list": "list", "uniform": f"U[{w.ctx[0]},{w.ctx[1]}]",
-            "lognormal_mix": "lognormal(1500, 1) + 4x30000"}[w.lengths]
+    if w.lengths == "fixed":
+        lens = f"{w.ctx[0]}"
+    elif w.lengths == "uniform":
+        lens = f"U[{w.ctx[0]},{w.ctx[1]}]"
+    elif w.lengths == "lognormal_mix":
+        lens = "lognormal(1500, 1) + 4x30000"
+    else:
+        lens = "list"
     return {"workload": f"{w.name}: B={w.batch} Hq={w.n_q_heads} Hk={w.n_kv_heads} D={w.head_dim} "
                         f"bs=16 ctx={lens}" + (f" +{w.bulk_append} bulk" if w.bulk_append else ""),
             "fmt": fmt, "batch": w.batch, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,

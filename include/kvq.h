@@ -41,17 +41,19 @@
  *   element  E = 1 byte (FP8 E4M3 code or int8 code) or 2 bytes (BF16)
  *   page     one (block, KV head): 16 tokens x head_dim elements = 16*D*E bytes,
  *            made of 16-byte chunks
- *   K cache  [num_blocks][n_kv_heads][D*E/16][16][16/E]: chunk (c, t) holds
+ *   K cache  [num_blocks][n_kv_heads][2][D*E/16][8][16/E]: chunk (c, t) holds
  *            elements d in [c*16/E, (c+1)*16/E) of token t, at page offset
- *            (c*16 + t)*16
+ *            (t/8)*8*D*E + c*128 + (t%8)*16 (each 8-token group stores its
+ *            16-byte chunks as 8 x 16-byte core matrices)
  *   V cache  [num_blocks][n_kv_heads][E][D][16/E]: chunk (u, d) holds tokens
  *            t in [u*16/E, (u+1)*16/E) of channel d, at page offset (u*D + d)*16
  *            (the page is stored transposed)
  *   scales   FP8:  [num_blocks][n_kv_heads][block_size]    BF16 scale
  *            INT8: [num_blocks][n_kv_heads][block_size][2] BF16 {scale, zero_point}
  *            BF16: none (pass NULL)
- * A thread that owns one token (K) or one channel (V) reads its row as whole
- * 16-byte chunks, and the threads of a page together read contiguous bytes.
+ * Both pages are tensor-core operands as stored: K is the K-major operand of
+ * S = K.q (rows = tokens), V the K-major operand of O^T = V^T.P (rows =
+ * channels); a page is one contiguous 1-D copy.
  * A token at sequence position p lives in slot
  *   block_tables[b][p / block_size] * block_size + p % block_size.
  */

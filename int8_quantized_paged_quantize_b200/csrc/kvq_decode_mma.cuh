@@ -1,0 +1,658 @@
+// Paged GQA decode attention with the cache codes fed to the 5th-generation
+// tensor cores as they are stored: FP8 E4M3 codes through kind::f8f6f4, INT8
+// codes through kind::i8 (exact integer sums), BF16 through kind::f16. No thread
+// dequantizes a K or V element; the per-token scales and zero points are applied
+// to the small S and P tiles instead. Included by kvq_kernels.cu.
+//
+// One CTA per (sequence b, KV head h, chunk of `part` tokens), 6 warps:
+//   warp 0      producer: lanes 0..7 each own one page of a 128-token tile and
+//               issue its 1-D bulk copy (K page, then V page) into a ring of
+//               smem stages; lanes 8..15 copy the pages' scales. The block ids
+//               of the next tile are loaded while the current one is issued.
+//   warp 1      allocates TMEM; one thread issues the MMAs.
+//   warps 2..5  softmax warps, one per TMEM lane quarter; thread r owns token r
+//               of the tile for S and P, channel r for O.
+// Per 128-token tile:
+//   S^T[tok x n] = Kcodes[tok x D] . Qp^T[D x n]    (A: K page ring, K-major;
+//                  B: the query group split into exact low-precision parts)
+//   softmax in FP32 registers: s = (sum of S parts) * k_scale (INT8: minus
+//     zero_point * sum(q)), online max / sum per query head.
+//   P[tok x n] = the weight p * v_scale * 2^e split into low-precision parts
+//     (FP8: 4 E4M3 parts, INT8: 3 unsigned bytes of a 24-bit fixed-point
+//     value, BF16: 3 bf16 parts), MN-major in smem.
+//   O^T[ch x n] = Vcodes^T[ch x tok] . P[tok x n]    (A: V page ring, K-major)
+//   O tile -> registers, parts recombined, rescaled and accumulated in FP32.
+// Each MMA result sits in TMEM; S, P and O are double-buffered so the MMA of
+// one tile overlaps the softmax of the next. Every byte of the chunk's K/V
+// crosses HBM once for the whole query group. Every wait is bounded: on expiry
+// the CTA sets KVQ_DEVERR_TIMEOUT, stops issuing work, drains what it issued,
+// frees TMEM and returns.
+
+#pragma once
+
+#include "kvq_tc.cuh"
+
+namespace kvq {
+
+constexpr long long kMmaWaitLimitCycles = 2000000000LL;   // about one second
+
+__host__ __device__ constexpr int round_up16(int x) { return x < 16 ? 16 : (x + 15) / 16 * 16; }
+
+template <int D, int G, int FMT>
+struct MmaCfg {
+  static constexpr bool BF = FMT == KVQ_BF16;
+  static constexpr bool F8 = FMT == KVQ_FP8_E4M3;
+  static constexpr bool I8 = FMT == KVQ_INT8_ASYM;
+  static constexpr int E = BF ? 2 : 1;                         // bytes per element
+  static constexpr int KIND = BF ? 0 : (F8 ? 1 : 2);           // mma_ss kind
+  static constexpr int PAGE = kBlockSize * D * E;              // bytes of one (block, head) page
+  static constexpr int NST = 3;                                // ring stages
+  static constexpr int MV = F8 ? 1 : (I8 ? 2 : 0);
+  static constexpr int METAB = kBlockSize * MV * 2;            // scale bytes per page
+  static constexpr int QPARTS = F8 ? 2 : (I8 ? 3 : 1);
+  static constexpr int PPARTS = F8 ? 4 : 3;
+  static constexpr int NS = round_up16(QPARTS * G);            // S columns (B rows of QK)
+  static constexpr int NO = round_up16(PPARTS * G);            // O columns (B rows of PV)
+  static_assert(NS <= 32 && NO <= 32, "query group too large");
+  static constexpr int S_MMAS = D * E / 32;                    // K extent of one MMA: 32 bytes
+  static constexpr int PV_MMAS = 128 * E / 32;
+  // operand strides (bytes)
+  static constexpr uint32_t K_LBO = 128, K_SBO = 8 * D * E;    // K page: [2][D*E/16][8 tok][16 B]
+  static constexpr uint32_t V_LBO = 16 * D, V_SBO = 128;       // V page: [E][D][16 B]
+  static constexpr uint32_t Q_SBO = 128, Q_LBO = (NS / 8) * 128;
+  static constexpr int PT = 16 / E;                            // P elements per 16-byte row
+  static constexpr uint32_t P_SBO = 128, P_LBO = (NO / PT) * 128;
+  static constexpr int QBYTES = NS * D * E;
+  static constexpr int PBYTES = NO * 128 * E;                  // one P buffer
+  // TMEM columns
+  static constexpr int COL_S = 0, COL_O = 64, TMEM_COLS = 128;
+  // shared memory carve-up (offsets from a 128-byte aligned base)
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + NST * 8 * PAGE;
+  static constexpr int OFF_KM = OFF_V + NST * 8 * PAGE;
+  static constexpr int OFF_VM = OFF_KM + NST * 8 * METAB;
+  static constexpr int OFF_Q = (OFF_VM + NST * 8 * METAB + 127) / 128 * 128;
+  static constexpr int OFF_P = OFF_Q + QBYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * PBYTES;
+  static constexpr int NBAR = 4 * NST + 10 + 1;
+  static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;           // float [2][4][16]
+  static constexpr int OFF_RED2 = OFF_RED + 2 * 4 * 16 * 4;    // float [2][4][8]
+  static constexpr int OFF_QSC = OFF_RED2 + 2 * 4 * 8 * 4;     // float [8] scale, float [8] sum(q)
+  static constexpr int OFF_PMASK = OFF_QSC + 16 * 4;           // uint32 [NST] valid-page masks
+  static constexpr int OFF_MISC = OFF_PMASK + 4 * NST;         // tmem base, abort flag
+  static constexpr int SMEM = OFF_MISC + 16 + 128;             // + alignment slack
+};
+
+template <int D, int G, int FMT>
+__global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_mma_kernel(
+    const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kc,
+    const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
+    const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
+    const int32_t* __restrict__ ctx_lens, int Hk, int NB, int W, int max_ctx, int part,
+    int max_splits, float qk_scale, float* __restrict__ part_o, float* __restrict__ part_ml) {
+  using C = MmaCfg<D, G, FMT>;
+  using namespace tc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x % max_splits;
+  const int bh = blockIdx.x / max_splits;
+  const int b = bh / Hk, h = bh % Hk;
+  const int Hq = Hk * G;
+
+  int ctx = ctx_lens[b];
+  if (ctx < 0 || ctx > max_ctx || int64_t(ctx) > int64_t(W) * kBlockSize) {
+    if (threadIdx.x == 0 && split == 0) flag_error(KVQ_DEVERR_CONTEXT);
+    ctx = 0;
+  }
+  const int n_splits = (ctx + part - 1) / part;
+  if (split >= n_splits) return;                         // uniform for the CTA
+  const int t0 = split * part, t1 = min(ctx, t0 + part);
+  const int ntiles = (t1 - t0 + 127) / 128;
+  const int32_t* trow = tables + int64_t(b) * W;
+
+  uint8_t* kring = smem + C::OFF_K;
+  uint8_t* vring = smem + C::OFF_V;
+  uint8_t* kmeta = smem + C::OFF_KM;
+  uint8_t* vmeta = smem + C::OFF_VM;
+  uint8_t* qop = smem + C::OFF_Q;
+  uint8_t* pop = smem + C::OFF_P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kfull = bars;
+  uint64_t* kempty = bars + C::NST;
+  uint64_t* vfull = bars + 2 * C::NST;
+  uint64_t* vempty = bars + 3 * C::NST;
+  uint64_t* sfull = bars + 4 * C::NST;      // [2]
+  uint64_t* sfree = sfull + 2;              // [2]
+  uint64_t* pready = sfree + 2;             // [2]
+  uint64_t* ofull = pready + 2;             // [2]
+  uint64_t* ofree = ofull + 2;              // [2]
+  uint64_t* drain = ofree + 2;
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  float* red2 = reinterpret_cast<float*>(smem + C::OFF_RED2);
+  float* qsc = reinterpret_cast<float*>(smem + C::OFF_QSC);
+  float* qsum = qsc + 8;
+  volatile uint32_t* pmask = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_PMASK);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  // ------------------------------------------------------------ set-up
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(kfull + s, 1);
+      mbar_init(kempty + s, 128);
+      mbar_init(vfull + s, 1);
+      mbar_init(vempty + s, 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(sfull + j, 1);
+      mbar_init(sfree + j, 128);
+      mbar_init(pready + j, 128);
+      mbar_init(ofull + j, 1);
+      mbar_init(ofree + j, 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    const int ct = threadIdx.x - 64;                       // 0..127
+    // zero the Q and P operands (padding rows stay zero)
+    for (int i = ct * 16; i < C::QBYTES + 2 * C::PBYTES; i += 128 * 16)
+      *reinterpret_cast<uint4*>(qop + i) = make_uint4(0, 0, 0, 0);
+    named_bar_sync(1, 128);
+    // Q parts, B operand of S (K-major, no swizzle): row n = part * G + g,
+    // element (n, d) at (n/8)*Q_SBO + (n%8)*16 + (d*E/16)*Q_LBO + (d*E)%16.
+    const int cw = warp - 2;
+    for (int g = cw; g < G; g += 4) {
+      const __nv_bfloat16* qr = q + (int64_t(b) * Hq + h * G + g) * D;
+      float v[D / 32];
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        v[i] = __bfloat162float(qr[lane + 32 * i]);
+        amax = fmaxf(amax, fabsf(v[i]));
+      }
+      amax = warp_max(amax);
+      // power-of-two scaling of the head: FP8 puts max|q| into [128, 256)
+      // (inside the E4M3 range), INT8 into [32, 64) (parts within +-64)
+      int e = 0;
+      if (!C::BF && amax > 0.f) e = (C::F8 ? 7 : 5) - ilogbf(amax);
+      e = max(-120, min(120, e));
+      const float up = __int_as_float((127 + e) << 23);
+      const float down = __int_as_float((127 - e) << 23);
+      int isum = 0;
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        const int d = lane + 32 * i;
+        auto at = [&](int n) -> uint8_t* {
+          return qop + (n >> 3) * C::Q_SBO + (n & 7) * 16 + ((d * C::E) >> 4) * C::Q_LBO +
+                 ((d * C::E) & 15);
+        };
+        if constexpr (C::BF) {
+          *reinterpret_cast<uint16_t*>(at(g)) = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+        } else if constexpr (C::F8) {
+          // x = hi + lo/16 with both parts E4M3: exact for a BF16 value unless
+          // it lies below the E4M3 normal range after scaling
+          const float x = v[i] * up;
+          const uint32_t hc = f32x2_to_e4m3x2(x, 0.f) & 0xFFu;
+          float hv, unused;
+          e4m3x2_to_f32x2(hc, hv, unused);
+          const uint32_t lc = f32x2_to_e4m3x2((x - hv) * 16.f, 0.f) & 0xFFu;
+          *at(g) = uint8_t(hc);
+          *at(G + g) = uint8_t(lc);
+        } else {
+          // x = x0 + x1/128 + x2/16384, every part an integer in [-64, 64]
+          const float x = v[i] * up;
+          const float x0 = rintf(x);
+          const float r0 = (x - x0) * 128.f;
+          const float x1 = rintf(r0);
+          const float x2 = rintf((r0 - x1) * 128.f);
+          const int i0 = int(x0), i1 = int(x1), i2 = int(x2);
+          *at(g) = uint8_t(int8_t(i0));
+          *at(G + g) = uint8_t(int8_t(i1));
+          *at(2 * G + g) = uint8_t(int8_t(i2));
+          isum += i0 * 16384 + i1 * 128 + i2;
+        }
+      }
+      if constexpr (C::I8) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+      }
+      if (lane == 0) {
+        qsc[g] = qk_scale * down;
+        qsum[g] = float(isum) * (1.f / 16384.f);           // sum of q in the units of S
+      }
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    const uint64_t pol = l2_evict_first_policy();
+    const int p8 = lane & 7;
+    auto load_id = [&](int i) -> int {
+      if (lane >= 8 || i >= ntiles) return -2;
+      const int tok0 = t0 + 128 * i;
+      const int npg = min(8, (t1 - tok0 + kBlockSize - 1) / kBlockSize);
+      return p8 < npg ? trow[tok0 / kBlockSize + p8] : -2;   // -2: no page here
+    };
+    int id_next = load_id(0);
+    bool kiss[C::NST], viss[C::NST];
+    uint32_t kpar[C::NST], vpar[C::NST];
+#pragma unroll
+    for (int s = 0; s < C::NST; ++s) { kiss[s] = viss[s] = false; kpar[s] = vpar[s] = 0; }
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % C::NST;
+      const uint32_t ph = (i / C::NST) & 1;
+      const int id = id_next;
+      id_next = load_id(i + 1);
+      if (lane < 8 && id != -2 && (id < 0 || id >= NB)) flag_error(KVQ_DEVERR_BLOCK);
+      const bool valid = lane < 8 && id >= 0 && id < NB;
+      const uint32_t mask = __ballot_sync(0xffffffffu, valid) & 0xFFu;
+      const int blk = __shfl_sync(0xffffffffu, id, p8);
+      const bool mine = ((mask >> p8) & 1u) != 0u;
+      const int64_t page = int64_t(blk) * Hk + h;
+      const uint32_t bytes = uint32_t(__popc(mask)) * uint32_t(C::PAGE + C::METAB);
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(kempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) {
+          pmask[s] = mask;                       // published by the arrive below
+          mbar_arrive_expect_tx(kfull + s, bytes);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
+      if (lane < 8 && mine) bulk_g2s(kring + (s * 8 + p8) * C::PAGE, kc + page * C::PAGE, C::PAGE, kfull + s, pol);
+      if constexpr (C::MV > 0) {
+        if (lane >= 8 && lane < 16 && mine)
+          bulk_g2s(kmeta + (s * 8 + p8) * C::METAB, reinterpret_cast<const uint8_t*>(ks) + page * C::METAB,
+                   C::METAB, kfull + s, pol);
+      }
+      kiss[s] = true;
+      kpar[s] = ph;
+      if (lane == 0) {
+        ok = mbar_wait(vempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) mbar_arrive_expect_tx(vfull + s, bytes);
+      }
+      if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
+      if (lane < 8 && mine) bulk_g2s(vring + (s * 8 + p8) * C::PAGE, vc + page * C::PAGE, C::PAGE, vfull + s, pol);
+      if constexpr (C::MV > 0) {
+        if (lane >= 8 && lane < 16 && mine)
+          bulk_g2s(vmeta + (s * 8 + p8) * C::METAB, reinterpret_cast<const uint8_t*>(vs) + page * C::METAB,
+                   C::METAB, vfull + s, pol);
+      }
+      viss[s] = true;
+      vpar[s] = ph;
+    }
+    if (lane == 0 && *abort_flag) {
+      // let the copies already issued land before the CTA's smem goes away
+      volatile int no_abort = 0;
+      for (int s = 0; s < C::NST; ++s) {
+        if (kiss[s]) mbar_wait(kfull + s, kpar[s], &no_abort, kMmaWaitLimitCycles);
+        if (viss[s]) mbar_wait(vfull + s, vpar[s], &no_abort, kMmaWaitLimitCycles);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t dfmt = C::I8 ? 2u : 1u;
+      constexpr uint32_t afmt = C::BF ? 1u : (C::I8 ? 1u : 0u);       // bf16 / s8 / E4M3
+      constexpr uint32_t qfmt = afmt;                                   // Q parts: same family
+      constexpr uint32_t pfmt = C::BF ? 1u : 0u;                        // bf16 / u8 / E4M3
+      constexpr uint32_t id_s = idesc_m128(dfmt, afmt, qfmt, false, C::NS);
+      constexpr uint32_t id_pv = idesc_m128(dfmt, afmt, pfmt, true, C::NO);
+      const uint32_t kbase = smem_u32(kring), vbase = smem_u32(vring);
+      const uint32_t qaddr = smem_u32(qop), paddr = smem_u32(pop);
+      bool ok = true;
+      for (int i = 0; ok && i <= ntiles; ++i) {
+        if (i < ntiles) {
+          const int s = i % C::NST;
+          ok = mbar_wait(kfull + s, (i / C::NST) & 1, abort_flag, kMmaWaitLimitCycles) &&
+               mbar_wait(sfree + (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, kMmaWaitLimitCycles);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a0 = kbase + s * 8 * C::PAGE;
+#pragma unroll
+          for (int kk = 0; kk < C::S_MMAS; ++kk)
+            mma_ss<C::KIND>(tmem + C::COL_S + (i & 1) * 32,
+                            sdesc_plain(a0 + kk * 2 * C::K_LBO, C::K_LBO, C::K_SBO),
+                            sdesc_plain(qaddr + kk * 2 * C::Q_LBO, C::Q_LBO, C::Q_SBO), id_s, kk > 0);
+          mma_commit(sfull + (i & 1));
+        }
+        if (i >= 1) {
+          const int j = i - 1, s = j % C::NST;
+          ok = mbar_wait(pready + (j & 1), (j >> 1) & 1, abort_flag, kMmaWaitLimitCycles) &&
+               mbar_wait(ofree + (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, kMmaWaitLimitCycles);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a0 = vbase + s * 8 * C::PAGE;
+          const uint32_t b0 = paddr + (j & 1) * C::PBYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::PV_MMAS; ++kk)
+            mma_ss<C::KIND>(tmem + C::COL_O + (j & 1) * 32,
+                            sdesc_plain(a0 + kk * 2 * C::V_LBO, C::V_LBO, C::V_SBO),
+                            sdesc_plain(b0 + kk * (4 / C::E) * C::P_LBO, C::P_LBO, C::P_SBO), id_pv,
+                            kk > 0);
+          mma_commit(ofull + (j & 1));
+          mma_commit(vempty + s);
+        }
+      }
+      // every MMA issued so far completes before TMEM is released
+      volatile int no_abort = 0;
+      mma_commit(drain);
+      mbar_wait(drain, 0, &no_abort, kMmaWaitLimitCycles);
+    }
+  } else {
+    // ---------------------------------------------------------- softmax warps
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                  // token / channel / TMEM lane
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    float qs[G], qz[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) { qs[g] = qsc[g]; qz[g] = qsum[g]; }
+    float m[G], l[G], corr[G], o[G], alpha_pend[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = -INFINITY; l[g] = 0.f; corr[g] = 0.f; o[g] = 0.f; alpha_pend[g] = 1.f;
+    }
+    float einv_pend = 1.f;
+    bool ok = true;
+    // this token's row of a P buffer (MN-major): element n at
+    // (n / PT) * P_SBO + (n % PT) * E, plus the row's own offset
+    const uint32_t prow = (r >> 3) * C::P_LBO + (r & 7) * 16;
+
+    auto accum_o = [&](int j) {
+      if (ok) ok = mbar_wait(ofull + (j & 1), (j >> 1) & 1, abort_flag, kMmaWaitLimitCycles);
+      tc_fence_after();
+      uint32_t ov[C::NO];
+      if (ok) {
+        const uint32_t col = tmem + lane_base + C::COL_O + (j & 1) * 32;
+        tmem_ld16(col, *reinterpret_cast<uint32_t(*)[16]>(&ov[0]));
+        if constexpr (C::NO == 32) tmem_ld16(col + 16, *reinterpret_cast<uint32_t(*)[16]>(&ov[16]));
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int e = 0; e < C::NO; ++e) ov[e] = 0u;
+      }
+      tc_fence_before();
+      mbar_arrive(ofree + (j & 1));
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float v;
+        if constexpr (C::F8) {
+          v = __uint_as_float(ov[g]) + __uint_as_float(ov[G + g]) * 0.0625f +
+              __uint_as_float(ov[2 * G + g]) * (1.f / 256.f) +
+              __uint_as_float(ov[3 * G + g]) * (1.f / 4096.f);
+        } else if constexpr (C::I8) {
+          v = float(int(ov[g])) + float(int(ov[G + g])) * (1.f / 256.f) +
+              float(int(ov[2 * G + g])) * (1.f / 65536.f);
+        } else {
+          v = __uint_as_float(ov[g]) + __uint_as_float(ov[G + g]) + __uint_as_float(ov[2 * G + g]);
+        }
+        o[g] = o[g] * alpha_pend[g] + v * einv_pend;
+      }
+    };
+
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % C::NST;
+      // ---- S of tile i
+      if (ok) ok = mbar_wait(sfull + (i & 1), (i >> 1) & 1, abort_flag, kMmaWaitLimitCycles);
+      tc_fence_after();
+      uint32_t sw[C::NS];
+      if (ok) {
+        const uint32_t col = tmem + lane_base + C::COL_S + (i & 1) * 32;
+        tmem_ld16(col, *reinterpret_cast<uint32_t(*)[16]>(&sw[0]));
+        if constexpr (C::NS == 32) tmem_ld16(col + 16, *reinterpret_cast<uint32_t(*)[16]>(&sw[16]));
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int e = 0; e < C::NS; ++e) sw[e] = 0u;
+      }
+      tc_fence_before();
+      mbar_arrive(sfree + (i & 1));
+
+      // ---- this token's scales (both copies acquired here, not through the MMA)
+      if (ok) ok = mbar_wait(kfull + s, (i / C::NST) & 1, abort_flag, kMmaWaitLimitCycles);
+      if (ok) ok = mbar_wait(vfull + s, (i / C::NST) & 1, abort_flag, kMmaWaitLimitCycles);
+      const uint32_t mask = ok ? pmask[s] : 0u;   // pages of tile i inside the chunk with legal ids
+      const int tile0 = t0 + 128 * i;
+      const int p = r >> 4, t = r & 15;
+      const bool valid = ok && ((mask >> p) & 1u) && (tile0 + r < t1);
+      float sk = 1.f, zk = 0.f, sv = 0.f, zv = 0.f;
+      if (valid) {
+        if constexpr (C::F8) {
+          sk = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(kmeta + (s * 8 + p) * C::METAB)[t]);
+          sv = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(vmeta + (s * 8 + p) * C::METAB)[t]);
+        } else if constexpr (C::I8) {
+          const __nv_bfloat162 km = reinterpret_cast<const __nv_bfloat162*>(kmeta + (s * 8 + p) * C::METAB)[t];
+          const __nv_bfloat162 vm = reinterpret_cast<const __nv_bfloat162*>(vmeta + (s * 8 + p) * C::METAB)[t];
+          sk = __low2float(km); zk = __high2float(km);
+          sv = __low2float(vm); zv = __high2float(vm);
+        } else {
+          sv = 1.f;
+        }
+      }
+      mbar_arrive(kempty + s);
+
+      // ---- scores (base 2) and the tile max of every head
+      float x[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float sc;
+        if constexpr (C::F8) {
+          sc = __uint_as_float(sw[g]) + __uint_as_float(sw[G + g]) * 0.0625f;
+        } else if constexpr (C::I8) {
+          sc = float(int(sw[g])) + float(int(sw[G + g])) * (1.f / 128.f) +
+               float(int(sw[2 * G + g])) * (1.f / 16384.f) - zk * qz[g];
+        } else {
+          sc = __uint_as_float(sw[g]);
+        }
+        x[g] = valid ? sc * sk * qs[g] : -INFINITY;
+      }
+      float* rb = red + (i & 1) * 64;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float tm = warp_max_f32(x[g]);
+        if (lane == 0) rb[quarter * 16 + g] = tm;
+      }
+      {
+        const float svm = warp_max_f32(sv);
+        if (lane == 0) rb[quarter * 16 + 8] = svm;
+      }
+      named_bar_sync(1, 128);
+      float alpha[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float tmax = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+        const float mn = fmaxf(m[g], tmax);
+        alpha[g] = (mn == -INFINITY) ? 1.f : exp2f(m[g] - mn);
+        m[g] = mn;
+      }
+      // P = p * v_scale * 2^ex with max(v_scale) * 2^ex in [128, 256): inside
+      // the E4M3 range, and below 2^8 for the 24-bit fixed point of INT8
+      const float svmax = fmaxf(fmaxf(rb[8], rb[24]), fmaxf(rb[40], rb[56]));
+      int ex = 0;
+      if (!C::BF && svmax > 0.f) ex = max(-120, min(120, 7 - ilogbf(svmax)));
+      const float escale = __int_as_float((127 + ex) << 23);
+      const float einv = __int_as_float((127 - ex) << 23);
+
+      // ---- tokens of this tile past the chunk end or on a missing page: their
+      // V rows in smem are stale or never written; zero them so that
+      // 0 * (stale code) cannot produce a NaN (integer codes need no care)
+      if constexpr (!C::I8) {
+        if (mask != 0xFFu || tile0 + 128 > t1) {          // uniform over the CTA
+          if (r < D) {
+#pragma unroll 1
+            for (int pp = 0; pp < 8; ++pp) {
+              int ntok = ((mask >> pp) & 1u) ? t1 - (tile0 + 16 * pp) : 0;
+              ntok = max(0, min(16, ntok));
+              if (ntok == 16) continue;
+              uint8_t* vpg = vring + (s * 8 + pp) * C::PAGE;
+#pragma unroll
+              for (int u = 0; u < C::E; ++u) {                 // 16-byte chunks of row r
+                uint4* cp = reinterpret_cast<uint4*>(vpg + u * (D * 16) + r * 16);
+                uint4 w = *cp;
+                uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  uint32_t keep = 0;
+#pragma unroll
+                  for (int bb = 0; bb < 4; ++bb) {
+                    const int tok = (u * 16 + e * 4 + bb) / C::E;   // token of byte bb of word e
+                    if (tok < ntok) keep |= 0xFFu << (8 * bb);
+                  }
+                  ww[e] &= keep;
+                }
+                *cp = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+              }
+            }
+          }
+        }
+      }
+
+      // ---- weights -> P buffer (i & 1), the row of token r
+      uint8_t* pb = pop + (i & 1) * C::PBYTES + prow;
+      if constexpr (C::F8) {
+        // y = y0 + y1/16 + y2/256 + y3/4096, each part E4M3 (RNE); the
+        // residual is exact in FP32 and 16x smaller than the part before
+        float y[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+          l[g] = l[g] * alpha[g] + pr;
+          y[g] = pr * sv * escale;
+        }
+        uint32_t words[C::NO / 4];
+#pragma unroll
+        for (int e = 0; e < C::NO / 4; ++e) words[e] = 0u;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+          for (int g = 0; g < G; g += 2) {
+            const float a = y[g];
+            const float c = (g + 1 < G) ? y[g + 1] : 0.f;
+            const uint32_t code2 = f32x2_to_e4m3x2(a, c);
+            const int n = jj * G + g;                        // byte index in the row
+            words[n >> 2] |= code2 << (8 * (n & 3));
+            if (jj < 3) {
+              float av, cv;
+              e4m3x2_to_f32x2(code2, av, cv);
+              y[g] = (a - av) * 16.f;
+              if (g + 1 < G) y[g + 1] = (c - cv) * 16.f;
+            }
+          }
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < C::NO / 16; ++c16)
+          *reinterpret_cast<uint4*>(pb + c16 * C::P_SBO) =
+              make_uint4(words[4 * c16], words[4 * c16 + 1], words[4 * c16 + 2], words[4 * c16 + 3]);
+      } else if constexpr (C::I8) {
+        // Y = rint(y * 2^16) < 2^24; its three bytes are the parts (weights
+        // 1, 1/256, 1/65536); zero_point * P is summed from the same Y
+        uint32_t yv[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+          l[g] = l[g] * alpha[g] + pr;
+          yv[g] = __float2uint_rn(pr * sv * escale * 65536.f);
+          corr[g] = corr[g] * alpha[g] + zv * float(yv[g]) * (1.f / 65536.f) * einv;
+        }
+        uint32_t words[C::NO / 4];
+#pragma unroll
+        for (int e = 0; e < C::NO / 4; ++e) words[e] = 0u;
+#pragma unroll
+        for (int jj = 0; jj < 3; ++jj) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const int n = jj * G + g;
+            words[n >> 2] |= ((yv[g] >> (16 - 8 * jj)) & 0xFFu) << (8 * (n & 3));
+          }
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < C::NO / 16; ++c16)
+          *reinterpret_cast<uint4*>(pb + c16 * C::P_SBO) =
+              make_uint4(words[4 * c16], words[4 * c16 + 1], words[4 * c16 + 2], words[4 * c16 + 3]);
+      } else {
+        // p = hi + mid + lo, each bf16: 24 significant bits
+        uint32_t words[C::NO / 2];
+#pragma unroll
+        for (int e = 0; e < C::NO / 2; ++e) words[e] = 0u;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+          l[g] = l[g] * alpha[g] + pr;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(pr);
+          const float r1 = pr - __bfloat162float(hi);
+          const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+          const uint16_t parts[3] = {__bfloat16_as_ushort(hi), __bfloat16_as_ushort(mid),
+                                     __bfloat16_as_ushort(lo)};
+#pragma unroll
+          for (int jj = 0; jj < 3; ++jj) {
+            const int n = jj * G + g;
+            words[n >> 1] |= uint32_t(parts[jj]) << (16 * (n & 1));
+          }
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < C::NO / 8; ++c8)
+          *reinterpret_cast<uint4*>(pb + c8 * C::P_SBO) =
+              make_uint4(words[4 * c8], words[4 * c8 + 1], words[4 * c8 + 2], words[4 * c8 + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(pready + (i & 1));
+
+      // ---- O of the previous tile
+      if (i > 0) accum_o(i - 1);
+#pragma unroll
+      for (int g = 0; g < G; ++g) alpha_pend[g] = alpha[g];
+      einv_pend = einv;
+    }
+    if (ntiles > 0) accum_o(ntiles - 1);
+
+    // ---- chunk partial: (max, sum, unnormalised output) per query head
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float ls = warp_sum(l[g]);
+      const float cs = C::I8 ? warp_sum(corr[g]) : 0.f;
+      if (lane == 0) {
+        red2[quarter * 8 + g] = ls;
+        red2[32 + quarter * 8 + g] = cs;
+      }
+    }
+    named_bar_sync(1, 128);
+    if (ok && !*abort_flag) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float L = red2[g] + red2[8 + g] + red2[16 + g] + red2[24 + g];
+        const float Cz = red2[32 + g] + red2[40 + g] + red2[48 + g] + red2[56 + g];
+        const int64_t row = (int64_t(b) * Hq + h * G + g) * max_splits + split;
+        if (r < D) part_o[row * D + r] = o[g] - Cz;
+        if (r == 0) {
+          part_ml[row * 2] = m[g];
+          part_ml[row * 2 + 1] = L;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) flag_error(KVQ_DEVERR_TIMEOUT);
+}
+
+}  // namespace kvq

@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
         const __half2 zsub = __float2half2_rn(1152.f + zk);      // (c + 1152) - (1152 + zp) = c - zp
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c) {
-          const uint4 u = *reinterpret_cast<const uint4*>(pg + c * 256 + t * 16);
+          const uint4 u = *reinterpret_cast<const uint4*>(pg + k_chunk_offset<D * C::ELT>(c, t));
           const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
           if constexpr (C::BF) {
 #pragma unroll

@@ -38,6 +38,15 @@ __device__ unsigned int g_error_word;
 __device__ __forceinline__ void flag_error(unsigned int bit) { atomicOr(&g_error_word, bit); }
 
 // ------------------------------------------------------------------ helpers
+// Byte offset, inside a K page whose token rows are ROWB bytes, of 16-byte
+// chunk c of token t: tokens come in two groups of 8, and a group stores its
+// chunk 0 for tokens 0..7, then chunk 1, ... (8 x 16-byte core matrices, the
+// K-major operand layout of the tensor cores).
+template <int ROWB>
+__host__ __device__ __forceinline__ int k_chunk_offset(int c, int t) {
+  return (t >> 3) * (8 * ROWB) + c * 128 + (t & 7) * 16;
+}
+
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
@@ -80,11 +89,13 @@ __device__ __forceinline__ void codes4_to_f32(uint32_t w, float* o) {
 
 }  // namespace kvq
 
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
 #include <utility>
 
 #include "kvq_decode_tc.cuh"
+#include "kvq_decode_mma.cuh"
 
 namespace kvq {
 
@@ -221,7 +232,7 @@ __global__ void __launch_bounds__(256) append_kernel(
     const int off = int(slot % kBlockSize);
     if (which == 0) {
       // this token's chunk(s) of the K page: element d at chunk d*ELT/16
-      uint8_t* dst = kc + page * PAGEB + ((d0 * ELT) / 16) * 256 + off * 16 + (d0 * ELT) % 16;
+      uint8_t* dst = kc + page * PAGEB + k_chunk_offset<ROWB>((d0 * ELT) / 16, off) + (d0 * ELT) % 16;
       if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
       else if constexpr (E * ELT == 4) *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
       else *reinterpret_cast<uint16_t*>(dst) = uint16_t(rc.w[0]);
@@ -252,9 +263,10 @@ __global__ void __launch_bounds__(256) append_kernel(
   const int64_t page = (s0 / kBlockSize) * Hk + h;
   uint8_t* kp = kc + page * PAGEB;
   uint8_t* vp = vc + page * PAGEB;
-  // K: chunk j = (c, t) <- bytes [16c, 16c+16) of token t's row
+  // K: chunk j = (token group t/8, c, t%8) <- bytes [16c, 16c+16) of token t's row
   for (int j = threadIdx.x; j < PAGEB / 16; j += blockDim.x) {
-    const int c = j >> 4, t = j & 15;
+    constexpr int NC = ROWB / 16;
+    const int c = (j >> 3) % NC, t = (j / (8 * NC)) * 8 + (j & 7);
     *reinterpret_cast<uint4*>(kp + j * 16) = *reinterpret_cast<const uint4*>(kbuf + t * PADB + c * 16);
   }
   // V: chunk j = (u, d) <- tokens [u*16/ELT, (u+1)*16/ELT) of channel d
@@ -383,7 +395,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
     const uint8_t* kpage = kc + page * C::PAGE_BYTES;
 #pragma unroll
     for (int i = 0; i < C::KU4; ++i)
-      kr[i] = __ldg(reinterpret_cast<const uint4*>(kpage + (half * C::KU4 + i) * 256 + t_in * 16));
+      kr[i] = __ldg(reinterpret_cast<const uint4*>(kpage + k_chunk_offset<D * ELT>(half * C::KU4 + i, t_in)));
     const uint8_t* vpage = vc + page * C::PAGE_BYTES;
 #pragma unroll
     for (int j = 0; j < C::ROWS; ++j) {
@@ -610,15 +622,41 @@ cudaError_t decode_tc_dispatch3(const void* q, int32_t B, const void* kc, const 
   return cudaGetLastError();
 }
 
-// The tensor-core kernel is the decode path; KVQ_DECODE_KERNEL=simt selects the
-// CUDA-core kernel instead (kept to measure one against the other).
-bool use_simt_decode() {
-  static const bool simt = [] {
-    const char* v = std::getenv("KVQ_DECODE_KERNEL");
-    return v != nullptr && std::strcmp(v, "simt") == 0;
-  }();
-  return simt;
+template <int D, int G, int FMT>
+cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
+                                 const void* ks, const void* vs, const int32_t* tables,
+                                 const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                                 const DecodePlan& plan, void* ws, const kvq_dims& d,
+                                 cudaStream_t st) {
+  using C = MmaCfg<D, G, FMT>;
+  auto kern = decode_mma_kernel<D, G, FMT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  float* po = static_cast<float*>(ws);
+  float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
+  const int64_t grid = int64_t(B) * d.n_kv_heads * plan.max_splits;
+  kern<<<dim3(unsigned(grid)), 192, C::SMEM, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
+      static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
+      static_cast<const __nv_bfloat16*>(vs), tables, ctx, d.n_kv_heads, d.num_blocks,
+      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml);
+  return cudaGetLastError();
 }
+
+// Decode kernel: the tensor-core kernel that multiplies the stored codes
+// directly. For measuring one design against another, KVQ_DECODE_KERNEL=tc
+// selects the tensor-core kernel that first converts the codes to f16 in
+// registers, and KVQ_DECODE_KERNEL=simt the CUDA-core kernel.
+int decode_kernel_choice() {
+  static const int choice = [] {
+    const char* v = std::getenv("KVQ_DECODE_KERNEL");
+    if (v != nullptr && std::strcmp(v, "simt") == 0) return 2;
+    if (v != nullptr && std::strcmp(v, "tc") == 0) return 1;
+    return 0;
+  }();
+  return choice;
+}
+bool use_simt_decode() { return decode_kernel_choice() == 2; }
 
 template <int D, int FMT>
 cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, const void* vc,
@@ -626,7 +664,15 @@ cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, co
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
                              const DecodePlan& plan, void* ws, const kvq_dims& d,
                              cudaStream_t st) {
-  if (!use_simt_decode()) {
+  if (decode_kernel_choice() == 0) {
+    switch (G) {
+      case 1: return decode_mma_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+      case 2: return decode_mma_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+      case 4: return decode_mma_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+      default: return decode_mma_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
+    }
+  }
+  if (decode_kernel_choice() == 1) {
     switch (G) {
       case 1: return decode_tc_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
       case 2: return decode_tc_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
 
 namespace kvq {
 namespace tc {
@@ -178,6 +179,74 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int k, int rows) {
   const int atom = k >> 6;
   const uint32_t logical = uint32_t(row) * 128u + uint32_t(k & 63) * 2u;
   return uint32_t(atom) * uint32_t(rows) * 128u + (logical ^ (uint32_t(row & 7) << 4));
+}
+
+// D[tmem] (+)= A[smem] x B[smem], both operands through shared-memory
+// descriptors. KIND selects the operand family: 0 = kind::f16 (f16/bf16),
+// 1 = kind::f8f6f4 (8-bit and narrower floats), 2 = kind::i8 (s8/u8, s32 sums).
+template <int KIND>
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  if constexpr (KIND == 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else if constexpr (KIND == 1) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
+// Instruction descriptor, M = 128: D format (1 = f32, 2 = s32), A and B formats
+// (kind::f16: 0 f16, 1 bf16; kind::f8f6f4: 0 E4M3; kind::i8: 0 u8, 1 s8), A
+// K-major, B K-major (b_mn = false) or MN-major (b_mn = true), N columns.
+__host__ __device__ constexpr uint32_t idesc_m128(uint32_t d_fmt, uint32_t a_fmt, uint32_t b_fmt,
+                                                 bool b_mn, int n) {
+  return (d_fmt << 4) | (a_fmt << 7) | (b_fmt << 10) | ((b_mn ? 1u : 0u) << 16) |
+         (uint32_t(n >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+}
+
+// Shared-memory descriptor of an operand in the no-swizzle (interleaved)
+// layout: 8 x 16-byte core matrices of 128 contiguous bytes. For a K-major
+// operand `lbo` is the byte distance between core matrices adjacent in K and
+// `sbo` between core matrices adjacent in M/N; for an MN-major operand `lbo`
+// steps K by 8 rows and `sbo` steps M/N by 16 bytes of elements.
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;                      // descriptor version (sm_100); layout 0 = none
+  return d;
+}
+
+// Two floats -> two E4M3 codes (RNE, saturating), `lo_val` in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo_val, float hi_val) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi_val), "f"(lo_val));
+  return r;
+}
+// Two E4M3 codes (low byte first) -> their exact values.
+__device__ __forceinline__ void e4m3x2_to_f32x2(uint32_t codes, float& lo_val, float& hi_val) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t}\n"
+      : "=r"(h2)
+      : "r"(codes));
+  const __half2 hv = *reinterpret_cast<const __half2*>(&h2);
+  lo_val = __low2float(hv);
+  hi_val = __high2float(hv);
 }
 
 // Two E4M3 codes per 16-bit half of `w` -> two packed f16x2 words (exact).

@@ -282,7 +282,7 @@ class LayerCache:
         nb, hk, D = d.num_blocks, d.n_kv_heads, d.head_dim
         E = ELEM_BYTES[fmt]
         edt = torch.bfloat16 if fmt == "bf16" else torch.uint8
-        k = torch.zeros((nb, hk, D * E // 16, BLOCK_SIZE, 16 // E), dtype=edt, device=device)
+        k = torch.zeros((nb, hk, 2, D * E // 16, 8, 16 // E), dtype=edt, device=device)
         v = torch.zeros((nb, hk, E, D, 16 // E), dtype=edt, device=device)
         mv = META_VALUES[fmt]
         if mv:
@@ -318,8 +318,8 @@ class LayerCache:
     def k_logical(self, blocks=None):
         """K of all blocks (or of the block ids `blocks`) as [n][Hk][block_size][D]."""
         k = self.k if blocks is None else self.k[blocks]
-        return k.permute(0, 1, 3, 2, 4).reshape(k.shape[0], k.shape[1], BLOCK_SIZE,
-                                                self.dims.head_dim)
+        return k.permute(0, 1, 2, 4, 3, 5).reshape(k.shape[0], k.shape[1], BLOCK_SIZE,
+                                                   self.dims.head_dim)
 
     def v_logical(self, blocks=None):
         """V of all blocks (or of the block ids `blocks`) as [n][Hk][block_size][D]."""
