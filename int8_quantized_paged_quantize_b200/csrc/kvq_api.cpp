@@ -49,10 +49,12 @@ int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kv
   const int64_t splits = std::max<int64_t>(1, (int64_t(max_ctx) + part - 1) / part);
   plan->partition = int32_t(part);
   plan->max_splits = int32_t(splits);
-  const size_t rows = size_t(batch) * d->n_q_heads * size_t(splits);
+  plan->slots = int32_t(splits + 1);
+  const size_t rows = size_t(batch) * d->n_q_heads * size_t(plan->slots);
   plan->o_bytes = round256(rows * d->head_dim * sizeof(float));
   plan->ml_bytes = round256(rows * 2 * sizeof(float));
-  plan->total = plan->o_bytes + plan->ml_bytes;
+  plan->cnt_bytes = round256(size_t(batch) * d->n_kv_heads * sizeof(int32_t));
+  plan->total = plan->o_bytes + plan->ml_bytes + plan->cnt_bytes;
   return KVQ_OK;
 }
 

@@ -4,14 +4,25 @@
 // dequantizes a K or V element; the per-token scales and zero points are applied
 // to the small S and P tiles instead. Included by kvq_kernels.cu.
 //
-// One CTA per (sequence b, KV head h, chunk of `part` tokens), 6 warps:
+// Work split (persistent, stream-K): the work list is every (sequence b, KV
+// head h, 128-token tile) in order of b, then h, then tile. Each of the N
+// resident CTAs takes one contiguous, equal share of it (N is cut so that a
+// share holds at least `unit_tiles` tiles). A share is a few "pieces", a piece
+// being the share's run of tiles of one (b, h); each piece ends in an
+// online-softmax partial (max, sum, unnormalised output) in a workspace slot,
+// and the piece holding the last tile of (b, h) records how many slots the
+// merge kernel must combine. The ring of K/V stages streams across piece
+// boundaries, so a CTA fills its pipeline once.
+//
+// 6 warps per CTA:
 //   warp 0      producer: lanes 0..7 each own one page of a 128-token tile and
 //               issue its 1-D bulk copy (K page, then V page) into a ring of
 //               smem stages; lanes 8..15 copy the pages' scales. The block ids
 //               of the next tile are loaded while the current one is issued.
 //   warp 1      allocates TMEM; one thread issues the MMAs.
 //   warps 2..5  softmax warps, one per TMEM lane quarter; thread r owns token r
-//               of the tile for S and P, channel r for O.
+//               of the tile for S and P, channel r for O. They also build the
+//               query operand of each piece, loading it one piece ahead.
 // Per 128-token tile:
 //   S^T[tok x n] = Kcodes[tok x D] . Qp^T[D x n]    (A: K page ring, K-major;
 //                  B: the query group split into exact low-precision parts)
@@ -23,10 +34,10 @@
 //   O^T[ch x n] = Vcodes^T[ch x tok] . P[tok x n]    (A: V page ring, K-major)
 //   O tile -> registers, parts recombined, rescaled and accumulated in FP32.
 // Each MMA result sits in TMEM; S, P and O are double-buffered so the MMA of
-// one tile overlaps the softmax of the next. Every byte of the chunk's K/V
-// crosses HBM once for the whole query group. Every wait is bounded: on expiry
-// the CTA sets KVQ_DEVERR_TIMEOUT, stops issuing work, drains what it issued,
-// frees TMEM and returns.
+// one tile overlaps the softmax of the next. Every byte of the K/V crosses HBM
+// once for the whole query group. Every wait is bounded: on expiry the CTA sets
+// KVQ_DEVERR_TIMEOUT, stops issuing work, drains what it issued, frees TMEM
+// and returns.
 
 #pragma once
 
@@ -35,6 +46,9 @@
 namespace kvq {
 
 constexpr long long kMmaWaitLimitCycles = 2000000000LL;   // about one second
+
+__device__ __forceinline__ long long ll_min(long long a, long long b) { return a < b ? a : b; }
+__device__ __forceinline__ long long ll_max(long long a, long long b) { return a > b ? a : b; }
 
 __host__ __device__ constexpr int round_up16(int x) { return x < 16 ? 16 : (x + 15) / 16 * 16; }
 
@@ -53,7 +67,10 @@ struct MmaCfg {
   static constexpr int PPARTS = F8 ? 4 : 3;
   static constexpr int NS = round_up16(QPARTS * G);            // S columns (B rows of QK)
   static constexpr int NO = round_up16(PPARTS * G);            // O columns (B rows of PV)
+  static constexpr int NSL = (QPARTS * G + 7) / 8 * 8;         // S columns read back
+  static constexpr int NOL = (PPARTS * G + 7) / 8 * 8;         // O columns read back
   static_assert(NS <= 32 && NO <= 32, "query group too large");
+  static constexpr int HPW = (G + 3) / 4;                      // query heads per softmax warp
   static constexpr int S_MMAS = D * E / 32;                    // K extent of one MMA: 32 bytes
   static constexpr int PV_MMAS = 128 * E / 32;
   // operand strides (bytes)
@@ -62,7 +79,7 @@ struct MmaCfg {
   static constexpr uint32_t Q_SBO = 128, Q_LBO = (NS / 8) * 128;
   static constexpr int PT = 16 / E;                            // P elements per 16-byte row
   static constexpr uint32_t P_SBO = 128, P_LBO = (NO / PT) * 128;
-  static constexpr int QBYTES = NS * D * E;
+  static constexpr int QBYTES = NS * D * E;                    // one query operand
   static constexpr int PBYTES = NO * 128 * E;                  // one P buffer
   // TMEM columns
   static constexpr int COL_S = 0, COL_O = 64, TMEM_COLS = 128;
@@ -72,45 +89,164 @@ struct MmaCfg {
   static constexpr int OFF_KM = OFF_V + NST * 8 * PAGE;
   static constexpr int OFF_VM = OFF_KM + NST * 8 * METAB;
   static constexpr int OFF_Q = (OFF_VM + NST * 8 * METAB + 127) / 128 * 128;
-  static constexpr int OFF_P = OFF_Q + QBYTES;
+  static constexpr int OFF_P = OFF_Q + QBYTES;                                  // [2]
   static constexpr int OFF_BAR = OFF_P + 2 * PBYTES;
-  static constexpr int NBAR = 4 * NST + 10 + 1;
-  static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;           // float [2][4][16]
-  static constexpr int OFF_RED2 = OFF_RED + 2 * 4 * 16 * 4;    // float [2][4][8]
-  static constexpr int OFF_QSC = OFF_RED2 + 2 * 4 * 8 * 4;     // float [8] scale, float [8] sum(q)
+  static constexpr int NBAR = 4 * NST + 12 + 1;
+  static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;           // float [2][4][16]; prologue scratch
+  static constexpr int OFF_RED2 = OFF_RED + 2 * 4 * 16 * 4;    // float [2][4][8]: sums, zero-point terms
+  static constexpr int OFF_QSC = OFF_RED2 + 2 * 4 * 8 * 4;     // float [8] scale, [8] sum(q)
   static constexpr int OFF_PMASK = OFF_QSC + 16 * 4;           // uint32 [NST] valid-page masks
-  static constexpr int OFF_MISC = OFF_PMASK + 4 * NST;         // tmem base, abort flag
-  static constexpr int SMEM = OFF_MISC + 16 + 128;             // + alignment slack
+  static constexpr int OFF_MISC = (OFF_PMASK + 4 * NST + 15) / 16 * 16;   // tmem base, abort flag, start (b, P)
+  static constexpr int OFF_WALK = OFF_MISC + 32;               // softmax piece cursor [2] + slots [2][2]
+  static constexpr int SMEM = OFF_WALK + 160 + 128;            // + alignment slack
 };
 
+// Context length of sequence b if it is legal, else 0.
+__device__ __forceinline__ int mma_seq_ctx(const int32_t* ctx_lens, int b, int max_ctx, int W) {
+  const int c = ctx_lens[b];
+  return (c < 0 || c > max_ctx || int64_t(c) > int64_t(W) * kBlockSize) ? 0 : c;
+}
+
+// Cursor over the pieces of one CTA's share [g, end) of the work list. Every
+// role walks it the same way; the next sequence's length is loaded one
+// sequence ahead so that stepping over a sequence boundary does not wait.
+struct PieceWalk {
+  int b, h, lo, hi;          // sequence, KV head, tiles [lo, hi) of that sequence
+  int nt, ctx;               // tiles and tokens of sequence b
+  int ctx_next;              // length of sequence b + 1 (0 past the batch)
+  long long P;               // tiles of sequences 0 .. b-1
+  long long g, end;          // work-list index of tile lo; end of the share
+  bool done;
+
+  __device__ __forceinline__ void load_next(const int32_t* ctx_lens, int B, int max_ctx, int W) {
+    ctx_next = (b + 1 < B) ? mma_seq_ctx(ctx_lens, b + 1, max_ctx, W) : 0;
+  }
+  __device__ __forceinline__ void init(int b0, long long P0, long long start, long long end_,
+                                       int Hk, const int32_t* ctx_lens, int B, int max_ctx, int W) {
+    b = b0; P = P0; g = start; end = end_;
+    ctx = mma_seq_ctx(ctx_lens, b, max_ctx, W);
+    nt = (ctx + 127) / 128;
+    load_next(ctx_lens, B, max_ctx, W);
+    done = g >= end || nt == 0;
+    const long long off = g - int64_t(Hk) * P;
+    h = done ? 0 : int(off / nt);
+    lo = done ? 0 : int(off % nt);
+    hi = done ? 0 : int(ll_min(nt, lo + (end - g)));
+  }
+  __device__ __forceinline__ void next(int Hk, const int32_t* ctx_lens, int B, int max_ctx, int W) {
+    g += hi - lo;
+    if (g >= end) { done = true; return; }
+    if (++h == Hk) {
+      h = 0;
+      P += nt;
+      ++b;
+      ctx = ctx_next;
+      nt = (ctx + 127) / 128;
+      load_next(ctx_lens, B, max_ctx, W);
+      while (nt == 0) {                          // empty sequences hold no tiles
+        ++b;
+        ctx = ctx_next;
+        nt = (ctx + 127) / 128;
+        load_next(ctx_lens, B, max_ctx, W);
+      }
+    }
+    lo = 0;
+    hi = int(ll_min(nt, end - g));
+  }
+};
+
+static_assert(2 * sizeof(PieceWalk) + 16 <= 160, "piece cursor area");
+
+// Columns [0, N) (N a multiple of 8, at most 32) of this warp's TMEM lanes.
+template <int N>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t* r) {
+  static_assert(N % 8 == 0 && N <= 32, "columns");
+  if constexpr (N >= 16) tc::tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+  if constexpr (N == 32) tc::tmem_ld16(taddr + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+  if constexpr (N % 16 == 8) tc::tmem_ld8(taddr + (N - 8), r + (N - 8));
+}
+
 template <int D, int G, int FMT>
-__global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_mma_kernel(
+__global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kc,
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
-    const int32_t* __restrict__ ctx_lens, int Hk, int NB, int W, int max_ctx, int part,
-    int max_splits, float qk_scale, float* __restrict__ part_o, float* __restrict__ part_ml) {
+    const int32_t* __restrict__ ctx_lens, int B, int Hk, int NB, int W, int max_ctx,
+    int unit_tiles, int slots, float qk_scale, float* __restrict__ part_o,
+    float* __restrict__ part_ml, int32_t* __restrict__ part_cnt) {
   using C = MmaCfg<D, G, FMT>;
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x % max_splits;
-  const int bh = blockIdx.x / max_splits;
-  const int b = bh / Hk, h = bh % Hk;
   const int Hq = Hk * G;
 
-  int ctx = ctx_lens[b];
-  if (ctx < 0 || ctx > max_ctx || int64_t(ctx) > int64_t(W) * kBlockSize) {
-    if (threadIdx.x == 0 && split == 0) flag_error(KVQ_DEVERR_CONTEXT);
-    ctx = 0;
+  // ------------------------------------------------------------ the share
+  // T = total tiles; each thread sums the tiles of some sequences
+  long long* red64 = reinterpret_cast<long long*>(smem + C::OFF_RED);   // [6] + 2
+  long long* miscll = reinterpret_cast<long long*>(smem + C::OFF_MISC + 16);
+  int* misci = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  {
+    long long tsum = 0;
+    for (int bb = threadIdx.x; bb < B; bb += blockDim.x) {
+      const int c = ctx_lens[bb];
+      if (c < 0 || c > max_ctx || int64_t(c) > int64_t(W) * kBlockSize) {
+        if (blockIdx.x == 0) flag_error(KVQ_DEVERR_CONTEXT);
+      } else {
+        tsum += (c + 127) / 128;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, o);
+    if (lane == 0) red64[warp] = tsum;
   }
-  const int n_splits = (ctx + part - 1) / part;
-  if (split >= n_splits) return;                         // uniform for the CTA
-  const int t0 = split * part, t1 = min(ctx, t0 + part);
-  const int ntiles = (t1 - t0 + 127) / 128;
-  const int32_t* trow = tables + int64_t(b) * W;
+  __syncthreads();
+  long long T = 0;
+#pragma unroll
+  for (int w = 0; w < 6; ++w) T += red64[w];
+  T *= Hk;
+  const long long N = ll_min(gridDim.x, ll_max(1, T / max(1, unit_tiles)));
+  if (T == 0 || blockIdx.x >= N) return;                 // uniform for the CTA
+  const long long start = (int64_t(blockIdx.x) * T) / N;
+  const long long end = (int64_t(blockIdx.x + 1) * T) / N;
+  // the sequence holding tile `start`: block-wide scan of tiles per sequence
+  {
+    if (threadIdx.x == 0) misci[0] = -1;
+    __syncthreads();
+    long long run = 0;
+    for (int base = 0; base < B; base += blockDim.x) {
+      const int bb = base + threadIdx.x;
+      const int tb = bb < B ? (mma_seq_ctx(ctx_lens, bb, max_ctx, W) + 127) / 128 : 0;
+      long long incl = tb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      __syncthreads();
+      if (lane == 31) red64[warp] = incl;
+      __syncthreads();
+      long long before = 0, total = 0;
+#pragma unroll
+      for (int w = 0; w < 6; ++w) {
+        before += (w < warp) ? red64[w] : 0;
+        total += red64[w];
+      }
+      const long long lo_t = run + before + incl - tb;          // tiles before sequence bb
+      if (bb < B && tb > 0 && int64_t(Hk) * lo_t <= start && start < int64_t(Hk) * (lo_t + tb)) {
+        misci[0] = bb;
+        miscll[0] = lo_t;
+      }
+      run += total;
+      __syncthreads();
+      if (misci[0] >= 0) break;                                 // uniform
+    }
+  }
+  const int b0 = misci[0];
+  const long long P0 = miscll[0];
+  // CTA that holds work-list tile x; the slot of a piece is its CTA's rank
+  // among the CTAs that share the piece's (b, h)
+  auto cta_of = [&](long long x) -> long long { return ((x + 1) * N - 1) / T; };
 
   uint8_t* kring = smem + C::OFF_K;
   uint8_t* vring = smem + C::OFF_V;
@@ -128,7 +264,9 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_mma_kerne
   uint64_t* pready = sfree + 2;             // [2]
   uint64_t* ofull = pready + 2;             // [2]
   uint64_t* ofree = ofull + 2;              // [2]
-  uint64_t* drain = ofree + 2;
+  uint64_t* qready = ofree + 2;
+  uint64_t* qfree = qready + 1;
+  uint64_t* drain = qfree + 1;
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
   float* red2 = reinterpret_cast<float*>(smem + C::OFF_RED2);
   float* qsc = reinterpret_cast<float*>(smem + C::OFF_QSC);
@@ -138,6 +276,7 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_mma_kerne
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   // ------------------------------------------------------------ set-up
+  __syncthreads();                                          // prologue scratch read by all
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(kfull + s, 1);
@@ -152,6 +291,8 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_mma_kerne
       mbar_init(ofull + j, 1);
       mbar_init(ofree + j, 128);
     }
+    mbar_init(qready, 128);
+    mbar_init(qfree, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -161,101 +302,48 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_mma_kerne
     tmem_relinquish();
   }
   if (warp >= 2) {
-    const int ct = threadIdx.x - 64;                       // 0..127
-    // zero the Q and P operands (padding rows stay zero)
+    // zero the query operand and both P buffers (padding rows stay zero)
+    const int ct = threadIdx.x - 64;
     for (int i = ct * 16; i < C::QBYTES + 2 * C::PBYTES; i += 128 * 16)
       *reinterpret_cast<uint4*>(qop + i) = make_uint4(0, 0, 0, 0);
-    named_bar_sync(1, 128);
-    // Q parts, B operand of S (K-major, no swizzle): row n = part * G + g,
-    // element (n, d) at (n/8)*Q_SBO + (n%8)*16 + (d*E/16)*Q_LBO + (d*E)%16.
-    const int cw = warp - 2;
-    for (int g = cw; g < G; g += 4) {
-      const __nv_bfloat16* qr = q + (int64_t(b) * Hq + h * G + g) * D;
-      float v[D / 32];
-      float amax = 0.f;
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) {
-        v[i] = __bfloat162float(qr[lane + 32 * i]);
-        amax = fmaxf(amax, fabsf(v[i]));
-      }
-      amax = warp_max(amax);
-      // power-of-two scaling of the head: FP8 puts max|q| into [128, 256)
-      // (inside the E4M3 range), INT8 into [32, 64) (parts within +-64)
-      int e = 0;
-      if (!C::BF && amax > 0.f) e = (C::F8 ? 7 : 5) - ilogbf(amax);
-      e = max(-120, min(120, e));
-      const float up = __int_as_float((127 + e) << 23);
-      const float down = __int_as_float((127 - e) << 23);
-      int isum = 0;
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) {
-        const int d = lane + 32 * i;
-        auto at = [&](int n) -> uint8_t* {
-          return qop + (n >> 3) * C::Q_SBO + (n & 7) * 16 + ((d * C::E) >> 4) * C::Q_LBO +
-                 ((d * C::E) & 15);
-        };
-        if constexpr (C::BF) {
-          *reinterpret_cast<uint16_t*>(at(g)) = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
-        } else if constexpr (C::F8) {
-          // x = hi + lo/16 with both parts E4M3: exact for a BF16 value unless
-          // it lies below the E4M3 normal range after scaling
-          const float x = v[i] * up;
-          const uint32_t hc = f32x2_to_e4m3x2(x, 0.f) & 0xFFu;
-          float hv, unused;
-          e4m3x2_to_f32x2(hc, hv, unused);
-          const uint32_t lc = f32x2_to_e4m3x2((x - hv) * 16.f, 0.f) & 0xFFu;
-          *at(g) = uint8_t(hc);
-          *at(G + g) = uint8_t(lc);
-        } else {
-          // x = x0 + x1/128 + x2/16384, every part an integer in [-64, 64]
-          const float x = v[i] * up;
-          const float x0 = rintf(x);
-          const float r0 = (x - x0) * 128.f;
-          const float x1 = rintf(r0);
-          const float x2 = rintf((r0 - x1) * 128.f);
-          const int i0 = int(x0), i1 = int(x1), i2 = int(x2);
-          *at(g) = uint8_t(int8_t(i0));
-          *at(G + g) = uint8_t(int8_t(i1));
-          *at(2 * G + g) = uint8_t(int8_t(i2));
-          isum += i0 * 16384 + i1 * 128 + i2;
-        }
-      }
-      if constexpr (C::I8) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
-      }
-      if (lane == 0) {
-        qsc[g] = qk_scale * down;
-        qsum[g] = float(isum) * (1.f / 16384.f);           // sum of q in the units of S
-      }
-    }
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  PieceWalk walk;
+  walk.init(b0, P0, start, end, Hk, ctx_lens, B, max_ctx, W);
+
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     const uint64_t pol = l2_evict_first_policy();
     const int p8 = lane & 7;
-    auto load_id = [&](int i) -> int {
-      if (lane >= 8 || i >= ntiles) return -2;
-      const int tok0 = t0 + 128 * i;
+    // block id of page p8 of tile `tile` of the current piece of `pw`
+    auto load_id = [&](const PieceWalk& pw, int tile) -> int {
+      if (lane >= 8 || pw.done) return -2;
+      const int tok0 = tile * 128;
+      const int t1 = min(pw.hi * 128, pw.ctx);
       const int npg = min(8, (t1 - tok0 + kBlockSize - 1) / kBlockSize);
-      return p8 < npg ? trow[tok0 / kBlockSize + p8] : -2;   // -2: no page here
+      return p8 < npg ? tables[int64_t(pw.b) * W + tok0 / kBlockSize + p8] : -2;   // -2: no page here
     };
-    int id_next = load_id(0);
+    PieceWalk nx = walk;                 // cursor of the next tile
+    int ntile = nx.lo;
+    int id_next = load_id(nx, ntile);
     bool kiss[C::NST], viss[C::NST];
     uint32_t kpar[C::NST], vpar[C::NST];
 #pragma unroll
     for (int s = 0; s < C::NST; ++s) { kiss[s] = viss[s] = false; kpar[s] = vpar[s] = 0; }
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i % C::NST;
-      const uint32_t ph = (i / C::NST) & 1;
+    for (int gt = 0; !nx.done; ++gt) {
+      const int s = gt % C::NST;
+      const uint32_t ph = (gt / C::NST) & 1;
+      const int h = nx.h;
       const int id = id_next;
-      id_next = load_id(i + 1);
+      if (++ntile >= nx.hi) {
+        nx.next(Hk, ctx_lens, B, max_ctx, W);
+        ntile = nx.lo;
+      }
+      id_next = load_id(nx, ntile);
       if (lane < 8 && id != -2 && (id < 0 || id >= NB)) flag_error(KVQ_DEVERR_BLOCK);
       const bool valid = lane < 8 && id >= 0 && id < NB;
       const uint32_t mask = __ballot_sync(0xffffffffu, valid) & 0xFFu;
@@ -314,39 +402,49 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_mma_kerne
       const uint32_t kbase = smem_u32(kring), vbase = smem_u32(vring);
       const uint32_t qaddr = smem_u32(qop), paddr = smem_u32(pop);
       bool ok = true;
-      for (int i = 0; ok && i <= ntiles; ++i) {
-        if (i < ntiles) {
-          const int s = i % C::NST;
-          ok = mbar_wait(kfull + s, (i / C::NST) & 1, abort_flag, kMmaWaitLimitCycles) &&
-               mbar_wait(sfree + (i & 1), ((i >> 1) & 1) ^ 1, abort_flag, kMmaWaitLimitCycles);
+      int gt = 0;
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % C::NST;
+        if (!mbar_wait(pready + (j & 1), (j >> 1) & 1, abort_flag, kMmaWaitLimitCycles)) return false;
+        if (!mbar_wait(ofree + (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, kMmaWaitLimitCycles)) return false;
+        tc_fence_after();
+        const uint32_t a0 = vbase + s * 8 * C::PAGE;
+        const uint32_t b0 = paddr + (j & 1) * C::PBYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::PV_MMAS; ++kk)
+          mma_ss<C::KIND>(tmem + C::COL_O + (j & 1) * 32,
+                          sdesc_plain(a0 + kk * 2 * C::V_LBO, C::V_LBO, C::V_SBO),
+                          sdesc_plain(b0 + kk * (4 / C::E) * C::P_LBO, C::P_LBO, C::P_SBO), id_pv,
+                          kk > 0);
+        mma_commit(ofull + (j & 1));
+        mma_commit(vempty + s);
+        return true;
+      };
+      for (int pc = 0; ok && !walk.done; ++pc) {
+        // the query operand of piece pc (one buffer: the softmax warps rewrite
+        // it only after every S product of the piece before has been read)
+        ok = mbar_wait(qready, pc & 1, abort_flag, kMmaWaitLimitCycles);
+        tc_fence_after();
+        const uint32_t qa = qaddr;
+        for (int i = walk.lo; ok && i < walk.hi; ++i, ++gt) {
+          const int s = gt % C::NST;
+          ok = mbar_wait(kfull + s, (gt / C::NST) & 1, abort_flag, kMmaWaitLimitCycles) &&
+               mbar_wait(sfree + (gt & 1), ((gt >> 1) & 1) ^ 1, abort_flag, kMmaWaitLimitCycles);
           if (!ok) break;
           tc_fence_after();
           const uint32_t a0 = kbase + s * 8 * C::PAGE;
 #pragma unroll
           for (int kk = 0; kk < C::S_MMAS; ++kk)
-            mma_ss<C::KIND>(tmem + C::COL_S + (i & 1) * 32,
+            mma_ss<C::KIND>(tmem + C::COL_S + (gt & 1) * 32,
                             sdesc_plain(a0 + kk * 2 * C::K_LBO, C::K_LBO, C::K_SBO),
-                            sdesc_plain(qaddr + kk * 2 * C::Q_LBO, C::Q_LBO, C::Q_SBO), id_s, kk > 0);
-          mma_commit(sfull + (i & 1));
+                            sdesc_plain(qa + kk * 2 * C::Q_LBO, C::Q_LBO, C::Q_SBO), id_s, kk > 0);
+          mma_commit(sfull + (gt & 1));
+          if (gt >= 1) ok = issue_pv(gt - 1);
         }
-        if (i >= 1) {
-          const int j = i - 1, s = j % C::NST;
-          ok = mbar_wait(pready + (j & 1), (j >> 1) & 1, abort_flag, kMmaWaitLimitCycles) &&
-               mbar_wait(ofree + (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, kMmaWaitLimitCycles);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t a0 = vbase + s * 8 * C::PAGE;
-          const uint32_t b0 = paddr + (j & 1) * C::PBYTES;
-#pragma unroll
-          for (int kk = 0; kk < C::PV_MMAS; ++kk)
-            mma_ss<C::KIND>(tmem + C::COL_O + (j & 1) * 32,
-                            sdesc_plain(a0 + kk * 2 * C::V_LBO, C::V_LBO, C::V_SBO),
-                            sdesc_plain(b0 + kk * (4 / C::E) * C::P_LBO, C::P_LBO, C::P_SBO), id_pv,
-                            kk > 0);
-          mma_commit(ofull + (j & 1));
-          mma_commit(vempty + s);
-        }
+        if (ok) mma_commit(qfree);                         // this piece's S products are issued
+        walk.next(Hk, ctx_lens, B, max_ctx, W);
       }
+      if (ok && gt >= 1) issue_pv(gt - 1);
       // every MMA issued so far completes before TMEM is released
       volatile int no_abort = 0;
       mma_commit(drain);
@@ -356,296 +454,425 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_mma_kerne
     // ---------------------------------------------------------- softmax warps
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                  // token / channel / TMEM lane
+    const int cw = warp - 2;                            // query heads cw, cw + 4 of a piece
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    float qs[G], qz[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) { qs[g] = qsc[g]; qz[g] = qsum[g]; }
-    float m[G], l[G], corr[G], o[G], alpha_pend[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      m[g] = -INFINITY; l[g] = 0.f; corr[g] = 0.f; o[g] = 0.f; alpha_pend[g] = 1.f;
-    }
-    float einv_pend = 1.f;
     bool ok = true;
     // this token's row of a P buffer (MN-major): element n at
     // (n / PT) * P_SBO + (n % PT) * E, plus the row's own offset
     const uint32_t prow = (r >> 3) * C::P_LBO + (r & 7) * 16;
-
-    auto accum_o = [&](int j) {
-      if (ok) ok = mbar_wait(ofull + (j & 1), (j >> 1) & 1, abort_flag, kMmaWaitLimitCycles);
-      tc_fence_after();
-      uint32_t ov[C::NO];
-      if (ok) {
-        const uint32_t col = tmem + lane_base + C::COL_O + (j & 1) * 32;
-        tmem_ld16(col, *reinterpret_cast<uint32_t(*)[16]>(&ov[0]));
-        if constexpr (C::NO == 32) tmem_ld16(col + 16, *reinterpret_cast<uint32_t(*)[16]>(&ov[16]));
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int e = 0; e < C::NO; ++e) ov[e] = 0u;
-      }
-      tc_fence_before();
-      mbar_arrive(ofree + (j & 1));
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float v;
-        if constexpr (C::F8) {
-          v = __uint_as_float(ov[g]) + __uint_as_float(ov[G + g]) * 0.0625f +
-              __uint_as_float(ov[2 * G + g]) * (1.f / 256.f) +
-              __uint_as_float(ov[3 * G + g]) * (1.f / 4096.f);
-        } else if constexpr (C::I8) {
-          v = float(int(ov[g])) + float(int(ov[G + g])) * (1.f / 256.f) +
-              float(int(ov[2 * G + g])) * (1.f / 65536.f);
-        } else {
-          v = __uint_as_float(ov[g]) + __uint_as_float(ov[G + g]) + __uint_as_float(ov[2 * G + g]);
-        }
-        o[g] = o[g] * alpha_pend[g] + v * einv_pend;
+    // The group's piece cursor lives in smem: wk[pc & 1] is piece pc, and
+    // thread r == 0 advances it (with the piece's partial slot in pinfo) so
+    // that no other thread keeps cursor state in registers.
+    PieceWalk* wk = reinterpret_cast<PieceWalk*>(smem + C::OFF_WALK);
+    int* pinfo = reinterpret_cast<int*>(smem + C::OFF_WALK + 2 * sizeof(PieceWalk));   // [2][2]
+    auto publish = [&](int idx, const PieceWalk& pw) {
+      wk[idx] = pw;
+      if (!pw.done) {
+        const long long first = int64_t(Hk) * pw.P + int64_t(pw.h) * pw.nt;   // tile 0 of (b, h)
+        pinfo[idx * 2] = int(int64_t(blockIdx.x) - cta_of(first));
+        pinfo[idx * 2 + 1] = pw.hi == pw.nt;
       }
     };
+    if (r == 0) {
+      publish(0, walk);
+      PieceWalk n = walk;
+      n.next(Hk, ctx_lens, B, max_ctx, W);
+      publish(1, n);
+    }
+    named_bar_sync(1, 128);
 
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i % C::NST;
-      // ---- S of tile i
-      if (ok) ok = mbar_wait(sfull + (i & 1), (i >> 1) & 1, abort_flag, kMmaWaitLimitCycles);
-      tc_fence_after();
-      uint32_t sw[C::NS];
-      if (ok) {
-        const uint32_t col = tmem + lane_base + C::COL_S + (i & 1) * 32;
-        tmem_ld16(col, *reinterpret_cast<uint32_t(*)[16]>(&sw[0]));
-        if constexpr (C::NS == 32) tmem_ld16(col + 16, *reinterpret_cast<uint32_t(*)[16]>(&sw[16]));
-        tmem_ld_wait();
-      } else {
+    // query operand of a piece: the BF16 query rows of its group, loaded early
+    // (qv) and written as exact parts later (store_q)
+    float qv[C::HPW][D / 32];
+    auto load_q = [&](bool none, int qb, int qh) {
 #pragma unroll
-        for (int e = 0; e < C::NS; ++e) sw[e] = 0u;
+      for (int hh = 0; hh < C::HPW; ++hh) {
+        const int g = cw + 4 * hh;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i)
+          qv[hh][i] = (g < G && !none)
+                          ? __bfloat162float(q[(int64_t(qb) * Hq + qh * G + g) * D + lane + 32 * i])
+                          : 0.f;
       }
+    };
+    // B operand of S (K-major, no swizzle): row n = part * G + g, element
+    // (n, d) at (n/8)*Q_SBO + (n%8)*16 + (d*E/16)*Q_LBO + (d*E)%16
+    auto store_q = [&]() {
+#pragma unroll
+      for (int hh = 0; hh < C::HPW; ++hh) {
+        const int g = cw + 4 * hh;
+        if (g >= G) continue;                                   // uniform per warp
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) amax = fmaxf(amax, fabsf(qv[hh][i]));
+        amax = warp_max(amax);
+        // power-of-two scaling of the head: FP8 puts max|q| into [128, 256)
+        // (inside the E4M3 range), INT8 into [32, 64) (parts within +-64)
+        int e = 0;
+        if (!C::BF && amax > 0.f) e = (C::F8 ? 7 : 5) - ilogbf(amax);
+        e = max(-120, min(120, e));
+        const float up = __int_as_float((127 + e) << 23);
+        const float down = __int_as_float((127 - e) << 23);
+        int isum = 0;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) {
+          const int d = lane + 32 * i;
+          auto at = [&](int n) -> uint8_t* {
+            return qop + (n >> 3) * C::Q_SBO + (n & 7) * 16 + ((d * C::E) >> 4) * C::Q_LBO +
+                   ((d * C::E) & 15);
+          };
+          if constexpr (C::BF) {
+            *reinterpret_cast<uint16_t*>(at(g)) = __bfloat16_as_ushort(__float2bfloat16_rn(qv[hh][i]));
+          } else if constexpr (C::F8) {
+            // x = hi + lo/16 with both parts E4M3: exact for a BF16 value unless
+            // it lies below the E4M3 normal range after scaling
+            const float x = qv[hh][i] * up;
+            const uint32_t hc = f32x2_to_e4m3x2(x, 0.f) & 0xFFu;
+            float hv, unused;
+            e4m3x2_to_f32x2(hc, hv, unused);
+            const uint32_t lc = f32x2_to_e4m3x2((x - hv) * 16.f, 0.f) & 0xFFu;
+            *at(g) = uint8_t(hc);
+            *at(G + g) = uint8_t(lc);
+          } else {
+            // x = x0 + x1/128 + x2/16384, every part an integer in [-64, 64]
+            const float x = qv[hh][i] * up;
+            const float x0 = rintf(x);
+            const float r0 = (x - x0) * 128.f;
+            const float x1 = rintf(r0);
+            const float x2 = rintf((r0 - x1) * 128.f);
+            const int i0 = int(x0), i1 = int(x1), i2 = int(x2);
+            *at(g) = uint8_t(int8_t(i0));
+            *at(G + g) = uint8_t(int8_t(i1));
+            *at(2 * G + g) = uint8_t(int8_t(i2));
+            isum += i0 * 16384 + i1 * 128 + i2;
+          }
+        }
+        if constexpr (C::I8) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+        }
+        if (lane == 0) {
+          qsc[g] = qk_scale * down;
+          qsum[g] = float(isum) * (1.f / 16384.f);             // sum of q in the units of S
+        }
+      }
+      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(sfree + (i & 1));
+    };
 
-      // ---- this token's scales (both copies acquired here, not through the MMA)
-      if (ok) ok = mbar_wait(kfull + s, (i / C::NST) & 1, abort_flag, kMmaWaitLimitCycles);
-      if (ok) ok = mbar_wait(vfull + s, (i / C::NST) & 1, abort_flag, kMmaWaitLimitCycles);
-      const uint32_t mask = ok ? pmask[s] : 0u;   // pages of tile i inside the chunk with legal ids
-      const int tile0 = t0 + 128 * i;
-      const int p = r >> 4, t = r & 15;
-      const bool valid = ok && ((mask >> p) & 1u) && (tile0 + r < t1);
-      float sk = 1.f, zk = 0.f, sv = 0.f, zv = 0.f;
-      if (valid) {
-        if constexpr (C::F8) {
-          sk = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(kmeta + (s * 8 + p) * C::METAB)[t]);
-          sv = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(vmeta + (s * 8 + p) * C::METAB)[t]);
-        } else if constexpr (C::I8) {
-          const __nv_bfloat162 km = reinterpret_cast<const __nv_bfloat162*>(kmeta + (s * 8 + p) * C::METAB)[t];
-          const __nv_bfloat162 vm = reinterpret_cast<const __nv_bfloat162*>(vmeta + (s * 8 + p) * C::METAB)[t];
-          sk = __low2float(km); zk = __high2float(km);
-          sv = __low2float(vm); zv = __high2float(vm);
+    // first piece's query operand
+    load_q(wk[0].done, wk[0].b, wk[0].h);
+    store_q();
+    mbar_arrive(qready);
+
+    int gt = 0;
+    for (int pc = 0;; ++pc) {
+      const PieceWalk* cur = wk + (pc & 1);
+      const PieceWalk* nxt = wk + ((pc + 1) & 1);
+      if (cur->done) break;                              // uniform
+      const int pb = cur->b, ph_ = cur->h, lo = cur->lo, hi = cur->hi;
+      const int t1 = min(hi * 128, cur->ctx);
+      const int slot = pinfo[(pc & 1) * 2], last = pinfo[(pc & 1) * 2 + 1];
+      const bool more = !nxt->done;
+      load_q(!more, nxt->b, nxt->h);                     // next piece's query, in flight
+      named_bar_sync(1, 128);                            // all read the cursor; qsc/qsum visible
+      if (r == 0) {                                      // piece pc + 2 into this piece's entry
+        PieceWalk n = *nxt;
+        if (!n.done) n.next(Hk, ctx_lens, B, max_ctx, W);
+        publish(pc & 1, n);
+      }
+      float qs[G], qz[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) { qs[g] = qsc[g]; qz[g] = qsum[g]; }
+      float m[G], l[G], corr[G], o[G], alpha[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        m[g] = -INFINITY; l[g] = 0.f; corr[g] = 0.f; o[g] = 0.f; alpha[g] = 1.f;
+      }
+      float einv_pend = 1.f;
+
+      // o (relative to the current max) += O tile j * 2^-e_j * alpha: alpha
+      // moves tile j from the max it was weighted with to the current one
+      auto accum_o = [&](int j) {
+        if (ok) ok = mbar_wait(ofull + (j & 1), (j >> 1) & 1, abort_flag, kMmaWaitLimitCycles);
+        tc_fence_after();
+        uint32_t ov[C::NOL];
+        if (ok) {
+          tmem_load_cols<C::NOL>(tmem + lane_base + C::COL_O + (j & 1) * 32, ov);
+          tmem_ld_wait();
         } else {
-          sv = 1.f;
-        }
-      }
-      mbar_arrive(kempty + s);
-
-      // ---- scores (base 2) and the tile max of every head
-      float x[G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float sc;
-        if constexpr (C::F8) {
-          sc = __uint_as_float(sw[g]) + __uint_as_float(sw[G + g]) * 0.0625f;
-        } else if constexpr (C::I8) {
-          sc = float(int(sw[g])) + float(int(sw[G + g])) * (1.f / 128.f) +
-               float(int(sw[2 * G + g])) * (1.f / 16384.f) - zk * qz[g];
+          for (int e = 0; e < C::NOL; ++e) ov[e] = 0u;
+        }
+        tc_fence_before();
+        mbar_arrive(ofree + (j & 1));
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float v;
+          if constexpr (C::F8) {
+            v = __uint_as_float(ov[g]) + __uint_as_float(ov[G + g]) * 0.0625f +
+                __uint_as_float(ov[2 * G + g]) * (1.f / 256.f) +
+                __uint_as_float(ov[3 * G + g]) * (1.f / 4096.f);
+          } else if constexpr (C::I8) {
+            v = float(int(ov[g])) + float(int(ov[G + g])) * (1.f / 256.f) +
+                float(int(ov[2 * G + g])) * (1.f / 65536.f);
+          } else {
+            v = __uint_as_float(ov[g]) + __uint_as_float(ov[G + g]) + __uint_as_float(ov[2 * G + g]);
+          }
+          o[g] += v * (einv_pend * alpha[g]);
+        }
+      };
+
+      for (int i = lo; i < hi; ++i, ++gt) {
+        const int s = gt % C::NST;
+        // ---- S of tile gt
+        if (ok) ok = mbar_wait(sfull + (gt & 1), (gt >> 1) & 1, abort_flag, kMmaWaitLimitCycles);
+        tc_fence_after();
+        uint32_t sw[C::NSL];
+        if (ok) {
+          tmem_load_cols<C::NSL>(tmem + lane_base + C::COL_S + (gt & 1) * 32, sw);
+          tmem_ld_wait();
         } else {
-          sc = __uint_as_float(sw[g]);
+#pragma unroll
+          for (int e = 0; e < C::NSL; ++e) sw[e] = 0u;
         }
-        x[g] = valid ? sc * sk * qs[g] : -INFINITY;
-      }
-      float* rb = red + (i & 1) * 64;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float tm = warp_max_f32(x[g]);
-        if (lane == 0) rb[quarter * 16 + g] = tm;
-      }
-      {
-        const float svm = warp_max_f32(sv);
-        if (lane == 0) rb[quarter * 16 + 8] = svm;
-      }
-      named_bar_sync(1, 128);
-      float alpha[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float tmax = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
-        const float mn = fmaxf(m[g], tmax);
-        alpha[g] = (mn == -INFINITY) ? 1.f : exp2f(m[g] - mn);
-        m[g] = mn;
-      }
-      // P = p * v_scale * 2^ex with max(v_scale) * 2^ex in [128, 256): inside
-      // the E4M3 range, and below 2^8 for the 24-bit fixed point of INT8
-      const float svmax = fmaxf(fmaxf(rb[8], rb[24]), fmaxf(rb[40], rb[56]));
-      int ex = 0;
-      if (!C::BF && svmax > 0.f) ex = max(-120, min(120, 7 - ilogbf(svmax)));
-      const float escale = __int_as_float((127 + ex) << 23);
-      const float einv = __int_as_float((127 - ex) << 23);
+        tc_fence_before();
+        mbar_arrive(sfree + (gt & 1));
 
-      // ---- tokens of this tile past the chunk end or on a missing page: their
-      // V rows in smem are stale or never written; zero them so that
-      // 0 * (stale code) cannot produce a NaN (integer codes need no care)
-      if constexpr (!C::I8) {
-        if (mask != 0xFFu || tile0 + 128 > t1) {          // uniform over the CTA
-          if (r < D) {
+        // ---- this token's scales (both copies acquired here, not through the MMA)
+        if (ok) ok = mbar_wait(kfull + s, (gt / C::NST) & 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) ok = mbar_wait(vfull + s, (gt / C::NST) & 1, abort_flag, kMmaWaitLimitCycles);
+        const uint32_t mask = ok ? pmask[s] : 0u;   // pages of the tile with legal ids
+        const int tile0 = i * 128;
+        const int p = r >> 4, t = r & 15;
+        const bool valid = ok && ((mask >> p) & 1u) && (tile0 + r < t1);
+        float sk = 1.f, zk = 0.f, sv = 0.f, zv = 0.f;
+        if (valid) {
+          if constexpr (C::F8) {
+            sk = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(kmeta + (s * 8 + p) * C::METAB)[t]);
+            sv = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(vmeta + (s * 8 + p) * C::METAB)[t]);
+          } else if constexpr (C::I8) {
+            const __nv_bfloat162 km = reinterpret_cast<const __nv_bfloat162*>(kmeta + (s * 8 + p) * C::METAB)[t];
+            const __nv_bfloat162 vm = reinterpret_cast<const __nv_bfloat162*>(vmeta + (s * 8 + p) * C::METAB)[t];
+            sk = __low2float(km); zk = __high2float(km);
+            sv = __low2float(vm); zv = __high2float(vm);
+          } else {
+            sv = 1.f;
+          }
+        }
+        mbar_arrive(kempty + s);
+
+        // ---- scores (base 2) and the tile max of every head
+        float x[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float sc;
+          if constexpr (C::F8) {
+            sc = __uint_as_float(sw[g]) + __uint_as_float(sw[G + g]) * 0.0625f;
+          } else if constexpr (C::I8) {
+            sc = float(int(sw[g])) + float(int(sw[G + g])) * (1.f / 128.f) +
+                 float(int(sw[2 * G + g])) * (1.f / 16384.f) - zk * qz[g];
+          } else {
+            sc = __uint_as_float(sw[g]);
+          }
+          x[g] = valid ? sc * sk * qs[g] : -INFINITY;
+        }
+        float* rb = red + (gt & 1) * 64;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float tm = warp_max_f32(x[g]);
+          if (lane == 0) rb[quarter * 16 + g] = tm;
+        }
+        {
+          const float svm = warp_max_f32(sv);
+          if (lane == 0) rb[quarter * 16 + 8] = svm;
+        }
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float tmax = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+          const float mn = fmaxf(m[g], tmax);
+          alpha[g] = (mn == -INFINITY) ? 1.f : exp2f(m[g] - mn);
+          m[g] = mn;
+          o[g] *= alpha[g];
+        }
+        // P = p * v_scale * 2^ex with max(v_scale) * 2^ex in [128, 256): inside
+        // the E4M3 range, and below 2^8 for the 24-bit fixed point of INT8
+        const float svmax = fmaxf(fmaxf(rb[8], rb[24]), fmaxf(rb[40], rb[56]));
+        int ex = 0;
+        if (!C::BF && svmax > 0.f) ex = max(-120, min(120, 7 - ilogbf(svmax)));
+        const float escale = __int_as_float((127 + ex) << 23);
+        const float einv = __int_as_float((127 - ex) << 23);
+
+        // ---- tokens of this tile past the sequence end or on a missing page:
+        // their V rows in smem are stale or never written; zero them so that
+        // 0 * (stale code) cannot produce a NaN (integer codes need no care)
+        if constexpr (!C::I8) {
+          if (mask != 0xFFu || tile0 + 128 > t1) {          // uniform over the CTA
+            if (r < D) {
 #pragma unroll 1
-            for (int pp = 0; pp < 8; ++pp) {
-              int ntok = ((mask >> pp) & 1u) ? t1 - (tile0 + 16 * pp) : 0;
-              ntok = max(0, min(16, ntok));
-              if (ntok == 16) continue;
-              uint8_t* vpg = vring + (s * 8 + pp) * C::PAGE;
+              for (int pp = 0; pp < 8; ++pp) {
+                int ntok = ((mask >> pp) & 1u) ? t1 - (tile0 + 16 * pp) : 0;
+                ntok = max(0, min(16, ntok));
+                if (ntok == 16) continue;
+                uint8_t* vpg = vring + (s * 8 + pp) * C::PAGE;
 #pragma unroll
-              for (int u = 0; u < C::E; ++u) {                 // 16-byte chunks of row r
-                uint4* cp = reinterpret_cast<uint4*>(vpg + u * (D * 16) + r * 16);
-                uint4 w = *cp;
-                uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                for (int u = 0; u < C::E; ++u) {                 // 16-byte chunks of row r
+                  uint4* cp = reinterpret_cast<uint4*>(vpg + u * (D * 16) + r * 16);
+                  uint4 w = *cp;
+                  uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  uint32_t keep = 0;
+                  for (int e = 0; e < 4; ++e) {
+                    uint32_t keep = 0;
 #pragma unroll
-                  for (int bb = 0; bb < 4; ++bb) {
-                    const int tok = (u * 16 + e * 4 + bb) / C::E;   // token of byte bb of word e
-                    if (tok < ntok) keep |= 0xFFu << (8 * bb);
+                    for (int bb = 0; bb < 4; ++bb) {
+                      const int tok = (u * 16 + e * 4 + bb) / C::E;   // token of byte bb of word e
+                      if (tok < ntok) keep |= 0xFFu << (8 * bb);
+                    }
+                    ww[e] &= keep;
                   }
-                  ww[e] &= keep;
+                  *cp = make_uint4(ww[0], ww[1], ww[2], ww[3]);
                 }
-                *cp = make_uint4(ww[0], ww[1], ww[2], ww[3]);
               }
             }
           }
         }
-      }
 
-      // ---- weights -> P buffer (i & 1), the row of token r
-      uint8_t* pb = pop + (i & 1) * C::PBYTES + prow;
-      if constexpr (C::F8) {
-        // y = y0 + y1/16 + y2/256 + y3/4096, each part E4M3 (RNE); the
-        // residual is exact in FP32 and 16x smaller than the part before
-        float y[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
-          l[g] = l[g] * alpha[g] + pr;
-          y[g] = pr * sv * escale;
-        }
-        uint32_t words[C::NO / 4];
-#pragma unroll
-        for (int e = 0; e < C::NO / 4; ++e) words[e] = 0u;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-#pragma unroll
-          for (int g = 0; g < G; g += 2) {
-            const float a = y[g];
-            const float c = (g + 1 < G) ? y[g + 1] : 0.f;
-            const uint32_t code2 = f32x2_to_e4m3x2(a, c);
-            const int n = jj * G + g;                        // byte index in the row
-            words[n >> 2] |= code2 << (8 * (n & 3));
-            if (jj < 3) {
-              float av, cv;
-              e4m3x2_to_f32x2(code2, av, cv);
-              y[g] = (a - av) * 16.f;
-              if (g + 1 < G) y[g + 1] = (c - cv) * 16.f;
-            }
-          }
-        }
-#pragma unroll
-        for (int c16 = 0; c16 < C::NO / 16; ++c16)
-          *reinterpret_cast<uint4*>(pb + c16 * C::P_SBO) =
-              make_uint4(words[4 * c16], words[4 * c16 + 1], words[4 * c16 + 2], words[4 * c16 + 3]);
-      } else if constexpr (C::I8) {
-        // Y = rint(y * 2^16) < 2^24; its three bytes are the parts (weights
-        // 1, 1/256, 1/65536); zero_point * P is summed from the same Y
-        uint32_t yv[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
-          l[g] = l[g] * alpha[g] + pr;
-          yv[g] = __float2uint_rn(pr * sv * escale * 65536.f);
-          corr[g] = corr[g] * alpha[g] + zv * float(yv[g]) * (1.f / 65536.f) * einv;
-        }
-        uint32_t words[C::NO / 4];
-#pragma unroll
-        for (int e = 0; e < C::NO / 4; ++e) words[e] = 0u;
-#pragma unroll
-        for (int jj = 0; jj < 3; ++jj) {
+        // ---- weights -> P buffer (gt & 1), the row of token r
+        uint8_t* pbuf = pop + (gt & 1) * C::PBYTES + prow;
+        if constexpr (C::F8) {
+          // y = y0 + y1/16 + y2/256 + y3/4096, each part E4M3 (RNE); the
+          // residual is exact in FP32 and 16x smaller than the part before
+          float y[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const int n = jj * G + g;
-            words[n >> 2] |= ((yv[g] >> (16 - 8 * jj)) & 0xFFu) << (8 * (n & 3));
+            const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+            l[g] = l[g] * alpha[g] + pr;
+            y[g] = pr * sv * escale;
           }
-        }
+          uint32_t words[C::NO / 4];
 #pragma unroll
-        for (int c16 = 0; c16 < C::NO / 16; ++c16)
-          *reinterpret_cast<uint4*>(pb + c16 * C::P_SBO) =
-              make_uint4(words[4 * c16], words[4 * c16 + 1], words[4 * c16 + 2], words[4 * c16 + 3]);
-      } else {
-        // p = hi + mid + lo, each bf16: 24 significant bits
-        uint32_t words[C::NO / 2];
+          for (int e = 0; e < C::NO / 4; ++e) words[e] = 0u;
 #pragma unroll
-        for (int e = 0; e < C::NO / 2; ++e) words[e] = 0u;
+          for (int jj = 0; jj < 4; ++jj) {
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
-          l[g] = l[g] * alpha[g] + pr;
-          const __nv_bfloat16 hi = __float2bfloat16_rn(pr);
-          const float r1 = pr - __bfloat162float(hi);
-          const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-          const uint16_t parts[3] = {__bfloat16_as_ushort(hi), __bfloat16_as_ushort(mid),
-                                     __bfloat16_as_ushort(lo)};
+            for (int g = 0; g < G; g += 2) {
+              const float a = y[g];
+              const float c = (g + 1 < G) ? y[g + 1] : 0.f;
+              const uint32_t code2 = f32x2_to_e4m3x2(a, c);
+              const int n = jj * G + g;                        // byte index in the row
+              words[n >> 2] |= code2 << (8 * (n & 3));
+              if (jj < 3) {
+                float av, cv;
+                e4m3x2_to_f32x2(code2, av, cv);
+                y[g] = (a - av) * 16.f;
+                if (g + 1 < G) y[g + 1] = (c - cv) * 16.f;
+              }
+            }
+          }
+#pragma unroll
+          for (int c16 = 0; c16 < C::NO / 16; ++c16)
+            *reinterpret_cast<uint4*>(pbuf + c16 * C::P_SBO) =
+                make_uint4(words[4 * c16], words[4 * c16 + 1], words[4 * c16 + 2], words[4 * c16 + 3]);
+        } else if constexpr (C::I8) {
+          // Y = rint(y * 2^16) < 2^24; its three bytes are the parts (weights
+          // 1, 1/256, 1/65536); zero_point * P is summed from the same Y
+          uint32_t yv[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+            l[g] = l[g] * alpha[g] + pr;
+            yv[g] = __float2uint_rn(pr * sv * escale * 65536.f);
+            corr[g] = corr[g] * alpha[g] + zv * float(yv[g]) * (1.f / 65536.f) * einv;
+          }
+          uint32_t words[C::NO / 4];
+#pragma unroll
+          for (int e = 0; e < C::NO / 4; ++e) words[e] = 0u;
 #pragma unroll
           for (int jj = 0; jj < 3; ++jj) {
-            const int n = jj * G + g;
-            words[n >> 1] |= uint32_t(parts[jj]) << (16 * (n & 1));
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              const int n = jj * G + g;
+              words[n >> 2] |= ((yv[g] >> (16 - 8 * jj)) & 0xFFu) << (8 * (n & 3));
+            }
           }
+#pragma unroll
+          for (int c16 = 0; c16 < C::NO / 16; ++c16)
+            *reinterpret_cast<uint4*>(pbuf + c16 * C::P_SBO) =
+                make_uint4(words[4 * c16], words[4 * c16 + 1], words[4 * c16 + 2], words[4 * c16 + 3]);
+        } else {
+          // p = hi + mid + lo, each bf16: 24 significant bits
+          uint32_t words[C::NO / 2];
+#pragma unroll
+          for (int e = 0; e < C::NO / 2; ++e) words[e] = 0u;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+            l[g] = l[g] * alpha[g] + pr;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(pr);
+            const float r1 = pr - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+            const uint16_t parts[3] = {__bfloat16_as_ushort(hi), __bfloat16_as_ushort(mid),
+                                       __bfloat16_as_ushort(lo)};
+#pragma unroll
+            for (int jj = 0; jj < 3; ++jj) {
+              const int n = jj * G + g;
+              words[n >> 1] |= uint32_t(parts[jj]) << (16 * (n & 1));
+            }
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < C::NO / 8; ++c8)
+            *reinterpret_cast<uint4*>(pbuf + c8 * C::P_SBO) =
+                make_uint4(words[4 * c8], words[4 * c8 + 1], words[4 * c8 + 2], words[4 * c8 + 3]);
         }
-#pragma unroll
-        for (int c8 = 0; c8 < C::NO / 8; ++c8)
-          *reinterpret_cast<uint4*>(pb + c8 * C::P_SBO) =
-              make_uint4(words[4 * c8], words[4 * c8 + 1], words[4 * c8 + 2], words[4 * c8 + 3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(pready + (i & 1));
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(pready + (gt & 1));
 
-      // ---- O of the previous tile
-      if (i > 0) accum_o(i - 1);
-#pragma unroll
-      for (int g = 0; g < G; ++g) alpha_pend[g] = alpha[g];
-      einv_pend = einv;
-    }
-    if (ntiles > 0) accum_o(ntiles - 1);
-
-    // ---- chunk partial: (max, sum, unnormalised output) per query head
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float ls = warp_sum(l[g]);
-      const float cs = C::I8 ? warp_sum(corr[g]) : 0.f;
-      if (lane == 0) {
-        red2[quarter * 8 + g] = ls;
-        red2[32 + quarter * 8 + g] = cs;
+        // ---- O of the previous tile of this piece
+        if (i > lo) accum_o(gt - 1);
+        einv_pend = einv;
       }
-    }
-    named_bar_sync(1, 128);
-    if (ok && !*abort_flag) {
+
+      // ---- the next piece's query operand, so that its first S can start
+      // while this piece's last O drains
+      if (more) {
+        if (ok) ok = mbar_wait(qfree, pc & 1, abort_flag, kMmaWaitLimitCycles);
+        store_q();
+        mbar_arrive(qready);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) alpha[g] = 1.f;
+      accum_o(gt - 1);
+
+      // ---- piece partial: (max, sum, unnormalised output) per query head
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float L = red2[g] + red2[8 + g] + red2[16 + g] + red2[24 + g];
-        const float Cz = red2[32 + g] + red2[40 + g] + red2[48 + g] + red2[56 + g];
-        const int64_t row = (int64_t(b) * Hq + h * G + g) * max_splits + split;
-        if (r < D) part_o[row * D + r] = o[g] - Cz;
-        if (r == 0) {
-          part_ml[row * 2] = m[g];
-          part_ml[row * 2 + 1] = L;
+        const float ls = warp_sum(l[g]);
+        const float cs = C::I8 ? warp_sum(corr[g]) : 0.f;
+        if (lane == 0) {
+          red2[quarter * 8 + g] = ls;
+          red2[32 + quarter * 8 + g] = cs;
         }
+      }
+      named_bar_sync(1, 128);
+      if (ok && !*abort_flag) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float L = red2[g] + red2[8 + g] + red2[16 + g] + red2[24 + g];
+          const float Cz = red2[32 + g] + red2[40 + g] + red2[48 + g] + red2[56 + g];
+          const int64_t row = (int64_t(pb) * Hq + ph_ * G + g) * slots + slot;
+          if (r < D) part_o[row * D + r] = o[g] - Cz;
+          if (r == 0) {
+            part_ml[row * 2] = m[g];
+            part_ml[row * 2 + 1] = L;
+          }
+        }
+        if (r == 0 && last) part_cnt[pb * Hk + ph_] = slot + 1;
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
     const int32_t* __restrict__ ctx_lens, int Hk, int NB, int W, int max_ctx, int part,
-    int max_splits, float qk_scale, float* __restrict__ part_o, float* __restrict__ part_ml) {
+    int max_splits, float qk_scale, float* __restrict__ part_o, float* __restrict__ part_ml,
+    int slots, int32_t* __restrict__ part_cnt) {
   using C = TcCfg<D, FMT>;
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
@@ -582,13 +583,14 @@ __global__ void __launch_bounds__(192, FMT == KVQ_BF16 ? 1 : 2) decode_tc_kernel
       for (int g = 0; g < G; ++g) {
         const float L = red2[g] + red2[8 + g] + red2[16 + g] + red2[24 + g];
         const float Cz = red2[32 + g] + red2[40 + g] + red2[48 + g] + red2[56 + g];
-        const int64_t row = (int64_t(b) * Hq + h * G + g) * max_splits + split;
+        const int64_t row = (int64_t(b) * Hq + h * G + g) * slots + split;
         if (r < D) part_o[row * D + r] = o[g] - Cz;
         if (r == 0) {
           part_ml[row * 2] = m[g];
           part_ml[row * 2 + 1] = L;
         }
       }
+      if (r == 0 && split == n_splits - 1) part_cnt[b * Hk + h] = n_splits;
     }
   }
 

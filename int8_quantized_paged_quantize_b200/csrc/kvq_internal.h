@@ -23,10 +23,13 @@ int check_dims(const kvq_dims* d);
 
 // Split-K plan of one decode call.
 struct DecodePlan {
-  int32_t partition;   // tokens per split (multiple of kTileTokens)
+  int32_t partition;   // tokens per split (multiple of kTileTokens); the smallest
+                       // run of one sequence's tokens a decode CTA takes
   int32_t max_splits;  // splits of the longest sequence
-  size_t o_bytes;      // partial outputs  [B][Hq][max_splits][D] f32
-  size_t ml_bytes;     // partial (max, sum) [B][Hq][max_splits][2] f32
+  int32_t slots;       // partial slots per (sequence, query head): max_splits + 1
+  size_t o_bytes;      // partial outputs  [B][Hq][slots][D] f32
+  size_t ml_bytes;     // partial (max, sum) [B][Hq][slots][2] f32
+  size_t cnt_bytes;    // partials written per (sequence, KV head) [B][Hk] int32
   size_t total;        // workspace bytes (256-aligned pieces)
 };
 // Fills `plan`; returns KVQ_OK or KVQ_ERR_ARG.

@@ -331,7 +331,8 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
     const int32_t* __restrict__ ctx_lens, int Hk, int NB, int W, int max_ctx, int part,
-    int max_splits, float qscale, float* __restrict__ part_o, float* __restrict__ part_ml) {
+    int max_splits, float qscale, float* __restrict__ part_o, float* __restrict__ part_ml,
+    int slots, int32_t* __restrict__ part_cnt) {
   using C = SimtCfg<D, G, FMT>;
   constexpr int ELT = C::ELT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -532,10 +533,11 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
       o += red_o[w][g][d] * f;
       l += red_l[w][g] * f;
     }
-    const int64_t r = (int64_t(b) * Hq + h * G + g) * max_splits + split;
+    const int64_t r = (int64_t(b) * Hq + h * G + g) * slots + split;
     part_o[r * D + d] = o;
     if (d == 0) { part_ml[r * 2] = M; part_ml[r * 2 + 1] = l; }
   }
+  if (threadIdx.x == 0 && split == n_splits - 1) part_cnt[b * Hk + h] = n_splits;
 }
 
 // ------------------------------------------------------------------ merge
@@ -543,17 +545,19 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
 // (m_i, l_i, o_i) as m = max m_i, l = sum l_i 2^(m_i - m), o = sum o_i 2^(m_i - m) / l.
 template <int D, typename OutT>
 __global__ void __launch_bounds__(128) merge_kernel(const int32_t* __restrict__ ctx_lens, int Hq,
-                                                    int part, int max_splits, int max_ctx, int W,
+                                                    int G, int slots, int max_ctx, int W,
                                                     const float* __restrict__ part_o,
                                                     const float* __restrict__ part_ml,
+                                                    const int32_t* __restrict__ part_cnt,
                                                     OutT* __restrict__ out) {
   const int bq = blockIdx.x;                 // b * Hq + head
   const int b = bq / Hq;
   const int d = threadIdx.x;
   int ctx = ctx_lens[b];
   if (ctx < 0 || ctx > max_ctx || int64_t(ctx) > int64_t(W) * kBlockSize) ctx = 0;
-  const int n = (ctx + part - 1) / part;
-  const int64_t r0 = int64_t(bq) * max_splits;
+  // partials written for this (sequence, KV head) by the decode kernel
+  const int n = ctx > 0 ? min(slots, max(0, part_cnt[bq / G])) : 0;
+  const int64_t r0 = int64_t(bq) * slots;
   float M = -INFINITY;
   for (int s = 0; s < n; ++s) M = fmaxf(M, part_ml[(r0 + s) * 2]);
   float o = 0.f, l = 0.f;
@@ -592,12 +596,14 @@ cudaError_t decode_dispatch3(const void* q, int32_t B, const void* kc, const voi
                              cudaStream_t st) {
   float* po = static_cast<float*>(ws);
   float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
+  int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
   const int64_t grid = int64_t(B) * d.n_kv_heads * plan.max_splits;
   decode_simt_kernel<D, G, FMT><<<dim3(unsigned(grid)), 128, 0, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
       static_cast<const __nv_bfloat16*>(vs), tables, ctx, d.n_kv_heads, d.num_blocks,
-      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml);
+      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml,
+      plan.slots, pcnt);
   return cudaGetLastError();
 }
 
@@ -613,12 +619,14 @@ cudaError_t decode_tc_dispatch3(const void* q, int32_t B, const void* kc, const 
   if (e != cudaSuccess) return e;
   float* po = static_cast<float*>(ws);
   float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
+  int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
   const int64_t grid = int64_t(B) * d.n_kv_heads * plan.max_splits;
   kern<<<dim3(unsigned(grid)), 192, C::SMEM, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
       static_cast<const __nv_bfloat16*>(vs), tables, ctx, d.n_kv_heads, d.num_blocks,
-      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml);
+      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml,
+      plan.slots, pcnt);
   return cudaGetLastError();
 }
 
@@ -632,14 +640,28 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
   auto kern = decode_mma_kernel<D, G, FMT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           int(cudaSharedmemCarveoutMaxShared));
+  if (e != cudaSuccess) return e;
+  // resident CTAs per SM: shared memory bounds it (registers are capped so
+  // that two 8-bit CTAs fit); the BF16 ring takes a whole SM
+  int dev = 0, smem_sm = 0, reserved = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  if (e != cudaSuccess) return e;
+  const int per_sm = std::max(1, std::min(FMT == KVQ_BF16 ? 1 : 2, smem_sm / (C::SMEM + reserved)));
   float* po = static_cast<float*>(ws);
   float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
-  const int64_t grid = int64_t(B) * d.n_kv_heads * plan.max_splits;
+  int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
+  // one CTA per resident slot; each takes an equal share of the tile list
+  const int64_t grid = int64_t(device_sm_count()) * per_sm;
   kern<<<dim3(unsigned(grid)), 192, C::SMEM, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
-      static_cast<const __nv_bfloat16*>(vs), tables, ctx, d.n_kv_heads, d.num_blocks,
-      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml);
+      static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, d.num_blocks,
+      d.max_blocks_per_seq, max_ctx, plan.partition / kTileTokens, plan.slots, sm_scale * kLog2e,
+      po, pml, pcnt);
   return cudaGetLastError();
 }
 
@@ -732,22 +754,26 @@ int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* ou
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float* po = static_cast<const float*>(ws);
   const float* pml = reinterpret_cast<const float*>(static_cast<const char*>(ws) + plan.o_bytes);
+  const int32_t* pcnt =
+      reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + plan.o_bytes + plan.ml_bytes);
   const dim3 grid(unsigned(int64_t(B) * d.n_q_heads));
-  const int W = d.max_blocks_per_seq, Hq = d.n_q_heads;
+  const int W = d.max_blocks_per_seq, Hq = d.n_q_heads, G = d.n_q_heads / d.n_kv_heads;
   if (d.head_dim == 128) {
     if (out_f32)
-      merge_kernel<128, float><<<grid, 128, 0, st>>>(ctx, Hq, plan.partition, plan.max_splits,
-          max_ctx, W, po, pml, static_cast<float*>(out));
+      merge_kernel<128, float><<<grid, 128, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W, po, pml,
+                                                     pcnt, static_cast<float*>(out));
     else
-      merge_kernel<128, __nv_bfloat16><<<grid, 128, 0, st>>>(ctx, Hq, plan.partition,
-          plan.max_splits, max_ctx, W, po, pml, static_cast<__nv_bfloat16*>(out));
+      merge_kernel<128, __nv_bfloat16><<<grid, 128, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W,
+                                                             po, pml, pcnt,
+                                                             static_cast<__nv_bfloat16*>(out));
   } else {
     if (out_f32)
-      merge_kernel<64, float><<<grid, 64, 0, st>>>(ctx, Hq, plan.partition, plan.max_splits,
-          max_ctx, W, po, pml, static_cast<float*>(out));
+      merge_kernel<64, float><<<grid, 64, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W, po, pml,
+                                                   pcnt, static_cast<float*>(out));
     else
-      merge_kernel<64, __nv_bfloat16><<<grid, 64, 0, st>>>(ctx, Hq, plan.partition,
-          plan.max_splits, max_ctx, W, po, pml, static_cast<__nv_bfloat16*>(out));
+      merge_kernel<64, __nv_bfloat16><<<grid, 64, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W, po,
+                                                           pml, pcnt,
+                                                           static_cast<__nv_bfloat16*>(out));
   }
   return int(cudaGetLastError());
 }
