@@ -17,8 +17,11 @@
 // 6 warps per CTA:
 //   warp 0      producer: lanes 0..7 each own one page of a 128-token tile and
 //               issue its 1-D bulk copy (K page, then V page) into a ring of
-//               smem stages; lanes 8..15 copy the pages' scales. The block ids
-//               of the next tile are loaded while the current one is issued.
+//               smem stages through the TMA engine. The pages' scales are
+//               loaded by every lane one tile ahead and stored into the stage
+//               before its arrive (as copies they would double the TMA
+//               requests, whose issue rate bounds the 8-bit tile). Block ids
+//               are loaded two tiles ahead.
 //   warp 1      allocates TMEM; one thread issues the MMAs.
 //   warps 2..5  softmax warps, one per TMEM lane quarter; thread r owns token r
 //               of the tile for S and P, channel r for O. They also build the
@@ -319,6 +322,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     // ---------------------------------------------------------- producer
     const uint64_t pol = l2_evict_first_policy();
     const int p8 = lane & 7;
+    constexpr int CPP = C::METAB / 16;                    // 16-byte scale chunks per page
     // block id of page p8 of tile `tile` of the current piece of `pw`
     auto load_id = [&](const PieceWalk& pw, int tile) -> int {
       if (lane >= 8 || pw.done) return -2;
@@ -327,60 +331,82 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       const int npg = min(8, (t1 - tok0 + kBlockSize - 1) / kBlockSize);
       return p8 < npg ? tables[int64_t(pw.b) * W + tok0 / kBlockSize + p8] : -2;   // -2: no page here
     };
-    PieceWalk nx = walk;                 // cursor of the next tile
-    int ntile = nx.lo;
-    int id_next = load_id(nx, ntile);
+    auto step = [&](PieceWalk& pw, int& tile) {
+      if (pw.done) return;
+      if (++tile >= pw.hi) {
+        pw.next(Hk, ctx_lens, B, max_ctx, W);
+        tile = pw.lo;
+      }
+    };
+    // this lane's 16-byte chunk of the K and V scales of a tile (lane = page *
+    // CPP + chunk), loaded one tile before it is stored into the stage
+    const int sp = lane / (CPP > 0 ? CPP : 1), sc = lane % (CPP > 0 ? CPP : 1);
+    auto load_scales = [&](int ids, int h, uint4& kv, uint4& vv) {
+      kv = vv = make_uint4(0, 0, 0, 0);
+      if constexpr (C::MV > 0) {
+        const int sblk = __shfl_sync(0xffffffffu, ids, sp & 7);
+        if (sp < 8 && sblk >= 0 && sblk < NB) {
+          const int64_t off = (int64_t(sblk) * Hk + h) * C::METAB + sc * 16;
+          kv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(ks) + off));
+          vv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vs) + off));
+        }
+      }
+    };
+    // cursors of tiles gt, gt + 1, gt + 2; block ids are loaded two tiles ahead
+    PieceWalk c0 = walk, c1 = walk, c2 = walk;
+    int i0 = walk.lo, i1 = walk.lo, i2 = walk.lo;
+    step(c1, i1);
+    step(c2, i2);
+    step(c2, i2);
+    int id0 = load_id(c0, i0), id1 = load_id(c1, i1);
+    uint4 ksc, vsc;
+    load_scales(id0, c0.h, ksc, vsc);
     bool kiss[C::NST], viss[C::NST];
     uint32_t kpar[C::NST], vpar[C::NST];
 #pragma unroll
     for (int s = 0; s < C::NST; ++s) { kiss[s] = viss[s] = false; kpar[s] = vpar[s] = 0; }
-    for (int gt = 0; !nx.done; ++gt) {
+    for (int gt = 0; !c0.done; ++gt) {
       const int s = gt % C::NST;
       const uint32_t ph = (gt / C::NST) & 1;
-      const int h = nx.h;
-      const int id = id_next;
-      if (++ntile >= nx.hi) {
-        nx.next(Hk, ctx_lens, B, max_ctx, W);
-        ntile = nx.lo;
-      }
-      id_next = load_id(nx, ntile);
+      const int h = c0.h;
+      const int id = id0;
+      const int id2 = load_id(c2, i2);
+      uint4 ksc_n, vsc_n;
+      load_scales(c1.done ? -2 : id1, c1.h, ksc_n, vsc_n);   // next tile's scales, in flight
       if (lane < 8 && id != -2 && (id < 0 || id >= NB)) flag_error(KVQ_DEVERR_BLOCK);
       const bool valid = lane < 8 && id >= 0 && id < NB;
       const uint32_t mask = __ballot_sync(0xffffffffu, valid) & 0xFFu;
       const int blk = __shfl_sync(0xffffffffu, id, p8);
       const bool mine = ((mask >> p8) & 1u) != 0u;
+      const bool smine = C::MV > 0 && sp < 8 && ((mask >> sp) & 1u) != 0u;
       const int64_t page = int64_t(blk) * Hk + h;
-      const uint32_t bytes = uint32_t(__popc(mask)) * uint32_t(C::PAGE + C::METAB);
+      const uint32_t bytes = uint32_t(__popc(mask)) * uint32_t(C::PAGE);
       bool ok = true;
-      if (lane == 0) {
-        ok = mbar_wait(kempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
-        if (ok) {
-          pmask[s] = mask;                       // published by the arrive below
-          mbar_arrive_expect_tx(kfull + s, bytes);
-        }
-      }
+      if (lane == 0) ok = mbar_wait(kempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
       if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
-      if (lane < 8 && mine) bulk_g2s(kring + (s * 8 + p8) * C::PAGE, kc + page * C::PAGE, C::PAGE, kfull + s, pol);
-      if constexpr (C::MV > 0) {
-        if (lane >= 8 && lane < 16 && mine)
-          bulk_g2s(kmeta + (s * 8 + p8) * C::METAB, reinterpret_cast<const uint8_t*>(ks) + page * C::METAB,
-                   C::METAB, kfull + s, pol);
+      if (smine) *reinterpret_cast<uint4*>(kmeta + (s * 8 + sp) * C::METAB + sc * 16) = ksc;
+      __syncwarp();                            // the scales, then the arrive that publishes them
+      if (lane == 0) {
+        pmask[s] = mask;
+        mbar_arrive_expect_tx(kfull + s, bytes);
       }
+      __syncwarp();
+      if (lane < 8 && mine) bulk_g2s(kring + (s * 8 + p8) * C::PAGE, kc + page * C::PAGE, C::PAGE, kfull + s, pol);
       kiss[s] = true;
       kpar[s] = ph;
-      if (lane == 0) {
-        ok = mbar_wait(vempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
-        if (ok) mbar_arrive_expect_tx(vfull + s, bytes);
-      }
+      if (lane == 0) ok = mbar_wait(vempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
       if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
+      if (smine) *reinterpret_cast<uint4*>(vmeta + (s * 8 + sp) * C::METAB + sc * 16) = vsc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(vfull + s, bytes);
+      __syncwarp();
       if (lane < 8 && mine) bulk_g2s(vring + (s * 8 + p8) * C::PAGE, vc + page * C::PAGE, C::PAGE, vfull + s, pol);
-      if constexpr (C::MV > 0) {
-        if (lane >= 8 && lane < 16 && mine)
-          bulk_g2s(vmeta + (s * 8 + p8) * C::METAB, reinterpret_cast<const uint8_t*>(vs) + page * C::METAB,
-                   C::METAB, vfull + s, pol);
-      }
       viss[s] = true;
       vpar[s] = ph;
+      // shift the cursors
+      c0 = c1; i0 = i1; id0 = id1; ksc = ksc_n; vsc = vsc_n;
+      c1 = c2; i1 = i2; id1 = id2;
+      step(c2, i2);
     }
     if (lane == 0 && *abort_flag) {
       // let the copies already issued land before the CTA's smem goes away
