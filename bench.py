@@ -89,10 +89,15 @@ class ClockSampler:
             self.path = tempfile.mktemp(suffix=".csv")
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.id}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "10"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # the timed region is short: wait until the sampler is producing lines
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
 
     def stop(self):
         if not self.proc:
@@ -123,6 +128,27 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def measured_traffic(workload, fmt):
+    """DRAM bytes per decode launch from the committed ncu capture of this
+    workload, or None when there is none or the kernel sources changed since."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    csrc = os.path.join(ROOT, "int8_quantized_paged_quantize_b200", "csrc")
+    for name, sha in rec.get("kernel_sha256", {}).items():
+        path = os.path.join(csrc, name)
+        if not os.path.exists(path):
+            return None
+        with open(path, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != sha:
+                return None
+    v = rec.get("bytes_per_launch", {}).get(f"{workload}/{fmt}")
+    return float(v) if v is not None else None
 
 
 # ----------------------------------------------------------------------------- distributed
@@ -522,7 +548,8 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "decode partial (kvq_decode_partial)",
                      "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
-                     "alg_bytes_per_launch": alg_step, "traffic": None},
+                     "alg_bytes_per_launch": alg_step,
+                     "traffic": measured_traffic(w.name, fmt)},
         "e2e": {"value": e2e_val, "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": t["launches"],
