@@ -503,6 +503,7 @@ def main():
     e2e_val = kv_total / (e2e_ms * 1e-3) / 1e9
 
     formats = {}
+    outs = {}
     if not args.no_formats:
         for f in ("fp8", "int8", "bf16"):
             if f == fmt:
@@ -528,7 +529,21 @@ def main():
                 "ms": {k: round(v, 5) for k, v in tf.items() if k != "launches"},
                 "kv_bytes_per_step": kvf,
             }
+            # step 0's attention again, in FP32: every format holds the same tokens
+            # up to that context, so the outputs compare directly
+            outs[f] = stf.cache.decode(stf.q[0], stf.tables, stf.ctx[0], stf.max_ctx,
+                                       sm_scale=wb.sm_scale, workspace=stf.ws,
+                                       out_dtype=torch.float32).cpu()
             st = stf
+        # quality number (reported, not a pass criterion): the quantized cache's
+        # attention output against the same kernel on the unquantized BF16 cache
+        for f in ("fp8", "int8"):
+            dev = (outs[f] - outs["bf16"]).abs()
+            ref = outs["bf16"].abs()
+            formats[f]["quality_vs_bf16_cache"] = {
+                "max_abs": float(dev.max()), "mean_abs": float(dev.mean()),
+                "rel_l2": float((outs[f] - outs["bf16"]).norm() / max(float(outs["bf16"].norm()), 1e-30)),
+                "mean_abs_ref": float(ref.mean()), "step": 0}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
