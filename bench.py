@@ -413,8 +413,11 @@ def run_reference(args):
     fmt = args.fmt or w.fmt
     vals = []
     t0 = time.perf_counter()
+    # each step samples the workload for a bounded time so that the whole run
+    # stays near two minutes whatever --steps / --warmup are
+    budget = min(args.ref_budget, 120.0 / max(1, args.warmup + args.steps))
     for s in range(args.warmup + args.steps):
-        gbs, tok_s, desc, threads = oracle_decode_sample(w, fmt, seed=0, budget_s=args.ref_budget)
+        gbs, tok_s, desc, threads = oracle_decode_sample(w, fmt, seed=0, budget_s=budget)
         if s >= args.warmup:
             vals.append(gbs)
     value = float(np.mean(vals))
