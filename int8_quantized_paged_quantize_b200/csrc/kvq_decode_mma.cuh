@@ -5,13 +5,14 @@
 // to the small S and P tiles instead. Included by kvq_kernels.cu.
 //
 // Work split (persistent, stream-K): the work list is every (sequence b, KV
-// head h, 128-token tile) in order of b, then h, then tile. Each of the N
-// resident CTAs takes one contiguous, equal share of it (N is cut so that a
-// share holds at least `unit_tiles` tiles). A share is a few "pieces", a piece
-// being the share's run of tiles of one (b, h); each piece ends in an
-// online-softmax partial (max, sum, unnormalised output) in a workspace slot,
-// and the piece holding the last tile of (b, h) records how many slots the
-// merge kernel must combine. The ring of K/V stages streams across piece
+// head h, 128-token tile) in order of b, then h, then tile, each (b, h) run
+// also costing kPieceCost units for opening and closing its piece. Each of
+// the N resident CTAs takes one contiguous, equal share of the total cost (N
+// is cut so that a share holds at least `unit_tiles` units). A share is a few
+// "pieces", a piece being the share's tiles of one (b, h); each piece ends in
+// an online-softmax partial (max, sum, unnormalised output) in a workspace
+// slot, and the piece holding the last tile of (b, h) records how many slots
+// the merge kernel must combine. The ring of K/V stages streams across piece
 // boundaries, so a CTA fills its pipeline once.
 //
 // 6 warps per CTA:
@@ -95,13 +96,14 @@ struct MmaCfg {
   static constexpr int OFF_P = OFF_Q + QBYTES;                                  // [2]
   static constexpr int OFF_BAR = OFF_P + 2 * PBYTES;
   static constexpr int NBAR = 4 * NST + 12 + 1;
-  static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;           // float [2][4][16]; prologue scratch
+  static constexpr int OFF_RED = (OFF_BAR + 8 * NBAR + 15) / 16 * 16;   // float [2][64]; prologue scratch
   static constexpr int OFF_RED2 = OFF_RED + 2 * 4 * 16 * 4;    // float [2][4][8]: sums, zero-point terms
   static constexpr int OFF_QSC = OFF_RED2 + 2 * 4 * 8 * 4;     // float [8] scale, [8] sum(q)
   static constexpr int OFF_PMASK = OFF_QSC + 16 * 4;           // uint32 [NST] valid-page masks
   static constexpr int OFF_MISC = (OFF_PMASK + 4 * NST + 15) / 16 * 16;   // tmem base, abort flag, start (b, P)
   static constexpr int OFF_WALK = OFF_MISC + 32;               // softmax piece cursor [2] + slots [2][2]
   static constexpr int SMEM = OFF_WALK + 160 + 128;            // + alignment slack
+  static_assert(OFF_RED % 16 == 0 && OFF_BAR % 8 == 0 && OFF_MISC % 16 == 0, "smem alignment");
 };
 
 // Context length of sequence b if it is legal, else 0.
@@ -110,19 +112,58 @@ __device__ __forceinline__ int mma_seq_ctx(const int32_t* ctx_lens, int b, int m
   return (c < 0 || c > max_ctx || int64_t(c) > int64_t(W) * kBlockSize) ? 0 : c;
 }
 
-// Cursor over the pieces of one CTA's share [g, end) of the work list. Every
-// role walks it the same way; the next sequence's length is loaded one
-// sequence ahead so that stepping over a sequence boundary does not wait.
+// Work-list cost of one (sequence, KV head) run: its tiles plus kPieceCost
+// virtual units in front of them, about what opening and closing a piece
+// costs in tile times, so that equal shares of cost take equal time.
+constexpr int kPieceCost = 1;
+
+// Cursor over the pieces of one CTA's share [g, end) of the work list (cost
+// units). Every role walks it the same way; the next sequence's length is
+// loaded one sequence ahead so that stepping over a sequence boundary does not
+// wait. A share that holds only a run's virtual units yields no piece there.
 struct PieceWalk {
   int b, h, lo, hi;          // sequence, KV head, tiles [lo, hi) of that sequence
   int nt, ctx;               // tiles and tokens of sequence b
   int ctx_next;              // length of sequence b + 1 (0 past the batch)
-  long long P;               // tiles of sequences 0 .. b-1
-  long long g, end;          // work-list index of tile lo; end of the share
+  long long P;               // cost per head of sequences 0 .. b-1
+  long long g, gend, end;    // cost positions: this piece's start and end; end of the share
   bool done;
 
   __device__ __forceinline__ void load_next(const int32_t* ctx_lens, int B, int max_ctx, int W) {
     ctx_next = (b + 1 < B) ? mma_seq_ctx(ctx_lens, b + 1, max_ctx, W) : 0;
+  }
+  __device__ __forceinline__ void next_run(int Hk, const int32_t* ctx_lens, int B, int max_ctx,
+                                           int W) {
+    if (++h < Hk) return;
+    h = 0;
+    P += nt + kPieceCost;
+    ++b;
+    ctx = ctx_next;
+    nt = (ctx + 127) / 128;
+    load_next(ctx_lens, B, max_ctx, W);
+    while (nt == 0) {                            // empty sequences hold no tiles
+      ++b;
+      ctx = ctx_next;
+      nt = (ctx + 127) / 128;
+      load_next(ctx_lens, B, max_ctx, W);
+    }
+  }
+  // the piece starting at cost position g, or the next non-empty one
+  __device__ __forceinline__ void settle(int Hk, const int32_t* ctx_lens, int B, int max_ctx,
+                                         int W) {
+    while (true) {
+      if (g >= end) { done = true; return; }
+      const long long L = nt + kPieceCost;
+      const long long u = g - (int64_t(Hk) * P + int64_t(h) * L);   // offset in the run
+      const long long uend = ll_min(L, u + (end - g));
+      lo = int(ll_max(0, u - kPieceCost));
+      hi = int(ll_max(0, uend - kPieceCost));
+      gend = g + (uend - u);
+      if (hi > lo) { done = false; return; }
+      g = gend;
+      if (g >= end) { done = true; return; }
+      next_run(Hk, ctx_lens, B, max_ctx, W);
+    }
   }
   __device__ __forceinline__ void init(int b0, long long P0, long long start, long long end_,
                                        int Hk, const int32_t* ctx_lens, int B, int max_ctx, int W) {
@@ -130,31 +171,21 @@ struct PieceWalk {
     ctx = mma_seq_ctx(ctx_lens, b, max_ctx, W);
     nt = (ctx + 127) / 128;
     load_next(ctx_lens, B, max_ctx, W);
-    done = g >= end || nt == 0;
-    const long long off = g - int64_t(Hk) * P;
-    h = done ? 0 : int(off / nt);
-    lo = done ? 0 : int(off % nt);
-    hi = done ? 0 : int(ll_min(nt, lo + (end - g)));
+    lo = hi = 0;
+    gend = g;
+    if (g >= end || nt == 0) { done = true; h = 0; return; }
+    h = int((g - int64_t(Hk) * P) / (nt + kPieceCost));
+    settle(Hk, ctx_lens, B, max_ctx, W);
   }
   __device__ __forceinline__ void next(int Hk, const int32_t* ctx_lens, int B, int max_ctx, int W) {
-    g += hi - lo;
+    g = gend;
     if (g >= end) { done = true; return; }
-    if (++h == Hk) {
-      h = 0;
-      P += nt;
-      ++b;
-      ctx = ctx_next;
-      nt = (ctx + 127) / 128;
-      load_next(ctx_lens, B, max_ctx, W);
-      while (nt == 0) {                          // empty sequences hold no tiles
-        ++b;
-        ctx = ctx_next;
-        nt = (ctx + 127) / 128;
-        load_next(ctx_lens, B, max_ctx, W);
-      }
-    }
-    lo = 0;
-    hi = int(ll_min(nt, end - g));
+    next_run(Hk, ctx_lens, B, max_ctx, W);
+    settle(Hk, ctx_lens, B, max_ctx, W);
+  }
+  // cost position of tile 0 of run (b, h)
+  __device__ __forceinline__ long long first_tile(int Hk) const {
+    return int64_t(Hk) * P + int64_t(h) * (nt + kPieceCost) + kPieceCost;
   }
 };
 
@@ -185,7 +216,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   const int Hq = Hk * G;
 
   // ------------------------------------------------------------ the share
-  // T = total tiles; each thread sums the tiles of some sequences
+  // T = total work-list cost; each thread sums the run costs of some sequences
   long long* red64 = reinterpret_cast<long long*>(smem + C::OFF_RED);   // [6] + 2
   long long* miscll = reinterpret_cast<long long*>(smem + C::OFF_MISC + 16);
   int* misci = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -195,8 +226,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       const int c = ctx_lens[bb];
       if (c < 0 || c > max_ctx || int64_t(c) > int64_t(W) * kBlockSize) {
         if (blockIdx.x == 0) flag_error(KVQ_DEVERR_CONTEXT);
-      } else {
-        tsum += (c + 127) / 128;
+      } else if (c > 0) {
+        tsum += (c + 127) / 128 + kPieceCost;
       }
     }
 #pragma unroll
@@ -212,14 +243,15 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   if (T == 0 || blockIdx.x >= N) return;                 // uniform for the CTA
   const long long start = (int64_t(blockIdx.x) * T) / N;
   const long long end = (int64_t(blockIdx.x + 1) * T) / N;
-  // the sequence holding tile `start`: block-wide scan of tiles per sequence
+  // the sequence holding cost position `start`: block-wide scan of run costs
   {
     if (threadIdx.x == 0) misci[0] = -1;
     __syncthreads();
     long long run = 0;
     for (int base = 0; base < B; base += blockDim.x) {
       const int bb = base + threadIdx.x;
-      const int tb = bb < B ? (mma_seq_ctx(ctx_lens, bb, max_ctx, W) + 127) / 128 : 0;
+      int tb = bb < B ? (mma_seq_ctx(ctx_lens, bb, max_ctx, W) + 127) / 128 : 0;
+      if (tb > 0) tb += kPieceCost;                           // run cost of sequence bb
       long long incl = tb;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -235,7 +267,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
         before += (w < warp) ? red64[w] : 0;
         total += red64[w];
       }
-      const long long lo_t = run + before + incl - tb;          // tiles before sequence bb
+      const long long lo_t = run + before + incl - tb;          // run cost before sequence bb
       if (bb < B && tb > 0 && int64_t(Hk) * lo_t <= start && start < int64_t(Hk) * (lo_t + tb)) {
         misci[0] = bb;
         miscll[0] = lo_t;
@@ -247,8 +279,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   }
   const int b0 = misci[0];
   const long long P0 = miscll[0];
-  // CTA that holds work-list tile x; the slot of a piece is its CTA's rank
-  // among the CTAs that share the piece's (b, h)
+  // CTA that holds work-list cost position x; the slot of a piece is its CTA's
+  // rank among the CTAs that hold real tiles of the piece's (b, h)
   auto cta_of = [&](long long x) -> long long { return ((x + 1) * N - 1) / T; };
 
   uint8_t* kring = smem + C::OFF_K;
@@ -382,27 +414,33 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       const int64_t page = int64_t(blk) * Hk + h;
       const uint32_t bytes = uint32_t(__popc(mask)) * uint32_t(C::PAGE);
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(kempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
-      if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
-      if (smine) *reinterpret_cast<uint4*>(kmeta + (s * 8 + sp) * C::METAB + sc * 16) = ksc;
-      __syncwarp();                            // the scales, then the arrive that publishes them
+      // per stage: byte count, the page copies, then the scale stores and the
+      // one arrival that publishes them (the copies need not wait for the scales)
       if (lane == 0) {
-        pmask[s] = mask;
-        mbar_arrive_expect_tx(kfull + s, bytes);
+        ok = mbar_wait(kempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) mbar_expect_tx(kfull + s, bytes);
       }
-      __syncwarp();
+      if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
       if (lane < 8 && mine) bulk_g2s(kring + (s * 8 + p8) * C::PAGE, kc + page * C::PAGE, C::PAGE, kfull + s, pol);
       kiss[s] = true;
       kpar[s] = ph;
-      if (lane == 0) ok = mbar_wait(vempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
+      if (smine) *reinterpret_cast<uint4*>(kmeta + (s * 8 + sp) * C::METAB + sc * 16) = ksc;
+      __syncwarp();
+      if (lane == 0) {
+        pmask[s] = mask;
+        mbar_arrive(kfull + s);
+      }
+      if (lane == 0) {
+        ok = mbar_wait(vempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) mbar_expect_tx(vfull + s, bytes);
+      }
       if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
-      if (smine) *reinterpret_cast<uint4*>(vmeta + (s * 8 + sp) * C::METAB + sc * 16) = vsc;
-      __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(vfull + s, bytes);
-      __syncwarp();
       if (lane < 8 && mine) bulk_g2s(vring + (s * 8 + p8) * C::PAGE, vc + page * C::PAGE, C::PAGE, vfull + s, pol);
       viss[s] = true;
       vpar[s] = ph;
+      if (smine) *reinterpret_cast<uint4*>(vmeta + (s * 8 + sp) * C::METAB + sc * 16) = vsc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(vfull + s);
       // shift the cursors
       c0 = c1; i0 = i1; id0 = id1; ksc = ksc_n; vsc = vsc_n;
       c1 = c2; i1 = i2; id1 = id2;
@@ -447,9 +485,12 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
         return true;
       };
       for (int pc = 0; ok && !walk.done; ++pc) {
+        // the last tile of the piece before: its PV goes first, so that the
+        // softmax warps can drain it while they build this piece's query
+        if (gt >= 1) ok = issue_pv(gt - 1);
         // the query operand of piece pc (one buffer: the softmax warps rewrite
         // it only after every S product of the piece before has been read)
-        ok = mbar_wait(qready, pc & 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) ok = mbar_wait(qready, pc & 1, abort_flag, kMmaWaitLimitCycles);
         tc_fence_after();
         const uint32_t qa = qaddr;
         for (int i = walk.lo; ok && i < walk.hi; ++i, ++gt) {
@@ -465,7 +506,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
                             sdesc_plain(a0 + kk * 2 * C::K_LBO, C::K_LBO, C::K_SBO),
                             sdesc_plain(qa + kk * 2 * C::Q_LBO, C::Q_LBO, C::Q_SBO), id_s, kk > 0);
           mma_commit(sfull + (gt & 1));
-          if (gt >= 1) ok = issue_pv(gt - 1);
+          if (i > walk.lo) ok = issue_pv(gt - 1);
         }
         if (ok) mma_commit(qfree);                         // this piece's S products are issued
         walk.next(Hk, ctx_lens, B, max_ctx, W);
@@ -494,8 +535,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     auto publish = [&](int idx, const PieceWalk& pw) {
       wk[idx] = pw;
       if (!pw.done) {
-        const long long first = int64_t(Hk) * pw.P + int64_t(pw.h) * pw.nt;   // tile 0 of (b, h)
-        pinfo[idx * 2] = int(int64_t(blockIdx.x) - cta_of(first));
+        pinfo[idx * 2] = int(int64_t(blockIdx.x) - cta_of(pw.first_tile(Hk)));
         pinfo[idx * 2 + 1] = pw.hi == pw.nt;
       }
     };
@@ -703,20 +743,22 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           }
           x[g] = valid ? sc * sk * qs[g] : -INFINITY;
         }
+        // per-head tile maxima of the four warps, head-major: rb[g][quarter]
         float* rb = red + (gt & 1) * 64;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float tm = warp_max_f32(x[g]);
-          if (lane == 0) rb[quarter * 16 + g] = tm;
+          if (lane == 0) rb[g * 4 + quarter] = tm;
         }
         {
           const float svm = warp_max_f32(sv);
-          if (lane == 0) rb[quarter * 16 + 8] = svm;
+          if (lane == 0) rb[8 * 4 + quarter] = svm;
         }
         named_bar_sync(1, 128);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float tmax = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+          const float4 t4 = *reinterpret_cast<const float4*>(rb + g * 4);
+          const float tmax = fmaxf(fmaxf(t4.x, t4.y), fmaxf(t4.z, t4.w));
           const float mn = fmaxf(m[g], tmax);
           alpha[g] = (mn == -INFINITY) ? 1.f : exp2f(m[g] - mn);
           m[g] = mn;
@@ -724,7 +766,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
         }
         // P = p * v_scale * 2^ex with max(v_scale) * 2^ex in [128, 256): inside
         // the E4M3 range, and below 2^8 for the 24-bit fixed point of INT8
-        const float svmax = fmaxf(fmaxf(rb[8], rb[24]), fmaxf(rb[40], rb[56]));
+        const float4 s4 = *reinterpret_cast<const float4*>(rb + 8 * 4);
+        const float svmax = fmaxf(fmaxf(s4.x, s4.y), fmaxf(s4.z, s4.w));
         int ex = 0;
         if (!C::BF && svmax > 0.f) ex = max(-120, min(120, 7 - ilogbf(svmax)));
         const float escale = __int_as_float((127 + ex) << 23);
@@ -814,12 +857,26 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           uint32_t words[C::NO / 4];
 #pragma unroll
           for (int e = 0; e < C::NO / 4; ++e) words[e] = 0u;
+          if constexpr (G % 4 == 0) {
+            // byte b = 2 - jj of four heads' Y into one word: three byte permutes
 #pragma unroll
-          for (int jj = 0; jj < 3; ++jj) {
+            for (int jj = 0; jj < 3; ++jj) {
+              const uint32_t sel = uint32_t(2 - jj) | (uint32_t(6 - jj) << 4);
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-              const int n = jj * G + g;
-              words[n >> 2] |= ((yv[g] >> (16 - 8 * jj)) & 0xFFu) << (8 * (n & 3));
+              for (int g = 0; g < G; g += 4) {
+                const uint32_t lo = __byte_perm(yv[g], yv[g + 1], sel);
+                const uint32_t hi = __byte_perm(yv[g + 2], yv[g + 3], sel);
+                words[(jj * G + g) >> 2] = __byte_perm(lo, hi, 0x5410);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 3; ++jj) {
+#pragma unroll
+              for (int g = 0; g < G; ++g) {
+                const int n = jj * G + g;
+                words[n >> 2] |= ((yv[g] >> (16 - 8 * jj)) & 0xFFu) << (8 * (n & 3));
+              }
             }
           }
 #pragma unroll

@@ -113,16 +113,20 @@ struct RowCodes {
   int zp;
 };
 
-template <int D, int FMT>
-__device__ __forceinline__ void quantize_row(const __nv_bfloat16* src, RowCodes<D, FMT>& rc) {
-  constexpr int E = D / 32;
-  uint32_t raw[E / 2];
-  if constexpr (E == 4) {
+// This lane's D/32 BF16 values of a row, as packed pairs.
+template <int D>
+__device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint32_t (&raw)[D / 64]) {
+  if constexpr (D / 64 == 2) {
     const uint2 u = *reinterpret_cast<const uint2*>(src);
     raw[0] = u.x; raw[1] = u.y;
   } else {
     raw[0] = *reinterpret_cast<const uint32_t*>(src);
   }
+}
+
+template <int D, int FMT>
+__device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowCodes<D, FMT>& rc) {
+  constexpr int E = D / 32;
   rc.zp = 0;
   rc.s = __float2bfloat16_rn(0.f);
   if constexpr (FMT == KVQ_BF16) {
@@ -206,7 +210,21 @@ __global__ void __launch_bounds__(256) append_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d0 = lane * E;
-  for (int rr = warp; rr < 2 * kBlockSize; rr += 8) {
+  // the warp's rows (row rr = 2 * token + {K, V}), loaded up front so that
+  // their latencies overlap
+  constexpr int RPW = 2 * kBlockSize / 8;
+  uint32_t raws[RPW][D / 64];
+#pragma unroll
+  for (int j = 0; j < RPW; ++j) {
+    const int rr = warp + 8 * j, i = rr >> 1, which = rr & 1;
+#pragma unroll
+    for (int e = 0; e < D / 64; ++e) raws[j][e] = 0u;
+    if (i < n && sl[i] >= 0 && sl[i] < int64_t(NB) * kBlockSize)
+      load_row<D>((which ? v : k) + ((tb + i) * Hk + h) * D + d0, raws[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < RPW; ++j) {
+    const int rr = warp + 8 * j;
     const int i = rr >> 1, which = rr & 1;          // token in the group, K or V
     if (i >= n) continue;
     const int64_t slot = sl[i];
@@ -216,7 +234,7 @@ __global__ void __launch_bounds__(256) append_kernel(
       continue;
     }
     RC rc;
-    quantize_row<D, FMT>((which ? v : k) + ((tb + i) * Hk + h) * D + d0, rc);
+    quantize_row<D, FMT>(raws[j], rc);
     if (fast) {
       uint8_t* dst = (which ? vbuf : kbuf) + i * PADB + d0 * ELT;
       if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);

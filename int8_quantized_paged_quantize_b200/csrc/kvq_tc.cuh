@@ -27,6 +27,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes) : "memory");
 }
+// Raise the transaction count of the current phase (no arrival).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes) : "memory");
+}
 // Test the phase; if it is not complete the thread is suspended in hardware
 // until it completes or about `suspend_ns` pass (no issue slots are spent).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
