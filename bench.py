@@ -297,24 +297,42 @@ def timed_loop(st, steps, warmup, world, flush):
 
 def e2e_loop(st, steps, warmup, world, flush):
     """The same step through the public API with host inputs: per step the
-    step's inputs are copied from pinned host memory (q, k, v, slots, context
-    lengths, the block tables) and the output is read back, inside the timing."""
+    step's inputs (q, k, v, slots, context lengths, the block tables) are copied
+    from pinned host memory and the output is read back, inside the timing. The
+    inputs of a step are packed into one pinned buffer (each at a 256-byte
+    aligned offset) and cross in one copy; the kernels take views into it."""
     w = st.w
+
+    def layout(tensors):
+        offs, o = [], 0
+        for t in tensors:
+            offs.append(o)
+            o += (t.numel() * t.element_size() + 255) // 256 * 256
+        return offs, o
+
+    def step_tensors(s):
+        return [st.q[s], st.k[s], st.v[s], st.slots[s], st.ctx[s], st.tables]
+
+    offs, nbytes = layout(step_tensors(0))
     host = []
     for s in range(st.steps):
-        host.append([t.cpu().pin_memory() for t in (st.q[s], st.k[s], st.v[s], st.slots[s], st.ctx[s])])
-    tables_h = st.tables.cpu().pin_memory()
+        hb = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+        for t, o in zip(step_tensors(s), offs):
+            n = t.numel() * t.element_size()
+            hb[o:o + n].copy_(t.contiguous().view(-1).view(torch.uint8).cpu())
+        host.append(hb)
+    dbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    views = []
+    for t, o in zip(step_tensors(0), offs):
+        n = t.numel() * t.element_size()
+        views.append(dbuf[o:o + n].view(t.dtype).view(t.shape))
     out_h = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-    dq = [torch.empty_like(t) for t in (st.q[0], st.k[0], st.v[0], st.slots[0], st.ctx[0])]
-    tables_d = torch.empty_like(st.tables)
-    h2d = sum(t.numel() * t.element_size() for t in host[0]) + tables_h.numel() * 4
+    h2d = nbytes
     d2h = out_h.numel() * out_h.element_size()
 
     def one(s):
-        for d, h in zip(dq, host[s]):
-            d.copy_(h, non_blocking=True)
-        tables_d.copy_(tables_h, non_blocking=True)
-        q, k, v, sl, cl = dq
+        dbuf.copy_(host[s], non_blocking=True)
+        q, k, v, sl, cl, tables_d = views
         st.cache.append(k, v, sl)
         st.cache.decode(q, tables_d, cl, st.max_ctx, sm_scale=w.sm_scale, out=st.out,
                         workspace=st.ws)

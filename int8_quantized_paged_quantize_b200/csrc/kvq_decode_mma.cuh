@@ -760,9 +760,12 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           const float4 t4 = *reinterpret_cast<const float4*>(rb + g * 4);
           const float tmax = fmaxf(fmaxf(t4.x, t4.y), fmaxf(t4.z, t4.w));
           const float mn = fmaxf(m[g], tmax);
-          alpha[g] = (mn == -INFINITY) ? 1.f : exp2f(m[g] - mn);
-          m[g] = mn;
-          o[g] *= alpha[g];
+          alpha[g] = 1.f;
+          if (mn != m[g]) {                      // the same for every thread of the CTA
+            alpha[g] = (mn == -INFINITY) ? 1.f : exp2f(m[g] - mn);
+            m[g] = mn;
+            o[g] *= alpha[g];
+          }
         }
         // P = p * v_scale * 2^ex with max(v_scale) * 2^ex in [128, 256): inside
         // the E4M3 range, and below 2^8 for the 24-bit fixed point of INT8
@@ -847,12 +850,14 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           // Y = rint(y * 2^16) < 2^24; its three bytes are the parts (weights
           // 1, 1/256, 1/65536); zero_point * P is summed from the same Y
           uint32_t yv[G];
+          const float ysc = sv * escale * 65536.f;
+          const float zsc = zv * einv * (1.f / 65536.f);
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
             l[g] = l[g] * alpha[g] + pr;
-            yv[g] = __float2uint_rn(pr * sv * escale * 65536.f);
-            corr[g] = corr[g] * alpha[g] + zv * float(yv[g]) * (1.f / 65536.f) * einv;
+            yv[g] = __float2uint_rn(pr * ysc);
+            corr[g] = corr[g] * alpha[g] + float(yv[g]) * zsc;
           }
           uint32_t words[C::NO / 4];
 #pragma unroll

@@ -85,6 +85,20 @@ def test_split_k_on_and_off_agree(fmt):
     assert (a.out - b.out).abs().max().item() < 1e-3
 
 
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("part", [0, 128])
+def test_many_short_sequences_split_across_ctas(fmt, part):
+    """The persistent kernel's work split: 120 sequences shorter than a few
+    tiles around the 128-token boundary, two long ones, GQA group 4. With
+    partition 128 every CTA's share crosses many (sequence, head) runs, and
+    some shares end inside a run's opening cost, so they hold no tile of it."""
+    rng = np.random.default_rng(7)
+    ctx = [int(c) for c in rng.integers(0, 300, size=120)] + [0, 126, 127, 128, 255, 3000, 5000]
+    w = _synthetic(fmt, 128, 4, Hk=2, ctx=ctx, kv_mean=0.3 if fmt == "int8" else 0.0)
+    run = GC.run_gpu(w, fmt, partition_tokens=part)
+    _check(run)
+
+
 @pytest.mark.parametrize("fmt", ["fp8", "int8"])
 def test_history_appended_in_chunks_is_identical(fmt):
     w = _synthetic(fmt, 128, 4, ctx=[100, 777, 31])
