@@ -205,8 +205,10 @@ int kvq_append(const void* k, const void* v, const int64_t* slot_mapping, int32_
 /* ------------------------------------------------------------------------ */
 /*
  * Scratch bytes kvq_decode_attn needs for these sizes. partition_tokens is the
- * split-K chunk (a positive multiple of 128), or 0 to let the library choose
- * from the batch, head count, max_context_len and the device's SM count.
+ * split-K chunk (a positive multiple of 128): the smallest run of one
+ * sequence's tokens a decode CTA takes, so one (sequence, KV head) produces at
+ * most ceil(max_context_len / partition_tokens) + 1 partials. 0 lets the
+ * library choose the smallest chunk that gives at most 16 partials.
  * Returns 0 for invalid arguments.
  */
 size_t kvq_decode_workspace_bytes(int32_t batch, int32_t max_context_len, int32_t partition_tokens,
@@ -232,9 +234,10 @@ size_t kvq_decode_workspace_bytes(int32_t batch, int32_t max_context_len, int32_
  * workspace     device scratch of at least kvq_decode_workspace_bytes(...) bytes;
  *               contents on entry do not matter.
  * partition_tokens  as for kvq_decode_workspace_bytes (0 = automatic).
- * The sequence's tokens are split into chunks of partition_tokens; each chunk
- * computes an online-softmax partial (max, sum, unnormalized output) and a
- * merge kernel combines the partials with a log-sum-exp rescale.
+ * The work (sequence, KV head, 128-token tile) is shared evenly over the
+ * GPU's resident CTAs; each CTA's run of one (sequence, head) computes an
+ * online-softmax partial (max, sum, unnormalized output) and a merge kernel
+ * combines the partials with a log-sum-exp rescale.
  */
 int kvq_decode_attn(const void* q, int32_t batch, const void* k_cache, const void* v_cache,
                     const void* const* scales, const int32_t* block_tables,

@@ -28,23 +28,20 @@ int device_sm_count() {
   return n;
 }
 
-// Split-K chunking. A chunk is a whole number of 128-token tiles. Automatic
-// choice: the smallest power-of-two chunk (>= 128 tokens) for which the grid of
-// (sequence, KV head, chunk) CTAs of the longest sequence fits in 16 CTAs per
-// SM, so long contexts are spread over every SM while short ones stay in one
-// chunk (no merge traffic to speak of).
+// Split-K chunking. A chunk is a whole number of 128-token tiles; it is the
+// smallest run of one sequence's tiles a decode CTA takes, so a (sequence, KV
+// head) yields at most ceil(max_ctx / chunk) + 1 partials (the workspace
+// slots). Automatic choice: the smallest chunk that cuts the longest sequence
+// into at most 15 runs. The persistent decode kernel then spreads any batch
+// over every resident CTA while the workspace stays at 16 partials per row.
 int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kvq_dims* d,
               DecodePlan* plan) {
   if (batch < 0 || max_ctx < 0 || partition_tokens < 0) return KVQ_ERR_ARG;
   if (partition_tokens % kTileTokens != 0) return KVQ_ERR_ARG;
   int64_t part = partition_tokens;
   if (part == 0) {
-    const int64_t budget = int64_t(16) * device_sm_count();
-    const int64_t rows = int64_t(batch) * d->n_kv_heads;
-    part = kTileTokens;
-    while (part < (int64_t(1) << 20) &&
-           rows * ((int64_t(max_ctx) + part - 1) / part) > budget)
-      part *= 2;
+    const int64_t tiles = std::max<int64_t>(1, (int64_t(max_ctx) + kTileTokens - 1) / kTileTokens);
+    part = int64_t(kTileTokens) * ((tiles + 14) / 15);
   }
   const int64_t splits = std::max<int64_t>(1, (int64_t(max_ctx) + part - 1) / part);
   plan->partition = int32_t(part);
