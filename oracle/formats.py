@@ -1,4 +1,5 @@
-"""Codecs of the quantized KV cache: OCP FP8 E4M3, INT8 asymmetric, BF16 scales.
+"""Codecs of the quantized KV cache: OCP FP8 E4M3 and E5M2, INT8 asymmetric,
+BF16 scales.
 
 Test infrastructure (see ``oracle/__init__``): plain numpy, element by element
 in meaning, vectorised only for speed.
@@ -21,6 +22,9 @@ Readings taken where the pages are silent (each is a stated choice)
 * FP8 scale: ``s = bf16_rne(f32(amax) / 448)`` with an IEEE f32 division; the
   code is ``e4m3_rne_satfinite(f32(x) / f32(s))``, again an IEEE f32 division
   by the *stored* BF16 scale (no reciprocal multiply).
+* E5M2 (the pages name it as the wider-range, lower-precision FP8 variant)
+  follows the same rule with its own maximum: ``s = bf16_rne(amax / 57344)``,
+  ``code = e5m2_rne_satfinite(x / s)``.
 * INT8: codes are signed [-128, 127]; the range is widened to contain 0,
   ``s = bf16_rne((xmax - xmin) / 255)`` in f32,
   ``zp = clamp(-128 - rint(xmin / s), -128, 127)`` (an integer, exact in BF16),
@@ -112,6 +116,81 @@ def e4m3_encode(x) -> np.ndarray:
     code = np.where(np.signbit(xf), code | 0x80, code)
     code = np.where(np.isnan(xf), E4M3_NAN_CODE, code)
     return code.astype(np.uint8)
+
+
+# --------------------------------------------------------------------------- E5M2
+E5M2_MAX = 57344.0
+E5M2_NAN_CODE = 0x7F
+
+
+def e5m2_decode(codes) -> np.ndarray:
+    """Value (float64) of each OCP E5M2 byte.
+
+    Bit 7 is the sign, bits 6..2 the exponent field e (bias 15), bits 1..0 the
+    mantissa m. e == 0 encodes subnormals m/4 * 2^-14; e == 31 encodes +-inf
+    (m == 0) and NaN (m != 0); otherwise the value is (1 + m/4) * 2^(e - 15),
+    so the largest finite magnitude is (1 + 3/4) * 2^15 = 57344.
+    """
+    c = np.asarray(codes).astype(np.int64) & 0xFF
+    sign = np.where((c & 0x80) != 0, -1.0, 1.0)
+    e = (c >> 2) & 0x1F
+    m = (c & 0x3).astype(np.float64)
+    subnormal = (m / 4.0) * 2.0 ** -14
+    normal = (1.0 + m / 4.0) * np.exp2(e.astype(np.float64) - 15.0)
+    val = sign * np.where(e == 0, subnormal, normal)
+    val = np.where((e == 31) & ((c & 0x3) == 0), sign * np.inf, val)
+    return np.where((e == 31) & ((c & 0x3) != 0), np.nan, val)
+
+
+# The 124 non-negative finite magnitudes, codes 0x00..0x7B, in value order.
+_E5M2_MAGNITUDES = e5m2_decode(np.arange(0x7C))
+
+
+def e5m2_encode(x) -> np.ndarray:
+    """Encode f32 values to OCP E5M2 codes (uint8): round to nearest, ties to even,
+    saturating to +-57344 (infinities too). Same definition as e4m3_encode over
+    the E5M2 value set: nearest finite value, the even code on a tie, the sign
+    kept (-0 -> 0x80), NaN -> 0x7F.
+    """
+    xf = np.asarray(x, dtype=np.float32)
+    mag = np.abs(xf.astype(np.float64))
+    tab = _E5M2_MAGNITUDES
+    top = len(tab) - 1                                    # 0x7B
+    hi = np.clip(np.searchsorted(tab, mag, side="left"), 0, top)
+    lo = np.clip(hi - 1, 0, top)
+    d_lo = mag - tab[lo]
+    d_hi = tab[hi] - mag
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(mag >= tab[hi], hi, code)            # exact hit (includes 0)
+    code = np.where(mag >= E5M2_MAX, top, code)          # satfinite
+    code = code.astype(np.int64)
+    code = np.where(np.signbit(xf), code | 0x80, code)
+    code = np.where(np.isnan(xf), E5M2_NAN_CODE, code)
+    return code.astype(np.uint8)
+
+
+def e5m2_scale(rows) -> np.ndarray:
+    """BF16 scale per row, as f32: ``s = bf16_rne(amax / 57344)`` (IEEE f32 division)."""
+    r = np.asarray(rows, dtype=np.float32)
+    amax = np.max(np.abs(r), axis=-1).astype(np.float32)
+    return bf16_round(amax / np.float32(E5M2_MAX))
+
+
+def e5m2_quantize(rows):
+    """(codes uint8[..., D], scales f32[...]): code = e5m2_encode(f32(x) / f32(s))
+    with the stored BF16 scale; a zero scale gives all-zero codes."""
+    r = np.asarray(rows, dtype=np.float32)
+    s = e5m2_scale(r)
+    safe = np.where(s == 0.0, np.float32(1.0), s).astype(np.float32)
+    codes = e5m2_encode(r / safe[..., None])
+    codes = np.where((s == 0.0)[..., None], np.uint8(0), codes).astype(np.uint8)
+    return codes, s
+
+
+def e5m2_dequantize(codes, scales) -> np.ndarray:
+    """float64 values of E5M2 codes: e5m2(c) * s, exact."""
+    return e5m2_decode(codes) * np.asarray(scales, dtype=np.float64)[..., None]
 
 
 # --------------------------------------------------------------------------- FP8 per-token scale

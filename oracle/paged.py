@@ -32,7 +32,7 @@ import numpy as np
 
 from . import formats
 
-FORMATS = ("bf16", "fp8", "int8")
+FORMATS = ("bf16", "fp8", "int8", "e5m2")
 
 
 def slot_of(block_table_row, pos, block_size):
@@ -47,6 +47,7 @@ class LogicalPool:
 
     bf16: codes hold the BF16 values themselves (as f32).
     fp8:  uint8 E4M3 codes + f32 scales (BF16 values).
+    e5m2: uint8 E5M2 codes + f32 scales (BF16 values).
     int8: int8 codes + f32 scales (BF16 values) + int64 zero points.
     """
 
@@ -57,7 +58,7 @@ class LogicalPool:
         self.num_blocks, self.n_kv_heads = num_blocks, n_kv_heads
         self.block_size, self.head_dim = block_size, head_dim
         shape = (num_blocks, n_kv_heads, block_size, head_dim)
-        dtype = {"bf16": np.float32, "fp8": np.uint8, "int8": np.int8}[fmt]
+        dtype = {"bf16": np.float32, "fp8": np.uint8, "int8": np.int8, "e5m2": np.uint8}[fmt]
         self.k = np.zeros(shape, dtype=dtype)
         self.v = np.zeros(shape, dtype=dtype)
         mshape = shape[:3]
@@ -94,6 +95,10 @@ class LogicalPool:
                 c, s = formats.fp8_quantize(src)
                 codes[blk, :, off, :] = c
                 scale[blk, :, off] = s
+            elif self.fmt == "e5m2":
+                c, s = formats.e5m2_quantize(src)
+                codes[blk, :, off, :] = c
+                scale[blk, :, off] = s
             else:
                 c, s, z = formats.int8_quantize(src)
                 codes[blk, :, off, :] = c
@@ -110,6 +115,8 @@ class LogicalPool:
             return codes.astype(np.float64)
         if self.fmt == "fp8":
             return formats.fp8_dequantize(codes, scale)
+        if self.fmt == "e5m2":
+            return formats.e5m2_dequantize(codes, scale)
         return formats.int8_dequantize(codes, scale, zp)
 
     def gather(self, block_table_row, ctx):

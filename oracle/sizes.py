@@ -22,7 +22,8 @@ from __future__ import annotations
 from fractions import Fraction
 
 BYTES_PER_ELEMENT = {"fp16": Fraction(2), "bf16": Fraction(2), "fp8": Fraction(1),
-                     "int8": Fraction(1), "int4": Fraction(1, 2), "int2": Fraction(1, 4)}
+                     "e5m2": Fraction(1), "int8": Fraction(1), "int4": Fraction(1, 2),
+                     "int2": Fraction(1, 4)}
 
 
 def kv_bytes(layers, n_kv_heads, head_dim, seq_len, batch, bytes_per_element):
@@ -38,5 +39,5 @@ def per_token_kv_bytes(layers, n_kv_heads, head_dim, bytes_per_element):
 def scale_bytes(layers, n_kv_heads, seq_len, batch, fmt):
     """Bytes of the per-token, per-KV-head BF16 metadata of K and V:
     one scale (FP8) or a scale and a zero point (INT8) per row; none for BF16."""
-    per_row = {"bf16": 0, "fp16": 0, "fp8": 2, "int8": 4}[fmt]
+    per_row = {"bf16": 0, "fp16": 0, "fp8": 2, "e5m2": 2, "int8": 4}[fmt]
     return 2 * layers * n_kv_heads * seq_len * batch * per_row
