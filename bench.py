@@ -38,10 +38,10 @@ sys.path.insert(0, ROOT)
 from int8_quantized_paged_quantize_b200 import workloads as WL  # noqa: E402
 
 DEFAULT_WORKLOAD = "llama3-8b-fp8"
-META_BYTES = {"fp8": 4, "int8": 8, "bf16": 0}       # per (token, KV head): K and V metadata
-ELEM = {"fp8": 1, "int8": 1, "bf16": 2}
+META_BYTES = {"fp8": 4, "int8": 8, "bf16": 0, "e5m2": 4}       # per (token, KV head): K and V metadata
+ELEM = {"fp8": 1, "int8": 1, "bf16": 2, "e5m2": 1}
 DTYPE_TAG = {"fp8": "e4m3 cache / f32 accumulate", "int8": "s8 cache / f32 accumulate",
-             "bf16": "bf16 cache / f32 accumulate"}
+             "bf16": "bf16 cache / f32 accumulate", "e5m2": "e5m2 cache / f32 accumulate"}
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -479,7 +479,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WL.WORKLOADS))
-    ap.add_argument("--fmt", default=None, choices=["fp8", "int8", "bf16"])
+    ap.add_argument("--fmt", default=None, choices=["fp8", "int8", "bf16", "e5m2"])
     ap.add_argument("--no-formats", action="store_true", help="skip the per-format comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--ref-budget", type=float, default=10.0)
@@ -526,7 +526,7 @@ def main():
     formats = {}
     outs = {}
     if not args.no_formats:
-        for f in ("fp8", "int8", "bf16"):
+        for f in ("fp8", "int8", "e5m2", "bf16"):
             if f == fmt:
                 tf, stf = t, st
             else:
@@ -558,7 +558,7 @@ def main():
             st = stf
         # quality number (reported, not a pass criterion): the quantized cache's
         # attention output against the same kernel on the unquantized BF16 cache
-        for f in ("fp8", "int8"):
+        for f in ("fp8", "int8", "e5m2"):
             dev = (outs[f] - outs["bf16"]).abs()
             ref = outs["bf16"].abs()
             formats[f]["quality_vs_bf16_cache"] = {

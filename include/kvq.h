@@ -48,7 +48,7 @@
  *   V cache  [num_blocks][n_kv_heads][E][D][16/E]: chunk (u, d) holds tokens
  *            t in [u*16/E, (u+1)*16/E) of channel d, at page offset (u*D + d)*16
  *            (the page is stored transposed)
- *   scales   FP8:  [num_blocks][n_kv_heads][block_size]    BF16 scale
+ *   scales   FP8 (E4M3, E5M2): [num_blocks][n_kv_heads][block_size] BF16 scale
  *            INT8: [num_blocks][n_kv_heads][block_size][2] BF16 {scale, zero_point}
  *            BF16: none (pass NULL)
  * Both pages are tensor-core operands as stored: K is the K-major operand of
@@ -73,7 +73,8 @@ typedef struct CUstream_st* kvq_stream_t;
 typedef enum {
   KVQ_BF16 = 0,      /* unquantized BF16 cache: the comparison baseline */
   KVQ_FP8_E4M3 = 1,  /* OCP E4M3 codes (max 448, RNE, saturating) + BF16 scale */
-  KVQ_INT8_ASYM = 2  /* signed int8 codes + BF16 {scale, zero_point} */
+  KVQ_INT8_ASYM = 2, /* signed int8 codes + BF16 {scale, zero_point} */
+  KVQ_FP8_E5M2 = 3   /* OCP E5M2 codes (max 57344, RNE, saturating) + BF16 scale */
 } kvq_fmt;
 
 typedef enum {

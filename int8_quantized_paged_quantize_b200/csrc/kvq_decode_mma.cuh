@@ -59,7 +59,7 @@ __host__ __device__ constexpr int round_up16(int x) { return x < 16 ? 16 : (x + 
 template <int D, int G, int FMT>
 struct MmaCfg {
   static constexpr bool BF = FMT == KVQ_BF16;
-  static constexpr bool F8 = FMT == KVQ_FP8_E4M3;
+  static constexpr bool F8 = FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2;   // either FP8 code
   static constexpr bool I8 = FMT == KVQ_INT8_ASYM;
   static constexpr int E = BF ? 2 : 1;                         // bytes per element
   static constexpr int KIND = BF ? 0 : (F8 ? 1 : 2);           // mma_ss kind
@@ -458,9 +458,11 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t dfmt = C::I8 ? 2u : 1u;
-      constexpr uint32_t afmt = C::BF ? 1u : (C::I8 ? 1u : 0u);       // bf16 / s8 / E4M3
-      constexpr uint32_t qfmt = afmt;                                   // Q parts: same family
-      constexpr uint32_t pfmt = C::BF ? 1u : 0u;                        // bf16 / u8 / E4M3
+      // A (cache codes): bf16 / s8 / E4M3 (0) or E5M2 (1); B (query and weight
+      // parts): bf16 / s8 and u8 / E4M3, whatever FP8 variant the cache holds
+      constexpr uint32_t afmt = (C::BF || C::I8 || FMT == KVQ_FP8_E5M2) ? 1u : 0u;
+      constexpr uint32_t qfmt = (C::BF || C::I8) ? 1u : 0u;
+      constexpr uint32_t pfmt = C::BF ? 1u : 0u;
       constexpr uint32_t id_s = idesc_m128(dfmt, afmt, qfmt, false, C::NS);
       constexpr uint32_t id_pv = idesc_m128(dfmt, afmt, pfmt, true, C::NO);
       const uint32_t kbase = smem_u32(kring), vbase = smem_u32(vring);

@@ -138,18 +138,20 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
 #pragma unroll
     for (int i = 0; i < E / 2; ++i) { x[2 * i] = bf16_lo(raw[i]); x[2 * i + 1] = bf16_hi(raw[i]); }
     uint32_t packed = 0;
-    if constexpr (FMT == KVQ_FP8_E4M3) {
+    if constexpr (FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2) {
+      // s = bf16(amax / max code), code = fp8_rne_satfinite(x / s)
+      constexpr bool E4 = FMT == KVQ_FP8_E4M3;
       float amax = 0.f;
 #pragma unroll
       for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(x[i]));
       amax = warp_max(amax);
-      rc.s = __float2bfloat16_rn(__fdiv_rn(amax, 448.0f));
+      rc.s = __float2bfloat16_rn(__fdiv_rn(amax, E4 ? 448.0f : 57344.0f));
       const float s = __bfloat162float(rc.s);
       if (s != 0.f) {
 #pragma unroll
         for (int i = 0; i < E; i += 2) {
           const float2 qv = make_float2(__fdiv_rn(x[i], s), __fdiv_rn(x[i + 1], s));
-          const uint32_t two = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
+          const uint32_t two = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, E4 ? __NV_E4M3 : __NV_E5M2);
           packed |= two << (8 * i);
         }
       }
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(256) append_kernel(
   constexpr int ROWB = D * ELT;                 // bytes of one token row
   constexpr int PADB = ROWB + 16;               // padded smem row (bank spread)
   constexpr int PAGEB = kBlockSize * ROWB;
-  constexpr int MV = (FMT == KVQ_FP8_E4M3) ? 1 : (FMT == KVQ_INT8_ASYM ? 2 : 0);
+  constexpr int MV = (FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2) ? 1 : (FMT == KVQ_INT8_ASYM ? 2 : 0);
   __shared__ __align__(16) uint8_t kbuf[kBlockSize * PADB];
   __shared__ __align__(16) uint8_t vbuf[kBlockSize * PADB];
   __shared__ __nv_bfloat16 kmb[kBlockSize][2], vmb[kBlockSize][2];
@@ -696,7 +698,6 @@ int decode_kernel_choice() {
   }();
   return choice;
 }
-bool use_simt_decode() { return decode_kernel_choice() == 2; }
 
 template <int D, int FMT>
 cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, const void* vc,
@@ -704,28 +705,22 @@ cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, co
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
                              const DecodePlan& plan, void* ws, const kvq_dims& d,
                              cudaStream_t st) {
-  if (decode_kernel_choice() == 0) {
-    switch (G) {
-      case 1: return decode_mma_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-      case 2: return decode_mma_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-      case 4: return decode_mma_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-      default: return decode_mma_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-    }
+#define KVQ_G_SWITCH(DISPATCH)                                                                   \
+  switch (G) {                                                                                   \
+    case 1: return DISPATCH<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st); \
+    case 2: return DISPATCH<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st); \
+    case 4: return DISPATCH<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st); \
+    default: return DISPATCH<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st); \
   }
-  if (decode_kernel_choice() == 1) {
-    switch (G) {
-      case 1: return decode_tc_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-      case 2: return decode_tc_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-      case 4: return decode_tc_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-      default: return decode_tc_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-    }
+  if constexpr (FMT == KVQ_FP8_E5M2) {
+    // E5M2 exists only in the tensor-core kernel that multiplies the codes
+    KVQ_G_SWITCH(decode_mma_dispatch3)
+  } else {
+    if (decode_kernel_choice() == 0) { KVQ_G_SWITCH(decode_mma_dispatch3) }
+    if (decode_kernel_choice() == 1) { KVQ_G_SWITCH(decode_tc_dispatch3) }
+    KVQ_G_SWITCH(decode_dispatch3)
   }
-  switch (G) {
-    case 1: return decode_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-    case 2: return decode_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-    case 4: return decode_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-    default: return decode_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st);
-  }
+#undef KVQ_G_SWITCH
 }
 }  // namespace
 
@@ -735,10 +730,12 @@ int launch_append(const void* k, const void* v, const int64_t* slots, int32_t T,
   cudaError_t e;
   if (d.head_dim == 128) {
     if (fmt == KVQ_FP8_E4M3) e = append_dispatch<128, KVQ_FP8_E4M3>(k, v, slots, T, kc, vc, ks, vs, d, st);
+    else if (fmt == KVQ_FP8_E5M2) e = append_dispatch<128, KVQ_FP8_E5M2>(k, v, slots, T, kc, vc, ks, vs, d, st);
     else if (fmt == KVQ_INT8_ASYM) e = append_dispatch<128, KVQ_INT8_ASYM>(k, v, slots, T, kc, vc, ks, vs, d, st);
     else e = append_dispatch<128, KVQ_BF16>(k, v, slots, T, kc, vc, ks, vs, d, st);
   } else {
     if (fmt == KVQ_FP8_E4M3) e = append_dispatch<64, KVQ_FP8_E4M3>(k, v, slots, T, kc, vc, ks, vs, d, st);
+    else if (fmt == KVQ_FP8_E5M2) e = append_dispatch<64, KVQ_FP8_E5M2>(k, v, slots, T, kc, vc, ks, vs, d, st);
     else if (fmt == KVQ_INT8_ASYM) e = append_dispatch<64, KVQ_INT8_ASYM>(k, v, slots, T, kc, vc, ks, vs, d, st);
     else e = append_dispatch<64, KVQ_BF16>(k, v, slots, T, kc, vc, ks, vs, d, st);
   }
@@ -756,10 +753,12 @@ int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* 
 #define KVQ_DEC(DD, FF) decode_dispatch2<DD, FF>(G, q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st)
   if (d.head_dim == 128) {
     if (fmt == KVQ_FP8_E4M3) e = KVQ_DEC(128, KVQ_FP8_E4M3);
+    else if (fmt == KVQ_FP8_E5M2) e = KVQ_DEC(128, KVQ_FP8_E5M2);
     else if (fmt == KVQ_INT8_ASYM) e = KVQ_DEC(128, KVQ_INT8_ASYM);
     else e = KVQ_DEC(128, KVQ_BF16);
   } else {
     if (fmt == KVQ_FP8_E4M3) e = KVQ_DEC(64, KVQ_FP8_E4M3);
+    else if (fmt == KVQ_FP8_E5M2) e = KVQ_DEC(64, KVQ_FP8_E5M2);
     else if (fmt == KVQ_INT8_ASYM) e = KVQ_DEC(64, KVQ_INT8_ASYM);
     else e = KVQ_DEC(64, KVQ_BF16);
   }

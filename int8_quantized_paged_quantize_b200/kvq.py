@@ -17,9 +17,9 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
 
-FMT = {"bf16": 0, "fp8": 1, "int8": 2}
-ELEM_BYTES = {"bf16": 2, "fp8": 1, "int8": 1}
-META_VALUES = {"bf16": 0, "fp8": 1, "int8": 2}
+FMT = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 3}
+ELEM_BYTES = {"bf16": 2, "fp8": 1, "int8": 1, "e5m2": 1}
+META_VALUES = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 1}
 BLOCK_SIZE = 16
 
 DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8

@@ -131,6 +131,10 @@ def oracle_sequence(run: GpuRun, b: int):
             c, s = OF.fp8_quantize(x)
             res[name + "_codes"], res[name + "_scale"] = c, s
             res[name.upper()] = OF.fp8_dequantize(c, s)
+        elif run.fmt == "e5m2":
+            c, s = OF.e5m2_quantize(x)
+            res[name + "_codes"], res[name + "_scale"] = c, s
+            res[name.upper()] = OF.e5m2_dequantize(c, s)
         elif run.fmt == "int8":
             c, s, z = OF.int8_quantize(x)
             res[name + "_codes"], res[name + "_scale"], res[name + "_zp"] = c, s, z
@@ -155,7 +159,7 @@ def gpu_sequence(run: GpuRun, b: int):
     if run.fmt != "bf16":
         for name, t in (("k", run.cache.k_scale), ("v", run.cache.v_scale)):
             m = t[ids]                                       # [pages][Hk][16](,2)
-            if run.fmt == "fp8":
+            if run.fmt in ("fp8", "e5m2"):
                 m = m.permute(0, 2, 1).reshape(pages * 16, -1)[:n].float().cpu().numpy()
                 out[name + "_scale"] = m
             else:
@@ -171,7 +175,7 @@ def assert_codes_equal(run: GpuRun, b: int, ref: dict):
         gc = g[name + "_codes"]
         if run.fmt == "bf16":
             assert torch.equal(gc.float(), torch.from_numpy(ref[name + "_codes"])), name
-        elif run.fmt == "fp8":
+        elif run.fmt in ("fp8", "e5m2"):
             assert np.array_equal(gc.numpy(), ref[name + "_codes"]), f"{name} codes b={b}"
         else:
             assert np.array_equal(gc.numpy().view(np.int8), ref[name + "_codes"]), f"{name} codes b={b}"

@@ -33,6 +33,11 @@ def test_llama3_8b_fp8_full():
     _run_and_check("llama3-8b-fp8", "fp8", extra=(7, 41))
 
 
+def test_llama3_8b_e5m2_full():
+    """The same workload on an E5M2 cache (the wider-range FP8 variant)."""
+    _run_and_check("llama3-8b-fp8", "e5m2", extra=(7, 41))
+
+
 def test_70b_32k_int8_full():
     _run_and_check("70b-32k-int8", "int8", extra=(9,))
 

@@ -21,7 +21,7 @@ from tests import gpu_cases as GC
 
 pytestmark = pytest.mark.gpu
 
-FORMATS = ["fp8", "int8", "bf16"]
+FORMATS = ["fp8", "int8", "bf16", "e5m2"]
 RAGGED = [1, 15, 16, 17, 127, 128, 129, 300, 555]
 
 
