@@ -124,6 +124,49 @@ __device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint32_t (&ra
   }
 }
 
+// a / c for a constant c > 0 and a >= 0: RN(a * RN(1/c)) corrected once on the
+// exact FMA residual. For c = 448 and c = 57344 over every BF16 a, and for
+// c = 255 over every a = RN(hi - lo) of BF16 hi >= 0 >= lo, this is the IEEE
+// quotient bit for bit (tests/test_scale_division.py enumerates all of them),
+// so the row scales are those of a plain division.
+template <int C>
+__device__ __forceinline__ float div_by_const(float a) {
+  constexpr float c = float(C), r = 1.0f / float(C);
+  const float q = __fmul_rn(a, r);
+  return __fmaf_rn(__fmaf_rn(-q, c, a), r, q);
+}
+
+// x / s for the row's BF16 scale s > 0, as the codes need it. For s >= 2^-100
+// it is RN(x * RN(1/s)) corrected once on the exact FMA residual (Markstein's
+// method; the test for a zero residual keeps the sign of -0): it may differ
+// from the IEEE quotient in the last bit, but the E4M3, E5M2 and rint codes
+// taken from it are the IEEE quotient's for every BF16 x with |x| <= 65536 s,
+// subnormal x included (enumerated by tests/test_scale_division.py). Rows with
+// a smaller scale take the IEEE division.
+struct ScaleDiv {
+  float s, r;
+  bool fast;
+  __device__ __forceinline__ explicit ScaleDiv(float s_) {
+    s = s_;
+    fast = s_ >= 7.88860905e-31f;                   // 2^-100
+    r = fast ? __frcp_rn(s_) : 0.f;
+  }
+  __device__ __forceinline__ float operator()(float x) const {
+    if (!fast) return __fdiv_rn(x, s);
+    const float q = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-q, s, x);
+    return e != 0.f ? __fmaf_rn(e, r, q) : q;
+  }
+};
+
+// Warp-wide max(0, max of v) for floats: non-negative floats order as their
+// bit patterns read as signed integers, and every negative float (-0 included)
+// reads as a negative integer, so one integer max-reduction with a floor of 0
+// gives the float maximum, +0 when nothing is positive.
+__device__ __forceinline__ float warp_max_floor0(int bits) {
+  return __int_as_float(__reduce_max_sync(0xffffffffu, max(bits, 0)));
+}
+
 template <int D, int FMT>
 __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowCodes<D, FMT>& rc) {
   constexpr int E = D / 32;
@@ -141,34 +184,39 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
     if constexpr (FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2) {
       // s = bf16(amax / max code), code = fp8_rne_satfinite(x / s)
       constexpr bool E4 = FMT == KVQ_FP8_E4M3;
-      float amax = 0.f;
+      int amax_bits = 0;
 #pragma unroll
-      for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(x[i]));
-      amax = warp_max(amax);
-      rc.s = __float2bfloat16_rn(__fdiv_rn(amax, E4 ? 448.0f : 57344.0f));
+      for (int i = 0; i < E; ++i) amax_bits = max(amax_bits, __float_as_int(fabsf(x[i])));
+      const float amax = warp_max_floor0(amax_bits);
+      rc.s = __float2bfloat16_rn(E4 ? div_by_const<448>(amax) : div_by_const<57344>(amax));
       const float s = __bfloat162float(rc.s);
       if (s != 0.f) {
+        const ScaleDiv div(s);
 #pragma unroll
         for (int i = 0; i < E; i += 2) {
-          const float2 qv = make_float2(__fdiv_rn(x[i], s), __fdiv_rn(x[i + 1], s));
+          const float2 qv = make_float2(div(x[i]), div(x[i + 1]));
           const uint32_t two = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, E4 ? __NV_E4M3 : __NV_E5M2);
           packed |= two << (8 * i);
         }
       }
-    } else {  // INT8 asymmetric
-      float lo = 0.f, hi = 0.f;
+    } else {  // INT8 asymmetric: range [lo, hi] widened to hold 0
+      int hi_bits = 0, nlo_bits = 0;
 #pragma unroll
-      for (int i = 0; i < E; ++i) { lo = fminf(lo, x[i]); hi = fmaxf(hi, x[i]); }
-      lo = warp_min(lo);
-      hi = warp_max(hi);
-      rc.s = __float2bfloat16_rn(__fdiv_rn(__fsub_rn(hi, lo), 255.0f));
+      for (int i = 0; i < E; ++i) {
+        hi_bits = max(hi_bits, __float_as_int(x[i]));
+        nlo_bits = max(nlo_bits, __float_as_int(-x[i]));
+      }
+      const float hi = warp_max_floor0(hi_bits);     // max(0, max x)
+      const float nlo = warp_max_floor0(nlo_bits);   // -min(0, min x)
+      rc.s = __float2bfloat16_rn(div_by_const<255>(__fadd_rn(hi, nlo)));
       const float s = __bfloat162float(rc.s);
       if (s != 0.f) {
-        const float zq = fminf(fmaxf(__fdiv_rn(lo, s), -1024.f), 1024.f);
+        const ScaleDiv div(s);
+        const float zq = fminf(fmaxf(-div(nlo), -1024.f), 1024.f);   // lo / s
         rc.zp = min(127, max(-128, -128 - __float2int_rn(zq)));
 #pragma unroll
         for (int i = 0; i < E; ++i) {
-          const float qf = fminf(fmaxf(__fdiv_rn(x[i], s), -1024.f), 1024.f);
+          const float qf = fminf(fmaxf(div(x[i]), -1024.f), 1024.f);
           const int c = min(127, max(-128, __float2int_rn(qf) + rc.zp));
           packed |= uint32_t(uint8_t(int8_t(c))) << (8 * i);
         }
@@ -178,42 +226,91 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
   }
 }
 
+// Bytes [p, e) of the 16-byte chunk at dst (16-byte aligned) from w, with the
+// widest aligned stores the range allows: one 16-byte store for a whole chunk,
+// else 8-, 4-, 2- and 1-byte pieces. Bytes outside [p, e) are not touched, so
+// writers of disjoint byte ranges of one chunk never clobber each other.
+__device__ __forceinline__ void store_bytes16(uint8_t* dst, const uint32_t (&w)[4], int p, int e) {
+  if (p == 0 && e == 16) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    return;
+  }
+#pragma unroll
+  for (int h8 = 0; h8 < 2; ++h8) {
+    const int a8 = max(p, 8 * h8), b8 = min(e, 8 * h8 + 8);
+    if (a8 >= b8) continue;
+    if (a8 == 8 * h8 && b8 == 8 * h8 + 8) {
+      *reinterpret_cast<uint2*>(dst + 8 * h8) = make_uint2(w[2 * h8], w[2 * h8 + 1]);
+      continue;
+    }
+#pragma unroll
+    for (int h4 = 0; h4 < 2; ++h4) {
+      const int base4 = 8 * h8 + 4 * h4;
+      const int a4 = max(a8, base4), b4 = min(b8, base4 + 4);
+      if (a4 >= b4) continue;
+      const uint32_t word = w[2 * h8 + h4];
+      if (a4 == base4 && b4 == base4 + 4) {
+        *reinterpret_cast<uint32_t*>(dst + base4) = word;
+        continue;
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int base2 = base4 + 2 * h2;
+        const int a2 = max(a4, base2), b2 = min(b4, base2 + 2);
+        if (a2 >= b2) continue;
+        const uint32_t half = word >> (16 * h2);
+        if (a2 == base2 && b2 == base2 + 2)
+          *reinterpret_cast<uint16_t*>(dst + base2) = uint16_t(half);
+        else
+          dst[a2] = uint8_t(half >> (8 * (a2 - base2)));
+      }
+    }
+  }
+}
+
 // One CTA of 8 warps per (16 consecutive input tokens, KV head); each warp
-// quantizes K and V rows of its tokens. When the 16 tokens fill one page in
-// order (the bulk / prefill case) the codes are staged in shared memory and the
-// page is written as whole 16-byte chunks: K in its chunk-major layout, V
-// transposed. Otherwise every row is stored on its own: its K chunks, and one
-// element per channel down the transposed V page.
+// quantizes K and V rows of its tokens into shared memory. The input rows are
+// requested before the slots arrive (a skipped token's row is read and
+// dropped), so the two loads overlap. The window is then written in page-sized
+// pieces:
+//   - the 16 tokens fill one page in order (the bulk / prefill case): the page
+//     is written as whole 16-byte chunks, K in its chunk-major layout and V
+//     transposed with byte permutes;
+//   - otherwise each token writes its K chunks, and the tokens are grouped into
+//     segments (runs of consecutive slots inside one page); a segment writes its
+//     byte range of each transposed V chunk once, with the widest aligned
+//     stores that range allows. A page continued from an offset (chunked
+//     prefill) thus costs one partial chunk per channel, not one byte store per
+//     token and channel.
+// Register use is capped at 32 so that 8 CTAs (64 warps) fit on an SM.
 template <int D, int FMT>
-__global__ void __launch_bounds__(256) append_kernel(
-    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-    const int64_t* __restrict__ slots, int T, int Hk, int NB, uint8_t* __restrict__ kc,
-    uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs) {
+__global__ void __launch_bounds__(256, 8)
+append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+              const int64_t* __restrict__ slots, int T, int Hk, int NB, uint8_t* __restrict__ kc,
+              uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs) {
   using RC = RowCodes<D, FMT>;
   constexpr int E = RC::E, ELT = RC::ELT;
   constexpr int ROWB = D * ELT;                 // bytes of one token row
   constexpr int PADB = ROWB + 16;               // padded smem row (bank spread)
   constexpr int PAGEB = kBlockSize * ROWB;
+  constexpr int NC = ROWB / 16;                 // 16-byte chunks of a K row
+  constexpr int UC = ELT;                       // 16-byte V chunks per channel
+  constexpr int TPC = 16 / ELT;                 // tokens per V chunk
   constexpr int MV = (FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2) ? 1 : (FMT == KVQ_INT8_ASYM ? 2 : 0);
   __shared__ __align__(16) uint8_t kbuf[kBlockSize * PADB];
   __shared__ __align__(16) uint8_t vbuf[kBlockSize * PADB];
   __shared__ __nv_bfloat16 kmb[kBlockSize][2], vmb[kBlockSize][2];
   __shared__ int64_t sl[kBlockSize];
+  __shared__ int seg_i0[kBlockSize], seg_len[kBlockSize], nseg, page_fast;
 
   const int h = blockIdx.y;
   const int64_t tb = int64_t(blockIdx.x) * kBlockSize;
   const int n = int(min(int64_t(kBlockSize), int64_t(T) - tb));
-  if (threadIdx.x < kBlockSize) sl[threadIdx.x] = threadIdx.x < n ? slots[tb + threadIdx.x] : -1;
-  __syncthreads();
-  const int64_t s0 = sl[0];
-  bool fast = n == kBlockSize && s0 >= 0 && s0 % kBlockSize == 0 && s0 < int64_t(NB) * kBlockSize;
-#pragma unroll
-  for (int i = 1; i < kBlockSize; ++i) fast = fast && sl[i] == s0 + i;
-
+  const int64_t nslots = int64_t(NB) * kBlockSize;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d0 = lane * E;
-  // the warp's rows (row rr = 2 * token + {K, V}), loaded up front so that
-  // their latencies overlap
+  // the warp's rows (row rr = 2 * token + {K, V}), requested up front so that
+  // their latencies overlap with each other and with the slot load
   constexpr int RPW = 2 * kBlockSize / 8;
   uint32_t raws[RPW][D / 64];
 #pragma unroll
@@ -221,9 +318,38 @@ __global__ void __launch_bounds__(256) append_kernel(
     const int rr = warp + 8 * j, i = rr >> 1, which = rr & 1;
 #pragma unroll
     for (int e = 0; e < D / 64; ++e) raws[j][e] = 0u;
-    if (i < n && sl[i] >= 0 && sl[i] < int64_t(NB) * kBlockSize)
-      load_row<D>((which ? v : k) + ((tb + i) * Hk + h) * D + d0, raws[j]);
+    if (i < n) load_row<D>((which ? v : k) + ((tb + i) * Hk + h) * D + d0, raws[j]);
   }
+  if (threadIdx.x < kBlockSize) sl[threadIdx.x] = threadIdx.x < n ? slots[tb + threadIdx.x] : -1;
+  __syncthreads();
+
+  if (warp == 0) {
+    const int64_t si = lane < kBlockSize ? sl[lane] : -1;
+    const int64_t sp = (lane > 0 && lane < kBlockSize) ? sl[lane - 1] : -1;
+    const int64_t s0 = sl[0];
+    // whole page in order: slot i = s0 + i for all 16 tokens, s0 page-aligned
+    const bool inpage = lane >= kBlockSize || (si == s0 + lane && s0 >= 0 && s0 % kBlockSize == 0 &&
+                                               s0 < nslots && n == kBlockSize);
+    const bool fast = __all_sync(0xffffffffu, inpage);
+    // segments: a token starts one unless it continues the previous token's
+    // slot inside the same page
+    const bool valid = si >= 0 && si < nslots;
+    const bool start = valid && !(sp >= 0 && sp < nslots && si == sp + 1 && si % kBlockSize != 0);
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    const unsigned smask = __ballot_sync(0xffffffffu, start);
+    if (start) {
+      const int idx = __popc(smask & ((1u << lane) - 1u));
+      // the run ends at the next start or at the first invalid token
+      const unsigned stop = (smask | ~vmask) & ~((2u << lane) - 1u);
+      seg_i0[idx] = lane;
+      seg_len[idx] = (stop ? __ffs(stop) - 1 : 32) - lane;
+    }
+    if (lane == 0) {
+      nseg = __popc(smask);
+      page_fast = fast;
+    }
+  }
+
 #pragma unroll
   for (int j = 0; j < RPW; ++j) {
     const int rr = warp + 8 * j;
@@ -231,93 +357,141 @@ __global__ void __launch_bounds__(256) append_kernel(
     if (i >= n) continue;
     const int64_t slot = sl[i];
     if (slot < 0) continue;
-    if (slot >= int64_t(NB) * kBlockSize) {
+    if (slot >= nslots) {
       if (lane == 0) flag_error(KVQ_DEVERR_SLOT);
       continue;
     }
     RC rc;
     quantize_row<D, FMT>(raws[j], rc);
-    if (fast) {
-      uint8_t* dst = (which ? vbuf : kbuf) + i * PADB + d0 * ELT;
-      if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
-      else if constexpr (E * ELT == 4) *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
-      else *reinterpret_cast<uint16_t*>(dst) = uint16_t(rc.w[0]);
-      if (lane == 0) {
-        (which ? vmb : kmb)[i][0] = rc.s;
-        (which ? vmb : kmb)[i][1] = __int2bfloat16_rn(rc.zp);
-      }
-      continue;
-    }
-    const int64_t page = (slot / kBlockSize) * Hk + h;
-    const int off = int(slot % kBlockSize);
-    if (which == 0) {
-      // this token's chunk(s) of the K page: element d at chunk d*ELT/16
-      uint8_t* dst = kc + page * PAGEB + k_chunk_offset<ROWB>((d0 * ELT) / 16, off) + (d0 * ELT) % 16;
-      if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
-      else if constexpr (E * ELT == 4) *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
-      else *reinterpret_cast<uint16_t*>(dst) = uint16_t(rc.w[0]);
-    } else {
-      // down the transposed V page: (token off, channel d) at chunk (off*ELT/16, d)
-      uint8_t* base = vc + page * PAGEB + ((off * ELT) / 16) * (D * 16) + (off * ELT) % 16;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const uint32_t word = rc.w[(e * ELT) / 4];
-        if constexpr (ELT == 2)
-          *reinterpret_cast<uint16_t*>(base + (d0 + e) * 16) = uint16_t(word >> (16 * (e & 1)));
-        else
-          base[(d0 + e) * 16] = uint8_t(word >> (8 * (e & 3)));
-      }
-    }
-    if (MV > 0 && lane == 0) {
-      __nv_bfloat16* meta = which ? vs : ks;
-      if (MV == 1) {
-        meta[page * kBlockSize + off] = rc.s;
-      } else {
-        meta[(page * kBlockSize + off) * 2] = rc.s;
-        meta[(page * kBlockSize + off) * 2 + 1] = __int2bfloat16_rn(rc.zp);
-      }
+    uint8_t* dst = (which ? vbuf : kbuf) + i * PADB + d0 * ELT;
+    if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
+    else if constexpr (E * ELT == 4) *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
+    else *reinterpret_cast<uint16_t*>(dst) = uint16_t(rc.w[0]);
+    if (lane == 0) {
+      (which ? vmb : kmb)[i][0] = rc.s;
+      (which ? vmb : kmb)[i][1] = __int2bfloat16_rn(rc.zp);
     }
   }
-  if (!fast) return;                                 // uniform over the CTA
   __syncthreads();
-  const int64_t page = (s0 / kBlockSize) * Hk + h;
-  uint8_t* kp = kc + page * PAGEB;
-  uint8_t* vp = vc + page * PAGEB;
-  // K: chunk j = (token group t/8, c, t%8) <- bytes [16c, 16c+16) of token t's row
-  for (int j = threadIdx.x; j < PAGEB / 16; j += blockDim.x) {
-    constexpr int NC = ROWB / 16;
-    const int c = (j >> 3) % NC, t = (j / (8 * NC)) * 8 + (j & 7);
-    *reinterpret_cast<uint4*>(kp + j * 16) = *reinterpret_cast<const uint4*>(kbuf + t * PADB + c * 16);
-  }
-  // V: chunk j = (u, d) <- tokens [u*16/ELT, (u+1)*16/ELT) of channel d
-  for (int j = threadIdx.x; j < ELT * D; j += blockDim.x) {
-    const int u = j / D, d = j % D;
-    uint32_t wv[4];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      uint32_t word = 0;
-      if constexpr (ELT == 1) {
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) word |= uint32_t(vbuf[(q4 * 4 + bb) * PADB + d]) << (8 * bb);
-      } else {
-        const int t0 = u * 8 + q4 * 2;
-        word = uint32_t(*reinterpret_cast<const uint16_t*>(vbuf + t0 * PADB + 2 * d)) |
-               (uint32_t(*reinterpret_cast<const uint16_t*>(vbuf + (t0 + 1) * PADB + 2 * d)) << 16);
+
+  if (page_fast) {                                   // uniform over the CTA
+    const int64_t page = (sl[0] / kBlockSize) * Hk + h;
+    uint8_t* kp = kc + page * PAGEB;
+    uint8_t* vp = vc + page * PAGEB;
+    // items [0, KN): K chunk j = (token group t/8, c, t%8) <- bytes [16c, 16c+16)
+    // of token t's row. Items [KN, KN + VN): a V piece, from 32-bit words of
+    // the staged rows transposed with byte permutes.
+    constexpr int KN = PAGEB / 16;
+    constexpr int VN = ELT == 1 ? 2 * (D / 4) : 2 * (D / 2);
+    for (int j = threadIdx.x; j < KN + VN; j += blockDim.x) {
+      if (j < KN) {
+        const int c = (j >> 3) % NC, t = (j / (8 * NC)) * 8 + (j & 7);
+        *reinterpret_cast<uint4*>(kp + j * 16) = *reinterpret_cast<const uint4*>(kbuf + t * PADB + c * 16);
+        continue;
       }
-      wv[q4] = word;
+      const int jv = j - KN;
+      if constexpr (ELT == 1) {
+        // channels 4c..4c+3, tokens 8h..8h+7: two 4x4 byte transposes; the
+        // result is the low or high 8 bytes of four channels' chunks
+        const int c = jv % (D / 4), hh = jv / (D / 4);
+        uint32_t o[4][2];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int t0 = 8 * hh + 4 * g;
+          const uint32_t r0 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 0) * PADB + 4 * c);
+          const uint32_t r1 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 1) * PADB + 4 * c);
+          const uint32_t r2 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 2) * PADB + 4 * c);
+          const uint32_t r3 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 3) * PADB + 4 * c);
+          const uint32_t a01 = __byte_perm(r0, r1, 0x5140), a23 = __byte_perm(r2, r3, 0x5140);
+          const uint32_t b01 = __byte_perm(r0, r1, 0x7362), b23 = __byte_perm(r2, r3, 0x7362);
+          o[0][g] = __byte_perm(a01, a23, 0x5410);
+          o[1][g] = __byte_perm(a01, a23, 0x7632);
+          o[2][g] = __byte_perm(b01, b23, 0x5410);
+          o[3][g] = __byte_perm(b01, b23, 0x7632);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint2*>(vp + (4 * c + m) * 16 + 8 * hh) = make_uint2(o[m][0], o[m][1]);
+      } else {
+        // channels 2c, 2c+1, tokens 8u..8u+7: 2x2 transposes of 16-bit halves
+        const int c = jv % (D / 2), u = jv / (D / 2);
+        uint32_t lo4[4], hi4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t0 = 8 * u + 2 * q;
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vbuf + t0 * PADB + 4 * c);
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 1) * PADB + 4 * c);
+          lo4[q] = __byte_perm(w0, w1, 0x5410);
+          hi4[q] = __byte_perm(w0, w1, 0x7632);
+        }
+        *reinterpret_cast<uint4*>(vp + (u * D + 2 * c) * 16) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+        *reinterpret_cast<uint4*>(vp + (u * D + 2 * c + 1) * 16) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+      }
     }
-    *reinterpret_cast<uint4*>(vp + j * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  } else {
+    // K: whole 16-byte chunks of each token's row
+    for (int j = threadIdx.x; j < n * NC; j += blockDim.x) {
+      const int i = j / NC, c = j % NC;
+      const int64_t slot = sl[i];
+      if (slot < 0 || slot >= nslots) continue;
+      const int64_t page = (slot / kBlockSize) * Hk + h;
+      *reinterpret_cast<uint4*>(kc + page * PAGEB + k_chunk_offset<ROWB>(c, int(slot % kBlockSize))) =
+          *reinterpret_cast<const uint4*>(kbuf + i * PADB + c * 16);
+    }
+    // V: per (segment, channel d, chunk u) the segment's bytes of that chunk
+    const int ns = nseg;
+    for (int j = threadIdx.x; j < ns * D * UC; j += blockDim.x) {
+      const int sg = j / (D * UC), d = (j / UC) % D, u = j % UC;
+      const int i0 = seg_i0[sg], len = seg_len[sg];
+      const int64_t slot0 = sl[i0];
+      const int o0 = int(slot0 % kBlockSize);
+      // token offsets of the segment inside chunk u
+      const int ta = max(o0, u * TPC), tz = min(o0 + len, (u + 1) * TPC);
+      if (ta >= tz) continue;
+      uint8_t* chunk = vc + ((slot0 / kBlockSize) * Hk + h) * PAGEB + (u * D + d) * 16;
+      if (tz - ta == 1) {                            // one token: one element
+        const int i = i0 + (ta - o0), b = (ta - u * TPC) * ELT;
+        if constexpr (ELT == 1) chunk[b] = vbuf[i * PADB + d];
+        else *reinterpret_cast<uint16_t*>(chunk + b) = *reinterpret_cast<const uint16_t*>(vbuf + i * PADB + 2 * d);
+        continue;
+      }
+      uint32_t wv[4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t word = 0;
+        const int w0 = u * TPC + q4 * (4 / ELT);      // first token offset of this word
+        if (w0 + 4 / ELT > ta && w0 < tz) {
+#pragma unroll
+          for (int bb = 0; bb < 4 / ELT; ++bb) {
+            const int t = w0 + bb;
+            if (t >= ta && t < tz) {
+              const int i = i0 + (t - o0);
+              if constexpr (ELT == 1)
+                word |= uint32_t(vbuf[i * PADB + d]) << (8 * bb);
+              else
+                word |= uint32_t(*reinterpret_cast<const uint16_t*>(vbuf + i * PADB + 2 * d)) << (16 * bb);
+            }
+          }
+        }
+        wv[q4] = word;
+      }
+      store_bytes16(chunk, wv, (ta - u * TPC) * ELT, (tz - u * TPC) * ELT);
+    }
   }
+  // metadata: one thread per (token, K or V)
   if (MV > 0 && threadIdx.x < 2 * kBlockSize) {
     const int t = threadIdx.x & 15;
-    const bool isv = threadIdx.x >= kBlockSize;
-    __nv_bfloat16* meta = isv ? vs : ks;
-    const __nv_bfloat16 (*mb)[2] = isv ? vmb : kmb;
-    if (MV == 1) {
-      meta[page * kBlockSize + t] = mb[t][0];
-    } else {
-      meta[(page * kBlockSize + t) * 2] = mb[t][0];
-      meta[(page * kBlockSize + t) * 2 + 1] = mb[t][1];
+    const int64_t slot = sl[t];
+    if (t < n && slot >= 0 && slot < nslots) {
+      const bool isv = threadIdx.x >= kBlockSize;
+      __nv_bfloat16* meta = isv ? vs : ks;
+      const __nv_bfloat16 (*mb)[2] = isv ? vmb : kmb;
+      const int64_t row = ((slot / kBlockSize) * Hk + h) * kBlockSize + slot % kBlockSize;
+      if (MV == 1) {
+        meta[row] = mb[t][0];
+      } else {
+        *reinterpret_cast<__nv_bfloat162*>(meta + row * 2) = __halves2bfloat162(mb[t][0], mb[t][1]);
+      }
     }
   }
 }

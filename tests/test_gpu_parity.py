@@ -284,3 +284,34 @@ def test_bulk_and_per_row_append_write_the_same_bytes(fmt, D):
     if fmt != "bf16":
         assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
     assert kvq.device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("D", [64, 128])
+def test_segmented_windows_write_the_same_bytes(fmt, D):
+    """Windows of 16 input tokens whose slots form runs inside pages (a page
+    continued from an offset, runs crossing a page edge, holes of skipped tokens,
+    runs of one token) are stored per run; a fully shuffled order stores every
+    token on its own. The caches must be identical byte for byte."""
+    d = kvq.dims(24, 2, 4, D, 24)
+    g = torch.Generator().manual_seed(11)
+    runs = [(16 + 5, 40), (16 * 6 + 15, 1), (16 * 8 + 3, 9), (16 * 10, 16), (16 * 12 + 7, 30),
+            (16 * 15 + 1, 2), (16 * 16 + 9, 7), (16 * 18, 5), (16 * 19 + 11, 21)]
+    parts = [torch.arange(s, s + n, dtype=torch.int64) for s, n in runs]
+    slots = torch.cat(parts)
+    skip = torch.randperm(slots.numel(), generator=g)[:7]
+    slots[skip] = -1
+    n = slots.numel()
+    k = (torch.randn(n, 2, D, generator=g) * 2 + 0.3).to(torch.bfloat16).cuda()
+    v = torch.randn(n, 2, D, generator=g).to(torch.bfloat16).cuda()
+    slots = slots.cuda()
+    a = kvq.LayerCache.allocate(fmt, d)
+    a.append(k, v, slots)
+    perm = torch.randperm(n, generator=g).cuda()
+    b = kvq.LayerCache.allocate(fmt, d)
+    b.append(k[perm].contiguous(), v[perm].contiguous(), slots[perm].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
+    if fmt != "bf16":
+        assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
+    assert kvq.device_error() == 0
