@@ -32,6 +32,17 @@ Readings taken where the pages are silent (each is a stated choice)
   ``rint`` rounds half to even.
 * A zero scale (all-zero row, or a BF16 underflow) stores ``s = 0, zp = 0`` and
   all-zero codes, so every value dequantises to 0.
+* Per-channel and per-tensor INT8 ([LIMITS] "Formats you will actually meet":
+  one scale per head_dim slice is faster on hardware and slightly less
+  accurate; one scale for the whole cache is cheapest and loses most). The
+  pages give one scale and no zero point, and say nothing of where the scale
+  comes from; read as symmetric codes with a static BF16 scale fixed before
+  the tokens arrive (given by the caller): ``c = clamp(rint(f32(x) / f32(s)),
+  -127, 127)``, ``deq = c * s``; ``s <= 0`` stores code 0. Per channel means
+  one scale per (KV head, channel), for K and for V separately; per tensor one
+  for all of K and one for all of V. ``int8_static_calibrate`` is one way to
+  fix such scales from sample data (max |x| / 127, rounded to BF16); the path
+  takes them as inputs.
 """
 
 from __future__ import annotations
@@ -271,3 +282,38 @@ def int8_clip_range(scales, zero_points):
     s = np.asarray(scales, dtype=np.float64)
     zp = np.asarray(zero_points, dtype=np.int64)
     return (-128 - zp) * s, (127 - zp) * s
+
+
+# --------------------------------------------------------------------------- INT8 symmetric, static scales
+def int8_static_quantize(x, scales) -> np.ndarray:
+    """int8 codes of values x[..., D] under given scales that broadcast against
+    x (per channel: [Hk][D] against [..., Hk, D]; per tensor: a scalar):
+    c = clamp(rint(f32(x) / f32(s)), -127, 127); 0 where s <= 0 or s is NaN."""
+    r = np.asarray(x, dtype=np.float32)
+    s = np.broadcast_to(np.asarray(scales, dtype=np.float32), r.shape)
+    ok = s > 0
+    safe = np.where(ok, s, np.float32(1.0)).astype(np.float32)
+    with np.errstate(over="ignore"):
+        q = np.rint(r / safe)
+    q = np.clip(q, -127, 127)
+    return np.where(ok, q, 0).astype(np.int8)
+
+
+def int8_static_dequantize(codes, scales) -> np.ndarray:
+    """float64 values of static-scale INT8 codes: c * s (s broadcast as in
+    int8_static_quantize)."""
+    c = np.asarray(codes).astype(np.float64)
+    return c * np.broadcast_to(np.asarray(scales, dtype=np.float64), c.shape)
+
+
+def int8_static_calibrate(x, per_channel=True) -> np.ndarray:
+    """Static scales from sample values x[..., Hk, D]: bf16_rne(f32(max |x|) /
+    127) over every axis but (Hk, D) (per channel, shape [Hk][D]) or over all
+    of x (per tensor, shape [1])."""
+    a = np.abs(np.asarray(x, dtype=np.float32))
+    if per_channel:
+        amax = a.reshape(-1, a.shape[-2], a.shape[-1]).max(axis=0)
+    else:
+        amax = np.array([a.max()], dtype=np.float32)
+    return bf16_round(amax.astype(np.float32) / np.float32(127.0))
+

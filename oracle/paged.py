@@ -32,7 +32,8 @@ import numpy as np
 
 from . import formats
 
-FORMATS = ("bf16", "fp8", "int8", "e5m2")
+FORMATS = ("bf16", "fp8", "int8", "e5m2", "int8c", "int8t")
+STATIC_FORMATS = ("int8c", "int8t")
 
 
 def slot_of(block_table_row, pos, block_size):
@@ -49,16 +50,24 @@ class LogicalPool:
     fp8:  uint8 E4M3 codes + f32 scales (BF16 values).
     e5m2: uint8 E5M2 codes + f32 scales (BF16 values).
     int8: int8 codes + f32 scales (BF16 values) + int64 zero points.
+    int8c / int8t: int8 codes under static scales given here (BF16 values):
+    [n_kv_heads][head_dim] per channel or [1] per tensor, for K and for V.
     """
 
-    def __init__(self, fmt, num_blocks, n_kv_heads, block_size, head_dim):
+    def __init__(self, fmt, num_blocks, n_kv_heads, block_size, head_dim, k_static=None,
+                 v_static=None):
         if fmt not in FORMATS:
             raise ValueError(fmt)
+        if fmt in STATIC_FORMATS:
+            shape = (n_kv_heads, head_dim) if fmt == "int8c" else (1,)
+            self.k_static = np.asarray(k_static, dtype=np.float32).reshape(shape)
+            self.v_static = np.asarray(v_static, dtype=np.float32).reshape(shape)
         self.fmt = fmt
         self.num_blocks, self.n_kv_heads = num_blocks, n_kv_heads
         self.block_size, self.head_dim = block_size, head_dim
         shape = (num_blocks, n_kv_heads, block_size, head_dim)
-        dtype = {"bf16": np.float32, "fp8": np.uint8, "int8": np.int8, "e5m2": np.uint8}[fmt]
+        dtype = {"bf16": np.float32, "fp8": np.uint8, "int8": np.int8, "e5m2": np.uint8,
+                 "int8c": np.int8, "int8t": np.int8}[fmt]
         self.k = np.zeros(shape, dtype=dtype)
         self.v = np.zeros(shape, dtype=dtype)
         mshape = shape[:3]
@@ -86,10 +95,13 @@ class LogicalPool:
             raise IndexError("slot beyond the pool")
         blk = slots[keep] // self.block_size
         off = slots[keep] % self.block_size
-        for src, codes, scale, zp in ((k[keep], self.k, self.k_scale, self.k_zp),
-                                      (v[keep], self.v, self.v_scale, self.v_zp)):
+        for which, src, codes, scale, zp in (("k", k[keep], self.k, self.k_scale, self.k_zp),
+                                             ("v", v[keep], self.v, self.v_scale, self.v_zp)):
             # src: [n][Hk][D]; codes[blk, :, off, :] is [n][Hk][D]
-            if self.fmt == "bf16":
+            if self.fmt in STATIC_FORMATS:
+                st = self.k_static if which == "k" else self.v_static
+                codes[blk, :, off, :] = formats.int8_static_quantize(src, st)
+            elif self.fmt == "bf16":
                 codes[blk, :, off, :] = formats.bf16_round(src)
             elif self.fmt == "fp8":
                 c, s = formats.fp8_quantize(src)
@@ -113,6 +125,8 @@ class LogicalPool:
         zp = (self.k_zp if which == "k" else self.v_zp)[blk, :, off]
         if self.fmt == "bf16":
             return codes.astype(np.float64)
+        if self.fmt in STATIC_FORMATS:
+            return formats.int8_static_dequantize(codes, self.k_static if which == "k" else self.v_static)
         if self.fmt == "fp8":
             return formats.fp8_dequantize(codes, scale)
         if self.fmt == "e5m2":

@@ -22,7 +22,8 @@ from __future__ import annotations
 from fractions import Fraction
 
 BYTES_PER_ELEMENT = {"fp16": Fraction(2), "bf16": Fraction(2), "fp8": Fraction(1),
-                     "e5m2": Fraction(1), "int8": Fraction(1), "int4": Fraction(1, 2),
+                     "e5m2": Fraction(1), "int8": Fraction(1), "int8c": Fraction(1),
+                     "int8t": Fraction(1), "int4": Fraction(1, 2),
                      "int2": Fraction(1, 4)}
 
 
@@ -39,5 +40,13 @@ def per_token_kv_bytes(layers, n_kv_heads, head_dim, bytes_per_element):
 def scale_bytes(layers, n_kv_heads, seq_len, batch, fmt):
     """Bytes of the per-token, per-KV-head BF16 metadata of K and V:
     one scale (FP8) or a scale and a zero point (INT8) per row; none for BF16."""
-    per_row = {"bf16": 0, "fp16": 0, "fp8": 2, "e5m2": 2, "int8": 4}[fmt]
+    per_row = {"bf16": 0, "fp16": 0, "fp8": 2, "e5m2": 2, "int8": 4, "int8c": 0, "int8t": 0}[fmt]
     return 2 * layers * n_kv_heads * seq_len * batch * per_row
+
+
+def static_scale_bytes(layers, n_kv_heads, head_dim, fmt):
+    """Bytes of the static BF16 scales of K and V: one per (KV head, channel)
+    for per-channel INT8, one per cache for per-tensor INT8; independent of the
+    number of tokens."""
+    per_cache = {"int8c": n_kv_heads * head_dim * 2, "int8t": 2}.get(fmt, 0)
+    return 2 * layers * per_cache
