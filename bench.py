@@ -38,10 +38,15 @@ sys.path.insert(0, ROOT)
 from int8_quantized_paged_quantize_b200 import workloads as WL  # noqa: E402
 
 DEFAULT_WORKLOAD = "llama3-8b-fp8"
-META_BYTES = {"fp8": 4, "int8": 8, "bf16": 0, "e5m2": 4}       # per (token, KV head): K and V metadata
-ELEM = {"fp8": 1, "int8": 1, "bf16": 2, "e5m2": 1}
+# per (token, KV head): K and V metadata (the static INT8 formats keep one
+# fixed scale per channel or per cache instead)
+META_BYTES = {"fp8": 4, "int8": 8, "bf16": 0, "e5m2": 4, "int8c": 0, "int8t": 0}
+ELEM = {"fp8": 1, "int8": 1, "bf16": 2, "e5m2": 1, "int8c": 1, "int8t": 1}
 DTYPE_TAG = {"fp8": "e4m3 cache / f32 accumulate", "int8": "s8 cache / f32 accumulate",
-             "bf16": "bf16 cache / f32 accumulate", "e5m2": "e5m2 cache / f32 accumulate"}
+             "bf16": "bf16 cache / f32 accumulate", "e5m2": "e5m2 cache / f32 accumulate",
+             "int8c": "s8 cache, static per-channel scales / f32 accumulate",
+             "int8t": "s8 cache, static per-tensor scales / f32 accumulate"}
+STATIC = ("int8c", "int8t")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -202,10 +207,14 @@ class Setup:
         self.ctx0 = WL.context_lengths(w, seed) + w.bulk_append
         d = kvq.dims(nb, w.n_kv_heads, w.n_q_heads, w.head_dim, self.tables_np.shape[1])
         self.dims = d
-        self.cache = kvq.LayerCache.allocate(fmt, d)
         dev = torch.device("cuda")
-        self.tables = torch.from_numpy(self.tables_np).to(dev)
         self.hist = hist if hist is not None else self.make_history(w, seed)
+        if fmt in STATIC:
+            ks, vs = self.static_scales(self.hist, fmt == "int8c")
+            self.cache = kvq.LayerCache.allocate(fmt, d, k_static=ks.to(dev), v_static=vs.to(dev))
+        else:
+            self.cache = kvq.LayerCache.allocate(fmt, d)
+        self.tables = torch.from_numpy(self.tables_np).to(dev)
         self.fill()
         # per-step inputs, resident in HBM
         self.q, self.k, self.v, self.slots, self.ctx = [], [], [], [], []
@@ -223,6 +232,17 @@ class Setup:
         self.max_ctx = int(self.ctx_np[-1].max())
         self.ws = self.cache.workspace(w.batch, self.max_ctx)
         self.out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+
+    @staticmethod
+    def static_scales(hist, per_channel):
+        """Static INT8 scales, calibrated on the cached history before anything is
+        timed (the caller's job in a deployment): bf16(max |x| / 127) per (KV
+        head, channel) or over the whole cache, for K and for V."""
+        out = []
+        for x in hist[:2]:
+            a = x.abs().amax(dim=0).float() if per_channel else x.abs().amax().float().reshape(1)
+            out.append((a / 127.0).to(torch.bfloat16).contiguous())
+        return out
 
     @staticmethod
     def make_history(w, seed):
@@ -373,6 +393,58 @@ def bulk_append_rate(st, tokens=32768, reps=5):
     return n / (ms * 1e-3), ms, n
 
 
+def bulk_append_probe(fmt, mode, reps=5, T=32768, Hk=8, D=128):
+    """One bulk append of T tokens (all Hk heads) into a fresh cache, timed with
+    CUDA events over `reps` calls after two untimed ones. `aligned`: 4 sequences
+    of T/4 tokens, so every 16-token window is one whole page. `continued`:
+    sequences of seeded lengths in [17, 3000) laid end to end in the input, so
+    most windows straddle two pages of two sequences. Returns one JSON-ready dict."""
+    from int8_quantized_paged_quantize_b200 import kvq
+    rng = np.random.default_rng(0)
+    if mode == "aligned":
+        lens = [T // 4] * 4
+    else:
+        lens = []
+        while sum(lens) < T:
+            lens.append(int(rng.integers(17, 3000)))
+        lens[-1] -= sum(lens) - T
+    nb = sum((n + 15) // 16 for n in lens) + 8
+    perm = rng.permutation(nb)
+    slots, p = [], 0
+    for n in lens:
+        npg = (n + 15) // 16
+        blocks = perm[p:p + npg]
+        p += npg
+        pos = np.arange(n)
+        slots.append(blocks[pos // 16].astype(np.int64) * 16 + pos % 16)
+    slots = torch.from_numpy(np.concatenate(slots)).cuda()
+    d = kvq.dims(nb, Hk, Hk * 4, D, max((n + 15) // 16 for n in lens))
+    g = torch.Generator(device="cuda").manual_seed(0)
+    k = torch.randn(T, Hk, D, dtype=torch.bfloat16, device="cuda", generator=g)
+    v = torch.randn(T, Hk, D, dtype=torch.bfloat16, device="cuda", generator=g)
+    if fmt in STATIC:
+        ks, vs = Setup.static_scales((k, v), fmt == "int8c")
+        cache = kvq.LayerCache.allocate(fmt, d, k_static=ks, v_static=vs)
+    else:
+        cache = kvq.LayerCache.allocate(fmt, d)
+    for _ in range(2):
+        cache.append(k, v, slots)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        cache.append(k, v, slots)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    by = T * append_bytes_per_token(dataclasses.replace(WL.WORKLOADS[DEFAULT_WORKLOAD],
+                                                        n_kv_heads=Hk, head_dim=D), fmt)
+    hbm, kind = peaks()
+    return {"bulk_append": mode, "fmt": fmt, "tokens": T, "sequences": len(lens), "us": ms * 1e3,
+            "tok_per_s": T / (ms * 1e-3), "gbs": by / (ms * 1e6), "frac": by / (ms * 1e6) / hbm,
+            "peak_kind": kind, "bytes": by}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_decode_sample(w, fmt, seed, budget_s=12.0):
     """Time the CPU oracle on a bounded sample of the workload: for sequences in
@@ -398,7 +470,14 @@ def oracle_decode_sample(w, fmt, seed, budget_s=12.0):
         v = torch.cat([v, vn[b:b + 1]]).float().numpy()
         n = k.shape[0]
         pages = (n + 15) // 16
-        pool = OP.LogicalPool(fmt, pages, w.n_kv_heads, 16, w.head_dim)
+        if fmt in STATIC:
+            from oracle import formats as OF
+            per_channel = fmt == "int8c"
+            pool = OP.LogicalPool(fmt, pages, w.n_kv_heads, 16, w.head_dim,
+                                  k_static=OF.int8_static_calibrate(k, per_channel),
+                                  v_static=OF.int8_static_calibrate(v, per_channel))
+        else:
+            pool = OP.LogicalPool(fmt, pages, w.n_kv_heads, 16, w.head_dim)
         row = np.arange(pages)
         t0 = time.perf_counter()
         pool.append(k, v, OP.slot_of(row, np.arange(n), 16))
@@ -479,11 +558,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WL.WORKLOADS))
-    ap.add_argument("--fmt", default=None, choices=["fp8", "int8", "bf16", "e5m2"])
+    ap.add_argument("--fmt", default=None, choices=["fp8", "int8", "bf16", "e5m2", "int8c", "int8t"])
     ap.add_argument("--no-formats", action="store_true", help="skip the per-format comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--ref-budget", type=float, default=10.0)
+    ap.add_argument("--bulk-append", choices=["aligned", "continued"], default=None,
+                    help="only time one bulk append of 32,768 tokens and print its line")
+    ap.add_argument("--reps", type=int, default=5, help="timed calls of --bulk-append")
     args = ap.parse_args()
+    if args.bulk_append:
+        print(json.dumps(bulk_append_probe(args.fmt or "fp8", args.bulk_append, args.reps)))
+        return 0
     if args.impl == "reference":
         return run_reference(args)
     if args.warmup < 3:
@@ -526,7 +611,7 @@ def main():
     formats = {}
     outs = {}
     if not args.no_formats:
-        for f in ("fp8", "int8", "e5m2", "bf16"):
+        for f in ("fp8", "int8", "e5m2", "int8c", "int8t", "bf16"):
             if f == fmt:
                 tf, stf = t, st
             else:
@@ -558,7 +643,7 @@ def main():
             st = stf
         # quality number (reported, not a pass criterion): the quantized cache's
         # attention output against the same kernel on the unquantized BF16 cache
-        for f in ("fp8", "int8", "e5m2"):
+        for f in ("fp8", "int8", "e5m2", "int8c", "int8t"):
             dev = (outs[f] - outs["bf16"]).abs()
             ref = outs["bf16"].abs()
             formats[f]["quality_vs_bf16_cache"] = {

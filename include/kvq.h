@@ -74,7 +74,11 @@ typedef enum {
   KVQ_BF16 = 0,      /* unquantized BF16 cache: the comparison baseline */
   KVQ_FP8_E4M3 = 1,  /* OCP E4M3 codes (max 448, RNE, saturating) + BF16 scale */
   KVQ_INT8_ASYM = 2, /* signed int8 codes + BF16 {scale, zero_point} */
-  KVQ_FP8_E5M2 = 3   /* OCP E5M2 codes (max 57344, RNE, saturating) + BF16 scale */
+  KVQ_FP8_E5M2 = 3,  /* OCP E5M2 codes (max 57344, RNE, saturating) + BF16 scale */
+  KVQ_INT8_CHANNEL = 4, /* signed int8 codes, symmetric, one static BF16 scale per
+                           (KV head, channel), given by the caller */
+  KVQ_INT8_TENSOR = 5   /* signed int8 codes, symmetric, one static BF16 scale for
+                           the whole K (and one for V) cache, given by the caller */
 } kvq_fmt;
 
 typedef enum {
@@ -120,7 +124,10 @@ const char* kvq_status_string(int status);
  * [COMPRESS] "1. The KV cache memory problem" gives the element count
  * 2 x layers x n_kv_heads x head_dim x tokens x bytes; one cache array is one
  * of the two halves of one layer for num_blocks * block_size tokens.
- * meta_bytes is 0 for KVQ_BF16. Host only; no CUDA call.
+ * meta_bytes is 0 for KVQ_BF16; for the per-token formats it is the per-token
+ * scale array of kvq_append; for KVQ_INT8_CHANNEL it is the static
+ * [n_kv_heads][head_dim] BF16 scale array, for KVQ_INT8_TENSOR one BF16 value
+ * (padded to 16 bytes). Host only; no CUDA call.
  */
 int kvq_cache_bytes(const kvq_dims* dims, kvq_fmt fmt, size_t* cache_bytes,
                     size_t* meta_bytes);
@@ -182,12 +189,20 @@ int kvq_pool_extend_seq(kvq_pool* pool, int32_t* block_table_row, int32_t cur_le
  *               block_size skips it and sets KVQ_DEVERR_SLOT. Slots must be
  *               distinct within one call.
  * k_cache, v_cache  device, the layouts in the file header.
- * k_scale, v_scale  device scale arrays (NULL for KVQ_BF16).
+ * k_scale, v_scale  device scale arrays (NULL for KVQ_BF16). Written per token
+ *               for FP8 / E5M2 / INT8_ASYM; read-only inputs for the static
+ *               formats: KVQ_INT8_CHANNEL [n_kv_heads][head_dim] BF16,
+ *               KVQ_INT8_TENSOR [1] BF16.
  * Per (token, KV head) row of D values:
  *   FP8:  s = bf16_rne(max|x| / 448); code = e4m3_rne_satfinite(x / s)
  *   INT8: xmin = min(0, min x), xmax = max(0, max x);
  *         s = bf16_rne((xmax - xmin) / 255); zp = clamp(-128 - rint(xmin / s), -128, 127);
  *         code = clamp(rint(x / s) + zp, -128, 127)
+ *   INT8_CHANNEL / INT8_TENSOR ([LIMITS] "Formats you will actually meet": a
+ *         per-channel scale per head_dim slice, or one per-tensor scale, fixed
+ *         ahead of the tokens): s = the given scale of the element's (head,
+ *         channel) or of the cache; code = clamp(rint(x / s), -127, 127);
+ *         s <= 0 (or NaN) stores code 0. Dequantized value: code * s.
  *   (all divisions IEEE f32, rint ties to even; s == 0 stores zero codes and zp 0)
  *   BF16: the values are copied.
  */
@@ -223,7 +238,11 @@ size_t kvq_decode_workspace_bytes(int32_t batch, int32_t max_context_len, int32_
  * q             device, [batch][n_q_heads][head_dim] BF16.
  * k_cache, v_cache  device, the layouts in the file header.
  * scales        host array of 2 device pointers {k_scale, v_scale} (both NULL, or
- *               scales itself NULL, for KVQ_BF16).
+ *               scales itself NULL, for KVQ_BF16): the per-token arrays of
+ *               kvq_append, or the static arrays of the INT8_CHANNEL / TENSOR
+ *               formats (for those the kernel multiplies the query by the K
+ *               scale of each channel and the output by the V scale of each
+ *               channel, since code * s_d factors out of both sums).
  * block_tables  device, [batch][max_blocks_per_seq] int32.
  * context_lens  device, [batch] int32: cached tokens per sequence, the token
  *               appended in this step included. 0 gives an all-zero output row.

@@ -60,12 +60,14 @@ template <int D, int G, int FMT>
 struct MmaCfg {
   static constexpr bool BF = FMT == KVQ_BF16;
   static constexpr bool F8 = FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2;   // either FP8 code
-  static constexpr bool I8 = FMT == KVQ_INT8_ASYM;
+  static constexpr bool SI = FMT == KVQ_INT8_CHANNEL;           // static per-channel / per-tensor scales
+  static constexpr bool I8 = FMT == KVQ_INT8_ASYM || SI;        // s8 codes
+  static constexpr bool ZP = FMT == KVQ_INT8_ASYM;              // per-token scale + zero point
   static constexpr int E = BF ? 2 : 1;                         // bytes per element
   static constexpr int KIND = BF ? 0 : (F8 ? 1 : 2);           // mma_ss kind
   static constexpr int PAGE = kBlockSize * D * E;              // bytes of one (block, head) page
   static constexpr int NST = 3;                                // ring stages
-  static constexpr int MV = F8 ? 1 : (I8 ? 2 : 0);
+  static constexpr int MV = F8 ? 1 : (ZP ? 2 : 0);            // per-token metadata values
   static constexpr int METAB = kBlockSize * MV * 2;            // scale bytes per page
   static constexpr int QPARTS = F8 ? 2 : (I8 ? 3 : 1);
   static constexpr int PPARTS = F8 ? 4 : 3;
@@ -206,7 +208,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
     const int32_t* __restrict__ ctx_lens, int B, int Hk, int NB, int W, int max_ctx,
-    int unit_tiles, int slots, float qk_scale, float* __restrict__ part_o,
+    int unit_tiles, int slots, float qk_scale, int per_tensor, float* __restrict__ part_o,
     float* __restrict__ part_ml, int32_t* __restrict__ part_cnt) {
   using C = MmaCfg<D, G, FMT>;
   using namespace tc;
@@ -552,6 +554,10 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     // query operand of a piece: the BF16 query rows of its group, loaded early
     // (qv) and written as exact parts later (store_q)
     float qv[C::HPW][D / 32];
+    // static INT8: K scale of channel lane + 32 i of the piece's KV head; the
+    // query is multiplied by it before the split, since sum_d q_d (s_d c_d) =
+    // sum_d (q_d s_d) c_d
+    [[maybe_unused]] float ksd[C::SI ? D / 32 : 1];
     auto load_q = [&](bool none, int qb, int qh) {
 #pragma unroll
       for (int hh = 0; hh < C::HPW; ++hh) {
@@ -562,6 +568,11 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
                           ? __bfloat162float(q[(int64_t(qb) * Hq + qh * G + g) * D + lane + 32 * i])
                           : 0.f;
       }
+      if constexpr (C::SI) {
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i)
+          ksd[i] = none ? 0.f : __bfloat162float(ks[per_tensor ? 0 : qh * D + lane + 32 * i]);
+      }
     };
     // B operand of S (K-major, no swizzle): row n = part * G + g, element
     // (n, d) at (n/8)*Q_SBO + (n%8)*16 + (d*E/16)*Q_LBO + (d*E)%16
@@ -570,6 +581,10 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       for (int hh = 0; hh < C::HPW; ++hh) {
         const int g = cw + 4 * hh;
         if (g >= G) continue;                                   // uniform per warp
+        if constexpr (C::SI) {
+#pragma unroll
+          for (int i = 0; i < D / 32; ++i) qv[hh][i] *= ksd[i];
+        }
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < D / 32; ++i) amax = fmaxf(amax, fabsf(qv[hh][i]));
@@ -615,7 +630,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
             isum += i0 * 16384 + i1 * 128 + i2;
           }
         }
-        if constexpr (C::I8) {
+        if constexpr (C::ZP) {
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
         }
@@ -719,13 +734,13 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           if constexpr (C::F8) {
             sk = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(kmeta + (s * 8 + p) * C::METAB)[t]);
             sv = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(vmeta + (s * 8 + p) * C::METAB)[t]);
-          } else if constexpr (C::I8) {
+          } else if constexpr (C::ZP) {
             const __nv_bfloat162 km = reinterpret_cast<const __nv_bfloat162*>(kmeta + (s * 8 + p) * C::METAB)[t];
             const __nv_bfloat162 vm = reinterpret_cast<const __nv_bfloat162*>(vmeta + (s * 8 + p) * C::METAB)[t];
             sk = __low2float(km); zk = __high2float(km);
             sv = __low2float(vm); zv = __high2float(vm);
           } else {
-            sv = 1.f;
+            sv = 1.f;                            // BF16 and static INT8: no per-token scales
           }
         }
         mbar_arrive(kempty + s);
@@ -739,7 +754,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
             sc = __uint_as_float(sw[g]) + __uint_as_float(sw[G + g]) * 0.0625f;
           } else if constexpr (C::I8) {
             sc = float(int(sw[g])) + float(int(sw[G + g])) * (1.f / 128.f) +
-                 float(int(sw[2 * G + g])) * (1.f / 16384.f) - zk * qz[g];
+                 float(int(sw[2 * G + g])) * (1.f / 16384.f);
+            if constexpr (C::ZP) sc -= zk * qz[g];
           } else {
             sc = __uint_as_float(sw[g]);
           }
@@ -853,13 +869,13 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           // 1, 1/256, 1/65536); zero_point * P is summed from the same Y
           uint32_t yv[G];
           const float ysc = sv * escale * 65536.f;
-          const float zsc = zv * einv * (1.f / 65536.f);
+          [[maybe_unused]] const float zsc = zv * einv * (1.f / 65536.f);
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
             l[g] = l[g] * alpha[g] + pr;
             yv[g] = __float2uint_rn(pr * ysc);
-            corr[g] = corr[g] * alpha[g] + float(yv[g]) * zsc;
+            if constexpr (C::ZP) corr[g] = corr[g] * alpha[g] + float(yv[g]) * zsc;
           }
           uint32_t words[C::NO / 4];
 #pragma unroll
@@ -940,20 +956,25 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float ls = warp_sum(l[g]);
-        const float cs = C::I8 ? warp_sum(corr[g]) : 0.f;
+        const float cs = C::ZP ? warp_sum(corr[g]) : 0.f;
         if (lane == 0) {
           red2[quarter * 8 + g] = ls;
           red2[32 + quarter * 8 + g] = cs;
         }
       }
       named_bar_sync(1, 128);
+      // static INT8: the V scale of channel r multiplies the finished sums
+      float vsd = 1.f;
+      if constexpr (C::SI) {
+        if (r < D) vsd = __bfloat162float(vs[per_tensor ? 0 : ph_ * D + r]);
+      }
       if (ok && !*abort_flag) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float L = red2[g] + red2[8 + g] + red2[16 + g] + red2[24 + g];
           const float Cz = red2[32 + g] + red2[40 + g] + red2[48 + g] + red2[56 + g];
           const int64_t row = (int64_t(pb) * Hq + ph_ * G + g) * slots + slot;
-          if (r < D) part_o[row * D + r] = o[g] - Cz;
+          if (r < D) part_o[row * D + r] = (o[g] - Cz) * vsd;
           if (r == 0) {
             part_ml[row * 2] = m[g];
             part_ml[row * 2 + 1] = L;

@@ -16,10 +16,11 @@ constexpr int kTileTokens = 128;   // partition_tokens granularity
 // Element bytes of the cache arrays and BF16 metadata values per (token, head).
 inline int elem_bytes(kvq_fmt f) { return f == KVQ_BF16 ? 2 : 1; }
 inline bool fmt_fp8(kvq_fmt f) { return f == KVQ_FP8_E4M3 || f == KVQ_FP8_E5M2; }
+// Per-token metadata values (0 for BF16 and the static-scale formats).
 inline int meta_values(kvq_fmt f) { return fmt_fp8(f) ? 1 : (f == KVQ_INT8_ASYM ? 2 : 0); }
-inline bool fmt_valid(int f) {
-  return f == KVQ_BF16 || f == KVQ_FP8_E4M3 || f == KVQ_INT8_ASYM || f == KVQ_FP8_E5M2;
-}
+// Static-scale INT8: one scale per (KV head, channel) or one per cache.
+inline bool fmt_static(kvq_fmt f) { return f == KVQ_INT8_CHANNEL || f == KVQ_INT8_TENSOR; }
+inline bool fmt_valid(int f) { return f >= KVQ_BF16 && f <= KVQ_INT8_TENSOR; }
 
 // Checks the shape rules of kvq.h. Returns KVQ_OK, KVQ_ERR_ARG or KVQ_ERR_UNSUPPORTED.
 int check_dims(const kvq_dims* d);

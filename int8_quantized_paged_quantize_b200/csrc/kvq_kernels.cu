@@ -226,6 +226,43 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
   }
 }
 
+// Static-scale INT8 (one given scale per channel, or one per cache): code =
+// clamp(rint(x / s), -127, 127), 0 where s <= 0 or s is NaN. s[i] and r[i] are
+// the scale of this lane's element i and its reciprocal RN(1/s), 0 when s is
+// below 2^-100 (those take the IEEE division). x is first clamped to
+// +-65536 s, which changes only quotients that saturate anyway and keeps the
+// corrected quotient inside the range where its rint equals that of the IEEE
+// quotient (tests/test_scale_division.py).
+template <int D>
+__device__ __forceinline__ void quantize_row_static(const uint32_t (&raw)[D / 64], const float (&sc)[D / 32],
+                                                    const float (&rc_)[D / 32], RowCodes<D, KVQ_INT8_CHANNEL>& rc) {
+  constexpr int E = D / 32;
+  rc.zp = 0;
+  rc.s = __float2bfloat16_rn(0.f);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const float x = (i & 1) ? bf16_hi(raw[i / 2]) : bf16_lo(raw[i / 2]);
+    const float s = sc[i], r = rc_[i];
+    int c = 0;
+    if (s > 0.f) {
+      const float lim = s * 65536.f;
+      const float xc = fminf(fmaxf(x, -lim), lim);
+      float q;
+      if (r != 0.f) {
+        const float q0 = __fmul_rn(xc, r);
+        const float e = __fmaf_rn(-q0, s, xc);
+        q = e != 0.f ? __fmaf_rn(e, r, q0) : q0;
+      } else {
+        q = __fdiv_rn(xc, s);
+      }
+      c = min(127, max(-127, __float2int_rn(fminf(fmaxf(q, -1024.f), 1024.f))));
+    }
+    packed |= uint32_t(uint8_t(int8_t(c))) << (8 * i);
+  }
+  rc.w[0] = packed;
+}
+
 // Bytes [p, e) of the 16-byte chunk at dst (16-byte aligned) from w, with the
 // widest aligned stores the range allows: one 16-byte store for a whole chunk,
 // else 8-, 4-, 2- and 1-byte pieces. Bytes outside [p, e) are not touched, so
@@ -282,12 +319,14 @@ __device__ __forceinline__ void store_bytes16(uint8_t* dst, const uint32_t (&w)[
 //     stores that range allows. A page continued from an offset (chunked
 //     prefill) thus costs one partial chunk per channel, not one byte store per
 //     token and channel.
-// Register use is capped at 32 so that 8 CTAs (64 warps) fit on an SM.
+// Register use is capped at 32 so that 8 CTAs (64 warps) fit on an SM (40 and
+// 6 CTAs for the static-scale format, which keeps its channels' scales).
 template <int D, int FMT>
-__global__ void __launch_bounds__(256, 8)
+__global__ void __launch_bounds__(256, FMT == KVQ_INT8_CHANNEL ? 6 : 8)
 append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
               const int64_t* __restrict__ slots, int T, int Hk, int NB, uint8_t* __restrict__ kc,
-              uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs) {
+              uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs,
+              int per_tensor) {
   using RC = RowCodes<D, FMT>;
   constexpr int E = RC::E, ELT = RC::ELT;
   constexpr int ROWB = D * ELT;                 // bytes of one token row
@@ -350,6 +389,17 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
     }
   }
 
+  // static scales: a warp's rows are all K (even warps) or all V (odd warps),
+  // so a lane's channels keep their scales for every row it quantizes
+  [[maybe_unused]] float ssc[E], rsc[E];
+  if constexpr (FMT == KVQ_INT8_CHANNEL) {
+    const __nv_bfloat16* sarr = (warp & 1) ? vs : ks;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      ssc[e] = __bfloat162float(sarr[per_tensor ? 0 : h * D + d0 + e]);
+      rsc[e] = ssc[e] >= 7.88860905e-31f ? __frcp_rn(ssc[e]) : 0.f;   // 2^-100
+    }
+  }
 #pragma unroll
   for (int j = 0; j < RPW; ++j) {
     const int rr = warp + 8 * j;
@@ -362,7 +412,8 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
       continue;
     }
     RC rc;
-    quantize_row<D, FMT>(raws[j], rc);
+    if constexpr (FMT == KVQ_INT8_CHANNEL) quantize_row_static<D>(raws[j], ssc, rsc, rc);
+    else quantize_row<D, FMT>(raws[j], rc);
     uint8_t* dst = (which ? vbuf : kbuf) + i * PADB + d0 * ELT;
     if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
     else if constexpr (E * ELT == 4) *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
@@ -773,12 +824,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D, int FMT>
 cudaError_t append_dispatch(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
-                            void* vc, void* ks, void* vs, const kvq_dims& d, cudaStream_t st) {
+                            void* vc, void* ks, void* vs, const kvq_dims& d, int per_tensor,
+                            cudaStream_t st) {
   const dim3 grid(unsigned((int64_t(T) + kBlockSize - 1) / kBlockSize), unsigned(d.n_kv_heads));
   append_kernel<D, FMT><<<grid, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), slots, T,
       d.n_kv_heads, d.num_blocks, static_cast<uint8_t*>(kc), static_cast<uint8_t*>(vc),
-      static_cast<__nv_bfloat16*>(ks), static_cast<__nv_bfloat16*>(vs));
+      static_cast<__nv_bfloat16*>(ks), static_cast<__nv_bfloat16*>(vs), per_tensor);
   return cudaGetLastError();
 }
 
@@ -786,7 +838,7 @@ template <int D, int G, int FMT>
 cudaError_t decode_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
                              const void* ks, const void* vs, const int32_t* tables,
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
-                             const DecodePlan& plan, void* ws, const kvq_dims& d,
+                             const DecodePlan& plan, void* ws, const kvq_dims& d, int,
                              cudaStream_t st) {
   float* po = static_cast<float*>(ws);
   float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
@@ -805,7 +857,7 @@ template <int D, int G, int FMT>
 cudaError_t decode_tc_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
                                 const void* ks, const void* vs, const int32_t* tables,
                                 const int32_t* ctx, int32_t max_ctx, float sm_scale,
-                                const DecodePlan& plan, void* ws, const kvq_dims& d,
+                                const DecodePlan& plan, void* ws, const kvq_dims& d, int,
                                 cudaStream_t st) {
   using C = TcCfg<D, FMT>;
   auto kern = decode_tc_kernel<D, G, FMT>;
@@ -829,7 +881,7 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
                                  const void* ks, const void* vs, const int32_t* tables,
                                  const int32_t* ctx, int32_t max_ctx, float sm_scale,
                                  const DecodePlan& plan, void* ws, const kvq_dims& d,
-                                 cudaStream_t st) {
+                                 int per_tensor, cudaStream_t st) {
   using C = MmaCfg<D, G, FMT>;
   auto kern = decode_mma_kernel<D, G, FMT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -855,7 +907,7 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
       static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, d.num_blocks,
       d.max_blocks_per_seq, max_ctx, plan.partition / kTileTokens, plan.slots, sm_scale * kLog2e,
-      po, pml, pcnt);
+      per_tensor, po, pml, pcnt);
   return cudaGetLastError();
 }
 
@@ -877,17 +929,18 @@ template <int D, int FMT>
 cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, const void* vc,
                              const void* ks, const void* vs, const int32_t* tables,
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
-                             const DecodePlan& plan, void* ws, const kvq_dims& d,
+                             const DecodePlan& plan, void* ws, const kvq_dims& d, int per_tensor,
                              cudaStream_t st) {
 #define KVQ_G_SWITCH(DISPATCH)                                                                   \
   switch (G) {                                                                                   \
-    case 1: return DISPATCH<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st); \
-    case 2: return DISPATCH<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st); \
-    case 4: return DISPATCH<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st); \
-    default: return DISPATCH<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st); \
+    case 1: return DISPATCH<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, st); \
+    case 2: return DISPATCH<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, st); \
+    case 4: return DISPATCH<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, st); \
+    default: return DISPATCH<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, st); \
   }
-  if constexpr (FMT == KVQ_FP8_E5M2) {
-    // E5M2 exists only in the tensor-core kernel that multiplies the codes
+  if constexpr (FMT == KVQ_FP8_E5M2 || FMT == KVQ_INT8_CHANNEL) {
+    // E5M2 and the static-scale INT8 formats exist only in the tensor-core
+    // kernel that multiplies the codes
     KVQ_G_SWITCH(decode_mma_dispatch3)
   } else {
     if (decode_kernel_choice() == 0) { KVQ_G_SWITCH(decode_mma_dispatch3) }
@@ -901,18 +954,23 @@ cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, co
 int launch_append(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
                   void* vc, void* ks, void* vs, kvq_fmt fmt, const kvq_dims& d, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int pt = fmt == KVQ_INT8_TENSOR;
   cudaError_t e;
+#define KVQ_APP(DD, FF) append_dispatch<DD, FF>(k, v, slots, T, kc, vc, ks, vs, d, pt, st)
   if (d.head_dim == 128) {
-    if (fmt == KVQ_FP8_E4M3) e = append_dispatch<128, KVQ_FP8_E4M3>(k, v, slots, T, kc, vc, ks, vs, d, st);
-    else if (fmt == KVQ_FP8_E5M2) e = append_dispatch<128, KVQ_FP8_E5M2>(k, v, slots, T, kc, vc, ks, vs, d, st);
-    else if (fmt == KVQ_INT8_ASYM) e = append_dispatch<128, KVQ_INT8_ASYM>(k, v, slots, T, kc, vc, ks, vs, d, st);
-    else e = append_dispatch<128, KVQ_BF16>(k, v, slots, T, kc, vc, ks, vs, d, st);
+    if (fmt == KVQ_FP8_E4M3) e = KVQ_APP(128, KVQ_FP8_E4M3);
+    else if (fmt == KVQ_FP8_E5M2) e = KVQ_APP(128, KVQ_FP8_E5M2);
+    else if (fmt == KVQ_INT8_ASYM) e = KVQ_APP(128, KVQ_INT8_ASYM);
+    else if (fmt_static(fmt)) e = KVQ_APP(128, KVQ_INT8_CHANNEL);
+    else e = KVQ_APP(128, KVQ_BF16);
   } else {
-    if (fmt == KVQ_FP8_E4M3) e = append_dispatch<64, KVQ_FP8_E4M3>(k, v, slots, T, kc, vc, ks, vs, d, st);
-    else if (fmt == KVQ_FP8_E5M2) e = append_dispatch<64, KVQ_FP8_E5M2>(k, v, slots, T, kc, vc, ks, vs, d, st);
-    else if (fmt == KVQ_INT8_ASYM) e = append_dispatch<64, KVQ_INT8_ASYM>(k, v, slots, T, kc, vc, ks, vs, d, st);
-    else e = append_dispatch<64, KVQ_BF16>(k, v, slots, T, kc, vc, ks, vs, d, st);
+    if (fmt == KVQ_FP8_E4M3) e = KVQ_APP(64, KVQ_FP8_E4M3);
+    else if (fmt == KVQ_FP8_E5M2) e = KVQ_APP(64, KVQ_FP8_E5M2);
+    else if (fmt == KVQ_INT8_ASYM) e = KVQ_APP(64, KVQ_INT8_ASYM);
+    else if (fmt_static(fmt)) e = KVQ_APP(64, KVQ_INT8_CHANNEL);
+    else e = KVQ_APP(64, KVQ_BF16);
   }
+#undef KVQ_APP
   return int(e);
 }
 
@@ -924,16 +982,19 @@ int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int G = d.n_q_heads / d.n_kv_heads;
   cudaError_t e;
-#define KVQ_DEC(DD, FF) decode_dispatch2<DD, FF>(G, q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, st)
+#define KVQ_DEC(DD, FF) decode_dispatch2<DD, FF>(G, q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, pt, st)
+  const int pt = fmt == KVQ_INT8_TENSOR;
   if (d.head_dim == 128) {
     if (fmt == KVQ_FP8_E4M3) e = KVQ_DEC(128, KVQ_FP8_E4M3);
     else if (fmt == KVQ_FP8_E5M2) e = KVQ_DEC(128, KVQ_FP8_E5M2);
     else if (fmt == KVQ_INT8_ASYM) e = KVQ_DEC(128, KVQ_INT8_ASYM);
+    else if (fmt_static(fmt)) e = KVQ_DEC(128, KVQ_INT8_CHANNEL);
     else e = KVQ_DEC(128, KVQ_BF16);
   } else {
     if (fmt == KVQ_FP8_E4M3) e = KVQ_DEC(64, KVQ_FP8_E4M3);
     else if (fmt == KVQ_FP8_E5M2) e = KVQ_DEC(64, KVQ_FP8_E5M2);
     else if (fmt == KVQ_INT8_ASYM) e = KVQ_DEC(64, KVQ_INT8_ASYM);
+    else if (fmt_static(fmt)) e = KVQ_DEC(64, KVQ_INT8_CHANNEL);
     else e = KVQ_DEC(64, KVQ_BF16);
   }
 #undef KVQ_DEC

@@ -50,7 +50,12 @@ int kvq_cache_bytes(const kvq_dims* dims, kvq_fmt fmt, size_t* cache_bytes, size
   if (rc != KVQ_OK) return rc;
   const size_t rows = size_t(dims->num_blocks) * dims->n_kv_heads * dims->block_size;
   *cache_bytes = rows * dims->head_dim * kvq::elem_bytes(fmt);
-  *meta_bytes = rows * kvq::meta_values(fmt) * 2;
+  if (fmt == KVQ_INT8_CHANNEL)
+    *meta_bytes = size_t(dims->n_kv_heads) * dims->head_dim * 2;
+  else if (fmt == KVQ_INT8_TENSOR)
+    *meta_bytes = 16;                 // one BF16 value, padded to the 16-byte alignment
+  else
+    *meta_bytes = rows * kvq::meta_values(fmt) * 2;
   return KVQ_OK;
 }
 

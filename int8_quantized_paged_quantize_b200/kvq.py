@@ -17,9 +17,12 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
 
-FMT = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 3}
-ELEM_BYTES = {"bf16": 2, "fp8": 1, "int8": 1, "e5m2": 1}
-META_VALUES = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 1}
+# int8c / int8t: symmetric INT8 with static BF16 scales given by the caller,
+# one per (KV head, channel) or one per cache (K and V separately)
+FMT = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 3, "int8c": 4, "int8t": 5}
+ELEM_BYTES = {"bf16": 2, "fp8": 1, "int8": 1, "e5m2": 1, "int8c": 1, "int8t": 1}
+META_VALUES = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 1, "int8c": 0, "int8t": 0}   # per token
+STATIC_FORMATS = ("int8c", "int8t")
 BLOCK_SIZE = 16
 
 DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
@@ -277,15 +280,24 @@ class LayerCache:
     v_scale: torch.Tensor | None
 
     @staticmethod
-    def allocate(fmt, d: Dims, device="cuda"):
-        """Zeroed K/V caches and scales in the library's page layout (include/kvq.h)."""
+    def allocate(fmt, d: Dims, device="cuda", k_static=None, v_static=None):
+        """Zeroed K/V caches and scales in the library's page layout (include/kvq.h).
+        The static formats take their scales here: BF16 [Hk][D] (int8c) or [1]
+        (int8t) tensors, kept by reference."""
         nb, hk, D = d.num_blocks, d.n_kv_heads, d.head_dim
         E = ELEM_BYTES[fmt]
         edt = torch.bfloat16 if fmt == "bf16" else torch.uint8
         k = torch.zeros((nb, hk, 2, D * E // 16, 8, 16 // E), dtype=edt, device=device)
         v = torch.zeros((nb, hk, E, D, 16 // E), dtype=edt, device=device)
         mv = META_VALUES[fmt]
-        if mv:
+        if fmt in STATIC_FORMATS:
+            shape = (hk, D) if fmt == "int8c" else (1,)
+            for name, t in (("k_static", k_static), ("v_static", v_static)):
+                if t is None or tuple(t.shape) != shape:
+                    raise KvqError(f"{fmt} needs {name} of shape {shape}")
+                _need(t, torch.bfloat16, name)
+            ks, vs = k_static, v_static
+        elif mv:
             shape = (nb, hk, BLOCK_SIZE) if mv == 1 else (nb, hk, BLOCK_SIZE, 2)
             ks = torch.zeros(shape, dtype=torch.bfloat16, device=device)
             vs = torch.zeros(shape, dtype=torch.bfloat16, device=device)

@@ -38,6 +38,8 @@ class GpuRun:
     v_new: torch.Tensor
     out: torch.Tensor           # [B][Hq][D] (CPU, dtype of the run)
     seed: int = 0
+    k_static: np.ndarray | None = None   # static INT8 scales (int8c [Hk][D], int8t [1])
+    v_static: np.ndarray | None = None
 
 
 def slots_for(tables, b, positions, bs=16):
@@ -52,6 +54,19 @@ def with_lengths(w: W.Workload, ctx_list):
 
 
 _INPUTS = {}
+STATIC = ("int8c", "int8t")
+
+
+def static_scales(w: W.Workload, fmt: str, seed=0):
+    """Static INT8 scales for a run, fixed by the oracle's calibration rule from
+    the workload's cached history (the sample a caller would calibrate on)."""
+    hist, _, (_, k_new, v_new) = inputs(w, seed)
+    ks = [h[0] for h in hist] + [k_new]
+    vs = [h[1] for h in hist] + [v_new]
+    K = torch.cat(ks).float().numpy()
+    V = torch.cat(vs).float().numpy()
+    per_channel = fmt == "int8c"
+    return OF.int8_static_calibrate(K, per_channel), OF.int8_static_calibrate(V, per_channel)
 
 
 def inputs(w: W.Workload, seed=0):
@@ -67,7 +82,7 @@ def inputs(w: W.Workload, seed=0):
 
 
 def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch.float32,
-            history_chunks=1):
+            history_chunks=1, static=None):
     """Append every sequence's cached history (in `history_chunks` calls), then the
     bulk append if the workload has one, then one token per sequence, and run one
     decode step over ctx + 1 tokens. Returns a GpuRun."""
@@ -75,8 +90,16 @@ def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch
     ctx = W.context_lengths(w, seed)
     hist, bulk, (q, k_new, v_new) = inputs(w, seed)
     d = kvq.dims(nb, w.n_kv_heads, w.n_q_heads, w.head_dim, tables.shape[1])
-    cache = kvq.LayerCache.allocate(fmt, d)
     dev = torch.device("cuda")
+    kst = vst = None
+    if fmt in STATIC:
+        kst, vst = static if static is not None else static_scales(w, fmt, seed)
+        kst = np.asarray(kst, dtype=np.float32)
+        vst = np.asarray(vst, dtype=np.float32)
+        cache = kvq.LayerCache.allocate(fmt, d, k_static=torch.from_numpy(kst).to(torch.bfloat16).to(dev),
+                                        v_static=torch.from_numpy(vst).to(torch.bfloat16).to(dev))
+    else:
+        cache = kvq.LayerCache.allocate(fmt, d)
     S = [torch.from_numpy(slots_for(tables, b, np.arange(ctx[b]))) for b in range(w.batch)]
     S = torch.cat(S) if S else torch.zeros(0, dtype=torch.int64)
     n = S.numel()
@@ -107,7 +130,7 @@ def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch
                        partition_tokens=partition_tokens, out_dtype=out_dtype)
     torch.cuda.synchronize()
     assert kvq.device_error(clear=True) == 0
-    return GpuRun(w, fmt, cache, tables, ctx, ctx_after, q, k_new, v_new, out.cpu(), seed)
+    return GpuRun(w, fmt, cache, tables, ctx, ctx_after, q, k_new, v_new, out.cpu(), seed, kst, vst)
 
 
 # ----------------------------------------------------------------------------- oracle side
@@ -135,6 +158,11 @@ def oracle_sequence(run: GpuRun, b: int):
             c, s = OF.e5m2_quantize(x)
             res[name + "_codes"], res[name + "_scale"] = c, s
             res[name.upper()] = OF.e5m2_dequantize(c, s)
+        elif run.fmt in STATIC:
+            st = run.k_static if name == "k" else run.v_static
+            c = OF.int8_static_quantize(x, st)
+            res[name + "_codes"] = c
+            res[name.upper()] = OF.int8_static_dequantize(c, st)
         elif run.fmt == "int8":
             c, s, z = OF.int8_quantize(x)
             res[name + "_codes"], res[name + "_scale"], res[name + "_zp"] = c, s, z
@@ -156,7 +184,7 @@ def gpu_sequence(run: GpuRun, b: int):
     kl = kl.permute(0, 2, 1, 3).reshape(pages * 16, kl.shape[1], kl.shape[3])[:n].cpu()
     vl = vl.permute(0, 2, 1, 3).reshape(pages * 16, vl.shape[1], vl.shape[3])[:n].cpu()
     out = {"k_codes": kl, "v_codes": vl}
-    if run.fmt != "bf16":
+    if run.fmt not in ("bf16",) + STATIC:
         for name, t in (("k", run.cache.k_scale), ("v", run.cache.v_scale)):
             m = t[ids]                                       # [pages][Hk][16](,2)
             if run.fmt in ("fp8", "e5m2"):
@@ -179,7 +207,7 @@ def assert_codes_equal(run: GpuRun, b: int, ref: dict):
             assert np.array_equal(gc.numpy(), ref[name + "_codes"]), f"{name} codes b={b}"
         else:
             assert np.array_equal(gc.numpy().view(np.int8), ref[name + "_codes"]), f"{name} codes b={b}"
-        if run.fmt != "bf16":
+        if run.fmt not in ("bf16",) + STATIC:
             assert np.array_equal(OF.bf16_bits(g[name + "_scale"]), OF.bf16_bits(ref[name + "_scale"])), \
                 f"{name} scales b={b}"
         if run.fmt == "int8":

@@ -50,6 +50,10 @@ def test_cache_bytes(kvq):
     assert kvq.cache_bytes(d, "fp8") == (100 * 8 * 16 * 128, 100 * 8 * 16 * 2)
     assert kvq.cache_bytes(d, "int8") == (100 * 8 * 16 * 128, 100 * 8 * 16 * 4)
     assert kvq.cache_bytes(d, "bf16") == (100 * 8 * 16 * 128 * 2, 0)
+    assert kvq.cache_bytes(d, "e5m2") == (100 * 8 * 16 * 128, 100 * 8 * 16 * 2)
+    # static INT8: the scales do not grow with the tokens
+    assert kvq.cache_bytes(d, "int8c") == (100 * 8 * 16 * 128, 8 * 128 * 2)
+    assert kvq.cache_bytes(d, "int8t") == (100 * 8 * 16 * 128, 16)
 
 
 def test_allocator_reproduces_printed_sizes(kvq):
