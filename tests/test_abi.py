@@ -125,6 +125,13 @@ def test_host_checks_need_no_gpu(kvq):
     assert L.kvq_append(fake, fake, fake, 4, fake, fake, fake, fake, 1, ctypes.byref(bad), None) == -2
     assert L.kvq_append(fake, fake, fake, 4, fake, fake, None, fake, 1, ctypes.byref(d), None) == -1
     assert L.kvq_append(fake, fake, fake, 0, None, None, None, None, 1, ctypes.byref(d), None) == 0
+    # the static INT8 formats need their scale arrays too; an unknown format is refused
+    for fmt in (4, 5):
+        assert L.kvq_append(fake, fake, fake, 4, fake, fake, fake, None, fmt, ctypes.byref(d), None) == -1
+        none = (ctypes.c_void_p * 2)(1 << 21, 0)
+        assert L.kvq_decode_attn(fake, 1, fake, fake, none, fake, fake, 100, ctypes.c_float(0.1), fake,
+                                 0, fake, 1 << 30, 0, fmt, ctypes.byref(d), None) == -1
+    assert L.kvq_append(fake, fake, fake, 4, fake, fake, fake, fake, 6, ctypes.byref(d), None) == -1
     # max_context_len beyond what the block table can hold
     assert kvq.lib().kvq_decode_workspace_bytes(1, 8 * 16 + 1, 0, 1, ctypes.byref(d)) == 0
     # partition must be a multiple of 128
