@@ -26,6 +26,12 @@ Readings taken
   the reference both for a quantised cache (fed the dequantised values) and for
   the unquantised BF16 values (the quality number).
 * A sequence with ctx == 0 has an all-zero output (nothing to attend).
+* Multi-query decode ([LIMITS] "How it interacts with speculative decoding":
+  the target model scores the K+1 proposed positions in one pass over the
+  quantised cache). Read as: the n_query new tokens are already appended, and
+  position j (0-based) sees the cached tokens before it and itself, i.e. the
+  first ``ctx - n_query + 1 + j`` positions (causal within the new tokens). A
+  position that sees no token has an all-zero output.
 """
 
 from __future__ import annotations
@@ -70,3 +76,25 @@ def softmax_weights(q, k, sm_scale):
     scores = (np.asarray(k, dtype=np.float64) @ np.asarray(q, dtype=np.float64)) * float(sm_scale)
     w = np.exp(scores - scores.max())
     return w / w.sum()
+
+
+def verify_attention(q, kv_per_seq, sm_scale, n_kv_heads):
+    """Multi-query outputs [B][Hq][n_query][D] float64.
+
+    q: [B][Hq][n_query][D]; kv_per_seq: list of (K, V), each [ctx_b][n_kv_heads][D]
+    with the n_query new tokens as its last positions. Position j of sequence b
+    attends to the first ctx_b - n_query + 1 + j positions."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, nq, D = q.shape
+    G = Hq // n_kv_heads
+    out = np.zeros((B, Hq, nq, D), dtype=np.float64)
+    for b in range(B):
+        K, V = kv_per_seq[b]
+        ctx = K.shape[0]
+        for h in range(Hq):
+            kh = h // G
+            for j in range(nq):
+                n = max(0, ctx - nq + 1 + j)
+                out[b, h, j] = attend_one(q[b, h, j], K[:n, kh, :], V[:n, kh, :], sm_scale)
+    return out
+
