@@ -315,6 +315,42 @@ int kvq_decode_attn_noalloc(const void* q, int32_t batch, const void* k_cache,
                             const kvq_dims* dims, kvq_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Multi-query decode (speculative verification).                              */
+/* [LIMITS] "How it interacts with speculative decoding": the target model     */
+/* scores all K+1 proposed positions in one pass that reads the quantized     */
+/* cache and dequantizes it on the fly.                                        */
+/* ------------------------------------------------------------------------ */
+/*
+ * Each sequence b has n_query new positions: the last n_query tokens of its
+ * context, already appended (context_lens[b] counts them). Position j
+ * (0 <= j < n_query) attends causally to tokens 0 .. context_lens[b] -
+ * n_query + j, i.e. to everything before it and to itself:
+ *   out[b][h][j] = softmax_t(sm_scale * q[b][h][j] . K_b[t][h/G]) weighted sum
+ *                  of V_b[t][h/G] over t < context_lens[b] - n_query + 1 + j.
+ * A position with no visible token gives an all-zero row.
+ *
+ * q    device, [batch][n_q_heads][n_query][head_dim] BF16.
+ * out  device, [batch][n_q_heads][n_query][head_dim], BF16 or FP32 per out_dtype.
+ * The cache, scales, block tables and the other arguments are those of
+ * kvq_decode_attn. The K/V of a (sequence, KV head) are read once for all
+ * n_query positions of all G query heads: the positions are extra heads of
+ * the GQA group. Supported when G * n_query is 1, 2, 4 or 8
+ * (KVQ_ERR_UNSUPPORTED otherwise; n_query outside 1..8 is KVQ_ERR_ARG).
+ * workspace  at least kvq_decode_verify_workspace_bytes(...) bytes; contents on
+ *            entry do not matter.
+ */
+size_t kvq_decode_verify_workspace_bytes(int32_t batch, int32_t n_query, int32_t max_context_len,
+                                         int32_t partition_tokens, kvq_fmt fmt,
+                                         const kvq_dims* dims);
+int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void* k_cache,
+                      const void* v_cache, const void* const* scales,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      int32_t max_context_len, float sm_scale, void* out,
+                      kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                      int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                      kvq_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Device error word.                                                          */
 /* ------------------------------------------------------------------------ */
 /* Read (and if `clear` is non-zero, reset) the current device's error word

@@ -190,4 +190,55 @@ int kvq_device_error(uint32_t* flags, int clear) {
   return *flags ? KVQ_ERR_DEVICE : KVQ_OK;
 }
 
+// Multi-query decode: the n_query positions of a query head are the heads
+// n_query * h .. n_query * h + n_query - 1 of a group n_query times larger, so
+// the single-query machinery runs on dims with n_q_heads * n_query query heads
+// and the kernel adds the causal limit of each position.
+namespace {
+int verify_dims(int32_t n_query, const kvq_dims* dims, kvq_dims* eff) {
+  if (!dims || n_query < 1 || n_query > 8) return KVQ_ERR_ARG;
+  *eff = *dims;
+  eff->n_q_heads = dims->n_q_heads * n_query;
+  return KVQ_OK;
+}
+}  // namespace
+
+size_t kvq_decode_verify_workspace_bytes(int32_t batch, int32_t n_query, int32_t max_context_len,
+                                         int32_t partition_tokens, kvq_fmt fmt,
+                                         const kvq_dims* dims) {
+  kvq_dims eff;
+  if (verify_dims(n_query, dims, &eff) != KVQ_OK) return 0;
+  return kvq_decode_workspace_bytes(batch, max_context_len, partition_tokens, fmt, &eff);
+}
+
+int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void* k_cache,
+                      const void* v_cache, const void* const* scales,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      int32_t max_context_len, float sm_scale, void* out,
+                      kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                      int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                      kvq_stream_t stream) {
+  kvq_dims eff;
+  int rc = verify_dims(n_query, dims, &eff);
+  if (rc != KVQ_OK) return rc;
+  DecodePlan plan;
+  rc = check_decode_common(batch, max_context_len, partition_tokens, fmt, &eff, &plan);
+  if (rc != KVQ_OK) return rc;                 // includes G * n_query outside {1, 2, 4, 8}
+  if (out_dtype != KVQ_OUT_BF16 && out_dtype != KVQ_OUT_F32) return KVQ_ERR_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!dev_ok(out)) return KVQ_ERR_ARG;
+  const void *ks, *vs;
+  rc = check_decode_inputs(q, k_cache, v_cache, scales, block_tables, context_lens, sm_scale, fmt,
+                           &ks, &vs);
+  if (rc != KVQ_OK) return rc;
+  if (!dev_ok(workspace)) return KVQ_ERR_ARG;
+  if (workspace_bytes < plan.total) return KVQ_ERR_WORKSPACE;
+  rc = cuda_rc(launch_decode_partial(q, batch, k_cache, v_cache, ks, vs, block_tables, context_lens,
+                                     max_context_len, sm_scale, plan, workspace, fmt, eff, stream,
+                                     n_query));
+  if (rc != KVQ_OK) return rc;
+  return cuda_rc(launch_decode_merge(batch, context_lens, max_context_len, out,
+                                     out_dtype == KVQ_OUT_F32, workspace, plan, eff, stream));
+}
+
 }  // extern "C"

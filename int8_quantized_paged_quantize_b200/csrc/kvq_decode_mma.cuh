@@ -208,7 +208,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
     const int32_t* __restrict__ ctx_lens, int B, int Hk, int NB, int W, int max_ctx,
-    int unit_tiles, int slots, float qk_scale, int per_tensor, float* __restrict__ part_o,
+    int unit_tiles, int slots, float qk_scale, int per_tensor, int n_query,
+    float* __restrict__ part_o,
     float* __restrict__ part_ml, int32_t* __restrict__ part_cnt) {
   using C = MmaCfg<D, G, FMT>;
   using namespace tc;
@@ -655,6 +656,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       if (cur->done) break;                              // uniform
       const int pb = cur->b, ph_ = cur->h, lo = cur->lo, hi = cur->hi;
       const int t1 = min(hi * 128, cur->ctx);
+      const int pctx = cur->ctx;
       const int slot = pinfo[(pc & 1) * 2], last = pinfo[(pc & 1) * 2 + 1];
       const bool more = !nxt->done;
       load_q(!more, nxt->b, nxt->h);                     // next piece's query, in flight
@@ -761,6 +763,15 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           }
           x[g] = valid ? sc * sk * qs[g] : -INFINITY;
         }
+        if (n_query > 1) {
+          // multi-query: head g is query position j = g % n_query of its
+          // group's head g / n_query, and position j sees the tokens before
+          // the last n_query - 1 - j of the context
+          const int after = pctx - 1 - (tile0 + r);       // tokens after this one
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            if (n_query - 1 - g % n_query > after) x[g] = -INFINITY;
+        }
         // per-head tile maxima of the four warps, head-major: rb[g][quarter]
         float* rb = red + (gt & 1) * 64;
 #pragma unroll
@@ -836,7 +847,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           float y[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+            const float pr = x[g] != -INFINITY ? exp2f(x[g] - m[g]) : 0.f;
             l[g] = l[g] * alpha[g] + pr;
             y[g] = pr * sv * escale;
           }
@@ -872,7 +883,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           [[maybe_unused]] const float zsc = zv * einv * (1.f / 65536.f);
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+            const float pr = x[g] != -INFINITY ? exp2f(x[g] - m[g]) : 0.f;
             l[g] = l[g] * alpha[g] + pr;
             yv[g] = __float2uint_rn(pr * ysc);
             if constexpr (C::ZP) corr[g] = corr[g] * alpha[g] + float(yv[g]) * zsc;
@@ -913,7 +924,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           for (int e = 0; e < C::NO / 2; ++e) words[e] = 0u;
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float pr = valid ? exp2f(x[g] - m[g]) : 0.f;
+            const float pr = x[g] != -INFINITY ? exp2f(x[g] - m[g]) : 0.f;
             l[g] = l[g] * alpha[g] + pr;
             const __nv_bfloat16 hi = __float2bfloat16_rn(pr);
             const float r1 = pr - __bfloat162float(hi);

@@ -51,7 +51,7 @@ int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* 
                           const void* ks, const void* vs, const int32_t* tables,
                           const int32_t* ctx, int32_t max_ctx, float sm_scale,
                           const DecodePlan& plan, void* ws, kvq_fmt fmt, const kvq_dims& d,
-                          void* stream);
+                          void* stream, int n_query = 1);
 int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* out, bool out_f32,
                         const void* ws, const DecodePlan& plan, const kvq_dims& d, void* stream);
 int read_device_error(uint32_t* flags, int clear);

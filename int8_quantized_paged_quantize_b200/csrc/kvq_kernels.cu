@@ -838,7 +838,7 @@ template <int D, int G, int FMT>
 cudaError_t decode_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
                              const void* ks, const void* vs, const int32_t* tables,
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
-                             const DecodePlan& plan, void* ws, const kvq_dims& d, int,
+                             const DecodePlan& plan, void* ws, const kvq_dims& d, int, int,
                              cudaStream_t st) {
   float* po = static_cast<float*>(ws);
   float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
@@ -857,7 +857,7 @@ template <int D, int G, int FMT>
 cudaError_t decode_tc_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
                                 const void* ks, const void* vs, const int32_t* tables,
                                 const int32_t* ctx, int32_t max_ctx, float sm_scale,
-                                const DecodePlan& plan, void* ws, const kvq_dims& d, int,
+                                const DecodePlan& plan, void* ws, const kvq_dims& d, int, int,
                                 cudaStream_t st) {
   using C = TcCfg<D, FMT>;
   auto kern = decode_tc_kernel<D, G, FMT>;
@@ -881,7 +881,7 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
                                  const void* ks, const void* vs, const int32_t* tables,
                                  const int32_t* ctx, int32_t max_ctx, float sm_scale,
                                  const DecodePlan& plan, void* ws, const kvq_dims& d,
-                                 int per_tensor, cudaStream_t st) {
+                                 int per_tensor, int n_query, cudaStream_t st) {
   using C = MmaCfg<D, G, FMT>;
   auto kern = decode_mma_kernel<D, G, FMT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -907,7 +907,7 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
       static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, d.num_blocks,
       d.max_blocks_per_seq, max_ctx, plan.partition / kTileTokens, plan.slots, sm_scale * kLog2e,
-      per_tensor, po, pml, pcnt);
+      per_tensor, n_query, po, pml, pcnt);
   return cudaGetLastError();
 }
 
@@ -930,20 +930,21 @@ cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, co
                              const void* ks, const void* vs, const int32_t* tables,
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
                              const DecodePlan& plan, void* ws, const kvq_dims& d, int per_tensor,
-                             cudaStream_t st) {
+                             int n_query, cudaStream_t st) {
 #define KVQ_G_SWITCH(DISPATCH)                                                                   \
   switch (G) {                                                                                   \
-    case 1: return DISPATCH<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, st); \
-    case 2: return DISPATCH<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, st); \
-    case 4: return DISPATCH<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, st); \
-    default: return DISPATCH<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, st); \
+    case 1: return DISPATCH<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st); \
+    case 2: return DISPATCH<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st); \
+    case 4: return DISPATCH<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st); \
+    default: return DISPATCH<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st); \
   }
   if constexpr (FMT == KVQ_FP8_E5M2 || FMT == KVQ_INT8_CHANNEL) {
     // E5M2 and the static-scale INT8 formats exist only in the tensor-core
     // kernel that multiplies the codes
     KVQ_G_SWITCH(decode_mma_dispatch3)
   } else {
-    if (decode_kernel_choice() == 0) { KVQ_G_SWITCH(decode_mma_dispatch3) }
+    // so does multi-query decode
+    if (decode_kernel_choice() == 0 || n_query > 1) { KVQ_G_SWITCH(decode_mma_dispatch3) }
     if (decode_kernel_choice() == 1) { KVQ_G_SWITCH(decode_tc_dispatch3) }
     KVQ_G_SWITCH(decode_dispatch3)
   }
@@ -978,11 +979,11 @@ int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* 
                           const void* ks, const void* vs, const int32_t* tables,
                           const int32_t* ctx, int32_t max_ctx, float sm_scale,
                           const DecodePlan& plan, void* ws, kvq_fmt fmt, const kvq_dims& d,
-                          void* stream) {
+                          void* stream, int n_query) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int G = d.n_q_heads / d.n_kv_heads;
   cudaError_t e;
-#define KVQ_DEC(DD, FF) decode_dispatch2<DD, FF>(G, q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, pt, st)
+#define KVQ_DEC(DD, FF) decode_dispatch2<DD, FF>(G, q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, pt, n_query, st)
   const int pt = fmt == KVQ_INT8_TENSOR;
   if (d.head_dim == 128) {
     if (fmt == KVQ_FP8_E4M3) e = KVQ_DEC(128, KVQ_FP8_E4M3);

@@ -53,6 +53,11 @@ _SIGNATURES = [
     ("kvq_decode_attn_noalloc", _c.c_int, [_P, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32,
                                            _c.c_float, _P, _c.c_int, _c.c_int32, _c.c_int, _P,
                                            _P]),
+    ("kvq_decode_verify_workspace_bytes", _c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32,
+                                                        _c.c_int32, _c.c_int, _P]),
+    ("kvq_decode_verify", _c.c_int, [_P, _c.c_int32, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32,
+                                     _c.c_float, _P, _c.c_int, _P, _c.c_size_t, _c.c_int32, _c.c_int,
+                                     _P, _P]),
 ]
 
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
@@ -257,6 +262,34 @@ def decode_attn_noalloc(q, k_cache, v_cache, k_scale, v_scale, block_tables, con
                                          _ptr(out), _out_dtype(out), partition_tokens, FMT[fmt],
                                          ctypes.byref(d), _stream(stream)),
            "kvq_decode_attn_noalloc")
+
+
+def decode_verify(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                  max_context_len, sm_scale, out, fmt: str, d: Dims, workspace=None,
+                  partition_tokens=0, stream=None):
+    """Multi-query decode for speculative verification (kvq_decode_verify).
+    q, out: [B][Hq][n_query][D]; position j of sequence b sees the tokens before
+    the last n_query - 1 - j of its context."""
+    _need(q, torch.bfloat16, "q")
+    _need(out, out.dtype, "out")
+    _need(block_tables, torch.int32, "block_tables")
+    _need(context_lens, torch.int32, "context_lens")
+    if q.dim() != 4 or tuple(out.shape) != tuple(q.shape):
+        raise KvqError("q and out must be [batch][n_q_heads][n_query][head_dim]")
+    B, nq = q.shape[0], q.shape[2]
+    if workspace is None:
+        n = lib().kvq_decode_verify_workspace_bytes(B, nq, int(max_context_len), partition_tokens,
+                                                    FMT[fmt], ctypes.byref(d))
+        if n == 0 and B > 0:
+            raise KvqError("kvq_decode_verify_workspace_bytes: invalid arguments")
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().kvq_decode_verify(_ptr(q), B, nq, _ptr(k_cache), _ptr(v_cache),
+                                   _scales(k_scale, v_scale), _ptr(block_tables),
+                                   _ptr(context_lens), int(max_context_len), float(sm_scale),
+                                   _ptr(out), _out_dtype(out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), partition_tokens,
+                                   FMT[fmt], ctypes.byref(d), _stream(stream)), "kvq_decode_verify")
+    return out
 
 
 def device_error(clear=True) -> int:

@@ -132,6 +132,14 @@ def test_host_checks_need_no_gpu(kvq):
         assert L.kvq_decode_attn(fake, 1, fake, fake, none, fake, fake, 100, ctypes.c_float(0.1), fake,
                                  0, fake, 1 << 30, 0, fmt, ctypes.byref(d), None) == -1
     assert L.kvq_append(fake, fake, fake, 4, fake, fake, fake, fake, 6, ctypes.byref(d), None) == -1
+    # multi-query decode: G * n_query must stay a supported group size
+    vargs = lambda nq: (fake, 1, nq, fake, fake, scales, fake, fake, 100, ctypes.c_float(0.1), fake,
+                        0, fake, 1 << 30, 0, 1, ctypes.byref(d), None)
+    assert L.kvq_decode_verify(*vargs(8)) == -2                   # G = 2: 16 heads per group
+    assert L.kvq_decode_verify(*vargs(0)) == -1
+    assert L.kvq_decode_verify(*vargs(9)) == -1
+    assert L.kvq_decode_verify_workspace_bytes(1, 4, 100, 0, 1, ctypes.byref(d)) == \
+        L.kvq_decode_workspace_bytes(1, 100, 0, 1, ctypes.byref(kvq.dims(64, 2, 16, 64, 8)))
     # max_context_len beyond what the block table can hold
     assert kvq.lib().kvq_decode_workspace_bytes(1, 8 * 16 + 1, 0, 1, ctypes.byref(d)) == 0
     # partition must be a multiple of 128

@@ -1,0 +1,117 @@
+"""GPU parity of multi-query decode (speculative verification) against the CPU
+oracle ("KV cache quantization: what FP8/INT8 K and V really give", "How it
+interacts with speculative decoding": the target model scores the K+1 proposed
+positions in one pass over the quantized cache).
+
+The n_query new tokens are appended first; position j sees the first
+ctx - n_query + 1 + j tokens. Every position's output (FP32) must be within max
+|err| 4e-3 and mean |err| 5e-4 of the oracle's FP64 attention over the same
+dequantized K/V, across formats, GQA groups, head_dims, ragged contexts
+(including contexts shorter than n_query, whose first positions see nothing)
+and split-K partitions that end inside the new tokens.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from int8_quantized_paged_quantize_b200 import kvq
+from int8_quantized_paged_quantize_b200 import workloads as W
+from oracle import attention as OA
+from oracle import formats as OF
+from oracle import paged as OP
+from tests import gpu_cases as GC
+
+pytestmark = pytest.mark.gpu
+
+CTX = [1, 2, 3, 15, 16, 17, 127, 128, 129, 300, 1000]
+
+
+def _run(fmt, D, G, nq, ctx=CTX, Hk=2, partition=0, seed=0):
+    w = W.Workload("synthetic", fmt, batch=len(ctx), n_q_heads=Hk * G, n_kv_heads=Hk, head_dim=D,
+                   lengths="list", ctx=tuple(ctx), kv_mean=0.3 if fmt == "int8" else 0.0)
+    tables, nb = W.block_tables(w, seed)
+    lens = W.context_lengths(w, seed)
+    hist = [W.kv_history(w, b, seed) for b in range(w.batch)]
+    d = kvq.dims(nb, Hk, Hk * G, D, tables.shape[1])
+    K = torch.cat([h[0] for h in hist])
+    V = torch.cat([h[1] for h in hist])
+    S = torch.cat([torch.from_numpy(GC.slots_for(tables, b, np.arange(lens[b]))) for b in range(w.batch)])
+    static = {}
+    if fmt in ("int8c", "int8t"):
+        pc = fmt == "int8c"
+        static = {"k_static": OF.int8_static_calibrate(K.float().numpy(), pc),
+                  "v_static": OF.int8_static_calibrate(V.float().numpy(), pc)}
+        cache = kvq.LayerCache.allocate(fmt, d, **{k: torch.from_numpy(v).to(torch.bfloat16).cuda()
+                                                   for k, v in static.items()})
+    else:
+        cache = kvq.LayerCache.allocate(fmt, d)
+    cache.append(K.cuda(), V.cuda(), S.cuda())
+    g = torch.Generator().manual_seed(100 + seed)
+    q = torch.randn(w.batch, Hk * G, nq, D, generator=g).to(torch.bfloat16)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    kvq.decode_verify(q.cuda(), cache.k, cache.v, cache.k_scale, cache.v_scale,
+                      torch.from_numpy(tables).cuda(), torch.from_numpy(lens.astype(np.int32)).cuda(),
+                      int(lens.max()), w.sm_scale, out, fmt, d, partition_tokens=partition)
+    torch.cuda.synchronize()
+    assert kvq.device_error() == 0
+    # oracle: the same tokens through the oracle's pool, then FP64 attention
+    pool = OP.LogicalPool(fmt, nb, Hk, 16, D, **static)
+    pool.append(K.float().numpy(), V.float().numpy(), S.numpy())
+    kv = [pool.gather(tables[b], lens[b]) for b in range(w.batch)]
+    ref = OA.verify_attention(q.float().numpy(), kv, w.sm_scale, Hk)
+    err = np.abs(out.cpu().numpy().astype(np.float64) - ref)
+    return err, out.cpu(), ref, lens
+
+
+def _check(err):
+    assert err.max() <= GC.MAX_ABS and err.mean() <= GC.MEAN_ABS, (err.max(), err.mean())
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G,nq", [(1, 2), (1, 4), (1, 8), (2, 2), (2, 4), (4, 2)])
+def test_verify_shapes(fmt, D, G, nq):
+    err, out, ref, lens = _run(fmt, D, G, nq)
+    _check(err)
+    # positions that see no token are exact zeros
+    for b, c in enumerate(lens):
+        for j in range(nq):
+            if c - nq + 1 + j <= 0:
+                assert torch.count_nonzero(out[b, :, j]) == 0
+
+
+@pytest.mark.parametrize("fmt", ["e5m2", "bf16", "int8c", "int8t"])
+def test_verify_other_formats(fmt):
+    _check(_run(fmt, 128, 2, 4)[0])
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+def test_verify_split_inside_the_new_tokens(fmt):
+    """Partitions of one tile: a sequence of 129 tokens ends in a piece of one
+    token, which the first positions do not see at all (an empty partial)."""
+    _check(_run(fmt, 128, 2, 4, ctx=[129, 130, 256, 257, 1000, 3], partition=128)[0])
+
+
+def test_one_position_equals_plain_decode():
+    fmt, D, G, Hk = "fp8", 128, 4, 2
+    ctx = [50, 700, 129]
+    w = W.Workload("synthetic", fmt, batch=len(ctx), n_q_heads=Hk * G, n_kv_heads=Hk, head_dim=D,
+                   lengths="list", ctx=tuple(ctx))
+    tables, nb = W.block_tables(w)
+    lens = W.context_lengths(w)
+    hist = [W.kv_history(w, b) for b in range(w.batch)]
+    d = kvq.dims(nb, Hk, Hk * G, D, tables.shape[1])
+    cache = kvq.LayerCache.allocate(fmt, d)
+    S = torch.cat([torch.from_numpy(GC.slots_for(tables, b, np.arange(lens[b]))) for b in range(w.batch)])
+    cache.append(torch.cat([h[0] for h in hist]).cuda(), torch.cat([h[1] for h in hist]).cuda(), S.cuda())
+    q = torch.randn(w.batch, Hk * G, 1, D, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16).cuda()
+    tb = torch.from_numpy(tables).cuda()
+    cl = torch.from_numpy(lens.astype(np.int32)).cuda()
+    out_v = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    kvq.decode_verify(q, cache.k, cache.v, cache.k_scale, cache.v_scale, tb, cl, int(lens.max()),
+                      w.sm_scale, out_v, fmt, d)
+    out_d = cache.decode(q[:, :, 0].contiguous(), tb, cl, int(lens.max()), sm_scale=w.sm_scale,
+                         out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(out_v[:, :, 0], out_d)
