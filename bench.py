@@ -422,6 +422,47 @@ def e2e_loop(st, steps, warmup, world, flush):
     return ms, h2d, d2h
 
 
+def verify_rate(st, flush, n_query=2, reps=10, warmup=3):
+    """Multi-query decode (speculative verification, kvq_decode_verify) over the
+    cache as the first timed step leaves it: the last n_query cached tokens of
+    every sequence are the positions being verified. L2 flushed before every
+    timed call. None when the GQA group times n_query exceeds 8."""
+    w, kvq, c = st.w, st.kvq, st.cache
+    if w.group * n_query > 8:
+        return None
+    g = torch.Generator(device="cuda").manual_seed(7)
+    q = torch.randn(w.batch, w.n_q_heads, n_query, w.head_dim, generator=g,
+                    device="cuda").to(torch.bfloat16)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    import ctypes
+    n = kvq.lib().kvq_decode_verify_workspace_bytes(w.batch, n_query, st.max_ctx, 0,
+                                                    kvq.FMT[st.fmt], ctypes.byref(st.dims))
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+
+    def call():
+        kvq.decode_verify(q, c.k, c.v, c.k_scale, c.v_scale, st.tables, st.ctx[0], st.max_ctx,
+                          w.sm_scale, out, st.fmt, st.dims, workspace=ws)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        call()
+        b.record()
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    kv, alg = kv_bytes_per_step(st.ctx_np[0], w, st.fmt)
+    hbm, _ = peaks()
+    return {"n_query": n_query, "ms": ms, "kv_gbs": kv / (ms * 1e-3) / 1e9,
+            "frac_of_peak": kv / (ms * 1e-3) / 1e9 / hbm,
+            "positions_per_s": w.batch * n_query / (ms * 1e-3),
+            "what": "decode partials + merge for n_query positions per sequence, pages read once"}
+
+
 def bulk_append_rate(st, tokens=32768, reps=5):
     """Append throughput for one bulk call of `tokens` tokens (prefill-style)."""
     K, V, S = st.hist
@@ -652,6 +693,10 @@ def main():
     seqs_s = sum_over_ranks(wb.batch, world) / (step_ms * 1e-3)
     app_tok_s = sum_over_ranks(wb.batch, world) / (max_over_ranks(t["append"], world) * 1e-3)
     bulk_tok_s, bulk_ms, bulk_n = bulk_append_rate(st)
+    try:
+        verify = verify_rate(st, flush)
+    except Exception as e:                        # reported, never fatal to the main line
+        verify = {"error": f"{type(e).__name__}: {e}"[:200]}
 
     e2e_ms, h2d, d2h = e2e_loop(st, args.steps, args.warmup, world, flush)
     e2e_ms = max_over_ranks(e2e_ms, world)
@@ -727,6 +772,7 @@ def main():
         "e2e": {"value": e2e_val, "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": t["launches"],
+        "verify": verify,
         "clocks": clk,
         "formats": formats,
         "cpu_baseline": cpu,
