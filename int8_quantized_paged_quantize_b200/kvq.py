@@ -359,6 +359,18 @@ class LayerCache:
                     partition_tokens, stream)
         return out
 
+    def verify(self, q, block_tables, context_lens, max_context_len, sm_scale=None, out=None,
+               workspace=None, partition_tokens=0, stream=None, out_dtype=torch.bfloat16):
+        """Multi-query decode (kvq_decode_verify): q [B][Hq][n_query][D], the
+        n_query newest cached tokens of each sequence being the positions."""
+        if sm_scale is None:
+            sm_scale = 1.0 / math.sqrt(self.dims.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        return decode_verify(q, self.k, self.v, self.k_scale, self.v_scale, block_tables,
+                             context_lens, max_context_len, sm_scale, out, self.fmt, self.dims,
+                             workspace=workspace, partition_tokens=partition_tokens, stream=stream)
+
     # ---- copies in the logical layout [NB][Hk][block_size][D] (for inspection and tests)
     def k_logical(self, blocks=None):
         """K of all blocks (or of the block ids `blocks`) as [n][Hk][block_size][D]."""
