@@ -1,8 +1,13 @@
 // Paged GQA decode attention with the cache codes fed to the 5th-generation
-// tensor cores as they are stored: FP8 E4M3 codes through kind::f8f6f4, INT8
-// codes through kind::i8 (exact integer sums), BF16 through kind::f16. No thread
-// dequantizes a K or V element; the per-token scales and zero points are applied
-// to the small S and P tiles instead. Included by kvq_kernels.cu.
+// tensor cores as they are stored: FP8 E4M3 or E5M2 codes through
+// kind::f8f6f4, INT8 codes through kind::i8 (exact integer sums), BF16 through
+// kind::f16. No thread dequantizes a K or V element; the per-token scales and
+// zero points are applied to the small S and P tiles instead. Static INT8
+// scales (one per channel, or one per cache) vary along the contraction, so
+// they multiply the query before its split (K) and the finished channel sums
+// (V). Multi-query decode (speculative verification) runs the n_query
+// positions of a query head as extra heads of its group, each with its causal
+// limit. Included by kvq_kernels.cu.
 //
 // Work split (persistent, stream-K): the work list is every (sequence b, KV
 // head h, 128-token tile) in order of b, then h, then tile, each (b, h) run
