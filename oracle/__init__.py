@@ -30,10 +30,12 @@ Modules
               paged gather + dequantisation.
 ``attention`` FP64 softmax attention over the gathered K/V (GQA head mapping).
 ``sizes``     the closed-form KV-cache byte count.
+``kivi``      KIVI-style low-bit codes (K per channel, V per token, BF16
+              residual); the CUDA path for it is not built.
 
 Parity status of each function is given in its docstring; the one result with
 no pin is the quality number (deviation from a BF16-cache attention), which is
 reported, not checked: "parity unpinned".
 """
 
-from . import formats, paged, attention, sizes  # noqa: F401
+from . import formats, paged, attention, sizes, kivi  # noqa: F401
