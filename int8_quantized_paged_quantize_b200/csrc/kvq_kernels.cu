@@ -52,11 +52,6 @@ __device__ __forceinline__ float warp_max(float x) {
   for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
   return x;
 }
-__device__ __forceinline__ float warp_min(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
-}
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -101,8 +96,8 @@ namespace kvq {
 
 // ------------------------------------------------------------------ append
 // Quantize one (token, KV head) row of D BF16 values held by a warp (E = D/32
-// values per lane): range by warp shuffles, the BF16 scale (+ zero point) on
-// every lane, codes in d order packed little-endian into `w`.
+// values per lane): the range by integer warp reductions, the BF16 scale (+
+// zero point) on every lane, codes in d order packed little-endian into `w`.
 template <int D, int FMT>
 struct RowCodes {
   static constexpr int E = D / 32;
