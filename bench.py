@@ -535,6 +535,18 @@ def bulk_append_probe(fmt, mode, reps=5, T=32768, Hk=8, D=128):
 
 
 # ----------------------------------------------------------------------------- CPU oracle
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def oracle_decode_sample(w, fmt, seed, budget_s=12.0):
     """Time the CPU oracle on a bounded sample of the workload: for sequences in
     order until the time budget is spent, quantize the sequence's cached K/V into
@@ -614,7 +626,7 @@ def run_reference(args):
             "dtype": "f64", "data": "synthetic (seeded)",
             "config": config_block(w, fmt, l2="host run (no GPU)"),
             "cpu_baseline": {"kind": "oracle", "value": value, "unit": "GB/s", "cores": threads,
-                             "sample": desc},
+                             "sample": desc, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -749,7 +761,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         gbs, tok_s, desc, threads = oracle_decode_sample(wb, fmt, seed=0)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
-               "append_tok_per_s": tok_s}
+               "append_tok_per_s": tok_s, "cpu_model": cpu_model()}
 
     line = {
         "metric": metric_name(fmt), "value": value, "unit": "GB/s", "n_gpus": world,
