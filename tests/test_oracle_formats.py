@@ -344,3 +344,46 @@ def test_int8_zero_point_landmarks():
     # symmetric range: zp near 0
     c, s, zp = F.int8_quantize(np.array([[-3.0, 3.0]], dtype=np.float32))
     assert abs(int(zp[0])) <= 1
+
+
+# ----------------------------------------------------------------------------- scale rounding
+
+
+def _scale_rows():
+    rows = read_golden("fp8_scale_rounding.txt")
+    return [(fmt, np.float32(amax), int(bits, 16)) for fmt, amax, bits, _ in rows]
+
+
+def test_scale_rounding_rows_are_exact_f32_inputs():
+    """The fixture's amax values are f32 numbers as written (no rounding on read)."""
+    for fmt, amax, _ in _scale_rows():
+        assert float(amax) == float(np.float64(amax))
+
+
+def test_fp8_and_e5m2_scale_rounding_rows():
+    """Hand-worked scales: RNE of the f32 quotient, ties to even, IEEE division.
+    Each row puts amax at the front of a row of smaller values, so the scale is
+    taken through the full quantize path too."""
+    for fmt, amax, bits in _scale_rows():
+        row = np.array([amax, amax / np.float32(4), -amax / np.float32(8)], dtype=np.float32)
+        if fmt == "fp8":
+            s = F.fp8_scale(row)
+            _, s2 = F.fp8_quantize(row)
+        else:
+            s = F.e5m2_scale(row)
+            _, s2 = F.e5m2_quantize(row)
+        assert int(F.bf16_bits(s)) == bits, (fmt, float(amax), hex(int(F.bf16_bits(s))), hex(bits))
+        assert int(F.bf16_bits(s2)) == bits
+        # the sign of amax does not matter
+        s3 = F.fp8_scale(-row) if fmt == "fp8" else F.e5m2_scale(-row)
+        assert int(F.bf16_bits(s3)) == bits
+
+
+def test_e5m2_worked_row():
+    rows = read_golden("e5m2_worked_row.txt")
+    scale_bits = int(rows[0][1], 16)
+    xs = np.array([float(r[0]) for r in rows[1:]], dtype=np.float32)
+    want = np.array([int(r[1], 16) for r in rows[1:]], dtype=np.uint8)
+    codes, s = F.e5m2_quantize(xs)
+    assert int(F.bf16_bits(s)) == scale_bits
+    assert np.array_equal(codes, want)

@@ -2,7 +2,8 @@
 
 This shows that the pins are not vacuous: a wrong exponent bias, a tie rule
 that rounds away from zero, a flipped zero-point sign, a GQA mapping that
-interleaves instead of grouping, or a dropped softmax scale each break at least
+interleaves instead of grouping, a dropped softmax scale, or an FP8 / E5M2 scale
+that truncates, rounds ties up or multiplies by a reciprocal each break at least
 one pin test.
 """
 
@@ -77,3 +78,32 @@ def test_dropped_softmax_scale_is_caught(monkeypatch):
     good = A.attend_one
     monkeypatch.setattr(A, "attend_one", lambda q, k, v, s: good(q, k, v, 1.0))
     assert _fails(TA.test_decode_attention_matches_torch_sdpa_gqa)
+
+
+# --------------------------------------------------------------------------- FP8 / E5M2 scale rounding
+def _bf16_truncate(x):
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    return (a.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+
+
+def _bf16_half_up(x):
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    return ((a.view(np.uint32) + np.uint32(0x8000)) & np.uint32(0xFFFF0000)).view(np.float32)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "e5m2"])
+@pytest.mark.parametrize("rounding", ["truncate", "half_up", "reciprocal"])
+def test_wrong_scale_rounding_is_caught(monkeypatch, fmt, rounding):
+    M = np.float32(F.E4M3_MAX if fmt == "fp8" else F.E5M2_MAX)
+
+    def scale(rows):
+        r = np.asarray(rows, dtype=np.float32)
+        amax = np.max(np.abs(r), axis=-1).astype(np.float32)
+        if rounding == "reciprocal":
+            return F.bf16_round(amax * (np.float32(1.0) / M))
+        q = amax / M
+        return _bf16_truncate(q) if rounding == "truncate" else _bf16_half_up(q)
+    monkeypatch.setattr(F, "fp8_scale" if fmt == "fp8" else "e5m2_scale", scale)
+    assert _fails(TF.test_fp8_and_e5m2_scale_rounding_rows)
+    if rounding == "truncate" and fmt == "e5m2":
+        assert _fails(TF.test_e5m2_worked_row)      # its quotient's low half is 0xDB6E
