@@ -101,8 +101,10 @@ typedef enum {
 #define KVQ_DEVERR_BLOCK 0x2u    /* decode: block id outside [0, num_blocks) */
 #define KVQ_DEVERR_CONTEXT 0x4u  /* decode: context_len < 0, > max_context_len,
                                     or > max_blocks_per_seq * block_size */
-#define KVQ_DEVERR_TIMEOUT 0x8u  /* decode: a pipeline wait ran out (about 1 s);
-                                    that chunk's output is not valid */
+#define KVQ_DEVERR_TIMEOUT 0x8u  /* decode: a pipeline wait ran out (about 1 s by
+                                    default, kvq_set_wait_limit); the output rows
+                                    of the sequences that CTA worked on come out
+                                    as NaN and the call's output is not valid */
 
 typedef struct {
   int32_t num_blocks;         /* blocks in the pool */
@@ -297,12 +299,16 @@ int kvq_decode_merge(int32_t batch, const int32_t* context_lens, int32_t max_con
  * cudaMalloc/cudaFree). The split-K scratch comes from one static device array
  * of KVQ_NOALLOC_SCRATCH_BYTES, held by every GPU that loads the library until
  * the process exits; the call allocates nothing.
- * - Returns KVQ_ERR_WORKSPACE, before touching the device, when the split plan
- *   (kvq_decode_workspace_bytes for the same arguments) needs more than
- *   KVQ_NOALLOC_SCRATCH_BYTES; use a larger partition_tokens or kvq_decode_attn.
+ * - Every argument check of kvq_decode_attn runs first, with the same result
+ *   (batch 0 included). Then KVQ_ERR_WORKSPACE, before touching the device,
+ *   when the split plan (kvq_decode_workspace_bytes for the same arguments)
+ *   needs more than KVQ_NOALLOC_SCRATCH_BYTES; use a larger partition_tokens
+ *   or kvq_decode_attn.
  * - The first call on each device looks up the array's device address (with
- *   that device current) and caches it; make that first call before any stream
- *   capture.
+ *   that device current) and caches it together with the id of the device's
+ *   context; after a cudaDeviceReset the next call sees a new context and
+ *   looks the address up again. Make the first call on a device (and the first
+ *   after a reset) before any stream capture.
  * - All calls share the array and it keeps the last call's contents (nothing in
  *   it needs to start at zero). Calls whose kernels overlap on the GPU (other
  *   streams, other host threads) race on it: serialise them.
@@ -351,8 +357,26 @@ int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void*
                       kvq_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
-/* Device error word.                                                          */
+/* Device error word and the decode wait bound.                               */
 /* ------------------------------------------------------------------------ */
+/*
+ * Every wait inside the decode kernels (for a page copy, an MMA, the softmax
+ * warps) gives up after a bounded number of SM clock cycles instead of hanging
+ * the GPU. A CTA whose wait runs out stops issuing work, waits for the copies
+ * and MMAs it already issued, writes NaN markers in place of its partials (so
+ * the affected output rows are NaN, not plausible values), frees its tensor
+ * memory, returns, and sets KVQ_DEVERR_TIMEOUT; the context stays usable.
+ * kvq_set_wait_limit sets that bound, in SM clock cycles, for decode launches
+ * made after the call on any device (0 restores the default of 2e9 cycles,
+ * about one second at 2 GHz). A bound far below a page's load time makes the
+ * waits run out on purpose, which is how the failure path is tested. The
+ * setting is process-wide and not ordered against launches from other host
+ * threads. Returns KVQ_ERR_ARG for a negative value.
+ */
+int kvq_set_wait_limit(int64_t cycles);
+/* The bound decode launches currently use, in SM clock cycles. */
+int64_t kvq_get_wait_limit(void);
+
 /* Read (and if `clear` is non-zero, reset) the current device's error word
  * (KVQ_DEVERR_* bits) into *flags (host). Synchronizes the device. Returns
  * KVQ_ERR_DEVICE if any bit was set, KVQ_OK otherwise. */

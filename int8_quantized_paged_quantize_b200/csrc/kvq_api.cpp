@@ -3,6 +3,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <atomic>
 #include <cstdint>
 
 #include <cuda_runtime.h>
@@ -55,11 +56,12 @@ int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kv
   return KVQ_OK;
 }
 
-}  // namespace kvq
-
-using namespace kvq;
-
 namespace {
+constexpr long long kDefaultWaitLimit = 2000000000LL;   // about one second of SM clock
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+}  // namespace
+
+long long decode_wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
 
 int check_decode_common(int32_t batch, int32_t max_ctx, int32_t partition_tokens, kvq_fmt fmt,
                         const kvq_dims* dims, DecodePlan* plan) {
@@ -86,7 +88,9 @@ int check_decode_inputs(const void* q, const void* kc, const void* vc, const voi
   return KVQ_OK;
 }
 
-}  // namespace
+}  // namespace kvq
+
+using namespace kvq;
 
 extern "C" {
 
@@ -182,6 +186,14 @@ int kvq_decode_attn(const void* q, int32_t batch, const void* k_cache, const voi
   return kvq_decode_merge(batch, context_lens, max_context_len, out, out_dtype, workspace,
                           workspace_bytes, partition_tokens, fmt, dims, stream);
 }
+
+int kvq_set_wait_limit(int64_t cycles) {
+  if (cycles < 0) return KVQ_ERR_ARG;
+  g_wait_limit.store(cycles == 0 ? kDefaultWaitLimit : (long long)cycles, std::memory_order_relaxed);
+  return KVQ_OK;
+}
+
+int64_t kvq_get_wait_limit(void) { return decode_wait_limit(); }
 
 int kvq_device_error(uint32_t* flags, int clear) {
   if (!flags) return KVQ_ERR_ARG;

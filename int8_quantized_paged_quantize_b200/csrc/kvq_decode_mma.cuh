@@ -45,8 +45,8 @@
 // Each MMA result sits in TMEM; S, P and O are double-buffered so the MMA of
 // one tile overlaps the softmax of the next. Every byte of the K/V crosses HBM
 // once for the whole query group. Every wait is bounded: on expiry the CTA sets
-// KVQ_DEVERR_TIMEOUT, stops issuing work, drains what it issued, frees TMEM
-// and returns.
+// KVQ_DEVERR_TIMEOUT, stops issuing work, drains what it issued, writes NaN
+// markers for its pieces' partials, frees TMEM and returns.
 
 #pragma once
 
@@ -54,6 +54,10 @@
 
 namespace kvq {
 
+// Bound on the waits that drain work already issued (copies in flight, the
+// last MMAs) before the CTA exits: those always complete, so this limit only
+// guards against a lost completion. The pipeline waits take the launch's
+// `wait_limit` (kvq_set_wait_limit; by default this same value).
 constexpr long long kMmaWaitLimitCycles = 2000000000LL;   // about one second
 
 __device__ __forceinline__ long long ll_min(long long a, long long b) { return a < b ? a : b; }
@@ -214,7 +218,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
     const int32_t* __restrict__ ctx_lens, int B, int Hk, int NB, int W, int max_ctx,
     int unit_tiles, int slots, float qk_scale, int per_tensor, int n_query,
-    float* __restrict__ part_o,
+    long long wait_limit, float* __restrict__ part_o,
     float* __restrict__ part_ml, int32_t* __restrict__ part_cnt) {
   using C = MmaCfg<D, G, FMT>;
   using namespace tc;
@@ -425,7 +429,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       // per stage: byte count, the page copies, then the scale stores and the
       // one arrival that publishes them (the copies need not wait for the scales)
       if (lane == 0) {
-        ok = mbar_wait(kempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
+        ok = mbar_wait(kempty + s, ph ^ 1, abort_flag, wait_limit);
         if (ok) mbar_expect_tx(kfull + s, bytes);
       }
       if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
@@ -439,7 +443,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
         mbar_arrive(kfull + s);
       }
       if (lane == 0) {
-        ok = mbar_wait(vempty + s, ph ^ 1, abort_flag, kMmaWaitLimitCycles);
+        ok = mbar_wait(vempty + s, ph ^ 1, abort_flag, wait_limit);
         if (ok) mbar_expect_tx(vfull + s, bytes);
       }
       if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
@@ -479,8 +483,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       int gt = 0;
       auto issue_pv = [&](int j) -> bool {
         const int s = j % C::NST;
-        if (!mbar_wait(pready + (j & 1), (j >> 1) & 1, abort_flag, kMmaWaitLimitCycles)) return false;
-        if (!mbar_wait(ofree + (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, kMmaWaitLimitCycles)) return false;
+        if (!mbar_wait(pready + (j & 1), (j >> 1) & 1, abort_flag, wait_limit)) return false;
+        if (!mbar_wait(ofree + (j & 1), ((j >> 1) & 1) ^ 1, abort_flag, wait_limit)) return false;
         tc_fence_after();
         const uint32_t a0 = vbase + s * 8 * C::PAGE;
         const uint32_t b0 = paddr + (j & 1) * C::PBYTES;
@@ -500,13 +504,13 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
         if (gt >= 1) ok = issue_pv(gt - 1);
         // the query operand of piece pc (one buffer: the softmax warps rewrite
         // it only after every S product of the piece before has been read)
-        if (ok) ok = mbar_wait(qready, pc & 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) ok = mbar_wait(qready, pc & 1, abort_flag, wait_limit);
         tc_fence_after();
         const uint32_t qa = qaddr;
         for (int i = walk.lo; ok && i < walk.hi; ++i, ++gt) {
           const int s = gt % C::NST;
-          ok = mbar_wait(kfull + s, (gt / C::NST) & 1, abort_flag, kMmaWaitLimitCycles) &&
-               mbar_wait(sfree + (gt & 1), ((gt >> 1) & 1) ^ 1, abort_flag, kMmaWaitLimitCycles);
+          ok = mbar_wait(kfull + s, (gt / C::NST) & 1, abort_flag, wait_limit) &&
+               mbar_wait(sfree + (gt & 1), ((gt >> 1) & 1) ^ 1, abort_flag, wait_limit);
           if (!ok) break;
           tc_fence_after();
           const uint32_t a0 = kbase + s * 8 * C::PAGE;
@@ -684,7 +688,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       // o (relative to the current max) += O tile j * 2^-e_j * alpha: alpha
       // moves tile j from the max it was weighted with to the current one
       auto accum_o = [&](int j) {
-        if (ok) ok = mbar_wait(ofull + (j & 1), (j >> 1) & 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) ok = mbar_wait(ofull + (j & 1), (j >> 1) & 1, abort_flag, wait_limit);
         tc_fence_after();
         uint32_t ov[C::NOL];
         if (ok) {
@@ -716,7 +720,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       for (int i = lo; i < hi; ++i, ++gt) {
         const int s = gt % C::NST;
         // ---- S of tile gt
-        if (ok) ok = mbar_wait(sfull + (gt & 1), (gt >> 1) & 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) ok = mbar_wait(sfull + (gt & 1), (gt >> 1) & 1, abort_flag, wait_limit);
         tc_fence_after();
         uint32_t sw[C::NSL];
         if (ok) {
@@ -730,8 +734,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
         mbar_arrive(sfree + (gt & 1));
 
         // ---- this token's scales (both copies acquired here, not through the MMA)
-        if (ok) ok = mbar_wait(kfull + s, (gt / C::NST) & 1, abort_flag, kMmaWaitLimitCycles);
-        if (ok) ok = mbar_wait(vfull + s, (gt / C::NST) & 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) ok = mbar_wait(kfull + s, (gt / C::NST) & 1, abort_flag, wait_limit);
+        if (ok) ok = mbar_wait(vfull + s, (gt / C::NST) & 1, abort_flag, wait_limit);
         const uint32_t mask = ok ? pmask[s] : 0u;   // pages of the tile with legal ids
         const int tile0 = i * 128;
         const int p = r >> 4, t = r & 15;
@@ -960,7 +964,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       // ---- the next piece's query operand, so that its first S can start
       // while this piece's last O drains
       if (more) {
-        if (ok) ok = mbar_wait(qfree, pc & 1, abort_flag, kMmaWaitLimitCycles);
+        if (ok) ok = mbar_wait(qfree, pc & 1, abort_flag, wait_limit);
         store_q();
         mbar_arrive(qready);
       }
@@ -984,20 +988,23 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       if constexpr (C::SI) {
         if (r < D) vsd = __bfloat162float(vs[per_tensor ? 0 : ph_ * D + r]);
       }
-      if (ok && !*abort_flag) {
+      // After a wait ran out the piece's sums are incomplete: it writes a
+      // marker instead (max +inf, sum and output NaN), so that every output row
+      // the piece contributes to merges to NaN rather than to a plausible value
+      // built from stale workspace.
+      const bool good = ok && !*abort_flag;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float L = red2[g] + red2[8 + g] + red2[16 + g] + red2[24 + g];
-          const float Cz = red2[32 + g] + red2[40 + g] + red2[48 + g] + red2[56 + g];
-          const int64_t row = (int64_t(pb) * Hq + ph_ * G + g) * slots + slot;
-          if (r < D) part_o[row * D + r] = (o[g] - Cz) * vsd;
-          if (r == 0) {
-            part_ml[row * 2] = m[g];
-            part_ml[row * 2 + 1] = L;
-          }
+      for (int g = 0; g < G; ++g) {
+        const float L = red2[g] + red2[8 + g] + red2[16 + g] + red2[24 + g];
+        const float Cz = red2[32 + g] + red2[40 + g] + red2[48 + g] + red2[56 + g];
+        const int64_t row = (int64_t(pb) * Hq + ph_ * G + g) * slots + slot;
+        if (r < D) part_o[row * D + r] = good ? (o[g] - Cz) * vsd : __int_as_float(0x7fc00000);
+        if (r == 0) {
+          part_ml[row * 2] = good ? m[g] : INFINITY;
+          part_ml[row * 2 + 1] = good ? L : __int_as_float(0x7fc00000);
         }
-        if (r == 0 && last) part_cnt[pb * Hk + ph_] = slot + 1;
       }
+      if (r == 0 && last) part_cnt[pb * Hk + ph_] = slot + 1;
     }
   }
   tc_fence_before();

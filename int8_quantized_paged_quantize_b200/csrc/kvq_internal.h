@@ -43,6 +43,20 @@ int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kv
 // Number of SMs of the current device (148 if no device can be queried).
 int device_sm_count();
 
+// Bound, in SM clock cycles, on each pipeline wait of the decode kernels
+// launched from now on (kvq_set_wait_limit; default about one second).
+long long decode_wait_limit();
+
+// Argument checks shared by every decode entry point (format, dims, sizes,
+// max_context_len against the block-table width) and the split plan.
+// Returns KVQ_OK, KVQ_ERR_ARG or KVQ_ERR_UNSUPPORTED.
+int check_decode_common(int32_t batch, int32_t max_ctx, int32_t partition_tokens, kvq_fmt fmt,
+                        const kvq_dims* dims, DecodePlan* plan);
+// Device-pointer checks of a decode call; *ks, *vs receive the scale arrays.
+int check_decode_inputs(const void* q, const void* kc, const void* vc, const void* const* scales,
+                        const int32_t* tables, const int32_t* ctx, float sm_scale, kvq_fmt fmt,
+                        const void** ks, const void** vs);
+
 // Kernel launchers (kvq_kernels.cu). They assume validated arguments and return
 // a cudaError_t value as int.
 int launch_append(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,

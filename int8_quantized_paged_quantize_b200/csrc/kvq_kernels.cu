@@ -1,5 +1,6 @@
-// CUDA kernels of libkvq for sm_100a: quantize-on-append, paged GQA decode
-// attention (split-K partials) and the log-sum-exp merge.
+// CUDA kernels of libkvq for sm_100a: quantize-on-append, the launch of the
+// paged GQA decode attention kernel (kvq_decode_mma.cuh, split-K partials) and
+// the log-sum-exp merge.
 //
 // Sources (web pages, by title and section):
 //  "KV cache quantization: what FP8/INT8 K and V really give, and their limits"
@@ -61,35 +62,11 @@ __device__ __forceinline__ float warp_sum(float x) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Two E4M3 codes (low byte first) -> two floats (exact).
-__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t two_codes) {
-  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu),
-                                              __NV_E4M3);
-  return __half22float2(*reinterpret_cast<__half2*>(&h));
-}
-
-// Eight 1-byte codes held in a uint2 / four in a uint32 -> floats.
-template <int FMT>
-__device__ __forceinline__ void codes4_to_f32(uint32_t w, float* o) {
-  if constexpr (FMT == KVQ_FP8_E4M3) {
-    const float2 a = e4m3x2_to_f2(w), b = e4m3x2_to_f2(w >> 16);
-    o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
-  } else {  // INT8: signed bytes
-    o[0] = float(int8_t(w & 0xff));
-    o[1] = float(int8_t((w >> 8) & 0xff));
-    o[2] = float(int8_t((w >> 16) & 0xff));
-    o[3] = float(int8_t(w >> 24));
-  }
-}
-
 }  // namespace kvq
 
 #include <algorithm>
-#include <cstdlib>
-#include <cstring>
 #include <utility>
 
-#include "kvq_decode_tc.cuh"
 #include "kvq_decode_mma.cuh"
 
 namespace kvq {
@@ -542,244 +519,6 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
   }
 }
 
-// ------------------------------------------------------------------ decode (CUDA cores)
-// One CTA of 4 warps per (sequence b, KV head h, chunk). Warp w takes pages
-// w, w+4, ... of the chunk. For a page of 16 tokens:
-//   QK: lane = (token t = lane & 15, half of head_dim); partial dot products
-//       over the half, completed with one xor-16 shuffle; every query head of
-//       the GQA group is done from the same K bytes, so each byte is read once.
-//   online softmax (base 2) per warp: page max by shuffles, rescale of the
-//       running sums by exp2(m_old - m_new).
-//   PV: the V page is stored transposed, so a lane owns D/32 channels and reads
-//       16 consecutive tokens per channel; the weights p*s_v of the page's 16
-//       tokens come from a small shared buffer.
-// Quantized values are never materialised: the K scale multiplies the finished
-// dot product, the V scale is folded into the softmax weight, and INT8 zero
-// points are subtracted as zp * sum(q) (K) and as sum(w * zp) (V).
-template <int D, int G, int FMT>
-struct SimtCfg {
-  static constexpr int ELT = (FMT == KVQ_BF16) ? 2 : 1;
-  static constexpr int KU4 = D * ELT / 32;          // uint4 per lane for a K half-row
-  static constexpr int ROWS = D / 32;               // V channels per lane
-  static constexpr int VU4 = ROWS * ELT;            // uint4 per lane for its V rows
-  static constexpr int PAGE_BYTES = kBlockSize * D * ELT;
-};
-
-template <int D, int G, int FMT>
-__global__ void __launch_bounds__(128) decode_simt_kernel(
-    const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kc,
-    const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
-    const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
-    const int32_t* __restrict__ ctx_lens, int Hk, int NB, int W, int max_ctx, int part,
-    int max_splits, float qscale, float* __restrict__ part_o, float* __restrict__ part_ml,
-    int slots, int32_t* __restrict__ part_cnt) {
-  using C = SimtCfg<D, G, FMT>;
-  constexpr int ELT = C::ELT;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x % max_splits;
-  const int bh = blockIdx.x / max_splits;
-  const int b = bh / Hk, h = bh % Hk;
-  const int Hq = Hk * G;
-
-  __shared__ __align__(16) float qs[G][D];
-  __shared__ float qsum[G];
-  __shared__ __align__(16) float wsm[4][kBlockSize][G];
-  __shared__ float red_m[4][G], red_l[4][G];
-  __shared__ __align__(16) float red_o[4][G][D];
-
-  int ctx = ctx_lens[b];
-  const int64_t cap = int64_t(W) * kBlockSize;
-  if (ctx < 0 || ctx > max_ctx || ctx > cap) {
-    if (threadIdx.x == 0 && split == 0) flag_error(KVQ_DEVERR_CONTEXT);
-    ctx = 0;
-  }
-  const int n_splits = (ctx + part - 1) / part;
-  if (split >= n_splits) return;                 // the merge never reads this chunk
-  const int t0 = split * part, t1 = min(ctx, t0 + part);
-  const int p0 = t0 / kBlockSize, p1 = (t1 + kBlockSize - 1) / kBlockSize;
-
-  // query group of this KV head, pre-scaled into the base-2 softmax domain
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int g = i / D, d = i % D;
-    qs[g][d] = __bfloat162float(q[(int64_t(b) * Hq + h * G + g) * D + d]) * qscale;
-  }
-  __syncthreads();
-  if (threadIdx.x < G) {
-    float s = 0.f;
-    for (int d = 0; d < D; ++d) s += qs[threadIdx.x][d];
-    qsum[threadIdx.x] = s;
-  }
-  __syncthreads();
-
-  const int t_in = lane & 15, half = lane >> 4;
-  float m_run[G], l_part[G], corr_part[G], acc[G][C::ROWS];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m_run[g] = -INFINITY; l_part[g] = 0.f; corr_part[g] = 0.f;
-#pragma unroll
-    for (int j = 0; j < C::ROWS; ++j) acc[g][j] = 0.f;
-  }
-
-  const int32_t* trow = tables + int64_t(b) * W;
-  for (int pg = p0 + warp; pg < p1; pg += 4) {
-    const int blk = trow[pg];
-    if (blk < 0 || blk >= NB) {
-      if (lane == 0) flag_error(KVQ_DEVERR_BLOCK);
-      continue;
-    }
-    const int64_t page = int64_t(blk) * Hk + h;
-    const int nvalid = min(kBlockSize, t1 - pg * kBlockSize);
-    const bool valid = t_in < nvalid && pg * kBlockSize + t_in >= t0;
-
-    // ---- loads (K: chunks of this lane's half row; V: this lane's channel rows)
-    uint4 kr[C::KU4], vr[C::VU4];
-    const uint8_t* kpage = kc + page * C::PAGE_BYTES;
-#pragma unroll
-    for (int i = 0; i < C::KU4; ++i)
-      kr[i] = __ldg(reinterpret_cast<const uint4*>(kpage + k_chunk_offset<D * ELT>(half * C::KU4 + i, t_in)));
-    const uint8_t* vpage = vc + page * C::PAGE_BYTES;
-#pragma unroll
-    for (int j = 0; j < C::ROWS; ++j) {
-#pragma unroll
-      for (int u = 0; u < ELT; ++u)
-        vr[j * ELT + u] = __ldg(reinterpret_cast<const uint4*>(vpage + u * (D * 16) + (lane * C::ROWS + j) * 16));
-    }
-    float sk = 1.f, sv = 1.f, zk = 0.f, zv = 0.f;
-    if constexpr (FMT == KVQ_FP8_E4M3) {
-      sk = __bfloat162float(ks[page * kBlockSize + t_in]);
-      sv = __bfloat162float(vs[page * kBlockSize + t_in]);
-    } else if constexpr (FMT == KVQ_INT8_ASYM) {
-      const __nv_bfloat162 mk = reinterpret_cast<const __nv_bfloat162*>(ks)[page * kBlockSize + t_in];
-      const __nv_bfloat162 mv = reinterpret_cast<const __nv_bfloat162*>(vs)[page * kBlockSize + t_in];
-      sk = __low2float(mk); zk = __high2float(mk);
-      sv = __low2float(mv); zv = __high2float(mv);
-    }
-
-    // ---- QK over this lane's half of head_dim
-    float dot[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) dot[g] = 0.f;
-    const uint32_t* kw = reinterpret_cast<const uint32_t*>(kr);
-#pragma unroll
-    for (int i = 0; i < C::KU4 * 4; ++i) {       // 32-bit words
-      float kv[4];
-      int nv;
-      if constexpr (FMT == KVQ_BF16) {
-        kv[0] = bf16_lo(kw[i]); kv[1] = bf16_hi(kw[i]); nv = 2;
-      } else {
-        codes4_to_f32<FMT>(kw[i], kv); nv = 4;
-      }
-      const int d0 = half * (D / 2) + i * nv;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (e < nv) dot[g] = fmaf(qs[g][d0 + e], kv[e], dot[g]);
-      }
-    }
-    float x[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float full = dot[g] + __shfl_xor_sync(0xffffffffu, dot[g], 16);
-      if constexpr (FMT == KVQ_FP8_E4M3) full *= sk;
-      if constexpr (FMT == KVQ_INT8_ASYM) full = (full - zk * qsum[g]) * sk;
-      x[g] = valid ? full : -INFINITY;
-    }
-
-    // ---- online softmax for the page
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float pm = x[g];
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, o));
-      const float m_new = fmaxf(m_run[g], pm);
-      const float alpha = exp2f(m_run[g] - m_new);     // 0 when m_run is -inf
-      const float p = valid ? exp2f(x[g] - m_new) : 0.f;
-      m_run[g] = m_new;
-      l_part[g] = l_part[g] * alpha + (half == 0 ? p : 0.f);
-#pragma unroll
-      for (int j = 0; j < C::ROWS; ++j) acc[g][j] *= alpha;
-      const float w = valid ? p * sv : 0.f;
-      if constexpr (FMT == KVQ_INT8_ASYM)
-        corr_part[g] = corr_part[g] * alpha + (half == 0 && valid ? w * zv : 0.f);
-      if (half == 0) wsm[warp][t_in][g] = w;
-    }
-    __syncwarp();
-
-    // ---- PV: this lane's channels, 16 tokens each
-    if (nvalid < kBlockSize) {                       // zero the tokens past the end
-#pragma unroll
-      for (int j = 0; j < C::ROWS; ++j) {
-#pragma unroll
-        for (int wd = 0; wd < 4 * ELT; ++wd) {
-          uint32_t* u = reinterpret_cast<uint32_t*>(&vr[j * ELT]) + wd;
-          const int tok0 = wd * 4 / ELT;           // first token in this word
-          uint32_t keep = 0;
-#pragma unroll
-          for (int bq = 0; bq < 4; ++bq)
-            if (tok0 + bq / ELT < nvalid) keep |= 0xffu << (8 * bq);
-          *u &= keep;
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < C::ROWS; ++j) {
-      const uint32_t* vw = reinterpret_cast<const uint32_t*>(&vr[j * ELT]);
-#pragma unroll
-      for (int wd = 0; wd < 4 * ELT; ++wd) {
-        float vv[4];
-        int nv;
-        if constexpr (FMT == KVQ_BF16) {
-          vv[0] = bf16_lo(vw[wd]); vv[1] = bf16_hi(vw[wd]); nv = 2;
-        } else {
-          codes4_to_f32<FMT>(vw[wd], vv); nv = 4;
-        }
-        const int tb = wd * nv;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (e < nv) {
-#pragma unroll
-            for (int g = 0; g < G; ++g) acc[g][j] = fmaf(wsm[warp][tb + e][g], vv[e], acc[g][j]);
-          }
-        }
-      }
-    }
-    __syncwarp();
-  }
-
-  // ---- combine the 4 warps of the CTA and write the chunk's partial
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float l = warp_sum(l_part[g]);
-    const float corr = warp_sum(corr_part[g]);
-    if (lane == 0) { red_m[warp][g] = m_run[g]; red_l[warp][g] = l; }
-#pragma unroll
-    for (int j = 0; j < C::ROWS; ++j) {
-      float a = acc[g][j];
-      if constexpr (FMT == KVQ_INT8_ASYM) a -= corr;
-      red_o[warp][g][lane * C::ROWS + j] = a;
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int g = i / D, d = i % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w][g]);
-    float o = 0.f, l = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float f = (M == -INFINITY) ? 0.f : exp2f(red_m[w][g] - M);
-      o += red_o[w][g][d] * f;
-      l += red_l[w][g] * f;
-    }
-    const int64_t r = (int64_t(b) * Hq + h * G + g) * slots + split;
-    part_o[r * D + d] = o;
-    if (d == 0) { part_ml[r * 2] = M; part_ml[r * 2 + 1] = l; }
-  }
-  if (threadIdx.x == 0 && split == n_splits - 1) part_cnt[b * Hk + h] = n_splits;
-}
-
 // ------------------------------------------------------------------ merge
 // One CTA of D threads per (sequence, query head): combine the chunk partials
 // (m_i, l_i, o_i) as m = max m_i, l = sum l_i 2^(m_i - m), o = sum o_i 2^(m_i - m) / l.
@@ -830,48 +569,6 @@ cudaError_t append_dispatch(const void* k, const void* v, const int64_t* slots, 
 }
 
 template <int D, int G, int FMT>
-cudaError_t decode_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
-                             const void* ks, const void* vs, const int32_t* tables,
-                             const int32_t* ctx, int32_t max_ctx, float sm_scale,
-                             const DecodePlan& plan, void* ws, const kvq_dims& d, int, int,
-                             cudaStream_t st) {
-  float* po = static_cast<float*>(ws);
-  float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
-  int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
-  const int64_t grid = int64_t(B) * d.n_kv_heads * plan.max_splits;
-  decode_simt_kernel<D, G, FMT><<<dim3(unsigned(grid)), 128, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
-      static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
-      static_cast<const __nv_bfloat16*>(vs), tables, ctx, d.n_kv_heads, d.num_blocks,
-      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml,
-      plan.slots, pcnt);
-  return cudaGetLastError();
-}
-
-template <int D, int G, int FMT>
-cudaError_t decode_tc_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
-                                const void* ks, const void* vs, const int32_t* tables,
-                                const int32_t* ctx, int32_t max_ctx, float sm_scale,
-                                const DecodePlan& plan, void* ws, const kvq_dims& d, int, int,
-                                cudaStream_t st) {
-  using C = TcCfg<D, FMT>;
-  auto kern = decode_tc_kernel<D, G, FMT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  float* po = static_cast<float*>(ws);
-  float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
-  int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
-  const int64_t grid = int64_t(B) * d.n_kv_heads * plan.max_splits;
-  kern<<<dim3(unsigned(grid)), 192, C::SMEM, st>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
-      static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
-      static_cast<const __nv_bfloat16*>(vs), tables, ctx, d.n_kv_heads, d.num_blocks,
-      d.max_blocks_per_seq, max_ctx, plan.partition, plan.max_splits, sm_scale * kLog2e, po, pml,
-      plan.slots, pcnt);
-  return cudaGetLastError();
-}
-
-template <int D, int G, int FMT>
 cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const void* vc,
                                  const void* ks, const void* vs, const int32_t* tables,
                                  const int32_t* ctx, int32_t max_ctx, float sm_scale,
@@ -902,22 +599,8 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
       static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, d.num_blocks,
       d.max_blocks_per_seq, max_ctx, plan.partition / kTileTokens, plan.slots, sm_scale * kLog2e,
-      per_tensor, n_query, po, pml, pcnt);
+      per_tensor, n_query, decode_wait_limit(), po, pml, pcnt);
   return cudaGetLastError();
-}
-
-// Decode kernel: the tensor-core kernel that multiplies the stored codes
-// directly. For measuring one design against another, KVQ_DECODE_KERNEL=tc
-// selects the tensor-core kernel that first converts the codes to f16 in
-// registers, and KVQ_DECODE_KERNEL=simt the CUDA-core kernel.
-int decode_kernel_choice() {
-  static const int choice = [] {
-    const char* v = std::getenv("KVQ_DECODE_KERNEL");
-    if (v != nullptr && std::strcmp(v, "simt") == 0) return 2;
-    if (v != nullptr && std::strcmp(v, "tc") == 0) return 1;
-    return 0;
-  }();
-  return choice;
 }
 
 template <int D, int FMT>
@@ -926,24 +609,12 @@ cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, co
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
                              const DecodePlan& plan, void* ws, const kvq_dims& d, int per_tensor,
                              int n_query, cudaStream_t st) {
-#define KVQ_G_SWITCH(DISPATCH)                                                                   \
-  switch (G) {                                                                                   \
-    case 1: return DISPATCH<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st); \
-    case 2: return DISPATCH<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st); \
-    case 4: return DISPATCH<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st); \
-    default: return DISPATCH<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st); \
+  switch (G) {
+    case 1: return decode_mma_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st);
+    case 2: return decode_mma_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st);
+    case 4: return decode_mma_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st);
+    default: return decode_mma_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st);
   }
-  if constexpr (FMT == KVQ_FP8_E5M2 || FMT == KVQ_INT8_CHANNEL) {
-    // E5M2 and the static-scale INT8 formats exist only in the tensor-core
-    // kernel that multiplies the codes
-    KVQ_G_SWITCH(decode_mma_dispatch3)
-  } else {
-    // so does multi-query decode
-    if (decode_kernel_choice() == 0 || n_query > 1) { KVQ_G_SWITCH(decode_mma_dispatch3) }
-    if (decode_kernel_choice() == 1) { KVQ_G_SWITCH(decode_tc_dispatch3) }
-    KVQ_G_SWITCH(decode_dispatch3)
-  }
-#undef KVQ_G_SWITCH
 }
 }  // namespace
 

@@ -63,13 +63,16 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the phase of `bar` with the given parity. Gives up after
 // `limit` SM clock cycles (or as soon as *abort is set by another thread) and
 // returns false; the caller then stops issuing work. A phase that is already
-// complete is seen by one non-blocking test.
+// complete is seen by one non-blocking test. The hardware suspend of each
+// try_wait is at most 1 ms and, for short limits, about half the limit in
+// nanoseconds (limit cycles at 2 GHz), so that a short limit is felt.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           long long limit) {
   if (mbar_test_wait(bar, parity)) return true;
-  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = limit >= 2000000LL ? 1000000u : uint32_t(limit / 2 + 1);
+  if (mbar_try_wait(bar, parity, hint)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait(bar, parity, hint)) {
     if (*abort) return false;
     if (clock64() - t0 > limit) {
       *abort = 1;

@@ -50,6 +50,8 @@ _SIGNATURES = [
     ("kvq_decode_merge", _c.c_int, [_c.c_int32, _P, _c.c_int32, _P, _c.c_int, _P, _c.c_size_t,
                                     _c.c_int32, _c.c_int, _P, _P]),
     ("kvq_device_error", _c.c_int, [_c.POINTER(_c.c_uint32), _c.c_int]),
+    ("kvq_set_wait_limit", _c.c_int, [_c.c_int64]),
+    ("kvq_get_wait_limit", _c.c_int64, []),
     ("kvq_decode_attn_noalloc", _c.c_int, [_P, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32,
                                            _c.c_float, _P, _c.c_int, _c.c_int32, _c.c_int, _P,
                                            _P]),
@@ -125,6 +127,13 @@ def _out_dtype(out):
 def _need(t, dtype, name):
     if not t.is_cuda or not t.is_contiguous() or t.dtype != dtype:
         raise KvqError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def _need_out(out):
+    """Decode outputs: a contiguous CUDA bfloat16 or float32 tensor."""
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise KvqError("out must be bfloat16 or float32")
+    _need(out, out.dtype, "out")
 
 
 # --------------------------------------------------------------------------- sizes / allocator
@@ -215,7 +224,7 @@ def decode_attn(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_len
                 partition_tokens=0, stream=None):
     """Paged GQA decode attention (kvq_decode_attn): partials + merge into out."""
     _need(q, torch.bfloat16, "q")
-    _need(out, out.dtype, "out")
+    _need_out(out)
     _need(block_tables, torch.int32, "block_tables")
     _need(context_lens, torch.int32, "context_lens")
     B = q.shape[0]
@@ -252,7 +261,7 @@ def decode_attn_noalloc(q, k_cache, v_cache, k_scale, v_scale, block_tables, con
     """kvq_decode_attn_noalloc: decode attention with the library's own static
     scratch instead of a caller workspace (for callers that cannot allocate)."""
     _need(q, torch.bfloat16, "q")
-    _need(out, out.dtype, "out")
+    _need_out(out)
     _need(block_tables, torch.int32, "block_tables")
     _need(context_lens, torch.int32, "context_lens")
     B = q.shape[0]
@@ -271,7 +280,7 @@ def decode_verify(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_l
     q, out: [B][Hq][n_query][D]; position j of sequence b sees the tokens before
     the last n_query - 1 - j of its context."""
     _need(q, torch.bfloat16, "q")
-    _need(out, out.dtype, "out")
+    _need_out(out)
     _need(block_tables, torch.int32, "block_tables")
     _need(context_lens, torch.int32, "context_lens")
     if q.dim() != 4 or tuple(out.shape) != tuple(q.shape):
@@ -290,6 +299,16 @@ def decode_verify(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_l
                                    workspace.numel() * workspace.element_size(), partition_tokens,
                                    FMT[fmt], ctypes.byref(d), _stream(stream)), "kvq_decode_verify")
     return out
+
+
+def set_wait_limit(cycles: int):
+    """Bound, in SM clock cycles, on each pipeline wait of later decode launches
+    (kvq_set_wait_limit); 0 restores the default of about one second."""
+    _check(lib().kvq_set_wait_limit(int(cycles)), "kvq_set_wait_limit")
+
+
+def wait_limit() -> int:
+    return int(lib().kvq_get_wait_limit())
 
 
 def device_error(clear=True) -> int:

@@ -80,3 +80,61 @@ def test_noalloc_rejects_plans_beyond_the_scratch():
                                    ctypes.c_float(0.1), fake, 0, 128, 1, ctypes.byref(d), None)
     assert rc == -3                                  # KVQ_ERR_WORKSPACE
     assert b"workspace" in L.kvq_status_string(rc)
+
+
+def test_noalloc_limit_is_the_header_constant():
+    """A plan of exactly KVQ_NOALLOC_SCRATCH_BYTES is accepted and the next larger
+    one refused: with null pointers the first call gets past the size check and
+    stops at the pointer check (KVQ_ERR_ARG), the second stops at the size check
+    (KVQ_ERR_WORKSPACE). Pins kvq.NOALLOC_SCRATCH_BYTES to the C macro."""
+    L = kvq.lib()
+    # D = 64, one KV head, one query head, 128-token chunks of max_context_len 384
+    # (4 partial slots per row): 63310 sequences need exactly 64 MiB
+    d = kvq.dims(1024, 1, 1, 64, 24)
+    B, max_ctx, part = 63310, 384, 128
+    assert L.kvq_decode_workspace_bytes(B, max_ctx, part, 1, ctypes.byref(d)) == kvq.NOALLOC_SCRATCH_BYTES
+    assert L.kvq_decode_workspace_bytes(B + 1, max_ctx, part, 1, ctypes.byref(d)) > kvq.NOALLOC_SCRATCH_BYTES
+    null = ctypes.c_void_p(0)
+    scales = (ctypes.c_void_p * 2)(0, 0)
+    args = (null, null, scales, null, null, max_ctx, ctypes.c_float(0.125), null, 0, part, 1,
+            ctypes.byref(d), None)
+    assert L.kvq_decode_attn_noalloc(null, B, *args) == -1            # KVQ_ERR_ARG: size accepted
+    assert L.kvq_decode_attn_noalloc(null, B + 1, *args) == -3        # KVQ_ERR_WORKSPACE
+
+
+def test_noalloc_checks_arguments_like_kvq_decode_attn():
+    """Batch 0 with a bad format or unsupported dims fails the same way in both
+    entry points; a valid batch 0 is a no-op in both."""
+    L = kvq.lib()
+    null = ctypes.c_void_p(0)
+    scales = (ctypes.c_void_p * 2)(0, 0)
+    good = kvq.dims(64, 2, 8, 128, 8)
+    bad_group = kvq.dims(64, 2, 6, 128, 8)
+    for d, fmt in ((good, 99), (bad_group, 1), (good, 1), (good, -1)):
+        ws_rc = L.kvq_decode_attn(null, 0, null, null, scales, null, null, 128, ctypes.c_float(0.1),
+                                  null, 0, null, 0, 0, fmt, ctypes.byref(d), None)
+        na_rc = L.kvq_decode_attn_noalloc(null, 0, null, null, scales, null, null, 128,
+                                          ctypes.c_float(0.1), null, 0, 0, fmt, ctypes.byref(d), None)
+        assert ws_rc == na_rc, (fmt, ws_rc, na_rc)
+    assert L.kvq_decode_attn_noalloc(null, 0, null, null, scales, null, null, 128, ctypes.c_float(0.1),
+                                     null, 0, 0, 99, ctypes.byref(good), None) == -1
+    # an output dtype outside the enum is refused too
+    assert L.kvq_decode_attn_noalloc(null, 0, null, null, scales, null, null, 128, ctypes.c_float(0.1),
+                                     null, 7, 0, 1, ctypes.byref(good), None) == -1
+
+
+@pytest.mark.gpu
+def test_noalloc_python_wrapper_matches_workspace_decode():
+    """The same through kvq.decode_attn_noalloc, BF16 output, twice in a row."""
+    for ctx, seed in (([2000, 129], 3), ([17], 4)):
+        w, c, tables, cl, q = _cache("fp8", ctx, seed)
+        max_ctx = int(max(ctx))
+        ref = c.decode(q, tables, cl, max_ctx, sm_scale=w.sm_scale)
+        out = torch.empty_like(ref)
+        kvq.decode_attn_noalloc(q, c.k, c.v, c.k_scale, c.v_scale, tables, cl, max_ctx, w.sm_scale,
+                                out, "fp8", c.dims)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)             # same kernels, same split plan: same bits
+        with pytest.raises(kvq.KvqError):
+            kvq.decode_attn_noalloc(q, c.k, c.v, c.k_scale, c.v_scale, tables, cl, max_ctx,
+                                    w.sm_scale, out.to(torch.float16), "fp8", c.dims)
