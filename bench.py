@@ -9,12 +9,23 @@ new token per sequence into the quantized paged cache (kvq_append), paged GQA
 decode attention split into chunk partials (kvq_decode_partial) and the
 log-sum-exp merge into the BF16 output (kvq_decode_merge).
 
+The default workload is the 70B-shaped layer at 32k context with the INT8
+cache (B=32, 64 query / 8 KV heads, head_dim 128), the largest single-GPU
+configuration; FP8, E5M2, static INT8 and a BF16 cache of the same kernels are
+timed beside it. A `configs` block adds the long-context workload as its
+specification runs it (4 sequences: a bulk append of 8,192 tokens each, then
+64 decode steps with one append each, for FP8, INT8 and BF16) and the mixed
+serving batch (256 sequences, block tables from the library's allocator after
+allocate/free churn).
+
 Headline `value`: decode KV bytes read per step (all ranks) / step time, GB/s.
 Inputs live in HBM before timing; L2 is flushed (a 256 MB write) before every
 timed step and each step is timed on its stream with CUDA events. A timed step
 is one CUDA graph replay of its three launches; the per-phase times come from
 the same steps launched one by one with events between the phases. K steps are
 bracketed by a barrier and a device synchronize; the max over ranks is taken.
+The roofline fraction is the decode attention's (partials + merge) algorithmic
+bytes over their event time, against the measured HBM copy peak.
 Multi-GPU runs are weak-scaled replicas: each rank holds its own batch of
 sequences (the path has no exchange step), so `value` sums all ranks' bytes.
 """
@@ -39,7 +50,7 @@ sys.path.insert(0, ROOT)
 
 from int8_quantized_paged_quantize_b200 import workloads as WL  # noqa: E402
 
-DEFAULT_WORKLOAD = "llama3-8b-fp8"
+DEFAULT_WORKLOAD = "70b-32k-int8"
 # per (token, KV head): K and V metadata (the static INT8 formats keep one
 # fixed scale per channel or per cache instead)
 META_BYTES = {"fp8": 4, "int8": 8, "bf16": 0, "e5m2": 4, "int8c": 0, "int8t": 0}
@@ -197,20 +208,79 @@ def sum_over_ranks(x, world, device="cuda"):
 
 
 # ----------------------------------------------------------------------------- GPU setup
+class Layout:
+    """Block tables and slots of one workload run, fixed on the host before
+    anything is timed: the cached history's slots per sequence, the bulk
+    append's (if the workload has one) and every decode step's. The fragmented
+    shared pool is grown through the library's block allocator (kvq_pool_*,
+    paging.py) after allocate/free churn; the other pools are laid out
+    directly by workloads.block_tables."""
+
+    def __init__(self, w, seed, fmt):
+        from int8_quantized_paged_quantize_b200 import paging
+        ctx = WL.context_lengths(w, seed)
+        if w.pool == "fragmented":
+            pb = paging.paged_batch(w, seed, fmt)
+            self.hist = [pb.extend(b, int(ctx[b])) for b in range(w.batch)]
+            self.bulk = [pb.extend(b, w.bulk_append) for b in range(w.batch)]
+            self.steps = [pb.extend_all(1) for _ in range(w.decode_steps)]
+            self.tables, self.num_blocks = pb.tables.copy(), pb.dims.num_blocks
+            self.source = "kvq_pool allocator after seeded allocate/free churn"
+            pb.close()
+            return
+        tables, nb = WL.block_tables(w, seed)
+
+        def slots(b, pos):
+            return tables[b][pos // 16].astype(np.int64) * 16 + pos % 16
+        self.hist = [slots(b, np.arange(ctx[b])) for b in range(w.batch)]
+        self.bulk = [slots(b, ctx[b] + np.arange(w.bulk_append)) for b in range(w.batch)]
+        c1 = ctx + w.bulk_append
+        self.steps = [np.array([slots(b, np.array([c1[b] + s]))[0] for b in range(w.batch)])
+                      for s in range(w.decode_steps)]
+        self.tables, self.num_blocks = tables, nb
+        self.source = f"workloads.block_tables ({w.pool})"
+
+
+def history(w, seed, bulk=True):
+    """BF16 K/V of every sequence's cached tokens (and its bulk append, when
+    `bulk`), concatenated sequence by sequence, drawn on host threads."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    def one(b):
+        k, v = WL.kv_history(w, b, seed)
+        if bulk and w.bulk_append:
+            kb, vb = WL.kv_bulk(w, b, seed)
+            k, v = torch.cat([k, kb]), torch.cat([v, vb])
+        return k, v
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        parts = list(ex.map(one, range(w.batch)))
+    return torch.cat([p[0] for p in parts]), torch.cat([p[1] for p in parts])
+
+
 class Setup:
     """Device-resident state of one workload in one format: the filled cache,
-    per-step inputs, slots, context lengths, workspace and output."""
+    per-step inputs, slots, context lengths, workspace and output. `with_bulk`
+    False leaves the workload's bulk append out of the fill (it is timed on its
+    own)."""
 
-    def __init__(self, w, fmt, steps, seed, hist=None):
+    def __init__(self, w, fmt, steps, seed, hist=None, layout=None, with_bulk=True):
         from int8_quantized_paged_quantize_b200 import kvq
         self.kvq = kvq
         self.w, self.fmt, self.steps = w, fmt, steps
-        self.tables_np, nb = WL.block_tables(w, seed)
-        self.ctx0 = WL.context_lengths(w, seed) + w.bulk_append
+        self.layout = layout if layout is not None else Layout(w, seed, fmt)
+        lay = self.layout
+        self.tables_np, nb = lay.tables, lay.num_blocks
+        bulk = w.bulk_append if with_bulk else 0
+        self.ctx0 = WL.context_lengths(w, seed) + bulk
         d = kvq.dims(nb, w.n_kv_heads, w.n_q_heads, w.head_dim, self.tables_np.shape[1])
         self.dims = d
         dev = torch.device("cuda")
-        self.hist = hist if hist is not None else self.make_history(w, seed)
+        self.hist = hist if hist is not None else history(w, seed, bulk=with_bulk)
+        if with_bulk:
+            hs = [np.concatenate([lay.hist[b], lay.bulk[b]]) for b in range(w.batch)]
+        else:
+            hs = lay.hist
+        self.hist_slots = torch.from_numpy(np.concatenate(hs).astype(np.int64))
         if fmt in STATIC:
             ks, vs = self.static_scales(self.hist, fmt == "int8c")
             self.cache = kvq.LayerCache.allocate(fmt, d, k_static=ks.to(dev), v_static=vs.to(dev))
@@ -218,19 +288,18 @@ class Setup:
             self.cache = kvq.LayerCache.allocate(fmt, d)
         self.tables = torch.from_numpy(self.tables_np).to(dev)
         self.fill()
-        # per-step inputs, resident in HBM
+        # per-step inputs, resident in HBM; the steps follow the bulk append
+        # whether or not the fill holds it
         self.q, self.k, self.v, self.slots, self.ctx = [], [], [], [], []
-        ctx = self.ctx0.copy()
         for s in range(steps):
             q, k, v = WL.step_inputs(w, s, seed)
             self.q.append(q.to(dev))
             self.k.append(k.to(dev))
             self.v.append(v.to(dev))
-            sl = self.tables_np[np.arange(w.batch), ctx // 16].astype(np.int64) * 16 + ctx % 16
-            self.slots.append(torch.from_numpy(sl).to(dev))
-            ctx = ctx + 1
-            self.ctx.append(torch.from_numpy(ctx.astype(np.int32)).to(dev))
-        self.ctx_np = [self.ctx0 + s + 1 for s in range(steps)]
+            self.slots.append(torch.from_numpy(np.asarray(lay.steps[s], dtype=np.int64)).to(dev))
+        self.ctx_np = [self.ctx0 + (0 if with_bulk else w.bulk_append) + s + 1 for s in range(steps)]
+        for c in self.ctx_np:
+            self.ctx.append(torch.from_numpy(c.astype(np.int32)).to(dev))
         self.max_ctx = int(self.ctx_np[-1].max())
         self.ws = self.cache.workspace(w.batch, self.max_ctx)
         self.out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
@@ -246,36 +315,13 @@ class Setup:
             out.append((a / 127.0).to(torch.bfloat16).contiguous())
         return out
 
-    @staticmethod
-    def make_history(w, seed):
-        """BF16 K/V of every sequence's cached tokens (history + bulk append),
-        concatenated, with their slots."""
-        tables, _ = WL.block_tables(w, seed)
-        ctx = WL.context_lengths(w, seed)
-        ks, vs, ss = [], [], []
-        for b in range(w.batch):
-            k, v = WL.kv_history(w, b, seed)
-            ks.append(k)
-            vs.append(v)
-            pos = np.arange(ctx[b])
-            if w.bulk_append:
-                kb, vb = WL.kv_bulk(w, b, seed)
-                ks.append(kb)
-                vs.append(vb)
-                pos = np.arange(ctx[b] + w.bulk_append)
-            ss.append(torch.from_numpy(tables[b][pos // 16].astype(np.int64) * 16 + pos % 16))
-        return torch.cat(ks), torch.cat(vs), torch.cat(ss)
-
     def fill(self, chunk=1 << 16):
-        K, V, S = self.hist
+        K, V = self.hist
+        S = self.hist_slots
         dev = torch.device("cuda")
         for a in range(0, S.numel(), chunk):
             self.cache.append(K[a:a + chunk].to(dev), V[a:a + chunk].to(dev), S[a:a + chunk].to(dev))
         torch.cuda.synchronize()
-
-    def reset_tail(self):
-        """Nothing to undo: step s appends at position ctx0 + s, so re-running the
-        steps overwrites the same slots with the same values."""
 
     # one step of the hot path, with events between its phases
     def step(self, s, ev=None):
@@ -422,50 +468,62 @@ def e2e_loop(st, steps, warmup, world, flush):
     return ms, h2d, d2h
 
 
-def verify_rate(st, flush, n_query=2, reps=10, warmup=3):
-    """Multi-query decode (speculative verification, kvq_decode_verify) over the
-    cache as the first timed step leaves it: the last n_query cached tokens of
-    every sequence are the positions being verified. L2 flushed before every
-    timed call. None when the GQA group times n_query exceeds 8."""
+def multi_query_rate(st, flush, n_query, call="verify", reps=10, warmup=3):
+    """Multi-query attention over the cache as the first timed step leaves it:
+    the last n_query cached tokens of every sequence are the positions
+    (speculative verification, kvq_decode_verify) or the prefill chunk
+    (kvq_prefill_attn). L2 flushed before every timed call. Reports KV bytes
+    over time (the pages are read from HBM once per KV head; row groups beyond
+    the first re-read them, mostly from L2) and the attention FLOPs."""
     w, kvq, c = st.w, st.kvq, st.cache
-    if w.group * n_query > 8:
-        return None
     g = torch.Generator(device="cuda").manual_seed(7)
     q = torch.randn(w.batch, w.n_q_heads, n_query, w.head_dim, generator=g,
                     device="cuda").to(torch.bfloat16)
     out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
     import ctypes
-    n = kvq.lib().kvq_decode_verify_workspace_bytes(w.batch, n_query, st.max_ctx, 0,
-                                                    kvq.FMT[st.fmt], ctypes.byref(st.dims))
+    size_fn = (kvq.lib().kvq_decode_verify_workspace_bytes if call == "verify"
+               else kvq.lib().kvq_prefill_attn_workspace_bytes)
+    n = size_fn(w.batch, n_query, st.max_ctx, 0, kvq.FMT[st.fmt], ctypes.byref(st.dims))
     ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    fn = kvq.decode_verify if call == "verify" else kvq.prefill_attn
 
-    def call():
-        kvq.decode_verify(q, c.k, c.v, c.k_scale, c.v_scale, st.tables, st.ctx[0], st.max_ctx,
-                          w.sm_scale, out, st.fmt, st.dims, workspace=ws)
+    def run():
+        fn(q, c.k, c.v, c.k_scale, c.v_scale, st.tables, st.ctx[0], st.max_ctx, w.sm_scale, out,
+           st.fmt, st.dims, workspace=ws)
 
     for _ in range(warmup):
-        call()
+        run()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(reps)]
     for a, b in evs:
         flush.zero_()
         a.record()
-        call()
+        run()
         b.record()
     torch.cuda.synchronize()
     ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
     kv, alg = kv_bytes_per_step(st.ctx_np[0], w, st.fmt)
     hbm, _ = peaks()
+    ctx = np.asarray(st.ctx_np[0], dtype=np.float64)
+    # causal: position j sees ctx - n_query + 1 + j tokens
+    seen = float(np.sum(np.maximum(0, ctx[:, None] - n_query + 1 + np.arange(n_query)[None, :])))
+    flops = 4.0 * w.n_q_heads * w.head_dim * seen
     return {"n_query": n_query, "ms": ms, "kv_gbs": kv / (ms * 1e-3) / 1e9,
-            "frac_of_peak": kv / (ms * 1e-3) / 1e9 / hbm,
+            "kv_frac_of_peak": kv / (ms * 1e-3) / 1e9 / hbm,
             "positions_per_s": w.batch * n_query / (ms * 1e-3),
-            "what": "decode partials + merge for n_query positions per sequence, pages read once"}
+            "attention_tflops": flops / (ms * 1e-3) / 1e12,
+            "row_groups_per_kv_head": (w.group * n_query) // max(
+                g_ for g_ in (8, 4, 2, 1) if (w.group * n_query) % g_ == 0),
+            "what": ("speculative verification: " if call == "verify" else "prefill chunk: ")
+            + "decode partials + merge for n_query causal positions per sequence"}
 
 
 def bulk_append_rate(st, tokens=32768, reps=5):
-    """Append throughput for one bulk call of `tokens` tokens (prefill-style)."""
-    K, V, S = st.hist
+    """Append throughput for one bulk call of the first `tokens` cached tokens
+    (prefill-style, re-appended to their own slots)."""
+    K, V = st.hist
+    S = st.hist_slots
     n = min(tokens, S.numel())
     dev = torch.device("cuda")
     k, v, s = K[:n].to(dev), V[:n].to(dev), S[:n].to(dev)
@@ -547,77 +605,97 @@ def cpu_model():
     return None
 
 
-def oracle_decode_sample(w, fmt, seed, budget_s=12.0):
-    """Time the CPU oracle on a bounded sample of the workload: for sequences in
-    order until the time budget is spent, quantize the sequence's cached K/V into
+ORACLE_SAMPLE_TOKENS = 65536
+_SAMPLE_INPUTS = {}
+
+
+def oracle_sample(w, seed):
+    """The fixed CPU sample of a workload: its first sequences, in order, until
+    they hold ORACLE_SAMPLE_TOKENS cached tokens (at least one sequence)."""
+    ctx = WL.context_lengths(w, seed) + w.bulk_append
+    n, tok = 0, 0
+    while n < w.batch and (n == 0 or tok < ORACLE_SAMPLE_TOKENS):
+        tok += int(ctx[n])
+        n += 1
+    return n
+
+
+def oracle_decode_sample(w, fmt, seed, threads=None):
+    """Time the CPU oracle on the fixed sample of the workload (oracle_sample):
+    for each sampled sequence, quantize its cached K/V and the step token into
     an oracle pool (append) and run the decode step's attention over it for all
-    query heads (dequantising gather + FP64 softmax attention). Returns
-    (decode KV GB/s, append tok/s, sample description, threads)."""
+    query heads (dequantising gather + FP64 softmax attention). `threads` caps
+    the BLAS / OpenMP threads (None: all the host's). Returns (decode KV GB/s,
+    append tok/s, sample description, threads used)."""
+    from threadpoolctl import threadpool_info, threadpool_limits
+
     from oracle import attention as OA
     from oracle import paged as OP
-    tables, nb = WL.block_tables(w, seed)
-    ctx = WL.context_lengths(w, seed)
-    q, kn, vn = WL.step_inputs(w, 0, seed)
+    key = (w.name, seed)
+    if key not in _SAMPLE_INPUTS:                 # drawn once, outside the timing
+        q, kn, vn = WL.step_inputs(w, 0, seed)
+        n_seq = oracle_sample(w, seed)
+        seqs = []
+        for b in range(n_seq):
+            k, v = WL.kv_history(w, b, seed)
+            if w.bulk_append:
+                kb, vb = WL.kv_bulk(w, b, seed)
+                k, v = torch.cat([k, kb]), torch.cat([v, vb])
+            seqs.append((torch.cat([k, kn[b:b + 1]]).float().numpy(),
+                         torch.cat([v, vn[b:b + 1]]).float().numpy()))
+        _SAMPLE_INPUTS.clear()
+        _SAMPLE_INPUTS[key] = (q, seqs)
+    q, seqs = _SAMPLE_INPUTS[key]
+    n_seq = len(seqs)
     t_app = t_dec = 0.0
     n_tok = 0
     kv_bytes = 0
-    done = []
-    t_start = time.perf_counter()
-    for b in range(w.batch):
-        if time.perf_counter() - t_start > budget_s and done:
-            break
-        k, v = WL.kv_history(w, b, seed)
-        k = torch.cat([k, kn[b:b + 1]]).float().numpy()
-        v = torch.cat([v, vn[b:b + 1]]).float().numpy()
-        n = k.shape[0]
-        pages = (n + 15) // 16
-        if fmt in STATIC:
-            from oracle import formats as OF
-            per_channel = fmt == "int8c"
-            pool = OP.LogicalPool(fmt, pages, w.n_kv_heads, 16, w.head_dim,
-                                  k_static=OF.int8_static_calibrate(k, per_channel),
-                                  v_static=OF.int8_static_calibrate(v, per_channel))
-        else:
-            pool = OP.LogicalPool(fmt, pages, w.n_kv_heads, 16, w.head_dim)
-        row = np.arange(pages)
-        t0 = time.perf_counter()
-        pool.append(k, v, OP.slot_of(row, np.arange(n), 16))
-        t1 = time.perf_counter()
-        K, V = pool.gather(row, n)
-        OA.decode_attention(q[b:b + 1].float().numpy(), [(K, V)], w.sm_scale, w.n_kv_heads)
-        t2 = time.perf_counter()
-        t_app += t1 - t0
-        t_dec += t2 - t1
-        n_tok += n
-        kv_bytes += n * w.n_kv_heads * (2 * w.head_dim * ELEM[fmt] + META_BYTES[fmt])
-        done.append(b)
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        threads = 1
-    desc = (f"{len(done)} of {w.batch} sequences ({n_tok} tokens, all {w.n_q_heads} query heads): "
+    with threadpool_limits(limits=threads):
+        used = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        for b in range(n_seq):
+            k, v = seqs[b]
+            n = k.shape[0]
+            pages = (n + 15) // 16
+            if fmt in STATIC:
+                from oracle import formats as OF
+                per_channel = fmt == "int8c"
+                pool = OP.LogicalPool(fmt, pages, w.n_kv_heads, 16, w.head_dim,
+                                      k_static=OF.int8_static_calibrate(k, per_channel),
+                                      v_static=OF.int8_static_calibrate(v, per_channel))
+            else:
+                pool = OP.LogicalPool(fmt, pages, w.n_kv_heads, 16, w.head_dim)
+            row = np.arange(pages)
+            t0 = time.perf_counter()
+            pool.append(k, v, OP.slot_of(row, np.arange(n), 16))
+            t1 = time.perf_counter()
+            K, V = pool.gather(row, n)
+            OA.decode_attention(q[b:b + 1].float().numpy(), [(K, V)], w.sm_scale, w.n_kv_heads)
+            t2 = time.perf_counter()
+            t_app += t1 - t0
+            t_dec += t2 - t1
+            n_tok += n
+            kv_bytes += n * w.n_kv_heads * (2 * w.head_dim * ELEM[fmt] + META_BYTES[fmt])
+    desc = (f"{n_seq} of {w.batch} sequences ({n_tok} tokens, all {w.n_q_heads} query heads): "
             f"oracle append of their cached tokens + one decode step")
-    return kv_bytes / t_dec / 1e9, n_tok / t_app, desc, threads
+    return kv_bytes / t_dec / 1e9, n_tok / t_app, desc, used
 
 
 def run_reference(args):
-    """The oracle as the reference arm: same metric/unit/config, each step a
-    bounded sample of the workload on the host cores."""
+    """The oracle as the reference arm: same metric/unit/config, each step the
+    workload's fixed CPU sample (oracle_sample) on all the host's cores."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     w = WL.WORKLOADS[args.workload]
     fmt = args.fmt or w.fmt
-    vals = []
+    vals, tok = [], []
     t0 = time.perf_counter()
-    # each step samples the workload for a bounded time so that the whole run
-    # stays near two minutes whatever --steps / --warmup are
-    budget = min(args.ref_budget, 120.0 / max(1, args.warmup + args.steps))
+    desc, threads = "", 1
     for s in range(args.warmup + args.steps):
-        gbs, tok_s, desc, threads = oracle_decode_sample(w, fmt, seed=0, budget_s=budget)
+        gbs, tok_s, desc, threads = oracle_decode_sample(w, fmt, seed=0)
         if s >= args.warmup:
             vals.append(gbs)
+            tok.append(tok_s)
     value = float(np.mean(vals))
     line = {"impl": "reference", "metric": metric_name(fmt), "value": value, "unit": "GB/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -626,10 +704,113 @@ def run_reference(args):
             "dtype": "f64", "data": "synthetic (seeded)",
             "config": config_block(w, fmt, l2="host run (no GPU)"),
             "cpu_baseline": {"kind": "oracle", "value": value, "unit": "GB/s", "cores": threads,
-                             "sample": desc, "cpu_model": cpu_model()},
+                             "sample": desc, "append_tok_per_s": float(np.mean(tok)),
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def step_metrics(st, t, fmt, world, hbm_peak, steps):
+    """The per-format numbers of one Setup timed by timed_loop: step and decode
+    throughput, fractions of the HBM peak (decode = partials + merge, as the
+    roofline counts it; the partials alone beside it), append rates."""
+    w = st.w
+    kv = float(np.mean([kv_bytes_per_step(st.ctx_np[i % st.steps], w, fmt)[0] for i in range(steps)]))
+    alg = float(np.mean([kv_bytes_per_step(st.ctx_np[i % st.steps], w, fmt)[1] for i in range(steps)]))
+    smax = max_over_ranks(t["step"], world)
+    dec = t["decode"] + t["merge"]
+    return {
+        "kv_gbs_step": sum_over_ranks(kv, world) / (smax * 1e-3) / 1e9,
+        "kv_frac_of_peak_step": kv / (smax * 1e-3) / 1e9 / hbm_peak,
+        "decode_gbs": alg / (dec * 1e-3) / 1e9,
+        "decode_frac_of_peak": alg / (dec * 1e-3) / 1e9 / hbm_peak,
+        "decode_partial_frac_of_peak": alg / (t["decode"] * 1e-3) / 1e9 / hbm_peak,
+        "decode_seqs_per_s": sum_over_ranks(w.batch, world) / (dec * 1e-3),
+        "step_seqs_per_s": sum_over_ranks(w.batch, world) / (smax * 1e-3),
+        "append_tok_per_s_step": sum_over_ranks(w.batch, world) / (t["append"] * 1e-3),
+        "ms": {k: round(v, 5) for k, v in t.items() if k != "launches"},
+        "kv_bytes_per_step": kv,
+        "alg_bytes_per_step": alg,
+    }
+
+
+def long_context_run(w, fmt, seed, hist, bulk_kv, layout, hbm_peak, flush):
+    """The long-context workload as specified: the cached history is filled
+    untimed; then ONE timed bulk append of every sequence's bulk tokens (w.batch
+    x w.bulk_append tokens in one call, slots in all sequences, prefill-style
+    quantize), then w.decode_steps timed decode steps, each appending one token
+    per sequence before its decode partials and merge. Both are first run once
+    untimed with the same values into the same slots, so each step sees the same
+    cache. L2 is flushed before the bulk append; each decode step reads far more
+    than L2 holds (no flush between steps)."""
+    st = Setup(w, fmt, w.decode_steps, seed, hist=hist, layout=layout, with_bulk=False)
+    dev = torch.device("cuda")
+    kb, vb = bulk_kv[0].to(dev), bulk_kv[1].to(dev)
+    sb = torch.from_numpy(np.concatenate(layout.bulk).astype(np.int64)).to(dev)
+    st.cache.append(kb, vb, sb)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush.zero_()
+    e0.record()
+    st.cache.append(kb, vb, sb)
+    e1.record()
+    torch.cuda.synchronize()
+    bulk_ms = e0.elapsed_time(e1)
+    n_bulk = sb.numel()
+    del kb, vb
+    for s in range(w.decode_steps):                    # untimed pass
+        st.step(s)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(w.decode_steps)]
+    for s in range(w.decode_steps):
+        evs[s][0].record()
+        st.step(s, evs[s])
+        evs[s][3].record()
+    torch.cuda.synchronize()
+    t = {"step": float(np.mean([e[0].elapsed_time(e[3]) for e in evs])),
+         "append": float(np.mean([e[0].elapsed_time(e[1]) for e in evs])),
+         "decode": float(np.mean([e[1].elapsed_time(e[2]) for e in evs])),
+         "merge": float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))}
+    r = step_metrics(st, t, fmt, 1, hbm_peak, w.decode_steps)
+    by = n_bulk * append_bytes_per_token(w, fmt)
+    r["bulk_append"] = {"tokens": n_bulk, "sequences": w.batch, "ms": bulk_ms,
+                        "tok_per_s": n_bulk / (bulk_ms * 1e-3), "gbs": by / (bulk_ms * 1e6),
+                        "frac_of_peak": by / (bulk_ms * 1e6) / hbm_peak}
+    r["decode_steps"] = w.decode_steps
+    r["context"] = [int(st.ctx_np[0].min()), int(st.ctx_np[-1].max())]
+    r["l2"] = "flushed before the bulk append; each step reads > L2"
+    del st
+    torch.cuda.empty_cache()
+    return r
+
+
+def configs_block(args, seed, hbm_peak, flush):
+    """Workloads beside the headline, each as its specification runs it."""
+    out = {}
+    w = WL.WORKLOADS["long-128k"]
+    hist = history(w, seed, bulk=False)
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        parts = list(ex.map(lambda b: WL.kv_bulk(w, b, seed), range(w.batch)))
+    bulk_kv = (torch.cat([p[0] for p in parts]), torch.cat([p[1] for p in parts]))
+    lay = Layout(w, seed, "fp8")
+    long_res = {}
+    for f in ("fp8", "int8", "bf16"):
+        long_res[f] = long_context_run(w, f, seed, hist, bulk_kv, lay, hbm_peak, flush)
+    out["long-128k"] = dict(long_res, workload=config_block(w, "fp8", "")["workload"])
+    del hist, bulk_kv
+    w = WL.WORKLOADS["mixed-serving-fp8"]
+    steps = min(args.steps, 10)
+    wb = dataclasses.replace(w, decode_steps=max(w.decode_steps, steps + args.warmup))
+    st = Setup(wb, "fp8", steps + args.warmup, seed)
+    t = timed_loop(st, steps, args.warmup, 1, flush)
+    r = step_metrics(st, t, "fp8", 1, hbm_peak, steps)
+    r["tables"] = st.layout.source
+    out["mixed-serving-fp8"] = {"fp8": r, "workload": config_block(w, "fp8", "")["workload"]}
+    del st
+    torch.cuda.empty_cache()
+    return out
 
 
 def metric_name(fmt):
@@ -661,8 +842,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WL.WORKLOADS))
     ap.add_argument("--fmt", default=None, choices=["fp8", "int8", "bf16", "e5m2", "int8c", "int8t"])
     ap.add_argument("--no-formats", action="store_true", help="skip the per-format comparison")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' block")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
-    ap.add_argument("--ref-budget", type=float, default=10.0)
     ap.add_argument("--bulk-append", choices=["aligned", "continued"], default=None,
                     help="only time one bulk append of 32,768 tokens and print its line")
     ap.add_argument("--reps", type=int, default=5, help="timed calls of --bulk-append")
@@ -684,8 +865,9 @@ def main():
     hbm_peak, peak_kind = peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
-    hist = Setup.make_history(wb, seed)
-    st = Setup(wb, fmt, steps_needed, seed, hist=hist)
+    hist = history(wb, seed)
+    lay = Layout(wb, seed, fmt)
+    st = Setup(wb, fmt, steps_needed, seed, hist=hist, layout=lay)
     clocks = ClockSampler(local)
     clocks.start()
     t = timed_loop(st, args.steps, args.warmup, world, flush)        # per-phase events
@@ -693,22 +875,25 @@ def main():
     clk = clocks.stop()
 
     step_ms = max_over_ranks(tg, world)
-    dec_ms = max_over_ranks(t["decode"], world)
-    # bytes of the timed steps (contexts grow by one per step)
-    kv_list, all_list = zip(*[kv_bytes_per_step(st.ctx_np[i % st.steps], wb, fmt)
-                              for i in range(args.steps)])
-    kv_step = float(np.mean(kv_list))
-    alg_step = float(np.mean(all_list))
+    head = step_metrics(st, t, fmt, world, hbm_peak, args.steps)
+    kv_step = head["kv_bytes_per_step"]
+    alg_step = head["alg_bytes_per_step"]
     kv_total = sum_over_ranks(kv_step, world)
     value = kv_total / (step_ms * 1e-3) / 1e9
-    achieved = alg_step / (t["decode"] * 1e-3) / 1e9
+    dec_ms = max_over_ranks(t["decode"] + t["merge"], world)
+    achieved = alg_step / (dec_ms * 1e-3) / 1e9
     seqs_s = sum_over_ranks(wb.batch, world) / (step_ms * 1e-3)
     app_tok_s = sum_over_ranks(wb.batch, world) / (max_over_ranks(t["append"], world) * 1e-3)
     bulk_tok_s, bulk_ms, bulk_n = bulk_append_rate(st)
+    verify, prefill = {}, {}
     try:
-        verify = verify_rate(st, flush)
+        verify = multi_query_rate(st, flush, 4, "verify")
     except Exception as e:                        # reported, never fatal to the main line
         verify = {"error": f"{type(e).__name__}: {e}"[:200]}
+    try:
+        prefill = multi_query_rate(st, flush, 64, "prefill", reps=3, warmup=1)
+    except Exception as e:
+        prefill = {"error": f"{type(e).__name__}: {e}"[:200]}
 
     e2e_ms, h2d, d2h = e2e_loop(st, args.steps, args.warmup, world, flush)
     e2e_ms = max_over_ranks(e2e_ms, world)
@@ -723,24 +908,11 @@ def main():
             else:
                 del st
                 torch.cuda.empty_cache()
-                stf = Setup(wb, f, steps_needed, seed, hist=hist)
+                stf = Setup(wb, f, steps_needed, seed, hist=hist, layout=lay)
                 tf = timed_loop(stf, args.steps, args.warmup, world, flush)
-            kvf = float(np.mean([kv_bytes_per_step(stf.ctx_np[i % stf.steps], wb, f)[0]
-                                 for i in range(args.steps)]))
-            algf = float(np.mean([kv_bytes_per_step(stf.ctx_np[i % stf.steps], wb, f)[1]
-                                  for i in range(args.steps)]))
             bt, _, _ = bulk_append_rate(stf)
-            smax = max_over_ranks(tf["step"], world)
-            formats[f] = {
-                "kv_gbs_step": sum_over_ranks(kvf, world) / (smax * 1e-3) / 1e9,
-                "decode_kernel_gbs": algf / (tf["decode"] * 1e-3) / 1e9,
-                "decode_frac_of_peak": algf / (tf["decode"] * 1e-3) / 1e9 / hbm_peak,
-                "decode_seqs_per_s": sum_over_ranks(wb.batch, world) / (smax * 1e-3),
-                "append_tok_per_s_step": sum_over_ranks(wb.batch, world) / (tf["append"] * 1e-3),
-                "append_tok_per_s_bulk": bt,
-                "ms": {k: round(v, 5) for k, v in tf.items() if k != "launches"},
-                "kv_bytes_per_step": kvf,
-            }
+            formats[f] = dict(step_metrics(stf, tf, f, world, hbm_peak, args.steps),
+                              append_tok_per_s_bulk=bt)
             # step 0's attention again, in FP32: every format holds the same tokens
             # up to that context, so the outputs compare directly
             outs[f] = stf.cache.decode(stf.q[0], stf.tables, stf.ctx[0], stf.max_ctx,
@@ -756,12 +928,20 @@ def main():
                 "max_abs": float(dev.max()), "mean_abs": float(dev.mean()),
                 "rel_l2": float((outs[f] - outs["bf16"]).norm() / max(float(outs["bf16"].norm()), 1e-30)),
                 "mean_abs_ref": float(ref.mean()), "step": 0}
+    del st, hist
+    torch.cuda.empty_cache()
+
+    configs = None
+    if world == 1 and not args.no_configs:
+        configs = configs_block(args, seed, hbm_peak, flush)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         gbs, tok_s, desc, threads = oracle_decode_sample(wb, fmt, seed=0)
+        gbs1, tok1, _, _ = oracle_decode_sample(wb, fmt, seed=0, threads=1)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
-               "append_tok_per_s": tok_s, "cpu_model": cpu_model()}
+               "append_tok_per_s": tok_s, "cpu_model": cpu_model(),
+               "single_thread": {"value": gbs1, "append_tok_per_s": tok1, "cores": 1}}
 
     line = {
         "metric": metric_name(fmt), "value": value, "unit": "GB/s", "n_gpus": world,
@@ -771,22 +951,27 @@ def main():
         "config": dict(config_block(wb, fmt, l2="flushed before every timed step (256 MB write)"),
                        launch="each timed step is one CUDA graph replay of its append, decode "
                               "and merge launches; phase_ms and the per-format table time the "
-                              "same steps launched one by one with events between the phases"),
+                              "same steps launched one by one with events between the phases",
+                       tables=lay.source),
         "decode_seqs_per_s": seqs_s, "append_tok_per_s_step": app_tok_s,
         "append_tok_per_s_bulk": bulk_tok_s, "kv_frac_of_peak_step": value / world / hbm_peak,
         "phase_ms": {k: round(v, 5) for k, v in t.items() if k != "launches"},
         "ms_per_step_eager": t["step"],
-        "roofline": {"bound": "hbm", "kernel": "decode partial (kvq_decode_partial)",
+        "roofline": {"bound": "hbm", "kernel": "decode attention: partials + merge "
+                                               "(kvq_decode_partial + kvq_decode_merge)",
                      "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                     "partial_only_frac": head["decode_partial_frac_of_peak"],
                      "alg_bytes_per_launch": alg_step,
                      "traffic": measured_traffic(w.name, fmt)},
         "e2e": {"value": e2e_val, "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": t["launches"],
         "verify": verify,
+        "prefill": prefill,
         "clocks": clk,
         "formats": formats,
+        "configs": configs,
         "cpu_baseline": cpu,
     }
     if rank == 0:

@@ -338,10 +338,11 @@ int kvq_decode_attn_noalloc(const void* q, int32_t batch, const void* k_cache,
  * q    device, [batch][n_q_heads][n_query][head_dim] BF16.
  * out  device, [batch][n_q_heads][n_query][head_dim], BF16 or FP32 per out_dtype.
  * The cache, scales, block tables and the other arguments are those of
- * kvq_decode_attn. The K/V of a (sequence, KV head) are read once for all
- * n_query positions of all G query heads: the positions are extra heads of
- * the GQA group. Supported when G * n_query is 1, 2, 4 or 8
- * (KVQ_ERR_UNSUPPORTED otherwise; n_query outside 1..8 is KVQ_ERR_ARG).
+ * kvq_decode_attn. n_query in 1 .. 1024 (KVQ_ERR_ARG otherwise). The G *
+ * n_query query rows of a KV head are taken in groups of up to 8 rows (the
+ * largest of 8, 4, 2, 1 that divides G * n_query); each group streams the KV
+ * head's pages once, and the groups of one KV head run side by side on the
+ * GPU, so their repeated reads of a page mostly come from L2.
  * workspace  at least kvq_decode_verify_workspace_bytes(...) bytes; contents on
  *            entry do not matter.
  */
@@ -355,6 +356,36 @@ int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void*
                       kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
                       int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
                       kvq_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Chunked-prefill attention over the quantized cache.                         */
+/* [GUIDE] "Core concepts 1)": prefill processes a prompt's tokens together,   */
+/* decode one token at a time against the cache. A long prompt prefilled in    */
+/* chunks appends each chunk's K/V (kvq_append, the bulk path) and then lets   */
+/* the chunk's queries attend, causally, to everything cached so far: the     */
+/* earlier chunks through the quantized pages and the chunk itself.           */
+/* ------------------------------------------------------------------------ */
+/*
+ * The chunk's chunk_len tokens are the last chunk_len tokens of each
+ * sequence's context, already appended (context_lens[b] counts them). Chunk
+ * position j attends to tokens 0 .. context_lens[b] - chunk_len + j (the same
+ * rule as kvq_decode_verify with n_query = chunk_len, and the same kernel):
+ *   out[b][h][j] = softmax_t(sm_scale * q[b][h][j] . K_b[t][h/G]) weighted sum
+ *                  of V_b[t][h/G] over t < context_lens[b] - chunk_len + 1 + j.
+ * q    device, [batch][n_q_heads][chunk_len][head_dim] BF16 (head-major).
+ * out  device, the same shape, BF16 or FP32 per out_dtype.
+ * chunk_len in 1 .. 1024; the other arguments and errors are those of
+ * kvq_decode_verify. workspace: kvq_prefill_attn_workspace_bytes(...) bytes.
+ */
+size_t kvq_prefill_attn_workspace_bytes(int32_t batch, int32_t chunk_len, int32_t max_context_len,
+                                        int32_t partition_tokens, kvq_fmt fmt,
+                                        const kvq_dims* dims);
+int kvq_prefill_attn(const void* q, int32_t batch, int32_t chunk_len, const void* k_cache,
+                     const void* v_cache, const void* const* scales, const int32_t* block_tables,
+                     const int32_t* context_lens, int32_t max_context_len, float sm_scale,
+                     void* out, kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                     int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                     kvq_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Device error word and the decode wait bound.                               */

@@ -36,7 +36,7 @@ int device_sm_count() {
 // into at most 15 runs. The persistent decode kernel then spreads any batch
 // over every resident CTA while the workspace stays at 16 partials per row.
 int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kvq_dims* d,
-              DecodePlan* plan) {
+              DecodePlan* plan, int32_t n_query) {
   if (batch < 0 || max_ctx < 0 || partition_tokens < 0) return KVQ_ERR_ARG;
   if (partition_tokens % kTileTokens != 0) return KVQ_ERR_ARG;
   int64_t part = partition_tokens;
@@ -48,10 +48,12 @@ int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kv
   plan->partition = int32_t(part);
   plan->max_splits = int32_t(splits);
   plan->slots = int32_t(splits + 1);
-  const size_t rows = size_t(batch) * d->n_q_heads * size_t(plan->slots);
+  int gp = 1;
+  const int groups = row_groups(d->n_q_heads / d->n_kv_heads * n_query, &gp);
+  const size_t rows = size_t(batch) * d->n_q_heads * size_t(n_query) * size_t(plan->slots);
   plan->o_bytes = round256(rows * d->head_dim * sizeof(float));
   plan->ml_bytes = round256(rows * 2 * sizeof(float));
-  plan->cnt_bytes = round256(size_t(batch) * d->n_kv_heads * sizeof(int32_t));
+  plan->cnt_bytes = round256(size_t(batch) * d->n_kv_heads * size_t(groups) * sizeof(int32_t));
   plan->total = plan->o_bytes + plan->ml_bytes + plan->cnt_bytes;
   return KVQ_OK;
 }
@@ -64,13 +66,13 @@ std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 long long decode_wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
 
 int check_decode_common(int32_t batch, int32_t max_ctx, int32_t partition_tokens, kvq_fmt fmt,
-                        const kvq_dims* dims, DecodePlan* plan) {
+                        const kvq_dims* dims, DecodePlan* plan, int32_t n_query) {
   if (!fmt_valid(fmt)) return KVQ_ERR_ARG;
   int rc = check_dims(dims);
   if (rc != KVQ_OK) return rc;
-  if (batch < 0 || max_ctx < 0) return KVQ_ERR_ARG;
+  if (batch < 0 || max_ctx < 0 || n_query < 1) return KVQ_ERR_ARG;
   if (int64_t(max_ctx) > int64_t(dims->max_blocks_per_seq) * dims->block_size) return KVQ_ERR_ARG;
-  return make_plan(batch, max_ctx, partition_tokens, dims, plan);
+  return make_plan(batch, max_ctx, partition_tokens, dims, plan, n_query);
 }
 
 int check_decode_inputs(const void* q, const void* kc, const void* vc, const void* const* scales,
@@ -202,40 +204,25 @@ int kvq_device_error(uint32_t* flags, int clear) {
   return *flags ? KVQ_ERR_DEVICE : KVQ_OK;
 }
 
-// Multi-query decode: the n_query positions of a query head are the heads
-// n_query * h .. n_query * h + n_query - 1 of a group n_query times larger, so
-// the single-query machinery runs on dims with n_q_heads * n_query query heads
-// and the kernel adds the causal limit of each position.
+// Multi-query decode: the n_query positions of a query head are the rows
+// n_query * h .. n_query * h + n_query - 1 of its KV head's G * n_query rows.
+// The decode kernel takes those rows in groups of up to 8 (row_groups), each
+// a virtual head of the work list with the KV head's pages, and adds the
+// causal limit of each position; the plan, the launch and the merge see
+// n_q_heads * n_query query rows per sequence.
 namespace {
-int verify_dims(int32_t n_query, const kvq_dims* dims, kvq_dims* eff) {
-  if (!dims || n_query < 1 || n_query > 8) return KVQ_ERR_ARG;
-  *eff = *dims;
-  eff->n_q_heads = dims->n_q_heads * n_query;
-  return KVQ_OK;
-}
-}  // namespace
+constexpr int32_t kMaxQueryPositions = 1024;
 
-size_t kvq_decode_verify_workspace_bytes(int32_t batch, int32_t n_query, int32_t max_context_len,
-                                         int32_t partition_tokens, kvq_fmt fmt,
-                                         const kvq_dims* dims) {
-  kvq_dims eff;
-  if (verify_dims(n_query, dims, &eff) != KVQ_OK) return 0;
-  return kvq_decode_workspace_bytes(batch, max_context_len, partition_tokens, fmt, &eff);
-}
-
-int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void* k_cache,
-                      const void* v_cache, const void* const* scales,
-                      const int32_t* block_tables, const int32_t* context_lens,
-                      int32_t max_context_len, float sm_scale, void* out,
-                      kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
-                      int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
-                      kvq_stream_t stream) {
-  kvq_dims eff;
-  int rc = verify_dims(n_query, dims, &eff);
-  if (rc != KVQ_OK) return rc;
+int verify_launch(const void* q, int32_t batch, int32_t n_query, const void* k_cache,
+                  const void* v_cache, const void* const* scales, const int32_t* block_tables,
+                  const int32_t* context_lens, int32_t max_context_len, float sm_scale, void* out,
+                  kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                  int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                  kvq_stream_t stream) {
+  if (n_query < 1 || n_query > kMaxQueryPositions) return KVQ_ERR_ARG;
   DecodePlan plan;
-  rc = check_decode_common(batch, max_context_len, partition_tokens, fmt, &eff, &plan);
-  if (rc != KVQ_OK) return rc;                 // includes G * n_query outside {1, 2, 4, 8}
+  int rc = check_decode_common(batch, max_context_len, partition_tokens, fmt, dims, &plan, n_query);
+  if (rc != KVQ_OK) return rc;
   if (out_dtype != KVQ_OUT_BF16 && out_dtype != KVQ_OUT_F32) return KVQ_ERR_ARG;
   if (batch == 0) return KVQ_OK;
   if (!dev_ok(out)) return KVQ_ERR_ARG;
@@ -245,12 +232,60 @@ int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void*
   if (rc != KVQ_OK) return rc;
   if (!dev_ok(workspace)) return KVQ_ERR_ARG;
   if (workspace_bytes < plan.total) return KVQ_ERR_WORKSPACE;
+  kvq_dims eff = *dims;
+  eff.n_q_heads = dims->n_q_heads * n_query;
   rc = cuda_rc(launch_decode_partial(q, batch, k_cache, v_cache, ks, vs, block_tables, context_lens,
                                      max_context_len, sm_scale, plan, workspace, fmt, eff, stream,
                                      n_query));
   if (rc != KVQ_OK) return rc;
   return cuda_rc(launch_decode_merge(batch, context_lens, max_context_len, out,
                                      out_dtype == KVQ_OUT_F32, workspace, plan, eff, stream));
+}
+
+size_t verify_ws(int32_t batch, int32_t n_query, int32_t max_context_len,
+                 int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims) {
+  if (n_query < 1 || n_query > kMaxQueryPositions) return 0;
+  DecodePlan plan;
+  if (check_decode_common(batch, max_context_len, partition_tokens, fmt, dims, &plan, n_query) !=
+      KVQ_OK)
+    return 0;
+  return plan.total;
+}
+}  // namespace
+
+size_t kvq_decode_verify_workspace_bytes(int32_t batch, int32_t n_query, int32_t max_context_len,
+                                         int32_t partition_tokens, kvq_fmt fmt,
+                                         const kvq_dims* dims) {
+  return verify_ws(batch, n_query, max_context_len, partition_tokens, fmt, dims);
+}
+
+int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void* k_cache,
+                      const void* v_cache, const void* const* scales,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      int32_t max_context_len, float sm_scale, void* out,
+                      kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                      int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                      kvq_stream_t stream) {
+  return verify_launch(q, batch, n_query, k_cache, v_cache, scales, block_tables, context_lens,
+                       max_context_len, sm_scale, out, out_dtype, workspace, workspace_bytes,
+                       partition_tokens, fmt, dims, stream);
+}
+
+size_t kvq_prefill_attn_workspace_bytes(int32_t batch, int32_t chunk_len, int32_t max_context_len,
+                                        int32_t partition_tokens, kvq_fmt fmt,
+                                        const kvq_dims* dims) {
+  return verify_ws(batch, chunk_len, max_context_len, partition_tokens, fmt, dims);
+}
+
+int kvq_prefill_attn(const void* q, int32_t batch, int32_t chunk_len, const void* k_cache,
+                     const void* v_cache, const void* const* scales, const int32_t* block_tables,
+                     const int32_t* context_lens, int32_t max_context_len, float sm_scale,
+                     void* out, kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                     int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
+                     kvq_stream_t stream) {
+  return verify_launch(q, batch, chunk_len, k_cache, v_cache, scales, block_tables, context_lens,
+                       max_context_len, sm_scale, out, out_dtype, workspace, workspace_bytes,
+                       partition_tokens, fmt, dims, stream);
 }
 
 }  // extern "C"

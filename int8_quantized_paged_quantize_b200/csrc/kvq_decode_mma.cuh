@@ -5,12 +5,15 @@
 // zero points are applied to the small S and P tiles instead. Static INT8
 // scales (one per channel, or one per cache) vary along the contraction, so
 // they multiply the query before its split (K) and the finished channel sums
-// (V). Multi-query decode (speculative verification) runs the n_query
-// positions of a query head as extra heads of its group, each with its causal
-// limit. Included by kvq_kernels.cu.
+// (V). Multi-query decode (speculative verification, chunked prefill) runs
+// the n_query positions of a query head as extra rows of its group, each with
+// its causal limit. A KV head's R = G * n_query rows are taken in row groups
+// of G rows (G = 1, 2, 4 or 8, the template parameter; nrg = R / G groups):
+// each group is a "virtual head" of the work list that reads the KV head's
+// pages; plain decode has nrg = 1. Included by kvq_kernels.cu.
 //
-// Work split (persistent, stream-K): the work list is every (sequence b, KV
-// head h, 128-token tile) in order of b, then h, then tile, each (b, h) run
+// Work split (persistent, stream-K): the work list is every (sequence b,
+// virtual head h, 128-token tile) in order of b, then h, then tile, each (b, h) run
 // also costing kPieceCost units for opening and closing its piece. Each of
 // the N resident CTAs takes one contiguous, equal share of the total cost (N
 // is cut so that a share holds at least `unit_tiles` units). A share is a few
@@ -216,7 +219,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kc,
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
-    const int32_t* __restrict__ ctx_lens, int B, int Hk, int NB, int W, int max_ctx,
+    const int32_t* __restrict__ ctx_lens, int B, int Hv, int nrg, int NB, int W, int max_ctx,
     int unit_tiles, int slots, float qk_scale, int per_tensor, int n_query,
     long long wait_limit, float* __restrict__ part_o,
     float* __restrict__ part_ml, int32_t* __restrict__ part_cnt) {
@@ -225,7 +228,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Hq = Hk * G;
+  const int Hq = Hv * G;                                   // query rows of a sequence
+  const int Hk = Hv / nrg;                                 // KV heads
 
   // ------------------------------------------------------------ the share
   // T = total work-list cost; each thread sums the run costs of some sequences
@@ -250,7 +254,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   long long T = 0;
 #pragma unroll
   for (int w = 0; w < 6; ++w) T += red64[w];
-  T *= Hk;
+  T *= Hv;
   const long long N = ll_min(gridDim.x, ll_max(1, T / max(1, unit_tiles)));
   if (T == 0 || blockIdx.x >= N) return;                 // uniform for the CTA
   const long long start = (int64_t(blockIdx.x) * T) / N;
@@ -280,7 +284,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
         total += red64[w];
       }
       const long long lo_t = run + before + incl - tb;          // run cost before sequence bb
-      if (bb < B && tb > 0 && int64_t(Hk) * lo_t <= start && start < int64_t(Hk) * (lo_t + tb)) {
+      if (bb < B && tb > 0 && int64_t(Hv) * lo_t <= start && start < int64_t(Hv) * (lo_t + tb)) {
         misci[0] = bb;
         miscll[0] = lo_t;
       }
@@ -360,7 +364,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   const uint32_t tmem = *tmem_slot;
 
   PieceWalk walk;
-  walk.init(b0, P0, start, end, Hk, ctx_lens, B, max_ctx, W);
+  walk.init(b0, P0, start, end, Hv, ctx_lens, B, max_ctx, W);
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
@@ -378,7 +382,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     auto step = [&](PieceWalk& pw, int& tile) {
       if (pw.done) return;
       if (++tile >= pw.hi) {
-        pw.next(Hk, ctx_lens, B, max_ctx, W);
+        pw.next(Hv, ctx_lens, B, max_ctx, W);
         tile = pw.lo;
       }
     };
@@ -390,7 +394,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       if constexpr (C::MV > 0) {
         const int sblk = __shfl_sync(0xffffffffu, ids, sp & 7);
         if (sp < 8 && sblk >= 0 && sblk < NB) {
-          const int64_t off = (int64_t(sblk) * Hk + h) * C::METAB + sc * 16;
+          const int64_t off = (int64_t(sblk) * Hk + h / nrg) * C::METAB + sc * 16;
           kv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(ks) + off));
           vv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vs) + off));
         }
@@ -423,7 +427,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       const int blk = __shfl_sync(0xffffffffu, id, p8);
       const bool mine = ((mask >> p8) & 1u) != 0u;
       const bool smine = C::MV > 0 && sp < 8 && ((mask >> sp) & 1u) != 0u;
-      const int64_t page = int64_t(blk) * Hk + h;
+      const int64_t page = int64_t(blk) * Hk + h / nrg;
       const uint32_t bytes = uint32_t(__popc(mask)) * uint32_t(C::PAGE);
       bool ok = true;
       // per stage: byte count, the page copies, then the scale stores and the
@@ -523,7 +527,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           if (i > walk.lo) ok = issue_pv(gt - 1);
         }
         if (ok) mma_commit(qfree);                         // this piece's S products are issued
-        walk.next(Hk, ctx_lens, B, max_ctx, W);
+        walk.next(Hv, ctx_lens, B, max_ctx, W);
       }
       if (ok && gt >= 1) issue_pv(gt - 1);
       // every MMA issued so far completes before TMEM is released
@@ -549,14 +553,14 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     auto publish = [&](int idx, const PieceWalk& pw) {
       wk[idx] = pw;
       if (!pw.done) {
-        pinfo[idx * 2] = int(int64_t(blockIdx.x) - cta_of(pw.first_tile(Hk)));
+        pinfo[idx * 2] = int(int64_t(blockIdx.x) - cta_of(pw.first_tile(Hv)));
         pinfo[idx * 2 + 1] = pw.hi == pw.nt;
       }
     };
     if (r == 0) {
       publish(0, walk);
       PieceWalk n = walk;
-      n.next(Hk, ctx_lens, B, max_ctx, W);
+      n.next(Hv, ctx_lens, B, max_ctx, W);
       publish(1, n);
     }
     named_bar_sync(1, 128);
@@ -581,7 +585,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       if constexpr (C::SI) {
 #pragma unroll
         for (int i = 0; i < D / 32; ++i)
-          ksd[i] = none ? 0.f : __bfloat162float(ks[per_tensor ? 0 : qh * D + lane + 32 * i]);
+          ksd[i] = none ? 0.f : __bfloat162float(ks[per_tensor ? 0 : (qh / nrg) * D + lane + 32 * i]);
       }
     };
     // B operand of S (K-major, no swizzle): row n = part * G + g, element
@@ -672,7 +676,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       named_bar_sync(1, 128);                            // all read the cursor; qsc/qsum visible
       if (r == 0) {                                      // piece pc + 2 into this piece's entry
         PieceWalk n = *nxt;
-        if (!n.done) n.next(Hk, ctx_lens, B, max_ctx, W);
+        if (!n.done) n.next(Hv, ctx_lens, B, max_ctx, W);
         publish(pc & 1, n);
       }
       float qs[G], qz[G];
@@ -773,13 +777,15 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           x[g] = valid ? sc * sk * qs[g] : -INFINITY;
         }
         if (n_query > 1) {
-          // multi-query: head g is query position j = g % n_query of its
-          // group's head g / n_query, and position j sees the tokens before
-          // the last n_query - 1 - j of the context
+          // multi-query: row rr = (virtual head % nrg) * G + g of the KV head's
+          // rows is query position j = rr % n_query of query head rr / n_query,
+          // and position j sees the tokens before the last n_query - 1 - j of
+          // the context
           const int after = pctx - 1 - (tile0 + r);       // tokens after this one
+          const int rr0 = (ph_ % nrg) * G;
 #pragma unroll
           for (int g = 0; g < G; ++g)
-            if (n_query - 1 - g % n_query > after) x[g] = -INFINITY;
+            if (n_query - 1 - (rr0 + g) % n_query > after) x[g] = -INFINITY;
         }
         // per-head tile maxima of the four warps, head-major: rb[g][quarter]
         float* rb = red + (gt & 1) * 64;
@@ -986,7 +992,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       // static INT8: the V scale of channel r multiplies the finished sums
       float vsd = 1.f;
       if constexpr (C::SI) {
-        if (r < D) vsd = __bfloat162float(vs[per_tensor ? 0 : ph_ * D + r]);
+        if (r < D) vsd = __bfloat162float(vs[per_tensor ? 0 : (ph_ / nrg) * D + r]);
       }
       // After a wait ran out the piece's sums are incomplete: it writes a
       // marker instead (max +inf, sum and output NaN), so that every output row
@@ -1004,7 +1010,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           part_ml[row * 2 + 1] = good ? L : __int_as_float(0x7fc00000);
         }
       }
-      if (r == 0 && last) part_cnt[pb * Hk + ph_] = slot + 1;
+      if (r == 0 && last) part_cnt[pb * Hv + ph_] = slot + 1;
     }
   }
   tc_fence_before();

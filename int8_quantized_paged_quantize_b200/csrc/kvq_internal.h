@@ -25,6 +25,18 @@ inline bool fmt_valid(int f) { return f >= KVQ_BF16 && f <= KVQ_INT8_TENSOR; }
 // Checks the shape rules of kvq.h. Returns KVQ_OK, KVQ_ERR_ARG or KVQ_ERR_UNSUPPORTED.
 int check_dims(const kvq_dims* d);
 
+// The query rows of one KV head (G query heads x n_query positions) are taken
+// by the decode kernel in row groups of gp rows, gp the largest of 8, 4, 2, 1
+// that divides the row count: each group is one "virtual head" of the work
+// list that reads the KV head's pages. Returns the number of groups per KV
+// head and writes gp.
+inline int row_groups(int rows, int* gp) {
+  int g = 8;
+  while (g > 1 && rows % g != 0) g /= 2;
+  *gp = g;
+  return rows / g;
+}
+
 // Split-K plan of one decode call.
 struct DecodePlan {
   int32_t partition;   // tokens per split (multiple of kTileTokens); the smallest
@@ -33,12 +45,13 @@ struct DecodePlan {
   int32_t slots;       // partial slots per (sequence, query head): max_splits + 1
   size_t o_bytes;      // partial outputs  [B][Hq][slots][D] f32
   size_t ml_bytes;     // partial (max, sum) [B][Hq][slots][2] f32
-  size_t cnt_bytes;    // partials written per (sequence, KV head) [B][Hk] int32
+  size_t cnt_bytes;    // partials written per (sequence, row group) [B][Hk * groups] int32
   size_t total;        // workspace bytes (256-aligned pieces)
 };
-// Fills `plan`; returns KVQ_OK or KVQ_ERR_ARG.
+// Fills `plan` for query rows n_q_heads * n_query per sequence; returns KVQ_OK
+// or KVQ_ERR_ARG.
 int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kvq_dims* d,
-              DecodePlan* plan);
+              DecodePlan* plan, int32_t n_query = 1);
 
 // Number of SMs of the current device (148 if no device can be queried).
 int device_sm_count();
@@ -51,7 +64,7 @@ long long decode_wait_limit();
 // max_context_len against the block-table width) and the split plan.
 // Returns KVQ_OK, KVQ_ERR_ARG or KVQ_ERR_UNSUPPORTED.
 int check_decode_common(int32_t batch, int32_t max_ctx, int32_t partition_tokens, kvq_fmt fmt,
-                        const kvq_dims* dims, DecodePlan* plan);
+                        const kvq_dims* dims, DecodePlan* plan, int32_t n_query = 1);
 // Device-pointer checks of a decode call; *ks, *vs receive the scale arrays.
 int check_decode_inputs(const void* q, const void* kc, const void* vc, const void* const* scales,
                         const int32_t* tables, const int32_t* ctx, float sm_scale, kvq_fmt fmt,

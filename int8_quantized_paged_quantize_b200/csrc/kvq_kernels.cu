@@ -573,7 +573,7 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
                                  const void* ks, const void* vs, const int32_t* tables,
                                  const int32_t* ctx, int32_t max_ctx, float sm_scale,
                                  const DecodePlan& plan, void* ws, const kvq_dims& d,
-                                 int per_tensor, int n_query, cudaStream_t st) {
+                                 int per_tensor, int n_query, int nrg, cudaStream_t st) {
   using C = MmaCfg<D, G, FMT>;
   auto kern = decode_mma_kernel<D, G, FMT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -597,23 +597,26 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
   kern<<<dim3(unsigned(grid)), 192, C::SMEM, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
-      static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, d.num_blocks,
+      static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads * nrg, nrg, d.num_blocks,
       d.max_blocks_per_seq, max_ctx, plan.partition / kTileTokens, plan.slots, sm_scale * kLog2e,
       per_tensor, n_query, decode_wait_limit(), po, pml, pcnt);
   return cudaGetLastError();
 }
 
 template <int D, int FMT>
-cudaError_t decode_dispatch2(int G, const void* q, int32_t B, const void* kc, const void* vc,
+cudaError_t decode_dispatch2(int R, const void* q, int32_t B, const void* kc, const void* vc,
                              const void* ks, const void* vs, const int32_t* tables,
                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
                              const DecodePlan& plan, void* ws, const kvq_dims& d, int per_tensor,
                              int n_query, cudaStream_t st) {
-  switch (G) {
-    case 1: return decode_mma_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st);
-    case 2: return decode_mma_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st);
-    case 4: return decode_mma_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st);
-    default: return decode_mma_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, st);
+  // R query rows per KV head, taken in groups of gp rows (one instantiation per gp)
+  int gp = 1;
+  const int nrg = row_groups(R, &gp);
+  switch (gp) {
+    case 1: return decode_mma_dispatch3<D, 1, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, nrg, st);
+    case 2: return decode_mma_dispatch3<D, 2, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, nrg, st);
+    case 4: return decode_mma_dispatch3<D, 4, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, nrg, st);
+    default: return decode_mma_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, nrg, st);
   }
 }
 }  // namespace
@@ -676,7 +679,10 @@ int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* ou
   const int32_t* pcnt =
       reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + plan.o_bytes + plan.ml_bytes);
   const dim3 grid(unsigned(int64_t(B) * d.n_q_heads));
-  const int W = d.max_blocks_per_seq, Hq = d.n_q_heads, G = d.n_q_heads / d.n_kv_heads;
+  // G: query rows per row group, the unit part_cnt is kept for
+  const int W = d.max_blocks_per_seq, Hq = d.n_q_heads;
+  int G = 1;
+  row_groups(d.n_q_heads / d.n_kv_heads, &G);
   if (d.head_dim == 128) {
     if (out_f32)
       merge_kernel<128, float><<<grid, 128, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W, po, pml,

@@ -60,6 +60,11 @@ _SIGNATURES = [
     ("kvq_decode_verify", _c.c_int, [_P, _c.c_int32, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32,
                                      _c.c_float, _P, _c.c_int, _P, _c.c_size_t, _c.c_int32, _c.c_int,
                                      _P, _P]),
+    ("kvq_prefill_attn_workspace_bytes", _c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32,
+                                                       _c.c_int32, _c.c_int, _P]),
+    ("kvq_prefill_attn", _c.c_int, [_P, _c.c_int32, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32,
+                                    _c.c_float, _P, _c.c_int, _P, _c.c_size_t, _c.c_int32, _c.c_int,
+                                    _P, _P]),
 ]
 
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
@@ -311,6 +316,34 @@ def wait_limit() -> int:
     return int(lib().kvq_get_wait_limit())
 
 
+def prefill_attn(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                 max_context_len, sm_scale, out, fmt: str, d: Dims, workspace=None,
+                 partition_tokens=0, stream=None):
+    """Chunked-prefill attention over the quantized cache (kvq_prefill_attn).
+    q, out: [B][Hq][chunk_len][D]; the chunk's tokens are the last chunk_len
+    cached tokens of each sequence and attend causally."""
+    _need(q, torch.bfloat16, "q")
+    _need_out(out)
+    _need(block_tables, torch.int32, "block_tables")
+    _need(context_lens, torch.int32, "context_lens")
+    if q.dim() != 4 or tuple(out.shape) != tuple(q.shape):
+        raise KvqError("q and out must be [batch][n_q_heads][chunk_len][head_dim]")
+    B, n = q.shape[0], q.shape[2]
+    if workspace is None:
+        nb = lib().kvq_prefill_attn_workspace_bytes(B, n, int(max_context_len), partition_tokens,
+                                                    FMT[fmt], ctypes.byref(d))
+        if nb == 0 and B > 0:
+            raise KvqError("kvq_prefill_attn_workspace_bytes: invalid arguments")
+        workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().kvq_prefill_attn(_ptr(q), B, n, _ptr(k_cache), _ptr(v_cache),
+                                  _scales(k_scale, v_scale), _ptr(block_tables),
+                                  _ptr(context_lens), int(max_context_len), float(sm_scale),
+                                  _ptr(out), _out_dtype(out), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), partition_tokens,
+                                  FMT[fmt], ctypes.byref(d), _stream(stream)), "kvq_prefill_attn")
+    return out
+
+
 def device_error(clear=True) -> int:
     """KVQ_DEVERR_* bits flagged by kernels on the current device (synchronizes)."""
     f = ctypes.c_uint32()
@@ -389,6 +422,18 @@ class LayerCache:
         return decode_verify(q, self.k, self.v, self.k_scale, self.v_scale, block_tables,
                              context_lens, max_context_len, sm_scale, out, self.fmt, self.dims,
                              workspace=workspace, partition_tokens=partition_tokens, stream=stream)
+
+    def prefill(self, q, block_tables, context_lens, max_context_len, sm_scale=None, out=None,
+                workspace=None, partition_tokens=0, stream=None, out_dtype=torch.bfloat16):
+        """Chunked-prefill attention (kvq_prefill_attn): q [B][Hq][chunk][D], the
+        chunk being the newest cached tokens of each sequence."""
+        if sm_scale is None:
+            sm_scale = 1.0 / math.sqrt(self.dims.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        return prefill_attn(q, self.k, self.v, self.k_scale, self.v_scale, block_tables,
+                            context_lens, max_context_len, sm_scale, out, self.fmt, self.dims,
+                            workspace=workspace, partition_tokens=partition_tokens, stream=stream)
 
     # ---- copies in the logical layout [NB][Hk][block_size][D] (for inspection and tests)
     def k_logical(self, blocks=None):

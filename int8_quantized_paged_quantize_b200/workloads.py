@@ -120,33 +120,43 @@ def final_lengths(w: Workload, seed: int = 0) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------- block tables
+def pool_blocks(w: Workload, seed: int = 0) -> int:
+    """Blocks in the pool of a workload: exactly what the sequences need for
+    their final lengths, except the fragmented shared pool (about 1.25x)."""
+    need = int(((final_lengths(w, seed) + w.block_size - 1) // w.block_size).sum())
+    if w.pool == "permutation16":
+        return 16
+    if w.pool == "fragmented":
+        return int(math.ceil(1.25 * need))
+    return need
+
+
 def block_tables(w: Workload, seed: int = 0):
-    """(block_tables int32 [B][W], num_blocks) covering final_lengths().
+    """(block_tables int32 [B][W], num_blocks) covering final_lengths(), for the
+    pools laid out directly (not through an allocator).
 
     Entries past a sequence's last block are -1.
       shuffled:      the pool holds exactly the blocks needed, handed out in a
                      seeded random order;
       permutation16: a 16-block pool, sequences take consecutive runs of one
-                     seeded permutation of 0..15;
-      fragmented:    the pool is ~1.25x what is needed and goes through seeded
-                     allocate/free churn before the sequences take their blocks.
+                     seeded permutation of 0..15.
+    The fragmented shared pool is built by the library's block allocator
+    instead (paging.paged_batch plays pool_churn() on it).
     """
     bs = w.block_size
     need = (final_lengths(w, seed) + bs - 1) // bs
     W = int(need.max()) if need.size else 0
     tables = np.full((w.batch, max(W, 1)), -1, dtype=np.int32)
     rng = _rng(seed, "blocks")
+    num_blocks = pool_blocks(w, seed)
     if w.pool == "permutation16":
-        num_blocks = 16
         if need.sum() > num_blocks:
             raise ValueError("permutation16 pool too small")
         order = rng.permutation(num_blocks)
     elif w.pool == "shuffled":
-        num_blocks = int(need.sum())
         order = rng.permutation(num_blocks)
     elif w.pool == "fragmented":
-        num_blocks = int(math.ceil(1.25 * need.sum()))
-        order = _fragmented_free_list(rng, num_blocks, int(need.sum()))
+        raise ValueError("the fragmented pool comes from the block allocator: use paging.paged_batch")
     else:
         raise ValueError(w.pool)
     at = 0
@@ -157,27 +167,36 @@ def block_tables(w: Workload, seed: int = 0):
     return tables, num_blocks
 
 
-def _fragmented_free_list(rng, num_blocks, n_needed, rounds=64):
-    """A free list after allocate/free churn: blocks are taken from the front in
-    runs of random size and a random half of the taken ones come back at the
-    end, in random order. Returns the free list (at least n_needed entries)."""
-    free = list(rng.permutation(num_blocks))
-    held = []
-    for _ in range(rounds):
-        take = int(rng.integers(1, max(2, num_blocks // 16)))
-        take = min(take, len(free) - 1)
-        if take > 0:
-            held.extend(free[:take])
-            free = free[take:]
-        if held:
-            n_back = len(held) // 2
-            idx = rng.permutation(len(held))
-            back = [held[i] for i in idx[:n_back]]
-            held = [held[i] for i in idx[n_back:]]
-            free.extend(back)
-    free.extend(rng.permutation(np.asarray(held, dtype=np.int64)).tolist() if held else [])
-    assert len(free) == num_blocks and len(free) >= n_needed
-    return np.asarray(free, dtype=np.int64)
+@dataclass(frozen=True)
+class ChurnRound:
+    take: int                     # blocks allocated in this round
+    give_back: tuple              # positions, in the list of held blocks, freed afterwards
+
+
+def pool_churn(w: Workload, seed: int = 0, rounds: int = 64):
+    """Seeded allocate/free schedule that fragments a shared pool before the
+    workload's sequences take their blocks (what other requests coming and
+    going leave behind). Only counts and positions are drawn here; the block
+    ids are whatever the allocator hands out. The first round fills the pool
+    but for one block (earlier requests holding it); every later round
+    allocates a run of 1 .. pool/16 blocks (never the last free one). After
+    each allocation a random half of all blocks held so far is freed, named by
+    their positions in the held list (held blocks in allocation order, freed
+    ones removed)."""
+    num_blocks = pool_blocks(w, seed)
+    rng = _rng(seed, "churn")
+    free, held = num_blocks, 0
+    out = []
+    for r in range(rounds):
+        take = num_blocks - 1 if r == 0 else int(rng.integers(1, max(2, num_blocks // 16)))
+        take = max(0, min(take, free - 1))
+        free -= take
+        held += take
+        idx = rng.permutation(held)[:held // 2] if held else np.zeros(0, dtype=np.int64)
+        out.append(ChurnRound(take, tuple(int(i) for i in idx)))
+        free += len(idx)
+        held -= len(idx)
+    return out
 
 
 # --------------------------------------------------------------------------- values

@@ -17,6 +17,7 @@ import numpy as np
 import torch
 
 from int8_quantized_paged_quantize_b200 import kvq
+from int8_quantized_paged_quantize_b200 import paging
 from int8_quantized_paged_quantize_b200 import workloads as W
 from oracle import attention as OA
 from oracle import formats as OF
@@ -74,8 +75,11 @@ def inputs(w: W.Workload, seed=0):
     history and bulk-append K/V (BF16, CPU) and the first step's q/k/v."""
     key = (w, seed)
     if key not in _INPUTS:
-        hist = [W.kv_history(w, b, seed) for b in range(w.batch)]
-        bulk = [W.kv_bulk(w, b, seed) for b in range(w.batch)] if w.bulk_append else None
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(16) as ex:                  # numpy draws release the GIL
+            hist = list(ex.map(lambda b: W.kv_history(w, b, seed), range(w.batch)))
+            bulk = (list(ex.map(lambda b: W.kv_bulk(w, b, seed), range(w.batch)))
+                    if w.bulk_append else None)
         _INPUTS.clear()                      # keep one workload's data at a time
         _INPUTS[key] = (hist, bulk, W.step_inputs(w, 0, seed))
     return _INPUTS[key]
@@ -86,9 +90,24 @@ def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch
     """Append every sequence's cached history (in `history_chunks` calls), then the
     bulk append if the workload has one, then one token per sequence, and run one
     decode step over ctx + 1 tokens. Returns a GpuRun."""
-    tables, nb = W.block_tables(w, seed)
     ctx = W.context_lengths(w, seed)
     hist, bulk, (q, k_new, v_new) = inputs(w, seed)
+    if w.pool == "fragmented":
+        # a shared pool fragmented by other requests: tables and slots come
+        # from the library's block allocator as the sequences grow
+        pb = paging.paged_batch(w, seed, fmt)
+        hist_slots = [pb.extend(b, int(ctx[b])) for b in range(w.batch)]
+        bulk_slots = [pb.extend(b, w.bulk_append) for b in range(w.batch)] if bulk is not None else None
+        step_np = np.array([pb.extend(b, 1)[0] for b in range(w.batch)], dtype=np.int64)
+        tables, nb = pb.tables.copy(), pb.dims.num_blocks
+        pb.close()
+    else:
+        tables, nb = W.block_tables(w, seed)
+        hist_slots = [slots_for(tables, b, np.arange(ctx[b])) for b in range(w.batch)]
+        bulk_slots = ([slots_for(tables, b, ctx[b] + np.arange(w.bulk_append)) for b in range(w.batch)]
+                      if bulk is not None else None)
+        c1 = ctx + w.bulk_append
+        step_np = np.array([slots_for(tables, b, [c1[b]])[0] for b in range(w.batch)], dtype=np.int64)
     d = kvq.dims(nb, w.n_kv_heads, w.n_q_heads, w.head_dim, tables.shape[1])
     dev = torch.device("cuda")
     kst = vst = None
@@ -100,7 +119,7 @@ def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch
                                         v_static=torch.from_numpy(vst).to(torch.bfloat16).to(dev))
     else:
         cache = kvq.LayerCache.allocate(fmt, d)
-    S = [torch.from_numpy(slots_for(tables, b, np.arange(ctx[b]))) for b in range(w.batch)]
+    S = [torch.from_numpy(x) for x in hist_slots]
     S = torch.cat(S) if S else torch.zeros(0, dtype=torch.int64)
     n = S.numel()
     if n:
@@ -115,13 +134,11 @@ def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch
         nb_tok = w.bulk_append
         K = torch.cat([x[0] for x in bulk]).to(dev)
         V = torch.cat([x[1] for x in bulk]).to(dev)
-        S = torch.cat([torch.from_numpy(slots_for(tables, b, ctx[b] + np.arange(nb_tok)))
-                       for b in range(w.batch)]).to(dev)
+        S = torch.cat([torch.from_numpy(x) for x in bulk_slots]).to(dev)
         cache.append(K, V, S)
         del K, V
         ctx = ctx + nb_tok
-    step_slots = torch.from_numpy(np.array([slots_for(tables, b, [ctx[b]])[0]
-                                            for b in range(w.batch)], dtype=np.int64))
+    step_slots = torch.from_numpy(step_np)
     cache.append(k_new.to(dev), v_new.to(dev), step_slots.to(dev))
     ctx_after = ctx + 1
     tbl = torch.from_numpy(tables).to(dev)
@@ -232,4 +249,103 @@ def attention_errors(run: GpuRun, seqs, check_codes=True):
         o = oracle_attention(run, b, ref)
         errs.append(np.abs(run.out[b].float().numpy().astype(np.float64) - o).ravel())
     e = np.concatenate(errs) if errs else np.zeros(1)
+    return float(e.max()), float(e.mean())
+
+
+# ----------------------------------------------------------------------------- many decode steps
+@dataclass
+class StepsRun:
+    w: W.Workload
+    fmt: str
+    cache: kvq.LayerCache
+    tables: np.ndarray
+    ctx_hist: np.ndarray        # cached tokens before the bulk append
+    steps: int
+    outs: list                  # per step: [B][Hq][D] FP32 (CPU)
+    q: list                     # per step: [B][Hq][D] BF16 (CPU)
+    k_new: list                 # per step: [B][Hk][D] BF16
+    v_new: list
+    seed: int = 0
+
+
+def run_gpu_steps(w: W.Workload, fmt: str, n_steps: int, seed=0):
+    """The workload as specified for long contexts: the cached history in one
+    append call per sequence, then ONE bulk append of every sequence's bulk
+    tokens (all sequences in one call), then n_steps decode steps, each
+    appending one token per sequence and decoding over the grown context
+    (automatic split plan, FP32 output). Returns a StepsRun."""
+    tables, nb = W.block_tables(w, seed)
+    ctx = W.context_lengths(w, seed)
+    hist, bulk, _ = inputs(w, seed)
+    d = kvq.dims(nb, w.n_kv_heads, w.n_q_heads, w.head_dim, tables.shape[1])
+    dev = torch.device("cuda")
+    cache = kvq.LayerCache.allocate(fmt, d)
+    for b in range(w.batch):
+        cache.append(hist[b][0].to(dev), hist[b][1].to(dev),
+                     torch.from_numpy(slots_for(tables, b, np.arange(ctx[b]))).to(dev))
+    if bulk is not None:
+        K = torch.cat([x[0] for x in bulk]).to(dev)
+        V = torch.cat([x[1] for x in bulk]).to(dev)
+        S = torch.cat([torch.from_numpy(slots_for(tables, b, ctx[b] + np.arange(w.bulk_append)))
+                       for b in range(w.batch)]).to(dev)
+        cache.append(K, V, S)
+        del K, V
+    c = ctx + w.bulk_append
+    tbl = torch.from_numpy(tables).to(dev)
+    max_ctx = int((c + n_steps).max())
+    ws = cache.workspace(w.batch, max_ctx)
+    outs, qs, ks, vs = [], [], [], []
+    for s in range(n_steps):
+        q, k, v = W.step_inputs(w, s, seed)
+        sl = np.array([slots_for(tables, b, [c[b]])[0] for b in range(w.batch)], dtype=np.int64)
+        cache.append(k.to(dev), v.to(dev), torch.from_numpy(sl).to(dev))
+        c = c + 1
+        cl = torch.from_numpy(c.astype(np.int32)).to(dev)
+        outs.append(cache.decode(q.to(dev), tbl, cl, max_ctx, sm_scale=w.sm_scale, workspace=ws,
+                                 out_dtype=torch.float32).cpu())
+        qs.append(q)
+        ks.append(k)
+        vs.append(v)
+    torch.cuda.synchronize()
+    assert kvq.device_error(clear=True) == 0
+    return StepsRun(w, fmt, cache, tables, ctx, n_steps, outs, qs, ks, vs, seed)
+
+
+def check_steps_run(run: StepsRun, b: int, steps):
+    """Codes and scales of sequence b after every step bit-exact against the
+    oracle's, and its attention output at each of `steps` within tolerance.
+    Returns (max err, mean err) over the checked steps."""
+    w = run.w
+    hist, bulk, _ = inputs(w, run.seed)
+    k = torch.cat([hist[b][0]] + ([bulk[b][0]] if bulk is not None else []) +
+                  [x[b:b + 1] for x in run.k_new]).float().numpy()
+    v = torch.cat([hist[b][1]] + ([bulk[b][1]] if bulk is not None else []) +
+                  [x[b:b + 1] for x in run.v_new]).float().numpy()
+    n = k.shape[0]
+    # the cache view of assert_codes_equal: every sequence's tokens after the last step
+    one = GpuRun(w, run.fmt, run.cache, run.tables, run.ctx_hist,
+                 run.ctx_hist + w.bulk_append + run.steps, None, None, None, None, run.seed)
+    assert int(one.ctx_after[b]) == n
+    res = {"Kraw": k.astype(np.float64), "Vraw": v.astype(np.float64)}
+    for name, x in (("k", k), ("v", v)):
+        if run.fmt == "fp8":
+            c, s = OF.fp8_quantize(x)
+            res[name + "_codes"], res[name + "_scale"] = c, s
+            res[name.upper()] = OF.fp8_dequantize(c, s)
+        elif run.fmt == "int8":
+            c, s, z = OF.int8_quantize(x)
+            res[name + "_codes"], res[name + "_scale"], res[name + "_zp"] = c, s, z
+            res[name.upper()] = OF.int8_dequantize(c, s, z)
+        else:
+            res[name + "_codes"] = OF.bf16_round(x)
+            res[name.upper()] = x.astype(np.float64)
+    assert_codes_equal(one, b, res)
+    errs = []
+    base = n - run.steps
+    for s in steps:
+        L = base + s + 1
+        q = run.q[s][b:b + 1].float().numpy().astype(np.float64)
+        o = OA.decode_attention(q, [(res["K"][:L], res["V"][:L])], w.sm_scale, w.n_kv_heads)[0]
+        errs.append(np.abs(run.outs[s][b].numpy().astype(np.float64) - o).ravel())
+    e = np.concatenate(errs)
     return float(e.max()), float(e.mean())

@@ -132,12 +132,13 @@ def test_host_checks_need_no_gpu(kvq):
         assert L.kvq_decode_attn(fake, 1, fake, fake, none, fake, fake, 100, ctypes.c_float(0.1), fake,
                                  0, fake, 1 << 30, 0, fmt, ctypes.byref(d), None) == -1
     assert L.kvq_append(fake, fake, fake, 4, fake, fake, fake, fake, 6, ctypes.byref(d), None) == -1
-    # multi-query decode: G * n_query must stay a supported group size
-    vargs = lambda nq: (fake, 1, nq, fake, fake, scales, fake, fake, 100, ctypes.c_float(0.1), fake,
-                        0, fake, 1 << 30, 0, 1, ctypes.byref(d), None)
-    assert L.kvq_decode_verify(*vargs(8)) == -2                   # G = 2: 16 heads per group
-    assert L.kvq_decode_verify(*vargs(0)) == -1
-    assert L.kvq_decode_verify(*vargs(9)) == -1
+    # multi-query decode: n_query in 1..1024; a workspace that is too small is
+    # refused before any launch (so these fake pointers never reach a kernel)
+    vargs = lambda nq, ws: (fake, 1, nq, fake, fake, scales, fake, fake, 100, ctypes.c_float(0.1),
+                            fake, 0, fake, ws, 0, 1, ctypes.byref(d), None)
+    assert L.kvq_decode_verify(*vargs(8, 0)) == -3                # G = 2: 16 rows, two groups
+    assert L.kvq_decode_verify(*vargs(0, 1 << 30)) == -1
+    assert L.kvq_decode_verify(*vargs(1025, 1 << 30)) == -1
     assert L.kvq_decode_verify_workspace_bytes(1, 4, 100, 0, 1, ctypes.byref(d)) == \
         L.kvq_decode_workspace_bytes(1, 100, 0, 1, ctypes.byref(kvq.dims(64, 2, 16, 64, 8)))
     # max_context_len beyond what the block table can hold
@@ -151,3 +152,32 @@ def test_workspace_plan_scales_with_splits(kvq):
     one = kvq.decode_workspace_bytes(32, 32769, "int8", d, partition_tokens=32768 + 128)
     many = kvq.decode_workspace_bytes(32, 32769, "int8", d, partition_tokens=128)
     assert many > one >= 32 * 64 * (128 + 2) * 4
+
+
+def test_multi_query_workspace_and_limits(kvq):
+    """Host checks of kvq_decode_verify / kvq_prefill_attn: any n_query in
+    1..1024 has a split plan (more query rows than one group of 8 included),
+    the plan grows with the positions, and out-of-range counts are refused
+    before any device work."""
+    import ctypes as C
+    L = kvq.lib()
+    d = kvq.dims(4096, 8, 64, 128, 256)            # G = 8
+    sizes = [L.kvq_decode_verify_workspace_bytes(4, nq, 4096, 0, 1, C.byref(d))
+             for nq in (1, 2, 4, 64, 1024)]
+    assert all(x > 0 for x in sizes) and sizes == sorted(sizes)
+    assert L.kvq_decode_verify_workspace_bytes(4, 1, 4096, 0, 1, C.byref(d)) == \
+        L.kvq_decode_workspace_bytes(4, 4096, 0, 1, C.byref(d))
+    assert L.kvq_prefill_attn_workspace_bytes(4, 64, 4096, 0, 1, C.byref(d)) == \
+        L.kvq_decode_verify_workspace_bytes(4, 64, 4096, 0, 1, C.byref(d))
+    for nq in (0, -1, 1025):
+        assert L.kvq_decode_verify_workspace_bytes(4, nq, 4096, 0, 1, C.byref(d)) == 0
+    null = C.c_void_p(0)
+    scales = (C.c_void_p * 2)(0, 0)
+    for fn in (L.kvq_decode_verify, L.kvq_prefill_attn):
+        assert fn(null, 1, 1025, null, null, scales, null, null, 64, C.c_float(0.1), null, 0,
+                  null, 0, 0, 1, C.byref(d), None) == -1
+        # a valid count with null device pointers stops at the pointer checks
+        assert fn(null, 1, 64, null, null, scales, null, null, 64, C.c_float(0.1), null, 0,
+                  null, 0, 0, 1, C.byref(d), None) == -1
+        assert fn(null, 0, 64, null, null, scales, null, null, 64, C.c_float(0.1), null, 0,
+                  null, 0, 0, 1, C.byref(d), None) == 0

@@ -53,3 +53,18 @@ def test_mixed_serving_fp8_full():
 @pytest.mark.parametrize("fmt", ["fp8", "int8", "bf16"])
 def test_long_128k_full(fmt):
     _run_and_check("long-128k", fmt)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+def test_long_128k_bulk_then_64_steps(fmt):
+    """The long-context workload as specified: one bulk append of 8,192 tokens
+    into each of the 4 sequences (one call), then 64 decode steps of one append
+    each. After step 64 every sequence's codes and scales are bit-exact and its
+    attention at the last step is within tolerance; sequence 0 is also checked
+    at steps 1 and 32 (the contexts grow by one token per step)."""
+    w = W.WORKLOADS["long-128k"]
+    run = GC.run_gpu_steps(w, fmt, w.decode_steps)
+    for b in range(w.batch):
+        steps = [0, 31, 63] if b == 0 else [63]
+        mx, mean = GC.check_steps_run(run, b, steps)
+        assert mx <= GC.MAX_ABS and mean <= GC.MEAN_ABS, (fmt, b, mx, mean)

@@ -8,7 +8,11 @@ ctx - n_query + 1 + j tokens. Every position's output (FP32) must be within max
 |err| 4e-3 and mean |err| 5e-4 of the oracle's FP64 attention over the same
 dequantized K/V, across formats, GQA groups, head_dims, ragged contexts
 (including contexts shorter than n_query, whose first positions see nothing)
-and split-K partitions that end inside the new tokens.
+and split-K partitions that end inside the new tokens. More query rows per KV
+head than one row group of the kernel holds (G * n_query > 8: 2 or 4 positions
+at the 70B-shaped G = 8) and a 64-token prefill chunk at G = 4 ("From FP8 KV
+cache to INT4 weight-only", Core concepts 1): a chunk's queries attend to the
+cached prefix and, causally, to the chunk) are checked the same way.
 """
 
 import numpy as np
@@ -27,7 +31,7 @@ pytestmark = pytest.mark.gpu
 CTX = [1, 2, 3, 15, 16, 17, 127, 128, 129, 300, 1000]
 
 
-def _run(fmt, D, G, nq, ctx=CTX, Hk=2, partition=0, seed=0):
+def _run(fmt, D, G, nq, ctx=CTX, Hk=2, partition=0, seed=0, call="verify"):
     w = W.Workload("synthetic", fmt, batch=len(ctx), n_q_heads=Hk * G, n_kv_heads=Hk, head_dim=D,
                    lengths="list", ctx=tuple(ctx), kv_mean=0.3 if fmt == "int8" else 0.0)
     tables, nb = W.block_tables(w, seed)
@@ -50,9 +54,10 @@ def _run(fmt, D, G, nq, ctx=CTX, Hk=2, partition=0, seed=0):
     g = torch.Generator().manual_seed(100 + seed)
     q = torch.randn(w.batch, Hk * G, nq, D, generator=g).to(torch.bfloat16)
     out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
-    kvq.decode_verify(q.cuda(), cache.k, cache.v, cache.k_scale, cache.v_scale,
-                      torch.from_numpy(tables).cuda(), torch.from_numpy(lens.astype(np.int32)).cuda(),
-                      int(lens.max()), w.sm_scale, out, fmt, d, partition_tokens=partition)
+    fn = kvq.decode_verify if call == "verify" else kvq.prefill_attn
+    fn(q.cuda(), cache.k, cache.v, cache.k_scale, cache.v_scale,
+       torch.from_numpy(tables).cuda(), torch.from_numpy(lens.astype(np.int32)).cuda(),
+       int(lens.max()), w.sm_scale, out, fmt, d, partition_tokens=partition)
     torch.cuda.synchronize()
     assert kvq.device_error() == 0
     # oracle: the same tokens through the oracle's pool, then FP64 attention
@@ -115,3 +120,34 @@ def test_one_position_equals_plain_decode():
                          out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(out_v[:, :, 0], out_d)
+
+
+def _zero_rows(out, lens, nq):
+    for b, c in enumerate(lens):
+        for j in range(nq):
+            if c - nq + 1 + j <= 0:
+                assert torch.count_nonzero(out[b, :, j]) == 0
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("G,nq", [(8, 2), (8, 4), (4, 4), (2, 8), (1, 16), (4, 3), (8, 5)])
+def test_verify_rows_beyond_one_group(fmt, G, nq):
+    """G * n_query > 8: the rows of a KV head span several row groups (3 and 5
+    positions give groups of 4 and 8 rows that split query heads apart)."""
+    err, out, ref, lens = _run(fmt, 128, G, nq)
+    _check(err)
+    _zero_rows(out, lens, nq)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "bf16", "e5m2"])
+def test_prefill_chunk_of_64_at_group_4(fmt):
+    """A 64-token prefill chunk at G = 4 (256 query rows per KV head): contexts
+    that are exactly the chunk, one token more, and long cached prefixes."""
+    err, out, ref, lens = _run(fmt, 128, 4, 64, ctx=[64, 65, 200, 1000, 4000], call="prefill")
+    _check(err)
+
+
+def test_prefill_equals_verify_with_the_same_positions():
+    e1, o1, _, _ = _run("fp8", 64, 2, 16, ctx=[40, 300], call="prefill")
+    e2, o2, _, _ = _run("fp8", 64, 2, 16, ctx=[40, 300], call="verify")
+    assert torch.equal(o1, o2)

@@ -6,7 +6,7 @@ import pytest
 from int8_quantized_paged_quantize_b200 import workloads as W
 
 
-@pytest.mark.parametrize("name", list(W.WORKLOADS))
+@pytest.mark.parametrize("name", [n for n, w in W.WORKLOADS.items() if w.pool != "fragmented"])
 def test_block_tables_are_valid(name):
     w = W.WORKLOADS[name]
     tables, nb = W.block_tables(w, seed=0)
@@ -49,9 +49,10 @@ def test_length_distributions():
     assert len(c) == 256 and np.sum(c == 30000) >= 4
     assert c.min() >= 16 and c.max() <= 32768
     assert 800 < np.median(c) < 2500
-    _, nb = W.block_tables(w)
     need = ((W.final_lengths(w) + 15) // 16).sum()
-    assert nb == int(np.ceil(1.25 * need))
+    assert W.pool_blocks(w) == int(np.ceil(1.25 * need))
+    with pytest.raises(ValueError):
+        W.block_tables(w)                      # comes from the allocator instead
 
 
 def test_outlier_structure():
@@ -66,3 +67,16 @@ def test_outlier_structure():
     k, _ = W.kv_history(w, 0, ctx=4000)
     frac = (k.float().abs() > 8).float().mean().item()
     assert 0.0003 < frac < 0.003
+
+
+def test_pool_churn_schedule_is_feasible_and_seeded():
+    w = W.WORKLOADS["mixed-serving-fp8"]
+    sched = W.pool_churn(w, seed=0)
+    assert sched == W.pool_churn(w, seed=0) and sched != W.pool_churn(w, seed=1)
+    nb, held = W.pool_blocks(w), 0
+    for rnd in sched:
+        assert 0 <= rnd.take and held + rnd.take < nb          # never the last free block
+        held += rnd.take
+        assert len(set(rnd.give_back)) == len(rnd.give_back) == held // 2
+        assert all(0 <= i < held for i in rnd.give_back)
+        held -= len(rnd.give_back)
