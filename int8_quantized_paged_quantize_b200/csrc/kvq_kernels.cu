@@ -72,27 +72,30 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 namespace kvq {
 
 // ------------------------------------------------------------------ append
-// Quantize one (token, KV head) row of D BF16 values held by a warp (E = D/32
-// values per lane): the range by integer warp reductions, the BF16 scale (+
-// zero point) on every lane, codes in d order packed little-endian into `w`.
+// A (token, KV head) row of D BF16 values is quantized by one half warp: 16
+// lanes with E = D/16 consecutive values each (one 16-byte load at D = 128),
+// so a warp instruction serves two rows. The range is an integer max over the
+// half warp, the BF16 scale (+ zero point) is formed on each of its lanes, and
+// the lane's codes are packed little-endian in d order into `w`.
 template <int D, int FMT>
 struct RowCodes {
-  static constexpr int E = D / 32;
+  static constexpr int E = D / 16;
   static constexpr int ELT = (FMT == KVQ_BF16) ? 2 : 1;
-  static constexpr int WORDS = (E * ELT + 3) / 4;
+  static constexpr int WORDS = E * ELT / 4;
   uint32_t w[WORDS];
   __nv_bfloat16 s;
   int zp;
 };
 
-// This lane's D/32 BF16 values of a row, as packed pairs.
+// This lane's D/16 BF16 values of a row, as packed pairs.
 template <int D>
-__device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint32_t (&raw)[D / 64]) {
-  if constexpr (D / 64 == 2) {
+__device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint32_t (&raw)[D / 32]) {
+  if constexpr (D == 128) {
+    const uint4 u = *reinterpret_cast<const uint4*>(src);
+    raw[0] = u.x; raw[1] = u.y; raw[2] = u.z; raw[3] = u.w;
+  } else {
     const uint2 u = *reinterpret_cast<const uint2*>(src);
     raw[0] = u.x; raw[1] = u.y;
-  } else {
-    raw[0] = *reinterpret_cast<const uint32_t*>(src);
   }
 }
 
@@ -110,11 +113,12 @@ __device__ __forceinline__ float div_by_const(float a) {
 
 // x / s for the row's BF16 scale s > 0, as the codes need it. For s >= 2^-100
 // it is RN(x * RN(1/s)) corrected once on the exact FMA residual (Markstein's
-// method; the test for a zero residual keeps the sign of -0): it may differ
-// from the IEEE quotient in the last bit, but the E4M3, E5M2 and rint codes
-// taken from it are the IEEE quotient's for every BF16 x with |x| <= 65536 s,
-// subnormal x included (enumerated by tests/test_scale_division.py). Rows with
-// a smaller scale take the IEEE division.
+// method), with the residual's sign folded so that a zero x keeps its sign
+// (-0 / s = -0) without a test: it may differ from the IEEE quotient in the
+// last bit, but the E4M3, E5M2 and rint codes taken from it are the IEEE
+// quotient's for every BF16 x with |x| <= 65536 s, subnormal x included
+// (enumerated by tests/test_scale_division.py). Rows with a smaller scale take
+// the IEEE division.
 struct ScaleDiv {
   float s, r;
   bool fast;
@@ -126,22 +130,27 @@ struct ScaleDiv {
   __device__ __forceinline__ float operator()(float x) const {
     if (!fast) return __fdiv_rn(x, s);
     const float q = __fmul_rn(x, r);
-    const float e = __fmaf_rn(-q, s, x);
-    return e != 0.f ? __fmaf_rn(e, r, q) : q;
+    const float e = __fmaf_rn(q, s, -x);             // minus the residual x - q s (exact)
+    return __fmaf_rn(-e, r, q);
   }
 };
 
-// Warp-wide max(0, max of v) for floats: non-negative floats order as their
-// bit patterns read as signed integers, and every negative float (-0 included)
-// reads as a negative integer, so one integer max-reduction with a floor of 0
-// gives the float maximum, +0 when nothing is positive.
-__device__ __forceinline__ float warp_max_floor0(int bits) {
-  return __int_as_float(__reduce_max_sync(0xffffffffu, max(bits, 0)));
+// Max over the 16 lanes of this half warp (both halves reduce at once).
+__device__ __forceinline__ int half_warp_max(int v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
 
+// The row maximum is taken on float bit patterns: non-negative floats order as
+// their bits read as signed integers and every negative float (-0 included)
+// reads as a negative integer, so an integer max with a floor of 0 gives the
+// float maximum, +0 when nothing is positive. Every lane of the warp must call
+// the quantizers (the half-warp reductions are warp-wide shuffles); a row that
+// is not stored is still quantized, from whatever its lanes hold.
 template <int D, int FMT>
-__device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowCodes<D, FMT>& rc) {
-  constexpr int E = D / 32;
+__device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 32], RowCodes<D, FMT>& rc) {
+  constexpr int E = D / 16;
   rc.zp = 0;
   rc.s = __float2bfloat16_rn(0.f);
   if constexpr (FMT == KVQ_BF16) {
@@ -152,14 +161,15 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
     float x[E];
 #pragma unroll
     for (int i = 0; i < E / 2; ++i) { x[2 * i] = bf16_lo(raw[i]); x[2 * i + 1] = bf16_hi(raw[i]); }
-    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < RowCodes<D, FMT>::WORDS; ++i) rc.w[i] = 0u;
     if constexpr (FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2) {
       // s = bf16(amax / max code), code = fp8_rne_satfinite(x / s)
       constexpr bool E4 = FMT == KVQ_FP8_E4M3;
       int amax_bits = 0;
 #pragma unroll
       for (int i = 0; i < E; ++i) amax_bits = max(amax_bits, __float_as_int(fabsf(x[i])));
-      const float amax = warp_max_floor0(amax_bits);
+      const float amax = __int_as_float(half_warp_max(amax_bits));
       rc.s = __float2bfloat16_rn(E4 ? div_by_const<448>(amax) : div_by_const<57344>(amax));
       const float s = __bfloat162float(rc.s);
       if (s != 0.f) {
@@ -168,7 +178,7 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
         for (int i = 0; i < E; i += 2) {
           const float2 qv = make_float2(div(x[i]), div(x[i + 1]));
           const uint32_t two = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, E4 ? __NV_E4M3 : __NV_E5M2);
-          packed |= two << (8 * i);
+          rc.w[i >> 2] |= two << (8 * (i & 3));
         }
       }
     } else {  // INT8 asymmetric: range [lo, hi] widened to hold 0
@@ -178,8 +188,8 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
         hi_bits = max(hi_bits, __float_as_int(x[i]));
         nlo_bits = max(nlo_bits, __float_as_int(-x[i]));
       }
-      const float hi = warp_max_floor0(hi_bits);     // max(0, max x)
-      const float nlo = warp_max_floor0(nlo_bits);   // -min(0, min x)
+      const float hi = __int_as_float(half_warp_max(hi_bits));     // max(0, max x)
+      const float nlo = __int_as_float(half_warp_max(nlo_bits));   // -min(0, min x)
       rc.s = __float2bfloat16_rn(div_by_const<255>(__fadd_rn(hi, nlo)));
       const float s = __bfloat162float(rc.s);
       if (s != 0.f) {
@@ -190,11 +200,10 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
         for (int i = 0; i < E; ++i) {
           const float qf = fminf(fmaxf(div(x[i]), -1024.f), 1024.f);
           const int c = min(127, max(-128, __float2int_rn(qf) + rc.zp));
-          packed |= uint32_t(uint8_t(int8_t(c))) << (8 * i);
+          rc.w[i >> 2] |= uint32_t(uint8_t(int8_t(c))) << (8 * (i & 3));
         }
       }
     }
-    rc.w[0] = packed;
   }
 }
 
@@ -206,12 +215,13 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 64], RowC
 // corrected quotient inside the range where its rint equals that of the IEEE
 // quotient (tests/test_scale_division.py).
 template <int D>
-__device__ __forceinline__ void quantize_row_static(const uint32_t (&raw)[D / 64], const float (&sc)[D / 32],
-                                                    const float (&rc_)[D / 32], RowCodes<D, KVQ_INT8_CHANNEL>& rc) {
-  constexpr int E = D / 32;
+__device__ __forceinline__ void quantize_row_static(const uint32_t (&raw)[D / 32], const float (&sc)[D / 16],
+                                                    const float (&rc_)[D / 16], RowCodes<D, KVQ_INT8_CHANNEL>& rc) {
+  constexpr int E = D / 16;
   rc.zp = 0;
   rc.s = __float2bfloat16_rn(0.f);
-  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < RowCodes<D, KVQ_INT8_CHANNEL>::WORDS; ++i) rc.w[i] = 0u;
 #pragma unroll
   for (int i = 0; i < E; ++i) {
     const float x = (i & 1) ? bf16_hi(raw[i / 2]) : bf16_lo(raw[i / 2]);
@@ -223,16 +233,15 @@ __device__ __forceinline__ void quantize_row_static(const uint32_t (&raw)[D / 64
       float q;
       if (r != 0.f) {
         const float q0 = __fmul_rn(xc, r);
-        const float e = __fmaf_rn(-q0, s, xc);
-        q = e != 0.f ? __fmaf_rn(e, r, q0) : q0;
+        const float e = __fmaf_rn(q0, s, -xc);
+        q = __fmaf_rn(-e, r, q0);
       } else {
         q = __fdiv_rn(xc, s);
       }
       c = min(127, max(-127, __float2int_rn(fminf(fmaxf(q, -1024.f), 1024.f))));
     }
-    packed |= uint32_t(uint8_t(int8_t(c))) << (8 * i);
+    rc.w[i >> 2] |= uint32_t(uint8_t(int8_t(c))) << (8 * (i & 3));
   }
-  rc.w[0] = packed;
 }
 
 // Bytes [p, e) of the 16-byte chunk at dst (16-byte aligned) from w, with the
@@ -277,11 +286,11 @@ __device__ __forceinline__ void store_bytes16(uint8_t* dst, const uint32_t (&w)[
   }
 }
 
-// One CTA of 8 warps per (16 consecutive input tokens, KV head); each warp
-// quantizes K and V rows of its tokens into shared memory. The input rows are
-// requested before the slots arrive (a skipped token's row is read and
-// dropped), so the two loads overlap. The window is then written in page-sized
-// pieces:
+// One CTA of 8 warps per (16 consecutive input tokens, KV head). Warp w takes
+// tokens 2w and 2w+1; for each, its lanes 0-15 quantize the token's K row and
+// lanes 16-31 its V row into shared memory. The input rows are requested before
+// the slots arrive (a skipped token's row is read and dropped), so the loads
+// overlap. The window is then written in page-sized pieces:
 //   - the 16 tokens fill one page in order (the bulk / prefill case): the page
 //     is written as whole 16-byte chunks, K in its chunk-major layout and V
 //     transposed with byte permutes;
@@ -291,10 +300,11 @@ __device__ __forceinline__ void store_bytes16(uint8_t* dst, const uint32_t (&w)[
 //     stores that range allows. A page continued from an offset (chunked
 //     prefill) thus costs one partial chunk per channel, not one byte store per
 //     token and channel.
-// Register use is capped at 32 so that 8 CTAs (64 warps) fit on an SM (40 and
-// 6 CTAs for the static-scale format, which keeps its channels' scales).
+// Register use is capped at 32 so that 8 CTAs (64 warps) fit on an SM (51 and
+// 5 CTAs for the static-scale format, whose lanes keep their channels' scales
+// and reciprocals).
 template <int D, int FMT>
-__global__ void __launch_bounds__(256, FMT == KVQ_INT8_CHANNEL ? 6 : 8)
+__global__ void __launch_bounds__(256, FMT == KVQ_INT8_CHANNEL ? 5 : 8)
 append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
               const int64_t* __restrict__ slots, int T, int Hk, int NB, uint8_t* __restrict__ kc,
               uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs,
@@ -319,17 +329,16 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
   const int n = int(min(int64_t(kBlockSize), int64_t(T) - tb));
   const int64_t nslots = int64_t(NB) * kBlockSize;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int d0 = lane * E;
-  // the warp's rows (row rr = 2 * token + {K, V}), requested up front so that
-  // their latencies overlap with each other and with the slot load
-  constexpr int RPW = 2 * kBlockSize / 8;
-  uint32_t raws[RPW][D / 64];
+  const int which = lane >> 4;                  // 0: K row, 1: V row
+  const int d0 = (lane & 15) * E;
+  // this half warp's rows: tokens 2 warp and 2 warp + 1, requested up front
+  const __nv_bfloat16* src = (which ? v : k) + ((tb + 2 * warp) * Hk + h) * D + d0;
+  uint32_t raws[2][D / 32];
 #pragma unroll
-  for (int j = 0; j < RPW; ++j) {
-    const int rr = warp + 8 * j, i = rr >> 1, which = rr & 1;
+  for (int p = 0; p < 2; ++p) {
 #pragma unroll
-    for (int e = 0; e < D / 64; ++e) raws[j][e] = 0u;
-    if (i < n) load_row<D>((which ? v : k) + ((tb + i) * Hk + h) * D + d0, raws[j]);
+    for (int e = 0; e < D / 32; ++e) raws[p][e] = 0u;
+    if (2 * warp + p < n) load_row<D>(src + int64_t(p) * Hk * D, raws[p]);
   }
   if (threadIdx.x < kBlockSize) sl[threadIdx.x] = threadIdx.x < n ? slots[tb + threadIdx.x] : -1;
   __syncthreads();
@@ -361,11 +370,11 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
     }
   }
 
-  // static scales: a warp's rows are all K (even warps) or all V (odd warps),
-  // so a lane's channels keep their scales for every row it quantizes
+  // static scales: a half warp's rows are all K (lanes 0-15) or all V, so a
+  // lane's channels keep their scales for every row it quantizes
   [[maybe_unused]] float ssc[E], rsc[E];
   if constexpr (FMT == KVQ_INT8_CHANNEL) {
-    const __nv_bfloat16* sarr = (warp & 1) ? vs : ks;
+    const __nv_bfloat16* sarr = which ? vs : ks;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       ssc[e] = __bfloat162float(sarr[per_tensor ? 0 : h * D + d0 + e]);
@@ -373,24 +382,23 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
     }
   }
 #pragma unroll
-  for (int j = 0; j < RPW; ++j) {
-    const int rr = warp + 8 * j;
-    const int i = rr >> 1, which = rr & 1;          // token in the group, K or V
-    if (i >= n) continue;
-    const int64_t slot = sl[i];
+  for (int p = 0; p < 2; ++p) {
+    const int i = 2 * warp + p;                     // token in the window
+    // every lane quantizes (the reductions span the warp); only real rows store
+    RC rc;
+    if constexpr (FMT == KVQ_INT8_CHANNEL) quantize_row_static<D>(raws[p], ssc, rsc, rc);
+    else quantize_row<D, FMT>(raws[p], rc);
+    const int64_t slot = i < n ? sl[i] : -1;
     if (slot < 0) continue;
     if (slot >= nslots) {
-      if (lane == 0) flag_error(KVQ_DEVERR_SLOT);
+      if ((lane & 15) == 0) flag_error(KVQ_DEVERR_SLOT);
       continue;
     }
-    RC rc;
-    if constexpr (FMT == KVQ_INT8_CHANNEL) quantize_row_static<D>(raws[j], ssc, rsc, rc);
-    else quantize_row<D, FMT>(raws[j], rc);
     uint8_t* dst = (which ? vbuf : kbuf) + i * PADB + d0 * ELT;
-    if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
-    else if constexpr (E * ELT == 4) *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
-    else *reinterpret_cast<uint16_t*>(dst) = uint16_t(rc.w[0]);
-    if (lane == 0) {
+    if constexpr (E * ELT == 16) *reinterpret_cast<uint4*>(dst) = make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]);
+    else if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
+    else *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
+    if ((lane & 15) == 0) {
       (which ? vmb : kmb)[i][0] = rc.s;
       (which ? vmb : kmb)[i][1] = __int2bfloat16_rn(rc.zp);
     }

@@ -11,7 +11,9 @@
  *
  * Mode "quot": the code quotient. For a BF16 scale s >= 2^-100 and every BF16
  * x with |x| <= 65536 s (subnormal x included), with r = RN(1/s):
- *     q = RN(x r), e = fma(-q, s, x), q2 = e != 0 ? fma(e, r, q) : q.
+ *     q = RN(x r), e = fma(q, s, -x), q2 = fma(-e, r, q)
+ * (e is minus the exact residual; with the sign folded this way a zero x keeps
+ * its sign through the correction, -0 giving -0).
  * q2 may differ from RN(x / s) in its last bit, but the E4M3 code (RNE,
  * saturating at 448), the E5M2 code (RNE, saturating at 57344) and the rint
  * integer taken from it must not. Scales below 2^-100 take the IEEE divide in
@@ -125,8 +127,8 @@ int main(int argc, char** argv) {
       for (int neg = 0; neg < 2; ++neg) {
         const float x = neg ? -xa : xa;
         const float q = x * r;
-        const float e = fmaf(-q, s, x);
-        const float q2 = e != 0.0f ? fmaf(e, r, q) : q;
+        const float e = fmaf(q, s, -x);          /* minus the residual x - q s, exact */
+        const float q2 = fmaf(-e, r, q);
         const float ref = x / s;
         ++checked;
         if (f32_bits(q2) == f32_bits(ref)) continue;

@@ -78,7 +78,7 @@ def test_a_dropped_correction_is_caught(tmp_path):
     """Planted mistake on the host: the plain product RN(x RN(1/s)) without the
     residual correction changes codes, so the check has teeth."""
     src = open(SRC).read()
-    planted = src.replace("const float q2 = e != 0.0f ? fmaf(e, r, q) : q;",
+    planted = src.replace("const float q2 = fmaf(-e, r, q);",
                           "const float q2 = q; (void)e;")
     assert planted != src
     p = tmp_path / "planted.c"
@@ -98,4 +98,19 @@ def test_a_plain_reciprocal_scale_is_caught(tmp_path):
     p.write_text(planted)
     exe = _compile(str(p), str(tmp_path / "planted"))
     rc, out, (_, _, bad) = _run(exe, "scale", 0, 0x10)
+    assert rc == 1 and bad > 0, out
+
+
+def test_a_correction_that_loses_the_sign_of_zero_is_caught(tmp_path):
+    """Planted mistake: the residual taken the other way round, e = fma(-q, s,
+    x) and q2 = fma(e, r, q), turns x = -0 into +0, whose E4M3 / E5M2 code
+    differs (0x00 against 0x80)."""
+    src = open(SRC).read()
+    planted = src.replace("const float e = fmaf(q, s, -x);", "const float e = fmaf(-q, s, x);")
+    planted = planted.replace("const float q2 = fmaf(-e, r, q);", "const float q2 = fmaf(e, r, q);")
+    assert planted != src
+    p = tmp_path / "planted.c"
+    p.write_text(planted)
+    exe = _compile(str(p), str(tmp_path / "planted"))
+    rc, out, (_, _, bad) = _run(exe, "quot", 0x3C00, 0x3C01)
     assert rc == 1 and bad > 0, out
