@@ -1,6 +1,5 @@
 """KIVI-style low-bit KV cache: K quantized per channel, V per token, the most
-recent tokens kept in full precision — test oracle (the CUDA path for this
-format is not built).
+recent tokens kept in full precision — test oracle.
 
 Test infrastructure (see ``oracle/__init__``).
 
@@ -30,7 +29,8 @@ Readings taken where the pages are silent
   most 127) stay in BF16, K and V alike; a group is quantized when it
   completes.
 * Metadata (s, z) is BF16: K 4 bytes per (group, KV head, channel), V 4 bytes
-  per (position, KV head).
+  per (position, KV head). A zero minimum or range is stored as +0 (the pages
+  give no sign of zero; numpy's min / max leave it to the order of the values).
 """
 
 from __future__ import annotations
@@ -47,8 +47,10 @@ def asym_params(x, axis, bits):
     a = np.asarray(x, dtype=np.float32)
     lo = np.min(a, axis=axis).astype(np.float32)
     hi = np.max(a, axis=axis).astype(np.float32)
-    z = bf16_round(lo)
-    s = bf16_round((hi - lo).astype(np.float32) / np.float32(2 ** bits - 1))
+    # a zero minimum or range is +0: numpy's reductions leave the sign of a
+    # zero result to the order they visit the values in (adding +0 maps -0 to +0)
+    z = bf16_round(lo) + np.float32(0.0)
+    s = bf16_round((hi - lo).astype(np.float32) / np.float32(2 ** bits - 1)) + np.float32(0.0)
     return s, z
 
 

@@ -120,3 +120,14 @@ def test_planted_mistakes_are_caught():
     c2, s2, z2 = Q.asym_quantize(g, axis=-1, bits=2)
     wrong_s = (g.max() - g.min()) / 4                          # 2^b instead of 2^b - 1 levels
     assert np.rint(g / wrong_s).tolist() != c2.tolist()
+
+
+def test_zero_minimum_and_range_are_plus_zero():
+    """Groups whose minimum or range is zero store +0 whatever the order of
+    +0 and -0 among the values (a canonical sign, reading in the oracle)."""
+    for row in ([0.0, -0.0, 0.0, -0.0], [-0.0, 0.0, -0.0, 0.0], [-0.0, -0.0, 1.0, 2.0]):
+        x = np.array([row], np.float32)
+        c, s, z = Q.asym_quantize(x, axis=-1, bits=2)
+        assert not np.signbit(z[0]) and z[0] == 0
+    c, s, z = Q.asym_quantize(np.array([[-0.0, 0.0, -0.0, 0.0]], np.float32), axis=-1, bits=4)
+    assert not np.signbit(s[0]) and s[0] == 0 and c.tolist() == [[0, 0, 0, 0]]
