@@ -77,8 +77,11 @@ typedef enum {
   KVQ_FP8_E5M2 = 3,  /* OCP E5M2 codes (max 57344, RNE, saturating) + BF16 scale */
   KVQ_INT8_CHANNEL = 4, /* signed int8 codes, symmetric, one static BF16 scale per
                            (KV head, channel), given by the caller */
-  KVQ_INT8_TENSOR = 5   /* signed int8 codes, symmetric, one static BF16 scale for
+  KVQ_INT8_TENSOR = 5,  /* signed int8 codes, symmetric, one static BF16 scale for
                            the whole K (and one for V) cache, given by the caller */
+  KVQ_KIVI2 = 6,        /* KIVI-style 2-bit codes: K per channel over 128-token
+                           groups, V per token; kvq_kivi_* calls only */
+  KVQ_KIVI4 = 7         /* the same with 4-bit codes */
 } kvq_fmt;
 
 typedef enum {
@@ -386,6 +389,82 @@ int kvq_prefill_attn(const void* q, int32_t batch, int32_t chunk_len, const void
                      void* out, kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
                      int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
                      kvq_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* KIVI-style low-bit cache (KVQ_KIVI2, KVQ_KIVI4).                            */
+/* [COMPRESS] "2.1": K has a few outlier channels and V a per-token spread, so */
+/* K is quantized per channel and V per token. [COMPRESS] "3.1", KIVI:         */
+/* asymmetric 2-bit codes, K per channel, V per token, the most recent tokens  */
+/* kept in full precision as a residual. [LIMITS] "Formats you will actually   */
+/* meet": the 4-bit variants do the same; 4-bit storage is a quarter of BF16.  */
+/* ------------------------------------------------------------------------ */
+/*
+ * A sequence's positions come in groups of 128 (eight 16-token blocks of its
+ * block table). A complete group is stored as b-bit codes (b = 2 or 4):
+ *   K, per (KV head, channel) over the group's 128 positions, and
+ *   V, per (position, KV head) over the head_dim channels:
+ *   z = bf16_rne(min x), s = bf16_rne(f32(max x - min x) / (2^b - 1)),
+ *   code = clamp(rint(f32(x - z) / s), 0, 2^b - 1) (IEEE f32 subtraction and
+ *   division, rint ties to even; s == 0 stores code 0; a zero z or s is +0);
+ *   the value read back is code * s + z.
+ * The positions after a sequence's last complete group (its residual) stay in
+ * BF16 in a separate cache of the KVQ_BF16 layout (kvq_append with KVQ_BF16,
+ * its own block tables); the caller quantizes a group once it is complete.
+ *
+ * Device layouts (one layer, K and V separate):
+ *   codes    [num_blocks][n_kv_heads][16 * head_dim * b / 8] bytes per page.
+ *            A page is made of 16-code units of 2b bytes. K: the unit of (token
+ *            t, channels 16c .. 16c+15) is unit ((t/8) * head_dim/16 + c) * 8 +
+ *            t%8 (the tensor-core K operand order); V: the unit of channel d
+ *            (tokens 0..15 of the page) is unit d. Inside a unit, code e = 4m + j
+ *            (m, j in 0..3): for b = 2 the unit is one 32-bit word and the code
+ *            is at bit 8j + 2m; for b = 4 it is word m/2, bit 8j + 4(m%2)
+ *            (little-endian words), so one shift and mask per m unpacks four
+ *            codes into bytes.
+ *   k_meta   [num_blocks][n_kv_heads][16][2] BF16 {s, z}: block i of a group
+ *            (i = its position in the sequence / 16, mod 8) holds channels
+ *            i*D/8 .. i*D/8 + D/8 - 1 of the group's K (entries 0 .. D/8-1).
+ *   v_meta   [num_blocks][n_kv_heads][16][2] BF16 {s, z} per token.
+ */
+
+/*
+ * Quantize whole groups. k, v: device [num_tokens][n_kv_heads][head_dim] BF16,
+ * num_tokens a multiple of 128: every run of 128 tokens is one complete group
+ * (positions 128g .. 128g+127 of one sequence, in order). slot_mapping: device
+ * [num_tokens] int64; the 16 tokens of a block must fill it in order (slot %
+ * 16 == token % 16, one block per 16 tokens). A group whose slots are all
+ * negative is skipped; one that breaks the rule above or leaves the pool is
+ * skipped and sets KVQ_DEVERR_SLOT. fmt: KVQ_KIVI2 or KVQ_KIVI4.
+ * Returns KVQ_ERR_ARG for a token count that is not a multiple of 128.
+ */
+int kvq_kivi_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                    void* k_codes, void* v_codes, void* k_meta, void* v_meta, kvq_fmt fmt,
+                    const kvq_dims* dims, kvq_stream_t stream);
+
+/*
+ * Decode attention over each sequence's quantized groups and its residual:
+ *   out[b][h] = softmax over the union of (quant_lens[b] tokens read through
+ *   block_tables[b], dequantized as above) and (res_lens[b] BF16 tokens read
+ *   through res_tables[b] from res_k / res_v), as kvq_decode_attn defines it.
+ * quant_lens[b] must be a multiple of 128 (a length that is not is cut to its
+ * whole groups and sets KVQ_DEVERR_CONTEXT); max_quant_len (a multiple of 128)
+ * and max_res_len bound them. dims describes the low-bit pool, res_dims the
+ * residual BF16 pool (same heads and head_dim). meta: host array {k_meta,
+ * v_meta}. The groups run on the tensor cores from the codes (the query is
+ * rebuilt per group with its channel scales), the residual through the BF16
+ * decode kernel, and one merge combines both. workspace: at least
+ * kvq_kivi_decode_workspace_bytes(...) bytes.
+ */
+size_t kvq_kivi_decode_workspace_bytes(int32_t batch, int32_t max_quant_len, int32_t max_res_len,
+                                       kvq_fmt fmt, const kvq_dims* dims,
+                                       const kvq_dims* res_dims);
+int kvq_kivi_decode_attn(const void* q, int32_t batch, const void* k_codes, const void* v_codes,
+                         const void* const* meta, const int32_t* block_tables,
+                         const int32_t* quant_lens, int32_t max_quant_len, const void* res_k,
+                         const void* res_v, const int32_t* res_tables, const int32_t* res_lens,
+                         int32_t max_res_len, float sm_scale, void* out, kvq_out_dtype out_dtype,
+                         void* workspace, size_t workspace_bytes, kvq_fmt fmt,
+                         const kvq_dims* dims, const kvq_dims* res_dims, kvq_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Device error word and the decode wait bound.                               */

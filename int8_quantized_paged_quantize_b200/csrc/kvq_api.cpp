@@ -288,4 +288,74 @@ int kvq_prefill_attn(const void* q, int32_t batch, int32_t chunk_len, const void
                        partition_tokens, fmt, dims, stream);
 }
 
+// ---------------------------------------------------------------- KIVI-style low-bit cache
+int kvq_kivi_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                    void* k_codes, void* v_codes, void* k_meta, void* v_meta, kvq_fmt fmt,
+                    const kvq_dims* dims, kvq_stream_t stream) {
+  if (!fmt_kivi(fmt) || num_tokens < 0 || num_tokens % 128 != 0) return KVQ_ERR_ARG;
+  int rc = check_dims(dims);
+  if (rc != KVQ_OK) return rc;
+  if (num_tokens == 0) return KVQ_OK;
+  if (!dev_ok(k) || !dev_ok(v) || !dev_ok(slot_mapping) || !dev_ok(k_codes) || !dev_ok(v_codes) ||
+      !dev_ok(k_meta) || !dev_ok(v_meta))
+    return KVQ_ERR_ARG;
+  return cuda_rc(launch_kivi_append(k, v, slot_mapping, num_tokens, k_codes, v_codes, k_meta, v_meta,
+                                    kivi_bits(fmt), *dims, stream));
+}
+
+namespace {
+int kivi_plans(int32_t batch, int32_t max_quant_len, int32_t max_res_len, kvq_fmt fmt,
+               const kvq_dims* dims, const kvq_dims* res_dims, DecodePlan* pa, DecodePlan* pb) {
+  if (!fmt_kivi(fmt) || batch < 0 || max_quant_len < 0 || max_res_len < 0) return KVQ_ERR_ARG;
+  int rc = check_dims(dims);
+  if (rc != KVQ_OK) return rc;
+  rc = check_dims(res_dims);
+  if (rc != KVQ_OK) return rc;
+  if (res_dims->n_kv_heads != dims->n_kv_heads || res_dims->n_q_heads != dims->n_q_heads ||
+      res_dims->head_dim != dims->head_dim)
+    return KVQ_ERR_ARG;
+  if (max_quant_len % 128 != 0) return KVQ_ERR_ARG;
+  if (int64_t(max_quant_len) > int64_t(dims->max_blocks_per_seq) * dims->block_size ||
+      int64_t(max_res_len) > int64_t(res_dims->max_blocks_per_seq) * res_dims->block_size)
+    return KVQ_ERR_ARG;
+  rc = make_plan(batch, max_quant_len, 0, dims, pa);
+  if (rc != KVQ_OK) return rc;
+  return make_plan(batch, max_res_len, 0, res_dims, pb);
+}
+}  // namespace
+
+size_t kvq_kivi_decode_workspace_bytes(int32_t batch, int32_t max_quant_len, int32_t max_res_len,
+                                       kvq_fmt fmt, const kvq_dims* dims,
+                                       const kvq_dims* res_dims) {
+  DecodePlan pa, pb;
+  if (kivi_plans(batch, max_quant_len, max_res_len, fmt, dims, res_dims, &pa, &pb) != KVQ_OK)
+    return 0;
+  return pa.total + pb.total;
+}
+
+int kvq_kivi_decode_attn(const void* q, int32_t batch, const void* k_codes, const void* v_codes,
+                         const void* const* meta, const int32_t* block_tables,
+                         const int32_t* quant_lens, int32_t max_quant_len, const void* res_k,
+                         const void* res_v, const int32_t* res_tables, const int32_t* res_lens,
+                         int32_t max_res_len, float sm_scale, void* out, kvq_out_dtype out_dtype,
+                         void* workspace, size_t workspace_bytes, kvq_fmt fmt,
+                         const kvq_dims* dims, const kvq_dims* res_dims, kvq_stream_t stream) {
+  DecodePlan pa, pb;
+  int rc = kivi_plans(batch, max_quant_len, max_res_len, fmt, dims, res_dims, &pa, &pb);
+  if (rc != KVQ_OK) return rc;
+  if (out_dtype != KVQ_OUT_BF16 && out_dtype != KVQ_OUT_F32) return KVQ_ERR_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!dev_ok(q) || !dev_ok(k_codes) || !dev_ok(v_codes) || !meta || !dev_ok(meta[0]) ||
+      !dev_ok(meta[1]) || !dev_ok(block_tables) || !dev_ok(quant_lens) || !dev_ok(res_k) ||
+      !dev_ok(res_v) || !dev_ok(res_tables) || !dev_ok(res_lens) || !dev_ok(out) ||
+      !dev_ok(workspace))
+    return KVQ_ERR_ARG;
+  if (!std::isfinite(sm_scale)) return KVQ_ERR_ARG;
+  if (workspace_bytes < pa.total + pb.total) return KVQ_ERR_WORKSPACE;
+  return cuda_rc(launch_kivi_decode(q, batch, k_codes, v_codes, meta[0], meta[1], block_tables,
+                                    quant_lens, max_quant_len, res_k, res_v, res_tables, res_lens,
+                                    max_res_len, sm_scale, out, out_dtype == KVQ_OUT_F32, workspace,
+                                    pa, pb, kivi_bits(fmt), *dims, *res_dims, stream));
+}
+
 }  // extern "C"

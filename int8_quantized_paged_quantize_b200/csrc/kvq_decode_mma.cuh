@@ -139,12 +139,13 @@ struct PieceWalk {
   int b, h, lo, hi;          // sequence, KV head, tiles [lo, hi) of that sequence
   int nt, ctx;               // tiles and tokens of sequence b
   int ctx_next;              // length of sequence b + 1 (0 past the batch)
+  int gmask;                 // lengths are ANDed with it (~127: whole 128-token groups)
   long long P;               // cost per head of sequences 0 .. b-1
   long long g, gend, end;    // cost positions: this piece's start and end; end of the share
   bool done;
 
   __device__ __forceinline__ void load_next(const int32_t* ctx_lens, int B, int max_ctx, int W) {
-    ctx_next = (b + 1 < B) ? mma_seq_ctx(ctx_lens, b + 1, max_ctx, W) : 0;
+    ctx_next = (b + 1 < B) ? (mma_seq_ctx(ctx_lens, b + 1, max_ctx, W) & gmask) : 0;
   }
   __device__ __forceinline__ void next_run(int Hk, const int32_t* ctx_lens, int B, int max_ctx,
                                            int W) {
@@ -180,9 +181,11 @@ struct PieceWalk {
     }
   }
   __device__ __forceinline__ void init(int b0, long long P0, long long start, long long end_,
-                                       int Hk, const int32_t* ctx_lens, int B, int max_ctx, int W) {
+                                       int Hk, const int32_t* ctx_lens, int B, int max_ctx, int W,
+                                       int gmask_ = -1) {
     b = b0; P = P0; g = start; end = end_;
-    ctx = mma_seq_ctx(ctx_lens, b, max_ctx, W);
+    gmask = gmask_;
+    ctx = mma_seq_ctx(ctx_lens, b, max_ctx, W) & gmask;
     nt = (ctx + 127) / 128;
     load_next(ctx_lens, B, max_ctx, W);
     lo = hi = 0;

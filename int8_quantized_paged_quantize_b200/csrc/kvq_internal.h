@@ -20,7 +20,11 @@ inline bool fmt_fp8(kvq_fmt f) { return f == KVQ_FP8_E4M3 || f == KVQ_FP8_E5M2; 
 inline int meta_values(kvq_fmt f) { return fmt_fp8(f) ? 1 : (f == KVQ_INT8_ASYM ? 2 : 0); }
 // Static-scale INT8: one scale per (KV head, channel) or one per cache.
 inline bool fmt_static(kvq_fmt f) { return f == KVQ_INT8_CHANNEL || f == KVQ_INT8_TENSOR; }
+// The 8-bit / BF16 formats of kvq_append and kvq_decode_attn.
 inline bool fmt_valid(int f) { return f >= KVQ_BF16 && f <= KVQ_INT8_TENSOR; }
+// The KIVI-style low-bit formats (kvq_kivi_* calls) and their code bits.
+inline bool fmt_kivi(int f) { return f == KVQ_KIVI2 || f == KVQ_KIVI4; }
+inline int kivi_bits(int f) { return f == KVQ_KIVI2 ? 2 : 4; }
 
 // Checks the shape rules of kvq.h. Returns KVQ_OK, KVQ_ERR_ARG or KVQ_ERR_UNSUPPORTED.
 int check_dims(const kvq_dims* d);
@@ -82,5 +86,14 @@ int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* 
 int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* out, bool out_f32,
                         const void* ws, const DecodePlan& plan, const kvq_dims& d, void* stream);
 int read_device_error(uint32_t* flags, int clear);
+int launch_kivi_decode(const void* q, int32_t B, const void* kc, const void* vc, const void* km,
+                       const void* vm, const int32_t* tables, const int32_t* qlens,
+                       int32_t max_qlen, const void* rk, const void* rv,
+                       const int32_t* rtables, const int32_t* rlens, int32_t max_rlen,
+                       float sm_scale, void* out, bool out_f32, void* ws, const DecodePlan& pa,
+                       const DecodePlan& pb, int bits, const kvq_dims& d, const kvq_dims& rd,
+                       void* stream);
+int launch_kivi_append(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
+                       void* vc, void* km, void* vm, int bits, const kvq_dims& d, void* stream);
 
 }  // namespace kvq

@@ -68,6 +68,8 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 #include <utility>
 
 #include "kvq_decode_mma.cuh"
+#include "kvq_decode_kivi.cuh"
+#include "kvq_kivi.cuh"
 
 namespace kvq {
 
@@ -560,6 +562,47 @@ __global__ void __launch_bounds__(128) merge_kernel(const int32_t* __restrict__ 
   else out[int64_t(bq) * D + d] = __float2bfloat16_rn(r);
 }
 
+// Merge of two partial sets of the same rows: the quantized groups' partials
+// (a) and the residual tokens' (b), each with its own context lengths, slot
+// count and per-(sequence, row group) counts.
+template <int D, typename OutT>
+__global__ void __launch_bounds__(128) merge2_kernel(
+    int Hq, int G, const int32_t* __restrict__ ctx_a, int slots_a, int max_a, int W_a,
+    const float* __restrict__ po_a, const float* __restrict__ pml_a, const int32_t* __restrict__ pc_a,
+    const int32_t* __restrict__ ctx_b, int slots_b, int max_b, int W_b,
+    const float* __restrict__ po_b, const float* __restrict__ pml_b, const int32_t* __restrict__ pc_b,
+    int group_mask_a, OutT* __restrict__ out) {
+  const int bq = blockIdx.x;
+  const int b = bq / Hq;
+  const int d = threadIdx.x;
+  int ca = ctx_a[b], cb = ctx_b[b];
+  if (ca < 0 || ca > max_a || int64_t(ca) > int64_t(W_a) * kBlockSize) ca = 0;
+  ca &= group_mask_a;
+  if (cb < 0 || cb > max_b || int64_t(cb) > int64_t(W_b) * kBlockSize) cb = 0;
+  const int na = ca > 0 ? min(slots_a, max(0, pc_a[bq / G])) : 0;
+  const int nb = cb > 0 ? min(slots_b, max(0, pc_b[bq / G])) : 0;
+  const int64_t ra = int64_t(bq) * slots_a, rb = int64_t(bq) * slots_b;
+  float M = -INFINITY;
+  for (int s = 0; s < na; ++s) M = fmaxf(M, pml_a[(ra + s) * 2]);
+  for (int s = 0; s < nb; ++s) M = fmaxf(M, pml_b[(rb + s) * 2]);
+  float o = 0.f, l = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < na; ++s) {
+      const float f = exp2f(pml_a[(ra + s) * 2] - M);
+      l += pml_a[(ra + s) * 2 + 1] * f;
+      o += po_a[(ra + s) * D + d] * f;
+    }
+    for (int s = 0; s < nb; ++s) {
+      const float f = exp2f(pml_b[(rb + s) * 2] - M);
+      l += pml_b[(rb + s) * 2 + 1] * f;
+      o += po_b[(rb + s) * D + d] * f;
+    }
+  }
+  const float r = l > 0.f ? o / l : 0.f;
+  if constexpr (sizeof(OutT) == 4) out[int64_t(bq) * D + d] = r;
+  else out[int64_t(bq) * D + d] = __float2bfloat16_rn(r);
+}
+
 // ------------------------------------------------------------------ launchers
 namespace {
 constexpr float kLog2e = 1.4426950408889634f;
@@ -708,6 +751,95 @@ int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* ou
                                                            pml, pcnt,
                                                            static_cast<__nv_bfloat16*>(out));
   }
+  return int(cudaGetLastError());
+}
+
+namespace {
+template <int D, int G, int BITS>
+cudaError_t kivi_dispatch3(const void* q, int32_t B, const void* kc, const void* vc, const void* km,
+                           const void* vm, const int32_t* tables, const int32_t* lens,
+                           int32_t max_len, float sm_scale, const DecodePlan& plan, void* ws,
+                           const kvq_dims& d, cudaStream_t st) {
+  using C = KiviCfg<D, G, BITS>;
+  auto kern = decode_kivi_kernel<D, G, BITS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           int(cudaSharedmemCarveoutMaxShared));
+  if (e != cudaSuccess) return e;
+  int dev = 0, smem_sm = 0, reserved = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  if (e != cudaSuccess) return e;
+  const int per_sm = std::max(1, std::min(2, smem_sm / (C::SMEM + reserved)));
+  float* po = static_cast<float*>(ws);
+  float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
+  int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
+  const int64_t grid = int64_t(device_sm_count()) * per_sm;
+  kern<<<dim3(unsigned(grid)), 256, C::SMEM, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
+      static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(km),
+      static_cast<const __nv_bfloat16*>(vm), tables, lens, B, d.n_kv_heads, d.num_blocks,
+      d.max_blocks_per_seq, max_len, plan.partition / kTileTokens, plan.slots, sm_scale * kLog2e,
+      decode_wait_limit(), po, pml, pcnt);
+  return cudaGetLastError();
+}
+
+template <int D, int BITS>
+cudaError_t kivi_dispatch2(int G, const void* q, int32_t B, const void* kc, const void* vc,
+                           const void* km, const void* vm, const int32_t* tables,
+                           const int32_t* lens, int32_t max_len, float sm_scale,
+                           const DecodePlan& plan, void* ws, const kvq_dims& d, cudaStream_t st) {
+  switch (G) {
+    case 1: return kivi_dispatch3<D, 1, BITS>(q, B, kc, vc, km, vm, tables, lens, max_len, sm_scale, plan, ws, d, st);
+    case 2: return kivi_dispatch3<D, 2, BITS>(q, B, kc, vc, km, vm, tables, lens, max_len, sm_scale, plan, ws, d, st);
+    case 4: return kivi_dispatch3<D, 4, BITS>(q, B, kc, vc, km, vm, tables, lens, max_len, sm_scale, plan, ws, d, st);
+    default: return kivi_dispatch3<D, 8, BITS>(q, B, kc, vc, km, vm, tables, lens, max_len, sm_scale, plan, ws, d, st);
+  }
+}
+}  // namespace
+
+int launch_kivi_decode(const void* q, int32_t B, const void* kc, const void* vc, const void* km,
+                       const void* vm, const int32_t* tables, const int32_t* qlens,
+                       int32_t max_qlen, const void* rk, const void* rv,
+                       const int32_t* rtables, const int32_t* rlens, int32_t max_rlen,
+                       float sm_scale, void* out, bool out_f32, void* ws, const DecodePlan& pa,
+                       const DecodePlan& pb, int bits, const kvq_dims& d, const kvq_dims& rd,
+                       void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = d.n_q_heads / d.n_kv_heads;
+  void* ws_b = static_cast<char*>(ws) + pa.total;
+  cudaError_t e;
+  // the quantized groups
+  if (d.head_dim == 128)
+    e = bits == 2 ? kivi_dispatch2<128, 2>(G, q, B, kc, vc, km, vm, tables, qlens, max_qlen, sm_scale, pa, ws, d, st)
+                  : kivi_dispatch2<128, 4>(G, q, B, kc, vc, km, vm, tables, qlens, max_qlen, sm_scale, pa, ws, d, st);
+  else
+    e = bits == 2 ? kivi_dispatch2<64, 2>(G, q, B, kc, vc, km, vm, tables, qlens, max_qlen, sm_scale, pa, ws, d, st)
+                  : kivi_dispatch2<64, 4>(G, q, B, kc, vc, km, vm, tables, qlens, max_qlen, sm_scale, pa, ws, d, st);
+  if (e != cudaSuccess) return int(e);
+  // the residual tokens, through the BF16 kernel
+  const int rc = launch_decode_partial(q, B, rk, rv, nullptr, nullptr, rtables, rlens, max_rlen,
+                                       sm_scale, pb, ws_b, KVQ_BF16, rd, stream, 1);
+  if (rc != 0) return rc;
+  const float* poa = static_cast<const float*>(ws);
+  const float* pmla = reinterpret_cast<const float*>(static_cast<const char*>(ws) + pa.o_bytes);
+  const int32_t* pca = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + pa.o_bytes + pa.ml_bytes);
+  const float* pob = static_cast<const float*>(ws_b);
+  const float* pmlb = reinterpret_cast<const float*>(static_cast<const char*>(ws_b) + pb.o_bytes);
+  const int32_t* pcb = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws_b) + pb.o_bytes + pb.ml_bytes);
+  const dim3 grid(unsigned(int64_t(B) * d.n_q_heads));
+  const int Hq = d.n_q_heads;
+#define KVQ_M2(DD, OT) merge2_kernel<DD, OT><<<grid, DD, 0, st>>>(Hq, G, qlens, pa.slots, max_qlen, \
+      d.max_blocks_per_seq, poa, pmla, pca, rlens, pb.slots, max_rlen, rd.max_blocks_per_seq, pob, pmlb, pcb, ~127, \
+      static_cast<OT*>(out))
+  if (d.head_dim == 128) {
+    if (out_f32) KVQ_M2(128, float); else KVQ_M2(128, __nv_bfloat16);
+  } else {
+    if (out_f32) KVQ_M2(64, float); else KVQ_M2(64, __nv_bfloat16);
+  }
+#undef KVQ_M2
   return int(cudaGetLastError());
 }
 

@@ -45,10 +45,17 @@ int check_dims(const kvq_dims* d) {
 extern "C" {
 
 int kvq_cache_bytes(const kvq_dims* dims, kvq_fmt fmt, size_t* cache_bytes, size_t* meta_bytes) {
-  if (!kvq::fmt_valid(fmt) || !cache_bytes || !meta_bytes) return KVQ_ERR_ARG;
+  if (!(kvq::fmt_valid(fmt) || kvq::fmt_kivi(fmt)) || !cache_bytes || !meta_bytes) return KVQ_ERR_ARG;
   const int rc = kvq::check_dims(dims);
   if (rc != KVQ_OK) return rc;
   const size_t rows = size_t(dims->num_blocks) * dims->n_kv_heads * dims->block_size;
+  if (kvq::fmt_kivi(fmt)) {
+    // b-bit codes; 16 BF16 (s, z) pairs per (block, KV head): a token's for V,
+    // D/8 channels' of the block's group for K (the same array size)
+    *cache_bytes = rows * dims->head_dim * kvq::kivi_bits(fmt) / 8;
+    *meta_bytes = rows * 2 * 2;
+    return KVQ_OK;
+  }
   *cache_bytes = rows * dims->head_dim * kvq::elem_bytes(fmt);
   if (fmt == KVQ_INT8_CHANNEL)
     *meta_bytes = size_t(dims->n_kv_heads) * dims->head_dim * 2;
@@ -60,7 +67,7 @@ int kvq_cache_bytes(const kvq_dims* dims, kvq_fmt fmt, size_t* cache_bytes, size
 }
 
 int kvq_pool_create(const kvq_dims* dims, kvq_fmt fmt, int32_t n_layers, kvq_pool** out) {
-  if (!out || !kvq::fmt_valid(fmt) || n_layers <= 0) return KVQ_ERR_ARG;
+  if (!out || !(kvq::fmt_valid(fmt) || kvq::fmt_kivi(fmt)) || n_layers <= 0) return KVQ_ERR_ARG;
   const int rc = kvq::check_dims(dims);
   if (rc != KVQ_OK) return rc;
   kvq_pool* p = new (std::nothrow) kvq_pool;

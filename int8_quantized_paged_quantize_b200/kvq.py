@@ -19,7 +19,9 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so"
 
 # int8c / int8t: symmetric INT8 with static BF16 scales given by the caller,
 # one per (KV head, channel) or one per cache (K and V separately)
-FMT = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 3, "int8c": 4, "int8t": 5}
+FMT = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 3, "int8c": 4, "int8t": 5, "kivi2": 6, "kivi4": 7}
+KIVI_BITS = {"kivi2": 2, "kivi4": 4}
+KIVI_GROUP = 128
 ELEM_BYTES = {"bf16": 2, "fp8": 1, "int8": 1, "e5m2": 1, "int8c": 1, "int8t": 1}
 META_VALUES = {"bf16": 0, "fp8": 1, "int8": 2, "e5m2": 1, "int8c": 0, "int8t": 0}   # per token
 STATIC_FORMATS = ("int8c", "int8t")
@@ -60,6 +62,12 @@ _SIGNATURES = [
     ("kvq_decode_verify", _c.c_int, [_P, _c.c_int32, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32,
                                      _c.c_float, _P, _c.c_int, _P, _c.c_size_t, _c.c_int32, _c.c_int,
                                      _P, _P]),
+    ("kvq_kivi_append", _c.c_int, [_P, _P, _P, _c.c_int32, _P, _P, _P, _P, _c.c_int, _P, _P]),
+    ("kvq_kivi_decode_workspace_bytes", _c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int,
+                                                      _P, _P]),
+    ("kvq_kivi_decode_attn", _c.c_int, [_P, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32, _P, _P, _P,
+                                        _P, _c.c_int32, _c.c_float, _P, _c.c_int, _P, _c.c_size_t,
+                                        _c.c_int, _P, _P, _P]),
     ("kvq_prefill_attn_workspace_bytes", _c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32,
                                                        _c.c_int32, _c.c_int, _P]),
     ("kvq_prefill_attn", _c.c_int, [_P, _c.c_int32, _c.c_int32, _P, _P, _P, _P, _P, _c.c_int32,
@@ -447,3 +455,80 @@ class LayerCache:
         v = self.v if blocks is None else self.v[blocks]
         return v.permute(0, 1, 2, 4, 3).reshape(v.shape[0], v.shape[1], BLOCK_SIZE,
                                                 self.dims.head_dim)
+
+
+# --------------------------------------------------------------------------- KIVI-style cache
+@dataclass
+class KiviCache:
+    """One layer's KIVI-style low-bit cache (torch-owned device memory): packed
+    b-bit K and V pages, their BF16 (scale, minimum) arrays, and a BF16 cache
+    of its own for each sequence's residual tokens (those after its last
+    complete 128-token group)."""
+    fmt: str
+    dims: Dims
+    k: torch.Tensor            # [NB][Hk][16 * D * b / 8] uint8, packed K pages
+    v: torch.Tensor            # [NB][Hk][16 * D * b / 8] uint8, packed V pages
+    k_meta: torch.Tensor       # [NB][Hk][16][2] bf16: page i of a group holds channels i*D/8..
+    v_meta: torch.Tensor       # [NB][Hk][16][2] bf16: per token
+    residual: LayerCache       # BF16 cache of the residual tokens
+
+    @staticmethod
+    def allocate(fmt, d: Dims, res_dims: Dims, device="cuda"):
+        if fmt not in KIVI_BITS:
+            raise KvqError("KIVI formats: kivi2, kivi4")
+        nb, hk, D = d.num_blocks, d.n_kv_heads, d.head_dim
+        pb = BLOCK_SIZE * D * KIVI_BITS[fmt] // 8
+        k = torch.zeros((nb, hk, pb), dtype=torch.uint8, device=device)
+        v = torch.zeros((nb, hk, pb), dtype=torch.uint8, device=device)
+        km = torch.zeros((nb, hk, BLOCK_SIZE, 2), dtype=torch.bfloat16, device=device)
+        vm = torch.zeros((nb, hk, BLOCK_SIZE, 2), dtype=torch.bfloat16, device=device)
+        return KiviCache(fmt, d, k, v, km, vm, LayerCache.allocate("bf16", res_dims, device))
+
+    def append_groups(self, k, v, slot_mapping, stream=None):
+        """Quantize whole 128-token groups (kvq_kivi_append): k, v [T][Hk][D] bf16
+        with T a multiple of 128, each run of 128 tokens one group whose slots fill
+        eight pages in order."""
+        _need(k, torch.bfloat16, "k")
+        _need(v, torch.bfloat16, "v")
+        _need(slot_mapping, torch.int64, "slot_mapping")
+        _check(lib().kvq_kivi_append(_ptr(k), _ptr(v), _ptr(slot_mapping), slot_mapping.numel(),
+                                     _ptr(self.k), _ptr(self.v), _ptr(self.k_meta), _ptr(self.v_meta),
+                                     FMT[self.fmt], ctypes.byref(self.dims), _stream(stream)),
+               "kvq_kivi_append")
+
+    def workspace(self, batch, max_quant_len, max_res_len, device="cuda"):
+        n = lib().kvq_kivi_decode_workspace_bytes(batch, int(max_quant_len), int(max_res_len),
+                                                  FMT[self.fmt], ctypes.byref(self.dims),
+                                                  ctypes.byref(self.residual.dims))
+        if n == 0 and batch > 0:
+            raise KvqError("kvq_kivi_decode_workspace_bytes: invalid arguments")
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+    def decode(self, q, block_tables, quant_lens, max_quant_len, res_tables, res_lens, max_res_len,
+               sm_scale=None, out=None, workspace=None, stream=None, out_dtype=torch.bfloat16):
+        """Decode attention over each sequence's quantized groups (quant_lens[b]
+        tokens, a multiple of 128) and its residual tokens (res_lens[b])."""
+        if sm_scale is None:
+            sm_scale = 1.0 / math.sqrt(self.dims.head_dim)
+        _need(q, torch.bfloat16, "q")
+        for t, name in ((block_tables, "block_tables"), (quant_lens, "quant_lens"),
+                        (res_tables, "res_tables"), (res_lens, "res_lens")):
+            _need(t, torch.int32, name)
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        _need_out(out)
+        B = q.shape[0]
+        if workspace is None:
+            workspace = self.workspace(B, max_quant_len, max_res_len, q.device)
+        meta = (ctypes.c_void_p * 2)(self.k_meta.data_ptr(), self.v_meta.data_ptr())
+        r = self.residual
+        _check(lib().kvq_kivi_decode_attn(_ptr(q), B, _ptr(self.k), _ptr(self.v), meta,
+                                          _ptr(block_tables), _ptr(quant_lens), int(max_quant_len),
+                                          _ptr(r.k), _ptr(r.v), _ptr(res_tables), _ptr(res_lens),
+                                          int(max_res_len), float(sm_scale), _ptr(out),
+                                          _out_dtype(out), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          FMT[self.fmt], ctypes.byref(self.dims),
+                                          ctypes.byref(r.dims), _stream(stream)),
+               "kvq_kivi_decode_attn")
+        return out

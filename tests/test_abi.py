@@ -181,3 +181,27 @@ def test_multi_query_workspace_and_limits(kvq):
                   null, 0, 0, 1, C.byref(d), None) == -1
         assert fn(null, 0, 64, null, null, scales, null, null, 64, C.c_float(0.1), null, 0,
                   null, 0, 0, 1, C.byref(d), None) == 0
+
+
+def test_kivi_host_checks(kvq):
+    """kvq_kivi_*: token counts and lengths in whole groups, matching residual
+    dims, workspace sizes; refused before any device work."""
+    import ctypes as C
+    L = kvq.lib()
+    d = kvq.dims(1024, 2, 8, 128, 64)
+    rd = kvq.dims(64, 2, 8, 128, 8)
+    null = C.c_void_p(0)
+    assert L.kvq_kivi_append(null, null, null, 100, null, null, null, null, 6, C.byref(d), None) == -1
+    assert L.kvq_kivi_append(null, null, null, 0, null, null, null, null, 6, C.byref(d), None) == 0
+    assert L.kvq_kivi_append(null, null, null, 128, null, null, null, null, 1, C.byref(d), None) == -1
+    assert L.kvq_kivi_append(null, null, null, 128, null, null, null, null, 7, C.byref(d), None) == -1
+    ws = L.kvq_kivi_decode_workspace_bytes(4, 1024, 100, 6, C.byref(d), C.byref(rd))
+    assert ws == L.kvq_decode_workspace_bytes(4, 1024, 0, 1, C.byref(d)) + \
+        L.kvq_decode_workspace_bytes(4, 100, 0, 0, C.byref(rd))
+    assert L.kvq_kivi_decode_workspace_bytes(4, 1000, 100, 6, C.byref(d), C.byref(rd)) == 0   # not whole groups
+    bad = kvq.dims(64, 2, 16, 128, 8)                                                           # other heads
+    assert L.kvq_kivi_decode_workspace_bytes(4, 1024, 100, 6, C.byref(d), C.byref(bad)) == 0
+    assert L.kvq_kivi_decode_workspace_bytes(4, 1024, 100, 2, C.byref(d), C.byref(rd)) == 0     # not KIVI
+    # sizes: 2-bit codes are a quarter of the 8-bit formats' bytes
+    assert kvq.cache_bytes(d, "kivi2")[0] * 4 == kvq.cache_bytes(d, "int8")[0]
+    assert kvq.cache_bytes(d, "kivi4")[0] * 2 == kvq.cache_bytes(d, "int8")[0]
