@@ -785,6 +785,90 @@ def long_context_run(w, fmt, seed, hist, bulk_kv, layout, hbm_peak, flush):
     return r
 
 
+def kivi_rate(w, hist, fmt, seed, hbm_peak, flush, reps=10, warmup=3):
+    """Decode over the KIVI-style cache (kvq_kivi_decode_attn) for the workload:
+    every sequence's complete 128-token groups quantized by kvq_kivi_append, the
+    rest (and one step token) in a BF16 residual cache. L2 flushed before every
+    timed call. Algorithmic bytes per token and KV head: the 2b-bit K and V
+    codes, V's (s, z) and K's (s, z) spread over its group."""
+    from int8_quantized_paged_quantize_b200 import kvq
+    bits = kvq.KIVI_BITS[fmt]
+    dev = torch.device("cuda")
+    ctx = WL.context_lengths(w, seed) + w.bulk_append
+    groups = ctx // 128
+    res = ctx % 128 + 1                               # + this step's token
+    rng = np.random.default_rng(seed)
+    nq = int(groups.sum()) * 8
+    perm = rng.permutation(max(nq, 1))
+    Wq = max(1, int(groups.max()) * 8)
+    qt = np.full((w.batch, Wq), -1, dtype=np.int32)
+    nr = int(((res + 15) // 16).sum())
+    rperm = rng.permutation(nr)
+    Wr = int(((res + 15) // 16).max())
+    rt = np.full((w.batch, Wr), -1, dtype=np.int32)
+    a = r = 0
+    for b in range(w.batch):
+        qt[b, :8 * groups[b]] = perm[a:a + 8 * groups[b]]
+        a += 8 * groups[b]
+        n = (res[b] + 15) // 16
+        rt[b, :n] = rperm[r:r + n]
+        r += n
+    d = kvq.dims(max(nq, 1), w.n_kv_heads, w.n_q_heads, w.head_dim, Wq)
+    rd = kvq.dims(nr, w.n_kv_heads, w.n_q_heads, w.head_dim, Wr)
+    cache = kvq.KiviCache.allocate(fmt, d, rd)
+    K, V = hist
+    q0, kn, vn = WL.step_inputs(w, 0, seed)
+    at = 0
+    for b in range(w.batch):
+        m = int(groups[b]) * 128
+        pos = np.arange(m)
+        if m:
+            sl = torch.from_numpy(qt[b][pos // 16].astype(np.int64) * 16 + pos % 16)
+            cache.append_groups(K[at:at + m].to(dev), V[at:at + m].to(dev), sl.to(dev))
+        rest = int(ctx[b]) - m
+        kr = torch.cat([K[at + m:at + m + rest], kn[b:b + 1]])
+        vr = torch.cat([V[at + m:at + m + rest], vn[b:b + 1]])
+        pos = np.arange(rest + 1)
+        sl = torch.from_numpy(rt[b][pos // 16].astype(np.int64) * 16 + pos % 16)
+        cache.residual.append(kr.to(dev), vr.to(dev), sl.to(dev))
+        at += int(ctx[b])
+    torch.cuda.synchronize()
+    q = q0.to(dev)
+    qtd, rtd = torch.from_numpy(qt).to(dev), torch.from_numpy(rt).to(dev)
+    qld = torch.from_numpy((groups * 128).astype(np.int32)).to(dev)
+    rld = torch.from_numpy(res.astype(np.int32)).to(dev)
+    maxq, maxr = int(groups.max()) * 128, int(res.max())
+    ws = cache.workspace(w.batch, maxq, maxr)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+
+    def call():
+        cache.decode(q, qtd, qld, maxq, rtd, rld, maxr, sm_scale=w.sm_scale, out=out, workspace=ws)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+    per_tok = w.n_kv_heads * (2 * w.head_dim * bits / 8 + 4 + w.head_dim * 4 / 128)
+    qbytes = float(groups.sum()) * 128 * per_tok
+    rbytes = float(res.sum()) * w.n_kv_heads * 2 * w.head_dim * 2
+    kv = qbytes + rbytes
+    del cache
+    torch.cuda.empty_cache()
+    return {"bits": bits, "ms": ms, "kv_gbs": kv / (ms * 1e-3) / 1e9,
+            "kv_frac_of_peak": kv / (ms * 1e-3) / 1e9 / hbm_peak,
+            "decode_seqs_per_s": w.batch / (ms * 1e-3),
+            "tokens_per_s": float(ctx.sum() + w.batch) / (ms * 1e-3),
+            "kv_bytes": kv, "bytes_per_token_head": per_tok / w.n_kv_heads,
+            "what": "groups on the tensor cores from the packed codes + BF16 residual + merge"}
+
+
 def configs_block(args, seed, hbm_peak, flush):
     """Workloads beside the headline, each as its specification runs it."""
     out = {}
@@ -928,6 +1012,13 @@ def main():
                 "max_abs": float(dev.max()), "mean_abs": float(dev.mean()),
                 "rel_l2": float((outs[f] - outs["bf16"]).norm() / max(float(outs["bf16"].norm()), 1e-30)),
                 "mean_abs_ref": float(ref.mean()), "step": 0}
+    kivi = {}
+    if not args.no_formats:
+        for f in ("kivi2", "kivi4"):
+            try:
+                kivi[f] = kivi_rate(wb, hist, f, seed, hbm_peak, flush)
+            except Exception as e:                # reported, never fatal to the main line
+                kivi[f] = {"error": f"{type(e).__name__}: {e}"[:200]}
     del st, hist
     torch.cuda.empty_cache()
 
@@ -971,6 +1062,7 @@ def main():
         "prefill": prefill,
         "clocks": clk,
         "formats": formats,
+        "kivi": kivi,
         "configs": configs,
         "cpu_baseline": cpu,
     }
