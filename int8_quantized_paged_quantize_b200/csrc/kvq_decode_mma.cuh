@@ -397,7 +397,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       if constexpr (C::MV > 0) {
         const int sblk = __shfl_sync(0xffffffffu, ids, sp & 7);
         if (sp < 8 && sblk >= 0 && sblk < NB) {
-          const int64_t off = (int64_t(sblk) * Hk + h / nrg) * C::METAB + sc * 16;
+          const int64_t off = (int64_t(sblk) * Hk + (nrg == 1 ? h : h / nrg)) * C::METAB + sc * 16;
           kv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(ks) + off));
           vv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vs) + off));
         }
@@ -430,7 +430,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       const int blk = __shfl_sync(0xffffffffu, id, p8);
       const bool mine = ((mask >> p8) & 1u) != 0u;
       const bool smine = C::MV > 0 && sp < 8 && ((mask >> sp) & 1u) != 0u;
-      const int64_t page = int64_t(blk) * Hk + h / nrg;
+      const int64_t page = int64_t(blk) * Hk + (nrg == 1 ? h : h / nrg);
       const uint32_t bytes = uint32_t(__popc(mask)) * uint32_t(C::PAGE);
       bool ok = true;
       // per stage: byte count, the page copies, then the scale stores and the

@@ -137,6 +137,19 @@ struct ScaleDiv {
   }
 };
 
+// Integer rounding by one addition: for |q| < 2^22, q + 1.5 * 2^23 lies in
+// [2^23, 2^24), where the float spacing is 1, so the sum is rint(q) (round to
+// nearest even) and its bit pattern is kRintBits + rint(q).
+constexpr float kRintMagic = 12582912.0f;
+constexpr int kRintBits = 0x4B400000;
+
+// The low bytes of four ints, packed little-endian.
+__device__ __forceinline__ uint32_t pack_low_bytes(int a, int b, int c, int d) {
+  const uint32_t lo = __byte_perm(uint32_t(a), uint32_t(b), 0x0040);
+  const uint32_t hi = __byte_perm(uint32_t(c), uint32_t(d), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
 // Max over the 16 lanes of this half warp (both halves reduce at once).
 __device__ __forceinline__ int half_warp_max(int v) {
 #pragma unroll
@@ -198,12 +211,16 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 32], RowC
         const ScaleDiv div(s);
         const float zq = fminf(fmaxf(-div(nlo), -1024.f), 1024.f);   // lo / s
         rc.zp = min(127, max(-128, -128 - __float2int_rn(zq)));
+        // code = clamp(rint(x / s) + zp, -128, 127): every x of the row lies in
+        // [lo, hi], so |x / s| stays near 255 and the rounding addition applies;
+        // the clamp runs on the sum's bits, shifted by zp
+        const int cmin = kRintBits - 128 - rc.zp, cmax = kRintBits + 127 - rc.zp;
+        int c[E];
 #pragma unroll
-        for (int i = 0; i < E; ++i) {
-          const float qf = fminf(fmaxf(div(x[i]), -1024.f), 1024.f);
-          const int c = min(127, max(-128, __float2int_rn(qf) + rc.zp));
-          rc.w[i >> 2] |= uint32_t(uint8_t(int8_t(c))) << (8 * (i & 3));
-        }
+        for (int i = 0; i < E; ++i)
+          c[i] = min(cmax, max(cmin, __float_as_int(__fadd_rn(div(x[i]), kRintMagic)))) + rc.zp;
+#pragma unroll
+        for (int i = 0; i < E; i += 4) rc.w[i >> 2] = pack_low_bytes(c[i], c[i + 1], c[i + 2], c[i + 3]);
       }
     }
   }
@@ -224,11 +241,12 @@ __device__ __forceinline__ void quantize_row_static(const uint32_t (&raw)[D / 32
   rc.s = __float2bfloat16_rn(0.f);
 #pragma unroll
   for (int i = 0; i < RowCodes<D, KVQ_INT8_CHANNEL>::WORDS; ++i) rc.w[i] = 0u;
+  int c[E];
 #pragma unroll
   for (int i = 0; i < E; ++i) {
     const float x = (i & 1) ? bf16_hi(raw[i / 2]) : bf16_lo(raw[i / 2]);
     const float s = sc[i], r = rc_[i];
-    int c = 0;
+    c[i] = 0;
     if (s > 0.f) {
       const float lim = s * 65536.f;
       const float xc = fminf(fmaxf(x, -lim), lim);
@@ -240,10 +258,12 @@ __device__ __forceinline__ void quantize_row_static(const uint32_t (&raw)[D / 32
       } else {
         q = __fdiv_rn(xc, s);
       }
-      c = min(127, max(-127, __float2int_rn(fminf(fmaxf(q, -1024.f), 1024.f))));
+      // |q| <= 65536 (x clamped above): the rounding addition applies
+      c[i] = min(kRintBits + 127, max(kRintBits - 127, __float_as_int(__fadd_rn(q, kRintMagic))));
     }
-    rc.w[i >> 2] |= uint32_t(uint8_t(int8_t(c))) << (8 * (i & 3));
   }
+#pragma unroll
+  for (int i = 0; i < E; i += 4) rc.w[i >> 2] = pack_low_bytes(c[i], c[i + 1], c[i + 2], c[i + 3]);
 }
 
 // Bytes [p, e) of the 16-byte chunk at dst (16-byte aligned) from w, with the
@@ -593,9 +613,11 @@ __global__ void __launch_bounds__(128) merge_kernel(const int32_t* __restrict__ 
       }
     }
   }
+  // l == 0: nothing attended (zeros); a NaN l (a piece that timed out wrote
+  // NaN markers) gives NaN
   float r[N];
 #pragma unroll
-  for (int i = 0; i < N; ++i) r[i] = l > 0.f ? o[i] / l : 0.f;
+  for (int i = 0; i < N; ++i) r[i] = l != 0.f ? o[i] / l : 0.f;
   OutT* dst = out + int64_t(bq) * D + lane * N;
   if constexpr (sizeof(OutT) == 4) {
     if constexpr (N == 4) *reinterpret_cast<float4*>(dst) = make_float4(r[0], r[1], r[2], r[3]);
@@ -647,7 +669,7 @@ __global__ void __launch_bounds__(128) merge2_kernel(
       o += po_b[(rb + s) * D + d] * f;
     }
   }
-  const float r = l > 0.f ? o / l : 0.f;
+  const float r = l != 0.f ? o / l : 0.f;            // NaN l (a timed-out piece): NaN
   if constexpr (sizeof(OutT) == 4) out[int64_t(bq) * D + d] = r;
   else out[int64_t(bq) * D + d] = __float2bfloat16_rn(r);
 }
