@@ -149,8 +149,9 @@ class ClockSampler:
 
 
 def measured_traffic(workload, fmt):
-    """DRAM bytes per decode launch from the committed ncu capture of this
-    workload, or None when there is none or the kernel sources changed since."""
+    """DRAM bytes (read + write) of one decode step's attention launches
+    (partials + merge) from the committed ncu capture of this workload, or None
+    when there is none or the kernel sources changed since."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -928,6 +929,7 @@ def main():
     ap.add_argument("--no-formats", action="store_true", help="skip the per-format comparison")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' block")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--no-multiquery", action="store_true", help="skip the verify / prefill entries")
     ap.add_argument("--bulk-append", choices=["aligned", "continued"], default=None,
                     help="only time one bulk append of 32,768 tokens and print its line")
     ap.add_argument("--reps", type=int, default=5, help="timed calls of --bulk-append")
@@ -970,14 +972,15 @@ def main():
     app_tok_s = sum_over_ranks(wb.batch, world) / (max_over_ranks(t["append"], world) * 1e-3)
     bulk_tok_s, bulk_ms, bulk_n = bulk_append_rate(st)
     verify, prefill = {}, {}
-    try:
-        verify = multi_query_rate(st, flush, 4, "verify")
-    except Exception as e:                        # reported, never fatal to the main line
-        verify = {"error": f"{type(e).__name__}: {e}"[:200]}
-    try:
-        prefill = multi_query_rate(st, flush, 64, "prefill", reps=3, warmup=1)
-    except Exception as e:
-        prefill = {"error": f"{type(e).__name__}: {e}"[:200]}
+    if not args.no_multiquery:
+        try:
+            verify = multi_query_rate(st, flush, 4, "verify")
+        except Exception as e:                    # reported, never fatal to the main line
+            verify = {"error": f"{type(e).__name__}: {e}"[:200]}
+        try:
+            prefill = multi_query_rate(st, flush, 64, "prefill", reps=3, warmup=1)
+        except Exception as e:
+            prefill = {"error": f"{type(e).__name__}: {e}"[:200]}
 
     e2e_ms, h2d, d2h = e2e_loop(st, args.steps, args.warmup, world, flush)
     e2e_ms = max_over_ranks(e2e_ms, world)

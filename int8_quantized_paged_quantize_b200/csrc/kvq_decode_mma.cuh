@@ -15,7 +15,7 @@
 // Work split (persistent, stream-K): the work list is every (sequence b,
 // virtual head h, 128-token tile) in order of b, then h, then tile, each (b, h) run
 // also costing kPieceCost units for opening and closing its piece. Each of
-// the N resident CTAs takes one contiguous, equal share of the total cost (N
+// the N CTA groups takes one contiguous, equal share of the total cost (N
 // is cut so that a share holds at least `unit_tiles` units). A share is a few
 // "pieces", a piece being the share's tiles of one (b, h); each piece ends in
 // an online-softmax partial (max, sum, unnormalised output) in a workspace
@@ -222,7 +222,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kc,
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
-    const int32_t* __restrict__ ctx_lens, int B, int Hv, int nrg, int NB, int W, int max_ctx,
+    const int32_t* __restrict__ ctx_lens, int B, int Hk, int nrg, int NB, int W, int max_ctx,
     int unit_tiles, int slots, float qk_scale, int per_tensor, int n_query,
     long long wait_limit, float* __restrict__ part_o,
     float* __restrict__ part_ml, int32_t* __restrict__ part_cnt) {
@@ -231,8 +231,12 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Hq = Hv * G;                                   // query rows of a sequence
-  const int Hk = Hv / nrg;                                 // KV heads
+  const int Hq = Hk * nrg * G;                             // query rows of a sequence
+  // nrg CTAs form a group: they walk the same share of the (sequence, KV head,
+  // tile) list in step, each for its own row group rg, so a page one of them
+  // copies from HBM is in L2 for the others
+  const int rg = int(blockIdx.x % nrg);
+  const long long grp = blockIdx.x / nrg, NG = gridDim.x / nrg;
 
   // ------------------------------------------------------------ the share
   // T = total work-list cost; each thread sums the run costs of some sequences
@@ -257,11 +261,11 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   long long T = 0;
 #pragma unroll
   for (int w = 0; w < 6; ++w) T += red64[w];
-  T *= Hv;
-  const long long N = ll_min(gridDim.x, ll_max(1, T / max(1, unit_tiles)));
-  if (T == 0 || blockIdx.x >= N) return;                 // uniform for the CTA
-  const long long start = (int64_t(blockIdx.x) * T) / N;
-  const long long end = (int64_t(blockIdx.x + 1) * T) / N;
+  T *= Hk;
+  const long long N = ll_min(NG, ll_max(1, T / max(1, unit_tiles)));
+  if (T == 0 || grp >= N) return;                        // uniform for the CTA
+  const long long start = (grp * T) / N;
+  const long long end = ((grp + 1) * T) / N;
   // the sequence holding cost position `start`: block-wide scan of run costs
   {
     if (threadIdx.x == 0) misci[0] = -1;
@@ -287,7 +291,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
         total += red64[w];
       }
       const long long lo_t = run + before + incl - tb;          // run cost before sequence bb
-      if (bb < B && tb > 0 && int64_t(Hv) * lo_t <= start && start < int64_t(Hv) * (lo_t + tb)) {
+      if (bb < B && tb > 0 && int64_t(Hk) * lo_t <= start && start < int64_t(Hk) * (lo_t + tb)) {
         misci[0] = bb;
         miscll[0] = lo_t;
       }
@@ -298,8 +302,8 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   }
   const int b0 = misci[0];
   const long long P0 = miscll[0];
-  // CTA that holds work-list cost position x; the slot of a piece is its CTA's
-  // rank among the CTAs that hold real tiles of the piece's (b, h)
+  // group that holds work-list cost position x; the slot of a piece is its
+  // group's rank among the groups that hold real tiles of the piece's (b, h)
   auto cta_of = [&](long long x) -> long long { return ((x + 1) * N - 1) / T; };
 
   uint8_t* kring = smem + C::OFF_K;
@@ -367,7 +371,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   const uint32_t tmem = *tmem_slot;
 
   PieceWalk walk;
-  walk.init(b0, P0, start, end, Hv, ctx_lens, B, max_ctx, W);
+  walk.init(b0, P0, start, end, Hk, ctx_lens, B, max_ctx, W);
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
@@ -385,7 +389,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     auto step = [&](PieceWalk& pw, int& tile) {
       if (pw.done) return;
       if (++tile >= pw.hi) {
-        pw.next(Hv, ctx_lens, B, max_ctx, W);
+        pw.next(Hk, ctx_lens, B, max_ctx, W);
         tile = pw.lo;
       }
     };
@@ -397,7 +401,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       if constexpr (C::MV > 0) {
         const int sblk = __shfl_sync(0xffffffffu, ids, sp & 7);
         if (sp < 8 && sblk >= 0 && sblk < NB) {
-          const int64_t off = (int64_t(sblk) * Hk + (nrg == 1 ? h : h / nrg)) * C::METAB + sc * 16;
+          const int64_t off = (int64_t(sblk) * Hk + h) * C::METAB + sc * 16;
           kv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(ks) + off));
           vv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(vs) + off));
         }
@@ -430,7 +434,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       const int blk = __shfl_sync(0xffffffffu, id, p8);
       const bool mine = ((mask >> p8) & 1u) != 0u;
       const bool smine = C::MV > 0 && sp < 8 && ((mask >> sp) & 1u) != 0u;
-      const int64_t page = int64_t(blk) * Hk + (nrg == 1 ? h : h / nrg);
+      const int64_t page = int64_t(blk) * Hk + h;
       const uint32_t bytes = uint32_t(__popc(mask)) * uint32_t(C::PAGE);
       bool ok = true;
       // per stage: byte count, the page copies, then the scale stores and the
@@ -530,7 +534,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           if (i > walk.lo) ok = issue_pv(gt - 1);
         }
         if (ok) mma_commit(qfree);                         // this piece's S products are issued
-        walk.next(Hv, ctx_lens, B, max_ctx, W);
+        walk.next(Hk, ctx_lens, B, max_ctx, W);
       }
       if (ok && gt >= 1) issue_pv(gt - 1);
       // every MMA issued so far completes before TMEM is released
@@ -556,14 +560,14 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
     auto publish = [&](int idx, const PieceWalk& pw) {
       wk[idx] = pw;
       if (!pw.done) {
-        pinfo[idx * 2] = int(int64_t(blockIdx.x) - cta_of(pw.first_tile(Hv)));
+        pinfo[idx * 2] = int(grp - cta_of(pw.first_tile(Hk)));
         pinfo[idx * 2 + 1] = pw.hi == pw.nt;
       }
     };
     if (r == 0) {
       publish(0, walk);
       PieceWalk n = walk;
-      n.next(Hv, ctx_lens, B, max_ctx, W);
+      n.next(Hk, ctx_lens, B, max_ctx, W);
       publish(1, n);
     }
     named_bar_sync(1, 128);
@@ -582,13 +586,13 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
 #pragma unroll
         for (int i = 0; i < D / 32; ++i)
           qv[hh][i] = (g < G && !none)
-                          ? __bfloat162float(q[(int64_t(qb) * Hq + qh * G + g) * D + lane + 32 * i])
+                          ? __bfloat162float(q[(int64_t(qb) * Hq + (qh * nrg + rg) * G + g) * D + lane + 32 * i])
                           : 0.f;
       }
       if constexpr (C::SI) {
 #pragma unroll
         for (int i = 0; i < D / 32; ++i)
-          ksd[i] = none ? 0.f : __bfloat162float(ks[per_tensor ? 0 : (qh / nrg) * D + lane + 32 * i]);
+          ksd[i] = none ? 0.f : __bfloat162float(ks[per_tensor ? 0 : qh * D + lane + 32 * i]);
       }
     };
     // B operand of S (K-major, no swizzle): row n = part * G + g, element
@@ -679,7 +683,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       named_bar_sync(1, 128);                            // all read the cursor; qsc/qsum visible
       if (r == 0) {                                      // piece pc + 2 into this piece's entry
         PieceWalk n = *nxt;
-        if (!n.done) n.next(Hv, ctx_lens, B, max_ctx, W);
+        if (!n.done) n.next(Hk, ctx_lens, B, max_ctx, W);
         publish(pc & 1, n);
       }
       float qs[G], qz[G];
@@ -780,12 +784,12 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           x[g] = valid ? sc * sk * qs[g] : -INFINITY;
         }
         if (n_query > 1) {
-          // multi-query: row rr = (virtual head % nrg) * G + g of the KV head's
-          // rows is query position j = rr % n_query of query head rr / n_query,
+          // multi-query: row rr = rg * G + g of the KV head's rows is query
+          // position j = rr % n_query of query head rr / n_query,
           // and position j sees the tokens before the last n_query - 1 - j of
           // the context
           const int after = pctx - 1 - (tile0 + r);       // tokens after this one
-          const int rr0 = (ph_ % nrg) * G;
+          const int rr0 = rg * G;
 #pragma unroll
           for (int g = 0; g < G; ++g)
             if (n_query - 1 - (rr0 + g) % n_query > after) x[g] = -INFINITY;
@@ -995,7 +999,7 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       // static INT8: the V scale of channel r multiplies the finished sums
       float vsd = 1.f;
       if constexpr (C::SI) {
-        if (r < D) vsd = __bfloat162float(vs[per_tensor ? 0 : (ph_ / nrg) * D + r]);
+        if (r < D) vsd = __bfloat162float(vs[per_tensor ? 0 : ph_ * D + r]);
       }
       // After a wait ran out the piece's sums are incomplete: it writes a
       // marker instead (max +inf, sum and output NaN), so that every output row
@@ -1006,14 +1010,14 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
       for (int g = 0; g < G; ++g) {
         const float L = red2[g] + red2[8 + g] + red2[16 + g] + red2[24 + g];
         const float Cz = red2[32 + g] + red2[40 + g] + red2[48 + g] + red2[56 + g];
-        const int64_t row = (int64_t(pb) * Hq + ph_ * G + g) * slots + slot;
+        const int64_t row = (int64_t(pb) * Hq + (ph_ * nrg + rg) * G + g) * slots + slot;
         if (r < D) part_o[row * D + r] = good ? (o[g] - Cz) * vsd : __int_as_float(0x7fc00000);
         if (r == 0) {
           part_ml[row * 2] = good ? m[g] : INFINITY;
           part_ml[row * 2 + 1] = good ? L : __int_as_float(0x7fc00000);
         }
       }
-      if (r == 0 && last) part_cnt[pb * Hv + ph_] = slot + 1;
+      if (r == 0 && last) part_cnt[(int64_t(pb) * Hk + ph_) * nrg + rg] = slot + 1;
     }
   }
   tc_fence_before();

@@ -309,44 +309,11 @@ __device__ __forceinline__ void store_bytes16(uint8_t* dst, const uint32_t (&w)[
   }
 }
 
-// cp.async copies of 16 and 8 bytes into shared memory (cached in L2 only),
-// committed as one group per window; wait_group<1> leaves the newest group in
-// flight.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(tc::smem_u32(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Heads per append window.
-constexpr int kAppendHeads = 2;
-
-// Dynamic shared memory of the append kernel (offsets in bytes, 16-aligned).
-template <int D, int FMT>
-struct AppendSmem {
-  static constexpr int ELT = FMT == KVQ_BF16 ? 2 : 1;
-  static constexpr int PADB = D * ELT + 16;
-  static constexpr int OFF_IN = 0;                                         // [2][2][16][HG*D] bf16
-  static constexpr int OFF_SL = OFF_IN + 2 * 2 * kBlockSize * kAppendHeads * D * 2;   // [2][16] int64
-  static constexpr int OFF_KB = OFF_SL + 2 * kBlockSize * 8;               // [HG][16 * PADB]
-  static constexpr int OFF_VB = OFF_KB + kAppendHeads * kBlockSize * PADB;
-  static constexpr int BYTES = OFF_VB + kAppendHeads * kBlockSize * PADB;
-};
-
-// Persistent append. A window is 16 consecutive input tokens x kAppendHeads KV
-// heads (one page per head when the tokens fill it); CTA c takes windows c,
-// c + gridDim.x, ... and copies the next window's K/V rows and slots into the
-// other of two shared-memory stages (cp.async) while it quantizes the current
-// one, so the loads of one window overlap the arithmetic and stores of the
-// last. Per window, each of the 8 warps quantizes four (token, head) pairs:
-// lanes 0-15 the K row, lanes 16-31 the V row. The codes are staged in shared
-// memory and written in page-sized pieces:
+// One CTA of 8 warps per (16 consecutive input tokens, KV head). Warp w takes
+// tokens 2w and 2w+1; for each, its lanes 0-15 quantize the token's K row and
+// lanes 16-31 its V row into shared memory. The input rows are requested before
+// the slots arrive (a skipped token's row is read and dropped), so the loads
+// overlap. The window is then written in page-sized pieces:
 //   - the 16 tokens fill one page in order (the bulk / prefill case): the page
 //     is written as whole 16-byte chunks, K in its chunk-major layout and V
 //     transposed with byte permutes;
@@ -356,292 +323,231 @@ struct AppendSmem {
 //     stores that range allows. A page continued from an offset (chunked
 //     prefill) thus costs one partial chunk per channel, not one byte store per
 //     token and channel.
+// Register use is capped at 32 so that 8 CTAs (64 warps) fit on an SM (51 and
+// 5 CTAs for the static-scale format, whose lanes keep their channels' scales
+// and reciprocals).
 template <int D, int FMT>
-__global__ void __launch_bounds__(256, FMT == KVQ_INT8_CHANNEL ? 4 : 5)
+__global__ void __launch_bounds__(256, FMT == KVQ_INT8_CHANNEL ? 5 : 8)
 append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
               const int64_t* __restrict__ slots, int T, int Hk, int NB, uint8_t* __restrict__ kc,
               uint8_t* __restrict__ vc, __nv_bfloat16* __restrict__ ks, __nv_bfloat16* __restrict__ vs,
               int per_tensor) {
   using RC = RowCodes<D, FMT>;
-  constexpr int HG = kAppendHeads;
   constexpr int E = RC::E, ELT = RC::ELT;
-  constexpr int ROWB = D * ELT;                 // bytes of one token row (output)
+  constexpr int ROWB = D * ELT;                 // bytes of one token row
   constexpr int PADB = ROWB + 16;               // padded smem row (bank spread)
   constexpr int PAGEB = kBlockSize * ROWB;
   constexpr int NC = ROWB / 16;                 // 16-byte chunks of a K row
   constexpr int UC = ELT;                       // 16-byte V chunks per channel
   constexpr int TPC = 16 / ELT;                 // tokens per V chunk
   constexpr int MV = (FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2) ? 1 : (FMT == KVQ_INT8_ASYM ? 2 : 0);
-  constexpr int INROW = HG * D;                 // bf16 elements of one token's rows of the window
-  using L = AppendSmem<D, FMT>;
-  // dynamic shared memory: input stages [2][K, V][16 tokens][HG heads][D]
-  // bf16, slots [2][16], staged codes [HG][16][PADB] for K and for V
-  extern __shared__ __align__(16) uint8_t app_smem[];
-  auto in = reinterpret_cast<__nv_bfloat16 (*)[2][kBlockSize][INROW]>(app_smem + L::OFF_IN);
-  auto sl2 = reinterpret_cast<int64_t (*)[kBlockSize]>(app_smem + L::OFF_SL);
-  auto kbuf = reinterpret_cast<uint8_t (*)[kBlockSize * PADB]>(app_smem + L::OFF_KB);
-  auto vbuf = reinterpret_cast<uint8_t (*)[kBlockSize * PADB]>(app_smem + L::OFF_VB);
-  __shared__ __nv_bfloat16 kmb[HG][kBlockSize][2], vmb[HG][kBlockSize][2];
+  __shared__ __align__(16) uint8_t kbuf[kBlockSize * PADB];
+  __shared__ __align__(16) uint8_t vbuf[kBlockSize * PADB];
+  __shared__ __nv_bfloat16 kmb[kBlockSize][2], vmb[kBlockSize][2];
+  __shared__ int64_t sl[kBlockSize];
   __shared__ int seg_i0[kBlockSize], seg_len[kBlockSize], nseg, page_fast;
 
-  const int n_hg = (Hk + HG - 1) / HG;
-  const int64_t n_win = ((int64_t(T) + kBlockSize - 1) / kBlockSize) * n_hg;
+  const int h = blockIdx.y;
+  const int64_t tb = int64_t(blockIdx.x) * kBlockSize;
+  const int n = int(min(int64_t(kBlockSize), int64_t(T) - tb));
   const int64_t nslots = int64_t(NB) * kBlockSize;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int which = lane >> 4;                  // 0: K row, 1: V row
   const int d0 = (lane & 15) * E;
+  // this half warp's rows: tokens 2 warp and 2 warp + 1, requested up front
+  const __nv_bfloat16* src = (which ? v : k) + ((tb + 2 * warp) * Hk + h) * D + d0;
+  uint32_t raws[2][D / 32];
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) raws[p][e] = 0u;
+    if (2 * warp + p < n) load_row<D>(src + int64_t(p) * Hk * D, raws[p]);
+  }
+  if (threadIdx.x < kBlockSize) sl[threadIdx.x] = threadIdx.x < n ? slots[tb + threadIdx.x] : -1;
+  __syncthreads();
 
-  // copies of window w into stage st: the rows of its tokens (one contiguous
-  // run of HG heads per token and tensor) and its slots
-  auto issue = [&](int64_t w, int st) {
-    const int64_t tb = (w / n_hg) * kBlockSize;
-    const int h0 = int(w % n_hg) * HG;
-    const int hn = min(HG, Hk - h0);
-    const int n = int(min(int64_t(kBlockSize), int64_t(T) - tb));
-    constexpr int CH = INROW * 2 / 16;          // 16-byte chunks of one token's rows
-    for (int j = threadIdx.x; j < 2 * kBlockSize * CH; j += blockDim.x) {
-      const int tens = j / (kBlockSize * CH), rem = j % (kBlockSize * CH);
-      const int t = rem / CH, c = rem % CH;
-      if (t < n && c < hn * D * 2 / 16) {
-        const __nv_bfloat16* src = (tens ? v : k) + ((tb + t) * Hk + h0) * D;
-        cp_async16(reinterpret_cast<uint8_t*>(&in[st][tens][t][0]) + c * 16,
-                   reinterpret_cast<const uint8_t*>(src) + c * 16);
-      }
+  if (warp == 0) {
+    const int64_t si = lane < kBlockSize ? sl[lane] : -1;
+    const int64_t sp = (lane > 0 && lane < kBlockSize) ? sl[lane - 1] : -1;
+    const int64_t s0 = sl[0];
+    // whole page in order: slot i = s0 + i for all 16 tokens, s0 page-aligned
+    const bool inpage = lane >= kBlockSize || (si == s0 + lane && s0 >= 0 && s0 % kBlockSize == 0 &&
+                                               s0 < nslots && n == kBlockSize);
+    const bool fast = __all_sync(0xffffffffu, inpage);
+    // segments: a token starts one unless it continues the previous token's
+    // slot inside the same page
+    const bool valid = si >= 0 && si < nslots;
+    const bool start = valid && !(sp >= 0 && sp < nslots && si == sp + 1 && si % kBlockSize != 0);
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    const unsigned smask = __ballot_sync(0xffffffffu, start);
+    if (start) {
+      const int idx = __popc(smask & ((1u << lane) - 1u));
+      // the run ends at the next start or at the first invalid token
+      const unsigned stop = (smask | ~vmask) & ~((2u << lane) - 1u);
+      seg_i0[idx] = lane;
+      seg_len[idx] = (stop ? __ffs(stop) - 1 : 32) - lane;
     }
-    if (threadIdx.x < kBlockSize) {
-      if (threadIdx.x < n) cp_async8(&sl2[st][threadIdx.x], slots + tb + threadIdx.x);
-      else sl2[st][threadIdx.x] = -1;
+    if (lane == 0) {
+      nseg = __popc(smask);
+      page_fast = fast;
     }
-  };
+  }
 
-  // static scales: a half warp's rows are all K (lanes 0-15) or all V; the
-  // lane's channels' scales and reciprocals, per head of the window
+  // static scales: a half warp's rows are all K (lanes 0-15) or all V, so a
+  // lane's channels keep their scales for every row it quantizes
   [[maybe_unused]] float ssc[E], rsc[E];
-  [[maybe_unused]] int ssc_head = -1;
-
-  int64_t w = blockIdx.x;
-  if (w < n_win) issue(w, 0);
-  cp_async_commit();
-  for (int it = 0; w < n_win; ++it, w += gridDim.x) {
-    const int st = it & 1;
-    const int64_t tb = (w / n_hg) * kBlockSize;
-    const int h0 = int(w % n_hg) * HG;
-    const int hn = min(HG, Hk - h0);
-    const int n = int(min(int64_t(kBlockSize), int64_t(T) - tb));
-    // the next window's copies go into the other stage (free: the last
-    // iteration ended with a barrier)
-    if (w + gridDim.x < n_win) issue(w + gridDim.x, st ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const int64_t* sl = sl2[st];
-
-    if (warp == 0) {
-      const int64_t si = lane < kBlockSize ? sl[lane] : -1;
-      const int64_t sp = (lane > 0 && lane < kBlockSize) ? sl[lane - 1] : -1;
-      const int64_t s0 = sl[0];
-      // whole page in order: slot i = s0 + i for all 16 tokens, s0 page-aligned
-      const bool inpage = lane >= kBlockSize || (si == s0 + lane && s0 >= 0 && s0 % kBlockSize == 0 &&
-                                                 s0 < nslots && n == kBlockSize);
-      const bool fast = __all_sync(0xffffffffu, inpage);
-      // segments: a token starts one unless it continues the previous token's
-      // slot inside the same page
-      const bool valid = si >= 0 && si < nslots;
-      const bool start = valid && !(sp >= 0 && sp < nslots && si == sp + 1 && si % kBlockSize != 0);
-      const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-      const unsigned smask = __ballot_sync(0xffffffffu, start);
-      if (start) {
-        const int idx = __popc(smask & ((1u << lane) - 1u));
-        // the run ends at the next start or at the first invalid token
-        const unsigned stop = (smask | ~vmask) & ~((2u << lane) - 1u);
-        seg_i0[idx] = lane;
-        seg_len[idx] = (stop ? __ffs(stop) - 1 : 32) - lane;
-      }
-      if (lane == 0) {
-        nseg = __popc(smask);
-        page_fast = fast;
-      }
+  if constexpr (FMT == KVQ_INT8_CHANNEL) {
+    const __nv_bfloat16* sarr = which ? vs : ks;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      ssc[e] = __bfloat162float(sarr[per_tensor ? 0 : h * D + d0 + e]);
+      rsc[e] = ssc[e] >= 7.88860905e-31f ? __frcp_rn(ssc[e]) : 0.f;   // 2^-100
     }
+  }
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const int i = 2 * warp + p;                     // token in the window
+    // every lane quantizes (the reductions span the warp); only real rows store
+    RC rc;
+    if constexpr (FMT == KVQ_INT8_CHANNEL) quantize_row_static<D>(raws[p], ssc, rsc, rc);
+    else quantize_row<D, FMT>(raws[p], rc);
+    const int64_t slot = i < n ? sl[i] : -1;
+    if (slot < 0) continue;
+    if (slot >= nslots) {
+      if ((lane & 15) == 0) flag_error(KVQ_DEVERR_SLOT);
+      continue;
+    }
+    uint8_t* dst = (which ? vbuf : kbuf) + i * PADB + d0 * ELT;
+    if constexpr (E * ELT == 16) *reinterpret_cast<uint4*>(dst) = make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]);
+    else if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
+    else *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
+    if ((lane & 15) == 0) {
+      (which ? vmb : kmb)[i][0] = rc.s;
+      (which ? vmb : kmb)[i][1] = __int2bfloat16_rn(rc.zp);
+    }
+  }
+  __syncthreads();
 
-    // ---- quantize: pair p of this warp is (token p % 16, head p / 16) of the
-    // window's 16 x HG pairs (whole warps share one head)
-#pragma unroll
-    for (int pp = 0; pp < kBlockSize * HG / 8; ++pp) {
-      const int p = warp * (kBlockSize * HG / 8) + pp;
-      const int i = p % kBlockSize, hh = p / kBlockSize;
-      uint32_t raw[D / 32];
-      {
-        const uint8_t* srow = reinterpret_cast<const uint8_t*>(&in[st][which][i][hh * D + d0]);
-        if constexpr (D == 128) {
-          const uint4 u = *reinterpret_cast<const uint4*>(srow);
-          raw[0] = u.x; raw[1] = u.y; raw[2] = u.z; raw[3] = u.w;
-        } else {
-          const uint2 u = *reinterpret_cast<const uint2*>(srow);
-          raw[0] = u.x; raw[1] = u.y;
-        }
-      }
-      RC rc;
-      if constexpr (FMT == KVQ_INT8_CHANNEL) {
-        if (ssc_head != h0 + hh) {                   // the window's head (warp-uniform)
-          ssc_head = h0 + hh;
-          const __nv_bfloat16* sarr = which ? vs : ks;
-          const int hs = min(h0 + hh, Hk - 1);
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            ssc[e] = __bfloat162float(sarr[per_tensor ? 0 : hs * D + d0 + e]);
-            rsc[e] = ssc[e] >= 7.88860905e-31f ? __frcp_rn(ssc[e]) : 0.f;   // 2^-100
-          }
-        }
-        quantize_row_static<D>(raw, ssc, rsc, rc);
-      } else {
-        quantize_row<D, FMT>(raw, rc);
-      }
-      const int64_t slot = (i < n && hh < hn) ? sl[i] : -1;
-      if (slot < 0) continue;
-      if (slot >= nslots) {
-        if ((lane & 15) == 0 && hh == 0) flag_error(KVQ_DEVERR_SLOT);
+  if (page_fast) {                                   // uniform over the CTA
+    const int64_t page = (sl[0] / kBlockSize) * Hk + h;
+    uint8_t* kp = kc + page * PAGEB;
+    uint8_t* vp = vc + page * PAGEB;
+    // items [0, KN): K chunk j = (token group t/8, c, t%8) <- bytes [16c, 16c+16)
+    // of token t's row. Items [KN, KN + VN): a V piece, from 32-bit words of
+    // the staged rows transposed with byte permutes.
+    constexpr int KN = PAGEB / 16;
+    constexpr int VN = ELT == 1 ? 2 * (D / 4) : 2 * (D / 2);
+    for (int j = threadIdx.x; j < KN + VN; j += blockDim.x) {
+      if (j < KN) {
+        const int c = (j >> 3) % NC, t = (j / (8 * NC)) * 8 + (j & 7);
+        *reinterpret_cast<uint4*>(kp + j * 16) = *reinterpret_cast<const uint4*>(kbuf + t * PADB + c * 16);
         continue;
       }
-      uint8_t* dst = (which ? vbuf[hh] : kbuf[hh]) + i * PADB + d0 * ELT;
-      if constexpr (E * ELT == 16) *reinterpret_cast<uint4*>(dst) = make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]);
-      else if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
-      else *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
-      if ((lane & 15) == 0) {
-        (which ? vmb : kmb)[hh][i][0] = rc.s;
-        (which ? vmb : kmb)[hh][i][1] = __int2bfloat16_rn(rc.zp);
+      const int jv = j - KN;
+      if constexpr (ELT == 1) {
+        // channels 4c..4c+3, tokens 8h..8h+7: two 4x4 byte transposes; the
+        // result is the low or high 8 bytes of four channels' chunks
+        const int c = jv % (D / 4), hh = jv / (D / 4);
+        uint32_t o[4][2];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int t0 = 8 * hh + 4 * g;
+          const uint32_t r0 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 0) * PADB + 4 * c);
+          const uint32_t r1 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 1) * PADB + 4 * c);
+          const uint32_t r2 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 2) * PADB + 4 * c);
+          const uint32_t r3 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 3) * PADB + 4 * c);
+          const uint32_t a01 = __byte_perm(r0, r1, 0x5140), a23 = __byte_perm(r2, r3, 0x5140);
+          const uint32_t b01 = __byte_perm(r0, r1, 0x7362), b23 = __byte_perm(r2, r3, 0x7362);
+          o[0][g] = __byte_perm(a01, a23, 0x5410);
+          o[1][g] = __byte_perm(a01, a23, 0x7632);
+          o[2][g] = __byte_perm(b01, b23, 0x5410);
+          o[3][g] = __byte_perm(b01, b23, 0x7632);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint2*>(vp + (4 * c + m) * 16 + 8 * hh) = make_uint2(o[m][0], o[m][1]);
+      } else {
+        // channels 2c, 2c+1, tokens 8u..8u+7: 2x2 transposes of 16-bit halves
+        const int c = jv % (D / 2), u = jv / (D / 2);
+        uint32_t lo4[4], hi4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t0 = 8 * u + 2 * q;
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vbuf + t0 * PADB + 4 * c);
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vbuf + (t0 + 1) * PADB + 4 * c);
+          lo4[q] = __byte_perm(w0, w1, 0x5410);
+          hi4[q] = __byte_perm(w0, w1, 0x7632);
+        }
+        *reinterpret_cast<uint4*>(vp + (u * D + 2 * c) * 16) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+        *reinterpret_cast<uint4*>(vp + (u * D + 2 * c + 1) * 16) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
       }
     }
-    __syncthreads();
-
-    if (page_fast) {                                   // uniform over the CTA
-      // items [0, KN): K chunk j = (token group t/8, c, t%8) <- bytes [16c, 16c+16)
-      // of token t's row. Items [KN, KN + VN): a V piece, from 32-bit words of
-      // the staged rows transposed with byte permutes. Per head of the window.
-      constexpr int KN = PAGEB / 16;
-      constexpr int VN = ELT == 1 ? 2 * (D / 4) : 2 * (D / 2);
-      for (int jj = threadIdx.x; jj < hn * (KN + VN); jj += blockDim.x) {
-        const int hh = jj / (KN + VN), j = jj % (KN + VN);
-        const int64_t page = (sl[0] / kBlockSize) * Hk + h0 + hh;
-        uint8_t* kp = kc + page * PAGEB;
-        uint8_t* vp = vc + page * PAGEB;
-        if (j < KN) {
-          const int c = (j >> 3) % NC, t = (j / (8 * NC)) * 8 + (j & 7);
-          *reinterpret_cast<uint4*>(kp + j * 16) = *reinterpret_cast<const uint4*>(kbuf[hh] + t * PADB + c * 16);
-          continue;
-        }
-        const int jv = j - KN;
-        const uint8_t* vb = vbuf[hh];
-        if constexpr (ELT == 1) {
-          // channels 4c..4c+3, tokens 8h..8h+7: two 4x4 byte transposes; the
-          // result is the low or high 8 bytes of four channels' chunks
-          const int c = jv % (D / 4), hx = jv / (D / 4);
-          uint32_t o[4][2];
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const int t0 = 8 * hx + 4 * g;
-            const uint32_t r0 = *reinterpret_cast<const uint32_t*>(vb + (t0 + 0) * PADB + 4 * c);
-            const uint32_t r1 = *reinterpret_cast<const uint32_t*>(vb + (t0 + 1) * PADB + 4 * c);
-            const uint32_t r2 = *reinterpret_cast<const uint32_t*>(vb + (t0 + 2) * PADB + 4 * c);
-            const uint32_t r3 = *reinterpret_cast<const uint32_t*>(vb + (t0 + 3) * PADB + 4 * c);
-            const uint32_t a01 = __byte_perm(r0, r1, 0x5140), a23 = __byte_perm(r2, r3, 0x5140);
-            const uint32_t b01 = __byte_perm(r0, r1, 0x7362), b23 = __byte_perm(r2, r3, 0x7362);
-            o[0][g] = __byte_perm(a01, a23, 0x5410);
-            o[1][g] = __byte_perm(a01, a23, 0x7632);
-            o[2][g] = __byte_perm(b01, b23, 0x5410);
-            o[3][g] = __byte_perm(b01, b23, 0x7632);
-          }
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            *reinterpret_cast<uint2*>(vp + (4 * c + m) * 16 + 8 * hx) = make_uint2(o[m][0], o[m][1]);
-        } else {
-          // channels 2c, 2c+1, tokens 8u..8u+7: 2x2 transposes of 16-bit halves
-          const int c = jv % (D / 2), u = jv / (D / 2);
-          uint32_t lo4[4], hi4[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int t0 = 8 * u + 2 * q;
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vb + t0 * PADB + 4 * c);
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vb + (t0 + 1) * PADB + 4 * c);
-            lo4[q] = __byte_perm(w0, w1, 0x5410);
-            hi4[q] = __byte_perm(w0, w1, 0x7632);
-          }
-          *reinterpret_cast<uint4*>(vp + (u * D + 2 * c) * 16) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
-          *reinterpret_cast<uint4*>(vp + (u * D + 2 * c + 1) * 16) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
-        }
+  } else {
+    // K: whole 16-byte chunks of each token's row
+    for (int j = threadIdx.x; j < n * NC; j += blockDim.x) {
+      const int i = j / NC, c = j % NC;
+      const int64_t slot = sl[i];
+      if (slot < 0 || slot >= nslots) continue;
+      const int64_t page = (slot / kBlockSize) * Hk + h;
+      *reinterpret_cast<uint4*>(kc + page * PAGEB + k_chunk_offset<ROWB>(c, int(slot % kBlockSize))) =
+          *reinterpret_cast<const uint4*>(kbuf + i * PADB + c * 16);
+    }
+    // V: per (segment, channel d, chunk u) the segment's bytes of that chunk
+    const int ns = nseg;
+    for (int j = threadIdx.x; j < ns * D * UC; j += blockDim.x) {
+      const int sg = j / (D * UC), d = (j / UC) % D, u = j % UC;
+      const int i0 = seg_i0[sg], len = seg_len[sg];
+      const int64_t slot0 = sl[i0];
+      const int o0 = int(slot0 % kBlockSize);
+      // token offsets of the segment inside chunk u
+      const int ta = max(o0, u * TPC), tz = min(o0 + len, (u + 1) * TPC);
+      if (ta >= tz) continue;
+      uint8_t* chunk = vc + ((slot0 / kBlockSize) * Hk + h) * PAGEB + (u * D + d) * 16;
+      if (tz - ta == 1) {                            // one token: one element
+        const int i = i0 + (ta - o0), b = (ta - u * TPC) * ELT;
+        if constexpr (ELT == 1) chunk[b] = vbuf[i * PADB + d];
+        else *reinterpret_cast<uint16_t*>(chunk + b) = *reinterpret_cast<const uint16_t*>(vbuf + i * PADB + 2 * d);
+        continue;
       }
-    } else {
-      // K: whole 16-byte chunks of each token's row
-      for (int jj = threadIdx.x; jj < hn * n * NC; jj += blockDim.x) {
-        const int hh = jj / (n * NC), j = jj % (n * NC);
-        const int i = j / NC, c = j % NC;
-        const int64_t slot = sl[i];
-        if (slot < 0 || slot >= nslots) continue;
-        const int64_t page = (slot / kBlockSize) * Hk + h0 + hh;
-        *reinterpret_cast<uint4*>(kc + page * PAGEB + k_chunk_offset<ROWB>(c, int(slot % kBlockSize))) =
-            *reinterpret_cast<const uint4*>(kbuf[hh] + i * PADB + c * 16);
-      }
-      // V: per (segment, channel d, chunk u) the segment's bytes of that chunk
-      const int ns = nseg;
-      for (int jj = threadIdx.x; jj < hn * ns * D * UC; jj += blockDim.x) {
-        const int hh = jj / (ns * D * UC), j = jj % (ns * D * UC);
-        const int sg = j / (D * UC), d = (j / UC) % D, u = j % UC;
-        const int i0 = seg_i0[sg], len = seg_len[sg];
-        const int64_t slot0 = sl[i0];
-        const int o0 = int(slot0 % kBlockSize);
-        const uint8_t* vb = vbuf[hh];
-        // token offsets of the segment inside chunk u
-        const int ta = max(o0, u * TPC), tz = min(o0 + len, (u + 1) * TPC);
-        if (ta >= tz) continue;
-        uint8_t* chunk = vc + ((slot0 / kBlockSize) * Hk + h0 + hh) * PAGEB + (u * D + d) * 16;
-        if (tz - ta == 1) {                            // one token: one element
-          const int i = i0 + (ta - o0), b = (ta - u * TPC) * ELT;
-          if constexpr (ELT == 1) chunk[b] = vb[i * PADB + d];
-          else *reinterpret_cast<uint16_t*>(chunk + b) = *reinterpret_cast<const uint16_t*>(vb + i * PADB + 2 * d);
-          continue;
-        }
-        uint32_t wv[4];
+      uint32_t wv[4];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t word = 0;
-          const int w0 = u * TPC + q4 * (4 / ELT);      // first token offset of this word
-          if (w0 + 4 / ELT > ta && w0 < tz) {
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t word = 0;
+        const int w0 = u * TPC + q4 * (4 / ELT);      // first token offset of this word
+        if (w0 + 4 / ELT > ta && w0 < tz) {
 #pragma unroll
-            for (int bb = 0; bb < 4 / ELT; ++bb) {
-              const int t = w0 + bb;
-              if (t >= ta && t < tz) {
-                const int i = i0 + (t - o0);
-                if constexpr (ELT == 1)
-                  word |= uint32_t(vb[i * PADB + d]) << (8 * bb);
-                else
-                  word |= uint32_t(*reinterpret_cast<const uint16_t*>(vb + i * PADB + 2 * d)) << (16 * bb);
-              }
+          for (int bb = 0; bb < 4 / ELT; ++bb) {
+            const int t = w0 + bb;
+            if (t >= ta && t < tz) {
+              const int i = i0 + (t - o0);
+              if constexpr (ELT == 1)
+                word |= uint32_t(vbuf[i * PADB + d]) << (8 * bb);
+              else
+                word |= uint32_t(*reinterpret_cast<const uint16_t*>(vbuf + i * PADB + 2 * d)) << (16 * bb);
             }
           }
-          wv[q4] = word;
         }
-        store_bytes16(chunk, wv, (ta - u * TPC) * ELT, (tz - u * TPC) * ELT);
+        wv[q4] = word;
       }
+      store_bytes16(chunk, wv, (ta - u * TPC) * ELT, (tz - u * TPC) * ELT);
     }
-    // metadata: one thread per (head, token, K or V)
-    if (MV > 0 && threadIdx.x < HG * 2 * kBlockSize) {
-      const int hh = threadIdx.x / (2 * kBlockSize);
-      const int t = threadIdx.x & 15;
-      const int64_t slot = sl[t];
-      if (hh < hn && t < n && slot >= 0 && slot < nslots) {
-        const bool isv = (threadIdx.x & 16) != 0;
-        __nv_bfloat16* meta = isv ? vs : ks;
-        const __nv_bfloat16 (*mb)[2] = isv ? vmb[hh] : kmb[hh];
-        const int64_t row = ((slot / kBlockSize) * Hk + h0 + hh) * kBlockSize + slot % kBlockSize;
-        if (MV == 1) {
-          meta[row] = mb[t][0];
-        } else {
-          *reinterpret_cast<__nv_bfloat162*>(meta + row * 2) = __halves2bfloat162(mb[t][0], mb[t][1]);
-        }
-      }
-    }
-    __syncthreads();                                  // staging and this stage are reused
   }
-  cp_async_wait<0>();
+  // metadata: one thread per (token, K or V)
+  if (MV > 0 && threadIdx.x < 2 * kBlockSize) {
+    const int t = threadIdx.x & 15;
+    const int64_t slot = sl[t];
+    if (t < n && slot >= 0 && slot < nslots) {
+      const bool isv = threadIdx.x >= kBlockSize;
+      __nv_bfloat16* meta = isv ? vs : ks;
+      const __nv_bfloat16 (*mb)[2] = isv ? vmb : kmb;
+      const int64_t row = ((slot / kBlockSize) * Hk + h) * kBlockSize + slot % kBlockSize;
+      if (MV == 1) {
+        meta[row] = mb[t][0];
+      } else {
+        *reinterpret_cast<__nv_bfloat162*>(meta + row * 2) = __halves2bfloat162(mb[t][0], mb[t][1]);
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------------ launchers
@@ -652,17 +558,8 @@ template <int D, int FMT>
 cudaError_t append_dispatch(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
                             void* vc, void* ks, void* vs, const kvq_dims& d, int per_tensor,
                             cudaStream_t st) {
-  // persistent: at most the resident CTAs, each taking windows in turn
-  const int64_t windows = ((int64_t(T) + kBlockSize - 1) / kBlockSize) *
-                          ((d.n_kv_heads + kAppendHeads - 1) / kAppendHeads);
-  constexpr int smem = AppendSmem<D, FMT>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(append_kernel<D, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_kernel<D, FMT>, 256, smem);
-  if (e != cudaSuccess) return e;
-  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(windows, int64_t(device_sm_count()) * std::max(1, per_sm)));
-  append_kernel<D, FMT><<<dim3(unsigned(grid)), 256, smem, st>>>(
+  const dim3 grid(unsigned((int64_t(T) + kBlockSize - 1) / kBlockSize), unsigned(d.n_kv_heads));
+  append_kernel<D, FMT><<<grid, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), slots, T,
       d.n_kv_heads, d.num_blocks, static_cast<uint8_t*>(kc), static_cast<uint8_t*>(vc),
       static_cast<__nv_bfloat16*>(ks), static_cast<__nv_bfloat16*>(vs), per_tensor);
@@ -693,12 +590,14 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
   float* po = static_cast<float*>(ws);
   float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
   int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
-  // one CTA per resident slot; each takes an equal share of the tile list
-  const int64_t grid = int64_t(device_sm_count()) * per_sm;
+  // one CTA per resident slot, in groups of nrg (one CTA per row group) that
+  // walk the same share of the tile list; at least one group
+  const int64_t slots_resident = int64_t(device_sm_count()) * per_sm;
+  const int64_t grid = std::max<int64_t>(1, slots_resident / nrg) * nrg;
   kern<<<dim3(unsigned(grid)), 192, C::SMEM, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
-      static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads * nrg, nrg, d.num_blocks,
+      static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, nrg, d.num_blocks,
       d.max_blocks_per_seq, max_ctx, plan.partition / kTileTokens, plan.slots, sm_scale * kLog2e,
       per_tensor, n_query, decode_wait_limit(), po, pml, pcnt);
   return cudaGetLastError();
