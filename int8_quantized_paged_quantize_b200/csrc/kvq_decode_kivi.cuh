@@ -474,38 +474,61 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
 
     // the BF16 query rows of a piece's group, loaded one piece ahead
     float qv[C::HPW][D / 32];
+    // lane owns the D/32 consecutive channels d0 .. d0 + D/32 - 1
+    constexpr int CPL = D / 32;
+    const int d0 = lane * CPL;
     auto load_q = [&](bool none, int qb, int qh) {
 #pragma unroll
       for (int hh = 0; hh < C::HPW; ++hh) {
         const int g = cw + 4 * hh;
+        uint32_t w[CPL / 2];
 #pragma unroll
-        for (int i = 0; i < D / 32; ++i)
-          qv[hh][i] = (g < G && !none)
-                          ? __bfloat162float(q[(int64_t(qb) * Hq + qh * G + g) * D + lane + 32 * i])
-                          : 0.f;
+        for (int i = 0; i < CPL / 2; ++i) w[i] = 0u;
+        if (g < G && !none) {
+          const __nv_bfloat16* src = q + (int64_t(qb) * Hq + qh * G + g) * D + d0;
+          if constexpr (CPL == 4) {
+            const uint2 u = *reinterpret_cast<const uint2*>(src);
+            w[0] = u.x; w[1] = u.y;
+          } else {
+            w[0] = *reinterpret_cast<const uint32_t*>(src);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < CPL / 2; ++i) {
+          qv[hh][2 * i] = __uint_as_float(w[i] << 16);
+          qv[hh][2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
       }
     };
     // query operand of tile gt: x = q s_d (the tile's channel scales) in three
-    // exact s8 parts after a power-of-two scaling of the head, and sum_d q z_d
+    // exact s8 parts after a power-of-two scaling of the head, and sum_d q z_d;
+    // the lane's consecutive channels make one word (or half word) per part
     auto store_q = [&](int gt_q, const float (&qcur)[C::HPW][D / 32]) {
       const int su = gt_q % C::NST;
-      const __nv_bfloat162* kmp = reinterpret_cast<const __nv_bfloat162*>(kmeta + su * 8 * C::META);
-      float sd[D / 32], zd[D / 32];
+      // channel d: page d / (D/8), entry d % (D/8); the lane's channels are
+      // consecutive entries of one page
+      const __nv_bfloat162* kmp = reinterpret_cast<const __nv_bfloat162*>(kmeta + su * 8 * C::META) +
+                                  (d0 / (D / 8)) * kBlockSize + d0 % (D / 8);
+      float sd[CPL], zd[CPL];
+      {
+        __nv_bfloat162 pr[CPL];
+        if constexpr (CPL == 4) {
+          const uint4 u = *reinterpret_cast<const uint4*>(kmp);
+          *reinterpret_cast<uint4*>(pr) = u;
+        } else {
+          const uint2 u = *reinterpret_cast<const uint2*>(kmp);
+          *reinterpret_cast<uint2*>(pr) = u;
+        }
 #pragma unroll
-      for (int i = 0; i < D / 32; ++i) {
-        // channel d = lane + 32 i: page d / (D/8), entry d % (D/8)
-        const int d = lane + 32 * i;
-        const __nv_bfloat162 pr = kmp[(d / (D / 8)) * kBlockSize + d % (D / 8)];
-        sd[i] = __low2float(pr);
-        zd[i] = __high2float(pr);
+        for (int i = 0; i < CPL; ++i) { sd[i] = __low2float(pr[i]); zd[i] = __high2float(pr[i]); }
       }
 #pragma unroll
       for (int hh = 0; hh < C::HPW; ++hh) {
         const int g = cw + 4 * hh;
         if (g >= G) continue;
-        float x[D / 32], zsum = 0.f, amax = 0.f;
+        float x[CPL], zsum = 0.f, amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < D / 32; ++i) {
+        for (int i = 0; i < CPL; ++i) {
           x[i] = qcur[hh][i] * sd[i];
           zsum = fmaf(qcur[hh][i], zd[i], zsum);
           amax = fmaxf(amax, fabsf(x[i]));
@@ -517,20 +540,24 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
         e = max(-120, min(120, e));
         const float up = __int_as_float((127 + e) << 23);
         const float down = __int_as_float((127 - e) << 23);
+        uint32_t part[3] = {0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < D / 32; ++i) {
-          const int d = lane + 32 * i;
-          auto at = [&](int n) -> uint8_t* {
-            return qop + (n >> 3) * C::Q_SBO + (n & 7) * 16 + (d >> 4) * C::Q_LBO + (d & 15);
-          };
+        for (int i = 0; i < CPL; ++i) {
           const float xs = x[i] * up;
           const float x0 = rintf(xs);
           const float r0 = (xs - x0) * 128.f;
           const float x1 = rintf(r0);
           const float x2 = rintf((r0 - x1) * 128.f);
-          *at(g) = uint8_t(int8_t(int(x0)));
-          *at(G + g) = uint8_t(int8_t(int(x1)));
-          *at(2 * G + g) = uint8_t(int8_t(int(x2)));
+          part[0] |= uint32_t(uint8_t(int8_t(int(x0)))) << (8 * i);
+          part[1] |= uint32_t(uint8_t(int8_t(int(x1)))) << (8 * i);
+          part[2] |= uint32_t(uint8_t(int8_t(int(x2)))) << (8 * i);
+        }
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const int n = j * G + g;                           // operand row of this part
+          uint8_t* at = qop + (n >> 3) * C::Q_SBO + (n & 7) * 16 + (d0 >> 4) * C::Q_LBO + (d0 & 15);
+          if constexpr (CPL == 4) *reinterpret_cast<uint32_t*>(at) = part[j];
+          else *reinterpret_cast<uint16_t*>(at) = uint16_t(part[j]);
         }
         if (lane == 0) {
           qsc[(gt_q & 1) * 8 + g] = qk_scale * down;
