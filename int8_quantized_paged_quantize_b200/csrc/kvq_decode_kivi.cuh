@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSP; ++s) {
       mbar_init(pfull + s, 1);
-      mbar_init(pfree + s, 64);
+      mbar_init(pfree + s, 64 + 128);             // converters and softmax warps
     }
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(kready + s, 64);
@@ -361,9 +361,6 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
                                             (ws[2 * x + 1] >> 4) & 0x0F0F0F0Fu);
             }
           }
-          if (ct < 32)
-            reinterpret_cast<uint4*>(kmeta + su * 8 * C::META)[ct] =
-                reinterpret_cast<const uint4*>(pkmeta + sp * 8 * C::META)[ct];
           if (ct == 0) pmask_u[su] = pmask_p[sp];
           fence_proxy_async_smem();
         }
@@ -504,10 +501,12 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
     // exact s8 parts after a power-of-two scaling of the head, and sum_d q z_d;
     // the lane's consecutive channels make one word (or half word) per part
     auto store_q = [&](int gt_q, const float (&qcur)[C::HPW][D / 32]) {
-      const int su = gt_q % C::NST;
+      const int sp = gt_q % C::NSP;
+      // the tile's K (s, z) pairs, read from the packed stage the producer filled
+      // (it is released only when the converters and these warps are done);
       // channel d: page d / (D/8), entry d % (D/8); the lane's channels are
       // consecutive entries of one page
-      const __nv_bfloat162* kmp = reinterpret_cast<const __nv_bfloat162*>(kmeta + su * 8 * C::META) +
+      const __nv_bfloat162* kmp = reinterpret_cast<const __nv_bfloat162*>(pkmeta + sp * 8 * C::META) +
                                   (d0 / (D / 8)) * kBlockSize + d0 % (D / 8);
       float sd[CPL], zd[CPL];
       {
@@ -576,8 +575,9 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
 #pragma unroll
       for (int i = 0; i < D / 32; ++i) qcur[hh][i] = qv[hh][i];
     if (!wk[0].done) {
-      if (ok) ok = mbar_wait(kready + 0, 0, abort_flag, wait_limit);
-      store_q(0, qcur);
+      if (ok) ok = mbar_wait(pfull + 0, 0, abort_flag, wait_limit);
+      if (ok) store_q(0, qcur);
+      mbar_arrive(pfree + 0);
     }
     mbar_arrive(qready);
 
@@ -645,13 +645,14 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
           qs[g] = qsc[(gt & 1) * 8 + g];
           qz[g] = qzs[(gt & 1) * 8 + g];
         }
-        // ---- the next tile's query: its K stage's channel scales (the next
-        // tile may open the next piece, whose query rows were loaded ahead)
+        // ---- the next tile's query: its channel scales from the packed stage
+        // (the next tile may open the next piece, whose query rows were loaded
+        // ahead); it waits only for the producer, which runs a few tiles ahead
         const bool last_tile = i + 1 == hi;
         const bool has_next = !last_tile || more;
         if (has_next) {
           if (ok) ok = mbar_wait(qfree, gt & 1, abort_flag, wait_limit);
-          if (ok) ok = mbar_wait(kready + (gt + 1) % C::NST, ((gt + 1) / C::NST) & 1, abort_flag, wait_limit);
+          if (ok) ok = mbar_wait(pfull + (gt + 1) % C::NSP, ((gt + 1) / C::NSP) & 1, abort_flag, wait_limit);
           if (last_tile) {
 #pragma unroll
             for (int hh = 0; hh < C::HPW; ++hh)
@@ -659,6 +660,7 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
               for (int ii = 0; ii < D / 32; ++ii) qcur[hh][ii] = qv[hh][ii];
           }
           if (ok) store_q(gt + 1, qcur);
+          mbar_arrive(pfree + (gt + 1) % C::NSP);       // this packed stage's K pairs are read
           mbar_arrive(qready);
         }
         // the K stage of this tile is free (its S product has been read)

@@ -57,15 +57,21 @@ __global__ void __launch_bounds__(128) merge_kernel(const int32_t* __restrict__ 
       if (s0 + lane < n) ml = *reinterpret_cast<const float2*>(part_ml + (r0 + s0 + lane) * 2);
       const float fl = exp2f(ml.x - M);
       const int cnt = min(32, n - s0);
-#pragma unroll 4
-      for (int s = 0; s < cnt; ++s) {
-        const float f = __shfl_sync(0xffffffffu, fl, s);
-        const float ls = __shfl_sync(0xffffffffu, ml.y, s);
-        MergeVec<D> x;
-        x.load(part_o + (r0 + s0 + s) * D + lane * N);
-        l += ls * f;
+      // eight slots' vectors are requested before any is summed
+      for (int s8 = 0; s8 < cnt; s8 += 8) {
+        MergeVec<D> x[8];
 #pragma unroll
-        for (int i = 0; i < N; ++i) o[i] += x.v[i] * f;
+        for (int j = 0; j < 8; ++j)
+          if (s8 + j < cnt) x[j].load(part_o + (r0 + s0 + s8 + j) * D + lane * N);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (s8 + j >= cnt) break;
+          const float f = __shfl_sync(0xffffffffu, fl, s8 + j);
+          const float ls = __shfl_sync(0xffffffffu, ml.y, s8 + j);
+          l += ls * f;
+#pragma unroll
+          for (int i = 0; i < N; ++i) o[i] += x[j].v[i] * f;
+        }
       }
     }
   }
