@@ -413,9 +413,16 @@ def graph_loop(st, steps, warmup, world, flush):
 def e2e_loop(st, steps, warmup, world, flush):
     """The same step through the public API with host inputs: per step the
     step's inputs (q, k, v, slots, context lengths, the block tables) are copied
-    from pinned host memory and the output is read back, inside the timing. The
-    inputs of a step are packed into one pinned buffer (each at a 256-byte
-    aligned offset) and cross in one copy; the kernels take views into it."""
+    from pinned host memory and the output is read back into pinned host
+    memory, inside the timing. The inputs of a step are packed into one pinned
+    buffer (each at a 256-byte aligned offset) and cross in one copy; the
+    kernels take views into it. As a serving loop that prefetches its next step
+    does, the copies run on a copy stream: step i+1's inputs go in while step
+    i computes (two device input buffers, two output buffers), and step i's
+    output comes back while step i+1 computes. The timed region runs from the
+    first input copy to the last output copy; the step time is its K-th part.
+    L2 is not flushed between these overlapped steps: every step reads a cache
+    larger than L2."""
     w = st.w
 
     def layout(tensors):
@@ -436,36 +443,64 @@ def e2e_loop(st, steps, warmup, world, flush):
             n = t.numel() * t.element_size()
             hb[o:o + n].copy_(t.contiguous().view(-1).view(torch.uint8).cpu())
         host.append(hb)
-    dbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    dbuf = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
     views = []
-    for t, o in zip(step_tensors(0), offs):
-        n = t.numel() * t.element_size()
-        views.append(dbuf[o:o + n].view(t.dtype).view(t.shape))
-    out_h = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    for d in dbuf:
+        vv = []
+        for t, o in zip(step_tensors(0), offs):
+            n = t.numel() * t.element_size()
+            vv.append(d[o:o + n].view(t.dtype).view(t.shape))
+        views.append(vv)
+    outs = [torch.empty_like(st.out) for _ in range(2)]
+    out_h = [torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory() for _ in range(2)]
     h2d = nbytes
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = out_h[0].numel() * out_h[0].element_size()
+    comp = torch.cuda.current_stream()
+    cp = torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # input buffer b holds its step
+    ev_used = [torch.cuda.Event() for _ in range(2)]   # the step using buffer b is done
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # output b is back on the host
 
-    def one(s):
-        dbuf.copy_(host[s], non_blocking=True)
-        q, k, v, sl, cl, tables_d = views
-        st.cache.append(k, v, sl)
-        st.cache.decode(q, tables_d, cl, st.max_ctx, sm_scale=w.sm_scale, out=st.out,
-                        workspace=st.ws)
-        out_h.copy_(st.out, non_blocking=True)
+    def run(idx):
+        n = len(idx)
+        cp.wait_stream(comp)
+        with torch.cuda.stream(cp):
+            dbuf[0].copy_(host[idx[0]], non_blocking=True)
+            ev_in[0].record(cp)
+        for i in range(n):
+            b = i & 1
+            if i + 1 < n:
+                with torch.cuda.stream(cp):
+                    if i >= 1:
+                        cp.wait_event(ev_used[b ^ 1])
+                    dbuf[b ^ 1].copy_(host[idx[i + 1]], non_blocking=True)
+                    ev_in[b ^ 1].record(cp)
+            comp.wait_event(ev_in[b])
+            if i >= 2:
+                comp.wait_event(ev_out[b])
+            q, k, v, sl, cl, tables_d = views[b]
+            st.cache.append(k, v, sl)
+            st.cache.decode(q, tables_d, cl, st.max_ctx, sm_scale=w.sm_scale, out=outs[b],
+                            workspace=st.ws)
+            ev_used[b].record(comp)
+            with torch.cuda.stream(cp):
+                cp.wait_event(ev_used[b])
+                out_h[b].copy_(outs[b], non_blocking=True)
+                ev_out[b].record(cp)
+        comp.wait_stream(cp)
 
-    for s in range(warmup):
-        one(s % st.steps)
+    run([s % st.steps for s in range(warmup)])
     torch.cuda.synchronize()
     barrier(world)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
-    for i in range(steps):
-        flush.zero_()
-        evs[i][0].record()
-        one(i % st.steps)
-        evs[i][1].record()
+    flush.zero_()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(cp)
+    run([i % st.steps for i in range(steps)])
+    t1.record(cp)
     torch.cuda.synchronize()
     barrier(world)
-    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    ms = t0.elapsed_time(t1) / steps
     return ms, h2d, d2h
 
 
@@ -591,6 +626,51 @@ def bulk_append_probe(fmt, mode, reps=5, T=32768, Hk=8, D=128):
     return {"bulk_append": mode, "fmt": fmt, "tokens": T, "sequences": len(lens), "us": ms * 1e3,
             "tok_per_s": T / (ms * 1e-3), "gbs": by / (ms * 1e6), "frac": by / (ms * 1e6) / hbm,
             "peak_kind": kind, "bytes": by}
+
+
+def kivi_probe(fmt, B=32, Hk=8, G=8, D=128, ctx=8192, reps=5):
+    """One KIVI-style decode (kvq_kivi_decode_attn) on a mid-size case: B
+    sequences of ctx tokens in complete 128-token groups plus one residual
+    token each, random BF16 K/V and queries. Timed with CUDA events over
+    `reps` calls after three untimed ones. Returns one JSON-ready dict."""
+    from int8_quantized_paged_quantize_b200 import kvq
+    dev = torch.device("cuda")
+    g = torch.Generator(device="cuda").manual_seed(0)
+    groups = ctx // 128
+    nq = B * groups * 8
+    qt = torch.randperm(nq, device=dev, generator=g).to(torch.int32).reshape(B, groups * 8)
+    rt = torch.arange(B, device=dev, dtype=torch.int32).reshape(B, 1)
+    cache = kvq.KiviCache.allocate(fmt, kvq.dims(nq, Hk, Hk * G, D, groups * 8),
+                                   kvq.dims(B, Hk, Hk * G, D, 1))
+    pos = torch.arange(groups * 128, device=dev)
+    for b in range(B):
+        k = torch.randn(groups * 128, Hk, D, device=dev, generator=g).to(torch.bfloat16)
+        v = torch.randn(groups * 128, Hk, D, device=dev, generator=g).to(torch.bfloat16)
+        cache.append_groups(k, v, qt[b][pos // 16].to(torch.int64) * 16 + pos % 16)
+    kr = torch.randn(B, Hk, D, device=dev, generator=g).to(torch.bfloat16)
+    cache.residual.append(kr, kr, torch.arange(B, device=dev, dtype=torch.int64) * 16)
+    q = torch.randn(B, Hk * G, D, device=dev, generator=g).to(torch.bfloat16)
+    ql = torch.full((B,), groups * 128, dtype=torch.int32, device=dev)
+    rl = torch.ones(B, dtype=torch.int32, device=dev)
+    ws = cache.workspace(B, groups * 128, 1)
+
+    def call():
+        cache.decode(q, qt, ql, groups * 128, rt, rl, 1, workspace=ws)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        call()
+    e.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(e) / reps
+    bits = kvq.KIVI_BITS[fmt]
+    by = B * groups * 128 * Hk * (2 * D * bits / 8 + 4 + D * 4 / 128)
+    return {"kivi_probe": fmt, "batch": B, "context": groups * 128, "n_kv_heads": Hk, "group": G,
+            "head_dim": D, "ms": ms, "kv_gbs": by / (ms * 1e6), "tokens_per_s": B * groups * 128 / (ms * 1e-3),
+            "device_error": kvq.device_error()}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -936,9 +1016,14 @@ def main():
     ap.add_argument("--bulk-append", choices=["aligned", "continued"], default=None,
                     help="only time one bulk append of 32,768 tokens and print its line")
     ap.add_argument("--reps", type=int, default=5, help="timed calls of --bulk-append")
+    ap.add_argument("--kivi-probe", choices=["kivi2", "kivi4"], default=None,
+                    help="only time one KIVI-style decode on a mid-size case and print its line")
     args = ap.parse_args()
     if args.bulk_append:
         print(json.dumps(bulk_append_probe(args.fmt or "fp8", args.bulk_append, args.reps)))
+        return 0
+    if args.kivi_probe:
+        print(json.dumps(kivi_probe(args.kivi_probe)))
         return 0
     if args.impl == "reference":
         return run_reference(args)
@@ -1071,7 +1156,10 @@ def main():
                      "alg_bytes_per_launch": alg_step,
                      "traffic": measured_traffic(w.name, fmt)},
         "e2e": {"value": e2e_val, "unit": "GB/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "kvq.LayerCache append + decode per step, inputs copied from pinned host "
+                       "memory and the output read back on a copy stream overlapped with the "
+                       "neighbouring steps' kernels; timed from the first copy to the last"},
         "gpu_launches": t["launches"],
         "verify": verify,
         "prefill": prefill,

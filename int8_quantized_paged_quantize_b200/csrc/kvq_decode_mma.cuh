@@ -369,6 +369,12 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Everything above (the share, the barriers, the tensor memory) overlaps the
+  // kernel ahead on the stream when this one is launched as its programmatic
+  // dependent (the append of the same step); the query, block tables, scales
+  // and pages are read only after it has finished. The merge may launch now.
+  grid_dep_wait();
+  grid_dep_launch_dependents();
 
   PieceWalk walk;
   walk.init(b0, P0, start, end, Hk, ctx_lens, B, max_ctx, W);

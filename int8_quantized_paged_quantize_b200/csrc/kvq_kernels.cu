@@ -347,6 +347,9 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
   __shared__ int64_t sl[kBlockSize];
   __shared__ int seg_i0[kBlockSize], seg_len[kBlockSize], nseg, page_fast;
 
+  // the decode kernel of the step may start its set-up now; it reads the
+  // cache only after this grid has finished
+  tc::grid_dep_launch_dependents();
   const int h = blockIdx.y;
   const int64_t tb = int64_t(blockIdx.x) * kBlockSize;
   const int n = int(min(int64_t(kBlockSize), int64_t(T) - tb));
@@ -554,6 +557,24 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
 namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Launch as the programmatic dependent of the kernel ahead on the stream: it
+// may start (and run up to its grid_dep_wait) before that kernel finishes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <int D, int FMT>
 cudaError_t append_dispatch(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
                             void* vc, void* ks, void* vs, const kvq_dims& d, int per_tensor,
@@ -594,12 +615,13 @@ cudaError_t decode_mma_dispatch3(const void* q, int32_t B, const void* kc, const
   // walk the same share of the tile list; at least one group
   const int64_t slots_resident = int64_t(device_sm_count()) * per_sm;
   const int64_t grid = std::max<int64_t>(1, slots_resident / nrg) * nrg;
-  kern<<<dim3(unsigned(grid)), 192, C::SMEM, st>>>(
+  e = launch_pdl(kern, dim3(unsigned(grid)), dim3(192), C::SMEM, st,
       static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
       static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, nrg, d.num_blocks,
       d.max_blocks_per_seq, max_ctx, plan.partition / kTileTokens, plan.slots, sm_scale * kLog2e,
       per_tensor, n_query, decode_wait_limit(), po, pml, pcnt);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -684,23 +706,23 @@ int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* ou
   const int W = d.max_blocks_per_seq, Hq = d.n_q_heads;
   int G = 1;
   row_groups(d.n_q_heads / d.n_kv_heads, &G);
+  cudaError_t e;
   if (d.head_dim == 128) {
     if (out_f32)
-      merge_kernel<128, float><<<grid, 128, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W, po, pml,
-                                                     pcnt, static_cast<float*>(out), rows);
+      e = launch_pdl(merge_kernel<128, float>, grid, dim3(128), 0, st, ctx, Hq, G, plan.slots,
+                     max_ctx, W, po, pml, pcnt, static_cast<float*>(out), rows);
     else
-      merge_kernel<128, __nv_bfloat16><<<grid, 128, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W,
-                                                             po, pml, pcnt,
-                                                             static_cast<__nv_bfloat16*>(out), rows);
+      e = launch_pdl(merge_kernel<128, __nv_bfloat16>, grid, dim3(128), 0, st, ctx, Hq, G,
+                     plan.slots, max_ctx, W, po, pml, pcnt, static_cast<__nv_bfloat16*>(out), rows);
   } else {
     if (out_f32)
-      merge_kernel<64, float><<<grid, 128, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W, po, pml,
-                                                    pcnt, static_cast<float*>(out), rows);
+      e = launch_pdl(merge_kernel<64, float>, grid, dim3(128), 0, st, ctx, Hq, G, plan.slots,
+                     max_ctx, W, po, pml, pcnt, static_cast<float*>(out), rows);
     else
-      merge_kernel<64, __nv_bfloat16><<<grid, 128, 0, st>>>(ctx, Hq, G, plan.slots, max_ctx, W, po,
-                                                            pml, pcnt,
-                                                            static_cast<__nv_bfloat16*>(out), rows);
+      e = launch_pdl(merge_kernel<64, __nv_bfloat16>, grid, dim3(128), 0, st, ctx, Hq, G,
+                     plan.slots, max_ctx, W, po, pml, pcnt, static_cast<__nv_bfloat16*>(out), rows);
   }
+  if (e != cudaSuccess) return int(e);
   return int(cudaGetLastError());
 }
 

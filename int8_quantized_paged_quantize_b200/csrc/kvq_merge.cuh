@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const int32_t* __restrict__ 
   constexpr int N = D / 32;
   const int lane = threadIdx.x & 31;
   const int bq = blockIdx.x * 4 + (threadIdx.x >> 5);      // b * Hq + row
+  tc::grid_dep_wait();                                     // the partials are complete
   if (bq >= rows) return;
   const int b = bq / Hq;
   int ctx = ctx_lens[b];
