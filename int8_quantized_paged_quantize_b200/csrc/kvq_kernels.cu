@@ -158,54 +158,121 @@ __device__ __forceinline__ int half_warp_max(int v) {
   return v;
 }
 
-// The row maximum is taken on float bit patterns: non-negative floats order as
-// their bits read as signed integers and every negative float (-0 included)
-// reads as a negative integer, so an integer max with a floor of 0 gives the
-// float maximum, +0 when nothing is positive. Every lane of the warp must call
-// the quantizers (the half-warp reductions are warp-wide shuffles); a row that
-// is not stored is still quantized, from whatever its lanes hold.
+// Lane-wise max of two pairs of 16-bit fields, unsigned or signed (the
+// signed form with a floor of 0).
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t vmax_relu_s16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.relu.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Field-wise max of a u16x2 word over the 16 lanes of this half warp.
+__device__ __forceinline__ uint32_t half_warp_vmax_u16x2(uint32_t v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v = vmax_u16x2(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// The two BF16 values of a packed pair as floats (low half first).
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) { return make_float2(bf16_lo(w), bf16_hi(w)); }
+
+// Markstein's corrected quotient on a pair: q = RN(x r), e = RN(q s - x)
+// (exact), q' = RN(q - e r), with -x and -r passed in so that a zero x keeps
+// its sign; the same arithmetic as ScaleDiv, two lanes per instruction.
+__device__ __forceinline__ float2 div_pair(float2 x, float2 r2, float2 nr2, float2 s2) {
+  const float2 nx = __fmul2_rn(x, make_float2(-1.f, -1.f));
+  const float2 q = __fmul2_rn(x, r2);
+  const float2 e = __ffma2_rn(q, s2, nx);
+  return __ffma2_rn(e, nr2, q);
+}
+
+// Two pairs of quotients as four E4M3 / E5M2 codes (RNE, satfinite),
+// little-endian: a.x in the low byte.
+template <bool E4>
+__device__ __forceinline__ uint32_t fp8x4(float2 a, float2 b) {
+  uint32_t w;
+  if constexpr (E4)
+    asm("{\n .reg .b16 lo, hi;\n cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n"
+        " cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n mov.b32 %0, {lo, hi};\n}"
+        : "=r"(w) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  else
+    asm("{\n .reg .b16 lo, hi;\n cvt.rn.satfinite.e5m2x2.f32 lo, %2, %1;\n"
+        " cvt.rn.satfinite.e5m2x2.f32 hi, %4, %3;\n mov.b32 %0, {lo, hi};\n}"
+        : "=r"(w) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return w;
+}
+
+// Two ints saturated to [-128, 127] in bytes 0 (b) and 1 (a), bytes 2-3 from
+// the low half of c.
+__device__ __forceinline__ uint32_t pack_sat_s8x2(int a, int b, uint32_t c) {
+  uint32_t d;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// The row maximum is taken on bit patterns: non-negative floats (and BF16
+// values) order as their bits read as integers and every negative one (-0
+// included) reads as a negative signed integer, so an integer max with a floor
+// of 0 gives the float maximum, +0 when nothing is positive. The lane's BF16
+// pairs are reduced as 16-bit fields, two values per instruction. Every lane
+// of the warp must call the quantizers (the half-warp reductions are warp-wide
+// shuffles); a row that is not stored is still quantized, from whatever its
+// lanes hold.
 template <int D, int FMT>
 __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 32], RowCodes<D, FMT>& rc) {
   constexpr int E = D / 16;
+  constexpr int NW = E / 2;                          // BF16 pairs of the lane
   rc.zp = 0;
   rc.s = __float2bfloat16_rn(0.f);
   if constexpr (FMT == KVQ_BF16) {
 #pragma unroll
-    for (int i = 0; i < E / 2; ++i) rc.w[i] = raw[i];
+    for (int i = 0; i < NW; ++i) rc.w[i] = raw[i];
     return;
   } else {
-    float x[E];
-#pragma unroll
-    for (int i = 0; i < E / 2; ++i) { x[2 * i] = bf16_lo(raw[i]); x[2 * i + 1] = bf16_hi(raw[i]); }
 #pragma unroll
     for (int i = 0; i < RowCodes<D, FMT>::WORDS; ++i) rc.w[i] = 0u;
     if constexpr (FMT == KVQ_FP8_E4M3 || FMT == KVQ_FP8_E5M2) {
       // s = bf16(amax / max code), code = fp8_rne_satfinite(x / s)
       constexpr bool E4 = FMT == KVQ_FP8_E4M3;
-      int amax_bits = 0;
+      uint32_t m = raw[0] & 0x7fff7fffu;             // |x| of both halves
 #pragma unroll
-      for (int i = 0; i < E; ++i) amax_bits = max(amax_bits, __float_as_int(fabsf(x[i])));
-      const float amax = __int_as_float(half_warp_max(amax_bits));
+      for (int i = 1; i < NW; ++i) m = vmax_u16x2(m, raw[i] & 0x7fff7fffu);
+      m = half_warp_vmax_u16x2(m);
+      const float amax = __uint_as_float(max(m & 0xffffu, m >> 16) << 16);
       rc.s = __float2bfloat16_rn(E4 ? div_by_const<448>(amax) : div_by_const<57344>(amax));
       const float s = __bfloat162float(rc.s);
-      if (s != 0.f) {
-        const ScaleDiv div(s);
+      if (s >= 7.88860905e-31f) {                    // 2^-100: the corrected quotient
+        const float r = __frcp_rn(s);
+        const float2 r2 = make_float2(r, r), nr2 = make_float2(-r, -r), s2 = make_float2(s, s);
 #pragma unroll
-        for (int i = 0; i < E; i += 2) {
-          const float2 qv = make_float2(div(x[i]), div(x[i + 1]));
-          const uint32_t two = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, E4 ? __NV_E4M3 : __NV_E5M2);
-          rc.w[i >> 2] |= two << (8 * (i & 3));
+        for (int i = 0; i < NW; i += 2)
+          rc.w[i >> 1] = fp8x4<E4>(div_pair(bf16x2_to_float2(raw[i]), r2, nr2, s2),
+                                   div_pair(bf16x2_to_float2(raw[i + 1]), r2, nr2, s2));
+      } else if (s != 0.f) {                         // tiny scale: the IEEE quotient
+#pragma unroll
+        for (int i = 0; i < NW; i += 2) {
+          const float2 a = bf16x2_to_float2(raw[i]), b = bf16x2_to_float2(raw[i + 1]);
+          rc.w[i >> 1] = fp8x4<E4>(make_float2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s)),
+                                   make_float2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s)));
         }
       }
     } else {  // INT8 asymmetric: range [lo, hi] widened to hold 0
-      int hi_bits = 0, nlo_bits = 0;
+      // hi = max(0, max x) and nlo = max(0, max -x), as 16-bit fields
+      uint32_t hw = vmax_relu_s16x2(raw[0], 0u), nw = vmax_relu_s16x2(raw[0] ^ 0x80008000u, 0u);
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        hi_bits = max(hi_bits, __float_as_int(x[i]));
-        nlo_bits = max(nlo_bits, __float_as_int(-x[i]));
+      for (int i = 1; i < NW; ++i) {
+        hw = vmax_relu_s16x2(hw, raw[i]);
+        nw = vmax_relu_s16x2(nw, raw[i] ^ 0x80008000u);
       }
-      const float hi = __int_as_float(half_warp_max(hi_bits));     // max(0, max x)
-      const float nlo = __int_as_float(half_warp_max(nlo_bits));   // -min(0, min x)
+      // both maxima in one word (hi low, nlo high), reduced over the half warp
+      const uint32_t hn = half_warp_vmax_u16x2(vmax_u16x2(__byte_perm(hw, nw, 0x5410),
+                                                           __byte_perm(hw, nw, 0x7632)));
+      const float hi = bf16_lo(hn), nlo = bf16_hi(hn);
       rc.s = __float2bfloat16_rn(div_by_const<255>(__fadd_rn(hi, nlo)));
       const float s = __bfloat162float(rc.s);
       if (s != 0.f) {
@@ -213,15 +280,30 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 32], RowC
         const float zq = fminf(fmaxf(-div(nlo), -1024.f), 1024.f);   // lo / s
         rc.zp = min(127, max(-128, -128 - __float2int_rn(zq)));
         // code = clamp(rint(x / s) + zp, -128, 127): every x of the row lies in
-        // [lo, hi], so |x / s| stays near 255 and the rounding addition applies;
-        // the clamp runs on the sum's bits, shifted by zp
-        const int cmin = kRintBits - 128 - rc.zp, cmax = kRintBits + 127 - rc.zp;
+        // [lo, hi], so |x / s| stays near 255 and the rounding addition
+        // applies; the sum's bits less kRintBits are rint(x / s), zp is added
+        // as an integer and the pack saturates
+        const int off = rc.zp - kRintBits;
         int c[E];
+        if (div.fast) {
+          const float2 r2 = make_float2(div.r, div.r), nr2 = make_float2(-div.r, -div.r);
+          const float2 s2 = make_float2(s, s), mg = make_float2(kRintMagic, kRintMagic);
 #pragma unroll
-        for (int i = 0; i < E; ++i)
-          c[i] = min(cmax, max(cmin, __float_as_int(__fadd_rn(div(x[i]), kRintMagic)))) + rc.zp;
+          for (int i = 0; i < NW; ++i) {
+            const float2 t = __fadd2_rn(div_pair(bf16x2_to_float2(raw[i]), r2, nr2, s2), mg);
+            c[2 * i] = __float_as_int(t.x) + off;
+            c[2 * i + 1] = __float_as_int(t.y) + off;
+          }
+        } else {
 #pragma unroll
-        for (int i = 0; i < E; i += 4) rc.w[i >> 2] = pack_low_bytes(c[i], c[i + 1], c[i + 2], c[i + 3]);
+          for (int i = 0; i < NW; ++i) {
+            const float2 x = bf16x2_to_float2(raw[i]);
+            c[2 * i] = __float_as_int(__fadd_rn(__fdiv_rn(x.x, s), kRintMagic)) + off;
+            c[2 * i + 1] = __float_as_int(__fadd_rn(__fdiv_rn(x.y, s), kRintMagic)) + off;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < E; i += 4) rc.w[i >> 2] = pack_sat_s8x2(c[i + 1], c[i], pack_sat_s8x2(c[i + 3], c[i + 2], 0u));
       }
     }
   }
