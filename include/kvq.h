@@ -31,11 +31,11 @@
  * - The decode kernels (kvq_decode_attn, _partial, _verify, kvq_prefill_attn)
  *   and the merge are launched as programmatic dependents of the kernel ahead
  *   of them on the stream: when that kernel signals early completion (the
- *   append kernel of kvq_append does), their set-up, which reads
- *   context_lens, overlaps its tail, and they read the query, block tables,
- *   scales and pages only after it has finished. Ordinary kernels never
- *   signal, so with them the order is the usual one; a caller's own kernel
- *   that signals early must have written context_lens before it does.
+ *   append kernel of kvq_append does), their set-up (barriers, tensor
+ *   memory) overlaps its tail, and they read every argument in device memory
+ *   (context lengths, query, block tables, scales, pages, workspace) only
+ *   after it has finished. Ordinary kernels never signal, so with them the
+ *   order is the usual one.
  * - Data-dependent faults (a slot or block id outside the pool, a context
  *   length beyond the block table or beyond max_context_len) cannot be seen on
  *   the host. Kernels skip the offending token, page or sequence and set a bit

@@ -238,6 +238,76 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   const int rg = int(blockIdx.x % nrg);
   const long long grp = blockIdx.x / nrg, NG = gridDim.x / nrg;
 
+  uint8_t* kring = smem + C::OFF_K;
+  uint8_t* vring = smem + C::OFF_V;
+  uint8_t* kmeta = smem + C::OFF_KM;
+  uint8_t* vmeta = smem + C::OFF_VM;
+  uint8_t* qop = smem + C::OFF_Q;
+  uint8_t* pop = smem + C::OFF_P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kfull = bars;
+  uint64_t* kempty = bars + C::NST;
+  uint64_t* vfull = bars + 2 * C::NST;
+  uint64_t* vempty = bars + 3 * C::NST;
+  uint64_t* sfull = bars + 4 * C::NST;      // [2]
+  uint64_t* sfree = sfull + 2;              // [2]
+  uint64_t* pready = sfree + 2;             // [2]
+  uint64_t* ofull = pready + 2;             // [2]
+  uint64_t* ofree = ofull + 2;              // [2]
+  uint64_t* qready = ofree + 2;
+  uint64_t* qfree = qready + 1;
+  uint64_t* drain = qfree + 1;
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  float* red2 = reinterpret_cast<float*>(smem + C::OFF_RED2);
+  float* qsc = reinterpret_cast<float*>(smem + C::OFF_QSC);
+  float* qsum = qsc + 8;
+  volatile uint32_t* pmask = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_PMASK);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  // ------------------------------------------------------------ set-up
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(kfull + s, 1);
+      mbar_init(kempty + s, 128);
+      mbar_init(vfull + s, 1);
+      mbar_init(vempty + s, 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(sfull + j, 1);
+      mbar_init(sfree + j, 128);
+      mbar_init(pready + j, 128);
+      mbar_init(ofull + j, 1);
+      mbar_init(ofree + j, 128);
+    }
+    mbar_init(qready, 128);
+    mbar_init(qfree, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // zero the query operand and both P buffers (padding rows stay zero)
+    const int ct = threadIdx.x - 64;
+    for (int i = ct * 16; i < C::QBYTES + 2 * C::PBYTES; i += 128 * 16)
+      *reinterpret_cast<uint4*>(qop + i) = make_uint4(0, 0, 0, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // Everything above (the barriers, the tensor memory) overlaps the kernel
+  // ahead on the stream when this one is launched as its programmatic
+  // dependent (the append of the same step) and touches no global memory: the
+  // context lengths, query, block tables, scales and pages are read only after
+  // that kernel has finished, whatever it wrote. The merge may launch now.
+  grid_dep_wait();
+  grid_dep_launch_dependents();
+
   // ------------------------------------------------------------ the share
   // T = total work-list cost; each thread sums the run costs of some sequences
   long long* red64 = reinterpret_cast<long long*>(smem + C::OFF_RED);   // [6] + 2
@@ -263,7 +333,10 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   for (int w = 0; w < 6; ++w) T += red64[w];
   T *= Hk;
   const long long N = ll_min(NG, ll_max(1, T / max(1, unit_tiles)));
-  if (T == 0 || grp >= N) return;                        // uniform for the CTA
+  if (T == 0 || grp >= N) {                               // uniform for the CTA
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+    return;
+  }
   const long long start = (grp * T) / N;
   const long long end = ((grp + 1) * T) / N;
   // the sequence holding cost position `start`: block-wide scan of run costs
@@ -305,76 +378,6 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
   // group that holds work-list cost position x; the slot of a piece is its
   // group's rank among the groups that hold real tiles of the piece's (b, h)
   auto cta_of = [&](long long x) -> long long { return ((x + 1) * N - 1) / T; };
-
-  uint8_t* kring = smem + C::OFF_K;
-  uint8_t* vring = smem + C::OFF_V;
-  uint8_t* kmeta = smem + C::OFF_KM;
-  uint8_t* vmeta = smem + C::OFF_VM;
-  uint8_t* qop = smem + C::OFF_Q;
-  uint8_t* pop = smem + C::OFF_P;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* kfull = bars;
-  uint64_t* kempty = bars + C::NST;
-  uint64_t* vfull = bars + 2 * C::NST;
-  uint64_t* vempty = bars + 3 * C::NST;
-  uint64_t* sfull = bars + 4 * C::NST;      // [2]
-  uint64_t* sfree = sfull + 2;              // [2]
-  uint64_t* pready = sfree + 2;             // [2]
-  uint64_t* ofull = pready + 2;             // [2]
-  uint64_t* ofree = ofull + 2;              // [2]
-  uint64_t* qready = ofree + 2;
-  uint64_t* qfree = qready + 1;
-  uint64_t* drain = qfree + 1;
-  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
-  float* red2 = reinterpret_cast<float*>(smem + C::OFF_RED2);
-  float* qsc = reinterpret_cast<float*>(smem + C::OFF_QSC);
-  float* qsum = qsc + 8;
-  volatile uint32_t* pmask = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_PMASK);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-
-  // ------------------------------------------------------------ set-up
-  __syncthreads();                                          // prologue scratch read by all
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NST; ++s) {
-      mbar_init(kfull + s, 1);
-      mbar_init(kempty + s, 128);
-      mbar_init(vfull + s, 1);
-      mbar_init(vempty + s, 1);
-    }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(sfull + j, 1);
-      mbar_init(sfree + j, 128);
-      mbar_init(pready + j, 128);
-      mbar_init(ofull + j, 1);
-      mbar_init(ofree + j, 128);
-    }
-    mbar_init(qready, 128);
-    mbar_init(qfree, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    mbar_init_fence();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  if (warp >= 2) {
-    // zero the query operand and both P buffers (padding rows stay zero)
-    const int ct = threadIdx.x - 64;
-    for (int i = ct * 16; i < C::QBYTES + 2 * C::PBYTES; i += 128 * 16)
-      *reinterpret_cast<uint4*>(qop + i) = make_uint4(0, 0, 0, 0);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  // Everything above (the share, the barriers, the tensor memory) overlaps the
-  // kernel ahead on the stream when this one is launched as its programmatic
-  // dependent (the append of the same step); the query, block tables, scales
-  // and pages are read only after it has finished. The merge may launch now.
-  grid_dep_wait();
-  grid_dep_launch_dependents();
 
   PieceWalk walk;
   walk.init(b0, P0, start, end, Hk, ctx_lens, B, max_ctx, W);
