@@ -380,13 +380,21 @@ int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void*
  * The chunk's chunk_len tokens are the last chunk_len tokens of each
  * sequence's context, already appended (context_lens[b] counts them). Chunk
  * position j attends to tokens 0 .. context_lens[b] - chunk_len + j (the same
- * rule as kvq_decode_verify with n_query = chunk_len, and the same kernel):
+ * rule as kvq_decode_verify with n_query = chunk_len):
  *   out[b][h][j] = softmax_t(sm_scale * q[b][h][j] . K_b[t][h/G]) weighted sum
  *                  of V_b[t][h/G] over t < context_lens[b] - chunk_len + 1 + j.
  * q    device, [batch][n_q_heads][chunk_len][head_dim] BF16 (head-major).
  * out  device, the same shape, BF16 or FP32 per out_dtype.
  * chunk_len in 1 .. 1024; the other arguments and errors are those of
- * kvq_decode_verify. workspace: kvq_prefill_attn_workspace_bytes(...) bytes.
+ * kvq_decode_verify. workspace: kvq_prefill_attn_workspace_bytes(...) bytes
+ * (the same size as kvq_decode_verify's for the same arguments).
+ * Unlike kvq_decode_verify (the cache tokens as the rows of the tensor-core
+ * products, at most 8 query rows per product), this call runs a kernel whose
+ * products take 128 query rows of a KV head at a time (the chunk's positions
+ * of its G query heads) against 64-token halves of the cache's 128-token
+ * tiles, with the 8-bit codes expanded to f16 / bf16 in shared memory: the
+ * scores are exact products accumulated in FP32 and the softmax weights keep
+ * 16 bits, so the outputs agree with kvq_decode_verify's to rounding.
  */
 size_t kvq_prefill_attn_workspace_bytes(int32_t batch, int32_t chunk_len, int32_t max_context_len,
                                         int32_t partition_tokens, kvq_fmt fmt,

@@ -53,7 +53,11 @@ int make_plan(int32_t batch, int32_t max_ctx, int32_t partition_tokens, const kv
   const size_t rows = size_t(batch) * d->n_q_heads * size_t(n_query) * size_t(plan->slots);
   plan->o_bytes = round256(rows * d->head_dim * sizeof(float));
   plan->ml_bytes = round256(rows * 2 * sizeof(float));
-  plan->cnt_bytes = round256(size_t(batch) * d->n_kv_heads * size_t(groups) * sizeof(int32_t));
+  // partial counts: one per (sequence, row group) for the decode kernel, one
+  // per query row for the prefill kernel
+  const size_t counts = std::max(size_t(batch) * d->n_kv_heads * size_t(groups),
+                                 size_t(batch) * d->n_q_heads * size_t(n_query));
+  plan->cnt_bytes = round256(counts * sizeof(int32_t));
   plan->total = plan->o_bytes + plan->ml_bytes + plan->cnt_bytes;
   return KVQ_OK;
 }
@@ -218,7 +222,7 @@ int verify_launch(const void* q, int32_t batch, int32_t n_query, const void* k_c
                   const int32_t* context_lens, int32_t max_context_len, float sm_scale, void* out,
                   kvq_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
                   int32_t partition_tokens, kvq_fmt fmt, const kvq_dims* dims,
-                  kvq_stream_t stream) {
+                  kvq_stream_t stream, bool prefill) {
   if (n_query < 1 || n_query > kMaxQueryPositions) return KVQ_ERR_ARG;
   DecodePlan plan;
   int rc = check_decode_common(batch, max_context_len, partition_tokens, fmt, dims, &plan, n_query);
@@ -234,6 +238,15 @@ int verify_launch(const void* q, int32_t batch, int32_t n_query, const void* k_c
   if (workspace_bytes < plan.total) return KVQ_ERR_WORKSPACE;
   kvq_dims eff = *dims;
   eff.n_q_heads = dims->n_q_heads * n_query;
+  if (prefill) {
+    // query rows as the MMA's M dimension (128-row blocks), one count per row
+    rc = cuda_rc(launch_prefill_partial(q, batch, k_cache, v_cache, ks, vs, block_tables,
+                                        context_lens, max_context_len, sm_scale, plan, workspace,
+                                        fmt, *dims, stream, n_query));
+    if (rc != KVQ_OK) return rc;
+    return cuda_rc(launch_decode_merge(batch, context_lens, max_context_len, out,
+                                       out_dtype == KVQ_OUT_F32, workspace, plan, eff, stream, 1));
+  }
   rc = cuda_rc(launch_decode_partial(q, batch, k_cache, v_cache, ks, vs, block_tables, context_lens,
                                      max_context_len, sm_scale, plan, workspace, fmt, eff, stream,
                                      n_query));
@@ -268,7 +281,7 @@ int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void*
                       kvq_stream_t stream) {
   return verify_launch(q, batch, n_query, k_cache, v_cache, scales, block_tables, context_lens,
                        max_context_len, sm_scale, out, out_dtype, workspace, workspace_bytes,
-                       partition_tokens, fmt, dims, stream);
+                       partition_tokens, fmt, dims, stream, false);
 }
 
 size_t kvq_prefill_attn_workspace_bytes(int32_t batch, int32_t chunk_len, int32_t max_context_len,
@@ -285,7 +298,7 @@ int kvq_prefill_attn(const void* q, int32_t batch, int32_t chunk_len, const void
                      kvq_stream_t stream) {
   return verify_launch(q, batch, chunk_len, k_cache, v_cache, scales, block_tables, context_lens,
                        max_context_len, sm_scale, out, out_dtype, workspace, workspace_bytes,
-                       partition_tokens, fmt, dims, stream);
+                       partition_tokens, fmt, dims, stream, true);
 }
 
 // ---------------------------------------------------------------- KIVI-style low-bit cache

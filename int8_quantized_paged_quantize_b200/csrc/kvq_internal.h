@@ -50,6 +50,7 @@ struct DecodePlan {
   size_t o_bytes;      // partial outputs  [B][Hq][slots][D] f32
   size_t ml_bytes;     // partial (max, sum) [B][Hq][slots][2] f32
   size_t cnt_bytes;    // partials written per (sequence, row group) [B][Hk * groups] int32
+                       // (decode kernel) or per query row [B][Hq * n_query] (prefill kernel)
   size_t total;        // workspace bytes (256-aligned pieces)
 };
 // Fills `plan` for query rows n_q_heads * n_query per sequence; returns KVQ_OK
@@ -83,8 +84,16 @@ int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* 
                           const int32_t* ctx, int32_t max_ctx, float sm_scale,
                           const DecodePlan& plan, void* ws, kvq_fmt fmt, const kvq_dims& d,
                           void* stream, int n_query = 1);
+// Chunked-prefill partials: the n_query positions of the G query heads of a KV
+// head as 128-row blocks of the query-row-major kernel; one count per row.
+int launch_prefill_partial(const void* q, int32_t B, const void* kc, const void* vc,
+                           const void* ks, const void* vs, const int32_t* tables,
+                           const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                           const DecodePlan& plan, void* ws, kvq_fmt fmt, const kvq_dims& d,
+                           void* stream, int n_query);
 int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* out, bool out_f32,
-                        const void* ws, const DecodePlan& plan, const kvq_dims& d, void* stream);
+                        const void* ws, const DecodePlan& plan, const kvq_dims& d, void* stream,
+                        int rows_per_count = 0);
 int read_device_error(uint32_t* flags, int clear);
 int launch_kivi_decode(const void* q, int32_t B, const void* kc, const void* vc, const void* km,
                        const void* vm, const int32_t* tables, const int32_t* qlens,

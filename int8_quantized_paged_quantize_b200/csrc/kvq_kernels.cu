@@ -71,6 +71,7 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 #include "kvq_decode_kivi.cuh"
 #include "kvq_kivi.cuh"
 #include "kvq_merge.cuh"
+#include "kvq_prefill.cuh"
 
 namespace kvq {
 
@@ -723,7 +724,61 @@ cudaError_t decode_dispatch2(int R, const void* q, int32_t B, const void* kc, co
     default: return decode_mma_dispatch3<D, 8, FMT>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, per_tensor, n_query, nrg, st);
   }
 }
+
+template <int D, int FMT>
+cudaError_t prefill_dispatch2(const void* q, int32_t B, const void* kc, const void* vc,
+                              const void* ks, const void* vs, const int32_t* tables,
+                              const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                              const DecodePlan& plan, void* ws, const kvq_dims& d, int per_tensor,
+                              int n_query, cudaStream_t st) {
+  using C = PfCfg<D, FMT>;
+  auto kern = prefill_mma_kernel<D, FMT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int G = d.n_q_heads / d.n_kv_heads;
+  const int R = G * n_query;                         // query rows of a KV head
+  const int nrb = (R + 127) / 128;                   // 128-row blocks, one CTA each
+  float* po = static_cast<float*>(ws);
+  float* pml = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.o_bytes);
+  int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
+  // one CTA per SM, in groups of nrb that walk the same share of the tile list
+  const int64_t grid = std::max<int64_t>(1, int64_t(device_sm_count()) / nrb) * nrb;
+  e = launch_pdl(kern, dim3(unsigned(grid)), dim3(256), C::SMEM, st,
+      static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
+      static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
+      static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, G, n_query, nrb,
+      d.num_blocks, d.max_blocks_per_seq, max_ctx, plan.partition / kTileTokens, plan.slots,
+      sm_scale * kLog2e, per_tensor, decode_wait_limit(), po, pml, pcnt);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 }  // namespace
+
+int launch_prefill_partial(const void* q, int32_t B, const void* kc, const void* vc,
+                           const void* ks, const void* vs, const int32_t* tables,
+                           const int32_t* ctx, int32_t max_ctx, float sm_scale,
+                           const DecodePlan& plan, void* ws, kvq_fmt fmt, const kvq_dims& d,
+                           void* stream, int n_query) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  const int pt = fmt == KVQ_INT8_TENSOR;
+#define KVQ_PF(DD, FF) prefill_dispatch2<DD, FF>(q, B, kc, vc, ks, vs, tables, ctx, max_ctx, sm_scale, plan, ws, d, pt, n_query, st)
+  if (d.head_dim == 128) {
+    if (fmt == KVQ_FP8_E4M3) e = KVQ_PF(128, KVQ_FP8_E4M3);
+    else if (fmt == KVQ_FP8_E5M2) e = KVQ_PF(128, KVQ_FP8_E5M2);
+    else if (fmt == KVQ_INT8_ASYM) e = KVQ_PF(128, KVQ_INT8_ASYM);
+    else if (fmt_static(fmt)) e = KVQ_PF(128, KVQ_INT8_CHANNEL);
+    else e = KVQ_PF(128, KVQ_BF16);
+  } else {
+    if (fmt == KVQ_FP8_E4M3) e = KVQ_PF(64, KVQ_FP8_E4M3);
+    else if (fmt == KVQ_FP8_E5M2) e = KVQ_PF(64, KVQ_FP8_E5M2);
+    else if (fmt == KVQ_INT8_ASYM) e = KVQ_PF(64, KVQ_INT8_ASYM);
+    else if (fmt_static(fmt)) e = KVQ_PF(64, KVQ_INT8_CHANNEL);
+    else e = KVQ_PF(64, KVQ_BF16);
+  }
+#undef KVQ_PF
+  return int(e);
+}
 
 int launch_append(const void* k, const void* v, const int64_t* slots, int32_t T, void* kc,
                   void* vc, void* ks, void* vs, kvq_fmt fmt, const kvq_dims& d, void* stream) {
@@ -776,7 +831,8 @@ int launch_decode_partial(const void* q, int32_t B, const void* kc, const void* 
 }
 
 int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* out, bool out_f32,
-                        const void* ws, const DecodePlan& plan, const kvq_dims& d, void* stream) {
+                        const void* ws, const DecodePlan& plan, const kvq_dims& d, void* stream,
+                        int rows_per_count) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float* po = static_cast<const float*>(ws);
   const float* pml = reinterpret_cast<const float*>(static_cast<const char*>(ws) + plan.o_bytes);
@@ -786,8 +842,8 @@ int launch_decode_merge(int32_t B, const int32_t* ctx, int32_t max_ctx, void* ou
   const dim3 grid(unsigned((rows + 3) / 4));
   // G: query rows per row group, the unit part_cnt is kept for
   const int W = d.max_blocks_per_seq, Hq = d.n_q_heads;
-  int G = 1;
-  row_groups(d.n_q_heads / d.n_kv_heads, &G);
+  int G = rows_per_count;
+  if (G <= 0) row_groups(d.n_q_heads / d.n_kv_heads, &G);
   cudaError_t e;
   if (d.head_dim == 128) {
     if (out_f32)

@@ -10,9 +10,12 @@ dequantized K/V, across formats, GQA groups, head_dims, ragged contexts
 (including contexts shorter than n_query, whose first positions see nothing)
 and split-K partitions that end inside the new tokens. More query rows per KV
 head than one row group of the kernel holds (G * n_query > 8: 2 or 4 positions
-at the 70B-shaped G = 8) and a 64-token prefill chunk at G = 4 ("From FP8 KV
-cache to INT4 weight-only", Core concepts 1): a chunk's queries attend to the
-cached prefix and, causally, to the chunk) are checked the same way.
+at the 70B-shaped G = 8) are checked the same way. Chunked prefill ("From FP8
+KV cache to INT4 weight-only", Core concepts 1): a chunk's queries attend to the
+cached prefix and, causally, to the chunk) runs its own kernel (128 query rows
+per tensor-core product): 64-token chunks at G = 4 and 8 in every format,
+row counts that leave a 128-row block partly empty, long prefixes split across
+CTAs, and agreement with the verification kernel on the same positions.
 """
 
 import numpy as np
@@ -139,15 +142,48 @@ def test_verify_rows_beyond_one_group(fmt, G, nq):
     _zero_rows(out, lens, nq)
 
 
-@pytest.mark.parametrize("fmt", ["fp8", "int8", "bf16", "e5m2"])
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "bf16", "e5m2", "int8c", "int8t"])
 def test_prefill_chunk_of_64_at_group_4(fmt):
-    """A 64-token prefill chunk at G = 4 (256 query rows per KV head): contexts
-    that are exactly the chunk, one token more, and long cached prefixes."""
+    """A 64-token prefill chunk at G = 4 (256 query rows per KV head, two
+    128-row blocks of the prefill kernel): contexts that are exactly the chunk,
+    one token more, and long cached prefixes."""
     err, out, ref, lens = _run(fmt, 128, 4, 64, ctx=[64, 65, 200, 1000, 4000], call="prefill")
     _check(err)
 
 
-def test_prefill_equals_verify_with_the_same_positions():
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_chunk_of_64_at_group_8(fmt, D):
+    """The 70B-shaped group: 512 query rows per KV head (four row blocks)."""
+    err, out, ref, lens = _run(fmt, D, 8, 64, ctx=[64, 129, 700, 2500], call="prefill")
+    _check(err)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("G,nq", [(1, 1), (2, 100), (8, 17), (4, 3), (1, 200)])
+def test_prefill_ragged_row_blocks(fmt, G, nq):
+    """Row counts that leave the last 128-row block partly empty (200 rows: 72
+    in the second block; 136 rows: 8), a single row, and contexts shorter than
+    the chunk, whose first positions see nothing (zero rows)."""
+    err, out, ref, lens = _run(fmt, 128, G, nq, ctx=[1, 5, 130, 333, 1000], call="prefill")
+    _check(err)
+    _zero_rows(out, lens, nq)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "bf16"])
+def test_prefill_split_across_ctas(fmt):
+    """Long prefixes cut into 256-token partitions: a row's partials come from
+    several CTAs and the merge combines them."""
+    err, out, ref, lens = _run(fmt, 128, 4, 32, ctx=[5000, 3100, 777], partition=256, call="prefill")
+    _check(err)
+
+
+def test_prefill_agrees_with_verify_on_the_same_positions():
+    """The same positions through the two kernels (query rows as the M
+    dimension against query rows as the N dimension of the products): both
+    within tolerance of the oracle and close to each other."""
     e1, o1, _, _ = _run("fp8", 64, 2, 16, ctx=[40, 300], call="prefill")
     e2, o2, _, _ = _run("fp8", 64, 2, 16, ctx=[40, 300], call="verify")
-    assert torch.equal(o1, o2)
+    _check(e1)
+    _check(e2)
+    assert (o1 - o2).abs().max().item() <= 2e-3
