@@ -674,6 +674,63 @@ def kivi_probe(fmt, B=32, Hk=8, G=8, D=128, ctx=8192, reps=5):
             "device_error": kvq.device_error()}
 
 
+def prefill_probe(fmt, B=8, Hk=8, G=8, D=128, ctx=8192, n_query=64, reps=5, call="prefill"):
+    """One chunked-prefill (kvq_prefill_attn) or verification (kvq_decode_verify)
+    call on a mid-size case: B sequences of ctx cached tokens (random BF16 K/V
+    appended through kvq_append, shuffled pages), the last n_query of them the
+    chunk. Timed with CUDA events over `reps` calls after three untimed ones.
+    Returns one JSON-ready dict (KV bytes read once per call, attention FLOPs
+    of the causal chunk)."""
+    from int8_quantized_paged_quantize_b200 import kvq
+    dev = torch.device("cuda")
+    g = torch.Generator(device="cuda").manual_seed(0)
+    npg = (ctx + 15) // 16
+    nb = B * npg
+    tables = torch.randperm(nb, device=dev, generator=g).to(torch.int32).reshape(B, npg)
+    d = kvq.dims(nb, Hk, Hk * G, D, npg)
+    k = torch.randn(B * ctx, Hk, D, device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn(B * ctx, Hk, D, device=dev, generator=g).to(torch.bfloat16)
+    pos = torch.arange(ctx, device=dev)
+    slots = torch.cat([tables[b][pos // 16].to(torch.int64) * 16 + pos % 16 for b in range(B)])
+    if fmt in STATIC:
+        ks, vs = Setup.static_scales((k, v), fmt == "int8c")
+        cache = kvq.LayerCache.allocate(fmt, d, k_static=ks, v_static=vs)
+    else:
+        cache = kvq.LayerCache.allocate(fmt, d)
+    cache.append(k, v, slots)
+    del k, v
+    q = torch.randn(B, Hk * G, n_query, D, device=dev, generator=g).to(torch.bfloat16)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    import ctypes
+    size_fn = (kvq.lib().kvq_prefill_attn_workspace_bytes if call == "prefill"
+               else kvq.lib().kvq_decode_verify_workspace_bytes)
+    n = size_fn(B, n_query, ctx, 0, kvq.FMT[fmt], ctypes.byref(d))
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    fn = kvq.prefill_attn if call == "prefill" else kvq.decode_verify
+
+    def run():
+        fn(q, cache.k, cache.v, cache.k_scale, cache.v_scale, tables, lens, ctx, D ** -0.5, out,
+           fmt, d, workspace=ws)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(e) / reps
+    seen = float(B * sum(ctx - n_query + 1 + j for j in range(n_query)))
+    flops = 4.0 * Hk * G * D * seen
+    kv = B * ctx * Hk * (2 * D * ELEM[fmt] + META_BYTES[fmt])
+    return {"probe": call, "fmt": fmt, "batch": B, "context": ctx, "n_query": n_query,
+            "n_kv_heads": Hk, "group": G, "head_dim": D, "ms": ms,
+            "attention_tflops": flops / (ms * 1e-3) / 1e12, "kv_gbs": kv / (ms * 1e6),
+            "device_error": kvq.device_error()}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def cpu_model():
     """The host CPU's model name (from /proc/cpuinfo), or None."""
@@ -1023,12 +1080,19 @@ def main():
     ap.add_argument("--reps", type=int, default=5, help="timed calls of --bulk-append")
     ap.add_argument("--kivi-probe", choices=["kivi2", "kivi4"], default=None,
                     help="only time one KIVI-style decode on a mid-size case and print its line")
+    ap.add_argument("--prefill-probe", choices=["prefill", "verify"], default=None,
+                    help="only time one chunked-prefill (or verification) call on a mid-size case")
+    ap.add_argument("--n-query", type=int, default=64, help="chunk length of --prefill-probe")
     args = ap.parse_args()
     if args.bulk_append:
         print(json.dumps(bulk_append_probe(args.fmt or "fp8", args.bulk_append, args.reps)))
         return 0
     if args.kivi_probe:
         print(json.dumps(kivi_probe(args.kivi_probe)))
+        return 0
+    if args.prefill_probe:
+        print(json.dumps(prefill_probe(args.fmt or "fp8", n_query=args.n_query, reps=args.reps,
+                                       call=args.prefill_probe)))
         return 0
     if args.impl == "reference":
         return run_reference(args)
