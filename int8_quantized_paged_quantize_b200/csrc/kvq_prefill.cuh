@@ -9,12 +9,16 @@
 //   softmax in FP32 registers, one row per thread, over the tile's tokens,
 //     with the per-token K scale (and zero point) applied to the columns
 //   O[128 x D] += P'[128 x 64] . V[64 x D]                     (P' in tensor
-//                              memory, V codes expanded to bf16)
-// where P' = p * v_scale of the token, kept exactly to 16 bits as two bf16
-// parts that share the FP32 accumulator. The cache codes are exact in f16 /
-// bf16 (E4M3, E5M2 and int8 values all are), the query is exact in bf16 and
-// in f16 after a per-row power-of-two scaling, and the products accumulate in
-// FP32, so the scores are those of the dequantized cache up to FP32 rounding.
+//                              memory, V codes expanded to f16)
+// where P' = p * v_scale of the token, kept to 22 bits as two f16 parts that
+// share the FP32 accumulator (bf16 parts and the bf16 V pages as stored, for
+// a BF16 cache). The cache codes are exact in f16 (E4M3, E5M2 and int8 values
+// all are), the query is exact in bf16 and in f16 after a per-row
+// power-of-two scaling, and the products accumulate in FP32, so the scores are
+// those of the dequantized cache up to FP32 rounding. The online softmax keeps
+// a lazily moved reference (it moves when the largest possible weight of a
+// half tile, the score's exponential times the half's largest V scale, would
+// exceed 2^8 relative to it), so P' stays within f16 range.
 // Static INT8 scales vary along the contraction: the query is multiplied by
 // the K scale of each channel and kept as two f16 parts; the V scale of each
 // channel multiplies the finished row. Included by kvq_kernels.cu after
@@ -26,15 +30,15 @@
 // for the others. Each piece ends in an online-softmax partial per row, and
 // the merge kernel combines a row's partials (one count per row).
 //
-// 8 warps per CTA:
+// 10 warps per CTA:
 //   warp 0      producer: lanes 0..7 copy one K and one V page each of a tile
 //               (1-D bulk copies) into a ring of raw stages and store the
 //               pages' scales beside them.
 //   warp 1      allocates TMEM; one thread issues the MMAs.
 //   warps 2..5  softmax warps, one per TMEM lane quarter: thread r owns query
 //               row r (S, P and O lane r); they also build the query operand.
-//   warps 6..7  converters: expand each half tile's K codes to f16 and V codes
-//               to bf16 in a converted stage, with V rows of tokens past the
+//   warps 6..9  converters: expand each half tile's K and V codes to f16 in a
+//               converted stage, with V rows of tokens past the
 //               sequence end or on invalid pages zeroed, and turn the
 //               per-token scales into FP32 column factors. For a BF16 cache
 //               they only zero those V rows in the raw stage.
@@ -55,21 +59,25 @@ struct PfCfg {
   static constexpr int PAGE = kBlockSize * D * E;                // raw page bytes
   static constexpr int MV = F8 ? 1 : (ZP ? 2 : 0);               // per-token metadata values
   static constexpr int METAB = kBlockSize * MV * 2;              // raw scale bytes per page
-  static constexpr int NST = (BF || SI) ? 2 : 3;                 // raw ring stages (tiles)
+  static constexpr int NST = 2;                                  // raw ring stages (tiles)
   static constexpr int HT = 64;                                  // tokens per half tile
   static constexpr int CPAGE = kBlockSize * D * 2;               // page bytes at 16 bits
   static constexpr int QP = SI ? 2 : 1;                          // query parts
   static constexpr int QBYTES = 128 * D * 2;                     // one query operand
-  static constexpr int NCS = BF ? 0 : 2;                         // converted half-tile stages
-  static constexpr int CMETA = 4 * HT * 4;                       // floats a, b, sv, zv per token
+  // converted half-tile stages: three let the converters run two halves ahead
+  // of the PV product (static INT8 keeps two: its query takes two operands)
+  static constexpr int NCS = BF ? 0 : (SI ? 2 : 3);
+  static constexpr int NCB = BF ? 2 : NCS;                        // half-tile slots of the barriers
+  static constexpr int CMETA = 4 * HT * 4 + 128;                 // floats a, b, sv, zv per token; max sv
   static constexpr int CSTAGE = 8 * CPAGE + CMETA;               // K (4 pages), V (4 pages), meta
   // operand strides (bytes): K pages and the query are K-major with 8-row
   // groups of 16-byte chunks; V pages are stored transposed (tokens contiguous)
   static constexpr uint32_t K_LBO = 128, K_SBO = 16 * D;          // 16-bit K page
   static constexpr uint32_t V_LBO = 16 * D, V_SBO = 128;          // 16-bit V page
   static constexpr uint32_t Q_LBO = 128, Q_SBO = 16 * D;
-  // TMEM: two S / P buffers of 64 columns, then O (D columns)
-  static constexpr int COL_S = 0, COL_O = 128, TMEM_COLS = 256;
+  // TMEM: three S / P buffers of 64 columns, then O (D columns)
+  static constexpr int NSB = 3;                                  // S / P buffers in TMEM
+  static constexpr int COL_S = 0, COL_O = 64 * NSB, TMEM_COLS = 512;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_RK = 0;                               // [NST][8 pages]
   static constexpr int OFF_RV = OFF_RK + NST * 8 * PAGE;
@@ -78,10 +86,10 @@ struct PfCfg {
   static constexpr int OFF_C = (OFF_RVM + NST * 8 * (METAB > 0 ? METAB : 16) + 127) / 128 * 128;
   static constexpr int OFF_Q = OFF_C + NCS * CSTAGE;             // [QP]
   static constexpr int OFF_BAR = OFF_Q + QP * QBYTES;
-  static constexpr int NBAR = 2 * NST + 4 * 2 + 2 + 2 + 1;       // rfull/rfree, cfull/sfull/pready/pvdone, q, ofree, drain
-  static constexpr int OFF_MASK = (OFF_BAR + 8 * NBAR + 15) / 16 * 16;   // uint32 [NST] raw, [2] conv
-  static constexpr int OFF_RED = (OFF_MASK + 4 * (NST + 2) + 15) / 16 * 16;   // long long [8] prologue
-  static constexpr int OFF_MISC = OFF_RED + 64;                  // tmem base, abort flag, start (b, P)
+  static constexpr int NBAR = 2 * NST + 2 * NCB + 3 * NSB + 3;  // rfull/rfree, cfull/cfree, sfull/pready/pvdone, q, ofree, drain
+  static constexpr int OFF_MASK = (OFF_BAR + 8 * NBAR + 15) / 16 * 16;   // uint32 [NST] raw, [NCB] conv
+  static constexpr int OFF_RED = (OFF_MASK + 4 * (NST + NCB) + 15) / 16 * 16;   // long long [8] prologue
+  static constexpr int OFF_MISC = OFF_RED + 128;                 // tmem base, abort flag, start (b, P)
   static constexpr int SMEM = OFF_MISC + 32 + 1024;              // + alignment slack
   static_assert(OFF_RKM % 16 == 0 && OFF_C % 128 == 0 && OFF_Q % 128 == 0 && OFF_BAR % 8 == 0,
                 "smem alignment");
@@ -114,12 +122,12 @@ __device__ __forceinline__ void s8x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t
   hi = *reinterpret_cast<const uint32_t*>(&h1);
 }
 
-// A packed f16x2 word -> the same two values as bf16x2 (exact for the values
-// of 8-bit codes, which need at most 8 significant bits).
-__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
-  const __half2 hv = *reinterpret_cast<const __half2*>(&h);
-  const __nv_bfloat162 b = __floats2bfloat162_rn(__low2float(hv), __high2float(hv));
-  return *reinterpret_cast<const uint32_t*>(&b);
+// 2^x by the hardware approximation (relative error about 2^-22; results below
+// 2^-126 flush to 0, 2^-inf = 0).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // 16 codes (one 16-byte chunk) -> 16 f16 values (32 bytes), little-endian.
@@ -146,7 +154,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, float up)
 }
 
 template <int D, int FMT>
-__global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
+__global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kc,
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
@@ -158,7 +166,7 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NWARPS = 8;
+  constexpr int NWARPS = 10;
   const int R = G * nq;                                    // query rows of a KV head
   const int rb = int(blockIdx.x % nrb);                    // this CTA's row block
   const long long grp = blockIdx.x / nrb, NG = gridDim.x / nrb;
@@ -172,15 +180,16 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* rfull = bars;                   // [NST] producer -> converters / MMA
   uint64_t* rfree = bars + C::NST;          // [NST]
-  uint64_t* cfull = bars + 2 * C::NST;      // [2] converters -> MMA, softmax
-  uint64_t* sfull = cfull + 2;              // [2] S of a half tile in TMEM
-  uint64_t* pready = sfull + 2;             // [2] P' of a half tile in TMEM
-  uint64_t* pvdone = pready + 2;            // [2] PV of a half tile complete
-  uint64_t* qready = pvdone + 2;            // the query operand of the next piece
+  uint64_t* cfull = bars + 2 * C::NST;      // [NCB] converters -> MMA, softmax
+  uint64_t* cfree = cfull + C::NCB;         // [NCB] a converted stage's PV product has completed
+  uint64_t* sfull = cfree + C::NCB;         // [NSB] S of a half tile in TMEM
+  uint64_t* pready = sfull + C::NSB;        // [NSB] P' of a half tile in TMEM
+  uint64_t* pvdone = pready + C::NSB;       // [NSB] PV of a half tile complete
+  uint64_t* qready = pvdone + C::NSB;       // the query operand of the next piece
   uint64_t* ofree = qready + 1;             // O of the last piece read
   uint64_t* drain = ofree + 1;
   volatile uint32_t* rmask = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MASK);   // [NST]
-  volatile uint32_t* cmask = rmask + C::NST;                                            // [2]
+  volatile uint32_t* cmask = rmask + C::NST;                                            // [NCB]
   long long* red64 = reinterpret_cast<long long*>(smem + C::OFF_RED);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -191,10 +200,13 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(rfull + s, 1);
-      mbar_init(rfree + s, C::BF ? 1 : 64);
+      mbar_init(rfree + s, C::BF ? 1 : 128);
     }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(cfull + j, 64);
+    for (int j = 0; j < C::NCB; ++j) {
+      mbar_init(cfull + j, 128);
+      mbar_init(cfree + j, 1);
+    }
+    for (int j = 0; j < C::NSB; ++j) {
       mbar_init(sfull + j, 1);
       mbar_init(pready + j, 128);
       mbar_init(pvdone + j, 1);
@@ -369,7 +381,7 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
     }
   } else if (warp >= 6) {
     // ---------------------------------------------------------- converters
-    const int ct = threadIdx.x - 192;                      // 0..63
+    const int ct = threadIdx.x - 192;                      // 0..127
     const float c0 = qk_scale;                             // sm_scale * log2(e): base-2 scores
     bool ok = true;
     int gt = 0, u = 0;
@@ -379,10 +391,10 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
         if (ok) ok = mbar_wait(rfull + s, (gt / C::NST) & 1, abort_flag, wait_limit);
         const uint32_t pm = rmask[s];
         for (int hh = 0; hh < 2; ++hh, ++u) {
-          const int cs = u & 1;
-          // the stage (and its page mask) of half u - 2 is free once that
+          const int cs = u % C::NCB;
+          // the stage (and its page mask) of half u - NCB is free once that
           // half's PV product has completed
-          if (ok && u >= 2) ok = mbar_wait(pvdone + cs, ((u - 2) >> 1) & 1, abort_flag, wait_limit);
+          if (ok && u >= C::NCB) ok = mbar_wait(cfree + cs, (u / C::NCB - 1) & 1, abort_flag, wait_limit);
           const int tok0 = i * 128 + hh * 64;              // first token of the half
           // tokens of page p of the half that hold cache entries (0 for an
           // invalid page)
@@ -397,7 +409,7 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
                 const int nv = nvalid(p);
                 if (nv == 16) continue;                    // uniform
                 uint8_t* pg = rv + (s * 8 + 4 * hh + p) * C::PAGE;
-                for (int x = ct; x < 2 * D; x += 64) {
+                for (int x = ct; x < 2 * D; x += 128) {
                   const int uu = x / D;                    // tokens 8 uu .. 8 uu + 7
                   uint4* ch = reinterpret_cast<uint4*>(pg + x * 16);
                   const int keep = max(0, min(8, nv - 8 * uu));
@@ -416,36 +428,55 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
               uint8_t* ck = cb;
               uint8_t* cv = cb + 4 * C::CPAGE;
               float* cm = reinterpret_cast<float*>(cb + 8 * C::CPAGE);
-              // K: raw 16-byte chunk k of a page holds 16 channels of one token
-              for (int x = ct; x < 4 * D; x += 64) {
+              // every raw chunk of the half is loaded before any converted one is
+              // stored (the stores could alias the loads as far as the compiler
+              // knows, which would serialize them)
+              constexpr int NIT = 4 * D / 128;
+              const uint8_t* rkh = rk + (s * 8 + 4 * hh) * C::PAGE;
+              const uint8_t* rvh = rv + (s * 8 + 4 * hh) * C::PAGE;
+              uint4 kraw[NIT], vraw[NIT];
+#pragma unroll
+              for (int it = 0; it < NIT; ++it) {
+                // K: raw 16-byte chunk k of a page holds 16 channels of one token;
+                // V: raw chunk d holds 16 tokens of channel d (in page units the
+                // two are the same byte offset)
+                const int x = ct + 128 * it;
+                kraw[it] = *reinterpret_cast<const uint4*>(rkh + (x / D) * C::PAGE + (x % D) * 16);
+                vraw[it] = *reinterpret_cast<const uint4*>(rvh + (x / D) * C::PAGE + (x % D) * 16);
+              }
+#pragma unroll
+              for (int it = 0; it < NIT; ++it) {
+                const int x = ct + 128 * it;
                 const int p = x / D, k = x % D;
                 const int g = k / (D / 2), rem = k % (D / 2), c = rem >> 3, tt = rem & 7;
-                const uint4 raw = *reinterpret_cast<const uint4*>(rk + (s * 8 + 4 * hh + p) * C::PAGE + k * 16);
                 uint4 o0, o1;
-                codes16_to_f16<FMT>(raw, o0, o1);
+                codes16_to_f16<FMT>(kraw[it], o0, o1);
                 uint8_t* dst = ck + p * C::CPAGE + g * 16 * D + (2 * c) * 128 + tt * 16;
                 *reinterpret_cast<uint4*>(dst) = o0;
                 *reinterpret_cast<uint4*>(dst + 128) = o1;
               }
-              // V: raw chunk d of a page holds 16 tokens of channel d
-              for (int x = ct; x < 4 * D; x += 64) {
+              // V (64 | D: the page, hence nv, is the same for every thread of a
+              // warp)
+#pragma unroll
+              for (int it = 0; it < NIT; ++it) {
+                const int x = ct + 128 * it;
                 const int p = x / D, d = x % D;
                 const int nv = nvalid(p);
-                const uint4 raw = *reinterpret_cast<const uint4*>(rv + (s * 8 + 4 * hh + p) * C::PAGE + d * 16);
                 uint4 o0, o1;
-                codes16_to_f16<FMT>(raw, o0, o1);
+                codes16_to_f16<FMT>(vraw[it], o0, o1);
                 uint32_t w[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+                if (nv < 16) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const uint32_t m = (2 * e < nv ? 0x0000FFFFu : 0u) | (2 * e + 1 < nv ? 0xFFFF0000u : 0u);
-                  w[e] = f16x2_to_bf16x2(w[e]) & m;
+                  for (int e = 0; e < 8; ++e)
+                    w[e] &= (2 * e < nv ? 0x0000FFFFu : 0u) | (2 * e + 1 < nv ? 0xFFFF0000u : 0u);
                 }
                 uint8_t* pg = cv + p * C::CPAGE;
                 *reinterpret_cast<uint4*>(pg + d * 16) = make_uint4(w[0], w[1], w[2], w[3]);
                 *reinterpret_cast<uint4*>(pg + (D + d) * 16) = make_uint4(w[4], w[5], w[6], w[7]);
               }
-              // per-token column factors: score = S a + b qsum, P' = p sv, V zero point zv
-              {
+              // per-token column factors: score = S a + b qsum, P' = p sv, V zero
+              // point zv (threads 0..63, one token each)
+              if (ct < C::HT) {
                 const int p = ct >> 4, tk = ct & 15;
                 const bool tv = tk < nvalid(p);
                 float a = 0.f, b = 0.f, sv = 0.f, zv = 0.f;
@@ -471,6 +502,8 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
                 cm[C::HT + ct] = b;
                 cm[2 * C::HT + ct] = sv;
                 cm[3 * C::HT + ct] = zv;
+                const float svw = warp_max(sv);              // V scales are >= 0
+                if ((ct & 31) == 0) cm[4 * C::HT + (ct >> 5)] = svw;
               }
             }
             fence_proxy_async_smem();
@@ -485,7 +518,7 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f16(C::HT, C::BF);   // Q x K^T: f16 (bf16 for a BF16 cache)
-      constexpr uint32_t id_pv = idesc_f16(D, true);        // P' x V: bf16
+      constexpr uint32_t id_pv = idesc_f16(D, C::BF);       // P' x V: f16 (bf16 for a BF16 cache)
       const uint32_t qaddr = smem_u32(qop), rkaddr = smem_u32(rk), rvaddr = smem_u32(rv);
       const uint32_t caddr = smem_u32(cst);
       bool ok = true;
@@ -494,14 +527,14 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
       int pend = -1, pend_s = 0, pend_hh = 0, pend_pc = 0;
       bool pend_first = false;
       auto issue_pv = [&]() -> bool {
-        const int cs = pend & 1;
-        if (!mbar_wait(pready + cs, (pend >> 1) & 1, abort_flag, wait_limit)) return false;
+        const int cs = pend % C::NSB, ck = pend % C::NCB;
+        if (!mbar_wait(pready + cs, (pend / C::NSB) & 1, abort_flag, wait_limit)) return false;
         // a piece's first product overwrites O: the softmax warps have read the last piece's
         if (pend_first && pend_pc > 0 && !mbar_wait(ofree, (pend_pc - 1) & 1, abort_flag, wait_limit))
           return false;
         tc_fence_after();
         const uint32_t vb = C::BF ? rvaddr + (pend_s * 8 + 4 * pend_hh) * C::PAGE
-                                  : caddr + cs * C::CSTAGE + 4 * C::CPAGE;
+                                  : caddr + ck * C::CSTAGE + 4 * C::CPAGE;
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -510,6 +543,7 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
                        sdesc_plain(vb + kk * C::CPAGE, C::V_LBO, C::V_SBO), id_pv,
                        (pend_first && j == 0 && kk == 0) ? 0u : 1u);
         mma_commit(pvdone + cs);
+        mma_commit(cfree + ck);
         if (C::BF && pend_hh == 1) mma_commit(rfree + pend_s);    // the raw stage is consumed
         return true;
       };
@@ -520,14 +554,14 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
         for (int i = pw.lo; ok && i < pw.hi; ++i, ++gt) {
           const int s = gt % C::NST;
           for (int hh = 0; hh < 2; ++hh, ++u) {
-            const int cs = u & 1;
+            const int cs = u % C::NSB, ck = u % C::NCB;
             // the half's K operand is ready; its S / P columns are free once the
-            // PV product of half u - 2 has completed
-            ok = mbar_wait(cfull + cs, (u >> 1) & 1, abort_flag, wait_limit) &&
-                 (u < 2 || mbar_wait(pvdone + cs, ((u - 2) >> 1) & 1, abort_flag, wait_limit));
+            // PV product of half u - NSB has completed
+            ok = mbar_wait(cfull + ck, (u / C::NCB) & 1, abort_flag, wait_limit) &&
+                 (u < C::NSB || mbar_wait(pvdone + cs, (u / C::NSB - 1) & 1, abort_flag, wait_limit));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t kb = C::BF ? rkaddr + (s * 8 + 4 * hh) * C::PAGE : caddr + cs * C::CSTAGE;
+            const uint32_t kb = C::BF ? rkaddr + (s * 8 + 4 * hh) * C::PAGE : caddr + ck * C::CSTAGE;
 #pragma unroll
             for (int qp = 0; qp < C::QP; ++qp)
 #pragma unroll
@@ -570,6 +604,26 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
       ok = __all_sync(0xffffffffu, ok);
     };
 
+    // a pair of P' parts in the PV product's operand type
+    struct P16 {
+      uint32_t bits;
+      __device__ __forceinline__ static P16 make(float a, float b) {
+        P16 r;
+        if constexpr (C::BF) {
+          const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+          r.bits = *reinterpret_cast<const uint32_t*>(&v);
+        } else {
+          const __half2 v = __floats2half2_rn(a, b);
+          r.bits = *reinterpret_cast<const uint32_t*>(&v);
+        }
+        return r;
+      }
+      __device__ __forceinline__ float2 f2() const {
+        if constexpr (C::BF) return make_float2(bf16_lo(bits), bf16_hi(bits));
+        const __half2 v = *reinterpret_cast<const __half2*>(&bits);
+        return __half22float2(v);
+      }
+    };
     // the query row of a piece as BF16 pairs (loaded when its operand is built:
     // once per piece, and a piece spans many tiles)
     uint32_t qw[D / 2];
@@ -654,9 +708,9 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
       float m_run = -INFINITY, l = 0.f, corr = 0.f;
       for (int i = pw.lo; i < pw.hi; ++i) {
         for (int hh = 0; hh < 2; ++hh, ++u) {
-          const int cs = u & 1;
-          wait_all(cfull + cs, (u >> 1) & 1);
-          wait_all(sfull + cs, (u >> 1) & 1);
+          const int cs = u % C::NSB, ck = u % C::NCB;      // TMEM buffer, converted stage
+          wait_all(cfull + ck, (u / C::NCB) & 1);
+          wait_all(sfull + cs, (u / C::NSB) & 1);
           tc_fence_after();
           if (i == pw.hi - 1 && hh == 1 && !nxt.done) {
             // every S product of this piece has completed: the next piece's
@@ -676,31 +730,49 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
 #pragma unroll
             for (int c = 0; c < C::HT; ++c) sr[c] = 0u;
           }
-          const float* cm = reinterpret_cast<const float*>(cst + cs * C::CSTAGE + 8 * C::CPAGE);
-          const uint32_t pmh = cmask[cs];
+          const float* cm = reinterpret_cast<const float*>(cst + ck * C::CSTAGE + 8 * C::CPAGE);
+          const uint32_t pmh = cmask[ck];
           const int t0 = i * 128 + hh * 64;
-          // scores in the operand's units (xs * down is the base-2 score)
-          float* xs = reinterpret_cast<float*>(sr);         // the scores replace S
-          float mt = -INFINITY;
+          // scores in the operand's units (x * down is the base-2 score), two
+          // columns per instruction, in place of S; columns are masked only in
+          // the halves where some row of the warp needs it
+          const bool full = __all_sync(0xffffffffu, t0 + C::HT <= lim && pmh == 0xFu);
+          float2* x2 = reinterpret_cast<float2*>(sr);
+          const float2* a2 = reinterpret_cast<const float2*>(cm);
+          const float2* b2 = reinterpret_cast<const float2*>(cm + C::HT);
+          const float2 qs2 = make_float2(qsum, qsum), k2 = make_float2(qk_scale, qk_scale);
+          float2 mx = make_float2(-INFINITY, -INFINITY);
 #pragma unroll
-          for (int c = 0; c < C::HT; ++c) {
-            const bool v = (t0 + c < lim) && ((pmh >> (c >> 4)) & 1u);
-            const float sv_ = __uint_as_float(sr[c]);
-            float x;
-            if constexpr (C::BF) x = sv_ * qk_scale;
-            else if constexpr (C::ZP) x = fmaf(sv_, cm[c], cm[C::HT + c] * qsum);
-            else x = sv_ * cm[c];
-            xs[c] = v ? x : -INFINITY;
-            mt = fmaxf(mt, xs[c]);
+          for (int k = 0; k < C::HT / 2; ++k) {
+            const float2 sv_ = make_float2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]));
+            float2 x;
+            if constexpr (C::BF) x = __fmul2_rn(sv_, k2);
+            else if constexpr (C::ZP) x = __ffma2_rn(sv_, a2[k], __fmul2_rn(b2[k], qs2));
+            else x = __fmul2_rn(sv_, a2[k]);
+            if (!full) {
+              const int c = 2 * k;
+              const bool pg = ((pmh >> (c >> 4)) & 1u) != 0u;
+              if (!(pg && t0 + c < lim)) x.x = -INFINITY;
+              if (!(pg && t0 + c + 1 < lim)) x.y = -INFINITY;
+            }
+            x2[k] = x;
+            mx.x = fmaxf(mx.x, x.x);
+            mx.y = fmaxf(mx.y, x.y);
           }
+          float mt = fmaxf(mx.x, mx.y);
           mt *= down;
-          // O holds the products of every earlier half of this piece
-          if (u >= 1) wait_all(pvdone + ((u - 1) & 1), ((u - 1) >> 1) & 1);
-          tc_fence_after();
-          // lazy rescaling: the reference max moves only when a score exceeds
-          // it by more than 8 (weights stay below 2^8); O (this piece's earlier
-          // halves, all complete) is rescaled in TMEM by the whole warp, with
-          // factor 1 for rows that keep their max
+          // the largest weight of the half is at most 2^(mt - m_run) * svmax: the
+          // reference moves with log2(svmax) too, so that P' stays below 2^8 and
+          // its f16 parts keep their precision whatever the V scales are (a
+          // zero largest scale counts as 2^-64: its tokens still count in l)
+          if constexpr (C::F8 || C::ZP) {
+            const float svm = fmaxf(cm[4 * C::HT], cm[4 * C::HT + 1]);
+            mt += svm > 0.f ? fmaxf(__log2f(svm), -64.f) : -64.f;
+          }
+          // lazy rescaling: the reference moves only when the largest weight
+          // would exceed 2^8 relative to it; O (this piece's earlier halves:
+          // their PV products are waited for only then) is rescaled in TMEM by
+          // the whole warp, with factor 1 for rows that keep their reference
           float alpha = 1.f;
           if (mt > m_run + 8.f) {
             if (m_run != -INFINITY) {
@@ -709,6 +781,10 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
               corr *= alpha;
             }
             m_run = mt;
+          }
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            if (u >= 1) wait_all(pvdone + ((u - 1) % C::NSB), ((u - 1) / C::NSB) & 1);
+            tc_fence_after();
           }
           if (ok && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
@@ -722,34 +798,40 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
             }
             tmem_st_wait();
           }
-          // P' = p * v_scale as two bf16 parts (16 bits), token pairs per word,
-          // written to TMEM 32 tokens at a time
+          // P' = p * v_scale as two 16-bit parts, token pairs per word, written
+          // to TMEM 32 tokens at a time
           const bool any = m_run != -INFINITY;
-          float ls = 0.f, cz = 0.f;
+          const float2 dn2 = make_float2(down, down), nm2 = make_float2(-m_run, -m_run);
+          const float2 m1 = make_float2(-1.f, -1.f);
+          const float2* sv2 = reinterpret_cast<const float2*>(cm + 2 * C::HT);
+          const float2* zv2 = reinterpret_cast<const float2*>(cm + 3 * C::HT);
+          float2 ls2 = make_float2(0.f, 0.f), cz2 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int h2 = 0; h2 < C::HT / 32; ++h2) {
             uint32_t ph[16], pl[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-              const int c = 32 * h2 + 2 * k;
-              const float p0 = any ? exp2f(fmaf(xs[c], down, -m_run)) : 0.f;
-              const float p1 = any ? exp2f(fmaf(xs[c + 1], down, -m_run)) : 0.f;
-              ls += p0 + p1;
-              float w0 = p0, w1 = p1;
-              if constexpr (C::F8 || C::ZP) { w0 *= cm[2 * C::HT + c]; w1 *= cm[2 * C::HT + c + 1]; }
-              const __nv_bfloat162 h2v = __floats2bfloat162_rn(w0, w1);
-              const __nv_bfloat162 l2v = __floats2bfloat162_rn(w0 - __low2float(h2v), w1 - __high2float(h2v));
-              ph[k] = *reinterpret_cast<const uint32_t*>(&h2v);
-              pl[k] = *reinterpret_cast<const uint32_t*>(&l2v);
+              const int kk = 16 * h2 + k;                   // column pair
+              const float2 e = __ffma2_rn(x2[kk], dn2, nm2);
+              const float2 p2 = any ? make_float2(ex2_ftz(e.x), ex2_ftz(e.y)) : make_float2(0.f, 0.f);
+              ls2 = __fadd2_rn(ls2, p2);
+              float2 w = p2;
+              if constexpr (C::F8 || C::ZP) w = __fmul2_rn(p2, sv2[kk]);
+              P16 hv = P16::make(w.x, w.y);
+              const float2 hf = hv.f2();
+              const float2 rr = __ffma2_rn(hf, m1, w);      // w - hi, exact
+              P16 lv = P16::make(rr.x, rr.y);
+              ph[k] = hv.bits;
+              pl[k] = lv.bits;
               if constexpr (C::ZP)
-                cz += (__low2float(h2v) + __low2float(l2v)) * cm[3 * C::HT + c] +
-                      (__high2float(h2v) + __high2float(l2v)) * cm[3 * C::HT + c + 1];
+                cz2 = __ffma2_rn(__fadd2_rn(hf, lv.f2()), zv2[kk], cz2);
             }
             if (ok) {
               tmem_st16(tmem + lane_base + C::COL_S + cs * 64 + 16 * h2, ph);
               tmem_st16(tmem + lane_base + C::COL_S + cs * 64 + 32 + 16 * h2, pl);
             }
           }
+          const float ls = ls2.x + ls2.y, cz = cz2.x + cz2.y;
           l += ls;
           corr += cz;
           if (ok) tmem_st_wait();
@@ -759,7 +841,7 @@ __global__ void __launch_bounds__(256, 1) prefill_mma_kernel(
       }
 
       // ---- piece partial: O of the last half, less the V zero-point term
-      wait_all(pvdone + ((u - 1) & 1), ((u - 1) >> 1) & 1);
+      wait_all(pvdone + ((u - 1) % C::NSB), ((u - 1) / C::NSB) & 1);
       tc_fence_after();
       const bool good = __all_sync(0xffffffffu, ok && !*abort_flag);
       const int64_t grow = (int64_t(pw.b) * Hk + pw.h) * R + rho;   // output row
