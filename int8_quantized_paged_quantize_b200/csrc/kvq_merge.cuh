@@ -10,8 +10,7 @@ namespace kvq {
 // partials (m_i, l_i, o_i) as m = max m_i, l = sum l_i 2^(m_i - m),
 // o = sum o_i 2^(m_i - m) / l. Lane i holds slot i's (m, l) (32 slots at a
 // time); each lane owns D/32 consecutive channels and reads them as one vector
-// per slot, so a row's partials stream in with every load in flight. The sums
-// run over the slots in order, as a single thread per channel would.
+// per slot, so a row's partials stream in with every load in flight.
 template <int D>
 struct MergeVec {
   static constexpr int N = D / 32;
@@ -35,43 +34,72 @@ __global__ void __launch_bounds__(128) merge_kernel(const int32_t* __restrict__ 
                                                     const int32_t* __restrict__ part_cnt,
                                                     OutT* __restrict__ out, int rows) {
   constexpr int N = D / 32;
+  constexpr int PRE = 8;                                   // slots whose vectors load up front
   const int lane = threadIdx.x & 31;
   const int bq = blockIdx.x * 4 + (threadIdx.x >> 5);      // b * Hq + row
   tc::grid_dep_wait();                                     // the partials are complete
   if (bq >= rows) return;
   const int b = bq / Hq;
-  int ctx = ctx_lens[b];
+  const int64_t r0 = int64_t(bq) * slots;
+  // The length, the count, the first 32 slots' (m, l) and the first PRE slots'
+  // vectors are requested together, before the count is known (every slot
+  // index below `slots` lies inside the workspace; values of slots past the
+  // count are never used), so a row costs one round trip to memory.
+  const int ctx_raw = ctx_lens[b];
+  const int cnt_raw = part_cnt[bq / G];
+  float2 ml = make_float2(-INFINITY, 0.f);
+  if (lane < slots) ml = *reinterpret_cast<const float2*>(part_ml + (r0 + lane) * 2);
+  MergeVec<D> x[PRE];
+#pragma unroll
+  for (int j = 0; j < PRE; ++j)
+    if (j < slots) x[j].load(part_o + (r0 + j) * D + lane * N);
+  int ctx = ctx_raw;
   if (ctx < 0 || ctx > max_ctx || int64_t(ctx) > int64_t(W) * kBlockSize) ctx = 0;
   // partials written for this (sequence, row group) by the decode kernel
-  const int n = ctx > 0 ? min(slots, max(0, part_cnt[bq / G])) : 0;
-  const int64_t r0 = int64_t(bq) * slots;
-  float M = -INFINITY;
-  for (int s0 = 0; s0 < n; s0 += 32)
+  const int n = ctx > 0 ? min(slots, max(0, cnt_raw)) : 0;
+  if (lane >= n) ml = make_float2(-INFINITY, 0.f);
+  float M = ml.x;
+  for (int s0 = 32; s0 < n; s0 += 32)
     if (s0 + lane < n) M = fmaxf(M, part_ml[(r0 + s0 + lane) * 2]);
   M = warp_max(M);
   float o[N], l = 0.f;
 #pragma unroll
   for (int i = 0; i < N; ++i) o[i] = 0.f;
   if (M != -INFINITY) {
+    // the sums run over the slots in order, as a single thread per channel would
+    const float fl0 = exp2f(ml.x - M);
+#pragma unroll
+    for (int j = 0; j < PRE; ++j) {
+      if (j >= n) break;
+      const float f = __shfl_sync(0xffffffffu, fl0, j);
+      const float ls = __shfl_sync(0xffffffffu, ml.y, j);
+      l += ls * f;
+#pragma unroll
+      for (int i = 0; i < N; ++i) o[i] += x[j].v[i] * f;
+    }
     for (int s0 = 0; s0 < n; s0 += 32) {
-      float2 ml = make_float2(-INFINITY, 0.f);
-      if (s0 + lane < n) ml = *reinterpret_cast<const float2*>(part_ml + (r0 + s0 + lane) * 2);
-      const float fl = exp2f(ml.x - M);
+      float2 mls = ml;
+      float fl = fl0;
+      if (s0 > 0) {
+        mls = make_float2(-INFINITY, 0.f);
+        if (s0 + lane < n) mls = *reinterpret_cast<const float2*>(part_ml + (r0 + s0 + lane) * 2);
+        fl = exp2f(mls.x - M);
+      }
       const int cnt = min(32, n - s0);
-      // eight slots' vectors are requested before any is summed
-      for (int s8 = 0; s8 < cnt; s8 += 8) {
-        MergeVec<D> x[8];
+      // slots past the first PRE: eight slots' vectors are requested before any is summed
+      for (int s8 = (s0 == 0 ? PRE : 0); s8 < cnt; s8 += 8) {
+        MergeVec<D> y[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (s8 + j < cnt) x[j].load(part_o + (r0 + s0 + s8 + j) * D + lane * N);
+          if (s8 + j < cnt) y[j].load(part_o + (r0 + s0 + s8 + j) * D + lane * N);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (s8 + j >= cnt) break;
           const float f = __shfl_sync(0xffffffffu, fl, s8 + j);
-          const float ls = __shfl_sync(0xffffffffu, ml.y, s8 + j);
+          const float ls = __shfl_sync(0xffffffffu, mls.y, s8 + j);
           l += ls * f;
 #pragma unroll
-          for (int i = 0; i < N; ++i) o[i] += x[j].v[i] * f;
+          for (int i = 0; i < N; ++i) o[i] += y[j].v[i] * f;
         }
       }
     }
