@@ -743,7 +743,7 @@ cudaError_t prefill_dispatch2(const void* q, int32_t B, const void* kc, const vo
   int32_t* pcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + plan.o_bytes + plan.ml_bytes);
   // one CTA per SM, in groups of nrb that walk the same share of the tile list
   const int64_t grid = std::max<int64_t>(1, int64_t(device_sm_count()) / nrb) * nrb;
-  e = launch_pdl(kern, dim3(unsigned(grid)), dim3(320), C::SMEM, st,
+  e = launch_pdl(kern, dim3(unsigned(grid)), dim3(448), C::SMEM, st,
       static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(kc),
       static_cast<const uint8_t*>(vc), static_cast<const __nv_bfloat16*>(ks),
       static_cast<const __nv_bfloat16*>(vs), tables, ctx, B, d.n_kv_heads, G, n_query, nrb,

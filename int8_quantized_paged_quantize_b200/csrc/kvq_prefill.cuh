@@ -30,14 +30,16 @@
 // for the others. Each piece ends in an online-softmax partial per row, and
 // the merge kernel combines a row's partials (one count per row).
 //
-// 10 warps per CTA:
+// 14 warps per CTA:
 //   warp 0      producer: lanes 0..7 copy one K and one V page each of a tile
 //               (1-D bulk copies) into a ring of raw stages and store the
 //               pages' scales beside them.
 //   warp 1      allocates TMEM; one thread issues the MMAs.
-//   warps 2..5  softmax warps, one per TMEM lane quarter: thread r owns query
-//               row r (S, P and O lane r); they also build the query operand.
-//   warps 6..9  converters: expand each half tile's K and V codes to f16 in a
+//   warps 2..9  softmax warps, two per TMEM lane quarter: thread r of a warp
+//               owns query row r (TMEM lane r) for one half of a half tile's
+//               columns (and of O's); the two exchange their row maxima and
+//               sums through shared memory. They also build the query operand.
+//   warps 10..13 converters: expand each half tile's K and V codes to f16 in a
 //               converted stage, with V rows of tokens past the
 //               sequence end or on invalid pages zeroed, and turn the
 //               per-token scales into FP32 column factors. For a BF16 cache
@@ -85,7 +87,8 @@ struct PfCfg {
   static constexpr int OFF_RVM = OFF_RKM + NST * 8 * (METAB > 0 ? METAB : 16);
   static constexpr int OFF_C = (OFF_RVM + NST * 8 * (METAB > 0 ? METAB : 16) + 127) / 128 * 128;
   static constexpr int OFF_Q = OFF_C + NCS * CSTAGE;             // [QP]
-  static constexpr int OFF_BAR = OFF_Q + QP * QBYTES;
+  static constexpr int OFF_XCH = OFF_Q + QP * QBYTES;            // float [2][2][128] maxima, [2][128][2] sums
+  static constexpr int OFF_BAR = OFF_XCH + (2 * 2 * 128 + 2 * 128 * 2) * 4;
   static constexpr int NBAR = 2 * NST + 2 * NCB + 3 * NSB + 3;  // rfull/rfree, cfull/cfree, sfull/pready/pvdone, q, ofree, drain
   static constexpr int OFF_MASK = (OFF_BAR + 8 * NBAR + 15) / 16 * 16;   // uint32 [NST] raw, [NCB] conv
   static constexpr int OFF_RED = (OFF_MASK + 4 * (NST + NCB) + 15) / 16 * 16;   // long long [8] prologue
@@ -154,7 +157,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, float up)
 }
 
 template <int D, int FMT>
-__global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
+__global__ void __launch_bounds__(448, 1) prefill_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ kc,
     const uint8_t* __restrict__ vc, const __nv_bfloat16* __restrict__ ks,
     const __nv_bfloat16* __restrict__ vs, const int32_t* __restrict__ tables,
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NWARPS = 10;
+  constexpr int NWARPS = 14;
   const int R = G * nq;                                    // query rows of a KV head
   const int rb = int(blockIdx.x % nrb);                    // this CTA's row block
   const long long grp = blockIdx.x / nrb, NG = gridDim.x / nrb;
@@ -208,11 +211,11 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
     }
     for (int j = 0; j < C::NSB; ++j) {
       mbar_init(sfull + j, 1);
-      mbar_init(pready + j, 128);
+      mbar_init(pready + j, 256);
       mbar_init(pvdone + j, 1);
     }
-    mbar_init(qready, 128);
-    mbar_init(ofree, 128);
+    mbar_init(qready, 256);
+    mbar_init(ofree, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -379,9 +382,9 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
       for (int s = 0; s < C::NST; ++s)
         if (iss[s]) mbar_wait(rfull + s, par[s], &no_abort, kMmaWaitLimitCycles);
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 10) {
     // ---------------------------------------------------------- converters
-    const int ct = threadIdx.x - 192;                      // 0..127
+    const int ct = threadIdx.x - 320;                      // 0..127
     const float c0 = qk_scale;                             // sm_scale * log2(e): base-2 scores
     bool ok = true;
     int gt = 0, u = 0;
@@ -592,7 +595,12 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
   } else {
     // ---------------------------------------------------------- softmax warps
     const int quarter = warp & 3;
+    const int set = (warp - 2) >> 2;                      // columns [32 set, 32 set + 32) of a half
     const int r = quarter * 32 + lane;                    // query row of the block, TMEM lane
+    constexpr int HC = C::HT / 2;                         // columns per thread and half
+    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XCH);          // [2][2][128]
+    float2* xsum = reinterpret_cast<float2*>(smem + C::OFF_XCH + 2 * 2 * 128 * 4);   // [2][128]
+    const int pair_bar = 2 + quarter;                     // the two warps of this lane quarter
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const int rho = rb * 128 + r;                         // row of the KV head: g * nq + j
     const bool row_ok = rho < R;
@@ -644,15 +652,19 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
     // write the row into the query operand (K-major 8-row groups of 16-byte
     // chunks); returns the factor that takes S back to the row's units and,
     // through qsum, the sum of the operand's values (the zero-point term)
+    // (both warp sets compute the row's factors; set 0 writes the operand)
     auto store_q = [&](int kvh, float& down, float& qsum) {
       down = 1.f;
       qsum = 0.f;
+      const bool wr = set == 0;
       uint8_t* row = qop + (r >> 3) * C::Q_SBO + (r & 7) * 16;
       if constexpr (C::BF) {
+        if (wr) {
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-          *reinterpret_cast<uint4*>(row + c * C::Q_LBO) =
-              make_uint4(qw[4 * c], qw[4 * c + 1], qw[4 * c + 2], qw[4 * c + 3]);
+          for (int c = 0; c < D / 8; ++c)
+            *reinterpret_cast<uint4*>(row + c * C::Q_LBO) =
+                make_uint4(qw[4 * c], qw[4 * c + 1], qw[4 * c + 2], qw[4 * c + 3]);
+        }
       } else {
         // x = q (static INT8: q times the K scale of the channel)
         auto xval = [&](int d) -> float {
@@ -683,9 +695,11 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
             }
             if constexpr (C::ZP) qsum += __low2float(h) + __high2float(h);
           }
-          *reinterpret_cast<uint4*>(row + c * C::Q_LBO) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          if constexpr (C::SI)
-            *reinterpret_cast<uint4*>(row + C::QBYTES + c * C::Q_LBO) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          if (wr) {
+            *reinterpret_cast<uint4*>(row + c * C::Q_LBO) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            if constexpr (C::SI)
+              *reinterpret_cast<uint4*>(row + C::QBYTES + c * C::Q_LBO) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
         }
       }
       fence_proxy_async_smem();
@@ -719,31 +733,31 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
             store_q(nxt.h, down_n, qsum_n);
             mbar_arrive(qready);
           }
-          uint32_t sr[C::HT];
+          uint32_t sr[HC];
           if (ok) {
 #pragma unroll
-            for (int c = 0; c < C::HT / 16; ++c)
-              tmem_ld16(tmem + lane_base + C::COL_S + cs * 64 + 16 * c,
+            for (int c = 0; c < HC / 16; ++c)
+              tmem_ld16(tmem + lane_base + C::COL_S + cs * 64 + HC * set + 16 * c,
                         *reinterpret_cast<uint32_t(*)[16]>(sr + 16 * c));
             tmem_ld_wait();
           } else {
 #pragma unroll
-            for (int c = 0; c < C::HT; ++c) sr[c] = 0u;
+            for (int c = 0; c < HC; ++c) sr[c] = 0u;
           }
           const float* cm = reinterpret_cast<const float*>(cst + ck * C::CSTAGE + 8 * C::CPAGE);
           const uint32_t pmh = cmask[ck];
-          const int t0 = i * 128 + hh * 64;
+          const int t0 = i * 128 + hh * 64 + HC * set;    // first token of this thread's columns
           // scores in the operand's units (x * down is the base-2 score), two
           // columns per instruction, in place of S; columns are masked only in
           // the halves where some row of the warp needs it
-          const bool full = __all_sync(0xffffffffu, t0 + C::HT <= lim && pmh == 0xFu);
+          const bool full = __all_sync(0xffffffffu, t0 + HC <= lim && pmh == 0xFu);
           float2* x2 = reinterpret_cast<float2*>(sr);
-          const float2* a2 = reinterpret_cast<const float2*>(cm);
-          const float2* b2 = reinterpret_cast<const float2*>(cm + C::HT);
+          const float2* a2 = reinterpret_cast<const float2*>(cm + HC * set);
+          const float2* b2 = reinterpret_cast<const float2*>(cm + C::HT + HC * set);
           const float2 qs2 = make_float2(qsum, qsum), k2 = make_float2(qk_scale, qk_scale);
           float2 mx = make_float2(-INFINITY, -INFINITY);
 #pragma unroll
-          for (int k = 0; k < C::HT / 2; ++k) {
+          for (int k = 0; k < HC / 2; ++k) {
             const float2 sv_ = make_float2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]));
             float2 x;
             if constexpr (C::BF) x = __fmul2_rn(sv_, k2);
@@ -751,7 +765,7 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
             else x = __fmul2_rn(sv_, a2[k]);
             if (!full) {
               const int c = 2 * k;
-              const bool pg = ((pmh >> (c >> 4)) & 1u) != 0u;
+              const bool pg = ((pmh >> ((HC * set + c) >> 4)) & 1u) != 0u;
               if (!(pg && t0 + c < lim)) x.x = -INFINITY;
               if (!(pg && t0 + c + 1 < lim)) x.y = -INFINITY;
             }
@@ -760,6 +774,10 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
             mx.y = fmaxf(mx.y, x.y);
           }
           float mt = fmaxf(mx.x, mx.y);
+          // the row maximum over both warps' columns (double-buffered by half)
+          xmax[((u & 1) * 2 + set) * 128 + r] = mt;
+          named_bar_sync(pair_bar, 64);
+          mt = fmaxf(mt, xmax[((u & 1) * 2 + (set ^ 1)) * 128 + r]);
           mt *= down;
           // the largest weight of the half is at most 2^(mt - m_run) * svmax: the
           // reference moves with log2(svmax) too, so that P' stays below 2^8 and
@@ -788,13 +806,14 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
           }
           if (ok && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-            for (int c = 0; c < D / 16; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
+              const uint32_t col = C::COL_O + (D / 2) * set + 16 * c;
               uint32_t ov[16];
-              tmem_ld16(tmem + lane_base + C::COL_O + 16 * c, ov);
+              tmem_ld16(tmem + lane_base + col, ov);
               tmem_ld_wait();
 #pragma unroll
               for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-              tmem_st16(tmem + lane_base + C::COL_O + 16 * c, ov);
+              tmem_st16(tmem + lane_base + col, ov);
             }
             tmem_st_wait();
           }
@@ -803,15 +822,14 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
           const bool any = m_run != -INFINITY;
           const float2 dn2 = make_float2(down, down), nm2 = make_float2(-m_run, -m_run);
           const float2 m1 = make_float2(-1.f, -1.f);
-          const float2* sv2 = reinterpret_cast<const float2*>(cm + 2 * C::HT);
-          const float2* zv2 = reinterpret_cast<const float2*>(cm + 3 * C::HT);
+          const float2* sv2 = reinterpret_cast<const float2*>(cm + 2 * C::HT + HC * set);
+          const float2* zv2 = reinterpret_cast<const float2*>(cm + 3 * C::HT + HC * set);
           float2 ls2 = make_float2(0.f, 0.f), cz2 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int h2 = 0; h2 < C::HT / 32; ++h2) {
+          {
             uint32_t ph[16], pl[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-              const int kk = 16 * h2 + k;                   // column pair
+              const int kk = k;                             // column pair of this thread
               const float2 e = __ffma2_rn(x2[kk], dn2, nm2);
               const float2 p2 = any ? make_float2(ex2_ftz(e.x), ex2_ftz(e.y)) : make_float2(0.f, 0.f);
               ls2 = __fadd2_rn(ls2, p2);
@@ -827,8 +845,8 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
                 cz2 = __ffma2_rn(__fadd2_rn(hf, lv.f2()), zv2[kk], cz2);
             }
             if (ok) {
-              tmem_st16(tmem + lane_base + C::COL_S + cs * 64 + 16 * h2, ph);
-              tmem_st16(tmem + lane_base + C::COL_S + cs * 64 + 32 + 16 * h2, pl);
+              tmem_st16(tmem + lane_base + C::COL_S + cs * 64 + 16 * set, ph);
+              tmem_st16(tmem + lane_base + C::COL_S + cs * 64 + 32 + 16 * set, pl);
             }
           }
           const float ls = ls2.x + ls2.y, cz = cz2.x + cz2.y;
@@ -844,13 +862,21 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
       wait_all(pvdone + ((u - 1) % C::NSB), ((u - 1) / C::NSB) & 1);
       tc_fence_after();
       const bool good = __all_sync(0xffffffffu, ok && !*abort_flag);
+      // the row's sums over both warps' columns
+      xsum[set * 128 + r] = make_float2(l, corr);
+      named_bar_sync(pair_bar, 64);
+      {
+        const float2 o2 = xsum[(set ^ 1) * 128 + r];
+        l += o2.x;
+        corr += o2.y;
+      }
       const int64_t grow = (int64_t(pw.b) * Hk + pw.h) * R + rho;   // output row
-      float* po = part_o + (grow * slots + slot) * D;
+      float* po = part_o + (grow * slots + slot) * D + (D / 2) * set;
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[16];
         if (good) {
-          tmem_ld16(tmem + lane_base + C::COL_O + 16 * c, ov);
+          tmem_ld16(tmem + lane_base + C::COL_O + (D / 2) * set + 16 * c, ov);
           tmem_ld_wait();
         }
         if (row_ok) {
@@ -859,7 +885,7 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
           for (int e = 0; e < 16; ++e) {
             float x = good ? __uint_as_float(ov[e]) - corr : __int_as_float(0x7fc00000);
             if constexpr (C::SI) {
-              if (good) x *= __bfloat162float(vs[per_tensor ? 0 : pw.h * D + 16 * c + e]);
+              if (good) x *= __bfloat162float(vs[per_tensor ? 0 : pw.h * D + (D / 2) * set + 16 * c + e]);
             }
             o[e] = x;
           }
@@ -868,7 +894,9 @@ __global__ void __launch_bounds__(320, 1) prefill_mma_kernel(
             *reinterpret_cast<float4*>(po + 16 * c + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         }
       }
-      if (row_ok) {
+      // the sums are read before the next piece overwrites them
+      named_bar_sync(pair_bar, 64);
+      if (row_ok && set == 0) {
         part_ml[(grow * slots + slot) * 2] = good ? m_run : INFINITY;
         part_ml[(grow * slots + slot) * 2 + 1] = good ? l : __int_as_float(0x7fc00000);
         if (last) part_cnt[grow] = slot + 1;
