@@ -69,7 +69,7 @@ struct PfCfg {
   // converted half-tile stages: three let the converters run two halves ahead
   // of the PV product (static INT8 keeps two: its query takes two operands)
   static constexpr int NCS = BF ? 0 : (SI ? 2 : 3);
-  static constexpr int NCB = BF ? 2 : NCS;                        // half-tile slots of the barriers
+  static constexpr int NCB = BF ? 3 : NCS;                        // half-tile slots of the barriers
   static constexpr int CMETA = 4 * HT * 4 + 128;                 // floats a, b, sv, zv per token; max sv
   static constexpr int CSTAGE = 8 * CPAGE + CMETA;               // K (4 pages), V (4 pages), meta
   // operand strides (bytes): K pages and the query are K-major with 8-row
