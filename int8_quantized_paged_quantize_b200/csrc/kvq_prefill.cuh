@@ -632,61 +632,55 @@ __global__ void __launch_bounds__(448, 1) prefill_mma_kernel(
         return __half22float2(v);
       }
     };
-    // the query row of a piece as BF16 pairs (loaded when its operand is built:
-    // once per piece, and a piece spans many tiles)
-    uint32_t qw[D / 2];
-    auto load_q = [&](const PieceWalk& pw) {
-      if (pw.done || !row_ok) {
-#pragma unroll
-        for (int i = 0; i < D / 2; ++i) qw[i] = 0u;
-        return;
-      }
-      const uint4* src = reinterpret_cast<const uint4*>(
-          q + ((int64_t(pw.b) * Hk + pw.h) * R + rho) * D);
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        const uint4 x = src[i];
-        qw[4 * i] = x.x; qw[4 * i + 1] = x.y; qw[4 * i + 2] = x.z; qw[4 * i + 3] = x.w;
-      }
-    };
-    // write the row into the query operand (K-major 8-row groups of 16-byte
-    // chunks); returns the factor that takes S back to the row's units and,
-    // through qsum, the sum of the operand's values (the zero-point term)
-    // (both warp sets compute the row's factors; set 0 writes the operand)
-    auto store_q = [&](int kvh, float& down, float& qsum) {
+    // The query row of a piece into the query operand (K-major 8-row groups of
+    // 16-byte chunks), once per piece (a piece spans many tiles): the row is
+    // streamed from global memory 8 channels at a time, twice (its largest
+    // element first), in rolled loops that keep the kernel's code small.
+    // Returns the factor that takes S back to the row's units and, through
+    // qsum, the sum of the operand's values (the zero-point term). Both warp
+    // sets compute the factors; set 0 writes the operand.
+    auto store_q = [&](const PieceWalk& pw, float& down, float& qsum) {
       down = 1.f;
       qsum = 0.f;
       const bool wr = set == 0;
+      const bool have = !pw.done && row_ok;
+      const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t(pw.b) * Hk + pw.h) * R + rho) * D);
       uint8_t* row = qop + (r >> 3) * C::Q_SBO + (r & 7) * 16;
+      auto chunk = [&](int c) -> uint4 { return have ? src[c] : make_uint4(0, 0, 0, 0); };
+      // x = q (static INT8: q times the K scale of the channel)
+      auto xval = [&](uint32_t w, int half, int d) -> float {
+        float x = half ? bf16_hi(w) : bf16_lo(w);
+        if constexpr (C::SI) x *= __bfloat162float(ks[per_tensor ? 0 : pw.h * D + d]);
+        return x;
+      };
       if constexpr (C::BF) {
         if (wr) {
-#pragma unroll
-          for (int c = 0; c < D / 8; ++c)
-            *reinterpret_cast<uint4*>(row + c * C::Q_LBO) =
-                make_uint4(qw[4 * c], qw[4 * c + 1], qw[4 * c + 2], qw[4 * c + 3]);
+#pragma unroll 2
+          for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4*>(row + c * C::Q_LBO) = chunk(c);
         }
       } else {
-        // x = q (static INT8: q times the K scale of the channel)
-        auto xval = [&](int d) -> float {
-          float x = (d & 1) ? bf16_hi(qw[d >> 1]) : bf16_lo(qw[d >> 1]);
-          if constexpr (C::SI) x *= __bfloat162float(ks[per_tensor ? 0 : kvh * D + d]);
-          return x;
-        };
         float amax = 0.f;
+#pragma unroll 2
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 u4 = chunk(c);
+          const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
-        for (int d = 0; d < D; ++d) amax = fmaxf(amax, fabsf(xval(d)));
+          for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(xval(w[k >> 1], k & 1, 8 * c + k)));
+        }
         // power-of-two scaling: the largest element lands in [2^14, 2^15)
         int e = 0;
         if (amax > 0.f) e = 14 - ilogbf(amax);
         e = max(-100, min(100, e));
         const float up = __int_as_float((127 + e) << 23);
         down = __int_as_float((127 - e) << 23);
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < D / 8; ++c) {
+          const uint4 u4 = chunk(c);
+          const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const float a = xval(8 * c + 2 * k) * up, b = xval(8 * c + 2 * k + 1) * up;
+            const float a = xval(w[k], 0, 8 * c + 2 * k) * up, b = xval(w[k], 1, 8 * c + 2 * k + 1) * up;
             const __half2 h = __floats2half2_rn(a, b);
             hi[k] = *reinterpret_cast<const uint32_t*>(&h);
             if constexpr (C::SI) {
@@ -706,8 +700,7 @@ __global__ void __launch_bounds__(448, 1) prefill_mma_kernel(
     };
 
     float down = 1.f, qsum = 0.f, down_n = 1.f, qsum_n = 0.f;
-    load_q(walk);
-    store_q(walk.h, down, qsum);
+    store_q(walk, down, qsum);
     mbar_arrive(qready);
 
     int u = 0;
@@ -729,8 +722,7 @@ __global__ void __launch_bounds__(448, 1) prefill_mma_kernel(
           if (i == pw.hi - 1 && hh == 1 && !nxt.done) {
             // every S product of this piece has completed: the next piece's
             // query may replace this one
-            load_q(nxt);
-            store_q(nxt.h, down_n, qsum_n);
+            store_q(nxt, down_n, qsum_n);
             mbar_arrive(qready);
           }
           uint32_t sr[HC];
@@ -805,7 +797,7 @@ __global__ void __launch_bounds__(448, 1) prefill_mma_kernel(
             tc_fence_after();
           }
           if (ok && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
               const uint32_t col = C::COL_O + (D / 2) * set + 16 * c;
               uint32_t ov[16];
@@ -872,7 +864,7 @@ __global__ void __launch_bounds__(448, 1) prefill_mma_kernel(
       }
       const int64_t grow = (int64_t(pw.b) * Hk + pw.h) * R + rho;   // output row
       float* po = part_o + (grow * slots + slot) * D + (D / 2) * set;
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[16];
         if (good) {
