@@ -532,24 +532,36 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
           zsum = fmaf(qcur[hh][i], zd[i], zsum);
           amax = fmaxf(amax, fabsf(x[i]));
         }
-        amax = warp_max(amax);
+        // the head's largest |x|: one integer reduction on the float bits (x >= 0)
+        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
         zsum = warp_sum(zsum);
         int e = 0;
         if (amax > 0.f) e = 5 - ilogbf(amax);
         e = max(-120, min(120, e));
         const float up = __int_as_float((127 + e) << 23);
         const float down = __int_as_float((127 - e) << 23);
-        uint32_t part[3] = {0u, 0u, 0u};
+        // the three parts by rounding additions (1.5 * 2^23 + v holds rint(v)
+        // in its low bits for |v| < 2^22): t_j's low byte is part j's code
+        constexpr float kMg = 12582912.0f;
+        uint32_t tb[3][CPL];
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
           const float xs = x[i] * up;
-          const float x0 = rintf(xs);
+          const float t0 = __fadd_rn(xs, kMg), x0 = __fsub_rn(t0, kMg);
           const float r0 = (xs - x0) * 128.f;
-          const float x1 = rintf(r0);
-          const float x2 = rintf((r0 - x1) * 128.f);
-          part[0] |= uint32_t(uint8_t(int8_t(int(x0)))) << (8 * i);
-          part[1] |= uint32_t(uint8_t(int8_t(int(x1)))) << (8 * i);
-          part[2] |= uint32_t(uint8_t(int8_t(int(x2)))) << (8 * i);
+          const float t1 = __fadd_rn(r0, kMg), x1 = __fsub_rn(t1, kMg);
+          const float t2 = __fadd_rn((r0 - x1) * 128.f, kMg);
+          tb[0][i] = __float_as_uint(t0);
+          tb[1][i] = __float_as_uint(t1);
+          tb[2][i] = __float_as_uint(t2);
+        }
+        uint32_t part[3];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          if constexpr (CPL == 4)
+            part[j] = __byte_perm(__byte_perm(tb[j][0], tb[j][1], 0x0040), __byte_perm(tb[j][2], tb[j][3], 0x0040), 0x5410);
+          else
+            part[j] = __byte_perm(tb[j][0], tb[j][1], 0x0040) & 0xFFFFu;
         }
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
