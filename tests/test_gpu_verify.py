@@ -34,7 +34,7 @@ pytestmark = pytest.mark.gpu
 CTX = [1, 2, 3, 15, 16, 17, 127, 128, 129, 300, 1000]
 
 
-def _run(fmt, D, G, nq, ctx=CTX, Hk=2, partition=0, seed=0, call="verify"):
+def _run(fmt, D, G, nq, ctx=CTX, Hk=2, partition=0, seed=0, call="verify", transform=None):
     w = W.Workload("synthetic", fmt, batch=len(ctx), n_q_heads=Hk * G, n_kv_heads=Hk, head_dim=D,
                    lengths="list", ctx=tuple(ctx), kv_mean=0.3 if fmt == "int8" else 0.0)
     tables, nb = W.block_tables(w, seed)
@@ -43,6 +43,8 @@ def _run(fmt, D, G, nq, ctx=CTX, Hk=2, partition=0, seed=0, call="verify"):
     d = kvq.dims(nb, Hk, Hk * G, D, tables.shape[1])
     K = torch.cat([h[0] for h in hist])
     V = torch.cat([h[1] for h in hist])
+    if transform is not None:
+        K, V = transform(K, V, lens)
     S = torch.cat([torch.from_numpy(GC.slots_for(tables, b, np.arange(lens[b]))) for b in range(w.batch)])
     static = {}
     if fmt in ("int8c", "int8t"):
@@ -187,3 +189,44 @@ def test_prefill_agrees_with_verify_on_the_same_positions():
     _check(e1)
     _check(e2)
     assert (o1 - o2).abs().max().item() <= 2e-3
+
+
+def _positions(lens):
+    """Each token's position inside its sequence, for the concatenated history."""
+    return torch.from_numpy(np.concatenate([np.arange(n) for n in lens]))
+
+
+def _check_scaled(err, ref):
+    """The attention tolerance relative to the outputs' magnitude."""
+    scale = max(1.0, float(np.abs(ref).max()))
+    assert err.max() <= GC.MAX_ABS * scale and err.mean() <= GC.MEAN_ABS * scale, (err.max(), scale)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "bf16"])
+def test_prefill_scores_that_grow_along_the_context(fmt):
+    """K grows 4x in the second half of every sequence, so the row maxima jump
+    by more than 2^8 after the first tiles: the prefill kernel's lazily moved
+    reference must rescale O in TMEM mid-piece (and more than once across the
+    split pieces of a long prefix)."""
+    def grow(K, V, lens):
+        pos = _positions(lens)
+        half = torch.from_numpy(np.concatenate([np.full(n, n // 2) for n in lens]))
+        f = torch.where(pos >= half, 4.0, 1.0).to(torch.float32)[:, None, None]
+        return (K.float() * f).to(torch.bfloat16), V
+    err, out, ref, lens = _run(fmt, 128, 4, 32, ctx=[600, 2500, 5000], partition=1024, call="prefill",
+                               transform=grow)
+    _check_scaled(err, ref)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+def test_prefill_v_scales_far_apart(fmt):
+    """V magnitudes that differ by 2^8 between the two halves of every sequence
+    (and so do the per-token V scales): the reference follows the half tiles'
+    largest V scale, so the f16 parts of P' neither overflow nor lose precision."""
+    def spread(K, V, lens):
+        pos = _positions(lens)
+        half = torch.from_numpy(np.concatenate([np.full(n, n // 2) for n in lens]))
+        f = torch.where(pos >= half, 16.0, 1.0 / 16.0).to(torch.float32)[:, None, None]
+        return K, (V.float() * f).to(torch.bfloat16)
+    err, out, ref, lens = _run(fmt, 128, 4, 32, ctx=[300, 2100, 4100], call="prefill", transform=spread)
+    _check_scaled(err, ref)
