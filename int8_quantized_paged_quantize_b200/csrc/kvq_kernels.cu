@@ -76,14 +76,18 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 namespace kvq {
 
 // ------------------------------------------------------------------ append
-// A (token, KV head) row of D BF16 values is quantized by one half warp: 16
-// lanes with E = D/16 consecutive values each (one 16-byte load at D = 128),
-// so a warp instruction serves two rows. The range is an integer max over the
-// half warp, the BF16 scale (+ zero point) is formed on each of its lanes, and
-// the lane's codes are packed little-endian in d order into `w`.
+// A (token, KV head) row of D BF16 values is quantized by a group of
+// kRowLanes = 8 lanes with E = D/8 consecutive values each (two 16-byte loads
+// at D = 128), so a warp instruction serves four rows and the per-row work
+// (range, scale, reciprocal, zero point) is shared by 16 values per lane. The
+// range is an integer max over the group, the BF16 scale (+ zero point) is
+// formed on each of its lanes, and the lane's codes are packed little-endian
+// in d order into `w`.
+constexpr int kRowLanes = 8;
+
 template <int D, int FMT>
 struct RowCodes {
-  static constexpr int E = D / 16;
+  static constexpr int E = D / kRowLanes;
   static constexpr int ELT = (FMT == KVQ_BF16) ? 2 : 1;
   static constexpr int WORDS = E * ELT / 4;
   uint32_t w[WORDS];
@@ -91,15 +95,13 @@ struct RowCodes {
   int zp;
 };
 
-// This lane's D/16 BF16 values of a row, as packed pairs.
+// This lane's D/8 BF16 values of a row, as packed pairs.
 template <int D>
-__device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint32_t (&raw)[D / 32]) {
-  if constexpr (D == 128) {
-    const uint4 u = *reinterpret_cast<const uint4*>(src);
-    raw[0] = u.x; raw[1] = u.y; raw[2] = u.z; raw[3] = u.w;
-  } else {
-    const uint2 u = *reinterpret_cast<const uint2*>(src);
-    raw[0] = u.x; raw[1] = u.y;
+__device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint32_t (&raw)[D / (2 * kRowLanes)]) {
+#pragma unroll
+  for (int c = 0; c < D / (8 * kRowLanes); ++c) {
+    const uint4 u = reinterpret_cast<const uint4*>(src)[c];
+    raw[4 * c] = u.x; raw[4 * c + 1] = u.y; raw[4 * c + 2] = u.z; raw[4 * c + 3] = u.w;
   }
 }
 
@@ -152,12 +154,6 @@ __device__ __forceinline__ uint32_t pack_low_bytes(int a, int b, int c, int d) {
   return __byte_perm(lo, hi, 0x5410);
 }
 
-// Max over the 16 lanes of this half warp (both halves reduce at once).
-__device__ __forceinline__ int half_warp_max(int v) {
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 
 // Lane-wise max of two pairs of 16-bit fields, unsigned or signed (the
 // signed form with a floor of 0).
@@ -172,10 +168,11 @@ __device__ __forceinline__ uint32_t vmax_relu_s16x2(uint32_t a, uint32_t b) {
   return d;
 }
 
-// Field-wise max of a u16x2 word over the 16 lanes of this half warp.
-__device__ __forceinline__ uint32_t half_warp_vmax_u16x2(uint32_t v) {
+// Field-wise max of a u16x2 word over the kRowLanes lanes of this row group
+// (the four groups of the warp reduce at once).
+__device__ __forceinline__ uint32_t row_vmax_u16x2(uint32_t v) {
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) v = vmax_u16x2(v, __shfl_xor_sync(0xffffffffu, v, o));
+  for (int o = kRowLanes / 2; o > 0; o >>= 1) v = vmax_u16x2(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
 
@@ -225,8 +222,8 @@ __device__ __forceinline__ uint32_t pack_sat_s8x2(int a, int b, uint32_t c) {
 // shuffles); a row that is not stored is still quantized, from whatever its
 // lanes hold.
 template <int D, int FMT>
-__device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 32], RowCodes<D, FMT>& rc) {
-  constexpr int E = D / 16;
+__device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / (2 * kRowLanes)], RowCodes<D, FMT>& rc) {
+  constexpr int E = D / kRowLanes;
   constexpr int NW = E / 2;                          // BF16 pairs of the lane
   rc.zp = 0;
   rc.s = __float2bfloat16_rn(0.f);
@@ -243,7 +240,7 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 32], RowC
       uint32_t m = raw[0] & 0x7fff7fffu;             // |x| of both halves
 #pragma unroll
       for (int i = 1; i < NW; ++i) m = vmax_u16x2(m, raw[i] & 0x7fff7fffu);
-      m = half_warp_vmax_u16x2(m);
+      m = row_vmax_u16x2(m);
       const float amax = __uint_as_float(max(m & 0xffffu, m >> 16) << 16);
       rc.s = __float2bfloat16_rn(E4 ? div_by_const<448>(amax) : div_by_const<57344>(amax));
       const float s = __bfloat162float(rc.s);
@@ -270,9 +267,9 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 32], RowC
         hw = vmax_relu_s16x2(hw, raw[i]);
         nw = vmax_relu_s16x2(nw, raw[i] ^ 0x80008000u);
       }
-      // both maxima in one word (hi low, nlo high), reduced over the half warp
-      const uint32_t hn = half_warp_vmax_u16x2(vmax_u16x2(__byte_perm(hw, nw, 0x5410),
-                                                           __byte_perm(hw, nw, 0x7632)));
+      // both maxima in one word (hi low, nlo high), reduced over the row group
+      const uint32_t hn = row_vmax_u16x2(vmax_u16x2(__byte_perm(hw, nw, 0x5410),
+                                                     __byte_perm(hw, nw, 0x7632)));
       const float hi = bf16_lo(hn), nlo = bf16_hi(hn);
       rc.s = __float2bfloat16_rn(div_by_const<255>(__fadd_rn(hi, nlo)));
       const float s = __bfloat162float(rc.s);
@@ -311,25 +308,35 @@ __device__ __forceinline__ void quantize_row(const uint32_t (&raw)[D / 32], RowC
 }
 
 // Static-scale INT8 (one given scale per channel, or one per cache): code =
-// clamp(rint(x / s), -127, 127), 0 where s <= 0 or s is NaN. s[i] and r[i] are
-// the scale of this lane's element i and its reciprocal RN(1/s), 0 when s is
-// below 2^-100 (those take the IEEE division). x is first clamped to
+// clamp(rint(x / s), -127, 127), 0 where s <= 0 or s is NaN. sc[i] and rc_[i]
+// (shared memory) are the scale of this lane's element i and its reciprocal
+// RN(1/s), 0 when s is below 2^-100 (those take the IEEE division). x is first clamped to
 // +-65536 s, which changes only quotients that saturate anyway and keeps the
 // corrected quotient inside the range where its rint equals that of the IEEE
 // quotient (tests/test_scale_division.py).
 template <int D>
-__device__ __forceinline__ void quantize_row_static(const uint32_t (&raw)[D / 32], const float (&sc)[D / 16],
-                                                    const float (&rc_)[D / 16], RowCodes<D, KVQ_INT8_CHANNEL>& rc) {
-  constexpr int E = D / 16;
+__device__ __forceinline__ void quantize_row_static(const uint32_t (&raw)[D / (2 * kRowLanes)],
+                                                    const float* sc, const float* rc_,
+                                                    RowCodes<D, KVQ_INT8_CHANNEL>& rc) {
+  constexpr int E = D / kRowLanes;
   rc.zp = 0;
   rc.s = __float2bfloat16_rn(0.f);
 #pragma unroll
   for (int i = 0; i < RowCodes<D, KVQ_INT8_CHANNEL>::WORDS; ++i) rc.w[i] = 0u;
+  // the lane's scales and reciprocals as 16-byte reads (sc, rc_ are 64-byte aligned)
+  float scv[E], rcv[E];
+#pragma unroll
+  for (int i = 0; i < E; i += 4) {
+    const float4 a = *reinterpret_cast<const float4*>(sc + i);
+    const float4 b = *reinterpret_cast<const float4*>(rc_ + i);
+    scv[i] = a.x; scv[i + 1] = a.y; scv[i + 2] = a.z; scv[i + 3] = a.w;
+    rcv[i] = b.x; rcv[i + 1] = b.y; rcv[i + 2] = b.z; rcv[i + 3] = b.w;
+  }
   int c[E];
 #pragma unroll
   for (int i = 0; i < E; ++i) {
     const float x = (i & 1) ? bf16_hi(raw[i / 2]) : bf16_lo(raw[i / 2]);
-    const float s = sc[i], r = rc_[i];
+    const float s = scv[i], r = rcv[i];
     c[i] = 0;
     if (s > 0.f) {
       const float lim = s * 65536.f;
@@ -393,10 +400,11 @@ __device__ __forceinline__ void store_bytes16(uint8_t* dst, const uint32_t (&w)[
 }
 
 // One CTA of 8 warps per (16 consecutive input tokens, KV head). Warp w takes
-// tokens 2w and 2w+1; for each, its lanes 0-15 quantize the token's K row and
-// lanes 16-31 its V row into shared memory. The input rows are requested before
-// the slots arrive (a skipped token's row is read and dropped), so the loads
-// overlap. The window is then written in page-sized pieces:
+// tokens 2w and 2w+1: its four lane groups quantize their K rows (lanes 0-15)
+// and V rows (lanes 16-31) into shared memory in one pass. The input rows are
+// requested before the slots arrive (a skipped token's row is read and
+// dropped), so the loads overlap. The window is then written in page-sized
+// pieces:
 //   - the 16 tokens fill one page in order (the bulk / prefill case): the page
 //     is written as whole 16-byte chunks, K in its chunk-major layout and V
 //     transposed with byte permutes;
@@ -406,9 +414,9 @@ __device__ __forceinline__ void store_bytes16(uint8_t* dst, const uint32_t (&w)[
 //     stores that range allows. A page continued from an offset (chunked
 //     prefill) thus costs one partial chunk per channel, not one byte store per
 //     token and channel.
-// Register use is capped at 32 so that 8 CTAs (64 warps) fit on an SM (51 and
-// 5 CTAs for the static-scale format, whose lanes keep their channels' scales
-// and reciprocals).
+// Register use is capped at 32 so that 8 CTAs (64 warps) fit on an SM (a few
+// bytes of spills for INT8 with its zero point cost less than 6 CTAs did); the
+// static-scale format takes 48 (5 CTAs), its scales in shared memory.
 template <int D, int FMT>
 __global__ void __launch_bounds__(256, FMT == KVQ_INT8_CHANNEL ? 5 : 8)
 append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
@@ -429,6 +437,9 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
   __shared__ __nv_bfloat16 kmb[kBlockSize][2], vmb[kBlockSize][2];
   __shared__ int64_t sl[kBlockSize];
   __shared__ int seg_i0[kBlockSize], seg_len[kBlockSize], nseg, page_fast;
+  // static scales of the head's K (0) and V (1) channels and their reciprocals
+  __shared__ __align__(16) float sscale[FMT == KVQ_INT8_CHANNEL ? 2 * D : 4];
+  __shared__ __align__(16) float srcp[FMT == KVQ_INT8_CHANNEL ? 2 * D : 4];
 
   // the decode kernel of the step may start its set-up now; it reads the
   // cache only after this grid has finished
@@ -438,18 +449,24 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
   const int n = int(min(int64_t(kBlockSize), int64_t(T) - tb));
   const int64_t nslots = int64_t(NB) * kBlockSize;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // lane group g = lane / 8: the K row (g = 0, 1) or the V row (g = 2, 3) of
+  // token 2 warp + (g & 1); requested before the slots arrive
   const int which = lane >> 4;                  // 0: K row, 1: V row
-  const int d0 = (lane & 15) * E;
-  // this half warp's rows: tokens 2 warp and 2 warp + 1, requested up front
-  const __nv_bfloat16* src = (which ? v : k) + ((tb + 2 * warp) * Hk + h) * D + d0;
-  uint32_t raws[2][D / 32];
+  const int ti = 2 * warp + ((lane >> 3) & 1);  // token of the window
+  const int d0 = (lane & (kRowLanes - 1)) * E;
+  const __nv_bfloat16* src = (which ? v : k) + ((tb + ti) * Hk + h) * D + d0;
+  uint32_t raw[D / (2 * kRowLanes)];
 #pragma unroll
-  for (int p = 0; p < 2; ++p) {
-#pragma unroll
-    for (int e = 0; e < D / 32; ++e) raws[p][e] = 0u;
-    if (2 * warp + p < n) load_row<D>(src + int64_t(p) * Hk * D, raws[p]);
-  }
+  for (int e = 0; e < D / (2 * kRowLanes); ++e) raw[e] = 0u;
+  if (ti < n) load_row<D>(src, raw);
   if (threadIdx.x < kBlockSize) sl[threadIdx.x] = threadIdx.x < n ? slots[tb + threadIdx.x] : -1;
+  if constexpr (FMT == KVQ_INT8_CHANNEL) {
+    for (int i = threadIdx.x; i < 2 * D; i += blockDim.x) {
+      const float sv = __bfloat162float((i >= D ? vs : ks)[per_tensor ? 0 : h * D + i % D]);
+      sscale[i] = sv;
+      srcp[i] = sv >= 7.88860905e-31f ? __frcp_rn(sv) : 0.f;   // 2^-100
+    }
+  }
   __syncthreads();
 
   if (warp == 0) {
@@ -479,37 +496,25 @@ append_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restri
     }
   }
 
-  // static scales: a half warp's rows are all K (lanes 0-15) or all V, so a
-  // lane's channels keep their scales for every row it quantizes
-  [[maybe_unused]] float ssc[E], rsc[E];
-  if constexpr (FMT == KVQ_INT8_CHANNEL) {
-    const __nv_bfloat16* sarr = which ? vs : ks;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      ssc[e] = __bfloat162float(sarr[per_tensor ? 0 : h * D + d0 + e]);
-      rsc[e] = ssc[e] >= 7.88860905e-31f ? __frcp_rn(ssc[e]) : 0.f;   // 2^-100
-    }
-  }
-#pragma unroll
-  for (int p = 0; p < 2; ++p) {
-    const int i = 2 * warp + p;                     // token in the window
+  {
     // every lane quantizes (the reductions span the warp); only real rows store
     RC rc;
-    if constexpr (FMT == KVQ_INT8_CHANNEL) quantize_row_static<D>(raws[p], ssc, rsc, rc);
-    else quantize_row<D, FMT>(raws[p], rc);
-    const int64_t slot = i < n ? sl[i] : -1;
-    if (slot < 0) continue;
+    if constexpr (FMT == KVQ_INT8_CHANNEL)
+      quantize_row_static<D>(raw, sscale + which * D + d0, srcp + which * D + d0, rc);
+    else quantize_row<D, FMT>(raw, rc);
+    const int64_t slot = ti < n ? sl[ti] : -1;
     if (slot >= nslots) {
-      if ((lane & 15) == 0) flag_error(KVQ_DEVERR_SLOT);
-      continue;
-    }
-    uint8_t* dst = (which ? vbuf : kbuf) + i * PADB + d0 * ELT;
-    if constexpr (E * ELT == 16) *reinterpret_cast<uint4*>(dst) = make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]);
-    else if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
-    else *reinterpret_cast<uint32_t*>(dst) = rc.w[0];
-    if ((lane & 15) == 0) {
-      (which ? vmb : kmb)[i][0] = rc.s;
-      (which ? vmb : kmb)[i][1] = __int2bfloat16_rn(rc.zp);
+      if ((lane & (kRowLanes - 1)) == 0) flag_error(KVQ_DEVERR_SLOT);
+    } else if (slot >= 0) {
+      uint8_t* dst = (which ? vbuf : kbuf) + ti * PADB + d0 * ELT;
+#pragma unroll
+      for (int c = 0; c < E * ELT / 16; ++c)
+        reinterpret_cast<uint4*>(dst)[c] = make_uint4(rc.w[4 * c], rc.w[4 * c + 1], rc.w[4 * c + 2], rc.w[4 * c + 3]);
+      if constexpr (E * ELT == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(rc.w[0], rc.w[1]);
+      if ((lane & (kRowLanes - 1)) == 0) {
+        (which ? vmb : kmb)[ti][0] = rc.s;
+        (which ? vmb : kmb)[ti][1] = __int2bfloat16_rn(rc.zp);
+      }
     }
   }
   __syncthreads();
