@@ -392,9 +392,10 @@ int kvq_decode_verify(const void* q, int32_t batch, int32_t n_query, const void*
  * products, at most 8 query rows per product), this call runs a kernel whose
  * products take 128 query rows of a KV head at a time (the chunk's positions
  * of its G query heads) against 64-token halves of the cache's 128-token
- * tiles, with the 8-bit codes expanded to f16 / bf16 in shared memory: the
- * scores are exact products accumulated in FP32 and the softmax weights keep
- * 16 bits, so the outputs agree with kvq_decode_verify's to rounding.
+ * tiles, with the 8-bit codes expanded to f16 in shared memory: the scores
+ * are exact products accumulated in FP32 and the softmax weights keep 22 bits
+ * (two f16 parts; 16 bits as two bf16 parts for a BF16 cache), so the outputs
+ * agree with kvq_decode_verify's to rounding.
  */
 size_t kvq_prefill_attn_workspace_bytes(int32_t batch, int32_t chunk_len, int32_t max_context_len,
                                         int32_t partition_tokens, kvq_fmt fmt,
