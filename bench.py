@@ -550,10 +550,14 @@ def multi_query_rate(st, flush, n_query, call="verify", reps=10, warmup=3):
             "kv_frac_of_peak": kv / (ms * 1e-3) / 1e9 / hbm,
             "positions_per_s": w.batch * n_query / (ms * 1e-3),
             "attention_tflops": flops / (ms * 1e-3) / 1e12,
-            "row_groups_per_kv_head": (w.group * n_query) // max(
+            **({"row_groups_per_kv_head": (w.group * n_query) // max(
                 g_ for g_ in (8, 4, 2, 1) if (w.group * n_query) % g_ == 0),
-            "what": ("speculative verification: " if call == "verify" else "prefill chunk: ")
-            + "decode partials + merge for n_query causal positions per sequence"}
+                "what": "speculative verification: decode partials (at most 8 query rows per "
+                        "tensor-core product) + merge for n_query causal positions per sequence"}
+               if call == "verify" else
+               {"row_blocks_per_kv_head": -(-w.group * n_query // 128),
+                "what": "prefill chunk: prefill partials (128 query rows per tensor-core "
+                        "product) + merge for n_query causal positions per sequence"})}
 
 
 def bulk_append_rate(st, tokens=32768, reps=5):
