@@ -12,10 +12,10 @@
 // kvq_kernels.cu after kvq_decode_mma.cuh (PieceWalk, tmem_load_cols).
 //
 // Pages arrive packed (b bits per code, 16 codes in 2b bytes) and are
-// expanded in shared memory by two converter warps into the 8-bit operand
-// layouts of the 8-bit formats (one shift and one mask per four output bytes). Rings: packed stages (producer -> converters) and
-// operand stages (converters -> MMA and softmax) are separate, so that more
-// copies are in flight than operand stages fit.
+// expanded in shared memory into the 8-bit operand layouts of the 8-bit
+// formats (one shift and one mask per four output bytes). Rings: packed
+// stages (producer -> expanding warps) and operand stages (-> MMA) are
+// separate, so that more copies are in flight than operand stages fit.
 //
 // 8 warps per CTA:
 //   warp 0      producer: lanes 0..7 copy one packed K and V page each of a
@@ -23,9 +23,12 @@
 //               the tile's K and V (s, z) pairs into the packed stage.
 //   warp 1      TMEM allocation; one thread issues the MMAs.
 //   warps 2..5  softmax warps: thread r owns token r (S, P) and channel r (O);
-//               they also rebuild the query operand for the next tile.
-//   warps 6..7  converters: expand the packed pages and move the (s, z) pairs
-//               into the operand stage.
+//               at the end of a tile they expand the next tile's V pages
+//               (whose stage the PV product two tiles back has released).
+//   warps 6..7  converters: expand the K pages and rebuild the query operand
+//               of every tile from its K channel scales (each warp half of the
+//               heads); they run ahead of the softmax warps, so the rebuild is
+//               off the softmax warps' per-tile chain.
 // Every wait is bounded as in the 8-bit kernel; on expiry the CTA drains what
 // it issued, writes NaN markers for its partials, frees TMEM and returns.
 // The tokens after the last complete group are not in this cache: a BF16
@@ -48,7 +51,6 @@ struct KiviCfg {
   static constexpr int NSL = (QPARTS * G + 7) / 8 * 8;
   static constexpr int NOL = (PPARTS * G + 7) / 8 * 8;
   static_assert(NS <= 32 && NO <= 32, "query group too large");
-  static constexpr int HPW = (G + 3) / 4;
   static constexpr int S_MMAS = D / 32;
   static constexpr int PV_MMAS = 128 / 32;
   static constexpr uint32_t K_LBO = 128, K_SBO = 8 * D;
@@ -61,26 +63,196 @@ struct KiviCfg {
   // shared memory (offsets from a 128-byte aligned base)
   static constexpr int OFF_K = 0;                                   // [NST][8 pages]
   static constexpr int OFF_V = OFF_K + NST * 8 * PAGE;
-  static constexpr int OFF_KM = OFF_V + NST * 8 * PAGE;             // [NST][8][META]
-  static constexpr int OFF_VM = OFF_KM + NST * 8 * META;
-  static constexpr int OFF_PK = OFF_VM + NST * 8 * META;            // [NSP][8 packed pages]
+  static constexpr int OFF_PK = OFF_V + NST * 8 * PAGE;             // [NSP][8 packed pages]
   static constexpr int OFF_PV = OFF_PK + NSP * 8 * PPAGE;
   static constexpr int OFF_PKM = OFF_PV + NSP * 8 * PPAGE;          // [NSP][8][META]
   static constexpr int OFF_PVM = OFF_PKM + NSP * 8 * META;
   static constexpr int OFF_Q = (OFF_PVM + NSP * 8 * META + 127) / 128 * 128;
   static constexpr int OFF_P = OFF_Q + QBYTES;                      // [2]
   static constexpr int OFF_BAR = OFF_P + 2 * PBYTES;
-  static constexpr int NBAR = 2 * NSP + 4 * NST + 10 + 3;
+  static constexpr int NBAR = 2 * NSP + 4 * NST + 10 + 3 + 4;
   static constexpr int OFF_RED = (OFF_BAR + 8 * NBAR + 15) / 16 * 16;   // float [2][64]; prologue
   static constexpr int OFF_RED2 = OFF_RED + 2 * 4 * 16 * 4;        // float [2][4][8]
-  static constexpr int OFF_QSC = OFF_RED2 + 2 * 4 * 8 * 4;         // float [2][8] scale, [2][8] sum(q z)
-  static constexpr int OFF_PMASK = OFF_QSC + 32 * 4;               // uint32 [NSP] packed, [NST] operand
-  static constexpr int OFF_MISC = (OFF_PMASK + 4 * (NSP + NST) + 15) / 16 * 16;
+  static constexpr int OFF_QSC = OFF_RED2 + 2 * 4 * 8 * 4;         // float [4][8] scale, [4][8] sum(q z)
+  static constexpr int OFF_PMASK = OFF_QSC + 64 * 4;               // uint32 [NSP] page masks
+  static constexpr int OFF_MISC = (OFF_PMASK + 4 * NSP + 15) / 16 * 16;
   static constexpr int OFF_WALK = OFF_MISC + 32;
   static constexpr int SMEM = OFF_WALK + 160 + 128;
   static_assert(OFF_RED % 16 == 0 && OFF_BAR % 8 == 0 && OFF_MISC % 16 == 0, "smem alignment");
-  static_assert(OFF_PK % 16 == 0 && OFF_PKM % 16 == 0 && OFF_KM % 16 == 0, "bulk copy alignment");
+  static_assert(OFF_PK % 16 == 0 && OFF_PKM % 16 == 0, "bulk copy alignment");
 };
+
+// Expand the packed codes of one 128-token tile's 8 pages (K or V) into the
+// 8-bit operand layout, by NT threads (t = 0 .. NT-1). 16 operand bytes (one
+// 16-byte row of a core matrix) come from one packed 32-bit word (2-bit codes:
+// bit pair k of packed byte j is operand byte 4k + j) or one 64-bit word
+// (4-bit: the low and high nibbles of packed byte j of word i are operand
+// bytes 8i + j and 8i + 4 + j). Consecutive threads take consecutive 16-byte
+// rows, so neither the packed reads nor the operand writes of a warp meet a
+// shared-memory bank twice; the packed words of a batch are all read before
+// any operand row is written (the two may alias as far as the compiler
+// knows), so a batch costs one shared-memory round trip.
+template <class C, int BITS, int NT>
+__device__ __forceinline__ void kivi_expand(const uint8_t* psrc, uint8_t* odst, int t) {
+  uint4* dst = reinterpret_cast<uint4*>(odst);
+  constexpr int PER = 8 * C::PAGE / 16 / NT;                // 16-byte rows per thread
+  constexpr int BATCH = PER < 8 ? PER : 8;
+  static_assert(PER * NT * 16 == 8 * C::PAGE && PER % BATCH == 0, "rows per thread");
+#pragma unroll
+  for (int b0 = 0; b0 < PER; b0 += BATCH) {
+    if constexpr (BITS == 2) {
+      uint32_t w[BATCH];
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k) w[k] = reinterpret_cast<const uint32_t*>(psrc)[t + NT * (b0 + k)];
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k)
+        dst[t + NT * (b0 + k)] = make_uint4(w[k] & 0x03030303u, (w[k] >> 2) & 0x03030303u,
+                                            (w[k] >> 4) & 0x03030303u, (w[k] >> 6) & 0x03030303u);
+    } else {
+      uint2 w[BATCH];
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k) w[k] = reinterpret_cast<const uint2*>(psrc)[t + NT * (b0 + k)];
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k)
+        dst[t + NT * (b0 + k)] = make_uint4(w[k].x & 0x0F0F0F0Fu, (w[k].x >> 4) & 0x0F0F0F0Fu,
+                                            w[k].y & 0x0F0F0F0Fu, (w[k].y >> 4) & 0x0F0F0F0Fu);
+    }
+  }
+}
+
+// The BF16 query rows of heads gs[0 .. HN) (-1: none) of one (sequence, KV
+// head) group starting at `rows`, as floats; lane owns the D/32 consecutive
+// channels lane * D/32 ...
+template <int D, int HN>
+__device__ __forceinline__ void kivi_load_query(float (&qr)[HN][D / 32], const int (&gs)[HN],
+                                                const __nv_bfloat16* rows, bool none, int lane) {
+  constexpr int CPL = D / 32;
+  const int d0 = lane * CPL;
+#pragma unroll
+  for (int hh = 0; hh < HN; ++hh) {
+    uint32_t w[CPL / 2];
+#pragma unroll
+    for (int i = 0; i < CPL / 2; ++i) w[i] = 0u;
+    if (gs[hh] >= 0 && !none) {
+      const __nv_bfloat16* src = rows + int64_t(gs[hh]) * D + d0;
+      if constexpr (CPL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(src);
+        w[0] = u.x; w[1] = u.y;
+      } else {
+        w[0] = *reinterpret_cast<const uint32_t*>(src);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < CPL / 2; ++i) {
+      qr[hh][2 * i] = __uint_as_float(w[i] << 16);
+      qr[hh][2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+}
+
+// The query operand rows of heads gs[0 .. HN) for one tile: x = q s_d (the
+// tile's K channel scales, from the (s, z) pairs `kpairs` of its packed stage)
+// in three exact s8 parts after a power-of-two scaling of the head, written
+// into `qop` (rows j * G + g); qsc_slot[g] = qk_scale * 2^-e and
+// qzs_slot[g] = qk_scale * sum_d q z_d. The lane's consecutive channels make
+// one word (or half word) per part. Warp-collective.
+template <class C, int D, int G, int HN>
+__device__ __forceinline__ void kivi_build_query(const float (&qc)[HN][D / 32], const int (&gs)[HN],
+                                                 const uint8_t* kpairs, uint8_t* qop, float* qsc_slot,
+                                                 float* qzs_slot, float qk_scale, int lane) {
+  using namespace tc;
+  constexpr int CPL = D / 32;
+  const int d0 = lane * CPL;
+  // the tile's K (s, z) pairs, in the packed stage the producer filled;
+  // channel d: page d / (D/8), entry d % (D/8); the lane's channels are
+  // consecutive entries of one page
+  const __nv_bfloat162* kmp = reinterpret_cast<const __nv_bfloat162*>(kpairs) +
+                              (d0 / (D / 8)) * kBlockSize + d0 % (D / 8);
+  float sd[CPL], zd[CPL];
+  {
+    __nv_bfloat162 pr[CPL];
+    if constexpr (CPL == 4) {
+      const uint4 u = *reinterpret_cast<const uint4*>(kmp);
+      *reinterpret_cast<uint4*>(pr) = u;
+    } else {
+      const uint2 u = *reinterpret_cast<const uint2*>(kmp);
+      *reinterpret_cast<uint2*>(pr) = u;
+    }
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) { sd[i] = __low2float(pr[i]); zd[i] = __high2float(pr[i]); }
+  }
+  // all of the warp's heads at once, so that their reductions overlap
+  float x[HN][CPL], zsum[HN];
+  uint32_t amax[HN];
+#pragma unroll
+  for (int hh = 0; hh < HN; ++hh) {
+    float zs = 0.f, am = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      x[hh][i] = qc[hh][i] * sd[i];
+      zs = fmaf(qc[hh][i], zd[i], zs);
+      am = fmaxf(am, fabsf(x[hh][i]));
+    }
+    zsum[hh] = zs;
+    amax[hh] = __float_as_uint(am);
+  }
+  // the head's largest |x|: one integer reduction on the float bits (x >= 0)
+#pragma unroll
+  for (int hh = 0; hh < HN; ++hh) amax[hh] = __reduce_max_sync(0xffffffffu, amax[hh]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int hh = 0; hh < HN; ++hh) zsum[hh] += __shfl_xor_sync(0xffffffffu, zsum[hh], o);
+#pragma unroll
+  for (int hh = 0; hh < HN; ++hh) {
+    const int g = gs[hh];
+    // e = 5 - floor(log2 amax) from the exponent field (zero and subnormal
+    // maxima clamp to 120, infinities to -120)
+    int e = 0;
+    if (amax[hh] != 0u) e = 5 - (int(amax[hh] >> 23) - 127);
+    e = max(-120, min(120, e));
+    const float up = __int_as_float((127 + e) << 23);
+    const float down = __int_as_float((127 - e) << 23);
+    // the three parts by rounding additions (1.5 * 2^23 + v holds rint(v)
+    // in its low bits for |v| < 2^22): t_j's low byte is part j's code
+    constexpr float kMg = 12582912.0f;
+    uint32_t tb[3][CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const float xs = x[hh][i] * up;
+      const float t0 = __fadd_rn(xs, kMg), x0 = __fsub_rn(t0, kMg);
+      const float r0 = (xs - x0) * 128.f;
+      const float t1 = __fadd_rn(r0, kMg), x1 = __fsub_rn(t1, kMg);
+      const float t2 = __fadd_rn((r0 - x1) * 128.f, kMg);
+      tb[0][i] = __float_as_uint(t0);
+      tb[1][i] = __float_as_uint(t1);
+      tb[2][i] = __float_as_uint(t2);
+    }
+    uint32_t part[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      if constexpr (CPL == 4)
+        part[j] = __byte_perm(__byte_perm(tb[j][0], tb[j][1], 0x0040), __byte_perm(tb[j][2], tb[j][3], 0x0040), 0x5410);
+      else
+        part[j] = __byte_perm(tb[j][0], tb[j][1], 0x0040) & 0xFFFFu;
+    }
+    if (g >= 0) {
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const int n = j * G + g;                         // operand row of this part
+        uint8_t* at = qop + (n >> 3) * C::Q_SBO + (n & 7) * 16 + (d0 >> 4) * C::Q_LBO + (d0 & 15);
+        if constexpr (CPL == 4) *reinterpret_cast<uint32_t*>(at) = part[j];
+        else *reinterpret_cast<uint16_t*>(at) = uint16_t(part[j]);
+      }
+      if (lane == 0) {
+        qsc_slot[g] = qk_scale * down;
+        qzs_slot[g] = qk_scale * zsum[hh];
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+}
 
 template <int D, int G, int BITS>
 __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
@@ -167,8 +339,6 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
 
   uint8_t* kring = smem + C::OFF_K;
   uint8_t* vring = smem + C::OFF_V;
-  uint8_t* kmeta = smem + C::OFF_KM;
-  uint8_t* vmeta = smem + C::OFF_VM;
   uint8_t* pkring = smem + C::OFF_PK;
   uint8_t* pvring = smem + C::OFF_PV;
   uint8_t* pkmeta = smem + C::OFF_PKM;
@@ -190,12 +360,12 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
   uint64_t* qready = ofree + 2;
   uint64_t* qfree = qready + 1;
   uint64_t* drain = qfree + 1;
+  uint64_t* qinfo = drain + 1;                 // [4] converters -> softmax (qsc, qzs)
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
   float* red2 = reinterpret_cast<float*>(smem + C::OFF_RED2);
-  float* qsc = reinterpret_cast<float*>(smem + C::OFF_QSC);      // [2][8]
-  float* qzs = qsc + 16;                                           // [2][8]
+  float* qsc = reinterpret_cast<float*>(smem + C::OFF_QSC);      // [4][8]
+  float* qzs = qsc + 32;                                           // [4][8]
   volatile uint32_t* pmask_p = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_PMASK);
-  volatile uint32_t* pmask_u = pmask_p + C::NSP;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -204,12 +374,12 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSP; ++s) {
       mbar_init(pfull + s, 1);
-      mbar_init(pfree + s, 64 + 128);             // converters and softmax warps
+      mbar_init(pfree + s, 64 + 128);             // converters (K) and softmax warps (V)
     }
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(kready + s, 64);
       mbar_init(kempty + s, 128);
-      mbar_init(vready + s, 64);
+      mbar_init(vready + s, 128);
       mbar_init(vempty + s, 1);
     }
     for (int j = 0; j < 2; ++j) {
@@ -219,8 +389,9 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
       mbar_init(ofull + j, 1);
       mbar_init(ofree + j, 128);
     }
-    mbar_init(qready, 128);
+    mbar_init(qready, 64);
     mbar_init(qfree, 1);
+    for (int j = 0; j < 4; ++j) mbar_init(qinfo + j, 64);
     mbar_init(drain, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -333,66 +504,49 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
   } else if (warp >= 6) {
     // ---------------------------------------------------------- converters
     const int ct = threadIdx.x - 192;                       // 0..63
+    const int cw = warp - 6;
+    // the query operand of every tile: heads cw, cw + 2, ... (the converters
+    // run several tiles ahead of the softmax warps, so the rebuild is off the
+    // softmax warps' per-tile chain)
+    constexpr int HPC = (G + 1) / 2;
+    constexpr int CPL = D / 32;
+    int gsc[HPC];
+#pragma unroll
+    for (int hh = 0; hh < HPC; ++hh) gsc[hh] = cw + 2 * hh < G ? cw + 2 * hh : -1;
+    auto rows_of = [&](const PieceWalk& pw) { return q + (int64_t(pw.b) * Hq + int64_t(pw.h) * G) * D; };
     bool ok = true;
     int gt = 0;
-    for (PieceWalk pw = walk; !pw.done; walk_next(pw)) {
+    float qcur[HPC][CPL], qnext[HPC][CPL];
+    kivi_load_query<D, HPC>(qcur, gsc, walk.done ? q : rows_of(walk), walk.done, lane);
+    for (PieceWalk pw = walk; !pw.done;) {
+      PieceWalk nx = pw;
+      walk_next(nx);
+      kivi_load_query<D, HPC>(qnext, gsc, nx.done ? q : rows_of(nx), nx.done, lane);   // a piece ahead
       for (int i = pw.lo; i < pw.hi; ++i, ++gt) {
         const int sp = gt % C::NSP, su = gt % C::NST;
         if (ok) ok = mbar_wait(pfull + sp, (gt / C::NSP) & 1, abort_flag, wait_limit);
         // K operand stage free: the S product of its last tile has been read
         if (ok) ok = mbar_wait(kempty + su, ((gt / C::NST) & 1) ^ 1, abort_flag, wait_limit);
         if (ok) {
-          // 16 packed bytes -> 16 x (8 / BITS) operand bytes per step
-          const uint4* src = reinterpret_cast<const uint4*>(pkring + sp * 8 * C::PPAGE);
-          uint4* dst = reinterpret_cast<uint4*>(kring + su * 8 * C::PAGE);
-          for (int u = ct; u < 8 * C::PPAGE / 16; u += 64) {
-            const uint4 w = src[u];
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-            if constexpr (BITS == 2) {
-#pragma unroll
-              for (int x = 0; x < 4; ++x)
-                dst[4 * u + x] = make_uint4(ws[x] & 0x03030303u, (ws[x] >> 2) & 0x03030303u,
-                                            (ws[x] >> 4) & 0x03030303u, (ws[x] >> 6) & 0x03030303u);
-            } else {
-#pragma unroll
-              for (int x = 0; x < 2; ++x)
-                dst[2 * u + x] = make_uint4(ws[2 * x] & 0x0F0F0F0Fu, (ws[2 * x] >> 4) & 0x0F0F0F0Fu,
-                                            ws[2 * x + 1] & 0x0F0F0F0Fu,
-                                            (ws[2 * x + 1] >> 4) & 0x0F0F0F0Fu);
-            }
-          }
-          if (ct == 0) pmask_u[su] = pmask_p[sp];
+          kivi_expand<C, BITS, 64>(pkring + sp * 8 * C::PPAGE, kring + su * 8 * C::PAGE, ct);
           fence_proxy_async_smem();
         }
         mbar_arrive(kready + su);
-        if (ok) ok = mbar_wait(vempty + su, ((gt / C::NST) & 1) ^ 1, abort_flag, wait_limit);
-        if (ok) {
-          const uint4* src = reinterpret_cast<const uint4*>(pvring + sp * 8 * C::PPAGE);
-          uint4* dst = reinterpret_cast<uint4*>(vring + su * 8 * C::PAGE);
-          for (int u = ct; u < 8 * C::PPAGE / 16; u += 64) {
-            const uint4 w = src[u];
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-            if constexpr (BITS == 2) {
-#pragma unroll
-              for (int x = 0; x < 4; ++x)
-                dst[4 * u + x] = make_uint4(ws[x] & 0x03030303u, (ws[x] >> 2) & 0x03030303u,
-                                            (ws[x] >> 4) & 0x03030303u, (ws[x] >> 6) & 0x03030303u);
-            } else {
-#pragma unroll
-              for (int x = 0; x < 2; ++x)
-                dst[2 * u + x] = make_uint4(ws[2 * x] & 0x0F0F0F0Fu, (ws[2 * x] >> 4) & 0x0F0F0F0Fu,
-                                            ws[2 * x + 1] & 0x0F0F0F0Fu,
-                                            (ws[2 * x + 1] >> 4) & 0x0F0F0F0Fu);
-            }
-          }
-          if (ct < 32)
-            reinterpret_cast<uint4*>(vmeta + su * 8 * C::META)[ct] =
-                reinterpret_cast<const uint4*>(pvmeta + sp * 8 * C::META)[ct];
-          fence_proxy_async_smem();
-        }
-        mbar_arrive(vready + su);
-        mbar_arrive(pfree + sp);
+        // this warp's heads of the tile's query operand (the previous tile's S
+        // product has read the operand)
+        if (ok && gt > 0) ok = mbar_wait(qfree, (gt - 1) & 1, abort_flag, wait_limit);
+        if (ok)
+          kivi_build_query<C, D, G, HPC>(qcur, gsc, pkmeta + sp * 8 * C::META, qop, qsc + (gt & 3) * 8,
+                                         qzs + (gt & 3) * 8, qk_scale, lane);
+        mbar_arrive(qready);
+        mbar_arrive(qinfo + (gt & 3));
+        mbar_arrive(pfree + sp);                          // the softmax warps expand V
       }
+#pragma unroll
+      for (int hh = 0; hh < HPC; ++hh)
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) qcur[hh][i] = qnext[hh][i];
+      pw = nx;
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -448,7 +602,6 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
     // ---------------------------------------------------------- softmax warps
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int cw = warp - 2;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     bool ok = true;
     const uint32_t prow = (r >> 3) * C::P_LBO + (r & 7) * 16;
@@ -469,129 +622,29 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
     }
     named_bar_sync(1, 128);
 
-    // the BF16 query rows of a piece's group, loaded one piece ahead
-    float qv[C::HPW][D / 32];
-    // lane owns the D/32 consecutive channels d0 .. d0 + D/32 - 1
-    constexpr int CPL = D / 32;
-    const int d0 = lane * CPL;
-    auto load_q = [&](bool none, int qb, int qh) {
-#pragma unroll
-      for (int hh = 0; hh < C::HPW; ++hh) {
-        const int g = cw + 4 * hh;
-        uint32_t w[CPL / 2];
-#pragma unroll
-        for (int i = 0; i < CPL / 2; ++i) w[i] = 0u;
-        if (g < G && !none) {
-          const __nv_bfloat16* src = q + (int64_t(qb) * Hq + qh * G + g) * D + d0;
-          if constexpr (CPL == 4) {
-            const uint2 u = *reinterpret_cast<const uint2*>(src);
-            w[0] = u.x; w[1] = u.y;
-          } else {
-            w[0] = *reinterpret_cast<const uint32_t*>(src);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < CPL / 2; ++i) {
-          qv[hh][2 * i] = __uint_as_float(w[i] << 16);
-          qv[hh][2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-        }
+    // the V codes of a tile, expanded by these warps one tile ahead (at the end
+    // of the previous tile, whose PV product has been issued by then), with
+    // the tile's page mask and this token's V (s, z) kept in registers
+    uint32_t vmask_n = 0u;
+    float sv_n = 0.f, zv_n = 0.f;
+    auto stage_v = [&](int gv) {
+      const int sp = gv % C::NSP, su = gv % C::NST;
+      if (ok) ok = mbar_wait(pfull + sp, (gv / C::NSP) & 1, abort_flag, wait_limit);
+      // V operand stage free: the PV product of its last tile has completed
+      if (ok) ok = mbar_wait(vempty + su, ((gv / C::NST) & 1) ^ 1, abort_flag, wait_limit);
+      if (ok) {
+        kivi_expand<C, BITS, 128>(pvring + sp * 8 * C::PPAGE, vring + su * 8 * C::PAGE, r);
+        vmask_n = pmask_p[sp];
+        const __nv_bfloat162 vmp =
+            reinterpret_cast<const __nv_bfloat162*>(pvmeta + (sp * 8 + (r >> 4)) * C::META)[r & 15];
+        sv_n = __low2float(vmp);
+        zv_n = __high2float(vmp);
+        fence_proxy_async_smem();
       }
+      mbar_arrive(vready + su);
+      mbar_arrive(pfree + sp);
     };
-    // query operand of tile gt: x = q s_d (the tile's channel scales) in three
-    // exact s8 parts after a power-of-two scaling of the head, and sum_d q z_d;
-    // the lane's consecutive channels make one word (or half word) per part
-    auto store_q = [&](int gt_q, const float (&qcur)[C::HPW][D / 32]) {
-      const int sp = gt_q % C::NSP;
-      // the tile's K (s, z) pairs, read from the packed stage the producer filled
-      // (it is released only when the converters and these warps are done);
-      // channel d: page d / (D/8), entry d % (D/8); the lane's channels are
-      // consecutive entries of one page
-      const __nv_bfloat162* kmp = reinterpret_cast<const __nv_bfloat162*>(pkmeta + sp * 8 * C::META) +
-                                  (d0 / (D / 8)) * kBlockSize + d0 % (D / 8);
-      float sd[CPL], zd[CPL];
-      {
-        __nv_bfloat162 pr[CPL];
-        if constexpr (CPL == 4) {
-          const uint4 u = *reinterpret_cast<const uint4*>(kmp);
-          *reinterpret_cast<uint4*>(pr) = u;
-        } else {
-          const uint2 u = *reinterpret_cast<const uint2*>(kmp);
-          *reinterpret_cast<uint2*>(pr) = u;
-        }
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) { sd[i] = __low2float(pr[i]); zd[i] = __high2float(pr[i]); }
-      }
-#pragma unroll
-      for (int hh = 0; hh < C::HPW; ++hh) {
-        const int g = cw + 4 * hh;
-        if (g >= G) continue;
-        float x[CPL], zsum = 0.f, amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-          x[i] = qcur[hh][i] * sd[i];
-          zsum = fmaf(qcur[hh][i], zd[i], zsum);
-          amax = fmaxf(amax, fabsf(x[i]));
-        }
-        // the head's largest |x|: one integer reduction on the float bits (x >= 0)
-        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
-        zsum = warp_sum(zsum);
-        int e = 0;
-        if (amax > 0.f) e = 5 - ilogbf(amax);
-        e = max(-120, min(120, e));
-        const float up = __int_as_float((127 + e) << 23);
-        const float down = __int_as_float((127 - e) << 23);
-        // the three parts by rounding additions (1.5 * 2^23 + v holds rint(v)
-        // in its low bits for |v| < 2^22): t_j's low byte is part j's code
-        constexpr float kMg = 12582912.0f;
-        uint32_t tb[3][CPL];
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-          const float xs = x[i] * up;
-          const float t0 = __fadd_rn(xs, kMg), x0 = __fsub_rn(t0, kMg);
-          const float r0 = (xs - x0) * 128.f;
-          const float t1 = __fadd_rn(r0, kMg), x1 = __fsub_rn(t1, kMg);
-          const float t2 = __fadd_rn((r0 - x1) * 128.f, kMg);
-          tb[0][i] = __float_as_uint(t0);
-          tb[1][i] = __float_as_uint(t1);
-          tb[2][i] = __float_as_uint(t2);
-        }
-        uint32_t part[3];
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          if constexpr (CPL == 4)
-            part[j] = __byte_perm(__byte_perm(tb[j][0], tb[j][1], 0x0040), __byte_perm(tb[j][2], tb[j][3], 0x0040), 0x5410);
-          else
-            part[j] = __byte_perm(tb[j][0], tb[j][1], 0x0040) & 0xFFFFu;
-        }
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          const int n = j * G + g;                           // operand row of this part
-          uint8_t* at = qop + (n >> 3) * C::Q_SBO + (n & 7) * 16 + (d0 >> 4) * C::Q_LBO + (d0 & 15);
-          if constexpr (CPL == 4) *reinterpret_cast<uint32_t*>(at) = part[j];
-          else *reinterpret_cast<uint16_t*>(at) = uint16_t(part[j]);
-        }
-        if (lane == 0) {
-          qsc[(gt_q & 1) * 8 + g] = qk_scale * down;
-          qzs[(gt_q & 1) * 8 + g] = qk_scale * zsum;
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-    };
-
-    // the first tile's query
-    load_q(wk[0].done, wk[0].b, wk[0].h);
-    float qcur[C::HPW][D / 32];
-#pragma unroll
-    for (int hh = 0; hh < C::HPW; ++hh)
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) qcur[hh][i] = qv[hh][i];
-    if (!wk[0].done) {
-      if (ok) ok = mbar_wait(pfull + 0, 0, abort_flag, wait_limit);
-      if (ok) store_q(0, qcur);
-      mbar_arrive(pfree + 0);
-    }
-    mbar_arrive(qready);
+    if (!wk[0].done) stage_v(0);
 
     int gt = 0;
     for (int pc = 0;; ++pc) {
@@ -602,7 +655,6 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
       const int t1 = min(hi * 128, cur->ctx);
       const int slot = pinfo[(pc & 1) * 2], last = pinfo[(pc & 1) * 2 + 1];
       const bool more = !nxt->done;
-      load_q(!more, nxt->b, nxt->h);                     // the next piece's query rows
       named_bar_sync(1, 128);
       if (r == 0) {
         PieceWalk n = *nxt;
@@ -651,45 +703,22 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
         }
         tc_fence_before();
         mbar_arrive(sfree + (gt & 1));
+        // the K stage of this tile is free (its S product has been read)
+        mbar_arrive(kempty + su);
+        // the tile's per-head query factors, written with its query operand
+        if (ok) ok = mbar_wait(qinfo + (gt & 3), (gt >> 2) & 1, abort_flag, wait_limit);
         float qs[G], qz[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          qs[g] = qsc[(gt & 1) * 8 + g];
-          qz[g] = qzs[(gt & 1) * 8 + g];
+          qs[g] = qsc[(gt & 3) * 8 + g];
+          qz[g] = qzs[(gt & 3) * 8 + g];
         }
-        // ---- the next tile's query: its channel scales from the packed stage
-        // (the next tile may open the next piece, whose query rows were loaded
-        // ahead); it waits only for the producer, which runs a few tiles ahead
-        const bool last_tile = i + 1 == hi;
-        const bool has_next = !last_tile || more;
-        if (has_next) {
-          if (ok) ok = mbar_wait(qfree, gt & 1, abort_flag, wait_limit);
-          if (ok) ok = mbar_wait(pfull + (gt + 1) % C::NSP, ((gt + 1) / C::NSP) & 1, abort_flag, wait_limit);
-          if (last_tile) {
-#pragma unroll
-            for (int hh = 0; hh < C::HPW; ++hh)
-#pragma unroll
-              for (int ii = 0; ii < D / 32; ++ii) qcur[hh][ii] = qv[hh][ii];
-          }
-          if (ok) store_q(gt + 1, qcur);
-          mbar_arrive(pfree + (gt + 1) % C::NSP);       // this packed stage's K pairs are read
-          mbar_arrive(qready);
-        }
-        // the K stage of this tile is free (its S product has been read)
-        mbar_arrive(kempty + su);
 
-        // ---- this token's V (s, z)
-        if (ok) ok = mbar_wait(vready + su, (gt / C::NST) & 1, abort_flag, wait_limit);
-        const uint32_t mask = ok ? pmask_u[su] : 0u;
+        // ---- this token's V (s, z), taken when the tile's V was expanded
+        const uint32_t mask = ok ? vmask_n : 0u;
         const int tile0 = i * 128;
-        const int p = r >> 4, t = r & 15;
-        const bool valid = ok && ((mask >> p) & 1u) && (tile0 + r < t1);
-        float sv = 0.f, zv = 0.f;
-        if (valid) {
-          const __nv_bfloat162 vmp = reinterpret_cast<const __nv_bfloat162*>(vmeta + (su * 8 + p) * C::META)[t];
-          sv = __low2float(vmp);
-          zv = __high2float(vmp);
-        }
+        const bool valid = ok && ((mask >> (r >> 4)) & 1u) && (tile0 + r < t1);
+        const float sv = valid ? sv_n : 0.f, zv = valid ? zv_n : 0.f;
         float x[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -723,7 +752,7 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
         const float4 s4 = *reinterpret_cast<const float4*>(rb + 8 * 4);
         const float svmax = fmaxf(fmaxf(s4.x, s4.y), fmaxf(s4.z, s4.w));
         int ex = 0;
-        if (svmax > 0.f) ex = max(-120, min(120, 7 - ilogbf(svmax)));
+        if (svmax > 0.f) ex = max(-120, min(120, 7 - (int(__float_as_uint(svmax) >> 23) - 127)));
         const float escale = __int_as_float((127 + ex) << 23);
         const float einv = __int_as_float((127 - ex) << 23);
 
@@ -759,6 +788,8 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
         mbar_arrive(pready + (gt & 1));
         if (i > lo) accum_o(gt - 1);
         einv_pend = einv;
+        // the next tile's V (it may open the next piece)
+        if (i + 1 < hi || more) stage_v(gt + 1);
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) alpha[g] = 1.f;
