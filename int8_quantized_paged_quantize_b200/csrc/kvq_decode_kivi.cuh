@@ -742,12 +742,13 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
           const float4 t4 = *reinterpret_cast<const float4*>(rb + g * 4);
           const float tmax = fmaxf(fmaxf(t4.x, t4.y), fmaxf(t4.z, t4.w));
           const float mn = fmaxf(m[g], tmax);
-          alpha[g] = 1.f;
-          if (mn != m[g]) {
-            alpha[g] = (mn == -INFINITY) ? 1.f : exp2f(m[g] - mn);
-            m[g] = mn;
-            o[g] *= alpha[g];
-          }
+          // 2^(m - mn) when the maximum moves, 1 while it stays (or while no
+          // token has been seen): selects rather than branches, so that the
+          // heads' exponentials overlap
+          const float a = exp2f(m[g] - mn);
+          alpha[g] = (mn == m[g] || mn == -INFINITY) ? 1.f : a;
+          m[g] = mn;
+          o[g] *= alpha[g];
         }
         const float4 s4 = *reinterpret_cast<const float4*>(rb + 8 * 4);
         const float svmax = fmaxf(fmaxf(s4.x, s4.y), fmaxf(s4.z, s4.w));
@@ -763,7 +764,8 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
         const float ysc = sv * escale * 65536.f;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float pr = x[g] != -INFINITY ? exp2f(x[g] - m[g]) : 0.f;
+          const float e2 = exp2f(x[g] - m[g]);
+          const float pr = x[g] != -INFINITY ? e2 : 0.f;
           l[g] = l[g] * alpha[g] + pr;
           yv[g] = __float2uint_rn(pr * ysc);
           corr[g] = corr[g] * alpha[g] + pr * zv;
