@@ -934,27 +934,38 @@ int launch_kivi_decode(const void* q, int32_t B, const void* kc, const void* vc,
     e = bits == 2 ? kivi_dispatch2<64, 2>(G, q, B, kc, vc, km, vm, tables, qlens, max_qlen, sm_scale, pa, ws, d, st)
                   : kivi_dispatch2<64, 4>(G, q, B, kc, vc, km, vm, tables, qlens, max_qlen, sm_scale, pa, ws, d, st);
   if (e != cudaSuccess) return int(e);
-  // the residual tokens, through the BF16 kernel
-  const int rc = launch_decode_partial(q, B, rk, rv, nullptr, nullptr, rtables, rlens, max_rlen,
-                                       sm_scale, pb, ws_b, KVQ_BF16, rd, stream, 1);
-  if (rc != 0) return rc;
+  // the residual tokens and the merge, one CTA per (sequence, KV head),
+  // launched as a programmatic dependent of the groups kernel
+  (void)pb;
   const float* poa = static_cast<const float*>(ws);
   const float* pmla = reinterpret_cast<const float*>(static_cast<const char*>(ws) + pa.o_bytes);
   const int32_t* pca = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + pa.o_bytes + pa.ml_bytes);
-  const float* pob = static_cast<const float*>(ws_b);
-  const float* pmlb = reinterpret_cast<const float*>(static_cast<const char*>(ws_b) + pb.o_bytes);
-  const int32_t* pcb = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws_b) + pb.o_bytes + pb.ml_bytes);
-  const dim3 grid(unsigned(int64_t(B) * d.n_q_heads));
-  const int Hq = d.n_q_heads;
-#define KVQ_M2(DD, OT) merge2_kernel<DD, OT><<<grid, DD, 0, st>>>(Hq, G, qlens, pa.slots, max_qlen, \
-      d.max_blocks_per_seq, poa, pmla, pca, rlens, pb.slots, max_rlen, rd.max_blocks_per_seq, pob, pmlb, pcb, ~127, \
-      static_cast<OT*>(out))
-  if (d.head_dim == 128) {
-    if (out_f32) KVQ_M2(128, float); else KVQ_M2(128, __nv_bfloat16);
-  } else {
-    if (out_f32) KVQ_M2(64, float); else KVQ_M2(64, __nv_bfloat16);
+  const dim3 grid(unsigned(int64_t(B) * d.n_kv_heads));
+  const float qk = sm_scale * kLog2e;
+  auto go = [&](auto kern, auto* o) {
+    return launch_pdl(kern, grid, dim3(128), 0, st, static_cast<const __nv_bfloat16*>(q), d.n_kv_heads,
+                      qlens, pa.slots, max_qlen, d.max_blocks_per_seq, poa, pmla, pca,
+                      static_cast<const __nv_bfloat16*>(rk), static_cast<const __nv_bfloat16*>(rv), rtables,
+                      rlens, rd.num_blocks, rd.max_blocks_per_seq, max_rlen, qk, o);
+  };
+#define KVQ_RM(DD, GG)                                                                        \
+  e = out_f32 ? go(kivi_residual_merge_kernel<DD, GG, float>, static_cast<float*>(out))       \
+              : go(kivi_residual_merge_kernel<DD, GG, __nv_bfloat16>, static_cast<__nv_bfloat16*>(out))
+#define KVQ_RM_G(DD)        \
+  switch (G) {              \
+    case 1: KVQ_RM(DD, 1); break; \
+    case 2: KVQ_RM(DD, 2); break; \
+    case 4: KVQ_RM(DD, 4); break; \
+    default: KVQ_RM(DD, 8); break; \
   }
-#undef KVQ_M2
+  if (d.head_dim == 128) {
+    KVQ_RM_G(128)
+  } else {
+    KVQ_RM_G(64)
+  }
+#undef KVQ_RM_G
+#undef KVQ_RM
+  if (e != cudaSuccess) return int(e);
   return int(cudaGetLastError());
 }
 

@@ -1,6 +1,7 @@
 // Log-sum-exp merge of the decode kernels' split-K partials into the output
-// rows: one set (kvq_decode_merge) or two sets of the same rows (the KIVI-style
-// cache's quantized groups and its BF16 residual). Included by kvq_kernels.cu.
+// rows (kvq_decode_merge), and the KIVI-style cache's BF16 residual attention
+// fused with the merge of its quantized groups' partials. Included by
+// kvq_kernels.cu.
 #pragma once
 
 namespace kvq {
@@ -124,45 +125,182 @@ __global__ void __launch_bounds__(128) merge_kernel(const int32_t* __restrict__ 
   }
 }
 
-// Merge of two partial sets of the same rows: the quantized groups' partials
-// (a) and the residual tokens' (b), each with its own context lengths, slot
-// count and per-(sequence, row group) counts.
-template <int D, typename OutT>
-__global__ void __launch_bounds__(128) merge2_kernel(
-    int Hq, int G, const int32_t* __restrict__ ctx_a, int slots_a, int max_a, int W_a,
-    const float* __restrict__ po_a, const float* __restrict__ pml_a, const int32_t* __restrict__ pc_a,
-    const int32_t* __restrict__ ctx_b, int slots_b, int max_b, int W_b,
-    const float* __restrict__ po_b, const float* __restrict__ pml_b, const int32_t* __restrict__ pc_b,
-    int group_mask_a, OutT* __restrict__ out) {
-  const int bq = blockIdx.x;
-  const int b = bq / Hq;
-  const int d = threadIdx.x;
-  int ca = ctx_a[b], cb = ctx_b[b];
-  if (ca < 0 || ca > max_a || int64_t(ca) > int64_t(W_a) * kBlockSize) ca = 0;
-  ca &= group_mask_a;
-  if (cb < 0 || cb > max_b || int64_t(cb) > int64_t(W_b) * kBlockSize) cb = 0;
-  const int na = ca > 0 ? min(slots_a, max(0, pc_a[bq / G])) : 0;
-  const int nb = cb > 0 ? min(slots_b, max(0, pc_b[bq / G])) : 0;
-  const int64_t ra = int64_t(bq) * slots_a, rb = int64_t(bq) * slots_b;
-  float M = -INFINITY;
-  for (int s = 0; s < na; ++s) M = fmaxf(M, pml_a[(ra + s) * 2]);
-  for (int s = 0; s < nb; ++s) M = fmaxf(M, pml_b[(rb + s) * 2]);
-  float o = 0.f, l = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < na; ++s) {
-      const float f = exp2f(pml_a[(ra + s) * 2] - M);
-      l += pml_a[(ra + s) * 2 + 1] * f;
-      o += po_a[(ra + s) * D + d] * f;
-    }
-    for (int s = 0; s < nb; ++s) {
-      const float f = exp2f(pml_b[(rb + s) * 2] - M);
-      l += pml_b[(rb + s) * 2 + 1] * f;
-      o += po_b[(rb + s) * D + d] * f;
-    }
+// ------------------------------------------------------- KIVI residual
+// The KIVI-style decode's second half: the BF16 residual tokens (those after
+// the last complete group) of one (sequence, KV head), attended in FP32 on the
+// CUDA cores, then the log-sum-exp merge with the quantized groups' partial
+// slots of the same rows. One CTA of 128 threads per (sequence, KV head)
+// covers the group's G query rows:
+//   scores   thread t takes token t of each 128-token chunk: its K row from
+//            the BF16 operand page (16-byte chunks 128 bytes apart), dot
+//            products with the G query rows (times sm_scale log2 e) held in
+//            shared memory;
+//   values   thread d < D accumulates O[g][d] over the chunk's tokens from the
+//            transposed V page: one 16-byte load per 8 tokens of its channel;
+//   softmax  online over the chunks in base 2, as the decode kernels do;
+//   merge    m = max(m_res, m_i), l and o summed with weights 2^(m_x - m).
+// Launched as a programmatic dependent of the groups kernel, which does not
+// signal early: the launch overlaps the groups kernel's end, and the
+// partials are read after the grid dependency wait, through plain pointers
+// and L2-coherent loads (never taken as invariant data that could be read
+// ahead of the wait).
+template <int D, int G, typename OutT>
+__global__ void __launch_bounds__(128) kivi_residual_merge_kernel(
+    const __nv_bfloat16* __restrict__ q, int Hk, const int32_t* ctx_a, int slots_a, int max_a,
+    int W_a, const float* po_a, const float* pml_a, const int32_t* pc_a,
+    const __nv_bfloat16* __restrict__ rk,
+    const __nv_bfloat16* __restrict__ rv, const int32_t* __restrict__ rtables,
+    const int32_t* __restrict__ rlens, int NBr, int Wr, int max_r, float qk_scale,
+    OutT* __restrict__ out) {
+  using namespace tc;
+  __shared__ __align__(16) float qsh[G][D];
+  __shared__ __align__(16) float psh[128][G];
+  __shared__ float red[4][G];
+  const int b = blockIdx.x / Hk, h = blockIdx.x % Hk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Hq = Hk * G;
+  const int64_t row0 = int64_t(b) * Hq + int64_t(h) * G;        // first query row of the group
+  int rl = rlens[b];
+  if (rl < 0 || rl > max_r || int64_t(rl) > int64_t(Wr) * kBlockSize) {
+    if (h == 0 && tid == 0) flag_error(KVQ_DEVERR_CONTEXT);
+    rl = 0;
   }
-  const float r = l != 0.f ? o / l : 0.f;            // NaN l (a timed-out piece): NaN
-  if constexpr (sizeof(OutT) == 4) out[int64_t(bq) * D + d] = r;
-  else out[int64_t(bq) * D + d] = __float2bfloat16_rn(r);
+  for (int i = tid; i < G * D; i += 128) qsh[i / D][i % D] = qk_scale * __bfloat162float(q[row0 * D + i]);
+  __syncthreads();
+
+  constexpr int64_t PAGE = int64_t(kBlockSize) * D * 2;           // bytes of one BF16 page
+  const uint8_t* rkb = reinterpret_cast<const uint8_t*>(rk);
+  const uint8_t* rvb = reinterpret_cast<const uint8_t*>(rv);
+  auto unpack8 = [](const uint4& u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  };
+  float m[G], lsum[G], o[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) { m[g] = -INFINITY; lsum[g] = 0.f; o[g] = 0.f; }
+  for (int t0 = 0; t0 < rl; t0 += 128) {
+    // ---- scores of token t0 + tid
+    const int t = t0 + tid;
+    float s[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) s[g] = -INFINITY;
+    if (t < rl) {
+      const int blk = rtables[int64_t(b) * Wr + t / kBlockSize];
+      if (blk < 0 || blk >= NBr) {
+        flag_error(KVQ_DEVERR_BLOCK);
+      } else {
+        const int tt = t % kBlockSize;
+        const uint8_t* krow = rkb + (int64_t(blk) * Hk + h) * PAGE + (tt / 8) * 8 * D * 2 + (tt % 8) * 16;
+        float acc[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) acc[g] = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          float kf[8];
+          unpack8(*reinterpret_cast<const uint4*>(krow + c * 128), kf);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float4 qa = *reinterpret_cast<const float4*>(&qsh[g][c * 8]);
+            const float4 qb = *reinterpret_cast<const float4*>(&qsh[g][c * 8 + 4]);
+            acc[g] = fmaf(qa.x, kf[0], acc[g]); acc[g] = fmaf(qa.y, kf[1], acc[g]);
+            acc[g] = fmaf(qa.z, kf[2], acc[g]); acc[g] = fmaf(qa.w, kf[3], acc[g]);
+            acc[g] = fmaf(qb.x, kf[4], acc[g]); acc[g] = fmaf(qb.y, kf[5], acc[g]);
+            acc[g] = fmaf(qb.z, kf[6], acc[g]); acc[g] = fmaf(qb.w, kf[7], acc[g]);
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) s[g] = acc[g];
+      }
+    }
+    // ---- the chunk's maxima, the new references, the weights
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float wm = warp_max_f32(s[g]);
+      if (lane == 0) red[warp][g] = wm;
+    }
+    __syncthreads();
+    float alpha[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float cm = fmaxf(fmaxf(red[0][g], red[1][g]), fmaxf(red[2][g], red[3][g]));
+      const float mn = fmaxf(m[g], cm);
+      const float a = exp2f(m[g] - mn);
+      alpha[g] = (mn == m[g] || mn == -INFINITY) ? 1.f : a;
+      m[g] = mn;
+      const float e2 = exp2f(s[g] - mn);
+      const float p = s[g] != -INFINITY ? e2 : 0.f;
+      psh[tid][g] = p;
+      lsum[g] = lsum[g] * alpha[g] + p;
+      o[g] *= alpha[g];
+    }
+    __syncthreads();
+    // ---- values: channel tid, the chunk's tokens 8 at a time (a page holds
+    // two 8-token halves; t0 is a multiple of 128, so no half straddles pages)
+    if (tid < D) {
+      const int nt = min(128, rl - t0);
+      for (int u = 0; u < nt; u += 8) {
+        const int tu = t0 + u;
+        const int blk = rtables[int64_t(b) * Wr + tu / kBlockSize];
+        if (blk < 0 || blk >= NBr) continue;                      // its weights are 0
+        float vf[8];
+        unpack8(*reinterpret_cast<const uint4*>(rvb + (int64_t(blk) * Hk + h) * PAGE +
+                                                (int64_t((tu % kBlockSize) / 8) * D + tid) * 16), vf);
+        const int ne = min(8, nt - u);                            // tokens past the end: not read
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (e < ne) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) o[g] = fmaf(psh[u + e][g], vf[e], o[g]);
+          }
+        }
+      }
+    }
+    __syncthreads();                                              // psh and red are rewritten
+  }
+  // ---- the residual's sums
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float ws = warp_sum(lsum[g]);
+    if (lane == 0) red[warp][g] = ws;
+  }
+  __syncthreads();
+  float lres[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) lres[g] = red[0][g] + red[1][g] + red[2][g] + red[3][g];
+
+  // ---- merge with the groups' partials (written by the preceding kernel)
+  grid_dep_wait();
+  if (tid >= D) return;
+  int ca = __ldcg(ctx_a + b);
+  if (ca < 0 || ca > max_a || int64_t(ca) > int64_t(W_a) * kBlockSize) ca = 0;
+  ca &= ~127;
+  const int na = ca > 0 ? min(slots_a, max(0, __ldcg(pc_a + int64_t(b) * Hk + h))) : 0;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int64_t row = row0 + g, ra = row * slots_a;
+    float M = m[g];
+    for (int sl = 0; sl < na; ++sl) M = fmaxf(M, __ldcg(pml_a + (ra + sl) * 2));
+    float oo = 0.f, ll = 0.f;
+    if (M != -INFINITY) {
+      for (int sl = 0; sl < na; ++sl) {
+        const float f = exp2f(__ldcg(pml_a + (ra + sl) * 2) - M);
+        ll += __ldcg(pml_a + (ra + sl) * 2 + 1) * f;
+        oo += __ldcg(po_a + (ra + sl) * D + tid) * f;
+      }
+      if (m[g] != -INFINITY) {
+        const float f = exp2f(m[g] - M);
+        ll += lres[g] * f;
+        oo += o[g] * f;
+      }
+    }
+    const float r = ll != 0.f ? oo / ll : 0.f;                    // NaN l (a timed-out piece): NaN
+    if constexpr (sizeof(OutT) == 4) out[row * D + tid] = r;
+    else out[row * D + tid] = __float2bfloat16_rn(r);
+  }
 }
 
 }  // namespace kvq
