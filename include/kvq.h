@@ -468,9 +468,12 @@ int kvq_kivi_append(const void* k, const void* v, const int64_t* slot_mapping, i
  * and max_res_len bound them. dims describes the low-bit pool, res_dims the
  * residual BF16 pool (same heads and head_dim). meta: host array {k_meta,
  * v_meta}. The groups run on the tensor cores from the codes (the query is
- * rebuilt per group with its channel scales), the residual through the BF16
- * decode kernel, and one merge combines both. workspace: at least
- * kvq_kivi_decode_workspace_bytes(...) bytes.
+ * rebuilt per group with its channel scales) into split-K partials; a second
+ * kernel attends the residual tokens in FP32 and merges them with those
+ * partials (a residual block id outside [0, res_dims->num_blocks) skips the
+ * token and sets KVQ_DEVERR_BLOCK; a residual length outside [0, max_res_len]
+ * or beyond the residual table counts as 0 and sets KVQ_DEVERR_CONTEXT).
+ * workspace: at least kvq_kivi_decode_workspace_bytes(...) bytes.
  */
 size_t kvq_kivi_decode_workspace_bytes(int32_t batch, int32_t max_quant_len, int32_t max_res_len,
                                        kvq_fmt fmt, const kvq_dims* dims,
