@@ -272,32 +272,67 @@ __global__ void __launch_bounds__(128) kivi_residual_merge_kernel(
 #pragma unroll
   for (int g = 0; g < G; ++g) lres[g] = red[0][g] + red[1][g] + red[2][g] + red[3][g];
 
-  // ---- merge with the groups' partials (written by the preceding kernel)
+  // ---- merge with the groups' partials (written by the preceding kernel),
+  // eight slots at a time: the slots' (m, l) of all G rows are loaded by one
+  // thread each into shared memory while every channel thread requests its
+  // G x 8 partial values, so a chunk costs one round trip to memory
   grid_dep_wait();
-  if (tid >= D) return;
   int ca = __ldcg(ctx_a + b);
   if (ca < 0 || ca > max_a || int64_t(ca) > int64_t(W_a) * kBlockSize) ca = 0;
   ca &= ~127;
   const int na = ca > 0 ? min(slots_a, max(0, __ldcg(pc_a + int64_t(b) * Hk + h))) : 0;
+  __shared__ float2 mls[G][8];
+  float M[G], ll[G], oo[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const int64_t row = row0 + g, ra = row * slots_a;
-    float M = m[g];
-    for (int sl = 0; sl < na; ++sl) M = fmaxf(M, __ldcg(pml_a + (ra + sl) * 2));
-    float oo = 0.f, ll = 0.f;
-    if (M != -INFINITY) {
-      for (int sl = 0; sl < na; ++sl) {
-        const float f = exp2f(__ldcg(pml_a + (ra + sl) * 2) - M);
-        ll += __ldcg(pml_a + (ra + sl) * 2 + 1) * f;
-        oo += __ldcg(po_a + (ra + sl) * D + tid) * f;
-      }
-      if (m[g] != -INFINITY) {
-        const float f = exp2f(m[g] - M);
-        ll += lres[g] * f;
-        oo += o[g] * f;
+    M[g] = m[g];                                                // the residual's (or -inf)
+    ll[g] = lres[g];
+    oo[g] = o[g];
+  }
+  for (int s0 = 0; s0 < na; s0 += 8) {
+    const int ns = min(8, na - s0);
+    __syncthreads();                                            // the previous chunk's mls are used
+    if (tid < G * 8) {
+      const int g = tid >> 3, j = tid & 7;
+      float2 v = make_float2(-INFINITY, 0.f);
+      if (j < ns) v = __ldcg(reinterpret_cast<const float2*>(pml_a + ((row0 + g) * slots_a + s0 + j) * 2));
+      mls[g][j] = v;
+    }
+    float pv[G][8];
+    if (tid < D) {
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          pv[g][j] = j < ns ? __ldcg(po_a + ((row0 + g) * slots_a + s0 + j) * D + tid) : 0.f;
+    }
+    __syncthreads();
+    if (tid < D) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float cm = M[g];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cm = fmaxf(cm, mls[g][j].x);
+        if (cm != -INFINITY) {
+          const float sc = exp2f(M[g] - cm);                    // 0 while nothing was seen
+          ll[g] *= sc;
+          oo[g] *= sc;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {                        // slots past ns: m = -inf, f = 0
+            const float f = exp2f(mls[g][j].x - cm);
+            ll[g] = fmaf(mls[g][j].y, f, ll[g]);
+            oo[g] = fmaf(pv[g][j], f, oo[g]);
+          }
+          M[g] = cm;
+        }
       }
     }
-    const float r = ll != 0.f ? oo / ll : 0.f;                    // NaN l (a timed-out piece): NaN
+  }
+  if (tid >= D) return;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int64_t row = row0 + g;
+    const float r = ll[g] != 0.f ? oo[g] / ll[g] : 0.f;        // NaN l (a timed-out piece): NaN
     if constexpr (sizeof(OutT) == 4) out[row * D + tid] = r;
     else out[row * D + tid] = __float2bfloat16_rn(r);
   }
