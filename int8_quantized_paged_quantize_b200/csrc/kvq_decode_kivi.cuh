@@ -535,6 +535,7 @@ __global__ void __launch_bounds__(256, 2) decode_kivi_kernel(
         // this warp's heads of the tile's query operand (the previous tile's S
         // product has read the operand)
         if (ok && gt > 0) ok = mbar_wait(qfree, (gt - 1) & 1, abort_flag, wait_limit);
+        ok = __all_sync(0xffffffffu, ok);                   // the build is warp-collective
         if (ok)
           kivi_build_query<C, D, G, HPC>(qcur, gsc, pkmeta + sp * 8 * C::META, qop, qsc + (gt & 3) * 8,
                                          qzs + (gt & 3) * 8, qk_scale, lane);
