@@ -27,7 +27,7 @@ MEAN_ABS = 5e-4
 
 
 @dataclass
-class GpuRun:
+class DeviceRun:
     w: W.Workload
     fmt: str
     cache: kvq.LayerCache
@@ -89,7 +89,7 @@ def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch
             history_chunks=1, static=None):
     """Append every sequence's cached history (in `history_chunks` calls), then the
     bulk append if the workload has one, then one token per sequence, and run one
-    decode step over ctx + 1 tokens. Returns a GpuRun."""
+    decode step over ctx + 1 tokens. Returns a DeviceRun."""
     ctx = W.context_lengths(w, seed)
     hist, bulk, (q, k_new, v_new) = inputs(w, seed)
     if w.pool == "fragmented":
@@ -147,11 +147,11 @@ def run_gpu(w: W.Workload, fmt: str, seed=0, partition_tokens=0, out_dtype=torch
                        partition_tokens=partition_tokens, out_dtype=out_dtype)
     torch.cuda.synchronize()
     assert kvq.device_error(clear=True) == 0
-    return GpuRun(w, fmt, cache, tables, ctx, ctx_after, q, k_new, v_new, out.cpu(), seed, kst, vst)
+    return DeviceRun(w, fmt, cache, tables, ctx, ctx_after, q, k_new, v_new, out.cpu(), seed, kst, vst)
 
 
 # ----------------------------------------------------------------------------- oracle side
-def oracle_sequence(run: GpuRun, b: int):
+def oracle_sequence(run: DeviceRun, b: int):
     """Oracle codes/scales and dequantised K/V of sequence b's ctx_after tokens,
     quantised by the oracle from the same seeded BF16 inputs.
 
@@ -190,7 +190,7 @@ def oracle_sequence(run: GpuRun, b: int):
     return res
 
 
-def gpu_sequence(run: GpuRun, b: int):
+def gpu_sequence(run: DeviceRun, b: int):
     """The GPU cache contents of sequence b's ctx_after tokens in logical order:
     codes [n][Hk][D] and metadata [n][Hk] (scale, zero point)."""
     n = int(run.ctx_after[b])
@@ -214,7 +214,7 @@ def gpu_sequence(run: GpuRun, b: int):
     return out
 
 
-def assert_codes_equal(run: GpuRun, b: int, ref: dict):
+def assert_codes_equal(run: DeviceRun, b: int, ref: dict):
     g = gpu_sequence(run, b)
     for name in ("k", "v"):
         gc = g[name + "_codes"]
@@ -231,7 +231,7 @@ def assert_codes_equal(run: GpuRun, b: int, ref: dict):
             assert np.array_equal(g[name + "_zp"], ref[name + "_zp"].astype(np.float32)), f"{name} zp b={b}"
 
 
-def oracle_attention(run: GpuRun, b: int, ref: dict, raw=False):
+def oracle_attention(run: DeviceRun, b: int, ref: dict, raw=False):
     """FP64 attention of sequence b, [Hq][D]: over the dequantised cache, or with
     raw=True over the unquantised BF16 values (the quality reference)."""
     K, V = (ref["Kraw"], ref["Vraw"]) if raw else (ref["K"], ref["V"])
@@ -239,7 +239,7 @@ def oracle_attention(run: GpuRun, b: int, ref: dict, raw=False):
     return OA.decode_attention(q, [(K, V)], run.w.sm_scale, run.w.n_kv_heads)[0]
 
 
-def attention_errors(run: GpuRun, seqs, check_codes=True):
+def attention_errors(run: DeviceRun, seqs, check_codes=True):
     """(max abs err, mean abs err) of the GPU output vs the oracle over `seqs`."""
     errs = []
     for b in seqs:
@@ -323,7 +323,7 @@ def check_steps_run(run: StepsRun, b: int, steps):
                   [x[b:b + 1] for x in run.v_new]).float().numpy()
     n = k.shape[0]
     # the cache view of assert_codes_equal: every sequence's tokens after the last step
-    one = GpuRun(w, run.fmt, run.cache, run.tables, run.ctx_hist,
+    one = DeviceRun(w, run.fmt, run.cache, run.tables, run.ctx_hist,
                  run.ctx_hist + w.bulk_append + run.steps, None, None, None, None, run.seed)
     assert int(one.ctx_after[b]) == n
     res = {"Kraw": k.astype(np.float64), "Vraw": v.astype(np.float64)}
