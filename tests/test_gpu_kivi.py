@@ -56,13 +56,15 @@ def unpack_v_page(page, D, bits):
     return codes
 
 
-def _build(fmt, lens, Hk=2, G=4, D=128, seed=0, kv_mean=0.0):
+def _build(fmt, lens, Hk=2, G=4, D=128, seed=0, kv_mean=0.0, quantized=None):
     bits = kvq.KIVI_BITS[fmt]
     w = W.Workload("kivi", "fp8", batch=len(lens), n_q_heads=Hk * G, n_kv_heads=Hk, head_dim=D,
                    lengths="list", ctx=tuple(lens), kv_mean=kv_mean)
     rng = np.random.default_rng(seed)
-    groups = [n // 128 for n in lens]
-    res = [n % 128 for n in lens]
+    # quantized[b]: the sequence's tokens in complete groups (default: all of
+    # its complete groups); the rest stays in the BF16 residual cache
+    groups = [n // 128 for n in lens] if quantized is None else [m // 128 for m in quantized]
+    res = [n - 128 * g for n, g in zip(lens, groups)]
     # low-bit pool: 8 blocks per group, shuffled; residual pool: its own blocks
     nq = max(1, sum(groups) * 8)
     perm = rng.permutation(nq)
@@ -132,8 +134,8 @@ def _check_codes(cache, bits, qt, hist, groups, b, D, Hk):
     return st
 
 
-def _run(fmt, lens, Hk=2, G=4, D=128, seed=0, kv_mean=0.0, check_codes=True):
-    w, bits, cache, qt, rt, hist, groups, res = _build(fmt, lens, Hk, G, D, seed, kv_mean)
+def _run(fmt, lens, Hk=2, G=4, D=128, seed=0, kv_mean=0.0, check_codes=True, quantized=None):
+    w, bits, cache, qt, rt, hist, groups, res = _build(fmt, lens, Hk, G, D, seed, kv_mean, quantized)
     g = torch.Generator().manual_seed(50 + seed)
     q = torch.randn(w.batch, Hk * G, D, generator=g).to(torch.bfloat16)
     ql = np.array([x * 128 for x in groups], dtype=np.int32)
@@ -147,9 +149,17 @@ def _run(fmt, lens, Hk=2, G=4, D=128, seed=0, kv_mean=0.0, check_codes=True):
     errs = []
     for b in range(w.batch):
         k, v = hist[b]
-        st = (_check_codes(cache, bits, qt, hist, groups, b, D, Hk) if check_codes else
-              OK.quantize_sequence(k.float().numpy(), v.float().numpy(), bits=bits))
-        K, V = OK.dequantize_sequence(st)
+        m = groups[b] * 128
+        if quantized is None:
+            st = (_check_codes(cache, bits, qt, hist, groups, b, D, Hk) if check_codes else
+                  OK.quantize_sequence(k.float().numpy(), v.float().numpy(), bits=bits))
+            K, V = OK.dequantize_sequence(st)
+        else:
+            # the first m tokens as groups, every later one in BF16
+            st = OK.quantize_sequence(k[:m].float().numpy(), v[:m].float().numpy(), bits=bits)
+            K, V = OK.dequantize_sequence(st)
+            K = np.concatenate([K, k[m:].float().numpy().astype(np.float64)])
+            V = np.concatenate([V, v[m:].float().numpy().astype(np.float64)])
         ref = OA.decode_attention(q[b:b + 1].float().numpy(), [(K, V)], w.sm_scale, Hk)[0]
         errs.append(np.abs(out[b].cpu().numpy().astype(np.float64) - ref).ravel())
     e = np.concatenate(errs)
@@ -175,4 +185,16 @@ def test_kivi_head_dim_64_nonzero_mean(fmt):
 def test_kivi_long_contexts():
     """Several CTAs per sequence (split-K) and many groups."""
     mx, mean = _run("kivi2", [8192 + 50, 4096, 12000], G=8, check_codes=False)
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
+
+
+@pytest.mark.parametrize("fmt", ["kivi2", "kivi4"])
+def test_kivi_residual_longer_than_a_group(fmt):
+    """Residuals of several hundred BF16 tokens (a caller that has not yet
+    quantized complete groups): the residual attention runs over several
+    128-token chunks, its online softmax moving between them; sequences with
+    no quantized group at all and with no residual are mixed in."""
+    lens = [900, 300, 2048, 129, 640]
+    quantized = [256, 0, 2048, 0, 128]
+    mx, mean = _run(fmt, lens, G=8, quantized=quantized)
     assert mx <= MAX_ABS and mean <= MEAN_ABS, (mx, mean)
