@@ -820,12 +820,13 @@ __global__ void __maxnreg__(FMT == KVQ_BF16 ? 168 : 120) decode_mma_kernel(
           const float4 t4 = *reinterpret_cast<const float4*>(rb + g * 4);
           const float tmax = fmaxf(fmaxf(t4.x, t4.y), fmaxf(t4.z, t4.w));
           const float mn = fmaxf(m[g], tmax);
-          alpha[g] = 1.f;
-          if (mn != m[g]) {                      // the same for every thread of the CTA
-            alpha[g] = (mn == -INFINITY) ? 1.f : exp2f(m[g] - mn);
-            m[g] = mn;
-            o[g] *= alpha[g];
-          }
+          // 2^(m - mn) when the maximum moves, 1 while it stays (or while no
+          // token has been seen): selects rather than branches, so that the
+          // heads' exponentials overlap
+          const float a = exp2f(m[g] - mn);
+          alpha[g] = (mn == m[g] || mn == -INFINITY) ? 1.f : a;
+          m[g] = mn;
+          o[g] *= alpha[g];
         }
         // P = p * v_scale * 2^ex with max(v_scale) * 2^ex in [128, 256): inside
         // the E4M3 range, and below 2^8 for the 24-bit fixed point of INT8
